@@ -1,0 +1,509 @@
+#!/usr/bin/env python
+"""Throughput of the POET layer hot path on B200: forward + backward (dX and
+packed-skew gradients, Cayley-Neumann for every primitive) over a LLaMA-shaped
+layer set, in tokens/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl poet|reference]
+                    [--workload llama1.3b|llama60m|llama350m|llama3b]
+
+One step = Cayley-Neumann of every primitive, then the forward of every
+linear of every layer, then the backward of every linear in reverse order;
+for the default workload both variants (fully stochastic and block-stochastic
+b=256 at LLaMA-1.3B shapes) run back to back, each over its own T tokens.
+Merge-then-reinitialize (every 400 steps in the pages' setup) is timed
+separately and reported amortized.  Under torchrun each rank trains its own
+replica on its own tokens (data parallel, weak scaling) and the packed-skew
+gradients are all-reduced over NCCL once per step.
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD_SETS = {
+    "llama1.3b": ["llama1.3b_fs", "llama1.3b_bs256"],
+    "llama60m": ["llama60m_fs"],
+    "llama350m": ["llama350m_bs256"],
+    "llama3b": ["llama3b_fs"],
+}
+METRIC = "POET layer fwd+bwd tokens/s at LLaMA-1.3B shapes; % of TC/HBM roofline"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["poet", "reference"], default="poet")
+    ap.add_argument("--workload", choices=sorted(WORKLOAD_SETS), default="llama1.3b")
+    ap.add_argument("--e2e-steps", type=int, default=1)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-merge", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="poet_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        busy = [s for s in sm if smax and s > 0.3 * smax] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- CUDA path
+
+class Variant:
+    """All POET linears of one workload, resident on the device."""
+
+    def __init__(self, wl, rank, device, w0_cache):
+        import torch
+
+        from orthogonal_reparameterized_poet_b200 import inputs as I
+        from orthogonal_reparameterized_poet_b200 import poet
+
+        self.wl = wl
+        self.T = wl.tokens
+        tdt = poet.torch_dtype(wl.dtype)
+        shapes = wl.linear_shapes()
+        self.layers = []
+        nth = []
+        for layer in range(wl.layers):
+            for t, (m, n) in enumerate(shapes):
+                key = (wl.seed, layer, t, m, n, wl.dtype)
+                if key not in w0_cache:
+                    w0_cache[key] = torch.from_numpy(I.w0(wl.seed, layer, t, m, n, wl.dtype)).to(device=device,
+                                                                                              dtype=tdt)
+                    W0 = w0_cache[key]
+                else:  # another variant of the same model: its own copy (merge updates W0 in place)
+                    W0 = w0_cache[key].clone()
+                nR, sR = poet.side_geometry(m, wl.mode, wl.b)
+                nP, sP = poet.side_geometry(n, wl.mode, wl.b)
+                thR = torch.from_numpy(I.theta(wl.seed, layer, t, 0, nR * sR * (sR - 1) // 2, wl.sigma)).to(device)
+                thP = torch.from_numpy(I.theta(wl.seed, layer, t, 1, nP * sP * (sP - 1) // 2, wl.sigma)).to(device)
+                L = poet.PoetLayer(W0, thR, thP, mode=wl.mode, b=wl.b, k=wl.k, seed=wl.seed,
+                                   layer_id=layer * len(shapes) + t)
+                L.prepare()
+                self.layers.append((layer, t, m, n, L))
+                nth.append((thR.numel(), thP.numel()))
+        # one flat gradient buffer (one all-reduce per step under data parallelism)
+        total = sum(a + b for a, b in nth)
+        self.dtheta = torch.zeros(max(total, 1), dtype=torch.float32, device=device)
+        self.dslices = []
+        off = 0
+        for a, b in nth:
+            self.dslices.append((self.dtheta[off:off + a], self.dtheta[off + a:off + a + b]))
+            off += a + b
+        # per-shape activations (each rank draws its own tokens)
+        self.x, self.dy, self.y, self.dx = {}, {}, {}, {}
+        for (m, n) in set(shapes):
+            if n not in self.x:
+                self.x[n] = torch.from_numpy(I.activations(wl.seed + 7919 * rank, n, self.T, n, wl.dtype)).to(
+                    device=device, dtype=tdt)
+                self.dx[n] = torch.empty(self.T, n, dtype=tdt, device=device)
+            if m not in self.dy:
+                self.dy[m] = torch.from_numpy(
+                    I.activations(wl.seed + 7919 * rank, m, self.T, m, wl.dtype, grad=True)).to(device=device,
+                                                                                             dtype=tdt)
+                self.y[m] = torch.empty(self.T, m, dtype=tdt, device=device)
+        self.saved = [L.saved_buffer(self.T) for (_, _, _, _, L) in self.layers]
+        for (_, _, _, _, L) in self.layers:
+            L.workspace(self.T)
+        self.input_bytes = sum(v.numel() * v.element_size() for v in list(self.x.values()) + list(self.dy.values()))
+
+    def step(self, world=1):
+        for (_, _, _, _, L) in self.layers:
+            L.cayley_neumann()
+        for i, (_, _, m, n, L) in enumerate(self.layers):
+            L.forward(self.x[n], y=self.y[m], saved=self.saved[i])
+        for i in reversed(range(len(self.layers))):
+            _, _, m, n, L = self.layers[i]
+            dR, dP = self.dslices[i]
+            L.backward(self.saved[i], self.dy[m], dx=self.dx[n], dtheta_R=dR, dtheta_P=dP)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.all_reduce(self.dtheta)
+
+    def merge_all(self):
+        for (_, _, _, _, L) in self.layers:
+            L.merge()
+            L.resample()
+
+
+def run_poet(args):
+    import torch
+
+    from orthogonal_reparameterized_poet_b200 import inputs as I
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    poet.lib()
+
+    wls = [I.WORKLOADS[name] for name in WORKLOAD_SETS[args.workload]]
+    w0_cache = {}
+    variants = [Variant(wl, rank, device, w0_cache) for wl in wls]
+    del w0_cache
+    torch.cuda.synchronize()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def step():
+        for v in variants:
+            v.step(world)
+
+    for _ in range(args.warmup):
+        step()
+    poet.poet_sync_status()
+
+    # ---- timed region
+    stream = torch.cuda.current_stream()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    smi_index = vis.split(",")[local] if vis else str(local)
+    clocks = ClockSampler(smi_index)
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in variants] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    poet.poet_trace_enable(True)
+    launches0 = poet.poet_launch_count()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s_ in range(args.steps):
+        for i, v in enumerate(variants):
+            ev[s_][i][0].record(stream)
+            v.step(world)
+            ev[s_][i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    per_variant_ms = [sum(ev[s_][i][0].elapsed_time(ev[s_][i][1]) for s_ in range(args.steps))
+                      for i in range(len(variants))]
+    launches = poet.poet_launch_count() - launches0
+    poet.poet_trace_enable(False)
+    clk = clocks.stop()
+    barrier()
+    elapsed = t0.elapsed_time(t1)
+    trace = poet.poet_trace_read()
+    poet.poet_sync_status()
+    if dist is not None:
+        t = torch.tensor([elapsed] + per_variant_ms, dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t[0])
+        per_variant_ms = [float(x) for x in t[1:]]
+
+    tokens_per_step = sum(v.T for v in variants) * world
+    ms_per_step = elapsed / args.steps
+    value = tokens_per_step / (ms_per_step / 1e3)
+
+    # ---- merge-then-reinitialize (timed once, amortized over the merge period)
+    merge = {}
+    if not args.no_merge:
+        for v in variants:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            v.merge_all()
+            b.record(stream)
+            b.synchronize()
+            merge[v.wl.name] = a.elapsed_time(b)
+        poet.poet_sync_status()
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, variants, world)
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    peaks = load_peaks()
+    rows = {k: dict(v) for k, v in trace.items()}
+    dominant = max(rows, key=lambda k: rows[k]["ms"]) if rows else None
+    roof = None
+    if dominant:
+        r = rows[dominant]
+        intensity = r["flop"] / r["bytes"] if r["bytes"] else float("inf")
+        ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        avg_ms = r["ms"] / r["launches"]
+        if intensity >= ridge:
+            achieved = r["flop"] / (r["ms"] / 1e3) / 1e12
+            peak = peaks["bf16_tflops_sustained"]
+            roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_kind": "bf16 sustained, " + peaks["source"]}
+        else:
+            achieved = r["bytes"] / (r["ms"] / 1e3) / 1e9
+            peak = peaks["hbm_gbs"]
+            roof = {"bound": "hbm", "unit": "GB/s", "peak_kind": "copy, " + peaks["source"]}
+        roof.update({"kernel": dominant, "achieved": round(achieved, 1), "peak": peak,
+                     "frac": round(achieved / peak, 4), "traffic": None, "avg_launch_ms": round(avg_ms, 4),
+                     "launches": r["launches"], "algorithmic_per_launch": {
+                         "flop": r["flop"] / r["launches"], "bytes": r["bytes"] / r["launches"]}})
+    kernels = {}
+    for k, r in sorted(rows.items(), key=lambda kv: -kv[1]["ms"]):
+        kernels[k] = {"launches": r["launches"], "ms_per_step": round(r["ms"] / args.steps, 3),
+                      "share": round(r["ms"] / sum(x["ms"] for x in rows.values()), 4),
+                      "tflops": round(r["flop"] / (r["ms"] / 1e3) / 1e12, 1) if r["ms"] and r["flop"] else None,
+                      "gbs": round(r["bytes"] / (r["ms"] / 1e3) / 1e9, 1) if r["ms"] else None}
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu = cpu_baseline([v.wl for v in variants])
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wls[0].dtype == I.BF16 else "f32",
+        "data": "synthetic (seeded N(0,1) tokens, normalized-Gaussian W0, random-init skew parameters)",
+        "config": {"workload": args.workload + "_" + "+".join(w.name.split("_", 1)[1] for w in wls),
+                   "hidden": wls[0].hidden, "ffn": wls[0].ffn, "layers": wls[0].layers,
+                   "linears_per_layer": len(wls[0].linear_shapes()), "tokens_per_variant": wls[0].tokens,
+                   "variants": [{"name": w.name, "mode": "FS" if w.mode == I.FS else "BS", "b": w.b, "k": w.k}
+                                for w in wls],
+                   "parallelism": f"dp{world}", "l2": "inputs larger than L2 (no flush needed)"},
+        "variants": {v.wl.name: {"ms_per_step": round(per_variant_ms[i] / args.steps, 3),
+                                 "tokens_per_s": round(v.T * world / (per_variant_ms[i] / args.steps / 1e3), 1),
+                                 "merge_ms": round(merge.get(v.wl.name, float("nan")), 3) if merge else None}
+                     for i, v in enumerate(variants)},
+        "value_merge_amortized": (round(tokens_per_step / ((ms_per_step + sum(merge.values()) / 400.0) / 1e3), 1)
+                                  if merge else None),
+        "roofline": roof, "kernels": kernels, "gpu_launches": int(launches), "clocks": clk,
+        "e2e": e2e, "cpu_baseline": cpu,
+    }
+    print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_e2e(args, variants, world):
+    """Same step through the public API with host buffers: every step copies the
+    step's inputs from pinned host memory and reads the results back."""
+    import torch
+
+    stream = torch.cuda.current_stream()
+    host_in, host_out = [], []
+    for v in variants:
+        for d in (v.x, v.dy):
+            for key, t in d.items():
+                host_in.append((t, t.cpu().pin_memory()))
+        host_out.append((v.dtheta, torch.empty(v.dtheta.shape, dtype=v.dtheta.dtype, pin_memory=True)))
+        last_m = v.layers[0][2]
+        last_n = v.layers[0][3]
+        host_out.append((v.y[last_m], torch.empty(v.y[last_m].shape, dtype=v.y[last_m].dtype, pin_memory=True)))
+        host_out.append((v.dx[last_n], torch.empty(v.dx[last_n].shape, dtype=v.dx[last_n].dtype, pin_memory=True)))
+    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
+    d2h = sum(h.numel() * h.element_size() for _, h in host_out)
+
+    def step():
+        for dev, host in host_in:
+            dev.copy_(host, non_blocking=True)
+        for v in variants:
+            v.step(world)
+        for dev, host in host_out:
+            host.copy_(dev, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    b.record(stream)
+    b.synchronize()
+    ms = a.elapsed_time(b) / args.e2e_steps
+    tokens = sum(v.T for v in variants) * world
+    return {"value": round(tokens / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 3),
+            "steps": args.e2e_steps, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(wls, budget_s=25.0):
+    """The float64 CPU oracle, as it stands, on a bounded sample of the same
+    workload, extrapolated to the full step in tokens/s."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from oracle import poet_oracle as O
+    from orthogonal_reparameterized_poet_b200 import inputs as I
+
+    cores = sum(p.get("num_threads", 1) for p in threadpool_info() if p.get("user_api") == "blas") or 1
+    total_s, total_tokens = 0.0, 0
+    sample_desc = []
+    t_start = time.perf_counter()
+    for wl in wls:
+        shapes = wl.linear_shapes()
+        Ts = 64
+        # token-independent part: Cayley-Neumann forward + backward, once per distinct primitive size
+        cnp_s = {}
+        for (m, n) in set(shapes):
+            for d in (m, n):
+                nprim, size = O.side_shape(d, wl.mode, wl.b)
+                if size in cnp_s or nprim == 0:
+                    continue
+                th = I.theta(wl.seed, 0, 0, 0, O.n_skew(size), wl.sigma).astype(np.float64)
+                G = np.random.default_rng(0).standard_normal((1, size, size))
+                t = time.perf_counter()
+                O.cayley_neumann(th, 1, size, wl.k)
+                O.theta_grad(G, th, size, wl.k)
+                cnp_s[size] = time.perf_counter() - t
+        # token-dependent part: dense forward + backward on Ts tokens, once per distinct linear shape
+        tok_s = {}
+        for t_idx, (m, n) in enumerate(shapes):
+            if (m, n) in tok_s:
+                continue
+            W0 = I.w0(wl.seed, 0, t_idx, m, n, wl.dtype).astype(np.float64)
+            nR, sR = O.side_shape(m, wl.mode, wl.b)
+            nP, sP = O.side_shape(n, wl.mode, wl.b)
+            permR, permP = O.draw_perm(wl.seed, t_idx, 0, 0, m), O.draw_perm(wl.seed, t_idx, 1, 0, n)
+            Rb = np.broadcast_to(np.eye(sR), (nR, sR, sR)) if nR else np.zeros((0, 0, 0))
+            Pb = np.broadcast_to(np.eye(sP), (nP, sP, sP)) if nP else np.zeros((0, 0, 0))
+            x = I.activations(wl.seed, n, Ts, n, wl.dtype).astype(np.float64)
+            dy = I.activations(wl.seed, m, Ts, m, wl.dtype, grad=True).astype(np.float64)
+            t = time.perf_counter()
+            R = O.dense_side(permR, Rb, wl.mode, wl.b)
+            P = O.dense_side(permP, Pb, wl.mode, wl.b)
+            O.forward(W0, R, P, x)
+            O.backward(W0, R, P, x, dy, permR, wl.mode, wl.b, permP, wl.mode, wl.b)
+            tok_s[(m, n)] = time.perf_counter() - t
+        per_layer = 0.0
+        for (m, n) in shapes:
+            for d in (m, n):
+                nprim, size = O.side_shape(d, wl.mode, wl.b)
+                if nprim:
+                    per_layer += nprim * cnp_s[size]
+            per_layer += tok_s[(m, n)] * wl.tokens / Ts
+        total_s += per_layer * wl.layers
+        total_tokens += wl.tokens
+        sample_desc.append(f"{wl.name}: Cayley-Neumann fwd+bwd once per distinct primitive size "
+                           f"{sorted(cnp_s)}, dense fwd+bwd of {Ts} tokens once per distinct linear shape")
+        if time.perf_counter() - t_start > budget_s:
+            break
+    wall = time.perf_counter() - t_start
+    return {"value": round(total_tokens / total_s, 3), "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
+            "sample": "; ".join(sample_desc) + f"; extrapolated linearly to all layers and tokens "
+                      f"({wall:.1f} s of CPU work)", "sample_wall_s": round(wall, 2)}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: rank 0 times it on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from orthogonal_reparameterized_poet_b200 import inputs as I
+
+    wls = [I.WORKLOADS[name] for name in WORKLOAD_SETS[args.workload]]
+    vals = []
+    res = None
+    for i in range(args.warmup + args.steps):
+        res = cpu_baseline(wls, budget_s=8.0)
+        if i >= args.warmup:
+            vals.append(res["value"])
+    value = statistics.median(vals) if vals else res["value"]
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sum(w.tokens for w in wls) / value * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload + "_" + "+".join(w.name.split("_", 1)[1] for w in wls),
+                   "tokens_per_variant": wls[0].tokens, "parallelism": "cpu"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": res["cores"], "kind": "oracle",
+                         "sample": res["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_poet(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,258 @@
+/*
+ * poet.h -- C ABI of libpoet, the B200 (sm_100a) hot path of the POET
+ * reparameterized linear layer   y = R . W0 . P . x
+ *
+ * Sources (web pages on POET / POET-X; cited by page title and section):
+ *   [P1] "Reparameterized LLM Training via Orthogonal Equivalence
+ *        Transformation" (atlas.scime.ai summary of arXiv 2506.08001):
+ *        Approach, Key results, Measured effects table, Limitations.
+ *   [P2] mlsanity page for arXiv 2506.08001: Abstract.
+ *   [P3] "POET-X: Memory-efficient LLM Training by Scaling Orthogonal
+ *        Transformation" (pith.science review): Core claim, What carries the
+ *        argument.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument named "device" is CUDA device memory on the
+ *    current device; the caller owns all memory.  The library never
+ *    allocates device memory: scratch comes from the caller's workspace.
+ *  - Every call is asynchronous and ordered on the given stream (NULL = the
+ *    legacy default stream).  Inputs must stay valid until the work is done.
+ *  - Row-major everywhere.  W0 is m x n (out x in).  Activations are
+ *    token-major: x is T x n, y is T x m (one row per token), so the per-token
+ *    y_t = R W0 P x_t of [P1] Approach is  Y = X P^T W0^T R^T.
+ *  - Element type: POET_F32 (float) or POET_BF16 (bfloat16, round to nearest
+ *    even) for W0, activations and materialized primitives.  Skew parameters
+ *    theta and their gradients are always float32.  Accumulation is float32.
+ *  - Status: arguments are validated on the host before anything is
+ *    launched; a bad argument returns POET_EINVAL and launches nothing.  A
+ *    failed CUDA launch returns POET_ECUDA.  Device-side errors (a bounded
+ *    wait that ran out) are recorded in a device status word that
+ *    poet_sync_status() reads.  poet_last_error() describes the last failure
+ *    of the calling thread.
+ *
+ * One side (R: dim = m, P: dim = n) -- readings of [P1] Key results
+ * ("POET-FS (b=1/2)", "POET-BS (b=256)"); the pages fix no layout:
+ *  - perm is a permutation of 0..dim-1.
+ *  - POET_BS: floor(dim/b) primitives of size b; primitive j acts on the
+ *    natural indices perm[j*b .. j*b+b-1]; the dim mod b leftover indices are
+ *    left unchanged (identity).
+ *  - POET_FS: one primitive of size s = floor(dim/2) acting on perm[0..s-1].
+ *  - As a matrix the side is  Pi^T diag(B_0, ..., B_{q-1}, I) Pi  with
+ *    (Pi v)_i = v[perm[i]].
+ *  - theta holds, for each primitive in order, size*(size-1)/2 floats: the
+ *    strict upper triangle of U packed row by row; Q = U - U^T.
+ *  - Each primitive is the truncated Cayley-Neumann map of order k >= 0
+ *    ([P1] Approach, Limitations):  B = (I + Q)(I + Q + Q^2 + ... + Q^k).
+ *
+ * The permuted frame.  The library keeps a copy of W0 with rows ordered by
+ * R.perm and columns by P.perm (W0f[i][j] = W0[R.perm[i]][P.perm[j]]), so
+ * that every primitive acts on a contiguous range of frame indices and every
+ * contraction on the hot path reads contiguous tiles.  Activations are
+ * gathered into the frame once on entry and scattered out once on exit.
+ */
+#ifndef POET_H
+#define POET_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define POET_API __attribute__((visibility("default")))
+#else
+#define POET_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t (a CUDA runtime stream handle). */
+typedef struct CUstream_st *poet_stream;
+
+typedef enum {
+  POET_OK = 0,
+  POET_EINVAL = 1,     /* bad argument; nothing was launched */
+  POET_ECUDA = 2,      /* a CUDA call or launch failed */
+  POET_ETIMEOUT = 3,   /* a device-side bounded wait ran out (see poet_sync_status) */
+  POET_ENOMEM_WS = 4   /* the workspace passed is smaller than required */
+} poet_status;
+
+typedef enum { POET_F32 = 0, POET_BF16 = 1 } poet_dtype;
+typedef enum { POET_BS = 0, POET_FS = 1 } poet_mode;
+
+typedef struct {
+  int32_t dim;     /* m for R, n for P; 1 <= dim <= 16384 */
+  int32_t mode;    /* POET_BS or POET_FS */
+  int32_t b;       /* POET_BS: block size, 1 <= b; ignored for POET_FS */
+  int32_t k;       /* Neumann order, 0 <= k <= 16 */
+  int32_t *perm;   /* device int32[dim]; written by poet_prepare/poet_resample */
+  float *theta;    /* device float[nprim * size*(size-1)/2]; zeroed by poet_merge */
+  void *state;     /* device, poet_side_state_bytes() bytes, written by
+                      poet_cayley_neumann.  It starts with the materialized
+                      primitives, element type dtype, [nprim][ld][ld] with
+                      ld = size rounded up to a multiple of 8 (padding zero);
+                      the rest (Neumann terms for the backward) is opaque. */
+} poet_side;
+
+typedef struct {
+  int64_t m;       /* output features (rows of W0) */
+  int64_t n;       /* input features (columns of W0) */
+  int32_t dtype;   /* poet_dtype of W0, W0f, activations, primitives */
+  int32_t layer_id;/* >= 0; keys the permutation draw */
+  int32_t epoch;   /* >= 0; advanced by poet_resample */
+  int32_t reserved;/* must be 0 */
+  uint64_t seed;   /* keys the permutation draw */
+  void *W0;        /* device m x n, row-major, natural order (the fixed weight) */
+  void *W0f;       /* device, poet_frame_bytes() bytes: W0 in the permuted frame */
+  poet_side R;     /* left side, dim = m */
+  poet_side P;     /* right side, dim = n */
+} poet_layer;
+
+/* ---------------------------------------------------------------- sizes */
+
+/* Bytes of side->state for element type dtype (0 if the side is invalid). */
+POET_API size_t poet_side_state_bytes(const poet_side *side, int32_t dtype);
+
+/* Bytes of L->W0f (0 if the layer is invalid). */
+POET_API size_t poet_frame_bytes(const poet_layer *L);
+
+/* Bytes of the buffer poet_forward saves for poet_backward at T tokens. */
+POET_API size_t poet_saved_bytes(const poet_layer *L, int64_t T);
+
+/* Bytes of workspace that poet_forward, poet_backward, poet_merge and
+ * poet_cayley_neumann(_grad) on this layer's sides need at T tokens
+ * (one size covers all of them; T may be 0 for merge / Cayley-Neumann). */
+POET_API size_t poet_workspace_bytes(const poet_layer *L, int64_t T);
+
+/* Bytes of workspace poet_cayley_neumann_grad needs for one side alone. */
+POET_API size_t poet_side_workspace_bytes(const poet_side *side, int32_t dtype);
+
+/* ---------------------------------------------------------------- a1 / a8 */
+
+/* a1: materialize every primitive of one side from side->theta into
+ * side->state ([P1] Approach: truncated Neumann-series Cayley
+ * parameterization).  ws: device scratch of ws_bytes bytes (may be NULL when
+ * poet_workspace_bytes(.., 0) is 0).  Overwrites side->state only. */
+POET_API poet_status poet_cayley_neumann(const poet_side *side, int32_t dtype,
+                                void *ws, size_t ws_bytes, poet_stream stream);
+
+/* a8: gradient of <G, B(Q)> with respect to the packed parameters of every
+ * primitive of one side (chain rule through the map of poet_cayley_neumann).
+ * G: device float[nprim][size][size] (dL/dB of each primitive, row-major).
+ * dtheta: device float[nprim * size*(size-1)/2], overwritten.
+ * Requires side->state from poet_cayley_neumann of the same theta. */
+POET_API poet_status poet_cayley_neumann_grad(const poet_side *side, int32_t dtype,
+                                     const float *G, float *dtheta,
+                                     void *ws, size_t ws_bytes, poet_stream stream);
+
+/* ---------------------------------------------------------------- a2..a4 */
+
+/* Forward: y = R W0 P x for T tokens ([P1] Approach; [P2] Abstract).
+ * x: device T x n (dtype), y: device T x m (dtype), both row-major and
+ * contiguous.  saved: device, poet_saved_bytes(L, T) bytes, written here and
+ * read by poet_backward.  Requires both sides' state from
+ * poet_cayley_neumann and W0f from poet_prepare/poet_resample/poet_merge.
+ * T = 0 is allowed (nothing is launched). */
+POET_API poet_status poet_forward(const poet_layer *L, const void *x, int64_t T, void *y,
+                         void *saved, void *ws, size_t ws_bytes, poet_stream stream);
+
+/* ---------------------------------------------------------------- a5..a8 */
+
+/* Backward for upstream gradient dy (device T x m, dtype): writes
+ * dx = P^T W0^T R^T dy (device T x n, dtype) and the gradients of the loss
+ * with respect to both sides' packed parameters (device float, overwritten,
+ * same layout as theta).  W0 is fixed ([P1] Approach), so there is no dW0.
+ * saved: the buffer poet_forward filled for the same x and T. */
+POET_API poet_status poet_backward(const poet_layer *L, const void *saved, const void *dy,
+                          int64_t T, void *dx, float *dtheta_R, float *dtheta_P,
+                          void *ws, size_t ws_bytes, poet_stream stream);
+
+/* ---------------------------------------------------------------- a9 */
+
+/* Merge-then-reinitialize ([P1] Approach: "merged periodically"; Measured
+ * effects: merge-then-reinitialize frequency):  W0 <- R W0 P using the
+ * primitives currently materialized in the side states (the same ones the
+ * forward used), then theta <- 0 for both sides and both states are
+ * re-materialized, so R = P = I exactly for any k.  Updates W0 and W0f;
+ * the permutations are unchanged (call poet_resample next for new ones). */
+POET_API poet_status poet_merge(poet_layer *L, void *ws, size_t ws_bytes, poet_stream stream);
+
+/* ---------------------------------------------------------------- a10 */
+
+/* Draw both sides' permutations for L->epoch and rebuild W0f from W0.
+ * Use once on a fresh layer; does not change L->epoch. */
+POET_API poet_status poet_prepare(poet_layer *L, poet_stream stream);
+
+/* Reinitialize's new sampling ([P1] Approach, "sampled sub-block
+ * primitives"): L->epoch += 1 (host struct), then as poet_prepare. */
+POET_API poet_status poet_resample(poet_layer *L, poet_stream stream);
+
+/* The permutation draw on its own (a reading: the pages fix no generator).
+ * key_i = i-th output of SplitMix64 (Steele, Lea, Flood 2014) seeded with
+ *   h = sm(seed ^ sm((layer_id << 32) ^ (epoch << 1) ^ side)),
+ * where sm(z) is one SplitMix64 step from state z; perm lists 0..dim-1
+ * ordered by (key_i, i) ascending.  side: 0 = R, 1 = P.
+ * perm: device int32[dim], overwritten.  1 <= dim <= 16384. */
+POET_API poet_status poet_draw_perm(uint64_t seed, int32_t layer_id, int32_t side, int32_t epoch,
+                           int32_t dim, int32_t *perm, poet_stream stream);
+
+/* ---------------------------------------------------------------- utilities */
+
+/* Batched dense product on the library's GEMM engine, exported so that the
+ * engine can be tested on its own (it is the same code the layer uses):
+ *   C[b][i][j] = alpha * sum_l A(b,i,l) * B(b,j,l) (+ beta * C[b][i][j])
+ * A(b,i,l) = A[b*sAb + i*sAm + l*sAk], B(b,j,l) = B[b*sBb + j*sBn + l*sBk]
+ * (element strides), C row-major with row stride ldc and batch stride sCb.
+ * dtype: element type of A, B and C.  Returns POET_EINVAL on a bad shape. */
+POET_API poet_status poet_gemm(int32_t dtype, int32_t M, int32_t N, int32_t K, int32_t batch,
+                      const void *A, int64_t sAm, int64_t sAk, int64_t sAb,
+                      const void *B, int64_t sBn, int64_t sBk, int64_t sBb,
+                      void *C, int64_t ldc, int64_t sCb, float alpha, float beta,
+                      poet_stream stream);
+
+/* Which GEMM engine poet_gemm and the layer use for dtype:
+ * 1 = tcgen05 tensor cores (bf16 with a supported operand layout),
+ * 0 = CUDA-core FMA (float32, and layouts tcgen05 cannot read). */
+POET_API int32_t poet_gemm_engine(int32_t dtype);
+
+/* ---------------------------------------------------------------- accounting */
+
+/* One kind of work with its recorded launches, CUDA-event time and
+ * algorithmic flops / bytes (the operation's own operand sizes, not counters). */
+typedef struct {
+  char kind[32];
+  int64_t launches;
+  double ms;
+  double flop;
+  double bytes;
+} poet_trace_row;
+
+/* Kernels this library has launched since it was loaded (all devices). */
+POET_API int64_t poet_launch_count(void);
+
+/* Start (on != 0) or stop recording a CUDA event pair on the launch stream
+ * around each unit of work, tagged by kind.  Recording adds host calls
+ * between launches but no device work. */
+POET_API poet_status poet_trace_enable(int32_t on);
+
+/* Wait for the recorded events, aggregate them by kind into rows (at most
+ * max_rows, sorted by kind), forget them, and return the rows written. */
+POET_API int32_t poet_trace_read(poet_trace_row *rows, int32_t max_rows);
+
+/* Synchronize the stream, then read and clear the device status word.
+ * Returns POET_ETIMEOUT if a kernel gave up a bounded wait since the last
+ * call, POET_ECUDA on a CUDA error, POET_OK otherwise. */
+POET_API poet_status poet_sync_status(poet_stream stream);
+
+/* Text of the last failure on the calling thread ("" if none). */
+POET_API const char *poet_last_error(void);
+
+/* Library version string. */
+POET_API const char *poet_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* POET_H */

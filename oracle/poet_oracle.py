@@ -167,7 +167,11 @@ def forward(W0: np.ndarray, R: np.ndarray, P: np.ndarray, X: np.ndarray) -> np.n
 
 
 def restrict_blocks(M: np.ndarray, perm: np.ndarray, mode: int, b: int) -> np.ndarray:
-    """The primitive-shaped pieces of a d x d matrix: out[j] = M[I_j][:, I_j]."""
+    """The primitive-shaped pieces of a d x d matrix: out[j] = M[I_j][:, I_j]
+    (an empty stack when the side has no primitive, e.g. b > d)."""
+    nprim, size = side_shape(len(perm), mode, b)
+    if nprim == 0:
+        return np.zeros((0, size, size))
     return np.stack([M[np.ix_(idx, idx)] for idx in block_index_sets(perm, mode, b)])
 
 

@@ -1,0 +1,223 @@
+// Cayley-Neumann parameterization of the orthogonal primitives (a1) and its
+// gradient with respect to the packed skew parameters (a8).
+//
+// POET summary page, Approach and Limitations: each primitive is the Cayley
+// map (I+Q)(I-Q)^-1 of a skew-symmetric Q with the inverse replaced by its
+// Neumann series truncated after Q^k:  B = (I + Q)(I + Q + ... + Q^k).
+//
+// Forward, by Horner's rule on the series:
+//   S_1 = I + Q,  S_{l+1} = I + Q S_l (l = 1..k-1),  B = S_k + Q S_k
+// (k GEMMs of size^3; k = 0 gives B = I + Q).  Q and S_1..S_k are kept in
+// the side state for the backward.
+//
+// Backward (reverse-mode through the same recurrence), G = dL/dB:
+//   A_k = (I + Q)^T G = G - Q G            (Q^T = -Q)
+//   dQ  = G S_k^T + sum_{l=k-1..0} A_{l+1} S_l^T,   A_l = Q^T A_{l+1} = -Q A_{l+1}
+// with S_0 = I, then dtheta[a,c] = dQ[a,c] - dQ[c,a] (a < c) because
+// Q[a,c] = theta and Q[c,a] = -theta.  2k GEMMs.
+#include "poet_internal.cuh"
+
+namespace poet {
+namespace {
+
+// index of (a, c), a < c, in the row-major packed strict upper triangle
+__device__ __forceinline__ int64_t packed_index(int a, int c, int size) {
+  return int64_t(a) * size - int64_t(a) * (a + 1) / 2 + (c - a - 1);
+}
+
+template <typename T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+// Q and S_1 = I + Q (or B = I + Q when k == 0) for every primitive; padding is zero.
+template <typename T>
+__global__ void unpack_kernel(const float *__restrict__ theta, int nprim, int size, int ld,
+                              T *__restrict__ Q, T *__restrict__ IplusQ) {
+  const int64_t blk = int64_t(ld) * ld;
+  const int64_t total = blk * nprim;
+  const int64_t per = int64_t(size) * (size - 1) / 2;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    const int j = int(e / blk);
+    const int a = int((e % blk) / ld), c = int(e % ld);
+    float q = 0.f, eye = 0.f;
+    if (a < size && c < size) {
+      if (a < c) q = theta[j * per + packed_index(a, c, size)];
+      else if (a > c) q = -theta[j * per + packed_index(c, a, size)];
+      else eye = 1.f;
+    }
+    Q[e] = from_f<T>(q);
+    IplusQ[e] = from_f<T>(q + eye);
+  }
+}
+
+// dtheta[j][idx(a,c)] = D[a,c] - D[c,a] with D = dQ (+ A1 when given)
+__global__ void pack_grad_kernel(const float *__restrict__ dQ, const float *__restrict__ A1, int nprim, int size,
+                                 int ld, float *__restrict__ dtheta) {
+  const int64_t blk = int64_t(ld) * ld;
+  const int64_t per = int64_t(size) * (size - 1) / 2;
+  const int64_t total = int64_t(nprim) * size * size;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    const int j = int(e / (int64_t(size) * size));
+    const int a = int((e / size) % size), c = int(e % size);
+    if (a >= c) continue;
+    const int64_t ac = j * blk + int64_t(a) * ld + c, ca = j * blk + int64_t(c) * ld + a;
+    float v = dQ[ac] - dQ[ca];
+    if (A1) v += A1[ac] - A1[ca];
+    dtheta[j * per + packed_index(a, c, size)] = v;
+  }
+}
+
+// out[j][a][c] = G[j][a][c] for a, c < size (G dense [nprim][size][size]); zero padding up to ld
+__global__ void pad_blocks_kernel(const float *__restrict__ G, int nprim, int size, int ld, float *__restrict__ out) {
+  const int64_t blk = int64_t(ld) * ld;
+  const int64_t total = blk * nprim;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t j = e / blk;
+    const int a = int((e % blk) / ld), c = int(e % ld);
+    out[e] = (a < size && c < size) ? G[(j * size + a) * size + c] : 0.f;
+  }
+}
+
+__global__ void f32_to_bf16_kernel(const float *__restrict__ in, bf16 *__restrict__ out, int64_t n) {
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x)
+    out[e] = __float2bfloat16_rn(in[e]);
+}
+
+int grid_for(int64_t n, int threads) {
+  int64_t g = (n + threads - 1) / threads;
+  const int64_t cap = int64_t(num_sms()) * 8;
+  return int(g < 1 ? 1 : (g > cap ? cap : g));
+}
+
+// C_j = alpha * X_j Y_j (+ beta * Add_j) (+ diag I), all ld x ld primitives of one side.
+// transY: false -> B(n, l) = Y[l][n] (Y read column-wise, "MN-major");
+//         true  -> B(n, l) = Y[n][l] (C = X Y^T).
+Gemm prim_gemm(const SideGeom &g, int dtype, const void *X, const void *Y, bool transY, const char *tag) {
+  Gemm p;
+  p.tag = tag;
+  p.M = p.N = p.K = g.size;
+  p.batch = g.nprim;
+  p.dtype = dtype;
+  p.A = X; p.a_m = g.ld; p.a_k = 1; p.a_b = g.blk_elems();
+  p.B = Y;
+  if (transY) { p.b_n = g.ld; p.b_k = 1; } else { p.b_n = 1; p.b_k = g.ld; }
+  p.b_b = g.blk_elems();
+  return p;
+}
+
+}  // namespace
+
+poet_status pad_blocks(const float *G, const SideGeom &g, float *out, cudaStream_t st) {
+  const int64_t n = g.all_elems();
+  pad_blocks_kernel<<<grid_for(n, 256), 256, 0, st>>>(G, g.nprim, g.size, g.ld, out);
+  count_launch();
+  return launch_status("pad blocks");
+}
+
+size_t cnp_scratch_bytes(const SideGeom &g, int dtype) {
+  const size_t f = align256(size_t(g.all_elems()) * 4);
+  const size_t d = align256(size_t(g.all_elems()) * esize(dtype));
+  // G operand copy (dtype), A ping-pong (f32 + dtype each), dQ (f32)
+  return d + 2 * (f + d) + f;
+}
+
+poet_status cnp_forward(const poet_side *side, const SideGeom &g, int dtype, cudaStream_t st) {
+  if (g.nprim == 0) return POET_OK;
+  const StateLayout L = state_layout(g, dtype);
+  char *base = static_cast<char *>(side->state);
+  void *R = base + L.R, *Q = base + L.Q;
+  const int64_t n = g.all_elems();
+  void *first = g.k == 0 ? R : static_cast<void *>(base + L.S1);
+  if (dtype == POET_BF16)
+    unpack_kernel<bf16><<<grid_for(n, 256), 256, 0, st>>>(side->theta, g.nprim, g.size, g.ld, static_cast<bf16 *>(Q),
+                                                          static_cast<bf16 *>(first));
+  else
+    unpack_kernel<float><<<grid_for(n, 256), 256, 0, st>>>(side->theta, g.nprim, g.size, g.ld, static_cast<float *>(Q),
+                                                           static_cast<float *>(first));
+  count_launch();
+  POET_TRY(launch_status("cnp unpack"));
+  for (int l = 1; l <= g.k; ++l) {
+    void *S = base + L.S1 + size_t(l - 1) * L.term;
+    Gemm p = prim_gemm(g, dtype, Q, S, false, "cnp_fwd");  // Q S_l
+    if (l < g.k) {                               // S_{l+1} = I + Q S_l
+      p.diag = 1.f;
+      p.outD = base + L.S1 + size_t(l) * L.term;
+    } else {                                     // B = S_k + Q S_k
+      p.add = S; p.add_dtype = dtype; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 1.f;
+      p.outD = R;
+    }
+    p.od_m = g.ld; p.od_b = g.blk_elems();
+    POET_TRY(gemm_run(p, st));
+  }
+  return POET_OK;
+}
+
+poet_status cnp_backward(const poet_side *side, const SideGeom &g, int dtype, const float *G, float *dtheta,
+                         void *scratch, cudaStream_t st) {
+  if (g.nprim == 0 || g.size < 2) return POET_OK;
+  const StateLayout L = state_layout(g, dtype);
+  char *base = static_cast<char *>(side->state);
+  const void *Q = base + L.Q;
+  const int64_t n = g.all_elems();
+  if (g.k == 0) {  // B = I + Q  ->  dQ = G
+    pack_grad_kernel<<<grid_for(n, 256), 256, 0, st>>>(G, nullptr, g.nprim, g.size, g.ld, dtheta);
+    count_launch();
+    return launch_status("cnp pack");
+  }
+  const size_t fb = align256(size_t(n) * 4), db = align256(size_t(n) * esize(dtype));
+  char *s = static_cast<char *>(scratch);
+  const void *Gop;
+  if (dtype == POET_BF16) {
+    f32_to_bf16_kernel<<<grid_for(n, 256), 256, 0, st>>>(G, reinterpret_cast<bf16 *>(s), n);
+    count_launch();
+    POET_TRY(launch_status("cnp G to bf16"));
+    Gop = s;
+  } else {
+    Gop = G;
+  }
+  s += db;
+  float *Af[2] = {reinterpret_cast<float *>(s), reinterpret_cast<float *>(s + fb + db)};
+  void *Ad[2] = {s + fb, s + 2 * fb + db};
+  if (dtype != POET_BF16) { Ad[0] = Af[0]; Ad[1] = Af[1]; }
+  float *dQ = reinterpret_cast<float *>(s + 2 * (fb + db));
+  auto S = [&](int l) -> const void * { return base + L.S1 + size_t(l - 1) * L.term; };
+
+  // A_k = G - Q G
+  {
+    Gemm p = prim_gemm(g, dtype, Q, Gop, false, "cnp_bwd");
+    p.alpha = -1.f;
+    p.add = G; p.add_dtype = POET_F32; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 1.f;
+    p.outF = Af[0]; p.of_m = g.ld; p.of_b = g.blk_elems();
+    if (dtype == POET_BF16) { p.outD = Ad[0]; p.od_m = g.ld; p.od_b = g.blk_elems(); }
+    POET_TRY(gemm_run(p, st));
+  }
+  // dQ = G S_k^T
+  {
+    Gemm p = prim_gemm(g, dtype, Gop, S(g.k), true, "cnp_bwd");
+    p.outF = dQ; p.of_m = g.ld; p.of_b = g.blk_elems();
+    POET_TRY(gemm_run(p, st));
+  }
+  int cur = 0;  // A_{l+1} lives in slot cur
+  for (int l = g.k - 1; l >= 1; --l) {
+    {  // dQ += A_{l+1} S_l^T
+      Gemm p = prim_gemm(g, dtype, Ad[cur], S(l), true, "cnp_bwd");
+      p.add = dQ; p.add_dtype = POET_F32; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 1.f;
+      p.outF = dQ; p.of_m = g.ld; p.of_b = g.blk_elems();
+      POET_TRY(gemm_run(p, st));
+    }
+    {  // A_l = -Q A_{l+1}
+      Gemm p = prim_gemm(g, dtype, Q, Ad[cur], false, "cnp_bwd");
+      p.alpha = -1.f;
+      p.outF = Af[cur ^ 1]; p.of_m = g.ld; p.of_b = g.blk_elems();
+      if (dtype == POET_BF16) { p.outD = Ad[cur ^ 1]; p.od_m = g.ld; p.od_b = g.blk_elems(); }
+      POET_TRY(gemm_run(p, st));
+    }
+    cur ^= 1;
+  }
+  // dQ += A_1 S_0^T = A_1, folded into the packing
+  pack_grad_kernel<<<grid_for(n, 256), 256, 0, st>>>(dQ, Af[cur], g.nprim, g.size, g.ld, dtheta);
+  count_launch();
+  return launch_status("cnp pack");
+}
+
+}  // namespace poet

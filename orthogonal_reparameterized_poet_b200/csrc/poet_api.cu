@@ -1,0 +1,557 @@
+// libpoet C ABI: argument validation and the order of the steps of the POET
+// layer y = R W0 P x (POET summary page, Approach).  Every arithmetic step
+// runs in this library's CUDA kernels; nothing falls back to the host.
+//
+// Data flow of one layer (frame = indices ordered by the side's permutation,
+// see poet.h), T tokens, q_R / q_P primitives of size s_R / s_P:
+//   forward   x --gather(P.perm)--> xf --blocks P_j--> uf --W0f--> vf
+//             --blocks R_j--> yf --scatter(R.perm)--> y           (saved: xf, vf)
+//   backward  dy --gather(R.perm)--> dyf --blocks R_j^T--> dvf --W0f^T--> duf
+//             --blocks P_j^T--> dxf --scatter(P.perm)--> dx
+//             G_R[j] = dyf_j^T vf_j,  G_P[j] = duf_j^T xf_j  (summed over tokens)
+//             dtheta = Cayley-Neumann backward of G
+// Frame indices past q*s (the leftover identity part) pass through unchanged.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "poet_internal.cuh"
+
+namespace poet {
+
+// ------------------------------------------------------------------ errors
+
+static thread_local char g_last_error[512] = "";
+
+void set_error(const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+}
+void clear_error() { g_last_error[0] = 0; }
+
+poet_status launch_status(const char *what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("%s: launch failed: %s", what, cudaGetErrorString(e));
+    return POET_ECUDA;
+  }
+  return POET_OK;
+}
+
+__device__ unsigned g_errword;
+
+unsigned *device_errword() {
+  static std::mutex mu;
+  static std::vector<unsigned *> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (int(cache.size()) <= dev) cache.resize(dev + 1, nullptr);
+  if (!cache[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_errword) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<unsigned *>(p);
+  }
+  return cache[dev];
+}
+
+int num_sms() {
+  static std::mutex mu;
+  static std::vector<int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (int(cache.size()) <= dev) cache.resize(dev + 1, 0);
+  if (!cache[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+// ------------------------------------------------------------------ geometry
+
+bool side_geom(const poet_side *s, SideGeom *g) {
+  if (!s || s->dim < 1 || s->dim > 16384 || s->k < 0 || s->k > 16) return false;
+  SideGeom r;
+  if (s->mode == POET_FS) {
+    r.size = s->dim / 2;
+    r.nprim = r.size >= 1 ? 1 : 0;
+  } else if (s->mode == POET_BS) {
+    if (s->b < 1) return false;
+    r.size = s->b;
+    r.nprim = s->dim / s->b;
+  } else {
+    return false;
+  }
+  if (r.nprim == 0) r.size = 0;
+  r.ld = int(round_up(r.size, 8));
+  r.covered = r.nprim * r.size;
+  r.k = s->k;
+  *g = r;
+  return true;
+}
+
+StateLayout state_layout(const SideGeom &g, int dtype) {
+  StateLayout L;
+  L.term = align256(size_t(g.all_elems()) * esize(dtype));
+  L.R = 0;
+  L.Q = L.term;
+  L.S1 = 2 * L.term;
+  L.bytes = size_t(2 + g.k) * L.term;
+  return L;
+}
+
+namespace {
+
+bool aligned256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+bool aligned_elem(const void *p, int dtype) { return (reinterpret_cast<uintptr_t>(p) % esize(dtype)) == 0; }
+
+struct LayerGeom {
+  SideGeom R, P;
+  int64_t m = 0, n = 0, ldm = 0, ldn = 0;
+  int dtype = 0;
+};
+
+poet_status check_layer(const poet_layer *L, LayerGeom *lg, bool need_state) {
+  POET_REQUIRE(L != nullptr, "layer is NULL");
+  POET_REQUIRE(L->m >= 1 && L->n >= 1 && L->m <= 16384 && L->n <= 16384, "layer shape %lld x %lld outside [1,16384]^2",
+               (long long)L->m, (long long)L->n);
+  POET_REQUIRE(L->dtype == POET_F32 || L->dtype == POET_BF16, "dtype %d is not POET_F32 or POET_BF16", L->dtype);
+  POET_REQUIRE(L->R.dim == L->m && L->P.dim == L->n, "side dims (%d, %d) do not match W0 (%lld x %lld)", L->R.dim,
+               L->P.dim, (long long)L->m, (long long)L->n);
+  POET_REQUIRE(side_geom(&L->R, &lg->R), "malformed R side (mode %d, b %d, k %d)", L->R.mode, L->R.b, L->R.k);
+  POET_REQUIRE(side_geom(&L->P, &lg->P), "malformed P side (mode %d, b %d, k %d)", L->P.mode, L->P.b, L->P.k);
+  POET_REQUIRE(L->layer_id >= 0 && L->epoch >= 0 && L->reserved == 0, "layer_id/epoch must be >= 0, reserved 0");
+  POET_REQUIRE(L->R.perm && L->P.perm, "perm pointers must not be NULL");
+  POET_REQUIRE(L->W0 && aligned_elem(L->W0, L->dtype), "W0 is NULL or misaligned");
+  POET_REQUIRE(L->W0f && aligned256(L->W0f), "W0f is NULL or not 256-byte aligned");
+  if (need_state) {
+    POET_REQUIRE(lg->R.nprim == 0 || (L->R.state && aligned256(L->R.state)), "R.state is NULL or not 256-byte aligned");
+    POET_REQUIRE(lg->P.nprim == 0 || (L->P.state && aligned256(L->P.state)), "P.state is NULL or not 256-byte aligned");
+  }
+  lg->m = L->m;
+  lg->n = L->n;
+  lg->ldm = frame_ld(L->m);
+  lg->ldn = frame_ld(L->n);
+  lg->dtype = L->dtype;
+  return POET_OK;
+}
+
+struct WsLayout {
+  size_t act1 = 0, act2 = 0, act3 = 0, GR = 0, GP = 0, cnp = 0, Z = 0, bytes = 0;
+};
+
+WsLayout ws_layout(const LayerGeom &lg, int64_t T) {
+  WsLayout w;
+  const size_t es = esize(lg.dtype);
+  const int64_t ldmax = lg.ldm > lg.ldn ? lg.ldm : lg.ldn;
+  size_t off = 0;
+  w.act1 = off; off += align256(size_t(T) * ldmax * es);
+  w.act2 = off; off += align256(size_t(T) * lg.ldm * es);
+  w.act3 = off; off += align256(size_t(T) * lg.ldn * es);
+  w.GR = off; off += align256(size_t(lg.R.all_elems()) * 4);
+  w.GP = off; off += align256(size_t(lg.P.all_elems()) * 4);
+  w.cnp = off;
+  const size_t cr = cnp_scratch_bytes(lg.R, lg.dtype), cp = cnp_scratch_bytes(lg.P, lg.dtype);
+  off += cr > cp ? cr : cp;
+  w.Z = off; off += align256(size_t(lg.m) * lg.ldn * es);
+  w.bytes = off;
+  return w;
+}
+
+size_t side_ws_bytes(const SideGeom &g, int dtype) {
+  return align256(size_t(g.all_elems()) * 4) + cnp_scratch_bytes(g, dtype);
+}
+
+// token-parallel block-diagonal product in the frame:
+//   C[t][j*s + a] = sum_c X[t][j*s + c] * (trans ? Blk_j[c][a] : Blk_j[a][c])
+Gemm blockdiag(const SideGeom &g, int dtype, int64_t T, const void *X, int64_t ldx, const void *Blk, bool trans,
+               void *C, int64_t ldc) {
+  Gemm p;
+  p.tag = trans ? "blk_bwd" : "blk_fwd";
+  p.M = int(T); p.N = g.size; p.K = g.size; p.batch = g.nprim;
+  p.dtype = dtype;
+  p.A = X; p.a_m = ldx; p.a_k = 1; p.a_b = g.size;
+  p.B = Blk;
+  if (trans) { p.b_n = 1; p.b_k = g.ld; } else { p.b_n = g.ld; p.b_k = 1; }
+  p.b_b = g.blk_elems();
+  p.outD = C; p.od_m = ldc; p.od_b = g.size;
+  return p;
+}
+
+// per-primitive gradient summed over tokens:
+//   Gout[j][a][c] += sum_t D[t][j*s + a] * V[t][j*s + c]
+Gemm blockgrad(const SideGeom &g, int dtype, int64_t T, const void *D, const void *V, int64_t ld, float *Gout) {
+  Gemm p;
+  p.tag = "blk_grad";
+  p.M = g.size; p.N = g.size; p.K = int(T); p.batch = g.nprim;
+  p.dtype = dtype;
+  p.A = D; p.a_m = 1; p.a_k = ld; p.a_b = g.size;
+  p.B = V; p.b_n = 1; p.b_k = ld; p.b_b = g.size;
+  p.outF = Gout; p.of_m = g.ld; p.of_b = g.blk_elems();
+  p.atomic = true;
+  return p;
+}
+
+const void *state_R(const poet_side *s, const SideGeom &g, int dtype) {
+  return static_cast<const char *>(s->state) + state_layout(g, dtype).R;
+}
+
+}  // namespace
+
+poet_status gemm_run(const Gemm &g, cudaStream_t st) {
+  if (g.M <= 0 || g.N <= 0 || g.batch <= 0) return POET_OK;
+  const double mnb = double(g.M) * g.N * g.batch;
+  const double bytes = double(esize(g.dtype)) * (double(g.M) + g.N) * g.K * g.batch +
+                       mnb * ((g.outF ? 4.0 : 0.0) + (g.outD ? double(esize(g.dtype)) : 0.0) +
+                              (g.add ? double(esize(g.add_dtype)) : 0.0));
+  TraceScope ts(g.tag, 2.0 * mnb * g.K, bytes, st);
+  if (gemm_tc_enabled() && gemm_tc_supported(g)) return gemm_tc(g, st);
+  return gemm_simt(g, st);
+}
+
+}  // namespace poet
+
+using namespace poet;
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+const char *poet_last_error(void) { return g_last_error; }
+
+const char *poet_version(void) { return "libpoet 0.1 (sm_100a)"; }
+
+size_t poet_side_state_bytes(const poet_side *side, int32_t dtype) {
+  SideGeom g;
+  if (!side_geom(side, &g) || (dtype != POET_F32 && dtype != POET_BF16)) return 0;
+  return state_layout(g, dtype).bytes;
+}
+
+size_t poet_frame_bytes(const poet_layer *L) {
+  if (!L || L->m < 1 || L->n < 1) return 0;
+  return align256(size_t(L->m) * frame_ld(L->n) * esize(L->dtype));
+}
+
+size_t poet_saved_bytes(const poet_layer *L, int64_t T) {
+  if (!L || L->m < 1 || L->n < 1 || T < 0) return 0;
+  const size_t es = esize(L->dtype);
+  return align256(size_t(T) * frame_ld(L->n) * es) + align256(size_t(T) * frame_ld(L->m) * es);
+}
+
+size_t poet_workspace_bytes(const poet_layer *L, int64_t T) {
+  LayerGeom lg;
+  if (T < 0 || check_layer(L, &lg, false) != POET_OK) {
+    clear_error();
+    // shape-only fallback so that sizes can be queried before pointers exist
+    if (!L || T < 0) return 0;
+    if (!side_geom(&L->R, &lg.R) || !side_geom(&L->P, &lg.P)) return 0;
+    lg.m = L->m; lg.n = L->n; lg.ldm = frame_ld(L->m); lg.ldn = frame_ld(L->n); lg.dtype = L->dtype;
+  }
+  return ws_layout(lg, T).bytes;
+}
+
+size_t poet_side_workspace_bytes(const poet_side *side, int32_t dtype) {
+  SideGeom g;
+  if (!side_geom(side, &g) || (dtype != POET_F32 && dtype != POET_BF16)) return 0;
+  return side_ws_bytes(g, dtype);
+}
+
+poet_status poet_cayley_neumann(const poet_side *side, int32_t dtype, void *ws, size_t ws_bytes, poet_stream stream) {
+  (void)ws; (void)ws_bytes;
+  clear_error();
+  SideGeom g;
+  POET_REQUIRE(side_geom(side, &g), "poet_cayley_neumann: malformed side");
+  POET_REQUIRE(dtype == POET_F32 || dtype == POET_BF16, "poet_cayley_neumann: bad dtype %d", dtype);
+  if (g.nprim == 0) return POET_OK;
+  POET_REQUIRE((side->theta || g.packed_per() == 0) && side->state && aligned256(side->state),
+               "poet_cayley_neumann: theta/state NULL or state not 256-byte aligned");
+  return cnp_forward(side, g, dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+poet_status poet_cayley_neumann_grad(const poet_side *side, int32_t dtype, const float *G, float *dtheta, void *ws,
+                                     size_t ws_bytes, poet_stream stream) {
+  clear_error();
+  SideGeom g;
+  POET_REQUIRE(side_geom(side, &g), "poet_cayley_neumann_grad: malformed side");
+  POET_REQUIRE(dtype == POET_F32 || dtype == POET_BF16, "poet_cayley_neumann_grad: bad dtype %d", dtype);
+  if (g.nprim == 0 || g.size < 2) return POET_OK;
+  POET_REQUIRE(side->state && aligned256(side->state) && G && dtheta, "poet_cayley_neumann_grad: NULL argument");
+  const size_t need = side_ws_bytes(g, dtype);
+  if (ws_bytes < need || !ws || !aligned256(ws)) {
+    set_error("poet_cayley_neumann_grad: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, need);
+    return POET_ENOMEM_WS;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float *Gpad = static_cast<float *>(ws);
+  POET_TRY(pad_blocks(G, g, Gpad, st));
+  void *scratch = static_cast<char *>(ws) + align256(size_t(g.all_elems()) * 4);
+  return cnp_backward(side, g, dtype, Gpad, dtheta, scratch, st);
+}
+
+poet_status poet_forward(const poet_layer *L, const void *x, int64_t T, void *y, void *saved, void *ws,
+                         size_t ws_bytes, poet_stream stream) {
+  clear_error();
+  LayerGeom lg;
+  POET_TRY(check_layer(L, &lg, true));
+  POET_REQUIRE(T >= 0 && T <= (int64_t(1) << 31) - 1, "poet_forward: T=%lld out of range", (long long)T);
+  if (T == 0) return POET_OK;
+  POET_REQUIRE(x && y && aligned_elem(x, lg.dtype) && aligned_elem(y, lg.dtype), "poet_forward: x/y NULL or misaligned");
+  POET_REQUIRE(saved && aligned256(saved), "poet_forward: saved NULL or not 256-byte aligned");
+  const WsLayout w = ws_layout(lg, T);
+  if (!ws || ws_bytes < w.bytes || !aligned256(ws)) {
+    set_error("poet_forward: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, w.bytes);
+    return POET_ENOMEM_WS;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int dt = lg.dtype;
+  const size_t es = esize(dt);
+  char *sv = static_cast<char *>(saved);
+  void *xf = sv;
+  void *vf = sv + align256(size_t(T) * lg.ldn * es);
+  char *wb = static_cast<char *>(ws);
+  void *uf = wb + w.act1;
+  void *yf = wb + w.act2;
+  const SideGeom &gR = lg.R, &gP = lg.P;
+
+  // a2: gather x into the P frame; the identity tail goes straight to uf
+  const bool tailP = gP.nprim > 0 && gP.covered < lg.n;
+  POET_TRY(gather_cols(dt, x, lg.n, nullptr, T, int(lg.n), L->P.perm, xf, lg.ldn, tailP ? uf : nullptr, lg.ldn,
+                       gP.covered, st));
+  const void *u = xf;
+  if (gP.nprim > 0) {
+    POET_TRY(gemm_run(blockdiag(gP, dt, T, xf, lg.ldn, state_R(&L->P, gP, dt), false, uf, lg.ldn), st));
+    u = uf;
+  }
+  // a3: v = u W0f^T
+  {
+    Gemm p;
+    p.tag = "w0_fwd";
+    p.M = int(T); p.N = int(lg.m); p.K = int(lg.n); p.dtype = dt;
+    p.A = u; p.a_m = lg.ldn; p.a_k = 1;
+    p.B = L->W0f; p.b_n = lg.ldn; p.b_k = 1;
+    p.outD = vf; p.od_m = lg.ldm;
+    POET_TRY(gemm_run(p, st));
+  }
+  // a4: R blocks, then scatter to natural order (tail straight from vf)
+  const void *ysrc = vf;
+  if (gR.nprim > 0) {
+    POET_TRY(gemm_run(blockdiag(gR, dt, T, vf, lg.ldm, state_R(&L->R, gR, dt), false, yf, lg.ldm), st));
+    ysrc = yf;
+  }
+  return scatter_cols(dt, ysrc, lg.ldm, vf, lg.ldm, gR.covered, T, int(lg.m), L->R.perm, y, lg.m, nullptr, st);
+}
+
+poet_status poet_backward(const poet_layer *L, const void *saved, const void *dy, int64_t T, void *dx,
+                          float *dtheta_R, float *dtheta_P, void *ws, size_t ws_bytes, poet_stream stream) {
+  clear_error();
+  LayerGeom lg;
+  POET_TRY(check_layer(L, &lg, true));
+  POET_REQUIRE(T >= 0 && T <= (int64_t(1) << 31) - 1, "poet_backward: T=%lld out of range", (long long)T);
+  const SideGeom &gR = lg.R, &gP = lg.P;
+  POET_REQUIRE(gR.nprim == 0 || gR.size < 2 || dtheta_R, "poet_backward: dtheta_R is NULL");
+  POET_REQUIRE(gP.nprim == 0 || gP.size < 2 || dtheta_P, "poet_backward: dtheta_P is NULL");
+  const WsLayout w = ws_layout(lg, T);
+  if (!ws || ws_bytes < w.bytes || !aligned256(ws)) {
+    set_error("poet_backward: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, w.bytes);
+    return POET_ENOMEM_WS;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int dt = lg.dtype;
+  const size_t es = esize(dt);
+  char *wb = static_cast<char *>(ws);
+  float *GR = reinterpret_cast<float *>(wb + w.GR);
+  float *GP = reinterpret_cast<float *>(wb + w.GP);
+  if (T > 0) {
+    POET_REQUIRE(dy && dx && aligned_elem(dy, dt) && aligned_elem(dx, dt), "poet_backward: dy/dx NULL or misaligned");
+    POET_REQUIRE(saved && aligned256(saved), "poet_backward: saved NULL or not 256-byte aligned");
+    const char *sv = static_cast<const char *>(saved);
+    const void *xf = sv;
+    const void *vf = sv + align256(size_t(T) * lg.ldn * es);
+    void *dyf = wb + w.act1, *dvf = wb + w.act2, *duf = wb + w.act3, *dxf = wb + w.act1;
+
+    // a5: gather dy into the R frame (tail straight to dvf), dv = R^T dy, G_R
+    const bool tailR = gR.nprim > 0 && gR.covered < lg.m;
+    POET_TRY(gather_cols(dt, dy, lg.m, nullptr, T, int(lg.m), L->R.perm, dyf, lg.ldm, tailR ? dvf : nullptr, lg.ldm,
+                         gR.covered, st));
+    const void *dv = dyf;
+    if (gR.nprim > 0) {
+      POET_TRY(gemm_run(blockdiag(gR, dt, T, dyf, lg.ldm, state_R(&L->R, gR, dt), true, dvf, lg.ldm), st));
+      dv = dvf;
+      POET_CUDA_TRY(cudaMemsetAsync(GR, 0, size_t(gR.all_elems()) * 4, st));
+      POET_TRY(gemm_run(blockgrad(gR, dt, T, dyf, vf, lg.ldm, GR), st));
+    }
+    // a6: du = dv W0f
+    {
+      Gemm p;
+      p.tag = "w0_bwd";
+      p.M = int(T); p.N = int(lg.n); p.K = int(lg.m); p.dtype = dt;
+      p.A = dv; p.a_m = lg.ldm; p.a_k = 1;
+      p.B = L->W0f; p.b_n = 1; p.b_k = lg.ldn;
+      p.outD = duf; p.od_m = lg.ldn;
+      POET_TRY(gemm_run(p, st));
+    }
+    // a7: G_P, dx = P^T du, scatter (tail straight from du)
+    const void *dxsrc = duf;
+    if (gP.nprim > 0) {
+      POET_CUDA_TRY(cudaMemsetAsync(GP, 0, size_t(gP.all_elems()) * 4, st));
+      POET_TRY(gemm_run(blockgrad(gP, dt, T, duf, xf, lg.ldn, GP), st));
+      POET_TRY(gemm_run(blockdiag(gP, dt, T, duf, lg.ldn, state_R(&L->P, gP, dt), true, dxf, lg.ldn), st));
+      dxsrc = dxf;
+    }
+    POET_TRY(scatter_cols(dt, dxsrc, lg.ldn, duf, lg.ldn, gP.covered, T, int(lg.n), L->P.perm, dx, lg.n, nullptr, st));
+  } else {
+    if (gR.nprim > 0) POET_CUDA_TRY(cudaMemsetAsync(GR, 0, size_t(gR.all_elems()) * 4, st));
+    if (gP.nprim > 0) POET_CUDA_TRY(cudaMemsetAsync(GP, 0, size_t(gP.all_elems()) * 4, st));
+  }
+  // a8: through the Cayley-Neumann map to the packed parameters
+  void *scratch = wb + w.cnp;
+  if (gR.nprim > 0 && gR.size >= 2) POET_TRY(cnp_backward(&L->R, gR, dt, GR, dtheta_R, scratch, st));
+  if (gP.nprim > 0 && gP.size >= 2) POET_TRY(cnp_backward(&L->P, gP, dt, GP, dtheta_P, scratch, st));
+  return POET_OK;
+}
+
+poet_status poet_prepare(poet_layer *L, poet_stream stream) {
+  clear_error();
+  LayerGeom lg;
+  POET_TRY(check_layer(L, &lg, false));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  POET_TRY(draw_perm_dev(L->seed, L->layer_id, 0, L->epoch, int(lg.m), L->R.perm, st));
+  POET_TRY(draw_perm_dev(L->seed, L->layer_id, 1, L->epoch, int(lg.n), L->P.perm, st));
+  // W0f[i][j] = W0[R.perm[i]][P.perm[j]]
+  return gather_cols(lg.dtype, L->W0, lg.n, L->R.perm, lg.m, int(lg.n), L->P.perm, L->W0f, lg.ldn, nullptr, 0,
+                     int(lg.n), st);
+}
+
+poet_status poet_resample(poet_layer *L, poet_stream stream) {
+  clear_error();
+  POET_REQUIRE(L != nullptr, "poet_resample: layer is NULL");
+  POET_REQUIRE(L->epoch >= 0 && L->epoch < 0x7FFFFFFF, "poet_resample: epoch %d cannot advance", L->epoch);
+  L->epoch += 1;
+  poet_status s = poet_prepare(L, stream);
+  if (s != POET_OK) L->epoch -= 1;
+  return s;
+}
+
+poet_status poet_draw_perm(uint64_t seed, int32_t layer_id, int32_t side, int32_t epoch, int32_t dim, int32_t *perm,
+                           poet_stream stream) {
+  clear_error();
+  return draw_perm_dev(seed, layer_id, side, epoch, dim, perm, reinterpret_cast<cudaStream_t>(stream));
+}
+
+poet_status poet_merge(poet_layer *L, void *ws, size_t ws_bytes, poet_stream stream) {
+  clear_error();
+  LayerGeom lg;
+  POET_TRY(check_layer(L, &lg, true));
+  POET_REQUIRE(lg.R.nprim == 0 || lg.R.packed_per() == 0 || L->R.theta, "poet_merge: R.theta is NULL");
+  POET_REQUIRE(lg.P.nprim == 0 || lg.P.packed_per() == 0 || L->P.theta, "poet_merge: P.theta is NULL");
+  const WsLayout w = ws_layout(lg, 0);
+  if (!ws || ws_bytes < w.bytes || !aligned256(ws)) {
+    set_error("poet_merge: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, w.bytes);
+    return POET_ENOMEM_WS;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int dt = lg.dtype;
+  const size_t es = esize(dt);
+  const SideGeom &gR = lg.R, &gP = lg.P;
+  char *W0f = static_cast<char *>(L->W0f);
+  char *Z = static_cast<char *>(ws) + w.Z;
+  const int64_t ldw = lg.ldn;
+  if (gR.nprim > 0 || gP.nprim > 0) {
+    // Z = blockdiag(R) W0f  (rows of each R primitive; leftover rows copied)
+    const char *src = W0f;
+    if (gR.nprim > 0) {
+      Gemm p;
+      p.tag = "merge";
+      p.M = gR.size; p.N = int(lg.n); p.K = gR.size; p.batch = gR.nprim; p.dtype = dt;
+      p.A = state_R(&L->R, gR, dt); p.a_m = gR.ld; p.a_k = 1; p.a_b = gR.blk_elems();
+      p.B = W0f; p.b_n = 1; p.b_k = ldw; p.b_b = int64_t(gR.size) * ldw;
+      p.outD = Z; p.od_m = ldw; p.od_b = int64_t(gR.size) * ldw;
+      POET_TRY(gemm_run(p, st));
+      if (gR.covered < lg.m)
+        POET_CUDA_TRY(cudaMemcpyAsync(Z + size_t(gR.covered) * ldw * es, W0f + size_t(gR.covered) * ldw * es,
+                                      size_t(lg.m - gR.covered) * ldw * es, cudaMemcpyDeviceToDevice, st));
+      src = Z;
+    }
+    // W0f = src blockdiag(P)  (columns of each P primitive; leftover columns copied)
+    if (gP.nprim > 0) {
+      Gemm p;
+      p.tag = "merge";
+      p.M = int(lg.m); p.N = gP.size; p.K = gP.size; p.batch = gP.nprim; p.dtype = dt;
+      p.A = src; p.a_m = ldw; p.a_k = 1; p.a_b = gP.size;
+      p.B = state_R(&L->P, gP, dt); p.b_n = 1; p.b_k = gP.ld; p.b_b = gP.blk_elems();
+      p.outD = W0f; p.od_m = ldw; p.od_b = gP.size;
+      if (src == W0f) {  // R had no primitives: the product cannot be written in place
+        POET_CUDA_TRY(cudaMemcpyAsync(Z, W0f, size_t(lg.m) * ldw * es, cudaMemcpyDeviceToDevice, st));
+        p.A = Z;
+        src = Z;
+      }
+      POET_TRY(gemm_run(p, st));
+      if (gP.covered < lg.n)
+        POET_CUDA_TRY(cudaMemcpy2DAsync(W0f + size_t(gP.covered) * es, ldw * es, src + size_t(gP.covered) * es,
+                                        ldw * es, size_t(lg.n - gP.covered) * es, size_t(lg.m),
+                                        cudaMemcpyDeviceToDevice, st));
+    } else {
+      POET_CUDA_TRY(cudaMemcpyAsync(W0f, Z, size_t(lg.m) * ldw * es, cudaMemcpyDeviceToDevice, st));
+    }
+    // W0[R.perm[i]][P.perm[j]] = W0f[i][j]
+    POET_TRY(scatter_cols(dt, W0f, ldw, W0f, ldw, int(lg.n), lg.m, int(lg.n), L->P.perm, L->W0, lg.n, L->R.perm, st));
+  }
+  // reinitialize: theta <- 0 and re-materialize (every primitive becomes I)
+  if (gR.nprim > 0) {
+    if (gR.packed_per() > 0)
+      POET_CUDA_TRY(cudaMemsetAsync(L->R.theta, 0, size_t(gR.nprim) * gR.packed_per() * 4, st));
+    POET_TRY(cnp_forward(&L->R, gR, dt, st));
+  }
+  if (gP.nprim > 0) {
+    if (gP.packed_per() > 0)
+      POET_CUDA_TRY(cudaMemsetAsync(L->P.theta, 0, size_t(gP.nprim) * gP.packed_per() * 4, st));
+    POET_TRY(cnp_forward(&L->P, gP, dt, st));
+  }
+  return POET_OK;
+}
+
+poet_status poet_gemm(int32_t dtype, int32_t M, int32_t N, int32_t K, int32_t batch, const void *A, int64_t sAm,
+                      int64_t sAk, int64_t sAb, const void *B, int64_t sBn, int64_t sBk, int64_t sBb, void *C,
+                      int64_t ldc, int64_t sCb, float alpha, float beta, poet_stream stream) {
+  clear_error();
+  POET_REQUIRE(dtype == POET_F32 || dtype == POET_BF16, "poet_gemm: bad dtype %d", dtype);
+  POET_REQUIRE(M >= 0 && N >= 0 && K >= 0 && batch >= 0, "poet_gemm: negative size");
+  if (M == 0 || N == 0 || batch == 0) return POET_OK;
+  POET_REQUIRE(A && B && C && ldc >= N, "poet_gemm: NULL operand or ldc < N");
+  Gemm p;
+  p.M = M; p.N = N; p.K = K; p.batch = batch; p.dtype = dtype;
+  p.A = A; p.a_m = sAm; p.a_k = sAk; p.a_b = sAb;
+  p.B = B; p.b_n = sBn; p.b_k = sBk; p.b_b = sBb;
+  p.alpha = alpha;
+  if (beta != 0.f) { p.add = C; p.add_dtype = dtype; p.add_m = ldc; p.add_b = sCb; p.beta = beta; }
+  p.outD = C; p.od_m = ldc; p.od_b = sCb;
+  return gemm_run(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int32_t poet_gemm_engine(int32_t dtype) { return (dtype == POET_BF16 && gemm_tc_enabled()) ? 1 : 0; }
+
+poet_status poet_sync_status(poet_stream stream) {
+  clear_error();
+  POET_CUDA_TRY(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  unsigned *ew = device_errword();
+  POET_REQUIRE(ew != nullptr, "poet_sync_status: no device status word");
+  unsigned word = 0;
+  POET_CUDA_TRY(cudaMemcpy(&word, ew, sizeof(word), cudaMemcpyDeviceToHost));
+  if (word) {
+    unsigned zero = 0;
+    POET_CUDA_TRY(cudaMemcpy(ew, &zero, sizeof(zero), cudaMemcpyHostToDevice));
+    set_error("device status word 0x%x (%s%s)", word, (word & ERR_TIMEOUT) ? "bounded wait ran out " : "",
+              (word & ERR_BOUNDS) ? "index out of bounds" : "");
+    return POET_ETIMEOUT;
+  }
+  return POET_OK;
+}
+
+}  // extern "C"

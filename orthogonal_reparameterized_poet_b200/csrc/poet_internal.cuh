@@ -1,0 +1,150 @@
+// Internal declarations of libpoet (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "poet.h"
+
+namespace poet {
+
+using bf16 = __nv_bfloat16;
+
+// ------------------------------------------------------------------ errors
+
+void set_error(const char *fmt, ...);
+void clear_error();
+
+#define POET_REQUIRE(cond, ...)                 \
+  do {                                          \
+    if (!(cond)) {                              \
+      ::poet::set_error(__VA_ARGS__);           \
+      return POET_EINVAL;                       \
+    }                                           \
+  } while (0)
+
+#define POET_CUDA_TRY(call)                                                         \
+  do {                                                                              \
+    cudaError_t e_ = (call);                                                        \
+    if (e_ != cudaSuccess) {                                                        \
+      ::poet::set_error("%s failed: %s", #call, cudaGetErrorString(e_));            \
+      return POET_ECUDA;                                                            \
+    }                                                                               \
+  } while (0)
+
+#define POET_TRY(expr)                 \
+  do {                                 \
+    poet_status s_ = (expr);           \
+    if (s_ != POET_OK) return s_;      \
+  } while (0)
+
+// Checks the last launch.
+poet_status launch_status(const char *what);
+
+// Device status word: kernels with bounded waits OR bits into it.
+enum : unsigned { ERR_TIMEOUT = 1u, ERR_BOUNDS = 2u };
+unsigned *device_errword();   // device address for the current device (nullptr on failure)
+
+// Multiprocessor count of the current device (cached per device).
+int num_sms();
+
+// ------------------------------------------------------------------ accounting
+//
+// Every kernel launch of the library is counted.  When tracing is on, a
+// TraceScope records a CUDA event pair on the launch stream around the work
+// it encloses, tagged with a kind and the work's algorithmic flops and bytes.
+void count_launch();
+bool trace_on();
+struct TraceScope {
+  TraceScope(const char *kind, double flop, double bytes, cudaStream_t st);
+  ~TraceScope();
+  int slot = -1;
+  cudaStream_t st = nullptr;
+};
+
+// ------------------------------------------------------------------ geometry
+
+inline size_t esize(int dtype) { return dtype == POET_BF16 ? 2 : 4; }
+inline int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// One side's primitives: nprim primitives of size `size`, stored with row
+// stride `ld` (size rounded up to 8 so that rows are 16-byte aligned);
+// covered = nprim * size frame indices are acted on, the rest is identity.
+struct SideGeom {
+  int nprim = 0, size = 0, ld = 0, covered = 0, k = 0;
+  int64_t blk_elems() const { return int64_t(ld) * ld; }          // one primitive
+  int64_t all_elems() const { return blk_elems() * nprim; }       // one side
+  int64_t packed_per() const { return int64_t(size) * (size - 1) / 2; }
+};
+bool side_geom(const poet_side *s, SideGeom *g);   // false if the side is malformed
+
+// Frame row stride of a dimension (elements): rows start on 128-byte lines.
+inline int64_t frame_ld(int64_t dim) { return round_up(dim, 64); }
+
+// Layout of a side's state buffer (byte offsets).
+struct StateLayout {
+  size_t R = 0, Q = 0, S1 = 0, bytes = 0;   // S_l at S1 + (l-1)*term
+  size_t term = 0;                          // bytes of one nprim x ld x ld array
+};
+StateLayout state_layout(const SideGeom &g, int dtype);
+
+// ------------------------------------------------------------------ GEMM engine
+//
+//   v(b,i,j) = alpha * sum_l A(b,i,l) * B(b,j,l)  (+ beta * Add(b,i,j)) (+ diag if i == j)
+//   A(b,i,l) = A[b*a_b + i*a_m + l*a_k], B(b,j,l) = B[b*b_b + j*b_n + l*b_k]
+// then v is stored to outF (float) and/or outD (element type `dtype`), or
+// added atomically into outF (split-K allowed).
+struct Gemm {
+  int M = 0, N = 0, K = 0, batch = 1;
+  int dtype = POET_F32;                       // type of A, B, outD
+  const void *A = nullptr; int64_t a_m = 0, a_k = 0, a_b = 0;
+  const void *B = nullptr; int64_t b_n = 0, b_k = 0, b_b = 0;
+  float alpha = 1.f;
+  const void *add = nullptr; int add_dtype = POET_F32; int64_t add_m = 0, add_b = 0; float beta = 0.f;
+  float diag = 0.f;
+  float *outF = nullptr; int64_t of_m = 0, of_b = 0;
+  void *outD = nullptr; int64_t od_m = 0, od_b = 0;
+  bool atomic = false;
+  const char *tag = "gemm";                   // kind for tracing
+};
+
+poet_status gemm_run(const Gemm &g, cudaStream_t st);       // picks the engine
+poet_status gemm_simt(const Gemm &g, cudaStream_t st);      // CUDA-core FMA engine
+bool gemm_tc_supported(const Gemm &g);                      // tcgen05 engine can take g
+poet_status gemm_tc(const Gemm &g, cudaStream_t st);        // tcgen05 engine
+bool gemm_tc_enabled();
+
+// ------------------------------------------------------------------ data movement
+
+// dst[r][i] = src[srcrow(r)][perm[i]] for i < d, r < rows; srcrow(r) = rowmap ? rowmap[r] : r.
+// If dst2 != nullptr, columns i >= split are also written to dst2.  Rows of
+// dst/dst2 are zero-padded up to round_up(d, 8).
+poet_status gather_cols(int dtype, const void *src, int64_t ld_src, const int32_t *rowmap,
+                        int64_t rows, int d, const int32_t *perm,
+                        void *dst, int64_t ld_dst, void *dst2, int64_t ld_dst2, int split,
+                        cudaStream_t st);
+
+// dst[dstrow(r)][perm[i]] = (i < split ? src1[r][i] : src2[r][i]); dstrow(r) = rowmap ? rowmap[r] : r.
+poet_status scatter_cols(int dtype, const void *src1, int64_t ld1, const void *src2, int64_t ld2,
+                         int split, int64_t rows, int d, const int32_t *perm,
+                         void *dst, int64_t ld_dst, const int32_t *rowmap, cudaStream_t st);
+
+// ------------------------------------------------------------------ Cayley-Neumann
+
+poet_status cnp_forward(const poet_side *side, const SideGeom &g, int dtype, cudaStream_t st);
+// G: float [nprim][ld][ld]; scratch: cnp_scratch_bytes(g, dtype) bytes.
+poet_status cnp_backward(const poet_side *side, const SideGeom &g, int dtype, const float *G,
+                         float *dtheta, void *scratch, cudaStream_t st);
+size_t cnp_scratch_bytes(const SideGeom &g, int dtype);
+// out = G (dense [nprim][size][size]) re-laid as [nprim][ld][ld] with zero padding
+poet_status pad_blocks(const float *G, const SideGeom &g, float *out, cudaStream_t st);
+
+// ------------------------------------------------------------------ permutations
+
+poet_status draw_perm_dev(uint64_t seed, int32_t layer_id, int32_t side, int32_t epoch,
+                          int32_t dim, int32_t *perm, cudaStream_t st);
+
+}  // namespace poet

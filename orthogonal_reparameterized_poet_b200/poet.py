@@ -1,0 +1,316 @@
+"""Thin Python binding of libpoet (the C ABI in include/poet.h).
+
+Argument marshalling only: every step of the POET layer runs in libpoet's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  If
+libpoet.so is missing or cannot be loaded, every call raises: there is no
+host fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+F32, BF16 = 0, 1
+BS, FS = 0, 1
+OK, EINVAL, ECUDA, ETIMEOUT, ENOMEM_WS = 0, 1, 2, 3, 4
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpoet.so")
+_lib = None
+
+
+class PoetError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"libpoet status {status}: {msg}")
+        self.status = status
+
+
+class poet_side(ctypes.Structure):
+    _fields_ = [("dim", ctypes.c_int32), ("mode", ctypes.c_int32), ("b", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("perm", ctypes.c_void_p), ("theta", ctypes.c_void_p), ("state", ctypes.c_void_p)]
+
+
+class poet_layer(ctypes.Structure):
+    _fields_ = [("m", ctypes.c_int64), ("n", ctypes.c_int64), ("dtype", ctypes.c_int32),
+                ("layer_id", ctypes.c_int32), ("epoch", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("seed", ctypes.c_uint64), ("W0", ctypes.c_void_p), ("W0f", ctypes.c_void_p),
+                ("R", poet_side), ("P", poet_side)]
+
+
+class poet_trace_row(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_char * 32), ("launches", ctypes.c_int64), ("ms", ctypes.c_double),
+                ("flop", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
+_SIGS = {
+    "poet_side_state_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_side), ctypes.c_int32]),
+    "poet_frame_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_layer)]),
+    "poet_saved_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_layer), ctypes.c_int64]),
+    "poet_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_layer), ctypes.c_int64]),
+    "poet_side_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_side), ctypes.c_int32]),
+    "poet_cayley_neumann": (ctypes.c_int, [ctypes.POINTER(poet_side), ctypes.c_int32, ctypes.c_void_p,
+                                           ctypes.c_size_t, ctypes.c_void_p]),
+    "poet_cayley_neumann_grad": (ctypes.c_int, [ctypes.POINTER(poet_side), ctypes.c_int32, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                                ctypes.c_void_p]),
+    "poet_forward": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "poet_backward": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.c_size_t, ctypes.c_void_p]),
+    "poet_merge": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "poet_prepare": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p]),
+    "poet_resample": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p]),
+    "poet_draw_perm": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                      ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]),
+    "poet_gemm": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                 ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                 ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                 ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_float, ctypes.c_float,
+                                 ctypes.c_void_p]),
+    "poet_gemm_engine": (ctypes.c_int32, [ctypes.c_int32]),
+    "poet_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "poet_launch_count": (ctypes.c_int64, []),
+    "poet_trace_enable": (ctypes.c_int, [ctypes.c_int32]),
+    "poet_trace_read": (ctypes.c_int32, [ctypes.POINTER(poet_trace_row), ctypes.c_int32]),
+    "poet_last_error": (ctypes.c_char_p, []),
+    "poet_version": (ctypes.c_char_p, []),
+}
+
+ABI_SYMBOLS = tuple(_SIGS)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libpoet (raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"libpoet.so not built at {_LIB_PATH}; run "
+                               "`python -m orthogonal_reparameterized_poet_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status):
+    if status != OK:
+        raise PoetError(status, lib().poet_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def torch_dtype(dtype: int):
+    return torch.bfloat16 if dtype == BF16 else torch.float32
+
+
+def side_geometry(dim, mode, b):
+    """(nprim, size) of one side, as libpoet computes it (host bookkeeping for buffer sizes)."""
+    if mode == FS:
+        s = dim // 2
+        return (1, s) if s >= 1 else (0, 0)
+    q = dim // b
+    return (q, b) if q > 0 else (0, 0)
+
+
+# ------------------------------------------------------------------ raw ABI calls
+
+def poet_side_state_bytes(side: poet_side, dtype: int) -> int:
+    return lib().poet_side_state_bytes(ctypes.byref(side), dtype)
+
+
+def poet_frame_bytes(layer: poet_layer) -> int:
+    return lib().poet_frame_bytes(ctypes.byref(layer))
+
+
+def poet_saved_bytes(layer: poet_layer, T: int) -> int:
+    return lib().poet_saved_bytes(ctypes.byref(layer), T)
+
+
+def poet_workspace_bytes(layer: poet_layer, T: int) -> int:
+    return lib().poet_workspace_bytes(ctypes.byref(layer), T)
+
+
+def poet_side_workspace_bytes(side: poet_side, dtype: int) -> int:
+    return lib().poet_side_workspace_bytes(ctypes.byref(side), dtype)
+
+
+def poet_cayley_neumann(side: poet_side, dtype: int, ws=None, stream=None):
+    _check(lib().poet_cayley_neumann(ctypes.byref(side), dtype, _ptr(ws), 0 if ws is None else ws.numel(),
+                                     _stream(stream)))
+
+
+def poet_cayley_neumann_grad(side: poet_side, dtype: int, G, dtheta, ws, stream=None):
+    _check(lib().poet_cayley_neumann_grad(ctypes.byref(side), dtype, _ptr(G), _ptr(dtheta), _ptr(ws), ws.numel(),
+                                          _stream(stream)))
+
+
+def poet_forward(layer: poet_layer, x, T: int, y, saved, ws, stream=None):
+    _check(lib().poet_forward(ctypes.byref(layer), _ptr(x), T, _ptr(y), _ptr(saved), _ptr(ws), ws.numel(),
+                              _stream(stream)))
+
+
+def poet_backward(layer: poet_layer, saved, dy, T: int, dx, dtheta_R, dtheta_P, ws, stream=None):
+    _check(lib().poet_backward(ctypes.byref(layer), _ptr(saved), _ptr(dy), T, _ptr(dx), _ptr(dtheta_R),
+                               _ptr(dtheta_P), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def poet_merge(layer: poet_layer, ws, stream=None):
+    _check(lib().poet_merge(ctypes.byref(layer), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def poet_prepare(layer: poet_layer, stream=None):
+    _check(lib().poet_prepare(ctypes.byref(layer), _stream(stream)))
+
+
+def poet_resample(layer: poet_layer, stream=None):
+    _check(lib().poet_resample(ctypes.byref(layer), _stream(stream)))
+
+
+def poet_draw_perm(seed: int, layer_id: int, side: int, epoch: int, dim: int, perm, stream=None):
+    _check(lib().poet_draw_perm(seed, layer_id, side, epoch, dim, _ptr(perm), _stream(stream)))
+
+
+def poet_gemm(dtype, M, N, K, batch, A, sA, B, sB, C, ldc, sCb, alpha=1.0, beta=0.0, stream=None):
+    """sA = (sAm, sAk, sAb), sB = (sBn, sBk, sBb) in elements."""
+    _check(lib().poet_gemm(dtype, M, N, K, batch, _ptr(A), *sA, _ptr(B), *sB, _ptr(C), ldc, sCb, alpha, beta,
+                           _stream(stream)))
+
+
+def poet_gemm_engine(dtype: int) -> int:
+    return lib().poet_gemm_engine(dtype)
+
+
+def poet_sync_status(stream=None):
+    _check(lib().poet_sync_status(_stream(stream)))
+
+
+def poet_launch_count() -> int:
+    return lib().poet_launch_count()
+
+
+def poet_trace_enable(on: bool):
+    _check(lib().poet_trace_enable(1 if on else 0))
+
+
+def poet_trace_read() -> dict:
+    """{kind: {"launches", "ms", "flop", "bytes"}} of the work recorded since tracing was enabled."""
+    rows = (poet_trace_row * 64)()
+    n = lib().poet_trace_read(rows, 64)
+    return {rows[i].kind.decode(): {"launches": rows[i].launches, "ms": rows[i].ms, "flop": rows[i].flop,
+                                    "bytes": rows[i].bytes} for i in range(n)}
+
+
+def poet_version() -> str:
+    return lib().poet_version().decode()
+
+
+# ------------------------------------------------------------------ owning wrapper
+
+class PoetLayer:
+    """Owns the device buffers of one POET linear and fills a poet_layer struct.
+
+    W0 (m x n, natural order) and theta_R / theta_P are given by the caller
+    (torch tensors on the device); the frame copy, permutations and side
+    states are allocated here.  Workspaces are allocated per token count and
+    cached.
+    """
+
+    def __init__(self, W0, theta_R, theta_P, *, mode, b, k, seed=0, layer_id=0, epoch=0,
+                 modeP=None, bP=None):
+        if not W0.is_cuda:
+            raise ValueError("W0 must be a CUDA tensor")
+        self.dtype = BF16 if W0.dtype == torch.bfloat16 else F32
+        if W0.dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError("W0 must be float32 or bfloat16")
+        self.m, self.n = W0.shape
+        dev = W0.device
+        self.W0 = W0.contiguous()
+        self.theta_R = theta_R.contiguous().float()
+        self.theta_P = theta_P.contiguous().float()
+        modeP = mode if modeP is None else modeP
+        bP = b if bP is None else bP
+        self.perm_R = torch.empty(self.m, dtype=torch.int32, device=dev)
+        self.perm_P = torch.empty(self.n, dtype=torch.int32, device=dev)
+        L = poet_layer()
+        L.m, L.n, L.dtype, L.layer_id, L.epoch, L.reserved, L.seed = self.m, self.n, self.dtype, layer_id, epoch, 0, seed
+        L.R.dim, L.R.mode, L.R.b, L.R.k = self.m, mode, b, k
+        L.P.dim, L.P.mode, L.P.b, L.P.k = self.n, modeP, bP, k
+        self.state_R = torch.empty(max(poet_side_state_bytes(L.R, self.dtype), 1), dtype=torch.uint8, device=dev)
+        self.state_P = torch.empty(max(poet_side_state_bytes(L.P, self.dtype), 1), dtype=torch.uint8, device=dev)
+        self.W0f = torch.empty(max(poet_frame_bytes(L), 1), dtype=torch.uint8, device=dev)
+        self._L = L
+        self._ws = {}
+        self._refresh()
+        nR, sR = side_geometry(self.m, mode, b)
+        nP, sP = side_geometry(self.n, modeP, bP)
+        self.geom_R, self.geom_P = (nR, sR), (nP, sP)
+        assert self.theta_R.numel() == nR * sR * (sR - 1) // 2 if nR else True, "theta_R has the wrong length"
+        assert self.theta_P.numel() == nP * sP * (sP - 1) // 2 if nP else True, "theta_P has the wrong length"
+
+    def _refresh(self):
+        L = self._L
+        L.W0, L.W0f = self.W0.data_ptr(), self.W0f.data_ptr()
+        L.R.perm, L.R.theta, L.R.state = self.perm_R.data_ptr(), self.theta_R.data_ptr(), self.state_R.data_ptr()
+        L.P.perm, L.P.theta, L.P.state = self.perm_P.data_ptr(), self.theta_P.data_ptr(), self.state_P.data_ptr()
+
+    @property
+    def struct(self) -> poet_layer:
+        return self._L
+
+    @property
+    def epoch(self) -> int:
+        return self._L.epoch
+
+    def workspace(self, T: int):
+        if T not in self._ws:
+            self._ws[T] = torch.empty(max(poet_workspace_bytes(self._L, T), 1), dtype=torch.uint8,
+                                      device=self.W0.device)
+        return self._ws[T]
+
+    def saved_buffer(self, T: int):
+        return torch.empty(max(poet_saved_bytes(self._L, T), 1), dtype=torch.uint8, device=self.W0.device)
+
+    def prepare(self, stream=None):
+        poet_prepare(self._L, stream)
+
+    def resample(self, stream=None):
+        poet_resample(self._L, stream)
+
+    def cayley_neumann(self, stream=None):
+        poet_cayley_neumann(self._L.R, self.dtype, None, stream)
+        poet_cayley_neumann(self._L.P, self.dtype, None, stream)
+
+    def forward(self, x, y=None, saved=None, stream=None):
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty(T, self.m, dtype=x.dtype, device=x.device)
+        if saved is None:
+            saved = self.saved_buffer(T)
+        poet_forward(self._L, x, T, y, saved, self.workspace(T), stream)
+        return y, saved
+
+    def backward(self, saved, dy, dx=None, dtheta_R=None, dtheta_P=None, stream=None):
+        T = dy.shape[0]
+        if dx is None:
+            dx = torch.empty(T, self.n, dtype=dy.dtype, device=dy.device)
+        if dtheta_R is None:
+            dtheta_R = torch.empty_like(self.theta_R)
+        if dtheta_P is None:
+            dtheta_P = torch.empty_like(self.theta_P)
+        poet_backward(self._L, saved, dy, T, dx, dtheta_R, dtheta_P, self.workspace(T), stream)
+        return dx, dtheta_R, dtheta_P
+
+    def merge(self, stream=None):
+        poet_merge(self._L, self.workspace(0), stream)

@@ -151,6 +151,20 @@ def check_side_shapes(O):
             and O.side_shape(2736, O.BS, 256) == (10, 256))
 
 
+def check_no_primitive_side(O):
+    """b > d: floor(d/b) = 0 primitives, the side is the identity, and the
+    layer reduces to the plain product y = W0 x with dx = W0^T dy."""
+    rng = _rng(9)
+    m, n, b = 7, 5, 8
+    W0 = rng.standard_normal((m, n))
+    X = rng.standard_normal((3, n))
+    dY = rng.standard_normal((3, m))
+    out = O.layer_step(W0, np.zeros(0), np.zeros(0), rng.permutation(m), rng.permutation(n), 0, b, 0, b, 2, X, dY)
+    return bool(np.allclose(out["Y"], X @ W0.T) and np.allclose(out["dX"], dY @ W0)
+                and out["dthetaR"].size == 0 and out["dthetaP"].size == 0
+                and np.allclose(out["W0_merged"], W0))
+
+
 # ---------------------------------------------------------------- spectrum, merge
 
 def check_spectrum_preservation(O, m=12, n=9):
@@ -317,7 +331,7 @@ def check_param_counts(O):
 ALL_CHECKS = [
     check_unpack_golden, check_cnp_2x2_closed_form, check_cnp_truncation_identity,
     check_orthogonality_identity, check_singular_values_closed_form, check_special_cases,
-    check_dense_side_golden, check_dense_side_vs_loops, check_side_shapes,
+    check_dense_side_golden, check_dense_side_vs_loops, check_side_shapes, check_no_primitive_side,
     check_spectrum_preservation, check_merge_invariance, check_backward_finite_differences,
     check_splitmix_golden, check_draw_perm, check_param_counts,
 ]

@@ -1,0 +1,91 @@
+"""The C-ABI library loads and exports every symbol include/poet.h declares;
+host-side size queries and argument validation (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from orthogonal_reparameterized_poet_b200 import poet
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "poet.h")).read()
+    return sorted(set(re.findall(r"POET_API\s+[\w\s\*]+?\b(poet_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for required in ("poet_cayley_neumann", "poet_forward", "poet_backward", "poet_merge", "poet_resample"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(poet._LIB_PATH)
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert sorted(poet.ABI_SYMBOLS) == _declared()
+
+
+def test_version_string():
+    assert "sm_100a" in poet.poet_version()
+
+
+def _side(dim, mode, b, k):
+    s = poet.poet_side()
+    s.dim, s.mode, s.b, s.k = dim, mode, b, k
+    return s
+
+
+def _layer(m, n, mode, b, k, dtype):
+    L = poet.poet_layer()
+    L.m, L.n, L.dtype = m, n, dtype
+    L.R = _side(m, mode, b, k)
+    L.P = _side(n, mode, b, k)
+    return L
+
+
+def test_state_and_frame_sizes():
+    # BS b=256 on d=5461: 21 primitives of 256 (ld 256); state = (2 + k) terms of 21*256*256 elements
+    assert poet.poet_side_state_bytes(_side(5461, poet.BS, 256, 4), poet.BF16) == 6 * 21 * 256 * 256 * 2
+    # FS on d=5461: one primitive of 2730, stored with ld 2736
+    term = (1 * 2736 * 2736 * 2 + 255) // 256 * 256
+    assert poet.poet_side_state_bytes(_side(5461, poet.FS, 0, 4), poet.BF16) == 6 * term
+    # k = 0 keeps only the primitive and Q
+    assert poet.poet_side_state_bytes(_side(256, poet.BS, 32, 0), poet.F32) == 2 * 8 * 32 * 32 * 4
+    # b > dim: no primitives
+    assert poet.poet_side_state_bytes(_side(100, poet.BS, 256, 4), poet.BF16) == 0
+    # malformed sides
+    assert poet.poet_side_state_bytes(_side(0, poet.BS, 256, 4), poet.BF16) == 0
+    assert poet.poet_side_state_bytes(_side(10, poet.BS, 0, 4), poet.BF16) == 0
+    assert poet.poet_side_state_bytes(_side(10, poet.BS, 2, 17), poet.BF16) == 0
+    L = _layer(5461, 2048, poet.BS, 256, 4, poet.BF16)
+    assert poet.poet_frame_bytes(L) == 5461 * 2048 * 2
+    assert poet.poet_saved_bytes(L, 32768) == 32768 * 2048 * 2 + 32768 * 5504 * 2
+    assert poet.poet_workspace_bytes(L, 32768) > poet.poet_workspace_bytes(L, 0) > 0
+
+
+def test_host_validation_rejects_bad_arguments():
+    lib = poet.lib()
+    L = _layer(256, 256, poet.BS, 32, 3, poet.F32)
+    st = poet.poet_forward.__globals__["ctypes"].c_void_p(0)
+    # NULL pointers everywhere: rejected before any launch
+    assert lib.poet_forward(ctypes.byref(L), None, 16, None, None, None, 0, st) == poet.EINVAL
+    assert "NULL" in lib.poet_last_error().decode() or "misaligned" in lib.poet_last_error().decode()
+    assert lib.poet_forward(None, None, 16, None, None, None, 0, st) == poet.EINVAL
+    assert lib.poet_draw_perm(0, 0, 0, 0, 0, None, st) == poet.EINVAL
+    assert lib.poet_draw_perm(0, 0, 0, 0, 16385, None, st) == poet.EINVAL
+    assert lib.poet_draw_perm(0, -1, 0, 0, 16, ctypes.c_void_p(256), st) == poet.EINVAL
+    bad = _layer(256, 255, poet.BS, 32, 3, poet.F32)  # side dim does not match W0
+    bad.P.dim = 256
+    assert lib.poet_merge(ctypes.byref(bad), None, 0, st) == poet.EINVAL
+    assert lib.poet_gemm(7, 1, 1, 1, 1, None, 0, 0, 0, None, 0, 0, 0, None, 1, 0, 1.0, 0.0, st) == poet.EINVAL
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(poet, "_lib", None)
+    monkeypatch.setattr(poet, "_LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        poet.lib()

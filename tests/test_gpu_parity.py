@@ -1,0 +1,189 @@
+"""CUDA path (through the C ABI) against the CPU oracle on the same seeded
+inputs.  Bar: bit-exact for permutations; relative Frobenius error <= 1e-5
+for float32 workloads and <= 2e-2 for bfloat16 workloads."""
+import numpy as np
+import pytest
+
+from oracle import poet_oracle as O
+from orthogonal_reparameterized_poet_b200 import inputs as I
+from tests.harness import TOL, Case, read_blocks, rel_fro, run_gpu, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cuda():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    poet.lib()  # raises if the library is missing: no fallback
+    return torch
+
+
+# ------------------------------------------------------------------ a10
+
+@pytest.mark.parametrize("dim", [1, 2, 3, 255, 256, 1376, 2736, 5461, 6912, 16384])
+def test_draw_perm_bit_exact(cuda, dim):
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    for (seed, layer_id, side, epoch) in [(0, 0, 0, 0), (0, 5, 1, 3), (123456789, 167, 0, 41)]:
+        p = cuda.empty(dim, dtype=cuda.int32, device="cuda")
+        poet.poet_draw_perm(seed, layer_id, side, epoch, dim, p)
+        got = p.cpu().numpy()
+        assert np.array_equal(got, O.draw_perm(seed, layer_id, side, epoch, dim))
+
+
+# ------------------------------------------------------------------ a1 / a8
+
+def _side_struct(cuda, dim, mode, b, k, theta, dtype):
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    s = poet.poet_side()
+    s.dim, s.mode, s.b, s.k = dim, mode, b, k
+    th = cuda.from_numpy(theta).cuda()
+    state = cuda.empty(max(poet.poet_side_state_bytes(s, dtype), 1), dtype=cuda.uint8, device="cuda")
+    perm = cuda.arange(dim, dtype=cuda.int32, device="cuda")
+    s.perm, s.theta, s.state = perm.data_ptr(), th.data_ptr(), state.data_ptr()
+    return s, (th, state, perm)
+
+
+CNP_CASES = [
+    # dim, mode, b, k, sigma, dtype
+    (256, I.BS, 32, 3, 0.01, I.F32),
+    (200, I.BS, 64, 0, 0.05, I.F32),
+    (90, I.BS, 7, 5, 0.1, I.F32),
+    (1024, I.BS, 256, 4, 0.02, I.BF16),
+    (1376, I.FS, 0, 4, 0.02, I.BF16),
+    (5461, I.FS, 0, 4, 0.02, I.BF16),
+    (301, I.FS, 0, 2, 0.03, I.F32),
+]
+
+
+@pytest.mark.parametrize("dim,mode,b,k,sigma,dtype", CNP_CASES)
+def test_cayley_neumann_forward_and_grad(cuda, dim, mode, b, k, sigma, dtype):
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    nprim, size = O.side_shape(dim, mode, b)
+    theta = I.theta(7, 0, 0, 0, nprim * O.n_skew(size), sigma)
+    s, keep = _side_struct(cuda, dim, mode, b, k, theta, dtype)
+    poet.poet_cayley_neumann(s, dtype)
+    got = read_blocks(keep[1], (nprim, size), dtype)
+    ref = O.cayley_neumann(theta.astype(np.float64), nprim, size, k)
+    assert rel_fro(got, ref) <= TOL[dtype]
+    # a8 on a random upstream gradient
+    G = np.random.default_rng(1).standard_normal((nprim, size, size)).astype(np.float32)
+    ws = cuda.empty(poet.poet_side_workspace_bytes(s, dtype), dtype=cuda.uint8, device="cuda")
+    dth = cuda.empty(theta.size, dtype=cuda.float32, device="cuda")
+    poet.poet_cayley_neumann_grad(s, dtype, cuda.from_numpy(G).cuda(), dth, ws)
+    poet.poet_sync_status()
+    ref_g = O.theta_grad(G.astype(np.float64), theta.astype(np.float64), size, k)
+    assert rel_fro(dth.cpu().numpy(), ref_g) <= TOL[dtype]
+
+
+# ------------------------------------------------------------------ whole layer
+
+LAYER_CASES = {
+    # the 256 x 256 float32 layer: b = 32, k = 3, 512 tokens, sigma 0.01
+    "single256_fp32_bs32": Case(256, 256, I.BS, 32, I.BS, 32, 3, 512, I.F32, 0.01),
+    # LLaMA-60M shapes, fully stochastic, k = 4, 8 x 256 tokens, bf16
+    "llama60m_fs_q": Case(512, 512, I.FS, 0, I.FS, 0, 4, 2048, I.BF16, 0.02, linear=0, layer_id=0),
+    "llama60m_fs_gate": Case(1376, 512, I.FS, 0, I.FS, 0, 4, 2048, I.BF16, 0.02, linear=4, layer_id=4),
+    "llama60m_fs_down": Case(512, 1376, I.FS, 0, I.FS, 0, 4, 2048, I.BF16, 0.02, linear=6, layer_id=6),
+    # ragged: leftover identity indices, token count not a tile multiple
+    "ragged_bs_fp32": Case(300, 200, I.BS, 64, I.BS, 64, 2, 333, I.F32, 0.05, layer_id=3, epoch=2),
+    "ragged_bs_bf16": Case(300, 200, I.BS, 64, I.BS, 64, 2, 333, I.BF16, 0.05, layer_id=3),
+    "ragged_fs_fp32": Case(301, 199, I.FS, 0, I.FS, 0, 3, 77, I.F32, 0.03, layer_id=9),
+    # block-stochastic b = 256 on LLaMA-350M FFN shapes (10 blocks + 176 leftover), few tokens
+    "bs256_ffn_bf16": Case(2736, 1024, I.BS, 256, I.BS, 256, 4, 300, I.BF16, 0.02, layer_id=11),
+    "bs256_down_bf16": Case(1024, 2736, I.BS, 256, I.BS, 256, 4, 130, I.BF16, 0.02, layer_id=12),
+    # mixed modes and degenerate sides
+    "mixed_fs_bs": Case(96, 160, I.FS, 0, I.BS, 16, 1, 40, I.F32, 0.05),
+    "k0": Case(64, 48, I.BS, 16, I.BS, 16, 0, 33, I.F32, 0.05),
+    "b1_no_params": Case(40, 24, I.BS, 1, I.BS, 1, 2, 9, I.F32, 0.05),
+    "b_gt_dim": Case(40, 24, I.BS, 64, I.BS, 64, 2, 9, I.F32, 0.05),
+    "single_token": Case(128, 64, I.BS, 32, I.FS, 0, 2, 1, I.F32, 0.05),
+}
+
+
+@pytest.mark.parametrize("name", list(LAYER_CASES))
+def test_layer_parity(cuda, name):
+    case = LAYER_CASES[name]
+    arrs = case.arrays()
+    ref = run_oracle(case, *arrs)
+    got = run_gpu(case, *arrs)
+    tol = TOL[case.dtype]
+    assert np.array_equal(got["permR"], ref["permR"]) and np.array_equal(got["permP"], ref["permP"])
+    if len(ref["R_blocks"]):
+        assert rel_fro(got["R_blocks"], ref["R_blocks"]) <= tol
+    if len(ref["P_blocks"]):
+        assert rel_fro(got["P_blocks"], ref["P_blocks"]) <= tol
+    errs = {
+        "Y": rel_fro(got["Y"], ref["Y"]),
+        "dX": rel_fro(got["dX"], ref["dX"]),
+        "W0_merged": rel_fro(got["W0_merged"], ref["W0_merged"]),
+    }
+    if ref["dthetaR"].size:
+        errs["dthetaR"] = rel_fro(got["dthetaR"], ref["dthetaR"])
+    if ref["dthetaP"].size:
+        errs["dthetaP"] = rel_fro(got["dthetaP"], ref["dthetaP"])
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, f"{name}: {bad} (tol {tol})"
+    # merge-then-reinitialize: theta reset, epoch advanced, output unchanged
+    assert not np.any(got["thetaR_after_merge"])
+    assert got["epoch_after"] == case.epoch + 1
+    assert np.array_equal(got["permR_after"], O.draw_perm(case.seed, case.layer_id, 0, case.epoch + 1, case.m))
+    assert rel_fro(got["Y_after_merge"], ref["Y"]) <= tol
+
+
+def test_zero_tokens(cuda):
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    case = LAYER_CASES["ragged_bs_fp32"]
+    W0, thR, thP, x, dy = case.arrays()
+    L = poet.PoetLayer(cuda.from_numpy(W0).cuda(), cuda.from_numpy(thR).cuda(), cuda.from_numpy(thP).cuda(),
+                       mode=case.modeR, b=case.bR, k=case.k)
+    L.prepare()
+    L.cayley_neumann()
+    x0 = cuda.empty(0, case.n, device="cuda")
+    y, saved = L.forward(x0)
+    dx, dthR, dthP = L.backward(saved, cuda.empty(0, case.m, device="cuda"))
+    poet.poet_sync_status()
+    assert y.shape == (0, case.m) and dx.shape == (0, case.n)
+    assert not dthR.any().item() and not dthP.any().item()
+
+
+# ------------------------------------------------------------------ GEMM engine
+
+GEMM_CASES = [
+    # dtype, M, N, K, batch, A major, B major, alpha, beta
+    (I.F32, 70, 50, 33, 2, "k", "k", 1.0, 0.0),
+    (I.F32, 64, 64, 64, 1, "m", "n", -0.5, 1.0),
+    (I.BF16, 300, 260, 200, 1, "k", "k", 1.0, 0.0),
+    (I.BF16, 129, 257, 65, 3, "k", "n", 1.0, 0.0),
+    (I.BF16, 256, 256, 1000, 2, "m", "n", 1.0, 0.0),
+    (I.BF16, 1000, 512, 512, 1, "k", "k", 2.0, 1.0),
+]
+
+
+@pytest.mark.parametrize("dtype,M,N,K,batch,amaj,bmaj,alpha,beta", GEMM_CASES)
+def test_gemm_engine(cuda, dtype, M, N, K, batch, amaj, bmaj, alpha, beta):
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    rng = np.random.default_rng(M * 7 + N)
+    tdt = poet.torch_dtype(dtype)
+    A = I.to_storage(rng.standard_normal((batch, M, K)).astype(np.float32), dtype)
+    B = I.to_storage(rng.standard_normal((batch, N, K)).astype(np.float32), dtype)
+    C0 = I.to_storage(rng.standard_normal((batch, M, N)).astype(np.float32), dtype)
+    # device layouts: "k" = row-major [M][K] (K contiguous), "m"/"n" = [K][M] (M contiguous)
+    Ad = cuda.from_numpy(A if amaj == "k" else np.ascontiguousarray(A.transpose(0, 2, 1))).to("cuda", tdt)
+    Bd = cuda.from_numpy(B if bmaj == "k" else np.ascontiguousarray(B.transpose(0, 2, 1))).to("cuda", tdt)
+    sA = (K, 1, M * K) if amaj == "k" else (1, M, M * K)
+    sB = (K, 1, N * K) if bmaj == "k" else (1, N, N * K)
+    C = cuda.from_numpy(C0).to("cuda", tdt)
+    poet.poet_gemm(dtype, M, N, K, batch, Ad, sA, Bd, sB, C, N, M * N, alpha, beta)
+    poet.poet_sync_status()
+    ref = alpha * np.einsum("bmk,bnk->bmn", A.astype(np.float64), B.astype(np.float64)) + beta * C0
+    assert rel_fro(C.float().cpu().numpy(), ref) <= (1e-5 if dtype == I.F32 else 8e-3)
