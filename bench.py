@@ -51,6 +51,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-merge", action="store_true")
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (small profiling cases)")
     return ap.parse_args()
 
 
@@ -124,7 +125,7 @@ class ClockSampler:
 class Variant:
     """All POET linears of one workload, resident on the device."""
 
-    def __init__(self, wl, rank, device, w0_cache):
+    def __init__(self, wl, rank, device, w0_cache, act_cache, saved_pool):
         import torch
 
         from orthogonal_reparameterized_poet_b200 import inputs as I
@@ -164,30 +165,45 @@ class Variant:
             off += a + b
         # per-shape activations (each rank draws its own tokens)
         self.x, self.dy, self.y, self.dx = {}, {}, {}, {}
+        def act(d, grad):
+            key = (wl.seed + 7919 * rank, d, self.T, wl.dtype, grad)
+            if key not in act_cache:  # the variants of one model see the same tokens
+                act_cache[key] = torch.from_numpy(
+                    I.activations(wl.seed + 7919 * rank, d, self.T, d, wl.dtype, grad=grad)).to(device=device,
+                                                                                             dtype=tdt)
+            return act_cache[key]
+
         for (m, n) in set(shapes):
             if n not in self.x:
-                self.x[n] = torch.from_numpy(I.activations(wl.seed + 7919 * rank, n, self.T, n, wl.dtype)).to(
-                    device=device, dtype=tdt)
+                self.x[n] = act(n, False)
                 self.dx[n] = torch.empty(self.T, n, dtype=tdt, device=device)
             if m not in self.dy:
-                self.dy[m] = torch.from_numpy(
-                    I.activations(wl.seed + 7919 * rank, m, self.T, m, wl.dtype, grad=True)).to(device=device,
-                                                                                             dtype=tdt)
+                self.dy[m] = act(m, True)
                 self.y[m] = torch.empty(self.T, m, dtype=tdt, device=device)
-        self.saved = [L.saved_buffer(self.T) for (_, _, _, _, L) in self.layers]
-        for (_, _, _, _, L) in self.layers:
-            L.workspace(self.T)
+        # saved activations: one buffer per linear position, shared by the variants (they run one after the other)
+        self.saved = []
+        for i, (_, _, _, _, L) in enumerate(self.layers):
+            need = poet.poet_saved_bytes(L.struct, self.T)
+            if i >= len(saved_pool) or saved_pool[i].numel() < need:
+                buf = torch.empty(need, dtype=torch.uint8, device=device)
+                if i < len(saved_pool):
+                    saved_pool[i] = buf
+                else:
+                    saved_pool.append(buf)
+            self.saved.append(saved_pool[i])
+        self.ws_need = max(max(L.workspace_bytes(self.T), L.workspace_bytes(0)) for (_, _, _, _, L) in self.layers)
+        self.ws = None
         self.input_bytes = sum(v.numel() * v.element_size() for v in list(self.x.values()) + list(self.dy.values()))
 
     def step(self, world=1):
         for (_, _, _, _, L) in self.layers:
             L.cayley_neumann()
         for i, (_, _, m, n, L) in enumerate(self.layers):
-            L.forward(self.x[n], y=self.y[m], saved=self.saved[i])
+            L.forward(self.x[n], y=self.y[m], saved=self.saved[i], ws=self.ws)
         for i in reversed(range(len(self.layers))):
             _, _, m, n, L = self.layers[i]
             dR, dP = self.dslices[i]
-            L.backward(self.saved[i], self.dy[m], dx=self.dx[n], dtheta_R=dR, dtheta_P=dP)
+            L.backward(self.saved[i], self.dy[m], dx=self.dx[n], dtheta_R=dR, dtheta_P=dP, ws=self.ws)
         if world > 1:
             import torch.distributed as dist
 
@@ -195,7 +211,7 @@ class Variant:
 
     def merge_all(self):
         for (_, _, _, _, L) in self.layers:
-            L.merge()
+            L.merge(ws=self.ws)
             L.resample()
 
 
@@ -223,9 +239,16 @@ def run_poet(args):
     poet.lib()
 
     wls = [I.WORKLOADS[name] for name in WORKLOAD_SETS[args.workload]]
-    w0_cache = {}
-    variants = [Variant(wl, rank, device, w0_cache) for wl in wls]
+    if args.layers:
+        import dataclasses
+
+        wls = [dataclasses.replace(w, layers=args.layers) for w in wls]
+    w0_cache, act_cache, saved_pool = {}, {}, []
+    variants = [Variant(wl, rank, device, w0_cache, act_cache, saved_pool) for wl in wls]
     del w0_cache
+    ws = torch.empty(max(v.ws_need for v in variants), dtype=torch.uint8, device=device)  # one shared workspace
+    for v in variants:
+        v.ws = ws
     torch.cuda.synchronize()
 
     def barrier():

@@ -1,10 +1,559 @@
-// tcgen05 (5th-generation tensor core) engine of the batched GEMM.
+// tcgen05 (5th-generation tensor core) engine of the batched GEMM, sm_100a.
+//
+//   C[b] = epilogue( A[b] . B[b]^T ),  A: M x K, B: N x K, bf16 in, fp32 accumulate
+//
+// Each operand is read by TMA (no multicast) in 64-element-wide slabs with the
+// 128-byte swizzle, either K-major (K contiguous) or MN-major (M/N contiguous);
+// the UMMA shared-memory descriptors describe both forms, so transposed
+// operands (W0f^T in the backward, the token-contracted per-primitive
+// gradients) need no transposed copy.
+//
+// Persistent, warp-specialized CTA (one per SM, 192 threads):
+//   warp 0     TMA producer (one elected lane) filling a STAGES-deep ring
+//   warp 1     TMEM allocator + MMA issuer (one elected lane):
+//              tcgen05.mma.cta_group::1.kind::f16, M=128, N=BN, K=16
+//   warps 2-5  epilogue: tcgen05.ld 32x32b rows out of TMEM, alpha/addend/
+//              diagonal, bf16 and/or fp32 stores, or fp32 atomics (split-K)
+// The accumulator is double-buffered in TMEM (2 x BN columns), so the
+// epilogue of one tile overlaps the MMAs of the next.  Every mbarrier wait is
+// bounded: after a time limit the CTA records ERR_TIMEOUT in the device status
+// word, stops, drains what it issued (bounded too), frees TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "poet_internal.cuh"
 
 namespace poet {
+namespace {
 
-bool gemm_tc_enabled() { return false; }
-bool gemm_tc_supported(const Gemm &) { return false; }
-poet_status gemm_tc(const Gemm &g, cudaStream_t st) { return gemm_simt(g, st); }
+constexpr int BM = 128;
+constexpr int BK = 64;                      // one 128-byte swizzle row of bf16
+constexpr int NTHREADS = 192;
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
+
+struct TcParams {
+  int M, N, K, batch;
+  int num_m, num_n, nk, kchunk, splits;
+  int64_t tiles;
+  float alpha, beta, diag;
+  const void *add; int add_f32; int64_t add_m, add_b;
+  float *outF; int64_t of_m, of_b;
+  bf16 *outD; int64_t od_m, od_b;
+  int atomic;
+  unsigned *errword;
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Returns false (after
+// recording ERR_TIMEOUT and raising the CTA's abort flag) if it runs out, or
+// if another role of the CTA has already aborted.
+__device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *errword) {
+  const uint32_t addr = smem_u32(bar);
+  if (mbar_try_wait(addr, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(addr, parity)) return true;
+    if ((it & 63) == 0) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > kTimeoutNs) {
+        if (errword) atomicOr(errword, ERR_TIMEOUT);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
+          "r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// UMMA shared-memory descriptor, 128-byte swizzle, sm_100 descriptor version.
+//   K-major slab (rows of 64 elements = 128 B): SBO = 1024 B between 8-row groups.
+//   MN-major slab (64 MN elements per 128-B row, one row per K):
+//     LBO = bytes between 64-element MN chunks, SBO = 1024 B between 8-row K groups.
+__device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFF);
+  d |= uint64_t((lbo >> 4) & 0x3FFF) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFF) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: D f32, A and B bf16, M = 128, N = BN.
+template <bool A_MN, bool B_MN, int BN>
+__device__ __forceinline__ uint32_t make_idesc() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(A_MN) << 15) | (uint32_t(B_MN) << 16) |
+         (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+}
+
+struct TileCoord {
+  int b, s, mt, nt;
+};
+__device__ __forceinline__ TileCoord decode(int64_t tile, const TcParams &p) {
+  TileCoord c;
+  c.nt = int(tile % p.num_n);
+  tile /= p.num_n;
+  c.mt = int(tile % p.num_m);
+  tile /= p.num_m;
+  c.s = int(tile % p.splits);
+  c.b = int(tile / p.splits);
+  return c;
+}
+
+template <int BN>
+struct Smem {
+  static constexpr int A_BYTES = BM * BK * 2;   // 16 KB
+  static constexpr int B_BYTES = BN * BK * 2;   // 32 KB (BN = 256)
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr size_t BYTES = size_t(STAGES) * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
+
+template <bool A_MN, bool B_MN, int BN>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                   const TcParams p) {
+  using S = Smem<BN>;
+  constexpr int STAGES = S::STAGES;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char *stage_base = smem;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + size_t(STAGES) * S::STAGE_BYTES);
+  uint64_t *full = bars;                 // [STAGES]
+  uint64_t *empty = bars + STAGES;       // [STAGES]
+  uint64_t *tfull = bars + 2 * STAGES;   // [2]
+  uint64_t *tempty = tfull + 2;          // [2]
+  uint64_t *drain = tempty + 2;          // [1]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_stage = -1;
+      uint32_t last_phase = 0;
+      for (int64_t tile = blockIdx.x; tile < p.tiles && !*abort; tile += gridDim.x) {
+        const TileCoord c = decode(tile, p);
+        const int kb0 = c.s * p.kchunk;
+        const int kb1 = min(p.nk, kb0 + p.kchunk);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort, p.errword)) break;
+          unsigned char *sa = stage_base + size_t(stage) * S::STAGE_BYTES;
+          unsigned char *sb = sa + S::A_BYTES;
+          mbar_expect_tx(&full[stage], S::STAGE_BYTES);
+          if (!A_MN) {
+            tma_load_3d(sa, &mapA, &full[stage], kb * BK, c.mt * BM, c.b);
+          } else {
+#pragma unroll
+            for (int q = 0; q < BM / 64; ++q) tma_load_3d(sa + q * 8192, &mapA, &full[stage], c.mt * BM + 64 * q, kb * BK, c.b);
+          }
+          if (!B_MN) {
+            tma_load_3d(sb, &mapB, &full[stage], kb * BK, c.nt * BN, c.b);
+          } else {
+#pragma unroll
+            for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, &mapB, &full[stage], c.nt * BN + 64 * q, kb * BK, c.b);
+          }
+          last_stage = stage;
+          last_phase = phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (*abort && last_stage >= 0) {
+        // drain: the most recent copies (bounded)
+        volatile int no_abort = 0;
+        mbar_wait(&full[last_stage], last_phase, &no_abort, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      const uint32_t idesc = make_idesc<A_MN, B_MN, BN>();
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool issued = false;
+      for (int64_t tile = blockIdx.x; tile < p.tiles && !*abort; tile += gridDim.x) {
+        const TileCoord c = decode(tile, p);
+        const int kb0 = c.s * p.kchunk;
+        const int kb1 = min(p.nk, kb0 + p.kchunk);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort, p.errword)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
+        bool ok = true;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort, p.errword)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_base + size_t(stage) * S::STAGE_BYTES);
+          const uint32_t sb = sa + S::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? make_desc(sa + kk * 2048, 8192, 1024) : make_desc(sa + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? make_desc(sb + kk * 2048, 8192, 1024) : make_desc(sb + kk * 32, 16, 1024);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          issued = true;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      if (*abort && issued) {
+        // drain: every MMA issued so far has completed once this commit arrives
+        umma_commit(drain);
+        volatile int no_abort = 0;
+        mbar_wait(drain, 0, &no_abort, nullptr);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp % 4;
+    const int row = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int64_t tile = blockIdx.x; tile < p.tiles && !*abort; tile += gridDim.x) {
+      const TileCoord c = decode(tile, p);
+      if (!mbar_wait(&tfull[acc], acc_phase, abort, p.errword)) break;
+      tc_fence_after();
+      const int gm = c.mt * BM + row;
+      const bool row_ok = gm < p.M;
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld32(tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN + cc * 32), r);
+        tmem_ld_wait();
+        const int gn0 = c.nt * BN + cc * 32;
+        if (!row_ok || gn0 >= p.N) continue;
+        const int nvalid = min(32, p.N - gn0);
+        if (p.atomic) {
+          float *o = p.outF + int64_t(c.b) * p.of_b + int64_t(gm) * p.of_m + gn0;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < nvalid) atomicAdd(o + j, p.alpha * __uint_as_float(r[j]));
+          continue;
+        }
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = p.alpha * __uint_as_float(r[j]);
+        if (p.add) {
+          const int64_t off = int64_t(c.b) * p.add_b + int64_t(gm) * p.add_m + gn0;
+          if (p.add_f32) {
+            const float *a = static_cast<const float *>(p.add) + off;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid) v[j] += p.beta * a[j];
+          } else {
+            const uint16_t *a = static_cast<const uint16_t *>(p.add) + off;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid) v[j] += p.beta * bf16_bits_to_float(a[j]);
+          }
+        }
+        if (p.diag != 0.f && gm >= gn0 && gm < gn0 + 32) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (gn0 + j == gm) v[j] += p.diag;
+        }
+        if (p.outF) {
+          float *o = p.outF + int64_t(c.b) * p.of_b + int64_t(gm) * p.of_m + gn0;
+          if (nvalid == 32 && (reinterpret_cast<uintptr_t>(o) & 15) == 0) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4 *>(o + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid) o[j] = v[j];
+          }
+        }
+        if (p.outD) {
+          bf16 *o = p.outD + int64_t(c.b) * p.od_b + int64_t(gm) * p.od_m + gn0;
+          if (nvalid == 32 && (reinterpret_cast<uintptr_t>(o) & 15) == 0) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              uint4 pk;
+              __nv_bfloat162 h0 = __floats2bfloat162_rn(v[j], v[j + 1]);
+              __nv_bfloat162 h1 = __floats2bfloat162_rn(v[j + 2], v[j + 3]);
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(v[j + 4], v[j + 5]);
+              __nv_bfloat162 h3 = __floats2bfloat162_rn(v[j + 6], v[j + 7]);
+              pk.x = *reinterpret_cast<uint32_t *>(&h0);
+              pk.y = *reinterpret_cast<uint32_t *>(&h1);
+              pk.z = *reinterpret_cast<uint32_t *>(&h2);
+              pk.w = *reinterpret_cast<uint32_t *>(&h3);
+              *reinterpret_cast<uint4 *>(o + j) = pk;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid) o[j] = __float2bfloat16_rn(v[j]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 3-D map (inner, outer, batch) over a bf16 operand; strides in elements.
+bool make_map(CUtensorMap *map, const void *base, int64_t inner, int64_t outer, int batch, int64_t outer_stride,
+              int64_t batch_stride, uint32_t box_inner, uint32_t box_outer) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(inner), cuuint64_t(outer), cuuint64_t(batch)};
+  int64_t bstride = batch > 1 ? batch_stride : outer_stride * outer;
+  bstride = round_up(bstride > 0 ? bstride : 8, 8);
+  cuuint64_t strides[2] = {cuuint64_t(outer_stride) * 2, cuuint64_t(bstride) * 2};
+  cuuint32_t box[3] = {box_inner, box_outer, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+template <bool A_MN, bool B_MN, int BN>
+poet_status launch(const Gemm &g, const TcParams &p, const CUtensorMap &ma, const CUtensorMap &mb, cudaStream_t st) {
+  using S = Smem<BN>;
+  auto kern = gemm_tc_kernel<A_MN, B_MN, BN>;
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    POET_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(S::BYTES)));
+    configured[dev] = true;
+  }
+  const int64_t grid = p.tiles < num_sms() ? p.tiles : num_sms();
+  kern<<<int(grid), NTHREADS, S::BYTES, st>>>(ma, mb, p);
+  count_launch();
+  return launch_status("gemm_tc");
+}
+
+}  // namespace
+
+bool gemm_tc_enabled() { return encoder() != nullptr; }
+
+bool gemm_tc_supported(const Gemm &g) {
+  if (g.dtype != POET_BF16 || g.K < 1 || g.M < 1 || g.N < 1) return false;
+  if (!aligned16(g.A) || !aligned16(g.B)) return false;
+  const bool a_k = g.a_k == 1 && g.a_m % 8 == 0 && g.a_m >= 1;
+  const bool a_mn = g.a_m == 1 && g.a_k % 8 == 0 && g.a_k >= 1;
+  const bool b_k = g.b_k == 1 && g.b_n % 8 == 0 && g.b_n >= 1;
+  const bool b_mn = g.b_n == 1 && g.b_k % 8 == 0 && g.b_k >= 1;
+  if (!(a_k || a_mn) || !(b_k || b_mn)) return false;
+  if (g.batch > 1 && (g.a_b % 8 != 0 || g.b_b % 8 != 0 || g.a_b <= 0 || g.b_b <= 0)) return false;
+  if (g.atomic && (g.add || g.outD || !g.outF)) return false;
+  return true;
+}
+
+poet_status gemm_tc(const Gemm &g, cudaStream_t st) {
+  const bool A_MN = !(g.a_k == 1 && g.a_m % 8 == 0);
+  const bool B_MN = !(g.b_k == 1 && g.b_n % 8 == 0);
+  const int BN = g.N <= 128 ? 128 : 256;
+  TcParams p{};
+  p.M = g.M; p.N = g.N; p.K = g.K; p.batch = g.batch;
+  p.num_m = (g.M + BM - 1) / BM;
+  p.num_n = (g.N + BN - 1) / BN;
+  p.nk = (g.K + BK - 1) / BK;
+  int splits = 1;
+  if (g.atomic) {
+    const int64_t base_tiles = int64_t(p.num_m) * p.num_n * g.batch;
+    const int64_t want = (int64_t(num_sms()) + base_tiles - 1) / base_tiles;
+    splits = int(want < p.nk ? want : p.nk);
+    if (splits < 1) splits = 1;
+  }
+  p.kchunk = (p.nk + splits - 1) / splits;
+  p.splits = (p.nk + p.kchunk - 1) / p.kchunk;
+  p.tiles = int64_t(p.num_m) * p.num_n * p.splits * g.batch;
+  p.alpha = g.alpha; p.beta = g.beta; p.diag = g.diag;
+  p.add = g.add; p.add_f32 = g.add_dtype == POET_F32; p.add_m = g.add_m; p.add_b = g.add_b;
+  p.outF = g.outF; p.of_m = g.of_m; p.of_b = g.of_b;
+  p.outD = static_cast<bf16 *>(g.outD); p.od_m = g.od_m; p.od_b = g.od_b;
+  p.atomic = g.atomic ? 1 : 0;
+  p.errword = device_errword();
+
+  CUtensorMap ma, mb;
+  bool ok;
+  if (!A_MN) ok = make_map(&ma, g.A, g.K, g.M, g.batch, g.a_m, g.a_b, 64, BM);
+  else ok = make_map(&ma, g.A, g.M, g.K, g.batch, g.a_k, g.a_b, 64, 64);
+  if (ok) {
+    if (!B_MN) ok = make_map(&mb, g.B, g.K, g.N, g.batch, g.b_n, g.b_b, 64, BN);
+    else ok = make_map(&mb, g.B, g.N, g.K, g.batch, g.b_k, g.b_b, 64, 64);
+  }
+  if (!ok) {
+    set_error("gemm_tc: tensor map encoding failed (M=%d N=%d K=%d)", g.M, g.N, g.K);
+    return POET_ECUDA;
+  }
+  if (BN == 128) {
+    if (!A_MN && !B_MN) return launch<false, false, 128>(g, p, ma, mb, st);
+    if (!A_MN && B_MN) return launch<false, true, 128>(g, p, ma, mb, st);
+    if (A_MN && !B_MN) return launch<true, false, 128>(g, p, ma, mb, st);
+    return launch<true, true, 128>(g, p, ma, mb, st);
+  }
+  if (!A_MN && !B_MN) return launch<false, false, 256>(g, p, ma, mb, st);
+  if (!A_MN && B_MN) return launch<false, true, 256>(g, p, ma, mb, st);
+  if (A_MN && !B_MN) return launch<true, false, 256>(g, p, ma, mb, st);
+  return launch<true, true, 256>(g, p, ma, mb, st);
+}
 
 }  // namespace poet

@@ -46,16 +46,10 @@ def normal(seed: int, key: tuple, shape, scale: float = 1.0) -> np.ndarray:
 
 def round_bf16(a: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even); returned as float32."""
-    a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16) << 16
-    nan = np.isnan(a)
-    out = (r & 0xFFFFFFFF).astype(np.uint32).view(np.float32)
-    if nan.any():
-        out = out.copy()
-        out[nan] = np.nan
-    return out
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return t.to(torch.bfloat16).to(torch.float32).numpy()
 
 
 def to_storage(a: np.ndarray, dtype: int) -> np.ndarray:
@@ -64,7 +58,7 @@ def to_storage(a: np.ndarray, dtype: int) -> np.ndarray:
 
 def w0(seed: int, layer: int, linear: int, m: int, n: int, dtype: int) -> np.ndarray:
     a = normal(seed, (layer, linear, _T_W0), (m, n))
-    a /= np.sqrt(np.sum(a.astype(np.float64) ** 2, axis=1, keepdims=True)).astype(np.float32)
+    a /= np.sqrt(np.einsum("ij,ij->i", a, a, dtype=np.float64)).astype(np.float32)[:, None]
     return to_storage(a, dtype)
 
 

@@ -292,16 +292,18 @@ class PoetLayer:
         poet_cayley_neumann(self._L.R, self.dtype, None, stream)
         poet_cayley_neumann(self._L.P, self.dtype, None, stream)
 
-    def forward(self, x, y=None, saved=None, stream=None):
+    def forward(self, x, y=None, saved=None, ws=None, stream=None):
+        """ws: optional caller workspace (uint8, >= poet_workspace_bytes(T)); work on
+        one stream is ordered, so layers may share one workspace."""
         T = x.shape[0]
         if y is None:
             y = torch.empty(T, self.m, dtype=x.dtype, device=x.device)
         if saved is None:
             saved = self.saved_buffer(T)
-        poet_forward(self._L, x, T, y, saved, self.workspace(T), stream)
+        poet_forward(self._L, x, T, y, saved, self.workspace(T) if ws is None else ws, stream)
         return y, saved
 
-    def backward(self, saved, dy, dx=None, dtheta_R=None, dtheta_P=None, stream=None):
+    def backward(self, saved, dy, dx=None, dtheta_R=None, dtheta_P=None, ws=None, stream=None):
         T = dy.shape[0]
         if dx is None:
             dx = torch.empty(T, self.n, dtype=dy.dtype, device=dy.device)
@@ -309,8 +311,12 @@ class PoetLayer:
             dtheta_R = torch.empty_like(self.theta_R)
         if dtheta_P is None:
             dtheta_P = torch.empty_like(self.theta_P)
-        poet_backward(self._L, saved, dy, T, dx, dtheta_R, dtheta_P, self.workspace(T), stream)
+        poet_backward(self._L, saved, dy, T, dx, dtheta_R, dtheta_P, self.workspace(T) if ws is None else ws,
+                      stream)
         return dx, dtheta_R, dtheta_P
 
-    def merge(self, stream=None):
-        poet_merge(self._L, self.workspace(0), stream)
+    def merge(self, ws=None, stream=None):
+        poet_merge(self._L, self.workspace(0) if ws is None else ws, stream)
+
+    def workspace_bytes(self, T: int) -> int:
+        return poet_workspace_bytes(self._L, T)

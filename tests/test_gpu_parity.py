@@ -165,7 +165,22 @@ GEMM_CASES = [
     (I.BF16, 129, 257, 65, 3, "k", "n", 1.0, 0.0),
     (I.BF16, 256, 256, 1000, 2, "m", "n", 1.0, 0.0),
     (I.BF16, 1000, 512, 512, 1, "k", "k", 2.0, 1.0),
+    # tensor-core eligible layouts: every operand-major pair, ragged M / N / K
+    (I.BF16, 300, 264, 200, 1, "k", "k", 1.0, 0.0),
+    (I.BF16, 129, 264, 72, 3, "k", "n", 1.0, 0.0),
+    (I.BF16, 136, 256, 136, 2, "m", "k", -1.0, 0.5),
+    (I.BF16, 72, 96, 130, 2, "m", "n", 1.0, 0.0),
+    (I.BF16, 64, 40, 8, 1, "k", "k", 1.0, 0.0),
+    (I.BF16, 2048, 1536, 2048, 1, "k", "k", 1.0, 0.0),
+    (I.BF16, 2048, 1536, 2048, 1, "k", "n", 1.0, 0.0),
 ]
+
+
+def test_tensor_core_engine_is_live(cuda):
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    assert poet.poet_gemm_engine(I.BF16) == 1
+    assert poet.poet_gemm_engine(I.F32) == 0
 
 
 @pytest.mark.parametrize("dtype,M,N,K,batch,amaj,bmaj,alpha,beta", GEMM_CASES)
