@@ -195,15 +195,40 @@ class Variant:
         self.ws = None
         self.input_bytes = sum(v.numel() * v.element_size() for v in list(self.x.values()) + list(self.dy.values()))
 
-    def step(self, world=1):
+    def alloc_grads(self, device, chunk):
+        """Per-primitive gradient buffers of every side (one flat buffer) and the
+        workspace of the grouped Cayley-Neumann backward over `chunk` layers."""
+        import torch
+
+        from orthogonal_reparameterized_poet_b200 import poet
+
+        sizes = []
         for (_, _, _, _, L) in self.layers:
-            L.cayley_neumann()
+            sizes.append((poet.poet_block_grad_bytes(L.struct.R) // 4, poet.poet_block_grad_bytes(L.struct.P) // 4))
+        total = sum(a + b for a, b in sizes)
+        self.gflat = torch.empty(max(total, 4), dtype=torch.float32, device=device)
+        self.G = []
+        off = 0
+        for a, b in sizes:
+            self.G.append((self.gflat[off:off + a], self.gflat[off + a:off + a + b]))
+            off += a + b
+        self.chunk = chunk
+        pl = [L for (_, _, _, _, L) in self.layers]
+        return max(poet.cayley_neumann_grad_many_workspace_bytes(pl[i:i + chunk]) for i in range(0, len(pl), chunk))
+
+    def step(self, world=1):
+        from orthogonal_reparameterized_poet_b200 import poet
+
+        pl = [L for (_, _, _, _, L) in self.layers]
+        poet.cayley_neumann_many(pl)  # a1 for every primitive of every layer
         for i, (_, _, m, n, L) in enumerate(self.layers):
             L.forward(self.x[n], y=self.y[m], saved=self.saved[i], ws=self.ws)
         for i in reversed(range(len(self.layers))):
             _, _, m, n, L = self.layers[i]
-            dR, dP = self.dslices[i]
-            L.backward(self.saved[i], self.dy[m], dx=self.dx[n], dtheta_R=dR, dtheta_P=dP, ws=self.ws)
+            L.backward_blocks(self.saved[i], self.dy[m], self.G[i][0], self.G[i][1], dx=self.dx[n], ws=self.ws)
+        for c0 in range(0, len(pl), self.chunk):  # a8 for every layer, in grouped launches
+            poet.cayley_neumann_grad_many(pl[c0:c0 + self.chunk], self.G[c0:c0 + self.chunk],
+                                          self.dslices[c0:c0 + self.chunk], self.gws)
         if world > 1:
             import torch.distributed as dist
 
@@ -247,8 +272,11 @@ def run_poet(args):
     variants = [Variant(wl, rank, device, w0_cache, act_cache, saved_pool) for wl in wls]
     del w0_cache
     ws = torch.empty(max(v.ws_need for v in variants), dtype=torch.uint8, device=device)  # one shared workspace
+    gws_need = max(v.alloc_grads(device, chunk=4 * len(v.wl.linear_shapes())) for v in variants)
+    gws = torch.empty(max(gws_need, 1), dtype=torch.uint8, device=device)
     for v in variants:
         v.ws = ws
+        v.gws = gws
     torch.cuda.synchronize()
 
     def barrier():

@@ -168,6 +168,39 @@ POET_API poet_status poet_backward(const poet_layer *L, const void *saved, const
                           int64_t T, void *dx, float *dtheta_R, float *dtheta_P,
                           void *ws, size_t ws_bytes, poet_stream stream);
 
+/* ---------------------------------------------------------------- many layers at once
+ *
+ * Training steps run a1 for every primitive of every layer and a8 for every
+ * layer; the calls below let many sides share each tensor-core launch (the
+ * primitives of one side are often too few to fill the GPU).  The per-side
+ * gradient G of a primitive is laid out like the materialized primitives at
+ * the start of the side state: float [nprim][ld][ld], ld = size rounded up to
+ * a multiple of 8 (padding ignored). */
+
+/* Bytes of the per-primitive gradient G of one side (float [nprim][ld][ld]). */
+POET_API size_t poet_block_grad_bytes(const poet_side *side);
+
+/* a1 for count sides (same result as poet_cayley_neumann on each). */
+POET_API poet_status poet_cayley_neumann_many(const poet_side *sides, int32_t count, int32_t dtype,
+                                              poet_stream stream);
+
+/* a5..a7 of poet_backward: writes dx and the per-primitive gradients
+ * G_R = dL/dR_j and G_P = dL/dP_j (device, poet_block_grad_bytes each,
+ * 16-byte aligned, overwritten) instead of dtheta. */
+POET_API poet_status poet_backward_blocks(const poet_layer *L, const void *saved, const void *dy,
+                                          int64_t T, void *dx, float *G_R, float *G_P,
+                                          void *ws, size_t ws_bytes, poet_stream stream);
+
+/* Workspace bytes of poet_cayley_neumann_grad_many for these sides. */
+POET_API size_t poet_cayley_neumann_grad_many_workspace_bytes(const poet_side *sides, int32_t count,
+                                                              int32_t dtype);
+
+/* a8 for count sides: dtheta[i] (device float, theta layout, overwritten) from
+ * G[i] (device, layout above).  Same result as poet_cayley_neumann_grad. */
+POET_API poet_status poet_cayley_neumann_grad_many(const poet_side *sides, const float *const *G,
+                                                   float *const *dtheta, int32_t count, int32_t dtype,
+                                                   void *ws, size_t ws_bytes, poet_stream stream);
+
 /* ---------------------------------------------------------------- a9 */
 
 /* Merge-then-reinitialize ([P1] Approach: "merged periodically"; Measured

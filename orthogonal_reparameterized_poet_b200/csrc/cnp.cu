@@ -15,6 +15,8 @@
 //   dQ  = G S_k^T + sum_{l=k-1..0} A_{l+1} S_l^T,   A_l = Q^T A_{l+1} = -Q A_{l+1}
 // with S_0 = I, then dtheta[a,c] = dQ[a,c] - dQ[c,a] (a < c) because
 // Q[a,c] = theta and Q[c,a] = -theta.  2k GEMMs.
+#include <vector>
+
 #include "poet_internal.cuh"
 
 namespace poet {
@@ -218,6 +220,163 @@ poet_status cnp_backward(const poet_side *side, const SideGeom &g, int dtype, co
   pack_grad_kernel<<<grid_for(n, 256), 256, 0, st>>>(dQ, Af[cur], g.nprim, g.size, g.ld, dtheta);
   count_launch();
   return launch_status("cnp pack");
+}
+
+// ---------------------------------------------------------------- many sides
+
+poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int count, int dtype, cudaStream_t st) {
+  int kmax = 0;
+  for (int i = 0; i < count; ++i) {
+    const SideGeom &g = geoms[i];
+    if (g.nprim == 0) continue;
+    const StateLayout L = state_layout(g, dtype);
+    char *base = static_cast<char *>(sides[i].state);
+    void *first = g.k == 0 ? static_cast<void *>(base + L.R) : static_cast<void *>(base + L.S1);
+    const int64_t n = g.all_elems();
+    if (dtype == POET_BF16)
+      unpack_kernel<bf16><<<grid_for(n, 256), 256, 0, st>>>(sides[i].theta, g.nprim, g.size, g.ld,
+                                                            reinterpret_cast<bf16 *>(base + L.Q),
+                                                            static_cast<bf16 *>(first));
+    else
+      unpack_kernel<float><<<grid_for(n, 256), 256, 0, st>>>(sides[i].theta, g.nprim, g.size, g.ld,
+                                                             reinterpret_cast<float *>(base + L.Q),
+                                                             static_cast<float *>(first));
+    count_launch();
+    POET_TRY(launch_status("cnp unpack"));
+    if (g.k > kmax) kmax = g.k;
+  }
+  std::vector<Gemm> gs;
+  for (int l = 1; l <= kmax; ++l) {
+    gs.clear();
+    for (int i = 0; i < count; ++i) {
+      const SideGeom &g = geoms[i];
+      if (g.nprim == 0 || g.k < l) continue;
+      const StateLayout L = state_layout(g, dtype);
+      char *base = static_cast<char *>(sides[i].state);
+      void *S = base + L.S1 + size_t(l - 1) * L.term;
+      Gemm p = prim_gemm(g, dtype, base + L.Q, S, false, "cnp_fwd");
+      if (l < g.k) {
+        p.diag = 1.f;
+        p.outD = base + L.S1 + size_t(l) * L.term;
+      } else {
+        p.add = S; p.add_dtype = dtype; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 1.f;
+        p.outD = base + L.R;
+      }
+      p.od_m = g.ld; p.od_b = g.blk_elems();
+      gs.push_back(p);
+    }
+    POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
+  }
+  return POET_OK;
+}
+
+poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int count, int dtype,
+                              const float *const *G, float *const *dtheta, void *const *scratch, cudaStream_t st) {
+  struct Work {
+    const void *Q, *Gop;
+    const char *S1;
+    size_t term;
+    float *Af[2];
+    void *Ad[2];
+    float *dQ;
+    int cur;
+  };
+  std::vector<Work> w(count);
+  int kmax = 0;
+  for (int i = 0; i < count; ++i) {
+    const SideGeom &g = geoms[i];
+    if (g.nprim == 0 || g.size < 2) continue;
+    const int64_t n = g.all_elems();
+    if (g.k == 0) {  // B = I + Q  ->  dQ = G
+      pack_grad_kernel<<<grid_for(n, 256), 256, 0, st>>>(G[i], nullptr, g.nprim, g.size, g.ld, dtheta[i]);
+      count_launch();
+      POET_TRY(launch_status("cnp pack"));
+      continue;
+    }
+    const StateLayout L = state_layout(g, dtype);
+    const char *base = static_cast<const char *>(sides[i].state);
+    const size_t fb = align256(size_t(n) * 4), db = align256(size_t(n) * esize(dtype));
+    char *s = static_cast<char *>(scratch[i]);
+    Work &x = w[i];
+    x.Q = base + L.Q;
+    x.S1 = base + L.S1;
+    x.term = L.term;
+    if (dtype == POET_BF16) {
+      f32_to_bf16_kernel<<<grid_for(n, 256), 256, 0, st>>>(G[i], reinterpret_cast<bf16 *>(s), n);
+      count_launch();
+      POET_TRY(launch_status("cnp G to bf16"));
+      x.Gop = s;
+    } else {
+      x.Gop = G[i];
+    }
+    s += db;
+    x.Af[0] = reinterpret_cast<float *>(s);
+    x.Af[1] = reinterpret_cast<float *>(s + fb + db);
+    x.Ad[0] = s + fb;
+    x.Ad[1] = s + 2 * fb + db;
+    if (dtype != POET_BF16) { x.Ad[0] = x.Af[0]; x.Ad[1] = x.Af[1]; }
+    x.dQ = reinterpret_cast<float *>(s + 2 * (fb + db));
+    x.cur = 0;
+    if (g.k > kmax) kmax = g.k;
+  }
+  auto active = [&](int i) { return geoms[i].nprim > 0 && geoms[i].size >= 2 && geoms[i].k > 0; };
+  std::vector<Gemm> gs;
+  // A_k = G - Q G  (all sides), then dQ = G S_k^T (all sides)
+  gs.clear();
+  for (int i = 0; i < count; ++i) {
+    if (!active(i)) continue;
+    const SideGeom &g = geoms[i];
+    Gemm p = prim_gemm(g, dtype, w[i].Q, w[i].Gop, false, "cnp_bwd");
+    p.alpha = -1.f;
+    p.add = G[i]; p.add_dtype = POET_F32; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 1.f;
+    p.outF = w[i].Af[0]; p.of_m = g.ld; p.of_b = g.blk_elems();
+    if (dtype == POET_BF16) { p.outD = w[i].Ad[0]; p.od_m = g.ld; p.od_b = g.blk_elems(); }
+    gs.push_back(p);
+  }
+  for (int i = 0; i < count; ++i) {
+    if (!active(i)) continue;
+    const SideGeom &g = geoms[i];
+    Gemm p = prim_gemm(g, dtype, w[i].Gop, w[i].S1 + size_t(g.k - 1) * w[i].term, true, "cnp_bwd");
+    p.outF = w[i].dQ; p.of_m = g.ld; p.of_b = g.blk_elems();
+    gs.push_back(p);
+  }
+  POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
+  for (int l = kmax - 1; l >= 1; --l) {
+    // dQ += A_{l+1} S_l^T
+    gs.clear();
+    for (int i = 0; i < count; ++i) {
+      if (!active(i) || l > geoms[i].k - 1) continue;
+      const SideGeom &g = geoms[i];
+      Gemm p = prim_gemm(g, dtype, w[i].Ad[w[i].cur], w[i].S1 + size_t(l - 1) * w[i].term, true, "cnp_bwd");
+      p.add = w[i].dQ; p.add_dtype = POET_F32; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 1.f;
+      p.outF = w[i].dQ; p.of_m = g.ld; p.of_b = g.blk_elems();
+      gs.push_back(p);
+    }
+    POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
+    // A_l = -Q A_{l+1}
+    gs.clear();
+    for (int i = 0; i < count; ++i) {
+      if (!active(i) || l > geoms[i].k - 1) continue;
+      const SideGeom &g = geoms[i];
+      const int cur = w[i].cur;
+      Gemm p = prim_gemm(g, dtype, w[i].Q, w[i].Ad[cur], false, "cnp_bwd");
+      p.alpha = -1.f;
+      p.outF = w[i].Af[cur ^ 1]; p.of_m = g.ld; p.of_b = g.blk_elems();
+      if (dtype == POET_BF16) { p.outD = w[i].Ad[cur ^ 1]; p.od_m = g.ld; p.od_b = g.blk_elems(); }
+      gs.push_back(p);
+      w[i].cur ^= 1;
+    }
+    POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
+  }
+  for (int i = 0; i < count; ++i) {
+    if (!active(i)) continue;
+    const SideGeom &g = geoms[i];
+    pack_grad_kernel<<<grid_for(g.all_elems(), 256), 256, 0, st>>>(w[i].dQ, w[i].Af[w[i].cur], g.nprim, g.size, g.ld,
+                                                                    dtheta[i]);
+    count_launch();
+    POET_TRY(launch_status("cnp pack"));
+  }
+  return POET_OK;
 }
 
 }  // namespace poet

@@ -32,15 +32,27 @@ constexpr int BK = 64;                      // one 128-byte swizzle row of bf16
 constexpr int NTHREADS = 192;
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
 
-struct TcParams {
+// One GEMM problem of a launch.
+struct TcProblem {
   int M, N, K, batch;
   int num_m, num_n, nk, kchunk, splits;
-  int64_t tiles;
   float alpha, beta, diag;
   const void *add; int add_f32; int64_t add_m, add_b;
   float *outF; int64_t of_m, of_b;
   bf16 *outD; int64_t od_m, od_b;
   int atomic;
+};
+
+// A launch: up to MAXP independent problems sharing operand majors and tile
+// width, with their TMA descriptors, passed whole as a __grid_constant__
+// kernel parameter.  Tiles of problem i are [tile_start[i], tile_start[i+1]).
+template <int MAXP>
+struct TcGroup {
+  CUtensorMap ma[MAXP];
+  CUtensorMap mb[MAXP];
+  TcProblem prob[MAXP];
+  int64_t tile_start[MAXP + 1];
+  int count;
   unsigned *errword;
 };
 
@@ -177,16 +189,25 @@ __device__ __forceinline__ uint32_t make_idesc() {
 }
 
 struct TileCoord {
-  int b, s, mt, nt;
+  int pi, b, s, mt, nt;
 };
-__device__ __forceinline__ TileCoord decode(int64_t tile, const TcParams &p) {
+template <int MAXP>
+__device__ __forceinline__ TileCoord decode(int64_t tile, const TcGroup<MAXP> &g) {
+  int lo = 0, hi = g.count - 1;  // last problem with tile_start <= tile
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) / 2;
+    if (g.tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
   TileCoord c;
-  c.nt = int(tile % p.num_n);
-  tile /= p.num_n;
-  c.mt = int(tile % p.num_m);
-  tile /= p.num_m;
-  c.s = int(tile % p.splits);
-  c.b = int(tile / p.splits);
+  c.pi = lo;
+  const TcProblem &p = g.prob[lo];
+  int64_t t = tile - g.tile_start[lo];
+  c.nt = int(t % p.num_n);
+  t /= p.num_n;
+  c.mt = int(t % p.num_m);
+  t /= p.num_m;
+  c.s = int(t % p.splits);
+  c.b = int(t / p.splits);
   return c;
 }
 
@@ -202,10 +223,8 @@ struct Smem {
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
 
-template <bool A_MN, bool B_MN, int BN>
-__global__ void __launch_bounds__(NTHREADS, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                   const TcParams p) {
+template <bool A_MN, bool B_MN, int BN, int MAXP>
+__global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_constant__ TcGroup<MAXP> g) {
   using S = Smem<BN>;
   constexpr int STAGES = S::STAGES;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -221,6 +240,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t tiles = g.tile_start[g.count];
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -234,8 +254,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(drain, 1);
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    tma_prefetch_desc(&mapA);
-    tma_prefetch_desc(&mapB);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, S::TMEM_COLS);
@@ -253,26 +271,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint32_t phase = 0;
       int last_stage = -1;
       uint32_t last_phase = 0;
-      for (int64_t tile = blockIdx.x; tile < p.tiles && !*abort; tile += gridDim.x) {
-        const TileCoord c = decode(tile, p);
+      int last_pi = -1;
+      for (int64_t tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
+        const TileCoord c = decode(tile, g);
+        const TcProblem &p = g.prob[c.pi];
+        const CUtensorMap *ma = &g.ma[c.pi];
+        const CUtensorMap *mb = &g.mb[c.pi];
+        if (c.pi != last_pi) {
+          tma_prefetch_desc(ma);
+          tma_prefetch_desc(mb);
+          last_pi = c.pi;
+        }
         const int kb0 = c.s * p.kchunk;
         const int kb1 = min(p.nk, kb0 + p.kchunk);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort, p.errword)) break;
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort, g.errword)) break;
           unsigned char *sa = stage_base + size_t(stage) * S::STAGE_BYTES;
           unsigned char *sb = sa + S::A_BYTES;
           mbar_expect_tx(&full[stage], S::STAGE_BYTES);
           if (!A_MN) {
-            tma_load_3d(sa, &mapA, &full[stage], kb * BK, c.mt * BM, c.b);
+            tma_load_3d(sa, ma, &full[stage], kb * BK, c.mt * BM, c.b);
           } else {
 #pragma unroll
-            for (int q = 0; q < BM / 64; ++q) tma_load_3d(sa + q * 8192, &mapA, &full[stage], c.mt * BM + 64 * q, kb * BK, c.b);
+            for (int q = 0; q < BM / 64; ++q) tma_load_3d(sa + q * 8192, ma, &full[stage], c.mt * BM + 64 * q, kb * BK, c.b);
           }
           if (!B_MN) {
-            tma_load_3d(sb, &mapB, &full[stage], kb * BK, c.nt * BN, c.b);
+            tma_load_3d(sb, mb, &full[stage], kb * BK, c.nt * BN, c.b);
           } else {
 #pragma unroll
-            for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, &mapB, &full[stage], c.nt * BN + 64 * q, kb * BK, c.b);
+            for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, mb, &full[stage], c.nt * BN + 64 * q, kb * BK, c.b);
           }
           last_stage = stage;
           last_phase = phase;
@@ -297,16 +324,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool issued = false;
-      for (int64_t tile = blockIdx.x; tile < p.tiles && !*abort; tile += gridDim.x) {
-        const TileCoord c = decode(tile, p);
+      for (int64_t tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
+        const TileCoord c = decode(tile, g);
+        const TcProblem &p = g.prob[c.pi];
         const int kb0 = c.s * p.kchunk;
         const int kb1 = min(p.nk, kb0 + p.kchunk);
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort, p.errword)) break;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort, g.errword)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort, p.errword)) { ok = false; break; }
+          if (!mbar_wait(&full[stage], phase, abort, g.errword)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + size_t(stage) * S::STAGE_BYTES);
           const uint32_t sb = sa + S::A_BYTES;
@@ -343,12 +371,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int64_t tile = blockIdx.x; tile < p.tiles && !*abort; tile += gridDim.x) {
-      const TileCoord c = decode(tile, p);
-      if (!mbar_wait(&tfull[acc], acc_phase, abort, p.errword)) break;
+    for (int64_t tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
+      const TileCoord c = decode(tile, g);
+      const TcProblem &p = g.prob[c.pi];
+      if (!mbar_wait(&tfull[acc], acc_phase, abort, g.errword)) break;
       tc_fence_after();
       const int gm = c.mt * BM + row;
       const bool row_ok = gm < p.M;
+      const float alpha = p.alpha, beta = p.beta, diag = p.diag;
       for (int cc = 0; cc < BN / 32; ++cc) {
         uint32_t r[32];
         __syncwarp();
@@ -361,30 +391,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           float *o = p.outF + int64_t(c.b) * p.of_b + int64_t(gm) * p.of_m + gn0;
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (j < nvalid) atomicAdd(o + j, p.alpha * __uint_as_float(r[j]));
+            if (j < nvalid) atomicAdd(o + j, alpha * __uint_as_float(r[j]));
           continue;
         }
         float v[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = p.alpha * __uint_as_float(r[j]);
+        for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(r[j]);
         if (p.add) {
           const int64_t off = int64_t(c.b) * p.add_b + int64_t(gm) * p.add_m + gn0;
           if (p.add_f32) {
             const float *a = static_cast<const float *>(p.add) + off;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (j < nvalid) v[j] += p.beta * a[j];
+              if (j < nvalid) v[j] += beta * a[j];
           } else {
             const uint16_t *a = static_cast<const uint16_t *>(p.add) + off;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (j < nvalid) v[j] += p.beta * bf16_bits_to_float(a[j]);
+              if (j < nvalid) v[j] += beta * bf16_bits_to_float(a[j]);
           }
         }
-        if (p.diag != 0.f && gm >= gn0 && gm < gn0 + 32) {
+        if (diag != 0.f && gm >= gn0 && gm < gn0 + 32) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (gn0 + j == gm) v[j] += p.diag;
+            if (gn0 + j == gm) v[j] += diag;
         }
         if (p.outF) {
           float *o = p.outF + int64_t(c.b) * p.of_b + int64_t(gm) * p.of_m + gn0;
@@ -472,10 +502,49 @@ bool make_map(CUtensorMap *map, const void *base, int64_t inner, int64_t outer, 
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-template <bool A_MN, bool B_MN, int BN>
-poet_status launch(const Gemm &g, const TcParams &p, const CUtensorMap &ma, const CUtensorMap &mb, cudaStream_t st) {
+// Operand majors and tile width of a supported problem.
+struct TcPlan {
+  bool A_MN, B_MN;
+  int BN;
+  bool operator==(const TcPlan &o) const { return A_MN == o.A_MN && B_MN == o.B_MN && BN == o.BN; }
+};
+TcPlan plan_of(const Gemm &g) {
+  TcPlan t;
+  t.A_MN = !(g.a_k == 1 && g.a_m % 8 == 0);
+  t.B_MN = !(g.b_k == 1 && g.b_n % 8 == 0);
+  t.BN = g.N <= 128 ? 128 : 256;
+  return t;
+}
+
+// Fill one problem of a group (tiles use split-K only for atomic outputs).
+bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, CUtensorMap *ma, CUtensorMap *mb) {
+  p->M = g.M; p->N = g.N; p->K = g.K; p->batch = g.batch;
+  p->num_m = (g.M + BM - 1) / BM;
+  p->num_n = (g.N + t.BN - 1) / t.BN;
+  p->nk = (g.K + BK - 1) / BK;
+  int splits = g.atomic ? (split_want < p->nk ? split_want : p->nk) : 1;
+  if (splits < 1) splits = 1;
+  p->kchunk = (p->nk + splits - 1) / splits;
+  p->splits = (p->nk + p->kchunk - 1) / p->kchunk;
+  p->alpha = g.alpha; p->beta = g.beta; p->diag = g.diag;
+  p->add = g.add; p->add_f32 = g.add_dtype == POET_F32; p->add_m = g.add_m; p->add_b = g.add_b;
+  p->outF = g.outF; p->of_m = g.of_m; p->of_b = g.of_b;
+  p->outD = static_cast<bf16 *>(g.outD); p->od_m = g.od_m; p->od_b = g.od_b;
+  p->atomic = g.atomic ? 1 : 0;
+  bool ok;
+  if (!t.A_MN) ok = make_map(ma, g.A, g.K, g.M, g.batch, g.a_m, g.a_b, 64, BM);
+  else ok = make_map(ma, g.A, g.M, g.K, g.batch, g.a_k, g.a_b, 64, 64);
+  if (ok) {
+    if (!t.B_MN) ok = make_map(mb, g.B, g.K, g.N, g.batch, g.b_n, g.b_b, 64, t.BN);
+    else ok = make_map(mb, g.B, g.N, g.K, g.batch, g.b_k, g.b_b, 64, 64);
+  }
+  return ok;
+}
+
+template <bool A_MN, bool B_MN, int BN, int MAXP>
+poet_status launch(const TcGroup<MAXP> &grp, cudaStream_t st) {
   using S = Smem<BN>;
-  auto kern = gemm_tc_kernel<A_MN, B_MN, BN>;
+  auto kern = gemm_tc_kernel<A_MN, B_MN, BN, MAXP>;
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -483,11 +552,46 @@ poet_status launch(const Gemm &g, const TcParams &p, const CUtensorMap &ma, cons
     POET_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(S::BYTES)));
     configured[dev] = true;
   }
-  const int64_t grid = p.tiles < num_sms() ? p.tiles : num_sms();
-  kern<<<int(grid), NTHREADS, S::BYTES, st>>>(ma, mb, p);
+  const int64_t tiles = grp.tile_start[grp.count];
+  const int64_t grid = tiles < num_sms() ? tiles : num_sms();
+  kern<<<int(grid), NTHREADS, S::BYTES, st>>>(grp);
   count_launch();
   return launch_status("gemm_tc");
 }
+
+template <int MAXP>
+poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
+  static thread_local TcGroup<MAXP> grp;  // large: keep it off the stack
+  int64_t base_tiles = 0;
+  for (int i = 0; i < n; ++i) {
+    const int64_t mt = (gs[i].M + BM - 1) / BM, nt = (gs[i].N + t.BN - 1) / t.BN;
+    base_tiles += mt * nt * gs[i].batch;
+  }
+  const int split_want = int((int64_t(num_sms()) + base_tiles - 1) / (base_tiles > 0 ? base_tiles : 1));
+  grp.count = n;
+  grp.errword = device_errword();
+  grp.tile_start[0] = 0;
+  for (int i = 0; i < n; ++i) {
+    TcProblem &p = grp.prob[i];
+    if (!fill_problem(gs[i], t, split_want, &p, &grp.ma[i], &grp.mb[i])) {
+      set_error("gemm_tc: tensor map encoding failed (M=%d N=%d K=%d)", gs[i].M, gs[i].N, gs[i].K);
+      return POET_ECUDA;
+    }
+    grp.tile_start[i + 1] = grp.tile_start[i] + int64_t(p.num_m) * p.num_n * p.splits * p.batch;
+  }
+  if (t.BN == 128) {
+    if (!t.A_MN && !t.B_MN) return launch<false, false, 128, MAXP>(grp, st);
+    if (!t.A_MN && t.B_MN) return launch<false, true, 128, MAXP>(grp, st);
+    if (t.A_MN && !t.B_MN) return launch<true, false, 128, MAXP>(grp, st);
+    return launch<true, true, 128, MAXP>(grp, st);
+  }
+  if (!t.A_MN && !t.B_MN) return launch<false, false, 256, MAXP>(grp, st);
+  if (!t.A_MN && t.B_MN) return launch<false, true, 256, MAXP>(grp, st);
+  if (t.A_MN && !t.B_MN) return launch<true, false, 256, MAXP>(grp, st);
+  return launch<true, true, 256, MAXP>(grp, st);
+}
+
+constexpr int kGroupMax = 48;
 
 }  // namespace
 
@@ -506,54 +610,30 @@ bool gemm_tc_supported(const Gemm &g) {
   return true;
 }
 
-poet_status gemm_tc(const Gemm &g, cudaStream_t st) {
-  const bool A_MN = !(g.a_k == 1 && g.a_m % 8 == 0);
-  const bool B_MN = !(g.b_k == 1 && g.b_n % 8 == 0);
-  const int BN = g.N <= 128 ? 128 : 256;
-  TcParams p{};
-  p.M = g.M; p.N = g.N; p.K = g.K; p.batch = g.batch;
-  p.num_m = (g.M + BM - 1) / BM;
-  p.num_n = (g.N + BN - 1) / BN;
-  p.nk = (g.K + BK - 1) / BK;
-  int splits = 1;
-  if (g.atomic) {
-    const int64_t base_tiles = int64_t(p.num_m) * p.num_n * g.batch;
-    const int64_t want = (int64_t(num_sms()) + base_tiles - 1) / base_tiles;
-    splits = int(want < p.nk ? want : p.nk);
-    if (splits < 1) splits = 1;
-  }
-  p.kchunk = (p.nk + splits - 1) / splits;
-  p.splits = (p.nk + p.kchunk - 1) / p.kchunk;
-  p.tiles = int64_t(p.num_m) * p.num_n * p.splits * g.batch;
-  p.alpha = g.alpha; p.beta = g.beta; p.diag = g.diag;
-  p.add = g.add; p.add_f32 = g.add_dtype == POET_F32; p.add_m = g.add_m; p.add_b = g.add_b;
-  p.outF = g.outF; p.of_m = g.of_m; p.of_b = g.of_b;
-  p.outD = static_cast<bf16 *>(g.outD); p.od_m = g.od_m; p.od_b = g.od_b;
-  p.atomic = g.atomic ? 1 : 0;
-  p.errword = device_errword();
+poet_status gemm_tc(const Gemm &g, cudaStream_t st) { return run_group<1>(&g, 1, plan_of(g), st); }
 
-  CUtensorMap ma, mb;
-  bool ok;
-  if (!A_MN) ok = make_map(&ma, g.A, g.K, g.M, g.batch, g.a_m, g.a_b, 64, BM);
-  else ok = make_map(&ma, g.A, g.M, g.K, g.batch, g.a_k, g.a_b, 64, 64);
-  if (ok) {
-    if (!B_MN) ok = make_map(&mb, g.B, g.K, g.N, g.batch, g.b_n, g.b_b, 64, BN);
-    else ok = make_map(&mb, g.B, g.N, g.K, g.batch, g.b_k, g.b_b, 64, 64);
+// Runs many independent problems: consecutive tensor-core problems that share
+// operand majors and tile width go into grouped launches of up to kGroupMax
+// problems each; the others run one by one on the CUDA-core engine.
+poet_status gemm_tc_many(const Gemm *gs, int count, cudaStream_t st) {
+  int i = 0;
+  while (i < count) {
+    if (gs[i].M <= 0 || gs[i].N <= 0 || gs[i].batch <= 0) { ++i; continue; }
+    if (!(gemm_tc_enabled() && gemm_tc_supported(gs[i]))) {
+      POET_TRY(gemm_simt(gs[i], st));
+      ++i;
+      continue;
+    }
+    const TcPlan t = plan_of(gs[i]);
+    int j = i + 1;
+    while (j < count && j - i < kGroupMax && gs[j].M > 0 && gs[j].N > 0 && gs[j].batch > 0 && gemm_tc_supported(gs[j]) &&
+           plan_of(gs[j]) == t)
+      ++j;
+    if (j - i == 1) POET_TRY(run_group<1>(gs + i, 1, t, st));
+    else POET_TRY(run_group<kGroupMax>(gs + i, j - i, t, st));
+    i = j;
   }
-  if (!ok) {
-    set_error("gemm_tc: tensor map encoding failed (M=%d N=%d K=%d)", g.M, g.N, g.K);
-    return POET_ECUDA;
-  }
-  if (BN == 128) {
-    if (!A_MN && !B_MN) return launch<false, false, 128>(g, p, ma, mb, st);
-    if (!A_MN && B_MN) return launch<false, true, 128>(g, p, ma, mb, st);
-    if (A_MN && !B_MN) return launch<true, false, 128>(g, p, ma, mb, st);
-    return launch<true, true, 128>(g, p, ma, mb, st);
-  }
-  if (!A_MN && !B_MN) return launch<false, false, 256>(g, p, ma, mb, st);
-  if (!A_MN && B_MN) return launch<false, true, 256>(g, p, ma, mb, st);
-  if (A_MN && !B_MN) return launch<true, false, 256>(g, p, ma, mb, st);
-  return launch<true, true, 256>(g, p, ma, mb, st);
+  return POET_OK;
 }
 
 }  // namespace poet

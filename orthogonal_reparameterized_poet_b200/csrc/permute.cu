@@ -4,224 +4,230 @@
 // (POET summary page, Approach: "sampled sub-block orthogonal primitives";
 // the index layout is a reading).  These kernels move whole rows between the
 // natural order and the frame order, so that every contraction downstream
-// reads contiguous blocks.  Each CTA stages a few rows in shared memory:
-// global reads and writes are 16-byte vectors on 16-byte boundaries (rows of
-// odd length are split into an aligned body and scalar edges), and only the
-// shared-memory side is accessed through the permutation.  HBM-bound.
+// reads contiguous blocks.  HBM-bound: one read and one write of each row.
+//
+// One kernel serves both directions as a row gather out[r][j] = in[r][map[j]]:
+//   gather  (natural -> frame): map = perm
+//   scatter (frame -> natural): map = perm^-1, built in shared memory
+// Each CTA keeps map (uint16) in shared memory and streams its rows through a
+// ring of NB row slots filled by cp.async 16-byte copies, prefetching NB-1
+// rows ahead, so the loads, the shared-memory gather and the 16-byte global
+// stores of different rows overlap; several CTAs per SM add more rows in
+// flight.  Rows whose start is not 16-byte aligned (natural rows of odd
+// length) use 16-byte copies for the aligned body and scalar copies for the
+// edges; shared and global addresses stay congruent modulo 16.
+#include <type_traits>
+
 #include "poet_internal.cuh"
 
 namespace poet {
 namespace {
 
-constexpr int NT = 512;
+constexpr int NT = 256;
+constexpr int NB = 4;  // ring depth (rows per CTA in flight)
 
-__device__ __forceinline__ int perm_bytes_dev(int d) { return (d * 4 + 15) & ~15; }
-
-// Row r of a chunk lives in shared memory at slot r (stride `slot` elements);
-// element e of the global row sits at slot position off_r + e, where off_r is
-// the row's misalignment (in elements) relative to 16 bytes, so that shared
-// and global addresses agree modulo 16 and both sides can use 16-byte vectors.
 template <typename T>
-struct RowIO {
-  static constexpr int VEC = 16 / sizeof(T);
-  __device__ static int misalign(const T *row) { return int((reinterpret_cast<uintptr_t>(row) & 15) / sizeof(T)); }
-  __device__ static int units(const T *row, int d) { return (misalign(row) + d + VEC - 1) / VEC; }
-  // copy unit u of a global row into the slot (the slot is 16-byte aligned)
-  __device__ static void load_unit(const T *row, int d, int u, T *slot) {
-    const int off = misalign(row);
-    const int first = u * VEC - off;  // row element of the unit's first lane
-    if (first >= 0 && first + VEC <= d) {
-      *reinterpret_cast<uint4 *>(slot + u * VEC) = __ldg(reinterpret_cast<const uint4 *>(row + first));
-    } else {
-      for (int v = 0; v < VEC; ++v) {
-        const int e = first + v;
-        if (e >= 0 && e < d) slot[u * VEC + v] = row[e];
-      }
-    }
-  }
-  __device__ static void store_unit(T *row, int d, int u, const T *slot) {
-    const int off = misalign(row);
-    const int first = u * VEC - off;
-    if (first >= 0 && first + VEC <= d) {
-      *reinterpret_cast<uint4 *>(row + first) = *reinterpret_cast<const uint4 *>(slot + u * VEC);
-    } else {
-      for (int v = 0; v < VEC; ++v) {
-        const int e = first + v;
-        if (e >= 0 && e < d) row[e] = slot[u * VEC + v];
-      }
-    }
-  }
+struct PermArgs {
+  const T *src1; int64_t ld1;         // source row = src1[0:split) ++ src2[split:d)
+  const T *src2; int64_t ld2; int split;
+  const int32_t *src_rowmap;          // source row of output row r (nullptr: r)
+  int64_t rows; int d;
+  const int32_t *perm; int inverse;
+  T *dst1; int64_t ldd1;              // output rows
+  T *dst2; int64_t ldd2; int dsplit;  // columns >= dsplit also go here (nullptr: none)
+  const int32_t *dst_rowmap;          // destination row of output row r (nullptr: r)
+  int slot;                           // slot stride (elements, multiple of 16 bytes)
 };
 
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_ring() { asm volatile("cp.async.wait_group %0;" ::"n"(NB - 1) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 template <typename T>
-__global__ void __launch_bounds__(NT) gather_cols_kernel(const T *__restrict__ src, int64_t ld_src,
-                                                        const int32_t *__restrict__ rowmap, int64_t rows, int d,
-                                                        const int32_t *__restrict__ perm, T *__restrict__ dst,
-                                                        int64_t ld_dst, T *__restrict__ dst2, int64_t ld_dst2,
-                                                        int split, int rows_per_cta, int slot) {
-  using IO = RowIO<T>;
-  constexpr int VEC = IO::VEC;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  int32_t *sperm = reinterpret_cast<int32_t *>(smem_raw);
-  T *srows = reinterpret_cast<T *>(smem_raw + perm_bytes_dev(d));
-  for (int i = threadIdx.x; i < d; i += NT) sperm[i] = perm[i];
-  const int dpad = (d + VEC - 1) / VEC * VEC;  // frame columns written (zero padded)
-  const int gpr = dpad / VEC;                  // vector groups per frame row
-  const int64_t nchunks = (rows + rows_per_cta - 1) / rows_per_cta;
-  for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x) {
-    const int64_t r0 = c * rows_per_cta;
-    const int nr = int(rows - r0 < rows_per_cta ? rows - r0 : rows_per_cta);
-    __syncthreads();  // previous chunk's readers are done (and sperm is ready)
-    // load: every unit of every row of the chunk
-    const T *row0 = src + (rowmap ? int64_t(rowmap[r0]) : r0) * ld_src;
-    const int upr = IO::units(row0, d) + 1;  // rows may differ in misalignment by one unit
-    for (int idx = threadIdx.x; idx < nr * upr; idx += NT) {
-      const int r = idx / upr, u = idx % upr;
-      const T *row = src + (rowmap ? int64_t(rowmap[r0 + r]) : (r0 + r)) * ld_src;
-      if (u < IO::units(row, d)) IO::load_unit(row, d, u, srows + int64_t(r) * slot);
-    }
-    __syncthreads();
-    // write: frame row r, vector group q covers frame columns q*VEC .. q*VEC+VEC-1
-    for (int idx = threadIdx.x; idx < nr * gpr; idx += NT) {
-      const int r = idx / gpr, q = idx % gpr;
-      const T *row = src + (rowmap ? int64_t(rowmap[r0 + r]) : (r0 + r)) * ld_src;
-      const T *s = srows + int64_t(r) * slot + IO::misalign(row);
-      alignas(16) T v[VEC];
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        const int i = q * VEC + e;
-        v[e] = i < d ? s[sperm[i]] : T(0.f);
-      }
-      const int i0 = q * VEC;
-      *reinterpret_cast<uint4 *>(dst + (r0 + r) * ld_dst + i0) = *reinterpret_cast<const uint4 *>(v);
-      if (dst2) {
-        if (i0 >= split) {
-          *reinterpret_cast<uint4 *>(dst2 + (r0 + r) * ld_dst2 + i0) = *reinterpret_cast<const uint4 *>(v);
-        } else if (i0 + VEC > split) {
-          for (int e = split - i0; e < VEC; ++e) dst2[(r0 + r) * ld_dst2 + i0 + e] = v[e];
-        }
-      }
-    }
-  }
+__device__ __forceinline__ int misalign(const T *p) {
+  return int((reinterpret_cast<uintptr_t>(p) & 15) / sizeof(T));
+}
+
+// Copies of elements [e0, e1) of a global row into slot[off + e]
+// (off = misalignment of the row start; the same for every part of a row).
+template <typename T>
+__device__ __forceinline__ void load_part(const T *row, int e0, int e1, T *slot, int off) {
+  constexpr int VEC = 16 / sizeof(T);
+  if (e1 <= e0) return;
+  const int b0 = ((off + e0 + VEC - 1) / VEC) * VEC - off;  // first 16B-aligned element >= e0
+  const int b1 = ((off + e1) / VEC) * VEC - off;            // end of the last whole aligned unit
+  if (b0 < b1)
+    for (int e = b0 + int(threadIdx.x) * VEC; e < b1; e += NT * VEC) cp_async16(slot + off + e, row + e);
+  const int h1 = b0 < e1 ? b0 : e1;
+  for (int e = e0 + int(threadIdx.x); e < h1; e += NT) slot[off + e] = row[e];
+  const int t0 = b1 > h1 ? b1 : h1;
+  for (int e = t0 + int(threadIdx.x); e < e1; e += NT) slot[off + e] = row[e];
 }
 
 template <typename T>
-__global__ void __launch_bounds__(NT) scatter_cols_kernel(const T *__restrict__ src1, int64_t ld1,
-                                                         const T *__restrict__ src2, int64_t ld2, int split,
-                                                         int64_t rows, int d, const int32_t *__restrict__ perm,
-                                                         T *__restrict__ dst, int64_t ld_dst,
-                                                         const int32_t *__restrict__ rowmap, int rows_per_cta,
-                                                         int slot) {
-  using IO = RowIO<T>;
-  constexpr int VEC = IO::VEC;
+__global__ void __launch_bounds__(NT) permute_rows_kernel(const PermArgs<T> a) {
+  constexpr int VEC = 16 / sizeof(T);
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  int32_t *sperm = reinterpret_cast<int32_t *>(smem_raw);
-  T *srows = reinterpret_cast<T *>(smem_raw + perm_bytes_dev(d));
-  for (int i = threadIdx.x; i < d; i += NT) sperm[i] = perm[i];
-  const int gpr = (d + VEC - 1) / VEC;
-  const int64_t nchunks = (rows + rows_per_cta - 1) / rows_per_cta;
-  for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x) {
-    const int64_t r0 = c * rows_per_cta;
-    const int nr = int(rows - r0 < rows_per_cta ? rows - r0 : rows_per_cta);
-    __syncthreads();
-    // load frame rows (aligned vectors), scatter into the slot at natural positions
-    for (int idx = threadIdx.x; idx < nr * gpr; idx += NT) {
-      const int r = idx / gpr, q = idx % gpr;
-      T *drow = dst + (rowmap ? int64_t(rowmap[r0 + r]) : (r0 + r)) * ld_dst;
-      T *s = srows + int64_t(r) * slot + IO::misalign(drow);
-      const int i0 = q * VEC;
+  uint16_t *map = reinterpret_cast<uint16_t *>(smem_raw);
+  T *ring = reinterpret_cast<T *>(smem_raw + ((a.d * 2 + 15) & ~15));
+  const int d = a.d;
+  if (a.inverse) {
+    for (int i = threadIdx.x; i < d; i += NT) map[a.perm[i]] = uint16_t(i);
+  } else {
+    for (int i = threadIdx.x; i < d; i += NT) map[i] = uint16_t(a.perm[i]);
+  }
+  const int split = a.split < d ? a.split : d;
+
+  // rows of this CTA: r_k = blockIdx.x + k * gridDim.x, k < count
+  const int64_t first = blockIdx.x, stride = gridDim.x;
+  const int64_t count = first < a.rows ? (a.rows - first + stride - 1) / stride : 0;
+  auto src1_row = [&](int64_t r) {
+    return a.src1 + (a.src_rowmap ? int64_t(a.src_rowmap[r]) : r) * a.ld1;
+  };
+  auto issue = [&](int64_t k) {
+    const int64_t r = first + k * stride;
+    T *slot = ring + int64_t(k % NB) * a.slot;
+    const T *r1 = src1_row(r);
+    const int off = misalign(r1);
+    load_part(r1, 0, split, slot, off);
+    if (split < d) {
+      const T *r2 = a.src2 + (a.src_rowmap ? int64_t(a.src_rowmap[r]) : r) * a.ld2;
+      load_part(r2, split, d, slot, off);
+    }
+  };
+
+  for (int k = 0; k < NB - 1; ++k) {
+    if (k < count) issue(k);
+    cp_async_commit();
+  }
+  __syncthreads();  // map is complete
+  for (int64_t k = 0; k < count; ++k) {
+    if (k + NB - 1 < count) issue(k + NB - 1);
+    cp_async_commit();
+    cp_async_wait_ring();  // this thread's copies of row k have landed
+    __syncthreads();       // ... and every other thread's
+    const int64_t r = first + k * stride;
+    const T *s = ring + int64_t(k % NB) * a.slot + misalign(src1_row(r));
+    T *drow = a.dst1 + (a.dst_rowmap ? int64_t(a.dst_rowmap[r]) : r) * a.ldd1;
+    T *d2row = a.dst2 ? a.dst2 + r * a.ldd2 : nullptr;
+    const int doff = misalign(drow);
+    const int units = (doff + d + VEC - 1) / VEC;
+    for (int u = threadIdx.x; u < units; u += NT) {
+      const int j0 = u * VEC - doff;  // output column of the unit's first lane
       alignas(16) T v[VEC];
-      if (i0 + VEC <= split) {
-        *reinterpret_cast<uint4 *>(v) = __ldg(reinterpret_cast<const uint4 *>(src1 + (r0 + r) * ld1 + i0));
-      } else if (i0 >= split) {
-        *reinterpret_cast<uint4 *>(v) = __ldg(reinterpret_cast<const uint4 *>(src2 + (r0 + r) * ld2 + i0));
+      if (j0 >= 0 && j0 + VEC <= d) {
+        if ((j0 & 7) == 0) {  // eight map entries in one 16-byte shared load
+          const uint4 mv = *reinterpret_cast<const uint4 *>(map + j0);
+          const uint16_t *mm = reinterpret_cast<const uint16_t *>(&mv);
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) v[e] = s[mm[e]];
+        } else {
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) v[e] = s[map[j0 + e]];
+        }
+        *reinterpret_cast<uint4 *>(drow + j0) = *reinterpret_cast<const uint4 *>(v);
+        if (d2row && j0 + VEC > a.dsplit) {
+          if (j0 >= a.dsplit && doff == 0) {
+            *reinterpret_cast<uint4 *>(d2row + j0) = *reinterpret_cast<const uint4 *>(v);
+          } else {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e)
+              if (j0 + e >= a.dsplit) d2row[j0 + e] = v[e];
+          }
+        }
       } else {
+#pragma unroll
         for (int e = 0; e < VEC; ++e) {
-          const int i = i0 + e;
-          if (i < d) v[e] = (i < split) ? src1[(r0 + r) * ld1 + i] : src2[(r0 + r) * ld2 + i];
+          const int j = j0 + e;
+          if (j >= 0 && j < d) {
+            const T x = s[map[j]];
+            drow[j] = x;
+            if (d2row && j >= a.dsplit) d2row[j] = x;
+          }
         }
       }
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        const int i = i0 + e;
-        if (i < d) s[sperm[i]] = v[e];
-      }
     }
-    __syncthreads();
-    const T *drow0 = dst + (rowmap ? int64_t(rowmap[r0]) : r0) * ld_dst;
-    const int upr = IO::units(drow0, d) + 1;
-    for (int idx = threadIdx.x; idx < nr * upr; idx += NT) {
-      const int r = idx / upr, u = idx % upr;
-      T *drow = dst + (rowmap ? int64_t(rowmap[r0 + r]) : (r0 + r)) * ld_dst;
-      if (u < IO::units(drow, d)) IO::store_unit(drow, d, u, srows + int64_t(r) * slot);
-    }
+    __syncthreads();  // slot k % NB may be refilled by the next iteration's prefetch
   }
+  cp_async_wait_all();
+}
+
+template <typename T>
+poet_status launch_permute(PermArgs<T> a, cudaStream_t st, const char *kind) {
+  if (a.rows <= 0 || a.d <= 0) return POET_OK;
+  POET_REQUIRE(a.d <= 65535, "permute: dimension %d too large", a.d);
+  constexpr int VEC = 16 / sizeof(T);
+  a.slot = int(round_up(a.d + VEC, VEC));
+  const size_t smem = size_t(round_up(int64_t(a.d) * 2, 16)) + size_t(NB) * a.slot * sizeof(T);
+  POET_REQUIRE(smem <= 220 * 1024, "permute: rows of %d elements do not fit in shared memory", a.d);
+  static int configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && configured[dev] < int(smem)) {
+    POET_CUDA_TRY(cudaFuncSetAttribute(permute_rows_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+    configured[dev] = int(smem);
+  }
+  int per_sm = 0;
+  POET_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_rows_kernel<T>, NT, smem));
+  if (per_sm < 1) per_sm = 1;
+  const int64_t cap = int64_t(num_sms()) * per_sm;
+  const int grid = int(a.rows < cap ? a.rows : cap);
+  TraceScope ts(kind, 0.0, double(a.rows) * a.d * sizeof(T) * 2.0, st);
+  permute_rows_kernel<T><<<grid, NT, smem, st>>>(a);
+  count_launch();
+  return launch_status(kind);
 }
 
 }  // namespace
 
-// shared-memory plan: permutation (d ints, rounded to 16 bytes) + rows
-static void plan_rows(int d, size_t esz, int64_t rows, int *rows_per_cta, int *slot, size_t *smem) {
-  const int vec = int(16 / esz);
-  *slot = int(round_up(d + 2 * vec, vec));  // misalignment offset + one spare unit
-  const size_t perm_bytes = size_t(round_up(int64_t(d) * 4, 16));
-  const size_t budget = 96 * 1024;
-  int r = int((budget > perm_bytes ? budget - perm_bytes : 0) / (size_t(*slot) * esz));
-  if (r < 1) r = 1;
-  if (r > 16) r = 16;
-  if (r > rows) r = int(rows > 0 ? rows : 1);
-  *rows_per_cta = r;
-  *smem = perm_bytes + size_t(r) * size_t(*slot) * esz;
-}
-
 poet_status gather_cols(int dtype, const void *src, int64_t ld_src, const int32_t *rowmap, int64_t rows, int d,
                         const int32_t *perm, void *dst, int64_t ld_dst, void *dst2, int64_t ld_dst2, int split,
                         cudaStream_t st) {
-  if (rows <= 0 || d <= 0) return POET_OK;
-  int rpc, slot;
-  size_t smem;
-  plan_rows(d, esize(dtype), rows, &rpc, &slot, &smem);
-  const int64_t chunks = (rows + rpc - 1) / rpc;
-  const int grid = int(chunks < 2 * num_sms() ? chunks : 2 * num_sms());
-  TraceScope ts("gather", 0.0, double(rows) * d * esize(dtype) * 2.0, st);
-  count_launch();
-  if (dtype == POET_BF16) {
-    POET_CUDA_TRY(cudaFuncSetAttribute(gather_cols_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
-    gather_cols_kernel<bf16><<<grid, NT, smem, st>>>(static_cast<const bf16 *>(src), ld_src, rowmap, rows, d, perm,
-                                                     static_cast<bf16 *>(dst), ld_dst, static_cast<bf16 *>(dst2),
-                                                     ld_dst2, split, rpc, slot);
-  } else {
-    POET_CUDA_TRY(cudaFuncSetAttribute(gather_cols_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
-    gather_cols_kernel<float><<<grid, NT, smem, st>>>(static_cast<const float *>(src), ld_src, rowmap, rows, d, perm,
-                                                      static_cast<float *>(dst), ld_dst, static_cast<float *>(dst2),
-                                                      ld_dst2, split, rpc, slot);
-  }
-  return launch_status("gather_cols");
+  POET_REQUIRE((reinterpret_cast<uintptr_t>(dst) & 15) == 0 && ld_dst * int64_t(esize(dtype)) % 16 == 0,
+               "gather: frame rows must be 16-byte aligned");
+  auto fill = [&](auto *tag) {
+    using T = std::remove_pointer_t<decltype(tag)>;
+    PermArgs<T> a{};
+    a.src1 = static_cast<const T *>(src); a.ld1 = ld_src;
+    a.src2 = nullptr; a.ld2 = 0; a.split = d;
+    a.src_rowmap = rowmap;
+    a.rows = rows; a.d = d;
+    a.perm = perm; a.inverse = 0;
+    a.dst1 = static_cast<T *>(dst); a.ldd1 = ld_dst;
+    a.dst2 = static_cast<T *>(dst2); a.ldd2 = ld_dst2; a.dsplit = dst2 ? split : d;
+    a.dst_rowmap = nullptr;
+    return launch_permute<T>(a, st, "gather");
+  };
+  return dtype == POET_BF16 ? fill(static_cast<bf16 *>(nullptr)) : fill(static_cast<float *>(nullptr));
 }
 
 poet_status scatter_cols(int dtype, const void *src1, int64_t ld1, const void *src2, int64_t ld2, int split,
                          int64_t rows, int d, const int32_t *perm, void *dst, int64_t ld_dst, const int32_t *rowmap,
                          cudaStream_t st) {
-  if (rows <= 0 || d <= 0) return POET_OK;
-  int rpc, slot;
-  size_t smem;
-  plan_rows(d, esize(dtype), rows, &rpc, &slot, &smem);
-  const int64_t chunks = (rows + rpc - 1) / rpc;
-  const int grid = int(chunks < 2 * num_sms() ? chunks : 2 * num_sms());
-  TraceScope ts("scatter", 0.0, double(rows) * d * esize(dtype) * 2.0, st);
-  count_launch();
-  if (dtype == POET_BF16) {
-    POET_CUDA_TRY(cudaFuncSetAttribute(scatter_cols_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
-    scatter_cols_kernel<bf16><<<grid, NT, smem, st>>>(static_cast<const bf16 *>(src1), ld1,
-                                                      static_cast<const bf16 *>(src2), ld2, split, rows, d, perm,
-                                                      static_cast<bf16 *>(dst), ld_dst, rowmap, rpc, slot);
-  } else {
-    POET_CUDA_TRY(cudaFuncSetAttribute(scatter_cols_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
-    scatter_cols_kernel<float><<<grid, NT, smem, st>>>(static_cast<const float *>(src1), ld1,
-                                                       static_cast<const float *>(src2), ld2, split, rows, d, perm,
-                                                       static_cast<float *>(dst), ld_dst, rowmap, rpc, slot);
-  }
-  return launch_status("scatter_cols");
+  const size_t es = esize(dtype);
+  POET_REQUIRE((reinterpret_cast<uintptr_t>(src1) & 15) == 0 && ld1 * int64_t(es) % 16 == 0 &&
+                   (split >= d || ((reinterpret_cast<uintptr_t>(src2) & 15) == 0 && ld2 * int64_t(es) % 16 == 0)),
+               "scatter: frame rows must be 16-byte aligned");
+  auto fill = [&](auto *tag) {
+    using T = std::remove_pointer_t<decltype(tag)>;
+    PermArgs<T> a{};
+    a.src1 = static_cast<const T *>(src1); a.ld1 = ld1;
+    a.src2 = static_cast<const T *>(src2); a.ld2 = ld2; a.split = split;
+    a.src_rowmap = nullptr;
+    a.rows = rows; a.d = d;
+    a.perm = perm; a.inverse = 1;
+    a.dst1 = static_cast<T *>(dst); a.ldd1 = ld_dst;
+    a.dst2 = nullptr; a.ldd2 = 0; a.dsplit = d;
+    a.dst_rowmap = rowmap;
+    return launch_permute<T>(a, st, "scatter");
+  };
+  return dtype == POET_BF16 ? fill(static_cast<bf16 *>(nullptr)) : fill(static_cast<float *>(nullptr));
 }
 
 }  // namespace poet

@@ -216,6 +216,21 @@ poet_status gemm_run(const Gemm &g, cudaStream_t st) {
   return gemm_simt(g, st);
 }
 
+poet_status gemm_run_many(const Gemm *gs, int count, cudaStream_t st) {
+  if (count <= 0) return POET_OK;
+  double flop = 0.0, bytes = 0.0;
+  for (int i = 0; i < count; ++i) {
+    const Gemm &g = gs[i];
+    const double mnb = double(g.M) * g.N * g.batch;
+    flop += 2.0 * mnb * g.K;
+    bytes += double(esize(g.dtype)) * (double(g.M) + g.N) * g.K * g.batch +
+             mnb * ((g.outF ? 4.0 : 0.0) + (g.outD ? double(esize(g.dtype)) : 0.0) +
+                    (g.add ? double(esize(g.add_dtype)) : 0.0));
+  }
+  TraceScope ts(gs[0].tag, flop, bytes, st);
+  return gemm_tc_many(gs, count, st);
+}
+
 }  // namespace poet
 
 using namespace poet;
@@ -348,29 +363,15 @@ poet_status poet_forward(const poet_layer *L, const void *x, int64_t T, void *y,
   return scatter_cols(dt, ysrc, lg.ldm, vf, lg.ldm, gR.covered, T, int(lg.m), L->R.perm, y, lg.m, nullptr, st);
 }
 
-poet_status poet_backward(const poet_layer *L, const void *saved, const void *dy, int64_t T, void *dx,
-                          float *dtheta_R, float *dtheta_P, void *ws, size_t ws_bytes, poet_stream stream) {
-  clear_error();
-  LayerGeom lg;
-  POET_TRY(check_layer(L, &lg, true));
-  POET_REQUIRE(T >= 0 && T <= (int64_t(1) << 31) - 1, "poet_backward: T=%lld out of range", (long long)T);
-  const SideGeom &gR = lg.R, &gP = lg.P;
-  POET_REQUIRE(gR.nprim == 0 || gR.size < 2 || dtheta_R, "poet_backward: dtheta_R is NULL");
-  POET_REQUIRE(gP.nprim == 0 || gP.size < 2 || dtheta_P, "poet_backward: dtheta_P is NULL");
-  const WsLayout w = ws_layout(lg, T);
-  if (!ws || ws_bytes < w.bytes || !aligned256(ws)) {
-    set_error("poet_backward: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, w.bytes);
-    return POET_ENOMEM_WS;
-  }
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+static poet_status backward_core(const poet_layer *L, const LayerGeom &lg, char *wb, const WsLayout &w,
+                                 const void *saved, const void *dy, int64_t T, void *dx, float *GR, float *GP,
+                                 cudaStream_t st) {
   const int dt = lg.dtype;
   const size_t es = esize(dt);
-  char *wb = static_cast<char *>(ws);
-  float *GR = reinterpret_cast<float *>(wb + w.GR);
-  float *GP = reinterpret_cast<float *>(wb + w.GP);
+  const SideGeom &gR = lg.R, &gP = lg.P;
   if (T > 0) {
-    POET_REQUIRE(dy && dx && aligned_elem(dy, dt) && aligned_elem(dx, dt), "poet_backward: dy/dx NULL or misaligned");
-    POET_REQUIRE(saved && aligned256(saved), "poet_backward: saved NULL or not 256-byte aligned");
+    POET_REQUIRE(dy && dx && aligned_elem(dy, dt) && aligned_elem(dx, dt), "backward: dy/dx NULL or misaligned");
+    POET_REQUIRE(saved && aligned256(saved), "backward: saved NULL or not 256-byte aligned");
     const char *sv = static_cast<const char *>(saved);
     const void *xf = sv;
     const void *vf = sv + align256(size_t(T) * lg.ldn * es);
@@ -410,11 +411,109 @@ poet_status poet_backward(const poet_layer *L, const void *saved, const void *dy
     if (gR.nprim > 0) POET_CUDA_TRY(cudaMemsetAsync(GR, 0, size_t(gR.all_elems()) * 4, st));
     if (gP.nprim > 0) POET_CUDA_TRY(cudaMemsetAsync(GP, 0, size_t(gP.all_elems()) * 4, st));
   }
+  return POET_OK;
+}
+
+poet_status poet_backward(const poet_layer *L, const void *saved, const void *dy, int64_t T, void *dx,
+                          float *dtheta_R, float *dtheta_P, void *ws, size_t ws_bytes, poet_stream stream) {
+  clear_error();
+  LayerGeom lg;
+  POET_TRY(check_layer(L, &lg, true));
+  POET_REQUIRE(T >= 0 && T <= (int64_t(1) << 31) - 1, "poet_backward: T=%lld out of range", (long long)T);
+  const SideGeom &gR = lg.R, &gP = lg.P;
+  POET_REQUIRE(gR.nprim == 0 || gR.size < 2 || dtheta_R, "poet_backward: dtheta_R is NULL");
+  POET_REQUIRE(gP.nprim == 0 || gP.size < 2 || dtheta_P, "poet_backward: dtheta_P is NULL");
+  const WsLayout w = ws_layout(lg, T);
+  if (!ws || ws_bytes < w.bytes || !aligned256(ws)) {
+    set_error("poet_backward: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, w.bytes);
+    return POET_ENOMEM_WS;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char *wb = static_cast<char *>(ws);
+  float *GR = reinterpret_cast<float *>(wb + w.GR);
+  float *GP = reinterpret_cast<float *>(wb + w.GP);
+  POET_TRY(backward_core(L, lg, wb, w, saved, dy, T, dx, GR, GP, st));
   // a8: through the Cayley-Neumann map to the packed parameters
   void *scratch = wb + w.cnp;
-  if (gR.nprim > 0 && gR.size >= 2) POET_TRY(cnp_backward(&L->R, gR, dt, GR, dtheta_R, scratch, st));
-  if (gP.nprim > 0 && gP.size >= 2) POET_TRY(cnp_backward(&L->P, gP, dt, GP, dtheta_P, scratch, st));
+  if (gR.nprim > 0 && gR.size >= 2) POET_TRY(cnp_backward(&L->R, gR, lg.dtype, GR, dtheta_R, scratch, st));
+  if (gP.nprim > 0 && gP.size >= 2) POET_TRY(cnp_backward(&L->P, gP, lg.dtype, GP, dtheta_P, scratch, st));
   return POET_OK;
+}
+
+poet_status poet_backward_blocks(const poet_layer *L, const void *saved, const void *dy, int64_t T, void *dx,
+                                 float *G_R, float *G_P, void *ws, size_t ws_bytes, poet_stream stream) {
+  clear_error();
+  LayerGeom lg;
+  POET_TRY(check_layer(L, &lg, true));
+  POET_REQUIRE(T >= 0 && T <= (int64_t(1) << 31) - 1, "poet_backward_blocks: T=%lld out of range", (long long)T);
+  POET_REQUIRE(lg.R.nprim == 0 || (G_R && (reinterpret_cast<uintptr_t>(G_R) & 15) == 0),
+               "poet_backward_blocks: G_R NULL or not 16-byte aligned");
+  POET_REQUIRE(lg.P.nprim == 0 || (G_P && (reinterpret_cast<uintptr_t>(G_P) & 15) == 0),
+               "poet_backward_blocks: G_P NULL or not 16-byte aligned");
+  const WsLayout w = ws_layout(lg, T);
+  if (!ws || ws_bytes < w.bytes || !aligned256(ws)) {
+    set_error("poet_backward_blocks: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, w.bytes);
+    return POET_ENOMEM_WS;
+  }
+  return backward_core(L, lg, static_cast<char *>(ws), w, saved, dy, T, dx, G_R, G_P,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t poet_block_grad_bytes(const poet_side *side) {
+  SideGeom g;
+  if (!side_geom(side, &g)) return 0;
+  return size_t(g.all_elems()) * 4;
+}
+
+poet_status poet_cayley_neumann_many(const poet_side *sides, int32_t count, int32_t dtype, poet_stream stream) {
+  clear_error();
+  POET_REQUIRE(count >= 0 && (count == 0 || sides), "poet_cayley_neumann_many: bad side list");
+  POET_REQUIRE(dtype == POET_F32 || dtype == POET_BF16, "poet_cayley_neumann_many: bad dtype %d", dtype);
+  std::vector<SideGeom> geoms(count);
+  for (int i = 0; i < count; ++i) {
+    POET_REQUIRE(side_geom(&sides[i], &geoms[i]), "poet_cayley_neumann_many: side %d malformed", i);
+    if (geoms[i].nprim == 0) continue;
+    POET_REQUIRE((sides[i].theta || geoms[i].packed_per() == 0) && sides[i].state && aligned256(sides[i].state),
+                 "poet_cayley_neumann_many: side %d theta/state NULL or misaligned", i);
+  }
+  return cnp_forward_many(sides, geoms.data(), count, dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t poet_cayley_neumann_grad_many_workspace_bytes(const poet_side *sides, int32_t count, int32_t dtype) {
+  if (count < 0 || (count > 0 && !sides) || (dtype != POET_F32 && dtype != POET_BF16)) return 0;
+  size_t total = 0;
+  for (int i = 0; i < count; ++i) {
+    SideGeom g;
+    if (!side_geom(&sides[i], &g)) return 0;
+    total += align256(cnp_scratch_bytes(g, dtype));
+  }
+  return total;
+}
+
+poet_status poet_cayley_neumann_grad_many(const poet_side *sides, const float *const *G, float *const *dtheta,
+                                          int32_t count, int32_t dtype, void *ws, size_t ws_bytes,
+                                          poet_stream stream) {
+  clear_error();
+  POET_REQUIRE(count >= 0 && (count == 0 || (sides && G && dtheta)), "poet_cayley_neumann_grad_many: bad lists");
+  POET_REQUIRE(dtype == POET_F32 || dtype == POET_BF16, "poet_cayley_neumann_grad_many: bad dtype %d", dtype);
+  std::vector<SideGeom> geoms(count);
+  std::vector<void *> scratch(count, nullptr);
+  size_t off = 0;
+  for (int i = 0; i < count; ++i) {
+    POET_REQUIRE(side_geom(&sides[i], &geoms[i]), "poet_cayley_neumann_grad_many: side %d malformed", i);
+    if (geoms[i].nprim == 0 || geoms[i].size < 2) continue;
+    POET_REQUIRE(sides[i].state && aligned256(sides[i].state) && G[i] && dtheta[i] &&
+                     (reinterpret_cast<uintptr_t>(G[i]) & 15) == 0,
+                 "poet_cayley_neumann_grad_many: side %d state/G/dtheta NULL or misaligned", i);
+    scratch[i] = static_cast<char *>(ws) + off;
+    off += align256(cnp_scratch_bytes(geoms[i], dtype));
+  }
+  if (off > 0 && (!ws || ws_bytes < off || !aligned256(ws))) {
+    set_error("poet_cayley_neumann_grad_many: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, off);
+    return POET_ENOMEM_WS;
+  }
+  return cnp_backward_many(sides, geoms.data(), count, dtype, G, dtheta, scratch.data(),
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 poet_status poet_prepare(poet_layer *L, poet_stream stream) {

@@ -115,6 +115,10 @@ poet_status gemm_run(const Gemm &g, cudaStream_t st);       // picks the engine
 poet_status gemm_simt(const Gemm &g, cudaStream_t st);      // CUDA-core FMA engine
 bool gemm_tc_supported(const Gemm &g);                      // tcgen05 engine can take g
 poet_status gemm_tc(const Gemm &g, cudaStream_t st);        // tcgen05 engine
+// Many independent problems: grouped tcgen05 launches where possible, the rest
+// on the CUDA-core engine.  gemm_run_many adds tracing around it.
+poet_status gemm_tc_many(const Gemm *gs, int count, cudaStream_t st);
+poet_status gemm_run_many(const Gemm *gs, int count, cudaStream_t st);
 bool gemm_tc_enabled();
 
 // ------------------------------------------------------------------ data movement
@@ -139,6 +143,11 @@ poet_status cnp_forward(const poet_side *side, const SideGeom &g, int dtype, cud
 poet_status cnp_backward(const poet_side *side, const SideGeom &g, int dtype, const float *G,
                          float *dtheta, void *scratch, cudaStream_t st);
 size_t cnp_scratch_bytes(const SideGeom &g, int dtype);
+// The same for many sides at once; their GEMM steps share grouped launches.
+// G[i]: float [nprim][ld][ld]; scratch[i]: cnp_scratch_bytes(geoms[i], dtype) bytes each.
+poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int count, int dtype, cudaStream_t st);
+poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int count, int dtype,
+                              const float *const *G, float *const *dtheta, void *const *scratch, cudaStream_t st);
 // out = G (dense [nprim][size][size]) re-laid as [nprim][ld][ld] with zero padding
 poet_status pad_blocks(const float *G, const SideGeom &g, float *out, cudaStream_t st);
 

@@ -70,6 +70,17 @@ _SIGS = {
                                  ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_float, ctypes.c_float,
                                  ctypes.c_void_p]),
     "poet_gemm_engine": (ctypes.c_int32, [ctypes.c_int32]),
+    "poet_block_grad_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_side)]),
+    "poet_cayley_neumann_many": (ctypes.c_int, [ctypes.POINTER(poet_side), ctypes.c_int32, ctypes.c_int32,
+                                                ctypes.c_void_p]),
+    "poet_backward_blocks": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p, ctypes.c_void_p,
+                                            ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "poet_cayley_neumann_grad_many_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_side), ctypes.c_int32,
+                                                                        ctypes.c_int32]),
+    "poet_cayley_neumann_grad_many": (ctypes.c_int, [ctypes.POINTER(poet_side), ctypes.POINTER(ctypes.c_void_p),
+                                                     ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32, ctypes.c_int32,
+                                                     ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "poet_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "poet_launch_count": (ctypes.c_int64, []),
     "poet_trace_enable": (ctypes.c_int, [ctypes.c_int32]),
@@ -196,6 +207,38 @@ def poet_sync_status(stream=None):
     _check(lib().poet_sync_status(_stream(stream)))
 
 
+def poet_block_grad_bytes(side: poet_side) -> int:
+    return lib().poet_block_grad_bytes(ctypes.byref(side))
+
+
+def _side_array(sides):
+    arr = (poet_side * max(len(sides), 1))()
+    for i, sd in enumerate(sides):
+        arr[i] = sd
+    return arr
+
+
+def poet_cayley_neumann_many(sides, dtype: int, stream=None):
+    _check(lib().poet_cayley_neumann_many(_side_array(sides), len(sides), dtype, _stream(stream)))
+
+
+def poet_backward_blocks(layer: poet_layer, saved, dy, T: int, dx, G_R, G_P, ws, stream=None):
+    _check(lib().poet_backward_blocks(ctypes.byref(layer), _ptr(saved), _ptr(dy), T, _ptr(dx), _ptr(G_R), _ptr(G_P),
+                                      _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def poet_cayley_neumann_grad_many_workspace_bytes(sides, dtype: int) -> int:
+    return lib().poet_cayley_neumann_grad_many_workspace_bytes(_side_array(sides), len(sides), dtype)
+
+
+def poet_cayley_neumann_grad_many(sides, G, dtheta, dtype: int, ws, stream=None):
+    n = len(sides)
+    gp = (ctypes.c_void_p * max(n, 1))(*[None if t is None else t.data_ptr() for t in G])
+    dp = (ctypes.c_void_p * max(n, 1))(*[None if t is None else t.data_ptr() for t in dtheta])
+    _check(lib().poet_cayley_neumann_grad_many(_side_array(sides), gp, dp, n, dtype, _ptr(ws),
+                                               0 if ws is None else ws.numel(), _stream(stream)))
+
+
 def poet_launch_count() -> int:
     return lib().poet_launch_count()
 
@@ -320,3 +363,41 @@ class PoetLayer:
 
     def workspace_bytes(self, T: int) -> int:
         return poet_workspace_bytes(self._L, T)
+
+    def block_grad_buffers(self):
+        """Float buffers for the per-primitive gradients of R and P ([nprim][ld][ld])."""
+        dev = self.W0.device
+        return (torch.empty(max(poet_block_grad_bytes(self._L.R) // 4, 4), dtype=torch.float32, device=dev),
+                torch.empty(max(poet_block_grad_bytes(self._L.P) // 4, 4), dtype=torch.float32, device=dev))
+
+    def backward_blocks(self, saved, dy, G_R, G_P, dx=None, ws=None, stream=None):
+        """a5..a7: dx and the per-primitive gradients (a8 left to cayley_neumann_grad_many)."""
+        T = dy.shape[0]
+        if dx is None:
+            dx = torch.empty(T, self.n, dtype=dy.dtype, device=dy.device)
+        poet_backward_blocks(self._L, saved, dy, T, dx, G_R, G_P, self.workspace(T) if ws is None else ws, stream)
+        return dx
+
+
+def cayley_neumann_many(layers, stream=None):
+    """a1 for both sides of every layer (all the same dtype) in shared launches."""
+    if not layers:
+        return
+    sides = [s for L in layers for s in (L.struct.R, L.struct.P)]
+    poet_cayley_neumann_many(sides, layers[0].dtype, stream)
+
+
+def cayley_neumann_grad_many_workspace_bytes(layers) -> int:
+    if not layers:
+        return 0
+    sides = [s for L in layers for s in (L.struct.R, L.struct.P)]
+    return poet_cayley_neumann_grad_many_workspace_bytes(sides, layers[0].dtype)
+
+
+def cayley_neumann_grad_many(layers, G, dtheta, ws, stream=None):
+    """a8 for every layer: G = [(G_R, G_P), ...], dtheta = [(dtheta_R, dtheta_P), ...]."""
+    if not layers:
+        return
+    sides = [s for L in layers for s in (L.struct.R, L.struct.P)]
+    poet_cayley_neumann_grad_many(sides, [t for pair in G for t in pair], [t for pair in dtheta for t in pair],
+                                  layers[0].dtype, ws, stream)

@@ -202,3 +202,61 @@ def test_gemm_engine(cuda, dtype, M, N, K, batch, amaj, bmaj, alpha, beta):
     poet.poet_sync_status()
     ref = alpha * np.einsum("bmk,bnk->bmn", A.astype(np.float64), B.astype(np.float64)) + beta * C0
     assert rel_fro(C.float().cpu().numpy(), ref) <= (1e-5 if dtype == I.F32 else 8e-3)
+
+
+# ------------------------------------------------------------------ many layers at once
+
+def _make_layer(cuda, case):
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    W0, thR, thP, x, dy = case.arrays()
+    tdt = poet.torch_dtype(case.dtype)
+    L = poet.PoetLayer(cuda.from_numpy(W0).to("cuda", tdt), cuda.from_numpy(thR).cuda(), cuda.from_numpy(thP).cuda(),
+                       mode=case.modeR, b=case.bR, modeP=case.modeP, bP=case.bP, k=case.k, seed=case.seed,
+                       layer_id=case.layer_id)
+    L.prepare()
+    return L, cuda.from_numpy(x).to("cuda", tdt), cuda.from_numpy(dy).to("cuda", tdt), (W0, thR, thP, x, dy)
+
+
+MANY_CASES = [  # different sizes, modes and Neumann orders in one call
+    Case(512, 512, I.FS, 0, I.FS, 0, 4, 300, I.BF16, 0.02, layer_id=21),
+    Case(1376, 512, I.FS, 0, I.FS, 0, 4, 300, I.BF16, 0.02, layer_id=22),
+    Case(1024, 768, I.BS, 256, I.BS, 256, 4, 300, I.BF16, 0.02, layer_id=23),
+    Case(640, 512, I.BS, 128, I.FS, 0, 2, 300, I.BF16, 0.03, layer_id=24),
+]
+
+
+def test_many_sides_match_single_calls_and_oracle(cuda):
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    built = [_make_layer(cuda, c) for c in MANY_CASES]
+    layers = [b[0] for b in built]
+    # a1: grouped launch vs one call per side (same tiles, same order: bitwise equal)
+    poet.cayley_neumann_many(layers)
+    many_R = [L.state_R.clone() for L in layers]
+    for L in layers:
+        L.cayley_neumann()
+    for L, r in zip(layers, many_R):
+        n = poet.poet_block_grad_bytes(L.struct.R) // 2
+        assert cuda.equal(L.state_R[:n], r[:n])
+    # a5..a8 split: backward_blocks + grouped a8 vs poet_backward, and both vs the oracle
+    G, dth, dth_ref = [], [], []
+    for (L, xt, dyt, arrs), case in zip(built, MANY_CASES):
+        y, saved = L.forward(xt)
+        gR, gP = L.block_grad_buffers()
+        dx = L.backward_blocks(saved, dyt, gR, gP)
+        G.append((gR, gP))
+        dth.append((cuda.empty_like(L.theta_R), cuda.empty_like(L.theta_P)))
+        dx1, dR1, dP1 = L.backward(saved, dyt)
+        assert cuda.equal(dx, dx1)
+        dth_ref.append((dR1, dP1))
+    ws = cuda.empty(max(poet.cayley_neumann_grad_many_workspace_bytes(layers), 1), dtype=cuda.uint8, device="cuda")
+    poet.cayley_neumann_grad_many(layers, G, dth, ws)
+    poet.poet_sync_status()
+    for (L, xt, dyt, arrs), case, (dR, dP), (dR1, dP1) in zip(built, MANY_CASES, dth, dth_ref):
+        ref = run_oracle(case, *arrs)
+        tol = TOL[case.dtype]
+        assert rel_fro(dR.cpu().numpy(), ref["dthetaR"]) <= tol
+        assert rel_fro(dP.cpu().numpy(), ref["dthetaP"]) <= tol
+        assert rel_fro(dR.cpu().numpy(), dR1.cpu().numpy()) <= 1e-3  # G sums differ only in atomic order
+        assert rel_fro(dP.cpu().numpy(), dP1.cpu().numpy()) <= 1e-3
