@@ -296,7 +296,8 @@ def run_poet(args):
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     smi_index = vis.split(",")[local] if vis else str(local)
     clocks = ClockSampler(smi_index)
-    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in variants] for _ in range(args.steps)]
+    # each variant runs its K steps back to back; the kernel trace is read per variant
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in variants]
     barrier()
     torch.cuda.synchronize()
     clocks.start()
@@ -305,21 +306,27 @@ def run_poet(args):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for s_ in range(args.steps):
-        for i, v in enumerate(variants):
-            ev[s_][i][0].record(stream)
+    traces = []
+    for i, v in enumerate(variants):
+        ev[i][0].record(stream)
+        for _ in range(args.steps):
             v.step(world)
-            ev[s_][i][1].record(stream)
+        ev[i][1].record(stream)
+        traces.append(poet.poet_trace_read())  # waits for this variant's recorded events
     t1.record(stream)
     torch.cuda.synchronize()
-    per_variant_ms = [sum(ev[s_][i][0].elapsed_time(ev[s_][i][1]) for s_ in range(args.steps))
-                      for i in range(len(variants))]
+    per_variant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(len(variants))]
     launches = poet.poet_launch_count() - launches0
     poet.poet_trace_enable(False)
     clk = clocks.stop()
     barrier()
     elapsed = t0.elapsed_time(t1)
-    trace = poet.poet_trace_read()
+    trace = {}
+    for tr in traces:
+        for k, r in tr.items():
+            a = trace.setdefault(k, {"launches": 0, "ms": 0.0, "flop": 0.0, "bytes": 0.0})
+            for f in a:
+                a[f] += r[f]
     poet.poet_sync_status()
     if dist is not None:
         t = torch.tensor([elapsed] + per_variant_ms, dtype=torch.float64, device=device)
@@ -398,7 +405,9 @@ def run_poet(args):
                    "parallelism": f"dp{world}", "l2": "inputs larger than L2 (no flush needed)"},
         "variants": {v.wl.name: {"ms_per_step": round(per_variant_ms[i] / args.steps, 3),
                                  "tokens_per_s": round(v.T * world / (per_variant_ms[i] / args.steps / 1e3), 1),
-                                 "merge_ms": round(merge.get(v.wl.name, float("nan")), 3) if merge else None}
+                                 "merge_ms": round(merge.get(v.wl.name, float("nan")), 3) if merge else None,
+                                 "kernels_ms_per_step": {k: round(r["ms"] / args.steps, 2) for k, r in
+                                                         sorted(traces[i].items(), key=lambda kv: -kv[1]["ms"])}}
                      for i, v in enumerate(variants)},
         "value_merge_amortized": (round(tokens_per_step / ((ms_per_step + sum(merge.values()) / 400.0) / 1e3), 1)
                                   if merge else None),

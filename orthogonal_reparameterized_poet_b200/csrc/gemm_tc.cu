@@ -223,6 +223,11 @@ struct Smem {
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
 
+// out[0..3] += (a, b, c, d) as one 16-byte reduction at L2
+__device__ __forceinline__ void red_add_v4(float *out, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(out), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
 template <bool A_MN, bool B_MN, int BN, int MAXP>
 __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_constant__ TcGroup<MAXP> g) {
   using S = Smem<BN>;
@@ -389,9 +394,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
         const int nvalid = min(32, p.N - gn0);
         if (p.atomic) {
           float *o = p.outF + int64_t(c.b) * p.of_b + int64_t(gm) * p.of_m + gn0;
+          if (nvalid == 32 && (reinterpret_cast<uintptr_t>(o) & 15) == 0) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j < nvalid) atomicAdd(o + j, alpha * __uint_as_float(r[j]));
+            for (int j = 0; j < 32; j += 4)
+              red_add_v4(o + j, alpha * __uint_as_float(r[j]), alpha * __uint_as_float(r[j + 1]),
+                         alpha * __uint_as_float(r[j + 2]), alpha * __uint_as_float(r[j + 3]));
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid) atomicAdd(o + j, alpha * __uint_as_float(r[j]));
+          }
           continue;
         }
         float v[32];
@@ -567,7 +579,8 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
     const int64_t mt = (gs[i].M + BM - 1) / BM, nt = (gs[i].N + t.BN - 1) / t.BN;
     base_tiles += mt * nt * gs[i].batch;
   }
-  const int split_want = int((int64_t(num_sms()) + base_tiles - 1) / (base_tiles > 0 ? base_tiles : 1));
+  // split K (atomic outputs only) as far as the tiles still fit in one wave
+  const int split_want = base_tiles > 0 && base_tiles < num_sms() ? int(num_sms() / base_tiles) : 1;
   grp.count = n;
   grp.errword = device_errword();
   grp.tile_start[0] = 0;

@@ -23,8 +23,9 @@
 namespace poet {
 namespace {
 
-constexpr int NT = 256;
-constexpr int NB = 4;  // ring depth (rows per CTA in flight)
+constexpr int MAX_WARPS = 8;          // warps per CTA (fewer for very long rows); each warp owns whole rows
+constexpr int NT = MAX_WARPS * 32;
+constexpr int NBW = 2;                // row slots per warp (one row prefetched while one is processed)
 
 template <typename T>
 struct PermArgs {
@@ -37,6 +38,7 @@ struct PermArgs {
   T *dst2; int64_t ldd2; int dsplit;  // columns >= dsplit also go here (nullptr: none)
   const int32_t *dst_rowmap;          // destination row of output row r (nullptr: r)
   int slot;                           // slot stride (elements, multiple of 16 bytes)
+  int map_len;                        // map entries allocated (>= round_up(d, 8) + 8)
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
@@ -46,7 +48,7 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem)), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_ring() { asm volatile("cp.async.wait_group %0;" ::"n"(NB - 1) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 template <typename T>
@@ -54,20 +56,94 @@ __device__ __forceinline__ int misalign(const T *p) {
   return int((reinterpret_cast<uintptr_t>(p) & 15) / sizeof(T));
 }
 
-// Copies of elements [e0, e1) of a global row into slot[off + e]
+// One warp copies elements [e0, e1) of a global row into slot[off + e]
 // (off = misalignment of the row start; the same for every part of a row).
 template <typename T>
-__device__ __forceinline__ void load_part(const T *row, int e0, int e1, T *slot, int off) {
+__device__ __forceinline__ void load_part(const T *row, int e0, int e1, T *slot, int off, int lane) {
   constexpr int VEC = 16 / sizeof(T);
   if (e1 <= e0) return;
   const int b0 = ((off + e0 + VEC - 1) / VEC) * VEC - off;  // first 16B-aligned element >= e0
   const int b1 = ((off + e1) / VEC) * VEC - off;            // end of the last whole aligned unit
   if (b0 < b1)
-    for (int e = b0 + int(threadIdx.x) * VEC; e < b1; e += NT * VEC) cp_async16(slot + off + e, row + e);
+    for (int e = b0 + lane * VEC; e < b1; e += 32 * VEC) cp_async16(slot + off + e, row + e);
   const int h1 = b0 < e1 ? b0 : e1;
-  for (int e = e0 + int(threadIdx.x); e < h1; e += NT) slot[off + e] = row[e];
+  for (int e = e0 + lane; e < h1; e += 32) slot[off + e] = row[e];
   const int t0 = b1 > h1 ? b1 : h1;
-  for (int e = t0 + int(threadIdx.x); e < e1; e += NT) slot[off + e] = row[e];
+  for (int e = t0 + lane; e < e1; e += 32) slot[off + e] = row[e];
+}
+
+// VEC consecutive map entries starting at j0 = u*VEC - DOFF, read as aligned
+// vectors (two when the destination row is misaligned).
+template <int VEC, int DOFF>
+__device__ __forceinline__ void map_entries(const uint16_t *map, int u, uint16_t (&m)[VEC]) {
+  if constexpr (VEC == 8) {
+    if constexpr (DOFF == 0) {
+      const uint4 a = *reinterpret_cast<const uint4 *>(map + 8 * u);
+      const uint16_t *pa = reinterpret_cast<const uint16_t *>(&a);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m[e] = pa[e];
+    } else {
+      const uint4 a = *reinterpret_cast<const uint4 *>(map + 8 * (u - 1));
+      const uint4 b = *reinterpret_cast<const uint4 *>(map + 8 * u);
+      const uint16_t *pa = reinterpret_cast<const uint16_t *>(&a);
+      const uint16_t *pb = reinterpret_cast<const uint16_t *>(&b);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m[e] = (8 - DOFF + e) < 8 ? pa[8 - DOFF + e] : pb[e - DOFF];
+    }
+  } else {  // VEC == 4: groups of four 16-bit entries
+    if constexpr (DOFF == 0) {
+      const uint2 a = *reinterpret_cast<const uint2 *>(map + 4 * u);
+      const uint16_t *pa = reinterpret_cast<const uint16_t *>(&a);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) m[e] = pa[e];
+    } else {
+      const uint2 a = *reinterpret_cast<const uint2 *>(map + 4 * (u - 1));
+      const uint2 b = *reinterpret_cast<const uint2 *>(map + 4 * u);
+      const uint16_t *pa = reinterpret_cast<const uint16_t *>(&a);
+      const uint16_t *pb = reinterpret_cast<const uint16_t *>(&b);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) m[e] = (4 - DOFF + e) < 4 ? pa[4 - DOFF + e] : pb[e - DOFF];
+    }
+  }
+}
+
+// Output row = slot gathered through map; drow misaligned by DOFF elements.
+template <typename T, int DOFF>
+__device__ __forceinline__ void emit_row(const PermArgs<T> &a, const uint16_t *map, const T *s, T *drow, T *d2row,
+                                         int lane) {
+  constexpr int VEC = 16 / sizeof(T);
+  const int d = a.d;
+  const int units = (DOFF + d + VEC - 1) / VEC;
+  for (int u = lane; u < units; u += 32) {
+    const int j0 = u * VEC - DOFF;  // output column of the unit's first lane
+    if (j0 >= 0 && j0 + VEC <= d) {
+      uint16_t m[VEC];
+      map_entries<VEC, DOFF>(map, u, m);
+      alignas(16) T v[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) v[e] = s[m[e]];
+      *reinterpret_cast<uint4 *>(drow + j0) = *reinterpret_cast<const uint4 *>(v);
+      if (d2row && j0 + VEC > a.dsplit) {
+        if (DOFF == 0 && j0 >= a.dsplit) {
+          *reinterpret_cast<uint4 *>(d2row + j0) = *reinterpret_cast<const uint4 *>(v);
+        } else {
+#pragma unroll
+          for (int e = 0; e < VEC; ++e)
+            if (j0 + e >= a.dsplit) d2row[j0 + e] = v[e];
+        }
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        const int j = j0 + e;
+        if (j >= 0 && j < d) {
+          const T x = s[map[j]];
+          drow[j] = x;
+          if (d2row && j >= a.dsplit) d2row[j] = x;
+        }
+      }
+    }
+  }
 }
 
 template <typename T>
@@ -75,85 +151,60 @@ __global__ void __launch_bounds__(NT) permute_rows_kernel(const PermArgs<T> a) {
   constexpr int VEC = 16 / sizeof(T);
   extern __shared__ __align__(16) unsigned char smem_raw[];
   uint16_t *map = reinterpret_cast<uint16_t *>(smem_raw);
-  T *ring = reinterpret_cast<T *>(smem_raw + ((a.d * 2 + 15) & ~15));
   const int d = a.d;
+  const int nthr = blockDim.x, warps = nthr / 32;
+  for (int i = threadIdx.x; i < a.map_len; i += nthr) map[i] = 0;
+  __syncthreads();
   if (a.inverse) {
-    for (int i = threadIdx.x; i < d; i += NT) map[a.perm[i]] = uint16_t(i);
+    for (int i = threadIdx.x; i < d; i += nthr) map[a.perm[i]] = uint16_t(i);
   } else {
-    for (int i = threadIdx.x; i < d; i += NT) map[i] = uint16_t(a.perm[i]);
+    for (int i = threadIdx.x; i < d; i += nthr) map[i] = uint16_t(a.perm[i]);
   }
-  const int split = a.split < d ? a.split : d;
+  __syncthreads();  // the only block-wide barriers: map is complete
 
-  // rows of this CTA: r_k = blockIdx.x + k * gridDim.x, k < count
-  const int64_t first = blockIdx.x, stride = gridDim.x;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  T *ring = reinterpret_cast<T *>(smem_raw + size_t(a.map_len) * 2) + int64_t(warp) * NBW * a.slot;
+  const int split = a.split < d ? a.split : d;
+  const int64_t first = int64_t(blockIdx.x) * warps + warp, stride = int64_t(gridDim.x) * warps;
   const int64_t count = first < a.rows ? (a.rows - first + stride - 1) / stride : 0;
+
   auto src1_row = [&](int64_t r) {
     return a.src1 + (a.src_rowmap ? int64_t(a.src_rowmap[r]) : r) * a.ld1;
   };
   auto issue = [&](int64_t k) {
     const int64_t r = first + k * stride;
-    T *slot = ring + int64_t(k % NB) * a.slot;
+    T *slot = ring + int64_t(k % NBW) * a.slot;
     const T *r1 = src1_row(r);
     const int off = misalign(r1);
-    load_part(r1, 0, split, slot, off);
+    load_part(r1, 0, split, slot, off, lane);
     if (split < d) {
       const T *r2 = a.src2 + (a.src_rowmap ? int64_t(a.src_rowmap[r]) : r) * a.ld2;
-      load_part(r2, split, d, slot, off);
+      load_part(r2, split, d, slot, off, lane);
     }
   };
 
-  for (int k = 0; k < NB - 1; ++k) {
-    if (k < count) issue(k);
-    cp_async_commit();
-  }
-  __syncthreads();  // map is complete
+  if (count > 0) issue(0);
+  cp_async_commit();
   for (int64_t k = 0; k < count; ++k) {
-    if (k + NB - 1 < count) issue(k + NB - 1);
+    if (k + 1 < count) issue(k + 1);
     cp_async_commit();
-    cp_async_wait_ring();  // this thread's copies of row k have landed
-    __syncthreads();       // ... and every other thread's
+    cp_async_wait_one();  // this lane's copies of row k have landed
+    __syncwarp();         // ... and every other lane's (scalar edges included)
     const int64_t r = first + k * stride;
-    const T *s = ring + int64_t(k % NB) * a.slot + misalign(src1_row(r));
+    const T *s = ring + int64_t(k % NBW) * a.slot + misalign(src1_row(r));
     T *drow = a.dst1 + (a.dst_rowmap ? int64_t(a.dst_rowmap[r]) : r) * a.ldd1;
     T *d2row = a.dst2 ? a.dst2 + r * a.ldd2 : nullptr;
-    const int doff = misalign(drow);
-    const int units = (doff + d + VEC - 1) / VEC;
-    for (int u = threadIdx.x; u < units; u += NT) {
-      const int j0 = u * VEC - doff;  // output column of the unit's first lane
-      alignas(16) T v[VEC];
-      if (j0 >= 0 && j0 + VEC <= d) {
-        if ((j0 & 7) == 0) {  // eight map entries in one 16-byte shared load
-          const uint4 mv = *reinterpret_cast<const uint4 *>(map + j0);
-          const uint16_t *mm = reinterpret_cast<const uint16_t *>(&mv);
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) v[e] = s[mm[e]];
-        } else {
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) v[e] = s[map[j0 + e]];
-        }
-        *reinterpret_cast<uint4 *>(drow + j0) = *reinterpret_cast<const uint4 *>(v);
-        if (d2row && j0 + VEC > a.dsplit) {
-          if (j0 >= a.dsplit && doff == 0) {
-            *reinterpret_cast<uint4 *>(d2row + j0) = *reinterpret_cast<const uint4 *>(v);
-          } else {
-#pragma unroll
-            for (int e = 0; e < VEC; ++e)
-              if (j0 + e >= a.dsplit) d2row[j0 + e] = v[e];
-          }
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          const int j = j0 + e;
-          if (j >= 0 && j < d) {
-            const T x = s[map[j]];
-            drow[j] = x;
-            if (d2row && j >= a.dsplit) d2row[j] = x;
-          }
-        }
-      }
+    switch (misalign(drow)) {
+      case 0: emit_row<T, 0>(a, map, s, drow, d2row, lane); break;
+      case 1: emit_row<T, 1>(a, map, s, drow, d2row, lane); break;
+      case 2: emit_row<T, 2>(a, map, s, drow, d2row, lane); break;
+      case 3: emit_row<T, 3>(a, map, s, drow, d2row, lane); break;
+      case 4: if constexpr (VEC == 8) emit_row<T, 4>(a, map, s, drow, d2row, lane); break;
+      case 5: if constexpr (VEC == 8) emit_row<T, 5>(a, map, s, drow, d2row, lane); break;
+      case 6: if constexpr (VEC == 8) emit_row<T, 6>(a, map, s, drow, d2row, lane); break;
+      default: if constexpr (VEC == 8) emit_row<T, 7>(a, map, s, drow, d2row, lane); break;
     }
-    __syncthreads();  // slot k % NB may be refilled by the next iteration's prefetch
+    __syncwarp();  // slot k % NBW may be refilled by the next iteration's prefetch
   }
   cp_async_wait_all();
 }
@@ -164,8 +215,12 @@ poet_status launch_permute(PermArgs<T> a, cudaStream_t st, const char *kind) {
   POET_REQUIRE(a.d <= 65535, "permute: dimension %d too large", a.d);
   constexpr int VEC = 16 / sizeof(T);
   a.slot = int(round_up(a.d + VEC, VEC));
-  const size_t smem = size_t(round_up(int64_t(a.d) * 2, 16)) + size_t(NB) * a.slot * sizeof(T);
-  POET_REQUIRE(smem <= 220 * 1024, "permute: rows of %d elements do not fit in shared memory", a.d);
+  a.map_len = int(round_up(a.d, 8) + 8);
+  const size_t budget = 220 * 1024, per_warp = size_t(NBW) * a.slot * sizeof(T);
+  int warps = int((budget - size_t(a.map_len) * 2) / per_warp);
+  if (warps > MAX_WARPS) warps = MAX_WARPS;
+  POET_REQUIRE(warps >= 1, "permute: rows of %d elements do not fit in shared memory", a.d);
+  const size_t smem = size_t(a.map_len) * 2 + size_t(warps) * per_warp;
   static int configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -174,12 +229,13 @@ poet_status launch_permute(PermArgs<T> a, cudaStream_t st, const char *kind) {
     configured[dev] = int(smem);
   }
   int per_sm = 0;
-  POET_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_rows_kernel<T>, NT, smem));
+  POET_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_rows_kernel<T>, warps * 32, smem));
   if (per_sm < 1) per_sm = 1;
+  const int64_t want = (a.rows + warps - 1) / warps;
   const int64_t cap = int64_t(num_sms()) * per_sm;
-  const int grid = int(a.rows < cap ? a.rows : cap);
+  const int grid = int(want < cap ? want : cap);
   TraceScope ts(kind, 0.0, double(a.rows) * a.d * sizeof(T) * 2.0, st);
-  permute_rows_kernel<T><<<grid, NT, smem, st>>>(a);
+  permute_rows_kernel<T><<<grid, warps * 32, smem, st>>>(a);
   count_launch();
   return launch_status(kind);
 }

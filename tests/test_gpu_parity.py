@@ -99,6 +99,10 @@ LAYER_CASES = {
     # block-stochastic b = 256 on LLaMA-350M FFN shapes (10 blocks + 176 leftover), few tokens
     "bs256_ffn_bf16": Case(2736, 1024, I.BS, 256, I.BS, 256, 4, 300, I.BF16, 0.02, layer_id=11),
     "bs256_down_bf16": Case(1024, 2736, I.BS, 256, I.BS, 256, 4, 130, I.BF16, 0.02, layer_id=12),
+    # LLaMA-3B down projection width (6912-wide rows through the permutes), block-stochastic
+    "bs256_3b_down_bf16": Case(2560, 6912, I.BS, 256, I.BS, 256, 4, 70, I.BF16, 0.02, layer_id=13),
+    # natural rows of odd width in float32 (every 16-byte misalignment of a row start)
+    "odd_width_fp32": Case(333, 517, I.BS, 40, I.FS, 0, 2, 45, I.F32, 0.04, layer_id=14),
     # mixed modes and degenerate sides
     "mixed_fs_bs": Case(96, 160, I.FS, 0, I.BS, 16, 1, 40, I.F32, 0.05),
     "k0": Case(64, 48, I.BS, 16, I.BS, 16, 0, 33, I.F32, 0.05),
