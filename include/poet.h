@@ -146,6 +146,25 @@ POET_API poet_status poet_cayley_neumann_grad(const poet_side *side, int32_t dty
                                      const float *G, float *dtheta,
                                      void *ws, size_t ws_bytes, poet_stream stream);
 
+/* The same computation as poet_cayley_neumann_grad, for callers that cannot
+ * allocate device memory (a host framework that owns all device memory and
+ * hands out none, a plug-in whose host forbids allocations, a caller that
+ * cannot keep a workspace between calls).  The POET pages have no counterpart
+ * of this call; it exists for those callers only.  Inputs and outputs as in
+ * poet_cayley_neumann_grad; the scratch is a 32 MiB array built into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  A side whose workspace (poet_side_workspace_bytes) exceeds 32 MiB is
+ * rejected with POET_EINVAL.  No allocation happens in this call.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and may load the library's code on that device:
+ *    make that first call before any stream capture begins.
+ *  - All calls on a device share the one array, which keeps the last call's
+ *    contents (nothing in it needs to start at zero).  Calls whose work
+ *    overlaps on the GPU race on it: order them on one stream. */
+POET_API poet_status poet_cayley_neumann_grad_noalloc(const poet_side *side, int32_t dtype,
+                                                      const float *G, float *dtheta,
+                                                      poet_stream stream);
+
 /* ---------------------------------------------------------------- a2..a4 */
 
 /* Forward: y = R W0 P x for T tokens ([P1] Approach; [P2] Abstract).

@@ -81,6 +81,8 @@ _SIGS = {
     "poet_cayley_neumann_grad_many": (ctypes.c_int, [ctypes.POINTER(poet_side), ctypes.POINTER(ctypes.c_void_p),
                                                      ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32, ctypes.c_int32,
                                                      ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "poet_cayley_neumann_grad_noalloc": (ctypes.c_int, [ctypes.POINTER(poet_side), ctypes.c_int32, ctypes.c_void_p,
+                                                        ctypes.c_void_p, ctypes.c_void_p]),
     "poet_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "poet_launch_count": (ctypes.c_int64, []),
     "poet_trace_enable": (ctypes.c_int, [ctypes.c_int32]),
@@ -165,6 +167,11 @@ def poet_cayley_neumann(side: poet_side, dtype: int, ws=None, stream=None):
 def poet_cayley_neumann_grad(side: poet_side, dtype: int, G, dtheta, ws, stream=None):
     _check(lib().poet_cayley_neumann_grad(ctypes.byref(side), dtype, _ptr(G), _ptr(dtheta), _ptr(ws), ws.numel(),
                                           _stream(stream)))
+
+
+def poet_cayley_neumann_grad_noalloc(side: poet_side, dtype: int, G, dtheta, stream=None):
+    """a8 without a caller workspace (the library's built-in 32 MiB scratch)."""
+    _check(lib().poet_cayley_neumann_grad_noalloc(ctypes.byref(side), dtype, _ptr(G), _ptr(dtheta), _stream(stream)))
 
 
 def poet_forward(layer: poet_layer, x, T: int, y, saved, ws, stream=None):
