@@ -39,6 +39,10 @@ WORKLOAD_SETS = {
 }
 METRIC = "POET layer fwd+bwd tokens/s at LLaMA-1.3B shapes; % of TC/HBM roofline"
 
+# DRAM traffic / algorithmic bytes of one launch, from an ncu capture, with the
+# kernel revision (as named in poet_version()) the counters were taken on.
+NCU_TRAFFIC_RATIO = {"w0_fwd": (0.920, "gemm_tc r3"), "w0_bwd": (0.979, "gemm_tc r3")}
+
 
 def parse_args():
     ap = argparse.ArgumentParser()
@@ -229,10 +233,10 @@ class Variant:
         for c0 in range(0, len(pl), self.chunk):  # a8 for every layer, in grouped launches
             poet.cayley_neumann_grad_many(pl[c0:c0 + self.chunk], self.G[c0:c0 + self.chunk],
                                           self.dslices[c0:c0 + self.chunk], self.gws)
-        if world > 1:
-            import torch.distributed as dist
+        if world > 1:  # data parallel: the one exchange of the step
+            from orthogonal_reparameterized_poet_b200 import dp
 
-            dist.all_reduce(self.dtheta)
+            dp.allreduce_gradients_(self.dtheta)
 
     def merge_all(self):
         for (_, _, _, _, L) in self.layers:
@@ -329,10 +333,10 @@ def run_poet(args):
                 a[f] += r[f]
     poet.poet_sync_status()
     if dist is not None:
-        t = torch.tensor([elapsed] + per_variant_ms, dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t[0])
-        per_variant_ms = [float(x) for x in t[1:]]
+        from orthogonal_reparameterized_poet_b200 import dp
+
+        mx = dp.max_over_ranks([elapsed] + per_variant_ms, device=device)
+        elapsed, per_variant_ms = mx[0], mx[1:]
 
     tokens_per_step = sum(v.T for v in variants) * world
     ms_per_step = elapsed / args.steps
@@ -377,10 +381,16 @@ def run_poet(args):
             achieved = r["bytes"] / (r["ms"] / 1e3) / 1e9
             peak = peaks["hbm_gbs"]
             roof = {"bound": "hbm", "unit": "GB/s", "peak_kind": "copy, " + peaks["source"]}
+        traffic = None
+        ratio = NCU_TRAFFIC_RATIO.get(dominant)
+        if ratio and ratio[1] in poet.poet_version():  # counters taken on this kernel revision
+            traffic = round(ratio[0] * r["bytes"] / r["launches"])
         roof.update({"kernel": dominant, "achieved": round(achieved, 1), "peak": peak,
-                     "frac": round(achieved / peak, 4), "traffic": None, "avg_launch_ms": round(avg_ms, 4),
+                     "frac": round(achieved / peak, 4), "traffic": traffic, "avg_launch_ms": round(avg_ms, 4),
                      "launches": r["launches"], "algorithmic_per_launch": {
-                         "flop": r["flop"] / r["launches"], "bytes": r["bytes"] / r["launches"]}})
+                         "flop": r["flop"] / r["launches"], "bytes": r["bytes"] / r["launches"]},
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one gate-shape launch "
+                                       "(profiles/w0_gemm_llama1.3b_gate_T32768.md), scaled by algorithmic bytes"})
     kernels = {}
     for k, r in sorted(rows.items(), key=lambda kv: -kv[1]["ms"]):
         kernels[k] = {"launches": r["launches"], "ms_per_step": round(r["ms"] / args.steps, 3),

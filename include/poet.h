@@ -292,6 +292,13 @@ POET_API poet_status poet_trace_enable(int32_t on);
  * max_rows, sorted by kind), forget them, and return the rows written. */
 POET_API int32_t poet_trace_read(poet_trace_row *rows, int32_t max_rows);
 
+/* Failure-detection self test.  Launches one CTA that waits, through the
+ * library's bounded mbarrier wait, on a barrier that nothing arrives on, with
+ * the limit set to timeout_us (1 .. 1e6).  The wait runs out, records a
+ * timeout in the device status word and the kernel returns normally, so the
+ * next poet_sync_status returns POET_ETIMEOUT and the context stays usable. */
+POET_API poet_status poet_selftest_bounded_wait(uint32_t timeout_us, poet_stream stream);
+
 /* Synchronize the stream, then read and clear the device status word.
  * Returns POET_ETIMEOUT if a kernel gave up a bounded wait since the last
  * call, POET_ECUDA on a CUDA error, POET_OK otherwise. */

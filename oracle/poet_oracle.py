@@ -155,6 +155,18 @@ def dense_side(perm: np.ndarray, blocks: np.ndarray, mode: int, b: int) -> np.nd
     return M
 
 
+def apply_side_rows(X: np.ndarray, perm: np.ndarray, blocks: np.ndarray, mode: int, b: int) -> np.ndarray:
+    """Rows of X (tokens) multiplied by the side matrix: returns X @ M^T for
+    M = dense_side(perm, blocks, mode, b), computed primitive by primitive
+    (out[:, I_j] = X[:, I_j] @ block_j^T, other columns copied) so that full
+    LLaMA widths stay cheap."""
+    X = np.asarray(X, dtype=np.float64)
+    out = X.copy()
+    for j, idx in enumerate(block_index_sets(perm, mode, b)):
+        out[:, idx] = X[:, idx] @ np.asarray(blocks[j], dtype=np.float64).T
+    return out
+
+
 # --------------------------------------------------------------------------
 # a2..a4: forward,  a5..a8: backward
 # --------------------------------------------------------------------------

@@ -95,7 +95,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
 // Bounded wait for the phase with the given parity.  Returns false (after
 // recording ERR_TIMEOUT and raising the CTA's abort flag) if it runs out, or
 // if another role of the CTA has already aborted.
-__device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *errword) {
+__device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *errword,
+                                       uint64_t timeout_ns = kTimeoutNs) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -103,7 +104,7 @@ __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile 
     if (mbar_try_wait(addr, parity)) return true;
     if ((it & 63) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kTimeoutNs) {
+      if (globaltimer() - t0 > timeout_ns) {
         if (errword) atomicOr(errword, ERR_TIMEOUT);
         *abort = 1;
         return false;
@@ -480,6 +481,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
   }
 }
 
+// Failure-detection self test: one thread waits, through the same bounded wait
+// the GEMM roles use, on a barrier that nothing arrives on.  The wait runs out
+// after timeout_ns, records ERR_TIMEOUT in the device status word and the
+// kernel returns normally (no trap, no fault: the context stays usable).
+__global__ void bounded_wait_selftest_kernel(unsigned *errword, uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, errword, timeout_ns);
+}
+
 // ------------------------------------------------------------------ host side
 
 PFN_cuTensorMapEncodeTiled_v12000 encoder() {
@@ -647,6 +664,16 @@ poet_status gemm_tc_many(const Gemm *gs, int count, cudaStream_t st) {
     i = j;
   }
   return POET_OK;
+}
+
+poet_status selftest_bounded_wait(uint32_t timeout_us, cudaStream_t st) {
+  POET_REQUIRE(timeout_us >= 1 && timeout_us <= 1000000, "poet_selftest_bounded_wait: timeout %u us outside [1, 1e6]",
+               timeout_us);
+  unsigned *ew = device_errword();
+  POET_REQUIRE(ew != nullptr, "poet_selftest_bounded_wait: no device status word");
+  bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(ew, uint64_t(timeout_us) * 1000ull);
+  count_launch();
+  return launch_status("bounded_wait_selftest");
 }
 
 }  // namespace poet

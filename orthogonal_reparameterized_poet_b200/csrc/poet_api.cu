@@ -241,7 +241,8 @@ extern "C" {
 
 const char *poet_last_error(void) { return g_last_error; }
 
-const char *poet_version(void) { return "libpoet 0.1 (sm_100a)"; }
+// The kernel revisions name the code that profiles/ counters were taken on.
+const char *poet_version(void) { return "libpoet 0.2 (sm_100a; gemm_tc r3; permute r3)"; }
 
 size_t poet_side_state_bytes(const poet_side *side, int32_t dtype) {
   SideGeom g;
@@ -632,6 +633,11 @@ poet_status poet_gemm(int32_t dtype, int32_t M, int32_t N, int32_t K, int32_t ba
   if (beta != 0.f) { p.add = C; p.add_dtype = dtype; p.add_m = ldc; p.add_b = sCb; p.beta = beta; }
   p.outD = C; p.od_m = ldc; p.od_b = sCb;
   return gemm_run(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+poet_status poet_selftest_bounded_wait(uint32_t timeout_us, poet_stream stream) {
+  clear_error();
+  return selftest_bounded_wait(timeout_us, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int32_t poet_gemm_engine(int32_t dtype) { return (dtype == POET_BF16 && gemm_tc_enabled()) ? 1 : 0; }

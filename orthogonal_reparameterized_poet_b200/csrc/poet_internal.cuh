@@ -119,6 +119,8 @@ poet_status gemm_tc(const Gemm &g, cudaStream_t st);        // tcgen05 engine
 // on the CUDA-core engine.  gemm_run_many adds tracing around it.
 poet_status gemm_tc_many(const Gemm *gs, int count, cudaStream_t st);
 poet_status gemm_run_many(const Gemm *gs, int count, cudaStream_t st);
+// One CTA whose bounded wait on a barrier nothing arrives on runs out (tests failure detection).
+poet_status selftest_bounded_wait(uint32_t timeout_us, cudaStream_t st);
 bool gemm_tc_enabled();
 
 // ------------------------------------------------------------------ data movement

@@ -83,6 +83,7 @@ _SIGS = {
                                                      ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "poet_cayley_neumann_grad_noalloc": (ctypes.c_int, [ctypes.POINTER(poet_side), ctypes.c_int32, ctypes.c_void_p,
                                                         ctypes.c_void_p, ctypes.c_void_p]),
+    "poet_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_void_p]),
     "poet_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "poet_launch_count": (ctypes.c_int64, []),
     "poet_trace_enable": (ctypes.c_int, [ctypes.c_int32]),
@@ -208,6 +209,10 @@ def poet_gemm(dtype, M, N, K, batch, A, sA, B, sB, C, ldc, sCb, alpha=1.0, beta=
 
 def poet_gemm_engine(dtype: int) -> int:
     return lib().poet_gemm_engine(dtype)
+
+
+def poet_selftest_bounded_wait(timeout_us: int, stream=None):
+    _check(lib().poet_selftest_bounded_wait(timeout_us, _stream(stream)))
 
 
 def poet_sync_status(stream=None):

@@ -145,6 +145,21 @@ def check_dense_side_vs_loops(O):
     return True
 
 
+def check_apply_side_rows(O):
+    """Blockwise application equals brute-force loops on every row."""
+    rng = _rng(10)
+    for d, mode, b in [(11, 0, 3), (10, 1, 0), (9, 0, 9)]:
+        perm = rng.permutation(d)
+        nprim, s = O.side_shape(d, mode, b)
+        blocks = rng.standard_normal((nprim, s, s))
+        X = rng.standard_normal((4, d))
+        got = O.apply_side_rows(X, perm, blocks, mode, b)
+        for t in range(4):
+            if not np.allclose(got[t], _apply_side_by_loops(perm, blocks, mode, b, X[t]), atol=1e-12):
+                return False
+    return True
+
+
 def check_side_shapes(O):
     return (O.side_shape(5461, O.BS, 256) == (21, 256) and O.side_shape(5461, O.FS, 0) == (1, 2730)
             and O.side_shape(1376, O.FS, 0) == (1, 688) and O.side_shape(256, O.BS, 32) == (8, 32)
@@ -331,7 +346,8 @@ def check_param_counts(O):
 ALL_CHECKS = [
     check_unpack_golden, check_cnp_2x2_closed_form, check_cnp_truncation_identity,
     check_orthogonality_identity, check_singular_values_closed_form, check_special_cases,
-    check_dense_side_golden, check_dense_side_vs_loops, check_side_shapes, check_no_primitive_side,
+    check_dense_side_golden, check_dense_side_vs_loops, check_apply_side_rows, check_side_shapes,
+    check_no_primitive_side,
     check_spectrum_preservation, check_merge_invariance, check_backward_finite_differences,
     check_splitmix_golden, check_draw_perm, check_param_counts,
 ]

@@ -1,0 +1,129 @@
+"""Parity at the benchmark's full size: LLaMA-1.3B shapes, 32768 tokens, layer
+0 of both variants (fully stochastic and block-stochastic b=256), built from
+the same seeded inputs and run through the same grouped calls bench.py times
+(poet_cayley_neumann_many, poet_forward, poet_backward_blocks,
+poet_cayley_neumann_grad_many, then poet_merge).
+
+The oracle cannot afford the whole layer at this size, so it computes sampled
+outputs one by one from their definitions:
+  * y and dx on 16 sampled tokens (per-token products through the primitives);
+  * dtheta of sampled primitives, whose block gradient sums over all 32768
+    tokens (only the primitive's own columns of v = W0 P x or du = W0^T R^T dy
+    are formed);
+  * sampled rows of the merged W0;
+  * every permutation, bit-exact.
+Fully stochastic sides of size 2730 are checked through y, dx and the merge
+(their dtheta costs minutes of float64 CPU time); their 1024-sized sides are
+checked directly."""
+import numpy as np
+import pytest
+
+from oracle import poet_oracle as O
+from orthogonal_reparameterized_poet_b200 import inputs as I
+from tests.harness import TOL, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cuda():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    poet.lib()
+    return torch
+
+
+CASES = [("llama1.3b_fs", 4), ("llama1.3b_fs", 6), ("llama1.3b_bs256", 4), ("llama1.3b_bs256", 6)]
+
+
+@pytest.mark.parametrize("name,linear", CASES)
+def test_fullsize_sampled_parity(cuda, name, linear):
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    wl = I.WORKLOADS[name]
+    layer, T, k, dt = 0, wl.tokens, wl.k, wl.dtype
+    m, n = wl.linear_shapes()[linear]
+    layer_id = layer * len(wl.linear_shapes()) + linear
+    nR, sR = O.side_shape(m, wl.mode, wl.b)
+    nP, sP = O.side_shape(n, wl.mode, wl.b)
+    # inputs exactly as bench.py draws them (rank 0)
+    W0 = I.w0(wl.seed, layer, linear, m, n, dt)
+    thR = I.theta(wl.seed, layer, linear, 0, nR * O.n_skew(sR), wl.sigma)
+    thP = I.theta(wl.seed, layer, linear, 1, nP * O.n_skew(sP), wl.sigma)
+    X = I.activations(wl.seed, n, T, n, dt)
+    dY = I.activations(wl.seed, m, T, m, dt, grad=True)
+
+    # ---------------- CUDA path, bench launch configuration
+    tdt = poet.torch_dtype(dt)
+    L = poet.PoetLayer(cuda.from_numpy(W0).to("cuda", tdt), cuda.from_numpy(thR).cuda(), cuda.from_numpy(thP).cuda(),
+                       mode=wl.mode, b=wl.b, k=k, seed=wl.seed, layer_id=layer_id)
+    L.prepare()
+    poet.cayley_neumann_many([L])
+    xt = cuda.from_numpy(X).to("cuda", tdt)
+    dyt = cuda.from_numpy(dY).to("cuda", tdt)
+    y, saved = L.forward(xt)
+    gR, gP = L.block_grad_buffers()
+    dx = L.backward_blocks(saved, dyt, gR, gP)
+    dthR, dthP = cuda.empty_like(L.theta_R), cuda.empty_like(L.theta_P)
+    ws = cuda.empty(max(poet.cayley_neumann_grad_many_workspace_bytes([L]), 1), dtype=cuda.uint8, device="cuda")
+    poet.cayley_neumann_grad_many([L], [(gR, gP)], [(dthR, dthP)], ws)
+    poet.poet_sync_status()
+    permR_gpu, permP_gpu = L.perm_R.cpu().numpy(), L.perm_P.cpu().numpy()
+    rows = np.random.default_rng(linear).choice(T, 16, replace=False)
+    y_s = y[rows].float().cpu().numpy()
+    dx_s = dx[rows].float().cpu().numpy()
+    dthR, dthP = dthR.cpu().numpy(), dthP.cpu().numpy()
+    del y, dx, saved, xt, dyt, gR, gP, ws
+    L.merge()
+    wrows = np.random.default_rng(100 + linear).choice(m, 12, replace=False)
+    W0m = L.W0[wrows].float().cpu().numpy()
+    del L
+
+    # ---------------- oracle, sampled
+    permR = O.draw_perm(wl.seed, layer_id, 0, 0, m)
+    permP = O.draw_perm(wl.seed, layer_id, 1, 0, n)
+    assert np.array_equal(permR_gpu, permR) and np.array_equal(permP_gpu, permP)
+    Rb = O.cayley_neumann(thR.astype(np.float64), nR, sR, k)
+    Pb = O.cayley_neumann(thP.astype(np.float64), nP, sP, k)
+    RbT, PbT = Rb.transpose(0, 2, 1), Pb.transpose(0, 2, 1)
+    W0d = W0.astype(np.float64)
+    tol = TOL[dt]
+    # y = R W0 P x and dx = P^T W0^T R^T dy on the sampled tokens
+    y_ref = O.apply_side_rows(O.apply_side_rows(X[rows], permP, Pb, wl.mode, wl.b) @ W0d.T, permR, Rb, wl.mode, wl.b)
+    dx_ref = O.apply_side_rows(O.apply_side_rows(dY[rows], permR, RbT, wl.mode, wl.b) @ W0d, permP, PbT,
+                               wl.mode, wl.b)
+    assert rel_fro(y_s, y_ref) <= tol
+    assert rel_fro(dx_s, dx_ref) <= tol
+    # dtheta of sampled primitives (block gradient over all tokens)
+    rng = np.random.default_rng(7)
+    if sP <= 1024:
+        dV = O.apply_side_rows(dY, permR, RbT, wl.mode, wl.b)  # R^T dy for every token
+        for j in sorted(rng.choice(nP, min(2, nP), replace=False)):
+            J = permP[j * sP:(j + 1) * sP]
+            dU_J = dV @ W0d[:, J]                                 # (W0^T R^T dy) on the primitive's columns
+            G = dU_J.T @ X[:, J].astype(np.float64)
+            per = O.n_skew(sP)
+            ref = O.theta_grad_block(G, thP[j * per:(j + 1) * per].astype(np.float64), sP, k)
+            assert rel_fro(dthP[j * per:(j + 1) * per], ref) <= tol
+        del dV
+    if sR <= 1024:
+        U = O.apply_side_rows(X, permP, Pb, wl.mode, wl.b)         # P x for every token
+        for j in sorted(rng.choice(nR, min(2, nR), replace=False)):
+            Iset = permR[j * sR:(j + 1) * sR]
+            V_I = U @ W0d[Iset, :].T                                 # (W0 P x) on the primitive's rows
+            G = dY[:, Iset].astype(np.float64).T @ V_I
+            per = O.n_skew(sR)
+            ref = O.theta_grad_block(G, thR[j * per:(j + 1) * per].astype(np.float64), sR, k)
+            assert rel_fro(dthR[j * per:(j + 1) * per], ref) <= tol
+    # merged W0 on sampled rows: (R W0 P)[i, :]
+    R_rows = np.zeros((len(wrows), m))
+    for r_i, i in enumerate(wrows):
+        e = np.zeros((1, m))
+        e[0, i] = 1.0
+        R_rows[r_i] = O.apply_side_rows(e, permR, RbT, wl.mode, wl.b)[0]  # row i of R = e_i^T R
+    W0m_ref = O.apply_side_rows(R_rows @ W0d, permP, PbT, wl.mode, wl.b)  # ... then times P
+    assert rel_fro(W0m, W0m_ref) <= tol
