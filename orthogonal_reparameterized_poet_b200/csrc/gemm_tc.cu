@@ -596,8 +596,24 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
     const int64_t mt = (gs[i].M + BM - 1) / BM, nt = (gs[i].N + t.BN - 1) / t.BN;
     base_tiles += mt * nt * gs[i].batch;
   }
-  // split K (atomic outputs only) as far as the tiles still fit in one wave
-  const int split_want = base_tiles > 0 && base_tiles < num_sms() ? int(num_sms() / base_tiles) : 1;
+  // Split K (atomic outputs only) into s parts, s chosen so that the tiles
+  // fill whole waves of persistent CTAs: take the smallest s within 2% of the
+  // best wave efficiency tiles / (ceil(tiles / SMs) * SMs), s <= 16.
+  int split_want = 1;
+  bool any_atomic = false;
+  for (int i = 0; i < n; ++i) any_atomic |= gs[i].atomic;
+  if (any_atomic && base_tiles > 0) {
+    const int64_t sms = num_sms();
+    double best = 0.0;
+    for (int sp = 1; sp <= 16; ++sp) {
+      const int64_t tiles = base_tiles * sp;
+      const double eff = double(tiles) / double(((tiles + sms - 1) / sms) * sms);
+      if (eff > best + 0.02) {
+        best = eff;
+        split_want = sp;
+      }
+    }
+  }
   grp.count = n;
   grp.errword = device_errword();
   grp.tile_start[0] = 0;
@@ -621,7 +637,8 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
   return launch<true, true, 256, MAXP>(grp, st);
 }
 
-constexpr int kGroupMax = 48;
+constexpr int kGroupMax = 64;  // ~25 KB of kernel parameters (limit 32 KB)
+static_assert(sizeof(TcGroup<kGroupMax>) <= 32000, "grouped launch parameters exceed the kernel parameter limit");
 
 }  // namespace
 
