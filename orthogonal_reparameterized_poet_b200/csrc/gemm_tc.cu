@@ -41,6 +41,7 @@ struct TcProblem {
   float *outF; int64_t of_m, of_b;
   bf16 *outD; int64_t od_m, od_b;
   int atomic;
+  int coalesced;  // plain bf16 output, 16-byte aligned rows: stores staged through shared memory
 };
 
 // A launch: up to MAXP independent problems sharing operand majors and tile
@@ -212,14 +213,26 @@ __device__ __forceinline__ TileCoord decode(int64_t tile, const TcGroup<MAXP> &g
   return c;
 }
 
-template <int BN>
+// Shared-memory plan.  Streaming mode: a ring of (A slab, B slab) stages.
+// B-stationary mode (BSTAT, problems with K <= 256 and one N tile): the whole
+// B operand of the current (problem, batch) stays resident (KB_MAX slabs) and
+// only A slabs stream through the ring.
+constexpr int KB_MAX = 4;  // B-stationary: K <= 256
+template <int BN, bool BSTAT = false>
 struct Smem {
   static constexpr int A_BYTES = BM * BK * 2;   // 16 KB
   static constexpr int B_BYTES = BN * BK * 2;   // 32 KB (BN = 256)
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int STAGE_BYTES = BSTAT ? A_BYTES : A_BYTES + B_BYTES;
+  static constexpr int STAGES = BSTAT ? 4 : (BN == 256 ? 4 : 6);
+  static constexpr int BRES_BYTES = BSTAT ? KB_MAX * B_BYTES : 0;  // resident B
+  // epilogue staging: per epilogue warp 32 rows x 128 B (one 64-column bf16
+  // chunk), rows padded to 144 B so row-wise writes and line-wise reads both
+  // take the minimum number of shared-memory wavefronts
+  static constexpr int EPI_ROW = 144;
+  static constexpr int EPI_BYTES = 4 * 32 * EPI_ROW;
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr size_t BYTES = size_t(STAGES) * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr size_t BYTES =
+      size_t(STAGES) * STAGE_BYTES + BRES_BYTES + EPI_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
@@ -229,24 +242,34 @@ __device__ __forceinline__ void red_add_v4(float *out, float a, float b, float c
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(out), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
-template <bool A_MN, bool B_MN, int BN, int MAXP>
+template <bool A_MN, bool B_MN, int BN, int MAXP, bool BSTAT>
 __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_constant__ TcGroup<MAXP> g) {
-  using S = Smem<BN>;
+  using S = Smem<BN, BSTAT>;
   constexpr int STAGES = S::STAGES;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char *stage_base = smem;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + size_t(STAGES) * S::STAGE_BYTES);
+  unsigned char *bres = smem + size_t(STAGES) * S::STAGE_BYTES;  // resident B (B-stationary only)
+  unsigned char *epi = bres + S::BRES_BYTES;                      // epilogue staging
+  uint64_t *bars = reinterpret_cast<uint64_t *>(epi + S::EPI_BYTES);
   uint64_t *full = bars;                 // [STAGES]
   uint64_t *empty = bars + STAGES;       // [STAGES]
   uint64_t *tfull = bars + 2 * STAGES;   // [2]
   uint64_t *tempty = tfull + 2;          // [2]
   uint64_t *drain = tempty + 2;          // [1]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  uint64_t *bfull = drain + 1;           // [1] resident B landed
+  uint64_t *bfree = bfull + 1;           // [1] MMAs reading the resident B are done
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bfree + 1);
   volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t tiles = g.tile_start[g.count];
+  // Tiles of this CTA: strided over the grid (streaming), or one contiguous
+  // range (B-stationary, so that consecutive tiles share their B operand).
+  const int64_t per_cta = (tiles + gridDim.x - 1) / gridDim.x;
+  const int64_t t_first = BSTAT ? int64_t(blockIdx.x) * per_cta : int64_t(blockIdx.x);
+  const int64_t t_step = BSTAT ? 1 : int64_t(gridDim.x);
+  const int64_t t_end = BSTAT ? (t_first + per_cta < tiles ? t_first + per_cta : tiles) : tiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -258,6 +281,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       mbar_init(&tempty[a], 4);
     }
     mbar_init(drain, 1);
+    mbar_init(bfull, 1);
+    mbar_init(bfree, 1);
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -278,7 +303,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       int last_stage = -1;
       uint32_t last_phase = 0;
       int last_pi = -1;
-      for (int64_t tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
+      int res_pi = -1, res_b = -1;   // B-stationary: operand currently resident
+      uint32_t bfree_phase = 0;
+      uint32_t bloads = 0;
+      for (int64_t tile = t_first; tile < t_end && !*abort; tile += t_step) {
         const TileCoord c = decode(tile, g);
         const TcProblem &p = g.prob[c.pi];
         const CUtensorMap *ma = &g.ma[c.pi];
@@ -287,6 +315,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
           tma_prefetch_desc(ma);
           tma_prefetch_desc(mb);
           last_pi = c.pi;
+        }
+        if constexpr (BSTAT) {
+          if (c.pi != res_pi || c.b != res_b) {  // load this (problem, batch)'s whole B once
+            if (res_pi >= 0) {
+              if (!mbar_wait(bfree, bfree_phase, abort, g.errword)) break;
+              bfree_phase ^= 1;
+            }
+            mbar_expect_tx(bfull, uint32_t(p.nk) * S::B_BYTES);
+            ++bloads;
+            for (int kb = 0; kb < p.nk; ++kb) {
+              unsigned char *sb = bres + size_t(kb) * S::B_BYTES;
+              if (!B_MN) {
+                tma_load_3d(sb, mb, bfull, kb * BK, c.nt * BN, c.b);
+              } else {
+#pragma unroll
+                for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, mb, bfull, c.nt * BN + 64 * q, kb * BK, c.b);
+              }
+            }
+            res_pi = c.pi;
+            res_b = c.b;
+          }
         }
         const int kb0 = c.s * p.kchunk;
         const int kb1 = min(p.nk, kb0 + p.kchunk);
@@ -301,11 +350,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
 #pragma unroll
             for (int q = 0; q < BM / 64; ++q) tma_load_3d(sa + q * 8192, ma, &full[stage], c.mt * BM + 64 * q, kb * BK, c.b);
           }
-          if (!B_MN) {
-            tma_load_3d(sb, mb, &full[stage], kb * BK, c.nt * BN, c.b);
-          } else {
+          if constexpr (!BSTAT) {
+            if (!B_MN) {
+              tma_load_3d(sb, mb, &full[stage], kb * BK, c.nt * BN, c.b);
+            } else {
 #pragma unroll
-            for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, mb, &full[stage], c.nt * BN + 64 * q, kb * BK, c.b);
+              for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, mb, &full[stage], c.nt * BN + 64 * q, kb * BK, c.b);
+            }
           }
           last_stage = stage;
           last_phase = phase;
@@ -320,6 +371,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
         volatile int no_abort = 0;
         mbar_wait(&full[last_stage], last_phase, &no_abort, nullptr);
       }
+      if (BSTAT && *abort && bloads > 0) {
+        volatile int no_abort = 0;
+        mbar_wait(bfull, (bloads - 1) & 1, &no_abort, nullptr);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -330,11 +385,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       int acc = 0;
       uint32_t acc_phase = 0;
       bool issued = false;
-      for (int64_t tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
+      int res_pi = -1, res_b = -1;  // B-stationary: operand currently resident
+      uint32_t bfull_phase = 0;
+      for (int64_t tile = t_first; tile < t_end && !*abort; tile += t_step) {
         const TileCoord c = decode(tile, g);
         const TcProblem &p = g.prob[c.pi];
         const int kb0 = c.s * p.kchunk;
         const int kb1 = min(p.nk, kb0 + p.kchunk);
+        if constexpr (BSTAT) {
+          if (c.pi != res_pi || c.b != res_b) {
+            if (!mbar_wait(bfull, bfull_phase, abort, g.errword)) break;
+            bfull_phase ^= 1;
+            res_pi = c.pi;
+            res_b = c.b;
+          }
+        }
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort, g.errword)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
@@ -343,7 +408,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
           if (!mbar_wait(&full[stage], phase, abort, g.errword)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + size_t(stage) * S::STAGE_BYTES);
-          const uint32_t sb = sa + S::A_BYTES;
+          const uint32_t sb = BSTAT ? smem_u32(bres + size_t(kb) * S::B_BYTES) : sa + S::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = A_MN ? make_desc(sa + kk * 2048, 8192, 1024) : make_desc(sa + kk * 32, 16, 1024);
@@ -359,6 +424,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
         }
         if (!ok) break;
         umma_commit(&tfull[acc]);
+        if constexpr (BSTAT) {
+          // the resident B is released after the last tile that reads it
+          bool last_use = tile + t_step >= t_end;
+          if (!last_use) {
+            const TileCoord nc = decode(tile + t_step, g);
+            last_use = nc.pi != c.pi || nc.b != c.b;
+          }
+          if (last_use) umma_commit(bfree);
+        }
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1;
@@ -377,7 +451,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int64_t tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
+    for (int64_t tile = t_first; tile < t_end && !*abort; tile += t_step) {
       const TileCoord c = decode(tile, g);
       const TcProblem &p = g.prob[c.pi];
       if (!mbar_wait(&tfull[acc], acc_phase, abort, g.errword)) break;
@@ -385,6 +459,58 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       const int gm = c.mt * BM + row;
       const bool row_ok = gm < p.M;
       const float alpha = p.alpha, beta = p.beta, diag = p.diag;
+      if (p.coalesced) {
+        // plain bf16 output: each 64-column chunk goes row-wise into this warp's
+        // staging rows, then out with every store instruction covering four
+        // rows x 128 contiguous bytes
+        unsigned char *ew = epi + quarter * (32 * S::EPI_ROW);
+        const int m_base = c.mt * BM + quarter * 32;
+        bf16 *obase = p.outD + int64_t(c.b) * p.od_b;
+        const int sub = lane & 7, rsub = lane >> 3;
+        for (int cc = 0; cc < BN / 64; ++cc) {
+          uint32_t r0[32], r1[32];
+          __syncwarp();
+          const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN + cc * 64);
+          tmem_ld32(taddr, r0);
+          tmem_ld32(taddr + 32, r1);
+          tmem_ld_wait();
+          const int gn0 = c.nt * BN + cc * 64;
+          if (gn0 >= p.N) continue;  // the same for the whole warp
+          unsigned char *myrow = ew + lane * S::EPI_ROW;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t *src = q < 4 ? r0 + 8 * q : r1 + 8 * (q - 4);
+            uint4 pk;
+            __nv_bfloat162 h0 = __floats2bfloat162_rn(alpha * __uint_as_float(src[0]), alpha * __uint_as_float(src[1]));
+            __nv_bfloat162 h1 = __floats2bfloat162_rn(alpha * __uint_as_float(src[2]), alpha * __uint_as_float(src[3]));
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(alpha * __uint_as_float(src[4]), alpha * __uint_as_float(src[5]));
+            __nv_bfloat162 h3 = __floats2bfloat162_rn(alpha * __uint_as_float(src[6]), alpha * __uint_as_float(src[7]));
+            pk.x = *reinterpret_cast<uint32_t *>(&h0);
+            pk.y = *reinterpret_cast<uint32_t *>(&h1);
+            pk.z = *reinterpret_cast<uint32_t *>(&h2);
+            pk.w = *reinterpret_cast<uint32_t *>(&h3);
+            *reinterpret_cast<uint4 *>(myrow + q * 16) = pk;
+          }
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + rsub;
+            const int gm = m_base + rr;
+            const int gn = gn0 + sub * 8;
+            const uint4 v = *reinterpret_cast<const uint4 *>(ew + rr * S::EPI_ROW + sub * 16);
+            if (gm < p.M && gn < p.N) {
+              bf16 *o = obase + int64_t(gm) * p.od_m + gn;
+              if (gn + 8 <= p.N) {
+                *reinterpret_cast<uint4 *>(o) = v;
+              } else {
+                const bf16 *pv = reinterpret_cast<const bf16 *>(&v);
+                for (int e = 0; e < 8; ++e)
+                  if (gn + e < p.N) o[e] = pv[e];
+              }
+            }
+          }
+        }
+      } else
       for (int cc = 0; cc < BN / 32; ++cc) {
         uint32_t r[32];
         __syncwarp();
@@ -535,13 +661,20 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 struct TcPlan {
   bool A_MN, B_MN;
   int BN;
-  bool operator==(const TcPlan &o) const { return A_MN == o.A_MN && B_MN == o.B_MN && BN == o.BN; }
+  bool bstat;  // B-stationary (whole B of a batch resident; contiguous tiles per CTA)
+  bool operator==(const TcPlan &o) const {
+    return A_MN == o.A_MN && B_MN == o.B_MN && BN == o.BN && bstat == o.bstat;
+  }
 };
 TcPlan plan_of(const Gemm &g) {
   TcPlan t;
   t.A_MN = !(g.a_k == 1 && g.a_m % 8 == 0);
   t.B_MN = !(g.b_k == 1 && g.b_n % 8 == 0);
   t.BN = g.N <= 128 ? 128 : 256;
+  // token-streaming products against a small operand (block-diagonal passes
+  // with 256-wide blocks): keep B resident when it fits and many M tiles
+  // share it
+  t.bstat = t.BN == 256 && g.N <= 256 && g.K <= KB_MAX * BK && g.M >= 8 * BM && !g.atomic;
   return t;
 }
 
@@ -560,6 +693,10 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   p->outF = g.outF; p->of_m = g.of_m; p->of_b = g.of_b;
   p->outD = static_cast<bf16 *>(g.outD); p->od_m = g.od_m; p->od_b = g.od_b;
   p->atomic = g.atomic ? 1 : 0;
+  p->coalesced = (g.outD && !g.outF && !g.add && g.diag == 0.f && !g.atomic && aligned16(g.outD) &&
+                  g.od_m % 8 == 0 && (g.batch == 1 || g.od_b % 8 == 0))
+                     ? 1
+                     : 0;
   bool ok;
   if (!t.A_MN) ok = make_map(ma, g.A, g.K, g.M, g.batch, g.a_m, g.a_b, 64, BM);
   else ok = make_map(ma, g.A, g.M, g.K, g.batch, g.a_k, g.a_b, 64, 64);
@@ -570,10 +707,10 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   return ok;
 }
 
-template <bool A_MN, bool B_MN, int BN, int MAXP>
+template <bool A_MN, bool B_MN, int BN, int MAXP, bool BSTAT = false>
 poet_status launch(const TcGroup<MAXP> &grp, cudaStream_t st) {
-  using S = Smem<BN>;
-  auto kern = gemm_tc_kernel<A_MN, B_MN, BN, MAXP>;
+  using S = Smem<BN, BSTAT>;
+  auto kern = gemm_tc_kernel<A_MN, B_MN, BN, MAXP, BSTAT>;
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -624,6 +761,12 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
       return POET_ECUDA;
     }
     grp.tile_start[i + 1] = grp.tile_start[i] + int64_t(p.num_m) * p.num_n * p.splits * p.batch;
+  }
+  if constexpr (MAXP == 1) {
+    if (t.bstat && !t.A_MN) {
+      if (!t.B_MN) return launch<false, false, 256, MAXP, true>(grp, st);
+      return launch<false, true, 256, MAXP, true>(grp, st);
+    }
   }
   if (t.BN == 128) {
     if (!t.A_MN && !t.B_MN) return launch<false, false, 128, MAXP>(grp, st);
