@@ -215,7 +215,10 @@ POET_API size_t poet_cayley_neumann_grad_many_workspace_bytes(const poet_side *s
                                                               int32_t dtype);
 
 /* a8 for count sides: dtheta[i] (device float, theta layout, overwritten) from
- * G[i] (device, layout above).  Same result as poet_cayley_neumann_grad. */
+ * G[i] (device, layout above).  The same gradient as poet_cayley_neumann_grad;
+ * its matrix products are grouped differently (every product of one Neumann
+ * order, across all sides, in one launch), so the two agree to rounding of
+ * the operand type, not bitwise. */
 POET_API poet_status poet_cayley_neumann_grad_many(const poet_side *sides, const float *const *G,
                                                    float *const *dtheta, int32_t count, int32_t dtype,
                                                    void *ws, size_t ws_bytes, poet_stream stream);

@@ -6,7 +6,7 @@
 // Neumann series truncated after Q^k:  B = (I + Q)(I + Q + ... + Q^k).
 //
 // Forward, by Horner's rule on the series:
-//   S_1 = I + Q,  S_{l+1} = I + Q S_l (l = 1..k-1),  B = S_k + Q S_k
+//   S_1 = I + Q,  S_{l+1} = I + Q S_l (l = 1..k-1),  B = (I + Q) S_k = S_1 S_k
 // (k GEMMs of size^3; k = 0 gives B = I + Q).  Q and S_1..S_k are kept in
 // the side state for the backward.
 //
@@ -66,6 +66,47 @@ __global__ void pack_grad_kernel(const float *__restrict__ dQ, const float *__re
     float v = dQ[ac] - dQ[ca];
     if (A1) v += A1[ac] - A1[ca];
     dtheta[j * per + packed_index(a, c, size)] = v;
+  }
+}
+
+// dtheta[j][idx(a,c)] = D[a,c] - D[c,a] with D = A1 + sum_t P_t (t < nterms,
+// P_t at P + t * pstride).  One block per pair of PACK_T x PACK_T tiles
+// (ta <= tc) of one primitive: both tiles are summed into shared memory with
+// row-contiguous loads, so the transposed read comes from shared memory.
+constexpr int PACK_T = 32;
+__global__ void pack_sum_kernel(const float *__restrict__ P, int nterms, int64_t pstride, const float *__restrict__ A1,
+                                int nprim, int size, int ld, float *__restrict__ dtheta) {
+  __shared__ float t1[PACK_T][PACK_T + 1], t2[PACK_T][PACK_T + 1];
+  // blockIdx.x enumerates (ta, tc), ta <= tc, row by row
+  int ta = 0, rem = blockIdx.x;
+  const int tiles = (size + PACK_T - 1) / PACK_T;
+  while (rem >= tiles - ta) { rem -= tiles - ta; ++ta; }
+  const int tc = ta + rem;
+  const int j = blockIdx.y;
+  const int64_t blk = int64_t(ld) * ld;
+  const int64_t per = int64_t(size) * (size - 1) / 2;
+  const int x = threadIdx.x;
+  for (int y = threadIdx.y; y < PACK_T; y += blockDim.y) {
+    const int a1 = ta * PACK_T + y, c1 = tc * PACK_T + x;  // tile (ta, tc)
+    const int a2 = tc * PACK_T + y, c2 = ta * PACK_T + x;  // tile (tc, ta)
+    float v1 = 0.f, v2 = 0.f;
+    if (a1 < size && c1 < size) {
+      const int64_t o = j * blk + int64_t(a1) * ld + c1;
+      v1 = A1[o];
+      for (int t = 0; t < nterms; ++t) v1 += P[t * pstride + o];
+    }
+    if (a2 < size && c2 < size) {
+      const int64_t o = j * blk + int64_t(a2) * ld + c2;
+      v2 = A1[o];
+      for (int t = 0; t < nterms; ++t) v2 += P[t * pstride + o];
+    }
+    t1[y][x] = v1;
+    t2[y][x] = v2;
+  }
+  __syncthreads();
+  for (int y = threadIdx.y; y < PACK_T; y += blockDim.y) {
+    const int a = ta * PACK_T + y, c = tc * PACK_T + x;
+    if (a < c && c < size) dtheta[j * per + packed_index(a, c, size)] = t1[y][x] - t2[x][y];
   }
 }
 
@@ -140,12 +181,13 @@ poet_status cnp_forward(const poet_side *side, const SideGeom &g, int dtype, cud
   POET_TRY(launch_status("cnp unpack"));
   for (int l = 1; l <= g.k; ++l) {
     void *S = base + L.S1 + size_t(l - 1) * L.term;
-    Gemm p = prim_gemm(g, dtype, Q, S, false, "cnp_fwd");  // Q S_l
+    Gemm p;
     if (l < g.k) {                               // S_{l+1} = I + Q S_l
+      p = prim_gemm(g, dtype, Q, S, false, "cnp_fwd");
       p.diag = 1.f;
       p.outD = base + L.S1 + size_t(l) * L.term;
-    } else {                                     // B = S_k + Q S_k
-      p.add = S; p.add_dtype = dtype; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 1.f;
+    } else {                                     // B = (I + Q) S_k = S_1 S_k
+      p = prim_gemm(g, dtype, base + L.S1, S, false, "cnp_fwd");
       p.outD = R;
     }
     p.od_m = g.ld; p.od_b = g.blk_elems();
@@ -254,12 +296,13 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
       const StateLayout L = state_layout(g, dtype);
       char *base = static_cast<char *>(sides[i].state);
       void *S = base + L.S1 + size_t(l - 1) * L.term;
-      Gemm p = prim_gemm(g, dtype, base + L.Q, S, false, "cnp_fwd");
-      if (l < g.k) {
+      Gemm p;
+      if (l < g.k) {  // S_{l+1} = I + Q S_l
+        p = prim_gemm(g, dtype, base + L.Q, S, false, "cnp_fwd");
         p.diag = 1.f;
         p.outD = base + L.S1 + size_t(l) * L.term;
-      } else {
-        p.add = S; p.add_dtype = dtype; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 1.f;
+      } else {        // B = (I + Q) S_k = S_1 S_k
+        p = prim_gemm(g, dtype, base + L.S1, S, false, "cnp_fwd");
         p.outD = base + L.R;
       }
       p.od_m = g.ld; p.od_b = g.blk_elems();
@@ -270,16 +313,32 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
   return POET_OK;
 }
 
+// Many sides: the same gradient reorganised so that every GEMM writes one
+// plain output (no addend), which the tensor-core engine stores through its
+// staged epilogue.  The chain A_k = S_1^T G, A_l = -Q A_{l+1} takes one
+// grouped launch per order (all sides); then one launch forms every partial
+// product P_k = G S_k^T, P_l = A_{l+1} S_l^T (l < k) of every side, and
+// dQ = P_1 + ... + P_k + A_1 is summed while packing.  (I + Q)^T = S_1^T is
+// read straight from the stored S_1 as a transposed operand.
+size_t cnp_many_scratch_bytes(const SideGeom &g, int dtype) {
+  if (g.nprim == 0 || g.size < 2 || g.k == 0) return 0;
+  const size_t f = align256(size_t(g.all_elems()) * 4);
+  const size_t d = align256(size_t(g.all_elems()) * esize(dtype));
+  // G operand copy, A_k..A_2 (dtype), A_1 (f32), P_1..P_k (f32)
+  return d + size_t(g.k - 1) * d + f + size_t(g.k) * f;
+}
+
 poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int count, int dtype,
                               const float *const *G, float *const *dtheta, void *const *scratch, cudaStream_t st) {
   struct Work {
     const void *Q, *Gop;
     const char *S1;
     size_t term;
-    float *Af[2];
-    void *Ad[2];
-    float *dQ;
-    int cur;
+    char *X;       // A_{l+1} for l = 1..k-1 at X + (l-1) * xb (dtype)
+    size_t xb;
+    float *A1;     // A_1 (f32)
+    float *P;      // P_l at P + (l-1) * pstride floats
+    int64_t pstride;
   };
   std::vector<Work> w(count);
   int kmax = 0;
@@ -310,69 +369,68 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
       x.Gop = G[i];
     }
     s += db;
-    x.Af[0] = reinterpret_cast<float *>(s);
-    x.Af[1] = reinterpret_cast<float *>(s + fb + db);
-    x.Ad[0] = s + fb;
-    x.Ad[1] = s + 2 * fb + db;
-    if (dtype != POET_BF16) { x.Ad[0] = x.Af[0]; x.Ad[1] = x.Af[1]; }
-    x.dQ = reinterpret_cast<float *>(s + 2 * (fb + db));
-    x.cur = 0;
+    x.X = s;
+    x.xb = db;
+    s += size_t(g.k - 1) * db;
+    x.A1 = reinterpret_cast<float *>(s);
+    s += fb;
+    x.P = reinterpret_cast<float *>(s);
+    x.pstride = int64_t(fb / 4);
     if (g.k > kmax) kmax = g.k;
   }
   auto active = [&](int i) { return geoms[i].nprim > 0 && geoms[i].size >= 2 && geoms[i].k > 0; };
+  // X_l, the left factor of P_l: G for l = k, else A_{l+1}
+  auto Xop = [&](int i, int l) -> const void * {
+    return l == geoms[i].k ? w[i].Gop : static_cast<const void *>(w[i].X + size_t(l - 1) * w[i].xb);
+  };
   std::vector<Gemm> gs;
-  // A_k = G - Q G  (all sides), then dQ = G S_k^T (all sides)
+  // the chain, one order per launch (sides with a smaller k finish early)
+  for (int step = 0; step < kmax; ++step) {
+    gs.clear();
+    for (int i = 0; i < count; ++i) {
+      if (!active(i)) continue;
+      const SideGeom &g = geoms[i];
+      const int l = g.k - step;  // order of the A made now
+      if (l < 1) continue;
+      const Work &x = w[i];
+      Gemm a;
+      if (l == g.k) {  // A_k = S_1^T G: S_1 read transposed (M contiguous)
+        a = prim_gemm(g, dtype, x.S1, x.Gop, false, "cnp_bwd");
+        a.a_m = 1; a.a_k = g.ld;
+      } else {         // A_l = -Q A_{l+1}
+        a = prim_gemm(g, dtype, x.Q, Xop(i, l), false, "cnp_bwd");
+        a.alpha = -1.f;
+      }
+      if (l == 1) {
+        a.outF = x.A1; a.of_m = g.ld; a.of_b = g.blk_elems();
+      } else if (dtype == POET_BF16) {
+        a.outD = x.X + size_t(l - 2) * x.xb; a.od_m = g.ld; a.od_b = g.blk_elems();
+      } else {
+        a.outF = reinterpret_cast<float *>(x.X + size_t(l - 2) * x.xb); a.of_m = g.ld; a.of_b = g.blk_elems();
+      }
+      gs.push_back(a);
+    }
+    POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
+  }
+  // every partial product P_l = X_l S_l^T of every side in one launch
   gs.clear();
   for (int i = 0; i < count; ++i) {
     if (!active(i)) continue;
     const SideGeom &g = geoms[i];
-    Gemm p = prim_gemm(g, dtype, w[i].Q, w[i].Gop, false, "cnp_bwd");
-    p.alpha = -1.f;
-    p.add = G[i]; p.add_dtype = POET_F32; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 1.f;
-    p.outF = w[i].Af[0]; p.of_m = g.ld; p.of_b = g.blk_elems();
-    if (dtype == POET_BF16) { p.outD = w[i].Ad[0]; p.od_m = g.ld; p.od_b = g.blk_elems(); }
-    gs.push_back(p);
-  }
-  for (int i = 0; i < count; ++i) {
-    if (!active(i)) continue;
-    const SideGeom &g = geoms[i];
-    Gemm p = prim_gemm(g, dtype, w[i].Gop, w[i].S1 + size_t(g.k - 1) * w[i].term, true, "cnp_bwd");
-    p.outF = w[i].dQ; p.of_m = g.ld; p.of_b = g.blk_elems();
-    gs.push_back(p);
+    for (int l = g.k; l >= 1; --l) {
+      Gemm p = prim_gemm(g, dtype, Xop(i, l), w[i].S1 + size_t(l - 1) * w[i].term, true, "cnp_bwd");
+      p.outF = w[i].P + (l - 1) * w[i].pstride; p.of_m = g.ld; p.of_b = g.blk_elems();
+      gs.push_back(p);
+    }
   }
   POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
-  for (int l = kmax - 1; l >= 1; --l) {
-    // dQ += A_{l+1} S_l^T
-    gs.clear();
-    for (int i = 0; i < count; ++i) {
-      if (!active(i) || l > geoms[i].k - 1) continue;
-      const SideGeom &g = geoms[i];
-      Gemm p = prim_gemm(g, dtype, w[i].Ad[w[i].cur], w[i].S1 + size_t(l - 1) * w[i].term, true, "cnp_bwd");
-      p.add = w[i].dQ; p.add_dtype = POET_F32; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 1.f;
-      p.outF = w[i].dQ; p.of_m = g.ld; p.of_b = g.blk_elems();
-      gs.push_back(p);
-    }
-    POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
-    // A_l = -Q A_{l+1}
-    gs.clear();
-    for (int i = 0; i < count; ++i) {
-      if (!active(i) || l > geoms[i].k - 1) continue;
-      const SideGeom &g = geoms[i];
-      const int cur = w[i].cur;
-      Gemm p = prim_gemm(g, dtype, w[i].Q, w[i].Ad[cur], false, "cnp_bwd");
-      p.alpha = -1.f;
-      p.outF = w[i].Af[cur ^ 1]; p.of_m = g.ld; p.of_b = g.blk_elems();
-      if (dtype == POET_BF16) { p.outD = w[i].Ad[cur ^ 1]; p.od_m = g.ld; p.od_b = g.blk_elems(); }
-      gs.push_back(p);
-      w[i].cur ^= 1;
-    }
-    POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
-  }
   for (int i = 0; i < count; ++i) {
     if (!active(i)) continue;
     const SideGeom &g = geoms[i];
-    pack_grad_kernel<<<grid_for(g.all_elems(), 256), 256, 0, st>>>(w[i].dQ, w[i].Af[w[i].cur], g.nprim, g.size, g.ld,
-                                                                    dtheta[i]);
+    const int tiles = (g.size + PACK_T - 1) / PACK_T;
+    dim3 grid(tiles * (tiles + 1) / 2, g.nprim);
+    pack_sum_kernel<<<grid, dim3(PACK_T, 8), 0, st>>>(w[i].P, g.k, w[i].pstride, w[i].A1, g.nprim, g.size, g.ld,
+                                                      dtheta[i]);
     count_launch();
     POET_TRY(launch_status("cnp pack"));
   }

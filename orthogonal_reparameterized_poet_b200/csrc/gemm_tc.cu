@@ -21,6 +21,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <vector>
 
 #include "poet_internal.cuh"
 
@@ -459,7 +460,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       const int gm = c.mt * BM + row;
       const bool row_ok = gm < p.M;
       const float alpha = p.alpha, beta = p.beta, diag = p.diag;
-      if (p.coalesced) {
+      if (p.coalesced == 1) {
         // plain bf16 output: each 64-column chunk goes row-wise into this warp's
         // staging rows, then out with every store instruction covering four
         // rows x 128 contiguous bytes
@@ -506,6 +507,49 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
                 const bf16 *pv = reinterpret_cast<const bf16 *>(&v);
                 for (int e = 0; e < 8; ++e)
                   if (gn + e < p.N) o[e] = pv[e];
+              }
+            }
+          }
+        }
+      } else if (p.coalesced == 2) {
+        // plain fp32 output: each 32-column chunk (128 B per row) goes row-wise
+        // into this warp's staging rows, then out four rows x 128 B at a time
+        unsigned char *ew = epi + quarter * (32 * S::EPI_ROW);
+        const int m_base = c.mt * BM + quarter * 32;
+        float *obase = p.outF + int64_t(c.b) * p.of_b;
+        const int sub = lane & 7, rsub = lane >> 3;
+        unsigned char *myrow = ew + lane * S::EPI_ROW;
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          uint32_t r[32];
+          __syncwarp();
+          tmem_ld32(tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN + cc * 32), r);
+          tmem_ld_wait();
+          const int gn0 = c.nt * BN + cc * 32;
+          if (gn0 >= p.N) continue;  // the same for the whole warp
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float4 f;
+            f.x = alpha * __uint_as_float(r[4 * q]);
+            f.y = alpha * __uint_as_float(r[4 * q + 1]);
+            f.z = alpha * __uint_as_float(r[4 * q + 2]);
+            f.w = alpha * __uint_as_float(r[4 * q + 3]);
+            *reinterpret_cast<float4 *>(myrow + q * 16) = f;
+          }
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + rsub;
+            const int gm = m_base + rr;
+            const int gn = gn0 + sub * 4;
+            const float4 f = *reinterpret_cast<const float4 *>(ew + rr * S::EPI_ROW + sub * 16);
+            if (gm < p.M && gn < p.N) {
+              float *o = obase + int64_t(gm) * p.of_m + gn;
+              if (gn + 4 <= p.N) {
+                *reinterpret_cast<float4 *>(o) = f;
+              } else {
+                o[0] = f.x;  // gn < N
+                if (gn + 1 < p.N) o[1] = f.y;
+                if (gn + 2 < p.N) o[2] = f.z;
               }
             }
           }
@@ -693,10 +737,15 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   p->outF = g.outF; p->of_m = g.of_m; p->of_b = g.of_b;
   p->outD = static_cast<bf16 *>(g.outD); p->od_m = g.od_m; p->od_b = g.od_b;
   p->atomic = g.atomic ? 1 : 0;
-  p->coalesced = (g.outD && !g.outF && !g.add && g.diag == 0.f && !g.atomic && aligned16(g.outD) &&
-                  g.od_m % 8 == 0 && (g.batch == 1 || g.od_b % 8 == 0))
-                     ? 1
-                     : 0;
+  // staged epilogue for a single plain output with 16-byte aligned rows
+  // (1: bf16, 2: fp32); the per-row path handles addends, pairs of outputs
+  // and split-K reductions
+  p->coalesced = 0;
+  const bool plain = !g.add && !g.atomic && g.diag == 0.f;
+  if (plain && g.outD && !g.outF && aligned16(g.outD) && g.od_m % 8 == 0 && (g.batch == 1 || g.od_b % 8 == 0))
+    p->coalesced = 1;
+  if (plain && g.outF && !g.outD && aligned16(g.outF) && g.of_m % 4 == 0 && (g.batch == 1 || g.of_b % 4 == 0))
+    p->coalesced = 2;
   bool ok;
   if (!t.A_MN) ok = make_map(ma, g.A, g.K, g.M, g.batch, g.a_m, g.a_b, 64, BM);
   else ok = make_map(ma, g.A, g.M, g.K, g.batch, g.a_k, g.a_b, 64, 64);
@@ -802,26 +851,32 @@ bool gemm_tc_supported(const Gemm &g) {
 
 poet_status gemm_tc(const Gemm &g, cudaStream_t st) { return run_group<1>(&g, 1, plan_of(g), st); }
 
-// Runs many independent problems: consecutive tensor-core problems that share
-// operand majors and tile width go into grouped launches of up to kGroupMax
-// problems each; the others run one by one on the CUDA-core engine.
+// Runs many independent problems: tensor-core problems that share operand
+// majors and tile width go into grouped launches of up to kGroupMax problems
+// each (buckets in order of first appearance, list order kept inside a
+// bucket); the others run one by one on the CUDA-core engine.
 poet_status gemm_tc_many(const Gemm *gs, int count, cudaStream_t st) {
-  int i = 0;
-  while (i < count) {
-    if (gs[i].M <= 0 || gs[i].N <= 0 || gs[i].batch <= 0) { ++i; continue; }
+  std::vector<TcPlan> plans;
+  std::vector<std::vector<Gemm>> buckets;
+  for (int i = 0; i < count; ++i) {
+    if (gs[i].M <= 0 || gs[i].N <= 0 || gs[i].batch <= 0) continue;
     if (!(gemm_tc_enabled() && gemm_tc_supported(gs[i]))) {
       POET_TRY(gemm_simt(gs[i], st));
-      ++i;
       continue;
     }
     const TcPlan t = plan_of(gs[i]);
-    int j = i + 1;
-    while (j < count && j - i < kGroupMax && gs[j].M > 0 && gs[j].N > 0 && gs[j].batch > 0 && gemm_tc_supported(gs[j]) &&
-           plan_of(gs[j]) == t)
-      ++j;
-    if (j - i == 1) POET_TRY(run_group<1>(gs + i, 1, t, st));
-    else POET_TRY(run_group<kGroupMax>(gs + i, j - i, t, st));
-    i = j;
+    size_t b = 0;
+    while (b < plans.size() && !(plans[b] == t)) ++b;
+    if (b == plans.size()) { plans.push_back(t); buckets.emplace_back(); }
+    buckets[b].push_back(gs[i]);
+  }
+  for (size_t b = 0; b < plans.size(); ++b) {
+    const std::vector<Gemm> &v = buckets[b];
+    for (size_t i = 0; i < v.size(); i += kGroupMax) {
+      const int n = int(v.size() - i < size_t(kGroupMax) ? v.size() - i : size_t(kGroupMax));
+      if (n == 1) POET_TRY(run_group<1>(v.data() + i, 1, plans[b], st));
+      else POET_TRY(run_group<kGroupMax>(v.data() + i, n, plans[b], st));
+    }
   }
   return POET_OK;
 }

@@ -242,7 +242,7 @@ extern "C" {
 const char *poet_last_error(void) { return g_last_error; }
 
 // The kernel revisions name the code that profiles/ counters were taken on.
-const char *poet_version(void) { return "libpoet 0.2 (sm_100a; gemm_tc r4; permute r3)"; }
+const char *poet_version(void) { return "libpoet 0.2 (sm_100a; gemm_tc r5; permute r3)"; }
 
 size_t poet_side_state_bytes(const poet_side *side, int32_t dtype) {
   SideGeom g;
@@ -486,7 +486,7 @@ size_t poet_cayley_neumann_grad_many_workspace_bytes(const poet_side *sides, int
   for (int i = 0; i < count; ++i) {
     SideGeom g;
     if (!side_geom(&sides[i], &g)) return 0;
-    total += align256(cnp_scratch_bytes(g, dtype));
+    total += align256(cnp_many_scratch_bytes(g, dtype));
   }
   return total;
 }
@@ -507,7 +507,7 @@ poet_status poet_cayley_neumann_grad_many(const poet_side *sides, const float *c
                      (reinterpret_cast<uintptr_t>(G[i]) & 15) == 0,
                  "poet_cayley_neumann_grad_many: side %d state/G/dtheta NULL or misaligned", i);
     scratch[i] = static_cast<char *>(ws) + off;
-    off += align256(cnp_scratch_bytes(geoms[i], dtype));
+    off += align256(cnp_many_scratch_bytes(geoms[i], dtype));
   }
   if (off > 0 && (!ws || ws_bytes < off || !aligned256(ws))) {
     set_error("poet_cayley_neumann_grad_many: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, off);

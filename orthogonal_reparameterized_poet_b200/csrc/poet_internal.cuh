@@ -146,10 +146,11 @@ poet_status cnp_backward(const poet_side *side, const SideGeom &g, int dtype, co
                          float *dtheta, void *scratch, cudaStream_t st);
 size_t cnp_scratch_bytes(const SideGeom &g, int dtype);
 // The same for many sides at once; their GEMM steps share grouped launches.
-// G[i]: float [nprim][ld][ld]; scratch[i]: cnp_scratch_bytes(geoms[i], dtype) bytes each.
+// G[i]: float [nprim][ld][ld]; scratch[i]: cnp_many_scratch_bytes(geoms[i], dtype) bytes each.
 poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int count, int dtype, cudaStream_t st);
 poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int count, int dtype,
                               const float *const *G, float *const *dtheta, void *const *scratch, cudaStream_t st);
+size_t cnp_many_scratch_bytes(const SideGeom &g, int dtype);
 // out = G (dense [nprim][size][size]) re-laid as [nprim][ld][ld] with zero padding
 poet_status pad_blocks(const float *G, const SideGeom &g, float *out, cudaStream_t st);
 

@@ -222,17 +222,30 @@ def _make_layer(cuda, case):
     return L, cuda.from_numpy(x).to("cuda", tdt), cuda.from_numpy(dy).to("cuda", tdt), (W0, thR, thP, x, dy)
 
 
-MANY_CASES = [  # different sizes, modes and Neumann orders in one call
-    Case(512, 512, I.FS, 0, I.FS, 0, 4, 300, I.BF16, 0.02, layer_id=21),
-    Case(1376, 512, I.FS, 0, I.FS, 0, 4, 300, I.BF16, 0.02, layer_id=22),
-    Case(1024, 768, I.BS, 256, I.BS, 256, 4, 300, I.BF16, 0.02, layer_id=23),
-    Case(640, 512, I.BS, 128, I.FS, 0, 2, 300, I.BF16, 0.03, layer_id=24),
-]
+MANY_SETS = {  # different sizes, modes and Neumann orders in one call
+    "bf16": [
+        Case(512, 512, I.FS, 0, I.FS, 0, 4, 300, I.BF16, 0.02, layer_id=21),
+        Case(1376, 512, I.FS, 0, I.FS, 0, 4, 300, I.BF16, 0.02, layer_id=22),
+        Case(1024, 768, I.BS, 256, I.BS, 256, 4, 300, I.BF16, 0.02, layer_id=23),
+        Case(640, 512, I.BS, 128, I.FS, 0, 2, 300, I.BF16, 0.03, layer_id=24),
+    ],
+    "f32": [  # odd sizes (ragged tiles), k = 3, 1 and 0
+        Case(301, 200, I.FS, 0, I.BS, 48, 3, 130, I.F32, 0.03, layer_id=25),
+        Case(200, 301, I.BS, 64, I.FS, 0, 1, 130, I.F32, 0.03, layer_id=26),
+        Case(96, 130, I.FS, 0, I.FS, 0, 0, 130, I.F32, 0.03, layer_id=27),
+    ],
+}
+# The grouped gradient computes (I + Q)^T G from the operand copy of G and
+# sums its partial products in another order than the one-side path, so the
+# two agree to a few roundings of the operand type.
+MANY_VS_SINGLE = {"bf16": 5e-3, "f32": 1e-5}
 
 
-def test_many_sides_match_single_calls_and_oracle(cuda):
+@pytest.mark.parametrize("which", sorted(MANY_SETS))
+def test_many_sides_match_single_calls_and_oracle(cuda, which):
     from orthogonal_reparameterized_poet_b200 import poet
 
+    MANY_CASES = MANY_SETS[which]
     built = [_make_layer(cuda, c) for c in MANY_CASES]
     layers = [b[0] for b in built]
     # a1: grouped launch vs one call per side (same tiles, same order: bitwise equal)
@@ -241,7 +254,7 @@ def test_many_sides_match_single_calls_and_oracle(cuda):
     for L in layers:
         L.cayley_neumann()
     for L, r in zip(layers, many_R):
-        n = poet.poet_block_grad_bytes(L.struct.R) // 2
+        n = poet.poet_block_grad_bytes(L.struct.R) // 4 * (2 if L.dtype == I.BF16 else 4)  # all of B
         assert cuda.equal(L.state_R[:n], r[:n])
     # a5..a8 split: backward_blocks + grouped a8 vs poet_backward, and both vs the oracle
     G, dth, dth_ref = [], [], []
@@ -262,5 +275,5 @@ def test_many_sides_match_single_calls_and_oracle(cuda):
         tol = TOL[case.dtype]
         assert rel_fro(dR.cpu().numpy(), ref["dthetaR"]) <= tol
         assert rel_fro(dP.cpu().numpy(), ref["dthetaP"]) <= tol
-        assert rel_fro(dR.cpu().numpy(), dR1.cpu().numpy()) <= 1e-3  # G sums differ only in atomic order
-        assert rel_fro(dP.cpu().numpy(), dP1.cpu().numpy()) <= 1e-3
+        assert rel_fro(dR.cpu().numpy(), dR1.cpu().numpy()) <= MANY_VS_SINGLE[which]
+        assert rel_fro(dP.cpu().numpy(), dP1.cpu().numpy()) <= MANY_VS_SINGLE[which]
