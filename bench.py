@@ -38,6 +38,8 @@ WORKLOAD_SETS = {
     "llama3b": ["llama3b_fs"],
 }
 METRIC = "POET layer fwd+bwd tokens/s at LLaMA-1.3B shapes; % of TC/HBM roofline"
+PLANS = {"auto": 0, "token": 1, "weight": 2}
+PLAN_NAMES = {1: "token", 2: "weight"}
 
 # DRAM traffic / algorithmic bytes of one launch, from an ncu capture, with the
 # kernel revision (as named in poet_version()) the counters were taken on.
@@ -55,6 +57,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-merge", action="store_true")
+    ap.add_argument("--plan", choices=sorted(PLANS), default="auto",
+                    help="where the primitives act: auto (cost model), token (activations) or weight (W0)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (small profiling cases)")
     return ap.parse_args()
 
@@ -129,7 +133,7 @@ class ClockSampler:
 class Variant:
     """All POET linears of one workload, resident on the device."""
 
-    def __init__(self, wl, rank, device, w0_cache, act_cache, saved_pool):
+    def __init__(self, wl, rank, device, w0_cache, act_cache, saved_pool, plan=0):
         import torch
 
         from orthogonal_reparameterized_poet_b200 import inputs as I
@@ -155,7 +159,7 @@ class Variant:
                 thR = torch.from_numpy(I.theta(wl.seed, layer, t, 0, nR * sR * (sR - 1) // 2, wl.sigma)).to(device)
                 thP = torch.from_numpy(I.theta(wl.seed, layer, t, 1, nP * sP * (sP - 1) // 2, wl.sigma)).to(device)
                 L = poet.PoetLayer(W0, thR, thP, mode=wl.mode, b=wl.b, k=wl.k, seed=wl.seed,
-                                   layer_id=layer * len(shapes) + t)
+                                   layer_id=layer * len(shapes) + t, plan=plan)
                 L.prepare()
                 self.layers.append((layer, t, m, n, L))
                 nth.append((thR.numel(), thP.numel()))
@@ -229,7 +233,8 @@ class Variant:
             L.forward(self.x[n], y=self.y[m], saved=self.saved[i], ws=self.ws)
         for i in reversed(range(len(self.layers))):
             _, _, m, n, L = self.layers[i]
-            L.backward_blocks(self.saved[i], self.dy[m], self.G[i][0], self.G[i][1], dx=self.dx[n], ws=self.ws)
+            L.backward_blocks(self.saved[i], self.dy[m], self.G[i][0], self.G[i][1], dx=self.dx[n], ws=self.ws,
+                              x=self.x[n])
         for c0 in range(0, len(pl), self.chunk):  # a8 for every layer, in grouped launches
             poet.cayley_neumann_grad_many(pl[c0:c0 + self.chunk], self.G[c0:c0 + self.chunk],
                                           self.dslices[c0:c0 + self.chunk], self.gws)
@@ -273,7 +278,7 @@ def run_poet(args):
 
         wls = [dataclasses.replace(w, layers=args.layers) for w in wls]
     w0_cache, act_cache, saved_pool = {}, {}, []
-    variants = [Variant(wl, rank, device, w0_cache, act_cache, saved_pool) for wl in wls]
+    variants = [Variant(wl, rank, device, w0_cache, act_cache, saved_pool, PLANS[args.plan]) for wl in wls]
     del w0_cache
     ws = torch.empty(max(v.ws_need for v in variants), dtype=torch.uint8, device=device)  # one shared workspace
     gws_need = max(v.alloc_grads(device, chunk=4 * len(v.wl.linear_shapes())) for v in variants)
@@ -410,8 +415,11 @@ def run_poet(args):
         "config": {"workload": args.workload + "_" + "+".join(w.name.split("_", 1)[1] for w in wls),
                    "hidden": wls[0].hidden, "ffn": wls[0].ffn, "layers": wls[0].layers,
                    "linears_per_layer": len(wls[0].linear_shapes()), "tokens_per_variant": wls[0].tokens,
-                   "variants": [{"name": w.name, "mode": "FS" if w.mode == I.FS else "BS", "b": w.b, "k": w.k}
-                                for w in wls],
+                   "variants": [{"name": v.wl.name, "mode": "FS" if v.wl.mode == I.FS else "BS", "b": v.wl.b,
+                                 "k": v.wl.k, "plan": "+".join(sorted({PLAN_NAMES[L.plan_for(v.T)]
+                                                                       for (_, _, _, _, L) in v.layers}))}
+                                for v in variants],
+                   "plan_requested": args.plan,
                    "parallelism": f"dp{world}", "l2": "inputs larger than L2 (no flush needed)"},
         "variants": {v.wl.name: {"ms_per_step": round(per_variant_ms[i] / args.steps, 3),
                                  "tokens_per_s": round(v.T * world / (per_variant_ms[i] / args.steps / 1e3), 1),

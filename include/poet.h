@@ -48,8 +48,22 @@
  * The permuted frame.  The library keeps a copy of W0 with rows ordered by
  * R.perm and columns by P.perm (W0f[i][j] = W0[R.perm[i]][P.perm[j]]), so
  * that every primitive acts on a contiguous range of frame indices and every
- * contraction on the hot path reads contiguous tiles.  Activations are
- * gathered into the frame once on entry and scattered out once on exit.
+ * contraction on the hot path reads contiguous tiles.
+ *
+ * Two plans compute the same layer (the pages fix what is computed, not the
+ * order of the products; both are exact rearrangements of y = R W0 P x):
+ *  - token plan: the primitives act on the activations.  Activations are
+ *    gathered into the frame once on entry, pass through the blocks of P,
+ *    W0f and the blocks of R, and are scattered out once on exit.  Cost per
+ *    token ~ 2mn + 2(sum of primitive sizes squared) flops plus four
+ *    activation-sized permutation passes (forward and backward).
+ *  - weight plan: the primitives act on W0.  The forward forms the
+ *    effective weight E = R W0 P (weight-sized work) and runs one GEMM
+ *    y = x E^T; the backward runs dx = dy E and D = dy^T x and takes the
+ *    per-primitive gradients from D (weight-sized work again).  Cost per
+ *    token ~ 3 x 2mn flops and no activation permutation.
+ *  poet_layer.plan selects one; POET_PLAN_AUTO picks the cheaper for the
+ *  token count (poet_plan_for tells which).
  */
 #ifndef POET_H
 #define POET_H
@@ -80,6 +94,7 @@ typedef enum {
 
 typedef enum { POET_F32 = 0, POET_BF16 = 1 } poet_dtype;
 typedef enum { POET_BS = 0, POET_FS = 1 } poet_mode;
+typedef enum { POET_PLAN_AUTO = 0, POET_PLAN_TOKEN = 1, POET_PLAN_WEIGHT = 2 } poet_plan;
 
 typedef struct {
   int32_t dim;     /* m for R, n for P; 1 <= dim <= 16384 */
@@ -101,7 +116,7 @@ typedef struct {
   int32_t dtype;   /* poet_dtype of W0, W0f, activations, primitives */
   int32_t layer_id;/* >= 0; keys the permutation draw */
   int32_t epoch;   /* >= 0; advanced by poet_resample */
-  int32_t reserved;/* must be 0 */
+  int32_t plan;    /* poet_plan: POET_PLAN_AUTO (0), _TOKEN or _WEIGHT */
   uint64_t seed;   /* keys the permutation draw */
   void *W0;        /* device m x n, row-major, natural order (the fixed weight) */
   void *W0f;       /* device, poet_frame_bytes() bytes: W0 in the permuted frame */
@@ -117,7 +132,17 @@ POET_API size_t poet_side_state_bytes(const poet_side *side, int32_t dtype);
 /* Bytes of L->W0f (0 if the layer is invalid). */
 POET_API size_t poet_frame_bytes(const poet_layer *L);
 
-/* Bytes of the buffer poet_forward saves for poet_backward at T tokens. */
+/* The plan poet_forward / poet_backward run for this layer at T tokens
+ * (POET_PLAN_TOKEN or POET_PLAN_WEIGHT; -1 if the layer is invalid).  With
+ * POET_PLAN_AUTO the choice depends only on the shapes, the sides' geometry
+ * and T: the plan with the smaller estimated device time, counting flops at
+ * the tensor-core rate and activation or weight passes at the HBM rate. */
+POET_API int32_t poet_plan_for(const poet_layer *L, int64_t T);
+
+/* Bytes of the buffer poet_forward saves for poet_backward at T tokens
+ * (token plan: the frame copies of x and of W0 P x; weight plan: the
+ * effective weight and two weight-sized factors, plus a 16-byte aligned copy
+ * of x when n is not a multiple of 8). */
 POET_API size_t poet_saved_bytes(const poet_layer *L, int64_t T);
 
 /* Bytes of workspace that poet_forward, poet_backward, poet_merge and
@@ -182,10 +207,13 @@ POET_API poet_status poet_forward(const poet_layer *L, const void *x, int64_t T,
  * dx = P^T W0^T R^T dy (device T x n, dtype) and the gradients of the loss
  * with respect to both sides' packed parameters (device float, overwritten,
  * same layout as theta).  W0 is fixed ([P1] Approach), so there is no dW0.
- * saved: the buffer poet_forward filled for the same x and T. */
-POET_API poet_status poet_backward(const poet_layer *L, const void *saved, const void *dy,
-                          int64_t T, void *dx, float *dtheta_R, float *dtheta_P,
-                          void *ws, size_t ws_bytes, poet_stream stream);
+ * x: the forward's input (device T x n), read by the weight plan (D = dy^T x)
+ * and ignored by the token plan (may be NULL there).  saved: the buffer
+ * poet_forward filled for the same x and T.  The layer's plan, state and
+ * W0f must be those of that forward. */
+POET_API poet_status poet_backward(const poet_layer *L, const void *x, const void *saved,
+                          const void *dy, int64_t T, void *dx, float *dtheta_R,
+                          float *dtheta_P, void *ws, size_t ws_bytes, poet_stream stream);
 
 /* ---------------------------------------------------------------- many layers at once
  *
@@ -206,9 +234,9 @@ POET_API poet_status poet_cayley_neumann_many(const poet_side *sides, int32_t co
 /* a5..a7 of poet_backward: writes dx and the per-primitive gradients
  * G_R = dL/dR_j and G_P = dL/dP_j (device, poet_block_grad_bytes each,
  * 16-byte aligned, overwritten) instead of dtheta. */
-POET_API poet_status poet_backward_blocks(const poet_layer *L, const void *saved, const void *dy,
-                                          int64_t T, void *dx, float *G_R, float *G_P,
-                                          void *ws, size_t ws_bytes, poet_stream stream);
+POET_API poet_status poet_backward_blocks(const poet_layer *L, const void *x, const void *saved,
+                                          const void *dy, int64_t T, void *dx, float *G_R,
+                                          float *G_P, void *ws, size_t ws_bytes, poet_stream stream);
 
 /* Workspace bytes of poet_cayley_neumann_grad_many for these sides. */
 POET_API size_t poet_cayley_neumann_grad_many_workspace_bytes(const poet_side *sides, int32_t count,

@@ -460,10 +460,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       const int gm = c.mt * BM + row;
       const bool row_ok = gm < p.M;
       const float alpha = p.alpha, beta = p.beta, diag = p.diag;
-      if (p.coalesced == 1) {
+      if (p.coalesced == 1 || p.coalesced == 3) {
         // plain bf16 output: each 64-column chunk goes row-wise into this warp's
         // staging rows, then out with every store instruction covering four
-        // rows x 128 contiguous bytes
+        // rows x 128 contiguous bytes (mode 1), or, for rows that are not
+        // 16-byte aligned (mode 3), one row x 128 bytes in 4-byte words
         unsigned char *ew = epi + quarter * (32 * S::EPI_ROW);
         const int m_base = c.mt * BM + quarter * 32;
         bf16 *obase = p.outD + int64_t(c.b) * p.od_b;
@@ -493,6 +494,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
             *reinterpret_cast<uint4 *>(myrow + q * 16) = pk;
           }
           __syncwarp();
+          if (p.coalesced == 3) {
+            const int nv = min(64, p.N - gn0);
+            const int rows = min(32, p.M - m_base);
+            for (int rr = 0; rr < rows; ++rr) {
+              const bf16 *srow = reinterpret_cast<const bf16 *>(ew + rr * S::EPI_ROW);
+              bf16 *o = obase + int64_t(m_base + rr) * p.od_m + gn0;
+              const int mis = int((reinterpret_cast<uintptr_t>(o) >> 1) & 1);  // o is 2 mod 4
+              const int e0 = 2 * lane - mis;  // lane's word covers elements e0, e0 + 1
+              if (e0 >= 0 && e0 + 1 < nv) {
+                __nv_bfloat162 h;
+                h.x = srow[e0];
+                h.y = srow[e0 + 1];
+                *reinterpret_cast<__nv_bfloat162 *>(o + e0) = h;
+              } else {
+                if (e0 >= 0 && e0 < nv) o[e0] = srow[e0];
+                if (e0 + 1 >= 0 && e0 + 1 < nv) o[e0 + 1] = srow[e0 + 1];
+              }
+              if (mis && lane == 0 && 63 < nv) o[63] = srow[63];
+            }
+            continue;
+          }
 #pragma unroll
           for (int it = 0; it < 8; ++it) {
             const int rr = it * 4 + rsub;
@@ -737,13 +759,13 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   p->outF = g.outF; p->of_m = g.of_m; p->of_b = g.of_b;
   p->outD = static_cast<bf16 *>(g.outD); p->od_m = g.od_m; p->od_b = g.od_b;
   p->atomic = g.atomic ? 1 : 0;
-  // staged epilogue for a single plain output with 16-byte aligned rows
-  // (1: bf16, 2: fp32); the per-row path handles addends, pairs of outputs
-  // and split-K reductions
+  // staged epilogue for a single plain output (1: bf16, 16-byte aligned rows;
+  // 3: bf16, any rows; 2: fp32, 16-byte aligned rows); the per-row path
+  // handles addends, pairs of outputs and split-K reductions
   p->coalesced = 0;
   const bool plain = !g.add && !g.atomic && g.diag == 0.f;
-  if (plain && g.outD && !g.outF && aligned16(g.outD) && g.od_m % 8 == 0 && (g.batch == 1 || g.od_b % 8 == 0))
-    p->coalesced = 1;
+  if (plain && g.outD && !g.outF)
+    p->coalesced = aligned16(g.outD) && g.od_m % 8 == 0 && (g.batch == 1 || g.od_b % 8 == 0) ? 1 : 3;
   if (plain && g.outF && !g.outD && aligned16(g.outF) && g.of_m % 4 == 0 && (g.batch == 1 || g.of_b % 4 == 0))
     p->coalesced = 2;
   bool ok;

@@ -155,7 +155,9 @@ __global__ void __launch_bounds__(NT) permute_rows_kernel(const PermArgs<T> a) {
   const int nthr = blockDim.x, warps = nthr / 32;
   for (int i = threadIdx.x; i < a.map_len; i += nthr) map[i] = 0;
   __syncthreads();
-  if (a.inverse) {
+  if (!a.perm) {  // identity: a plain row copy (re-striding)
+    for (int i = threadIdx.x; i < d; i += nthr) map[i] = uint16_t(i);
+  } else if (a.inverse) {
     for (int i = threadIdx.x; i < d; i += nthr) map[a.perm[i]] = uint16_t(i);
   } else {
     for (int i = threadIdx.x; i < d; i += nthr) map[i] = uint16_t(a.perm[i]);
@@ -209,6 +211,53 @@ __global__ void __launch_bounds__(NT) permute_rows_kernel(const PermArgs<T> a) {
   cp_async_wait_all();
 }
 
+// Plain row copy to 16-byte aligned destination rows (re-striding rows whose
+// start is only element-aligned).  Destination unit u (16 bytes) of a row is
+// assembled from the two aligned 16-byte source words u and u + 1 of that
+// row, shifted by the row's misalignment; every word read overlaps the row.
+// Columns past d in the last unit receive bytes of the source's next
+// elements (padding, never read as data).
+template <int H>  // shift by H 16-bit halves (0..7)
+__device__ __forceinline__ uint4 shift_pair(const uint4 &a, const uint4 &b) {
+  const uint32_t c[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if constexpr (H % 2 == 0) o[i] = c[i + H / 2];
+    else o[i] = __byte_perm(c[i + H / 2], c[i + H / 2 + 1], 0x5432);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__global__ void __launch_bounds__(256) restride_kernel(const unsigned char *__restrict__ src, int64_t ld_src_bytes,
+                                                       int64_t rows, int row_bytes, unsigned char *__restrict__ dst,
+                                                       int64_t ld_dst_bytes) {
+  const int units = (row_bytes + 15) / 16;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const unsigned char *srow = src + r * ld_src_bytes;
+    const int off = int(reinterpret_cast<uintptr_t>(srow) & 15);  // even: elements are >= 2 bytes
+    const uint4 *wp = reinterpret_cast<const uint4 *>(srow - off);
+    const int nwords = (off + row_bytes + 15) / 16;  // aligned words overlapping the row
+    uint4 *drow = reinterpret_cast<uint4 *>(dst + r * ld_dst_bytes);
+    for (int u = threadIdx.x; u < units; u += blockDim.x) {
+      const uint4 w0 = wp[u];
+      const uint4 w1 = u + 1 < nwords ? wp[u + 1] : make_uint4(0, 0, 0, 0);
+      uint4 v;
+      switch (off >> 1) {
+        case 0: v = w0; break;
+        case 1: v = shift_pair<1>(w0, w1); break;
+        case 2: v = shift_pair<2>(w0, w1); break;
+        case 3: v = shift_pair<3>(w0, w1); break;
+        case 4: v = shift_pair<4>(w0, w1); break;
+        case 5: v = shift_pair<5>(w0, w1); break;
+        case 6: v = shift_pair<6>(w0, w1); break;
+        default: v = shift_pair<7>(w0, w1); break;
+      }
+      drow[u] = v;
+    }
+  }
+}
+
 template <typename T>
 poet_status launch_permute(PermArgs<T> a, cudaStream_t st, const char *kind) {
   if (a.rows <= 0 || a.d <= 0) return POET_OK;
@@ -244,7 +293,7 @@ poet_status launch_permute(PermArgs<T> a, cudaStream_t st, const char *kind) {
 
 poet_status gather_cols(int dtype, const void *src, int64_t ld_src, const int32_t *rowmap, int64_t rows, int d,
                         const int32_t *perm, void *dst, int64_t ld_dst, void *dst2, int64_t ld_dst2, int split,
-                        cudaStream_t st) {
+                        cudaStream_t st, const char *kind) {
   POET_REQUIRE((reinterpret_cast<uintptr_t>(dst) & 15) == 0 && ld_dst * int64_t(esize(dtype)) % 16 == 0,
                "gather: frame rows must be 16-byte aligned");
   auto fill = [&](auto *tag) {
@@ -258,14 +307,30 @@ poet_status gather_cols(int dtype, const void *src, int64_t ld_src, const int32_
     a.dst1 = static_cast<T *>(dst); a.ldd1 = ld_dst;
     a.dst2 = static_cast<T *>(dst2); a.ldd2 = ld_dst2; a.dsplit = dst2 ? split : d;
     a.dst_rowmap = nullptr;
-    return launch_permute<T>(a, st, "gather");
+    return launch_permute<T>(a, st, kind);
   };
   return dtype == POET_BF16 ? fill(static_cast<bf16 *>(nullptr)) : fill(static_cast<float *>(nullptr));
 }
 
+poet_status copy_rows(int dtype, const void *src, int64_t ld_src, int64_t rows, int d, void *dst, int64_t ld_dst,
+                      cudaStream_t st) {
+  const int64_t es = int64_t(esize(dtype));
+  POET_REQUIRE((reinterpret_cast<uintptr_t>(dst) & 15) == 0 && ld_dst * es % 16 == 0 && ld_dst >= round_up(d, 16 / es),
+               "copy_rows: destination rows must be 16-byte aligned and hold whole 16-byte units");
+  POET_REQUIRE((reinterpret_cast<uintptr_t>(src) % es) == 0, "copy_rows: source misaligned");
+  if (rows <= 0 || d <= 0) return POET_OK;
+  TraceScope ts("pad", 0.0, double(rows) * d * es * 2.0, st);
+  const int64_t cap = int64_t(num_sms()) * 8;
+  const int grid = int(rows < cap ? rows : cap);
+  restride_kernel<<<grid, 256, 0, st>>>(static_cast<const unsigned char *>(src), ld_src * es, rows, int(d * es),
+                                        static_cast<unsigned char *>(dst), ld_dst * es);
+  count_launch();
+  return launch_status("pad");
+}
+
 poet_status scatter_cols(int dtype, const void *src1, int64_t ld1, const void *src2, int64_t ld2, int split,
                          int64_t rows, int d, const int32_t *perm, void *dst, int64_t ld_dst, const int32_t *rowmap,
-                         cudaStream_t st) {
+                         cudaStream_t st, const char *kind) {
   const size_t es = esize(dtype);
   POET_REQUIRE((reinterpret_cast<uintptr_t>(src1) & 15) == 0 && ld1 * int64_t(es) % 16 == 0 &&
                    (split >= d || ((reinterpret_cast<uintptr_t>(src2) & 15) == 0 && ld2 * int64_t(es) % 16 == 0)),
@@ -281,7 +346,7 @@ poet_status scatter_cols(int dtype, const void *src1, int64_t ld1, const void *s
     a.dst1 = static_cast<T *>(dst); a.ldd1 = ld_dst;
     a.dst2 = nullptr; a.ldd2 = 0; a.dsplit = d;
     a.dst_rowmap = rowmap;
-    return launch_permute<T>(a, st, "scatter");
+    return launch_permute<T>(a, st, kind);
   };
   return dtype == POET_BF16 ? fill(static_cast<bf16 *>(nullptr)) : fill(static_cast<float *>(nullptr));
 }

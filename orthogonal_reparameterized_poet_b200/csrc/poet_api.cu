@@ -11,6 +11,14 @@
 //             G_R[j] = dyf_j^T vf_j,  G_P[j] = duf_j^T xf_j  (summed over tokens)
 //             dtheta = Cayley-Neumann backward of G
 // Frame indices past q*s (the leftover identity part) pass through unchanged.
+//
+// The weight plan computes the same layer with the primitives applied to W0:
+//   forward   H = R W0f, F = W0f P, E_f = H P (frame, weight-sized),
+//             E = E_f unframed (natural order),  y = x E^T       (saved: E, F, H)
+//   backward  dx = dy E,  D = dy^T x (natural),  D_f = D framed,
+//             G_R[j] = D_f[rows j] F[rows j]^T,  G_P[j] = H[:, cols j]^T D_f[:, cols j]
+// (G_R = sum_t dyf_t vf_t^T with vf_t = F xf_t, and G_P = sum_t duf_t xf_t^T with
+// duf_t = H^T dyf_t, so both plans give the same gradients.)
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -116,6 +124,7 @@ struct LayerGeom {
   SideGeom R, P;
   int64_t m = 0, n = 0, ldm = 0, ldn = 0;
   int dtype = 0;
+  int plan = POET_PLAN_AUTO;  // as requested; resolve_plan() gives the one that runs
 };
 
 poet_status check_layer(const poet_layer *L, LayerGeom *lg, bool need_state) {
@@ -127,7 +136,9 @@ poet_status check_layer(const poet_layer *L, LayerGeom *lg, bool need_state) {
                L->P.dim, (long long)L->m, (long long)L->n);
   POET_REQUIRE(side_geom(&L->R, &lg->R), "malformed R side (mode %d, b %d, k %d)", L->R.mode, L->R.b, L->R.k);
   POET_REQUIRE(side_geom(&L->P, &lg->P), "malformed P side (mode %d, b %d, k %d)", L->P.mode, L->P.b, L->P.k);
-  POET_REQUIRE(L->layer_id >= 0 && L->epoch >= 0 && L->reserved == 0, "layer_id/epoch must be >= 0, reserved 0");
+  POET_REQUIRE(L->layer_id >= 0 && L->epoch >= 0, "layer_id/epoch must be >= 0");
+  POET_REQUIRE(L->plan == POET_PLAN_AUTO || L->plan == POET_PLAN_TOKEN || L->plan == POET_PLAN_WEIGHT,
+               "plan %d is not a poet_plan", L->plan);
   POET_REQUIRE(L->R.perm && L->P.perm, "perm pointers must not be NULL");
   POET_REQUIRE(L->W0 && aligned_elem(L->W0, L->dtype), "W0 is NULL or misaligned");
   POET_REQUIRE(L->W0f && aligned256(L->W0f), "W0f is NULL or not 256-byte aligned");
@@ -140,29 +151,78 @@ poet_status check_layer(const poet_layer *L, LayerGeom *lg, bool need_state) {
   lg->ldm = frame_ld(L->m);
   lg->ldn = frame_ld(L->n);
   lg->dtype = L->dtype;
+  lg->plan = L->plan;
   return POET_OK;
 }
 
+// Plan choice for POET_PLAN_AUTO: estimated device time of fwd + bwd in
+// tensor-core flop equivalents, one HBM byte counted as kFlopPerByte flops
+// (about the ratio of the B200's dense bf16 rate to its HBM bandwidth).
+constexpr double kFlopPerByte = 200.0;
+int resolve_plan(const LayerGeom &lg, int64_t T) {
+  if (lg.plan == POET_PLAN_TOKEN || lg.plan == POET_PLAN_WEIGHT) return lg.plan;
+  const double m = double(lg.m), n = double(lg.n), t = double(T), es = double(esize(lg.dtype));
+  const double cR = double(lg.R.nprim) * lg.R.size * lg.R.size, cP = double(lg.P.nprim) * lg.P.size * lg.P.size;
+  // token plan: W0f forward and backward, three block products per side,
+  // four permutation passes and the block passes' activation traffic
+  const double tok = t * (4.0 * m * n + 6.0 * (cR + cP) + kFlopPerByte * es * 8.0 * (m + n));
+  // weight plan: three T x m x n GEMMs, the weight-sized block products and
+  // passes, and re-striding copies of x / dy whose rows are not 16-byte aligned
+  double wt = t * 6.0 * m * n + 4.0 * n * cR + 6.0 * m * cP + kFlopPerByte * es * 12.0 * m * n;
+  if (lg.n % 8) wt += kFlopPerByte * es * 2.0 * t * n;
+  if (lg.m % 8) wt += kFlopPerByte * es * 2.0 * t * m;
+  return wt < tok ? POET_PLAN_WEIGHT : POET_PLAN_TOKEN;
+}
+
 struct WsLayout {
-  size_t act1 = 0, act2 = 0, act3 = 0, GR = 0, GP = 0, cnp = 0, Z = 0, bytes = 0;
+  size_t act1 = 0, act2 = 0, act3 = 0, GR = 0, GP = 0, cnp = 0, Z = 0, D = 0, D2 = 0, bytes = 0;
 };
 
-WsLayout ws_layout(const LayerGeom &lg, int64_t T) {
+// token plan: act1..act3 activation frames;  weight plan: act1 = re-strided
+// dy, D / D2 = float m x ldn (D and its framed copy).  Both: GR, GP, the
+// Cayley-Neumann scratch and Z (m x ldn, merge and the weight plan's E_f).
+WsLayout ws_layout(const LayerGeom &lg, int64_t T, int plan) {
   WsLayout w;
   const size_t es = esize(lg.dtype);
   const int64_t ldmax = lg.ldm > lg.ldn ? lg.ldm : lg.ldn;
+  const size_t wsz = size_t(lg.m) * lg.ldn;
   size_t off = 0;
-  w.act1 = off; off += align256(size_t(T) * ldmax * es);
-  w.act2 = off; off += align256(size_t(T) * lg.ldm * es);
-  w.act3 = off; off += align256(size_t(T) * lg.ldn * es);
+  if (plan == POET_PLAN_WEIGHT) {
+    w.act1 = off; off += align256(size_t(T) * lg.ldm * es);
+  } else {
+    w.act1 = off; off += align256(size_t(T) * ldmax * es);
+    w.act2 = off; off += align256(size_t(T) * lg.ldm * es);
+    w.act3 = off; off += align256(size_t(T) * lg.ldn * es);
+  }
   w.GR = off; off += align256(size_t(lg.R.all_elems()) * 4);
   w.GP = off; off += align256(size_t(lg.P.all_elems()) * 4);
   w.cnp = off;
   const size_t cr = cnp_scratch_bytes(lg.R, lg.dtype), cp = cnp_scratch_bytes(lg.P, lg.dtype);
   off += cr > cp ? cr : cp;
-  w.Z = off; off += align256(size_t(lg.m) * lg.ldn * es);
+  w.Z = off; off += align256(wsz * es);
+  if (plan == POET_PLAN_WEIGHT) {
+    w.D = off; off += align256(wsz * 4);
+    w.D2 = off; off += align256(wsz * 4);
+  }
   w.bytes = off;
   return w;
+}
+
+// Weight plan saved buffer: E (natural), F, H (frame), all m x ldn, then a
+// T x ldn re-strided copy of x (used when x's rows are not 16-byte aligned).
+struct WeightSaved {
+  size_t E = 0, F = 0, H = 0, xp = 0, bytes = 0;
+};
+WeightSaved weight_saved(const LayerGeom &lg, int64_t T) {
+  WeightSaved v;
+  const size_t w = align256(size_t(lg.m) * lg.ldn * esize(lg.dtype));
+  v.E = 0; v.F = w; v.H = 2 * w; v.xp = 3 * w;
+  v.bytes = 3 * w + align256(size_t(T) * lg.ldn * esize(lg.dtype));
+  return v;
+}
+
+bool rows16(const void *p, int64_t ld, int dtype) {
+  return (reinterpret_cast<uintptr_t>(p) & 15) == 0 && (ld * int64_t(esize(dtype))) % 16 == 0;
 }
 
 size_t side_ws_bytes(const SideGeom &g, int dtype) {
@@ -201,6 +261,51 @@ Gemm blockgrad(const SideGeom &g, int dtype, int64_t T, const void *D, const voi
 
 const void *state_R(const poet_side *s, const SideGeom &g, int dtype) {
   return static_cast<const char *>(s->state) + state_layout(g, dtype).R;
+}
+
+// out = blockdiag(R) src on the rows of an m x ldn frame matrix: the rows of
+// each R primitive are multiplied by it, the leftover rows are copied.
+Gemm left_blocks(const poet_layer *L, const LayerGeom &lg, const void *src, void *out, const char *tag) {
+  const SideGeom &g = lg.R;
+  const int64_t ldw = lg.ldn;
+  Gemm p;
+  p.tag = tag;
+  p.M = g.size; p.N = int(lg.n); p.K = g.size; p.batch = g.nprim; p.dtype = lg.dtype;
+  p.A = state_R(&L->R, g, lg.dtype); p.a_m = g.ld; p.a_k = 1; p.a_b = g.blk_elems();
+  p.B = src; p.b_n = 1; p.b_k = ldw; p.b_b = int64_t(g.size) * ldw;
+  p.outD = out; p.od_m = ldw; p.od_b = int64_t(g.size) * ldw;
+  return p;
+}
+poet_status left_tail(const LayerGeom &lg, const void *src, void *out, cudaStream_t st) {
+  if (lg.R.covered >= lg.m) return POET_OK;
+  const size_t es = esize(lg.dtype), row = size_t(lg.ldn) * es;
+  POET_CUDA_TRY(cudaMemcpyAsync(static_cast<char *>(out) + size_t(lg.R.covered) * row,
+                                static_cast<const char *>(src) + size_t(lg.R.covered) * row,
+                                size_t(lg.m - lg.R.covered) * row, cudaMemcpyDeviceToDevice, st));
+  return POET_OK;
+}
+
+// out = src blockdiag(P) on the columns of an m x ldn frame matrix: the
+// columns of each P primitive are multiplied by it, the leftover columns are
+// copied.
+Gemm right_blocks(const poet_layer *L, const LayerGeom &lg, const void *src, void *out, const char *tag) {
+  const SideGeom &g = lg.P;
+  const int64_t ldw = lg.ldn;
+  Gemm p;
+  p.tag = tag;
+  p.M = int(lg.m); p.N = g.size; p.K = g.size; p.batch = g.nprim; p.dtype = lg.dtype;
+  p.A = src; p.a_m = ldw; p.a_k = 1; p.a_b = g.size;
+  p.B = state_R(&L->P, g, lg.dtype); p.b_n = 1; p.b_k = g.ld; p.b_b = g.blk_elems();
+  p.outD = out; p.od_m = ldw; p.od_b = g.size;
+  return p;
+}
+poet_status right_tail(const LayerGeom &lg, const void *src, void *out, cudaStream_t st) {
+  if (lg.P.covered >= lg.n) return POET_OK;
+  const size_t es = esize(lg.dtype), row = size_t(lg.ldn) * es;
+  POET_CUDA_TRY(cudaMemcpy2DAsync(static_cast<char *>(out) + size_t(lg.P.covered) * es, row,
+                                  static_cast<const char *>(src) + size_t(lg.P.covered) * es, row,
+                                  size_t(lg.n - lg.P.covered) * es, size_t(lg.m), cudaMemcpyDeviceToDevice, st));
+  return POET_OK;
 }
 
 }  // namespace
@@ -255,22 +360,35 @@ size_t poet_frame_bytes(const poet_layer *L) {
   return align256(size_t(L->m) * frame_ld(L->n) * esize(L->dtype));
 }
 
+// Shapes only, so that sizes can be queried before the pointers exist.
+static bool shape_geom(const poet_layer *L, LayerGeom *lg) {
+  if (!L || L->m < 1 || L->n < 1 || L->m > 16384 || L->n > 16384) return false;
+  if (L->dtype != POET_F32 && L->dtype != POET_BF16) return false;
+  if (L->plan != POET_PLAN_AUTO && L->plan != POET_PLAN_TOKEN && L->plan != POET_PLAN_WEIGHT) return false;
+  if (!side_geom(&L->R, &lg->R) || !side_geom(&L->P, &lg->P)) return false;
+  lg->m = L->m; lg->n = L->n; lg->ldm = frame_ld(L->m); lg->ldn = frame_ld(L->n);
+  lg->dtype = L->dtype; lg->plan = L->plan;
+  return true;
+}
+
+int32_t poet_plan_for(const poet_layer *L, int64_t T) {
+  LayerGeom lg;
+  if (T < 0 || !shape_geom(L, &lg)) return -1;
+  return resolve_plan(lg, T);
+}
+
 size_t poet_saved_bytes(const poet_layer *L, int64_t T) {
-  if (!L || L->m < 1 || L->n < 1 || T < 0) return 0;
+  LayerGeom lg;
+  if (T < 0 || !shape_geom(L, &lg)) return 0;
+  if (resolve_plan(lg, T) == POET_PLAN_WEIGHT) return weight_saved(lg, T).bytes;
   const size_t es = esize(L->dtype);
-  return align256(size_t(T) * frame_ld(L->n) * es) + align256(size_t(T) * frame_ld(L->m) * es);
+  return align256(size_t(T) * lg.ldn * es) + align256(size_t(T) * lg.ldm * es);
 }
 
 size_t poet_workspace_bytes(const poet_layer *L, int64_t T) {
   LayerGeom lg;
-  if (T < 0 || check_layer(L, &lg, false) != POET_OK) {
-    clear_error();
-    // shape-only fallback so that sizes can be queried before pointers exist
-    if (!L || T < 0) return 0;
-    if (!side_geom(&L->R, &lg.R) || !side_geom(&L->P, &lg.P)) return 0;
-    lg.m = L->m; lg.n = L->n; lg.ldm = frame_ld(L->m); lg.ldn = frame_ld(L->n); lg.dtype = L->dtype;
-  }
-  return ws_layout(lg, T).bytes;
+  if (T < 0 || !shape_geom(L, &lg)) return 0;
+  return ws_layout(lg, T, resolve_plan(lg, T)).bytes;
 }
 
 size_t poet_side_workspace_bytes(const poet_side *side, int32_t dtype) {
@@ -311,6 +429,129 @@ poet_status poet_cayley_neumann_grad(const poet_side *side, int32_t dtype, const
   return cnp_backward(side, g, dtype, Gpad, dtheta, scratch, st);
 }
 
+// ------------------------------------------------------------------ weight plan
+
+// E_f = R W0f P in the frame (H = R W0f and F = W0f P kept for the backward),
+// then E = E_f in natural order.  Weight-sized work only.
+static poet_status weight_factors(const poet_layer *L, const LayerGeom &lg, char *sv, const WeightSaved &ly, void *Ef,
+                                  cudaStream_t st) {
+  const int dt = lg.dtype;
+  const void *W0f = L->W0f;
+  const void *Hs = W0f, *Es = W0f;
+  if (lg.R.nprim > 0) {
+    POET_TRY(gemm_run(left_blocks(L, lg, W0f, sv + ly.H, "w_prep"), st));
+    POET_TRY(left_tail(lg, W0f, sv + ly.H, st));
+    Hs = sv + ly.H;
+    Es = Hs;
+  }
+  if (lg.P.nprim > 0) {
+    Gemm two[2] = {right_blocks(L, lg, W0f, sv + ly.F, "w_prep"), right_blocks(L, lg, Hs, Ef, "w_prep")};
+    POET_TRY(gemm_run_many(two, 2, st));
+    POET_TRY(right_tail(lg, W0f, sv + ly.F, st));
+    POET_TRY(right_tail(lg, Hs, Ef, st));
+    Es = Ef;
+  }
+  // E[R.perm[i]][P.perm[j]] = E_f[i][j]
+  return scatter_cols(dt, Es, lg.ldn, Es, lg.ldn, int(lg.n), lg.m, int(lg.n), L->P.perm, sv + ly.E, lg.ldn,
+                      L->R.perm, st, "unframe");
+}
+
+static poet_status forward_weight(const poet_layer *L, const LayerGeom &lg, const void *x, int64_t T, void *y,
+                                  void *saved, char *wb, const WsLayout &w, cudaStream_t st) {
+  const int dt = lg.dtype;
+  char *sv = static_cast<char *>(saved);
+  const WeightSaved ly = weight_saved(lg, T);
+  POET_TRY(weight_factors(L, lg, sv, ly, wb + w.Z, st));
+  // x as a GEMM operand needs 16-byte aligned rows
+  const void *xa = x;
+  int64_t ldx = lg.n;
+  if (!rows16(x, lg.n, dt)) {
+    POET_TRY(copy_rows(dt, x, lg.n, T, int(lg.n), sv + ly.xp, lg.ldn, st));
+    xa = sv + ly.xp;
+    ldx = lg.ldn;
+  }
+  Gemm p;  // y = x E^T
+  p.tag = "w0_fwd";
+  p.M = int(T); p.N = int(lg.m); p.K = int(lg.n); p.dtype = dt;
+  p.A = xa; p.a_m = ldx; p.a_k = 1;
+  p.B = sv + ly.E; p.b_n = lg.ldn; p.b_k = 1;
+  p.outD = y; p.od_m = lg.m;
+  return gemm_run(p, st);
+}
+
+static poet_status backward_weight(const poet_layer *L, const LayerGeom &lg, char *wb, const WsLayout &w,
+                                   const void *x, const void *saved, const void *dy, int64_t T, void *dx, float *GR,
+                                   float *GP, cudaStream_t st) {
+  const int dt = lg.dtype;
+  const SideGeom &gR = lg.R, &gP = lg.P;
+  const char *sv = static_cast<const char *>(saved);
+  const WeightSaved ly = weight_saved(lg, T);
+  const void *xa = x;
+  int64_t ldx = lg.n;
+  if (!rows16(x, lg.n, dt)) { xa = sv + ly.xp; ldx = lg.ldn; }  // the forward's re-strided copy
+  const void *dya = dy;
+  int64_t ldy = lg.m;
+  if (!rows16(dy, lg.m, dt)) {
+    POET_TRY(copy_rows(dt, dy, lg.m, T, int(lg.m), wb + w.act1, lg.ldm, st));
+    dya = wb + w.act1;
+    ldy = lg.ldm;
+  }
+  {  // dx = dy E
+    Gemm p;
+    p.tag = "w0_bwd";
+    p.M = int(T); p.N = int(lg.n); p.K = int(lg.m); p.dtype = dt;
+    p.A = dya; p.a_m = ldy; p.a_k = 1;
+    p.B = sv + ly.E; p.b_n = 1; p.b_k = lg.ldn;
+    p.outD = dx; p.od_m = lg.n;
+    POET_TRY(gemm_run(p, st));
+  }
+  if (gR.nprim == 0 && gP.nprim == 0) return POET_OK;
+  // D = dy^T x (natural order, float, split over tokens)
+  float *D = reinterpret_cast<float *>(wb + w.D);
+  float *D2 = reinterpret_cast<float *>(wb + w.D2);
+  const size_t wsz = size_t(lg.m) * lg.ldn;
+  POET_CUDA_TRY(cudaMemsetAsync(D, 0, wsz * 4, st));
+  {
+    Gemm p;
+    p.tag = "w_grad";
+    p.M = int(lg.m); p.N = int(lg.n); p.K = int(T); p.dtype = dt;
+    p.A = dya; p.a_m = 1; p.a_k = ldy;
+    p.B = xa; p.b_n = 1; p.b_k = ldx;
+    p.outF = D; p.of_m = lg.ldn;
+    p.atomic = true;
+    POET_TRY(gemm_run(p, st));
+  }
+  // D_f[i][j] = D[R.perm[i]][P.perm[j]], in the element type of the GEMMs
+  POET_TRY(gather_cols(POET_F32, D, lg.ldn, L->R.perm, lg.m, int(lg.n), L->P.perm, D2, lg.ldn, nullptr, 0,
+                       int(lg.n), st, "frame"));
+  const void *Df = D2;
+  if (dt == POET_BF16) {
+    POET_TRY(f32_to_bf16(D2, wb + w.Z, int64_t(wsz), st));
+    Df = wb + w.Z;
+  }
+  const void *Fs = gP.nprim > 0 ? static_cast<const void *>(sv + ly.F) : L->W0f;
+  const void *Hs = gR.nprim > 0 ? static_cast<const void *>(sv + ly.H) : L->W0f;
+  Gemm g2[2];
+  int ng = 0;
+  if (gR.nprim > 0) {  // G_R[j] = D_f[rows j] F[rows j]^T
+    Gemm &p = g2[ng++];
+    p.tag = "blk_grad";
+    p.M = gR.size; p.N = gR.size; p.K = int(lg.n); p.batch = gR.nprim; p.dtype = dt;
+    p.A = Df; p.a_m = lg.ldn; p.a_k = 1; p.a_b = int64_t(gR.size) * lg.ldn;
+    p.B = Fs; p.b_n = lg.ldn; p.b_k = 1; p.b_b = int64_t(gR.size) * lg.ldn;
+    p.outF = GR; p.of_m = gR.ld; p.of_b = gR.blk_elems();
+  }
+  if (gP.nprim > 0) {  // G_P[j] = H[:, cols j]^T D_f[:, cols j]
+    Gemm &p = g2[ng++];
+    p.tag = "blk_grad";
+    p.M = gP.size; p.N = gP.size; p.K = int(lg.m); p.batch = gP.nprim; p.dtype = dt;
+    p.A = Hs; p.a_m = 1; p.a_k = lg.ldn; p.a_b = gP.size;
+    p.B = Df; p.b_n = 1; p.b_k = lg.ldn; p.b_b = gP.size;
+    p.outF = GP; p.of_m = gP.ld; p.of_b = gP.blk_elems();
+  }
+  return gemm_run_many(g2, ng, st);
+}
+
 poet_status poet_forward(const poet_layer *L, const void *x, int64_t T, void *y, void *saved, void *ws,
                          size_t ws_bytes, poet_stream stream) {
   clear_error();
@@ -320,12 +561,14 @@ poet_status poet_forward(const poet_layer *L, const void *x, int64_t T, void *y,
   if (T == 0) return POET_OK;
   POET_REQUIRE(x && y && aligned_elem(x, lg.dtype) && aligned_elem(y, lg.dtype), "poet_forward: x/y NULL or misaligned");
   POET_REQUIRE(saved && aligned256(saved), "poet_forward: saved NULL or not 256-byte aligned");
-  const WsLayout w = ws_layout(lg, T);
+  const int plan = resolve_plan(lg, T);
+  const WsLayout w = ws_layout(lg, T, plan);
   if (!ws || ws_bytes < w.bytes || !aligned256(ws)) {
     set_error("poet_forward: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, w.bytes);
     return POET_ENOMEM_WS;
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (plan == POET_PLAN_WEIGHT) return forward_weight(L, lg, x, T, y, saved, static_cast<char *>(ws), w, st);
   const int dt = lg.dtype;
   const size_t es = esize(dt);
   char *sv = static_cast<char *>(saved);
@@ -364,12 +607,18 @@ poet_status poet_forward(const poet_layer *L, const void *x, int64_t T, void *y,
   return scatter_cols(dt, ysrc, lg.ldm, vf, lg.ldm, gR.covered, T, int(lg.m), L->R.perm, y, lg.m, nullptr, st);
 }
 
-static poet_status backward_core(const poet_layer *L, const LayerGeom &lg, char *wb, const WsLayout &w,
-                                 const void *saved, const void *dy, int64_t T, void *dx, float *GR, float *GP,
-                                 cudaStream_t st) {
+static poet_status backward_core(const poet_layer *L, const LayerGeom &lg, int plan, char *wb, const WsLayout &w,
+                                 const void *x, const void *saved, const void *dy, int64_t T, void *dx, float *GR,
+                                 float *GP, cudaStream_t st) {
   const int dt = lg.dtype;
   const size_t es = esize(dt);
   const SideGeom &gR = lg.R, &gP = lg.P;
+  if (T > 0 && plan == POET_PLAN_WEIGHT) {
+    POET_REQUIRE(dy && dx && aligned_elem(dy, dt) && aligned_elem(dx, dt), "backward: dy/dx NULL or misaligned");
+    POET_REQUIRE(x && aligned_elem(x, dt), "backward: x NULL or misaligned (the weight plan reads x)");
+    POET_REQUIRE(saved && aligned256(saved), "backward: saved NULL or not 256-byte aligned");
+    return backward_weight(L, lg, wb, w, x, saved, dy, T, dx, GR, GP, st);
+  }
   if (T > 0) {
     POET_REQUIRE(dy && dx && aligned_elem(dy, dt) && aligned_elem(dx, dt), "backward: dy/dx NULL or misaligned");
     POET_REQUIRE(saved && aligned256(saved), "backward: saved NULL or not 256-byte aligned");
@@ -415,8 +664,8 @@ static poet_status backward_core(const poet_layer *L, const LayerGeom &lg, char 
   return POET_OK;
 }
 
-poet_status poet_backward(const poet_layer *L, const void *saved, const void *dy, int64_t T, void *dx,
-                          float *dtheta_R, float *dtheta_P, void *ws, size_t ws_bytes, poet_stream stream) {
+poet_status poet_backward(const poet_layer *L, const void *x, const void *saved, const void *dy, int64_t T,
+                          void *dx, float *dtheta_R, float *dtheta_P, void *ws, size_t ws_bytes, poet_stream stream) {
   clear_error();
   LayerGeom lg;
   POET_TRY(check_layer(L, &lg, true));
@@ -424,7 +673,8 @@ poet_status poet_backward(const poet_layer *L, const void *saved, const void *dy
   const SideGeom &gR = lg.R, &gP = lg.P;
   POET_REQUIRE(gR.nprim == 0 || gR.size < 2 || dtheta_R, "poet_backward: dtheta_R is NULL");
   POET_REQUIRE(gP.nprim == 0 || gP.size < 2 || dtheta_P, "poet_backward: dtheta_P is NULL");
-  const WsLayout w = ws_layout(lg, T);
+  const int plan = resolve_plan(lg, T);
+  const WsLayout w = ws_layout(lg, T, plan);
   if (!ws || ws_bytes < w.bytes || !aligned256(ws)) {
     set_error("poet_backward: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, w.bytes);
     return POET_ENOMEM_WS;
@@ -433,7 +683,7 @@ poet_status poet_backward(const poet_layer *L, const void *saved, const void *dy
   char *wb = static_cast<char *>(ws);
   float *GR = reinterpret_cast<float *>(wb + w.GR);
   float *GP = reinterpret_cast<float *>(wb + w.GP);
-  POET_TRY(backward_core(L, lg, wb, w, saved, dy, T, dx, GR, GP, st));
+  POET_TRY(backward_core(L, lg, plan, wb, w, x, saved, dy, T, dx, GR, GP, st));
   // a8: through the Cayley-Neumann map to the packed parameters
   void *scratch = wb + w.cnp;
   if (gR.nprim > 0 && gR.size >= 2) POET_TRY(cnp_backward(&L->R, gR, lg.dtype, GR, dtheta_R, scratch, st));
@@ -441,8 +691,8 @@ poet_status poet_backward(const poet_layer *L, const void *saved, const void *dy
   return POET_OK;
 }
 
-poet_status poet_backward_blocks(const poet_layer *L, const void *saved, const void *dy, int64_t T, void *dx,
-                                 float *G_R, float *G_P, void *ws, size_t ws_bytes, poet_stream stream) {
+poet_status poet_backward_blocks(const poet_layer *L, const void *x, const void *saved, const void *dy, int64_t T,
+                                 void *dx, float *G_R, float *G_P, void *ws, size_t ws_bytes, poet_stream stream) {
   clear_error();
   LayerGeom lg;
   POET_TRY(check_layer(L, &lg, true));
@@ -451,12 +701,13 @@ poet_status poet_backward_blocks(const poet_layer *L, const void *saved, const v
                "poet_backward_blocks: G_R NULL or not 16-byte aligned");
   POET_REQUIRE(lg.P.nprim == 0 || (G_P && (reinterpret_cast<uintptr_t>(G_P) & 15) == 0),
                "poet_backward_blocks: G_P NULL or not 16-byte aligned");
-  const WsLayout w = ws_layout(lg, T);
+  const int plan = resolve_plan(lg, T);
+  const WsLayout w = ws_layout(lg, T, plan);
   if (!ws || ws_bytes < w.bytes || !aligned256(ws)) {
     set_error("poet_backward_blocks: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, w.bytes);
     return POET_ENOMEM_WS;
   }
-  return backward_core(L, lg, static_cast<char *>(ws), w, saved, dy, T, dx, G_R, G_P,
+  return backward_core(L, lg, plan, static_cast<char *>(ws), w, x, saved, dy, T, dx, G_R, G_P,
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -551,7 +802,7 @@ poet_status poet_merge(poet_layer *L, void *ws, size_t ws_bytes, poet_stream str
   POET_TRY(check_layer(L, &lg, true));
   POET_REQUIRE(lg.R.nprim == 0 || lg.R.packed_per() == 0 || L->R.theta, "poet_merge: R.theta is NULL");
   POET_REQUIRE(lg.P.nprim == 0 || lg.P.packed_per() == 0 || L->P.theta, "poet_merge: P.theta is NULL");
-  const WsLayout w = ws_layout(lg, 0);
+  const WsLayout w = ws_layout(lg, 0, POET_PLAN_TOKEN);
   if (!ws || ws_bytes < w.bytes || !aligned256(ws)) {
     set_error("poet_merge: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, w.bytes);
     return POET_ENOMEM_WS;
@@ -564,39 +815,21 @@ poet_status poet_merge(poet_layer *L, void *ws, size_t ws_bytes, poet_stream str
   char *Z = static_cast<char *>(ws) + w.Z;
   const int64_t ldw = lg.ldn;
   if (gR.nprim > 0 || gP.nprim > 0) {
-    // Z = blockdiag(R) W0f  (rows of each R primitive; leftover rows copied)
+    // Z = blockdiag(R) W0f
     const char *src = W0f;
     if (gR.nprim > 0) {
-      Gemm p;
-      p.tag = "merge";
-      p.M = gR.size; p.N = int(lg.n); p.K = gR.size; p.batch = gR.nprim; p.dtype = dt;
-      p.A = state_R(&L->R, gR, dt); p.a_m = gR.ld; p.a_k = 1; p.a_b = gR.blk_elems();
-      p.B = W0f; p.b_n = 1; p.b_k = ldw; p.b_b = int64_t(gR.size) * ldw;
-      p.outD = Z; p.od_m = ldw; p.od_b = int64_t(gR.size) * ldw;
-      POET_TRY(gemm_run(p, st));
-      if (gR.covered < lg.m)
-        POET_CUDA_TRY(cudaMemcpyAsync(Z + size_t(gR.covered) * ldw * es, W0f + size_t(gR.covered) * ldw * es,
-                                      size_t(lg.m - gR.covered) * ldw * es, cudaMemcpyDeviceToDevice, st));
+      POET_TRY(gemm_run(left_blocks(L, lg, W0f, Z, "merge"), st));
+      POET_TRY(left_tail(lg, W0f, Z, st));
       src = Z;
     }
-    // W0f = src blockdiag(P)  (columns of each P primitive; leftover columns copied)
+    // W0f = src blockdiag(P)
     if (gP.nprim > 0) {
-      Gemm p;
-      p.tag = "merge";
-      p.M = int(lg.m); p.N = gP.size; p.K = gP.size; p.batch = gP.nprim; p.dtype = dt;
-      p.A = src; p.a_m = ldw; p.a_k = 1; p.a_b = gP.size;
-      p.B = state_R(&L->P, gP, dt); p.b_n = 1; p.b_k = gP.ld; p.b_b = gP.blk_elems();
-      p.outD = W0f; p.od_m = ldw; p.od_b = gP.size;
       if (src == W0f) {  // R had no primitives: the product cannot be written in place
         POET_CUDA_TRY(cudaMemcpyAsync(Z, W0f, size_t(lg.m) * ldw * es, cudaMemcpyDeviceToDevice, st));
-        p.A = Z;
         src = Z;
       }
-      POET_TRY(gemm_run(p, st));
-      if (gP.covered < lg.n)
-        POET_CUDA_TRY(cudaMemcpy2DAsync(W0f + size_t(gP.covered) * es, ldw * es, src + size_t(gP.covered) * es,
-                                        ldw * es, size_t(lg.n - gP.covered) * es, size_t(lg.m),
-                                        cudaMemcpyDeviceToDevice, st));
+      POET_TRY(gemm_run(right_blocks(L, lg, src, W0f, "merge"), st));
+      POET_TRY(right_tail(lg, src, W0f, st));
     } else {
       POET_CUDA_TRY(cudaMemcpyAsync(W0f, Z, size_t(lg.m) * ldw * es, cudaMemcpyDeviceToDevice, st));
     }

@@ -131,12 +131,20 @@ bool gemm_tc_enabled();
 poet_status gather_cols(int dtype, const void *src, int64_t ld_src, const int32_t *rowmap,
                         int64_t rows, int d, const int32_t *perm,
                         void *dst, int64_t ld_dst, void *dst2, int64_t ld_dst2, int split,
-                        cudaStream_t st);
+                        cudaStream_t st, const char *kind = "gather");
+
+// dst[r][j] = src[r][j] for j < d: rows re-strided to 16-byte aligned rows.
+poet_status copy_rows(int dtype, const void *src, int64_t ld_src, int64_t rows, int d, void *dst, int64_t ld_dst,
+                      cudaStream_t st);
+
+// out[e] = bf16(in[e]) for e < n.
+poet_status f32_to_bf16(const float *in, void *out, int64_t n, cudaStream_t st);
 
 // dst[dstrow(r)][perm[i]] = (i < split ? src1[r][i] : src2[r][i]); dstrow(r) = rowmap ? rowmap[r] : r.
 poet_status scatter_cols(int dtype, const void *src1, int64_t ld1, const void *src2, int64_t ld2,
                          int split, int64_t rows, int d, const int32_t *perm,
-                         void *dst, int64_t ld_dst, const int32_t *rowmap, cudaStream_t st);
+                         void *dst, int64_t ld_dst, const int32_t *rowmap, cudaStream_t st,
+                         const char *kind = "scatter");
 
 // ------------------------------------------------------------------ Cayley-Neumann
 

@@ -14,6 +14,7 @@ import torch
 
 F32, BF16 = 0, 1
 BS, FS = 0, 1
+PLAN_AUTO, PLAN_TOKEN, PLAN_WEIGHT = 0, 1, 2
 OK, EINVAL, ECUDA, ETIMEOUT, ENOMEM_WS = 0, 1, 2, 3, 4
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpoet.so")
@@ -33,7 +34,7 @@ class poet_side(ctypes.Structure):
 
 class poet_layer(ctypes.Structure):
     _fields_ = [("m", ctypes.c_int64), ("n", ctypes.c_int64), ("dtype", ctypes.c_int32),
-                ("layer_id", ctypes.c_int32), ("epoch", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("layer_id", ctypes.c_int32), ("epoch", ctypes.c_int32), ("plan", ctypes.c_int32),
                 ("seed", ctypes.c_uint64), ("W0", ctypes.c_void_p), ("W0f", ctypes.c_void_p),
                 ("R", poet_side), ("P", poet_side)]
 
@@ -46,6 +47,7 @@ class poet_trace_row(ctypes.Structure):
 _SIGS = {
     "poet_side_state_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_side), ctypes.c_int32]),
     "poet_frame_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_layer)]),
+    "poet_plan_for": (ctypes.c_int32, [ctypes.POINTER(poet_layer), ctypes.c_int64]),
     "poet_saved_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_layer), ctypes.c_int64]),
     "poet_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_layer), ctypes.c_int64]),
     "poet_side_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_side), ctypes.c_int32]),
@@ -56,9 +58,9 @@ _SIGS = {
                                                 ctypes.c_void_p]),
     "poet_forward": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
-    "poet_backward": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
-                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-                                     ctypes.c_size_t, ctypes.c_void_p]),
+    "poet_backward": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "poet_merge": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "poet_prepare": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p]),
     "poet_resample": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p]),
@@ -74,8 +76,8 @@ _SIGS = {
     "poet_cayley_neumann_many": (ctypes.c_int, [ctypes.POINTER(poet_side), ctypes.c_int32, ctypes.c_int32,
                                                 ctypes.c_void_p]),
     "poet_backward_blocks": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p, ctypes.c_void_p,
-                                            ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+                                            ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "poet_cayley_neumann_grad_many_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_side), ctypes.c_int32,
                                                                         ctypes.c_int32]),
     "poet_cayley_neumann_grad_many": (ctypes.c_int, [ctypes.POINTER(poet_side), ctypes.POINTER(ctypes.c_void_p),
@@ -148,6 +150,10 @@ def poet_frame_bytes(layer: poet_layer) -> int:
     return lib().poet_frame_bytes(ctypes.byref(layer))
 
 
+def poet_plan_for(layer: poet_layer, T: int) -> int:
+    return lib().poet_plan_for(ctypes.byref(layer), T)
+
+
 def poet_saved_bytes(layer: poet_layer, T: int) -> int:
     return lib().poet_saved_bytes(ctypes.byref(layer), T)
 
@@ -180,8 +186,8 @@ def poet_forward(layer: poet_layer, x, T: int, y, saved, ws, stream=None):
                               _stream(stream)))
 
 
-def poet_backward(layer: poet_layer, saved, dy, T: int, dx, dtheta_R, dtheta_P, ws, stream=None):
-    _check(lib().poet_backward(ctypes.byref(layer), _ptr(saved), _ptr(dy), T, _ptr(dx), _ptr(dtheta_R),
+def poet_backward(layer: poet_layer, x, saved, dy, T: int, dx, dtheta_R, dtheta_P, ws, stream=None):
+    _check(lib().poet_backward(ctypes.byref(layer), _ptr(x), _ptr(saved), _ptr(dy), T, _ptr(dx), _ptr(dtheta_R),
                                _ptr(dtheta_P), _ptr(ws), ws.numel(), _stream(stream)))
 
 
@@ -234,9 +240,9 @@ def poet_cayley_neumann_many(sides, dtype: int, stream=None):
     _check(lib().poet_cayley_neumann_many(_side_array(sides), len(sides), dtype, _stream(stream)))
 
 
-def poet_backward_blocks(layer: poet_layer, saved, dy, T: int, dx, G_R, G_P, ws, stream=None):
-    _check(lib().poet_backward_blocks(ctypes.byref(layer), _ptr(saved), _ptr(dy), T, _ptr(dx), _ptr(G_R), _ptr(G_P),
-                                      _ptr(ws), ws.numel(), _stream(stream)))
+def poet_backward_blocks(layer: poet_layer, x, saved, dy, T: int, dx, G_R, G_P, ws, stream=None):
+    _check(lib().poet_backward_blocks(ctypes.byref(layer), _ptr(x), _ptr(saved), _ptr(dy), T, _ptr(dx), _ptr(G_R),
+                                      _ptr(G_P), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def poet_cayley_neumann_grad_many_workspace_bytes(sides, dtype: int) -> int:
@@ -283,7 +289,7 @@ class PoetLayer:
     """
 
     def __init__(self, W0, theta_R, theta_P, *, mode, b, k, seed=0, layer_id=0, epoch=0,
-                 modeP=None, bP=None):
+                 modeP=None, bP=None, plan=PLAN_AUTO):
         if not W0.is_cuda:
             raise ValueError("W0 must be a CUDA tensor")
         self.dtype = BF16 if W0.dtype == torch.bfloat16 else F32
@@ -299,7 +305,7 @@ class PoetLayer:
         self.perm_R = torch.empty(self.m, dtype=torch.int32, device=dev)
         self.perm_P = torch.empty(self.n, dtype=torch.int32, device=dev)
         L = poet_layer()
-        L.m, L.n, L.dtype, L.layer_id, L.epoch, L.reserved, L.seed = self.m, self.n, self.dtype, layer_id, epoch, 0, seed
+        L.m, L.n, L.dtype, L.layer_id, L.epoch, L.plan, L.seed = self.m, self.n, self.dtype, layer_id, epoch, plan, seed
         L.R.dim, L.R.mode, L.R.b, L.R.k = self.m, mode, b, k
         L.P.dim, L.P.mode, L.P.b, L.P.k = self.n, modeP, bP, k
         self.state_R = torch.empty(max(poet_side_state_bytes(L.R, self.dtype), 1), dtype=torch.uint8, device=dev)
@@ -334,6 +340,10 @@ class PoetLayer:
                                       device=self.W0.device)
         return self._ws[T]
 
+    def plan_for(self, T: int) -> int:
+        """PLAN_TOKEN or PLAN_WEIGHT: the plan forward/backward run at T tokens."""
+        return poet_plan_for(self._L, T)
+
     def saved_buffer(self, T: int):
         return torch.empty(max(poet_saved_bytes(self._L, T), 1), dtype=torch.uint8, device=self.W0.device)
 
@@ -358,7 +368,8 @@ class PoetLayer:
         poet_forward(self._L, x, T, y, saved, self.workspace(T) if ws is None else ws, stream)
         return y, saved
 
-    def backward(self, saved, dy, dx=None, dtheta_R=None, dtheta_P=None, ws=None, stream=None):
+    def backward(self, saved, dy, dx=None, dtheta_R=None, dtheta_P=None, ws=None, stream=None, x=None):
+        """x: the forward's input (read by the weight plan)."""
         T = dy.shape[0]
         if dx is None:
             dx = torch.empty(T, self.n, dtype=dy.dtype, device=dy.device)
@@ -366,7 +377,7 @@ class PoetLayer:
             dtheta_R = torch.empty_like(self.theta_R)
         if dtheta_P is None:
             dtheta_P = torch.empty_like(self.theta_P)
-        poet_backward(self._L, saved, dy, T, dx, dtheta_R, dtheta_P, self.workspace(T) if ws is None else ws,
+        poet_backward(self._L, x, saved, dy, T, dx, dtheta_R, dtheta_P, self.workspace(T) if ws is None else ws,
                       stream)
         return dx, dtheta_R, dtheta_P
 
@@ -382,12 +393,13 @@ class PoetLayer:
         return (torch.empty(max(poet_block_grad_bytes(self._L.R) // 4, 4), dtype=torch.float32, device=dev),
                 torch.empty(max(poet_block_grad_bytes(self._L.P) // 4, 4), dtype=torch.float32, device=dev))
 
-    def backward_blocks(self, saved, dy, G_R, G_P, dx=None, ws=None, stream=None):
-        """a5..a7: dx and the per-primitive gradients (a8 left to cayley_neumann_grad_many)."""
+    def backward_blocks(self, saved, dy, G_R, G_P, dx=None, ws=None, stream=None, x=None):
+        """a5..a7: dx and the per-primitive gradients (a8 left to cayley_neumann_grad_many).
+        x: the forward's input (read by the weight plan)."""
         T = dy.shape[0]
         if dx is None:
             dx = torch.empty(T, self.n, dtype=dy.dtype, device=dy.device)
-        poet_backward_blocks(self._L, saved, dy, T, dx, G_R, G_P, self.workspace(T) if ws is None else ws, stream)
+        poet_backward_blocks(self._L, x, saved, dy, T, dx, G_R, G_P, self.workspace(T) if ws is None else ws, stream)
         return dx
 
 

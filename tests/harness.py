@@ -64,9 +64,9 @@ def run_oracle(case: Case, W0, thR, thP, x, dy):
     return out
 
 
-def run_gpu(case: Case, W0, thR, thP, x, dy, device="cuda"):
+def run_gpu(case: Case, W0, thR, thP, x, dy, device="cuda", plan=0):
     """prepare -> Cayley-Neumann -> forward -> backward -> merge -> resample ->
-    Cayley-Neumann -> forward, all through libpoet."""
+    Cayley-Neumann -> forward, all through libpoet (plan: poet.PLAN_*)."""
     import torch
     from orthogonal_reparameterized_poet_b200 import poet
 
@@ -74,15 +74,16 @@ def run_gpu(case: Case, W0, thR, thP, x, dy, device="cuda"):
     L = poet.PoetLayer(torch.from_numpy(W0).to(device=device, dtype=tdt),
                        torch.from_numpy(thR).to(device), torch.from_numpy(thP).to(device),
                        mode=case.modeR, b=case.bR, modeP=case.modeP, bP=case.bP, k=case.k,
-                       seed=case.seed, layer_id=case.layer_id, epoch=case.epoch)
+                       seed=case.seed, layer_id=case.layer_id, epoch=case.epoch, plan=plan)
     xt = torch.from_numpy(x).to(device=device, dtype=tdt)
     dyt = torch.from_numpy(dy).to(device=device, dtype=tdt)
     L.prepare()
     L.cayley_neumann()
     y, saved = L.forward(xt)
-    dx, dthR, dthP = L.backward(saved, dyt)
+    dx, dthR, dthP = L.backward(saved, dyt, x=xt)
     poet.poet_sync_status()
     res = {
+        "plan": L.plan_for(xt.shape[0]),
         "permR": L.perm_R.cpu().numpy(), "permP": L.perm_P.cpu().numpy(),
         "Y": y.float().cpu().numpy(), "dX": dx.float().cpu().numpy(),
         "dthetaR": dthR.cpu().numpy(), "dthetaP": dthP.cpu().numpy(),

@@ -63,8 +63,46 @@ def test_state_and_frame_sizes():
     assert poet.poet_side_state_bytes(_side(10, poet.BS, 2, 17), poet.BF16) == 0
     L = _layer(5461, 2048, poet.BS, 256, 4, poet.BF16)
     assert poet.poet_frame_bytes(L) == 5461 * 2048 * 2
+    L.plan = poet.PLAN_TOKEN  # frame copies of x (ld 2048) and of W0 P x (ld 5504)
     assert poet.poet_saved_bytes(L, 32768) == 32768 * 2048 * 2 + 32768 * 5504 * 2
     assert poet.poet_workspace_bytes(L, 32768) > poet.poet_workspace_bytes(L, 0) > 0
+    L.plan = poet.PLAN_WEIGHT  # E, F, H (m x ld 2048, 256-byte rounded) and a re-strided x
+    w = (5461 * 2048 * 2 + 255) // 256 * 256
+    assert poet.poet_saved_bytes(L, 32768) == 3 * w + 32768 * 2048 * 2
+    assert poet.poet_workspace_bytes(L, 32768) > poet.poet_workspace_bytes(L, 0) > 0
+
+
+@pytest.mark.parametrize("m,n,mode,b", [(2048, 2048, poet.BS, 256), (5461, 2048, poet.BS, 256),
+                                        (2048, 5461, poet.FS, 0), (2048, 2048, poet.FS, 0)])
+def test_auto_plan_follows_token_count(m, n, mode, b):
+    L = _layer(m, n, mode, b, 4, poet.BF16)
+    # many tokens per weight element: the primitives go on W0; few tokens: on the activations
+    assert poet.poet_plan_for(L, 32768) == poet.PLAN_WEIGHT
+    assert poet.poet_plan_for(L, 64) == poet.PLAN_TOKEN
+    assert poet.poet_plan_for(L, 0) == poet.PLAN_TOKEN
+    for forced in (poet.PLAN_TOKEN, poet.PLAN_WEIGHT):
+        L.plan = forced
+        assert poet.poet_plan_for(L, 32768) == forced and poet.poet_plan_for(L, 64) == forced
+    L.plan = 3
+    assert poet.poet_plan_for(L, 64) == -1
+    assert poet.poet_saved_bytes(L, 64) == 0 and poet.poet_workspace_bytes(L, 64) == 0
+
+
+def test_weight_plan_backward_requires_x():
+    lib = poet.lib()
+    st = ctypes.c_void_p(0)
+    L = _layer(256, 256, poet.BS, 32, 3, poet.BF16)
+    L.plan = poet.PLAN_WEIGHT
+    fake = 1 << 20  # 256-byte aligned, never dereferenced: validation fails first
+    L.W0, L.W0f = fake, fake
+    for sd in (L.R, L.P):
+        sd.perm, sd.theta, sd.state = fake, fake, fake
+    ws_bytes = poet.poet_workspace_bytes(L, 16)
+    args = (ctypes.c_void_p(fake), ctypes.c_void_p(fake), 16, ctypes.c_void_p(fake), ctypes.c_void_p(fake),
+            ctypes.c_void_p(fake), ctypes.c_void_p(fake), ws_bytes, st)
+    assert lib.poet_backward(ctypes.byref(L), None, *args) == poet.EINVAL
+    assert "x NULL" in lib.poet_last_error().decode()
+    assert lib.poet_backward_blocks(ctypes.byref(L), None, *args) == poet.EINVAL
 
 
 def test_host_validation_rejects_bad_arguments():

@@ -38,10 +38,13 @@ def cuda():
 
 
 CASES = [("llama1.3b_fs", 4), ("llama1.3b_fs", 6), ("llama1.3b_bs256", 4), ("llama1.3b_bs256", 6)]
+# auto: the plan bench.py runs at this size (the weight plan); token: the other one
+PLANS = {"auto": 0, "token": 1}
 
 
+@pytest.mark.parametrize("plan", list(PLANS))
 @pytest.mark.parametrize("name,linear", CASES)
-def test_fullsize_sampled_parity(cuda, name, linear):
+def test_fullsize_sampled_parity(cuda, name, linear, plan):
     from orthogonal_reparameterized_poet_b200 import poet
 
     wl = I.WORKLOADS[name]
@@ -60,14 +63,15 @@ def test_fullsize_sampled_parity(cuda, name, linear):
     # ---------------- CUDA path, bench launch configuration
     tdt = poet.torch_dtype(dt)
     L = poet.PoetLayer(cuda.from_numpy(W0).to("cuda", tdt), cuda.from_numpy(thR).cuda(), cuda.from_numpy(thP).cuda(),
-                       mode=wl.mode, b=wl.b, k=k, seed=wl.seed, layer_id=layer_id)
+                       mode=wl.mode, b=wl.b, k=k, seed=wl.seed, layer_id=layer_id, plan=PLANS[plan])
+    assert L.plan_for(T) == (poet.PLAN_WEIGHT if plan == "auto" else poet.PLAN_TOKEN)
     L.prepare()
     poet.cayley_neumann_many([L])
     xt = cuda.from_numpy(X).to("cuda", tdt)
     dyt = cuda.from_numpy(dY).to("cuda", tdt)
     y, saved = L.forward(xt)
     gR, gP = L.block_grad_buffers()
-    dx = L.backward_blocks(saved, dyt, gR, gP)
+    dx = L.backward_blocks(saved, dyt, gR, gP, x=xt)
     dthR, dthP = cuda.empty_like(L.theta_R), cuda.empty_like(L.theta_P)
     ws = cuda.empty(max(poet.cayley_neumann_grad_many_workspace_bytes([L]), 1), dtype=cuda.uint8, device="cuda")
     poet.cayley_neumann_grad_many([L], [(gR, gP)], [(dthR, dthP)], ws)

@@ -112,12 +112,17 @@ LAYER_CASES = {
 }
 
 
+PLANS = {"token": 1, "weight": 2}
+
+
+@pytest.mark.parametrize("plan", list(PLANS))
 @pytest.mark.parametrize("name", list(LAYER_CASES))
-def test_layer_parity(cuda, name):
+def test_layer_parity(cuda, name, plan):
     case = LAYER_CASES[name]
     arrs = case.arrays()
     ref = run_oracle(case, *arrs)
-    got = run_gpu(case, *arrs)
+    got = run_gpu(case, *arrs, plan=PLANS[plan])
+    assert got["plan"] == PLANS[plan]
     tol = TOL[case.dtype]
     assert np.array_equal(got["permR"], ref["permR"]) and np.array_equal(got["permP"], ref["permP"])
     if len(ref["R_blocks"]):
@@ -142,18 +147,19 @@ def test_layer_parity(cuda, name):
     assert rel_fro(got["Y_after_merge"], ref["Y"]) <= tol
 
 
-def test_zero_tokens(cuda):
+@pytest.mark.parametrize("plan", list(PLANS))
+def test_zero_tokens(cuda, plan):
     from orthogonal_reparameterized_poet_b200 import poet
 
     case = LAYER_CASES["ragged_bs_fp32"]
     W0, thR, thP, x, dy = case.arrays()
     L = poet.PoetLayer(cuda.from_numpy(W0).cuda(), cuda.from_numpy(thR).cuda(), cuda.from_numpy(thP).cuda(),
-                       mode=case.modeR, b=case.bR, k=case.k)
+                       mode=case.modeR, b=case.bR, k=case.k, plan=PLANS[plan])
     L.prepare()
     L.cayley_neumann()
     x0 = cuda.empty(0, case.n, device="cuda")
     y, saved = L.forward(x0)
-    dx, dthR, dthP = L.backward(saved, cuda.empty(0, case.m, device="cuda"))
+    dx, dthR, dthP = L.backward(saved, cuda.empty(0, case.m, device="cuda"), x=x0)
     poet.poet_sync_status()
     assert y.shape == (0, case.m) and dx.shape == (0, case.n)
     assert not dthR.any().item() and not dthP.any().item()
@@ -210,14 +216,14 @@ def test_gemm_engine(cuda, dtype, M, N, K, batch, amaj, bmaj, alpha, beta):
 
 # ------------------------------------------------------------------ many layers at once
 
-def _make_layer(cuda, case):
+def _make_layer(cuda, case, plan=0):
     from orthogonal_reparameterized_poet_b200 import poet
 
     W0, thR, thP, x, dy = case.arrays()
     tdt = poet.torch_dtype(case.dtype)
     L = poet.PoetLayer(cuda.from_numpy(W0).to("cuda", tdt), cuda.from_numpy(thR).cuda(), cuda.from_numpy(thP).cuda(),
                        mode=case.modeR, b=case.bR, modeP=case.modeP, bP=case.bP, k=case.k, seed=case.seed,
-                       layer_id=case.layer_id)
+                       layer_id=case.layer_id, plan=plan)
     L.prepare()
     return L, cuda.from_numpy(x).to("cuda", tdt), cuda.from_numpy(dy).to("cuda", tdt), (W0, thR, thP, x, dy)
 
@@ -241,12 +247,13 @@ MANY_SETS = {  # different sizes, modes and Neumann orders in one call
 MANY_VS_SINGLE = {"bf16": 5e-3, "f32": 1e-5}
 
 
+@pytest.mark.parametrize("plan", list(PLANS))
 @pytest.mark.parametrize("which", sorted(MANY_SETS))
-def test_many_sides_match_single_calls_and_oracle(cuda, which):
+def test_many_sides_match_single_calls_and_oracle(cuda, which, plan):
     from orthogonal_reparameterized_poet_b200 import poet
 
     MANY_CASES = MANY_SETS[which]
-    built = [_make_layer(cuda, c) for c in MANY_CASES]
+    built = [_make_layer(cuda, c, PLANS[plan]) for c in MANY_CASES]
     layers = [b[0] for b in built]
     # a1: grouped launch vs one call per side (same tiles, same order: bitwise equal)
     poet.cayley_neumann_many(layers)
@@ -261,10 +268,10 @@ def test_many_sides_match_single_calls_and_oracle(cuda, which):
     for (L, xt, dyt, arrs), case in zip(built, MANY_CASES):
         y, saved = L.forward(xt)
         gR, gP = L.block_grad_buffers()
-        dx = L.backward_blocks(saved, dyt, gR, gP)
+        dx = L.backward_blocks(saved, dyt, gR, gP, x=xt)
         G.append((gR, gP))
         dth.append((cuda.empty_like(L.theta_R), cuda.empty_like(L.theta_P)))
-        dx1, dR1, dP1 = L.backward(saved, dyt)
+        dx1, dR1, dP1 = L.backward(saved, dyt, x=xt)
         assert cuda.equal(dx, dx1)
         dth_ref.append((dR1, dP1))
     ws = cuda.empty(max(poet.cayley_neumann_grad_many_workspace_bytes(layers), 1), dtype=cuda.uint8, device="cuda")
