@@ -495,23 +495,38 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
           }
           __syncwarp();
           if (p.coalesced == 3) {
+            // one row per store instruction: lane l writes the 4-byte word
+            // holding elements e0 = 2l - mis and e0 + 1 (mis = 1 when the row
+            // segment starts 2 bytes past a 4-byte boundary; element 63 then
+            // goes separately).  Eight rows are read from shared memory before
+            // their stores are issued.
             const int nv = min(64, p.N - gn0);
-            const int rows = min(32, p.M - m_base);
-            for (int rr = 0; rr < rows; ++rr) {
-              const bf16 *srow = reinterpret_cast<const bf16 *>(ew + rr * S::EPI_ROW);
-              bf16 *o = obase + int64_t(m_base + rr) * p.od_m + gn0;
-              const int mis = int((reinterpret_cast<uintptr_t>(o) >> 1) & 1);  // o is 2 mod 4
-              const int e0 = 2 * lane - mis;  // lane's word covers elements e0, e0 + 1
-              if (e0 >= 0 && e0 + 1 < nv) {
-                __nv_bfloat162 h;
-                h.x = srow[e0];
-                h.y = srow[e0 + 1];
-                *reinterpret_cast<__nv_bfloat162 *>(o + e0) = h;
-              } else {
-                if (e0 >= 0 && e0 < nv) o[e0] = srow[e0];
-                if (e0 + 1 >= 0 && e0 + 1 < nv) o[e0 + 1] = srow[e0 + 1];
+            uint16_t *orow0 = reinterpret_cast<uint16_t *>(obase + int64_t(m_base) * p.od_m + gn0);
+            for (int r0 = 0; r0 < 32 && m_base + r0 < p.M; r0 += 8) {
+              uint32_t val[8];
+              uint16_t last[8];
+              int mis[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const uint16_t *srow = reinterpret_cast<const uint16_t *>(ew + (r0 + j) * S::EPI_ROW);
+                mis[j] = int((reinterpret_cast<uintptr_t>(orow0 + int64_t(r0 + j) * p.od_m) >> 1) & 1);
+                const int e0 = 2 * lane - mis[j];  // >= -1; e0 + 1 <= 63
+                val[j] = uint32_t(srow[e0 < 0 ? 0 : e0]) | (uint32_t(srow[e0 + 1]) << 16);
+                last[j] = srow[63];
               }
-              if (mis && lane == 0 && 63 < nv) o[63] = srow[63];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                if (m_base + r0 + j >= p.M) break;  // the same for the whole warp
+                uint16_t *o = orow0 + int64_t(r0 + j) * p.od_m;
+                const int e0 = 2 * lane - mis[j];
+                if (e0 >= 0 && e0 + 1 < nv) {
+                  *reinterpret_cast<uint32_t *>(o + e0) = val[j];
+                } else {
+                  if (e0 >= 0 && e0 < nv) o[e0] = uint16_t(val[j]);
+                  if (e0 + 1 < nv) o[e0 + 1] = uint16_t(val[j] >> 16);
+                }
+                if (mis[j] && lane == 0 && 63 < nv) o[63] = last[j];
+              }
             }
             continue;
           }
@@ -871,7 +886,19 @@ bool gemm_tc_supported(const Gemm &g) {
   return true;
 }
 
-poet_status gemm_tc(const Gemm &g, cudaStream_t st) { return run_group<1>(&g, 1, plan_of(g), st); }
+// A launch whose 128 x 256 tiles would not give every SM one tile and that
+// has no split-K output runs 128 x 128 tiles instead (twice as many CTAs).
+int64_t wide_tiles(const Gemm &g) {
+  return int64_t((g.M + BM - 1) / BM) * ((g.N + 255) / 256) * g.batch;
+}
+TcPlan narrowed(TcPlan t, int64_t tiles, bool any_atomic) {
+  if (t.BN == 256 && !t.bstat && !any_atomic && tiles < num_sms()) t.BN = 128;
+  return t;
+}
+
+poet_status gemm_tc(const Gemm &g, cudaStream_t st) {
+  return run_group<1>(&g, 1, narrowed(plan_of(g), wide_tiles(g), g.atomic), st);
+}
 
 // Runs many independent problems: tensor-core problems that share operand
 // majors and tile width go into grouped launches of up to kGroupMax problems
@@ -896,8 +923,15 @@ poet_status gemm_tc_many(const Gemm *gs, int count, cudaStream_t st) {
     const std::vector<Gemm> &v = buckets[b];
     for (size_t i = 0; i < v.size(); i += kGroupMax) {
       const int n = int(v.size() - i < size_t(kGroupMax) ? v.size() - i : size_t(kGroupMax));
-      if (n == 1) POET_TRY(run_group<1>(v.data() + i, 1, plans[b], st));
-      else POET_TRY(run_group<kGroupMax>(v.data() + i, n, plans[b], st));
+      int64_t tiles = 0;
+      bool any_atomic = false;
+      for (int j = 0; j < n; ++j) {
+        tiles += wide_tiles(v[i + j]);
+        any_atomic |= v[i + j].atomic;
+      }
+      const TcPlan t = narrowed(plans[b], tiles, any_atomic);
+      if (n == 1) POET_TRY(run_group<1>(v.data() + i, 1, t, st));
+      else POET_TRY(run_group<kGroupMax>(v.data() + i, n, t, st));
     }
   }
   return POET_OK;

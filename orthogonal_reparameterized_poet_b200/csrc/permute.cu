@@ -258,6 +258,27 @@ __global__ void __launch_bounds__(256) restride_kernel(const unsigned char *__re
   }
 }
 
+// out[a][c] = bf16(D[rowmap[a]][perm[c]]): a float matrix gathered into the
+// frame and rounded in one pass.  One block per output row at a time; the
+// source row is read through L1 (it is reused by the block's gathers).
+__global__ void __launch_bounds__(256) frame_f32_to_bf16_kernel(const float *__restrict__ D, int64_t ldD,
+                                                                const int32_t *__restrict__ rowmap, int64_t rows,
+                                                                int d, const int32_t *__restrict__ perm,
+                                                                bf16 *__restrict__ out, int64_t ld_out) {
+  for (int64_t a = blockIdx.x; a < rows; a += gridDim.x) {
+    const float *src = D + int64_t(__ldg(rowmap + a)) * ldD;
+    bf16 *orow = out + a * ld_out;
+    for (int c = 2 * threadIdx.x; c < d; c += 2 * blockDim.x) {
+      if (c + 1 < d) {
+        const int2 pc = *reinterpret_cast<const int2 *>(perm + c);
+        *reinterpret_cast<__nv_bfloat162 *>(orow + c) = __floats2bfloat162_rn(__ldg(src + pc.x), __ldg(src + pc.y));
+      } else {
+        orow[c] = __float2bfloat16_rn(__ldg(src + perm[c]));
+      }
+    }
+  }
+}
+
 template <typename T>
 poet_status launch_permute(PermArgs<T> a, cudaStream_t st, const char *kind) {
   if (a.rows <= 0 || a.d <= 0) return POET_OK;
@@ -310,6 +331,20 @@ poet_status gather_cols(int dtype, const void *src, int64_t ld_src, const int32_
     return launch_permute<T>(a, st, kind);
   };
   return dtype == POET_BF16 ? fill(static_cast<bf16 *>(nullptr)) : fill(static_cast<float *>(nullptr));
+}
+
+poet_status frame_f32_to_bf16(const float *D, int64_t ldD, const int32_t *rowmap, int64_t rows, int d,
+                              const int32_t *perm, void *out, int64_t ld_out, cudaStream_t st) {
+  POET_REQUIRE((reinterpret_cast<uintptr_t>(out) & 3) == 0 && ld_out % 2 == 0 &&
+                   (reinterpret_cast<uintptr_t>(perm) & 7) == 0,
+               "frame: output rows must be 4-byte aligned and perm 8-byte aligned");
+  if (rows <= 0 || d <= 0) return POET_OK;
+  TraceScope ts("frame", 0.0, double(rows) * d * 6.0, st);
+  const int64_t cap = int64_t(num_sms()) * 8;
+  const int grid = int(rows < cap ? rows : cap);
+  frame_f32_to_bf16_kernel<<<grid, 256, 0, st>>>(D, ldD, rowmap, rows, d, perm, static_cast<bf16 *>(out), ld_out);
+  count_launch();
+  return launch_status("frame");
 }
 
 poet_status copy_rows(int dtype, const void *src, int64_t ld_src, int64_t rows, int d, void *dst, int64_t ld_dst,

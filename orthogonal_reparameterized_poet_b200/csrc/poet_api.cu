@@ -179,8 +179,9 @@ struct WsLayout {
 };
 
 // token plan: act1..act3 activation frames;  weight plan: act1 = re-strided
-// dy, D / D2 = float m x ldn (D and its framed copy).  Both: GR, GP, the
-// Cayley-Neumann scratch and Z (m x ldn, merge and the weight plan's E_f).
+// dy, D = float m x ldn, D2 = its framed copy (float layers; bf16 layers frame
+// D into Z).  Both: GR, GP, the Cayley-Neumann scratch and Z (m x ldn: merge,
+// the weight plan's E_f and framed D).
 WsLayout ws_layout(const LayerGeom &lg, int64_t T, int plan) {
   WsLayout w;
   const size_t es = esize(lg.dtype);
@@ -202,7 +203,7 @@ WsLayout ws_layout(const LayerGeom &lg, int64_t T, int plan) {
   w.Z = off; off += align256(wsz * es);
   if (plan == POET_PLAN_WEIGHT) {
     w.D = off; off += align256(wsz * 4);
-    w.D2 = off; off += align256(wsz * 4);
+    if (lg.dtype == POET_F32) { w.D2 = off; off += align256(wsz * 4); }  // bf16 frames D into Z
   }
   w.bytes = off;
   return w;
@@ -347,7 +348,7 @@ extern "C" {
 const char *poet_last_error(void) { return g_last_error; }
 
 // The kernel revisions name the code that profiles/ counters were taken on.
-const char *poet_version(void) { return "libpoet 0.2 (sm_100a; gemm_tc r5; permute r3)"; }
+const char *poet_version(void) { return "libpoet 0.3 (sm_100a; gemm_tc r6; permute r3; restride r1)"; }
 
 size_t poet_side_state_bytes(const poet_side *side, int32_t dtype) {
   SideGeom g;
@@ -522,17 +523,22 @@ static poet_status backward_weight(const poet_layer *L, const LayerGeom &lg, cha
     POET_TRY(gemm_run(p, st));
   }
   // D_f[i][j] = D[R.perm[i]][P.perm[j]], in the element type of the GEMMs
-  POET_TRY(gather_cols(POET_F32, D, lg.ldn, L->R.perm, lg.m, int(lg.n), L->P.perm, D2, lg.ldn, nullptr, 0,
-                       int(lg.n), st, "frame"));
-  const void *Df = D2;
+  const void *Df;
   if (dt == POET_BF16) {
-    POET_TRY(f32_to_bf16(D2, wb + w.Z, int64_t(wsz), st));
+    POET_TRY(frame_f32_to_bf16(D, lg.ldn, L->R.perm, lg.m, int(lg.n), L->P.perm, wb + w.Z, lg.ldn, st));
     Df = wb + w.Z;
+  } else {
+    POET_TRY(gather_cols(POET_F32, D, lg.ldn, L->R.perm, lg.m, int(lg.n), L->P.perm, D2, lg.ldn, nullptr, 0,
+                         int(lg.n), st, "frame"));
+    Df = D2;
   }
   const void *Fs = gP.nprim > 0 ? static_cast<const void *>(sv + ly.F) : L->W0f;
   const void *Hs = gR.nprim > 0 ? static_cast<const void *>(sv + ly.H) : L->W0f;
+  // the per-primitive products are small (K = n or m): split over K, summed in place
   Gemm g2[2];
   int ng = 0;
+  if (gR.nprim > 0) POET_CUDA_TRY(cudaMemsetAsync(GR, 0, size_t(gR.all_elems()) * 4, st));
+  if (gP.nprim > 0) POET_CUDA_TRY(cudaMemsetAsync(GP, 0, size_t(gP.all_elems()) * 4, st));
   if (gR.nprim > 0) {  // G_R[j] = D_f[rows j] F[rows j]^T
     Gemm &p = g2[ng++];
     p.tag = "blk_grad";
@@ -540,6 +546,7 @@ static poet_status backward_weight(const poet_layer *L, const LayerGeom &lg, cha
     p.A = Df; p.a_m = lg.ldn; p.a_k = 1; p.a_b = int64_t(gR.size) * lg.ldn;
     p.B = Fs; p.b_n = lg.ldn; p.b_k = 1; p.b_b = int64_t(gR.size) * lg.ldn;
     p.outF = GR; p.of_m = gR.ld; p.of_b = gR.blk_elems();
+    p.atomic = true;
   }
   if (gP.nprim > 0) {  // G_P[j] = H[:, cols j]^T D_f[:, cols j]
     Gemm &p = g2[ng++];
@@ -548,6 +555,7 @@ static poet_status backward_weight(const poet_layer *L, const LayerGeom &lg, cha
     p.A = Hs; p.a_m = 1; p.a_k = lg.ldn; p.a_b = gP.size;
     p.B = Df; p.b_n = 1; p.b_k = lg.ldn; p.b_b = gP.size;
     p.outF = GP; p.of_m = gP.ld; p.of_b = gP.blk_elems();
+    p.atomic = true;
   }
   return gemm_run_many(g2, ng, st);
 }

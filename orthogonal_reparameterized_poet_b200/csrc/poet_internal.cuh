@@ -137,6 +137,10 @@ poet_status gather_cols(int dtype, const void *src, int64_t ld_src, const int32_
 poet_status copy_rows(int dtype, const void *src, int64_t ld_src, int64_t rows, int d, void *dst, int64_t ld_dst,
                       cudaStream_t st);
 
+// out[a][c] = bf16(D[rowmap[a]][perm[c]]) for a < rows, c < d (out: bf16).
+poet_status frame_f32_to_bf16(const float *D, int64_t ldD, const int32_t *rowmap, int64_t rows, int d,
+                              const int32_t *perm, void *out, int64_t ld_out, cudaStream_t st);
+
 // out[e] = bf16(in[e]) for e < n.
 poet_status f32_to_bf16(const float *in, void *out, int64_t n, cudaStream_t st);
 
