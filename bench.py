@@ -59,6 +59,8 @@ def parse_args():
     ap.add_argument("--no-merge", action="store_true")
     ap.add_argument("--plan", choices=sorted(PLANS), default="auto",
                     help="where the primitives act: auto (cost model), token (activations) or weight (W0)")
+    ap.add_argument("--no-token-plan", action="store_true",
+                    help="skip the second timed pass that runs every layer on the token plan")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (small profiling cases)")
     return ap.parse_args()
 
@@ -203,6 +205,24 @@ class Variant:
         self.ws = None
         self.input_bytes = sum(v.numel() * v.element_size() for v in list(self.x.values()) + list(self.dy.values()))
 
+    def use_plan(self, plan, saved_pool, device):
+        """Run every layer on `plan` from now on; grow the shared saved buffers to fit."""
+        import torch
+
+        from orthogonal_reparameterized_poet_b200 import poet
+
+        for i, (_, _, _, _, L) in enumerate(self.layers):
+            L.struct.plan = plan
+            need = poet.poet_saved_bytes(L.struct, self.T)
+            if saved_pool[i].numel() < need:
+                saved_pool[i] = None
+                saved_pool[i] = torch.empty(need, dtype=torch.uint8, device=device)
+            self.saved[i] = saved_pool[i]
+        self.ws_need = max(max(L.workspace_bytes(self.T), L.workspace_bytes(0)) for (_, _, _, _, L) in self.layers)
+
+    def plan_names(self):
+        return "+".join(sorted({PLAN_NAMES[L.plan_for(self.T)] for (_, _, _, _, L) in self.layers}))
+
     def alloc_grads(self, device, chunk):
         """Per-primitive gradient buffers of every side (one flat buffer) and the
         workspace of the grouped Cayley-Neumann backward over `chunk` layers."""
@@ -247,6 +267,26 @@ class Variant:
         for (_, _, _, _, L) in self.layers:
             L.merge(ws=self.ws)
             L.resample()
+
+
+def kernel_table(rows, steps):
+    """Per trace kind: launches, ms per step, share, and the fraction of the
+    roofline that bounds it (tensor when its flop/byte is above the ridge of
+    the measured peaks, HBM otherwise)."""
+    peaks = load_peaks()
+    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    total = sum(x["ms"] for x in rows.values()) or 1.0
+    out = {}
+    for k, r in sorted(rows.items(), key=lambda kv: -kv[1]["ms"]):
+        sec = r["ms"] / 1e3
+        tf = r["flop"] / sec / 1e12 if sec and r["flop"] else None
+        gb = r["bytes"] / sec / 1e9 if sec else None
+        tensor = r["flop"] and r["bytes"] and r["flop"] / r["bytes"] >= ridge
+        frac = (tf / peaks["bf16_tflops_sustained"]) if tensor else (gb / peaks["hbm_gbs"] if gb else None)
+        out[k] = {"launches": r["launches"], "ms_per_step": round(r["ms"] / steps, 3), "share": round(r["ms"] / total, 4),
+                  "tflops": round(tf, 1) if tf else None, "gbs": round(gb, 1) if gb else None,
+                  "bound": "tensor" if tensor else "hbm", "frac": round(frac, 4) if frac is not None else None}
+    return out
 
 
 def run_poet(args):
@@ -304,48 +344,80 @@ def run_poet(args):
     stream = torch.cuda.current_stream()
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     smi_index = vis.split(",")[local] if vis else str(local)
-    clocks = ClockSampler(smi_index)
-    # each variant runs its K steps back to back; the kernel trace is read per variant
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in variants]
-    barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    poet.poet_trace_enable(True)
-    launches0 = poet.poet_launch_count()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    traces = []
-    for i, v in enumerate(variants):
-        ev[i][0].record(stream)
-        for _ in range(args.steps):
-            v.step(world)
-        ev[i][1].record(stream)
-        traces.append(poet.poet_trace_read())  # waits for this variant's recorded events
-    t1.record(stream)
-    torch.cuda.synchronize()
-    per_variant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(len(variants))]
-    launches = poet.poet_launch_count() - launches0
-    poet.poet_trace_enable(False)
-    clk = clocks.stop()
-    barrier()
-    elapsed = t0.elapsed_time(t1)
-    trace = {}
-    for tr in traces:
-        for k, r in tr.items():
-            a = trace.setdefault(k, {"launches": 0, "ms": 0.0, "flop": 0.0, "bytes": 0.0})
-            for f in a:
-                a[f] += r[f]
-    poet.poet_sync_status()
-    if dist is not None:
-        from orthogonal_reparameterized_poet_b200 import dp
 
-        mx = dp.max_over_ranks([elapsed] + per_variant_ms, device=device)
-        elapsed, per_variant_ms = mx[0], mx[1:]
+    def timed(steps, clocks=None):
+        """K steps of every variant back to back, the kernel trace read per variant.
+        Returns (elapsed ms, per-variant ms, merged trace, per-variant traces, launches)."""
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in variants]
+        barrier()
+        torch.cuda.synchronize()
+        if clocks:
+            clocks.start()
+        poet.poet_trace_enable(True)
+        launches0 = poet.poet_launch_count()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        traces = []
+        for i, v in enumerate(variants):
+            ev[i][0].record(stream)
+            for _ in range(steps):
+                v.step(world)
+            ev[i][1].record(stream)
+            traces.append(poet.poet_trace_read())  # waits for this variant's recorded events
+        t1.record(stream)
+        torch.cuda.synchronize()
+        per_variant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(len(variants))]
+        launches = poet.poet_launch_count() - launches0
+        poet.poet_trace_enable(False)
+        clk = clocks.stop() if clocks else None
+        barrier()
+        elapsed = t0.elapsed_time(t1)
+        trace = {}
+        for tr in traces:
+            for k, r in tr.items():
+                a = trace.setdefault(k, {"launches": 0, "ms": 0.0, "flop": 0.0, "bytes": 0.0})
+                for f in a:
+                    a[f] += r[f]
+        poet.poet_sync_status()
+        if dist is not None:
+            from orthogonal_reparameterized_poet_b200 import dp
+
+            mx = dp.max_over_ranks([elapsed] + per_variant_ms, device=device)
+            elapsed, per_variant_ms = mx[0], mx[1:]
+        return elapsed, per_variant_ms, trace, traces, launches, clk
+
+    elapsed, per_variant_ms, trace, traces, launches, clk = timed(args.steps, ClockSampler(smi_index))
+    plans_run = [v.plan_names() for v in variants]
 
     tokens_per_step = sum(v.T for v in variants) * world
     ms_per_step = elapsed / args.steps
     value = tokens_per_step / (ms_per_step / 1e3)
+
+    # ---- the same steps with every layer on the token plan (primitives on the
+    # activations): the block contractions and permutations the cost model
+    # replaced, measured against their own rooflines
+    token = None
+    if not args.no_token_plan and any(p != "token" for p in plans_run):
+        for v in variants:
+            v.use_plan(1, saved_pool, device)
+        need = max(v.ws_need for v in variants)
+        if ws.numel() < need:
+            ws = None
+            ws = torch.empty(need, dtype=torch.uint8, device=device)
+        for v in variants:
+            v.ws = ws
+        for _ in range(max(1, min(args.warmup, 2))):
+            step()
+        t_el, t_pv, t_trace, t_traces, _, _ = timed(args.steps)
+        token = {"ms_per_step": round(t_el / args.steps, 3),
+                 "tokens_per_s": round(sum(v.T for v in variants) * world / (t_el / args.steps / 1e3), 1),
+                 "variants": {v.wl.name: round(t_pv[i] / args.steps, 3) for i, v in enumerate(variants)},
+                 "kernels": None}
+        t_kernels = kernel_table(t_trace, args.steps)
+        token["kernels"] = t_kernels
+        for v in variants:
+            v.use_plan(PLANS[args.plan], saved_pool, device)
 
     # ---- merge-then-reinitialize (timed once, amortized over the merge period)
     merge = {}
@@ -396,12 +468,7 @@ def run_poet(args):
                          "flop": r["flop"] / r["launches"], "bytes": r["bytes"] / r["launches"]},
                      "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one gate-shape launch "
                                        "(profiles/w0_gemm_llama1.3b_gate_T32768.md), scaled by algorithmic bytes"})
-    kernels = {}
-    for k, r in sorted(rows.items(), key=lambda kv: -kv[1]["ms"]):
-        kernels[k] = {"launches": r["launches"], "ms_per_step": round(r["ms"] / args.steps, 3),
-                      "share": round(r["ms"] / sum(x["ms"] for x in rows.values()), 4),
-                      "tflops": round(r["flop"] / (r["ms"] / 1e3) / 1e12, 1) if r["ms"] and r["flop"] else None,
-                      "gbs": round(r["bytes"] / (r["ms"] / 1e3) / 1e9, 1) if r["ms"] else None}
+    kernels = kernel_table(rows, args.steps)
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
@@ -416,9 +483,7 @@ def run_poet(args):
                    "hidden": wls[0].hidden, "ffn": wls[0].ffn, "layers": wls[0].layers,
                    "linears_per_layer": len(wls[0].linear_shapes()), "tokens_per_variant": wls[0].tokens,
                    "variants": [{"name": v.wl.name, "mode": "FS" if v.wl.mode == I.FS else "BS", "b": v.wl.b,
-                                 "k": v.wl.k, "plan": "+".join(sorted({PLAN_NAMES[L.plan_for(v.T)]
-                                                                       for (_, _, _, _, L) in v.layers}))}
-                                for v in variants],
+                                 "k": v.wl.k, "plan": plans_run[i]} for i, v in enumerate(variants)],
                    "plan_requested": args.plan,
                    "parallelism": f"dp{world}", "l2": "inputs larger than L2 (no flush needed)"},
         "variants": {v.wl.name: {"ms_per_step": round(per_variant_ms[i] / args.steps, 3),
@@ -430,7 +495,7 @@ def run_poet(args):
         "value_merge_amortized": (round(tokens_per_step / ((ms_per_step + sum(merge.values()) / 400.0) / 1e3), 1)
                                   if merge else None),
         "roofline": roof, "kernels": kernels, "gpu_launches": int(launches), "clocks": clk,
-        "e2e": e2e, "cpu_baseline": cpu,
+        "e2e": e2e, "cpu_baseline": cpu, "token_plan": token,
     }
     print(json.dumps(out), flush=True)
     if dist is not None:
