@@ -43,7 +43,10 @@ PLAN_NAMES = {1: "token", 2: "weight"}
 
 # DRAM traffic / algorithmic bytes of one launch, from an ncu capture, with the
 # kernel revision (as named in poet_version()) the counters were taken on.
-NCU_TRAFFIC_RATIO = {"w0_fwd": (0.920, "gemm_tc r3"), "w0_bwd": (0.979, "gemm_tc r3")}
+NCU_TRAFFIC_RATIO = {"w0_fwd": (0.901, "gemm_tc r6"), "w0_bwd": (0.917, "gemm_tc r6"), "w_grad": (1.830, "gemm_tc r6")}
+NCU_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of every launch of one LLaMA-1.3B layer "
+                      "(profiles/weight_plan_llama1.3b_layer_T32768.md), as a ratio to the algorithmic bytes of the "
+                      "same launches, scaled to this run's launches")
 
 
 def parse_args():
@@ -414,8 +417,7 @@ def run_poet(args):
                  "tokens_per_s": round(sum(v.T for v in variants) * world / (t_el / args.steps / 1e3), 1),
                  "variants": {v.wl.name: round(t_pv[i] / args.steps, 3) for i, v in enumerate(variants)},
                  "kernels": None}
-        t_kernels = kernel_table(t_trace, args.steps)
-        token["kernels"] = t_kernels
+        token["kernels"] = {v.wl.name: kernel_table(t_traces[i], args.steps) for i, v in enumerate(variants)}
         for v in variants:
             v.use_plan(PLANS[args.plan], saved_pool, device)
 
@@ -466,8 +468,7 @@ def run_poet(args):
                      "frac": round(achieved / peak, 4), "traffic": traffic, "avg_launch_ms": round(avg_ms, 4),
                      "launches": r["launches"], "algorithmic_per_launch": {
                          "flop": r["flop"] / r["launches"], "bytes": r["bytes"] / r["launches"]},
-                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one gate-shape launch "
-                                       "(profiles/w0_gemm_llama1.3b_gate_T32768.md), scaled by algorithmic bytes"})
+                     "traffic_source": NCU_TRAFFIC_SOURCE})
     kernels = kernel_table(rows, args.steps)
 
     cpu = None

@@ -20,6 +20,7 @@
 // word, stops, drains what it issued (bounded too), frees TMEM and returns.
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 #include <vector>
 
@@ -43,6 +44,7 @@ struct TcProblem {
   bf16 *outD; int64_t od_m, od_b;
   int atomic;
   int coalesced;  // plain bf16 output, 16-byte aligned rows: stores staged through shared memory
+  int m_fast;     // tile order: M tiles fastest (N > M: CTAs of a wave share B slabs)
 };
 
 // A launch: up to MAXP independent problems sharing operand majors and tile
@@ -156,6 +158,78 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
                : "memory");
 }
 
+// ---- CTA pairs (cta_group::2): two CTAs of a cluster share one 256-row MMA.
+// The pair's MMAs are issued by rank 0; each CTA loads its half of A (128
+// rows) and of B (half the N columns) and holds its 128 accumulator rows.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// address of the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on an
+// mbarrier of either CTA of the pair (no multicast)
+__device__ __forceinline__ void tma_load_3d_pair(void *dst, const CUtensorMap *map, uint32_t bar_cluster, int c0,
+                                                 int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive on the mbarrier at this offset in both CTAs of the pair once the pair's MMAs so far are done
+__device__ __forceinline__ void umma_commit_pair_both(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(uint16_t(3))
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -184,11 +258,11 @@ __device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint
   return d;
 }
 
-// Instruction descriptor, kind::f16: D f32, A and B bf16, M = 128, N = BN.
-template <bool A_MN, bool B_MN, int BN>
+// Instruction descriptor, kind::f16: D f32, A and B bf16, M = MM, N = BN.
+template <bool A_MN, bool B_MN, int BN, int MM = BM>
 __device__ __forceinline__ uint32_t make_idesc() {
   return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(A_MN) << 15) | (uint32_t(B_MN) << 16) |
-         (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+         (uint32_t(BN >> 3) << 17) | (uint32_t(MM >> 4) << 24);
 }
 
 struct TileCoord {
@@ -205,10 +279,17 @@ __device__ __forceinline__ TileCoord decode(int64_t tile, const TcGroup<MAXP> &g
   c.pi = lo;
   const TcProblem &p = g.prob[lo];
   int64_t t = tile - g.tile_start[lo];
-  c.nt = int(t % p.num_n);
-  t /= p.num_n;
-  c.mt = int(t % p.num_m);
-  t /= p.num_m;
+  if (p.m_fast) {
+    c.mt = int(t % p.num_m);
+    t /= p.num_m;
+    c.nt = int(t % p.num_n);
+    t /= p.num_n;
+  } else {
+    c.nt = int(t % p.num_n);
+    t /= p.num_n;
+    c.mt = int(t % p.num_m);
+    t /= p.num_m;
+  }
   c.s = int(t % p.splits);
   c.b = int(t / p.splits);
   return c;
@@ -219,12 +300,12 @@ __device__ __forceinline__ TileCoord decode(int64_t tile, const TcGroup<MAXP> &g
 // B operand of the current (problem, batch) stays resident (KB_MAX slabs) and
 // only A slabs stream through the ring.
 constexpr int KB_MAX = 4;  // B-stationary: K <= 256
-template <int BN, bool BSTAT = false>
+template <int BN, bool BSTAT = false, int CG = 1>
 struct Smem {
-  static constexpr int A_BYTES = BM * BK * 2;   // 16 KB
-  static constexpr int B_BYTES = BN * BK * 2;   // 32 KB (BN = 256)
+  static constexpr int A_BYTES = BM * BK * 2;          // 16 KB
+  static constexpr int B_BYTES = (BN / CG) * BK * 2;   // 32 KB (BN = 256), 16 KB per CTA of a pair
   static constexpr int STAGE_BYTES = BSTAT ? A_BYTES : A_BYTES + B_BYTES;
-  static constexpr int STAGES = BSTAT ? 4 : (BN == 256 ? 4 : 6);
+  static constexpr int STAGES = BSTAT ? 4 : (CG == 2 ? 6 : (BN == 256 ? 4 : 6));
   static constexpr int BRES_BYTES = BSTAT ? KB_MAX * B_BYTES : 0;  // resident B
   // epilogue staging: per epilogue warp 32 rows x 128 B (one 64-column bf16
   // chunk), rows padded to 144 B so row-wise writes and line-wise reads both
@@ -243,9 +324,10 @@ __device__ __forceinline__ void red_add_v4(float *out, float a, float b, float c
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(out), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
-template <bool A_MN, bool B_MN, int BN, int MAXP, bool BSTAT>
+template <bool A_MN, bool B_MN, int BN, int MAXP, bool BSTAT, int CG>
 __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_constant__ TcGroup<MAXP> g) {
-  using S = Smem<BN, BSTAT>;
+  static_assert(CG == 1 || (CG == 2 && BN == 256 && !BSTAT), "CTA pairs run 256 x 256 streaming tiles");
+  using S = Smem<BN, BSTAT, CG>;
   constexpr int STAGES = S::STAGES;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -265,11 +347,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t tiles = g.tile_start[g.count];
-  // Tiles of this CTA: strided over the grid (streaming), or one contiguous
-  // range (B-stationary, so that consecutive tiles share their B operand).
-  const int64_t per_cta = (tiles + gridDim.x - 1) / gridDim.x;
-  const int64_t t_first = BSTAT ? int64_t(blockIdx.x) * per_cta : int64_t(blockIdx.x);
-  const int64_t t_step = BSTAT ? 1 : int64_t(gridDim.x);
+  // CTA pairs: rank 0 issues the pair's MMAs; rank r holds rows r*128.. of each 256-row tile
+  const uint32_t rank = CG == 2 ? cluster_rank() : 0;
+  const bool leader = rank == 0;
+  const int64_t units = CG == 2 ? int64_t(cluster_count()) : int64_t(gridDim.x);
+  const int64_t unit = CG == 2 ? int64_t(cluster_id()) : int64_t(blockIdx.x);
+  // Tiles of this CTA (pair): strided over the grid (streaming), or one
+  // contiguous range (B-stationary, so that consecutive tiles share their B operand).
+  const int64_t per_cta = (tiles + units - 1) / units;
+  const int64_t t_first = BSTAT ? unit * per_cta : unit;
+  const int64_t t_step = BSTAT ? 1 : units;
   const int64_t t_end = BSTAT ? (t_first + per_cta < tiles ? t_first + per_cta : tiles) : tiles;
 
   if (threadIdx.x == 0) {
@@ -279,7 +366,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], 4 * CG);  // the epilogue warps of every CTA of the pair
     }
     mbar_init(drain, 1);
     mbar_init(bfull, 1);
@@ -287,12 +374,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, S::TMEM_COLS);
-    tmem_relinquish();
+  if (warp == 1) {  // a pair allocates collectively (the same warp of both CTAs)
+    if constexpr (CG == 2) {
+      tmem_alloc_pair(tmem_slot, S::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, S::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) cluster_sync_all();  // barriers initialised in both CTAs before any remote use
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -307,6 +400,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       int res_pi = -1, res_b = -1;   // B-stationary: operand currently resident
       uint32_t bfree_phase = 0;
       uint32_t bloads = 0;
+      const uint32_t full0 = CG == 2 ? mapa_shared(smem_u32(full), 0) : 0;  // rank 0's full[0]
       for (int64_t tile = t_first; tile < t_end && !*abort; tile += t_step) {
         const TileCoord c = decode(tile, g);
         const TcProblem &p = g.prob[c.pi];
@@ -344,6 +438,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
           if (!mbar_wait(&empty[stage], phase ^ 1, abort, g.errword)) break;
           unsigned char *sa = stage_base + size_t(stage) * S::STAGE_BYTES;
           unsigned char *sb = sa + S::A_BYTES;
+          if constexpr (CG == 2) {
+            // both halves land on rank 0's full barrier, which expects the pair's bytes
+            if (leader) mbar_expect_tx(&full[stage], 2 * S::STAGE_BYTES);
+            const uint32_t fb = full0 + uint32_t(stage) * 8u;
+            const int row0 = c.mt * (2 * BM) + int(rank) * BM;
+            const int col0 = c.nt * BN + int(rank) * (BN / 2);
+            if (!A_MN) {
+              tma_load_3d_pair(sa, ma, fb, kb * BK, row0, c.b);
+            } else {
+#pragma unroll
+              for (int q = 0; q < BM / 64; ++q) tma_load_3d_pair(sa + q * 8192, ma, fb, row0 + 64 * q, kb * BK, c.b);
+            }
+            if (!B_MN) {
+              tma_load_3d_pair(sb, mb, fb, kb * BK, col0, c.b);
+            } else {
+#pragma unroll
+              for (int q = 0; q < BN / 128; ++q) tma_load_3d_pair(sb + q * 8192, mb, fb, col0 + 64 * q, kb * BK, c.b);
+            }
+          } else {
           mbar_expect_tx(&full[stage], S::STAGE_BYTES);
           if (!A_MN) {
             tma_load_3d(sa, ma, &full[stage], kb * BK, c.mt * BM, c.b);
@@ -359,6 +472,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
               for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * 8192, mb, &full[stage], c.nt * BN + 64 * q, kb * BK, c.b);
             }
           }
+          }
           last_stage = stage;
           last_phase = phase;
           if (++stage == STAGES) {
@@ -368,9 +482,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
         }
       }
       if (*abort && last_stage >= 0) {
-        // drain: the most recent copies (bounded)
-        volatile int no_abort = 0;
-        mbar_wait(&full[last_stage], last_phase, &no_abort, nullptr);
+        if (CG == 1 || leader) {
+          // drain: the most recent copies (bounded)
+          volatile int no_abort = 0;
+          mbar_wait(&full[last_stage], last_phase, &no_abort, nullptr);
+        } else {
+          // the second CTA of a pair cannot wait on rank 0's barrier: give its
+          // copies in flight a fixed 200 us to land
+          const uint64_t t0 = globaltimer();
+          while (globaltimer() - t0 < 200000ull) {
+          }
+        }
       }
       if (BSTAT && *abort && bloads > 0) {
         volatile int no_abort = 0;
@@ -378,9 +500,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && (CG == 1 || leader)) {
       // ---------------------------------------------------------- MMA issuer
-      const uint32_t idesc = make_idesc<A_MN, B_MN, BN>();
+      const uint32_t idesc = make_idesc<A_MN, B_MN, BN, BM * CG>();
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -414,9 +536,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = A_MN ? make_desc(sa + kk * 2048, 8192, 1024) : make_desc(sa + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? make_desc(sb + kk * 2048, 8192, 1024) : make_desc(sb + kk * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+            if constexpr (CG == 2) umma_bf16_pair(d_tmem, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+            else umma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(&empty[stage]);
+          if constexpr (CG == 2) umma_commit_pair_both(&empty[stage]);
+          else umma_commit(&empty[stage]);
           issued = true;
           if (++stage == STAGES) {
             stage = 0;
@@ -424,7 +548,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        if constexpr (CG == 2) umma_commit_pair_both(&tfull[acc]);
+        else umma_commit(&tfull[acc]);
         if constexpr (BSTAT) {
           // the resident B is released after the last tile that reads it
           bool last_use = tile + t_step >= t_end;
@@ -441,7 +566,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       }
       if (*abort && issued) {
         // drain: every MMA issued so far has completed once this commit arrives
-        umma_commit(drain);
+        if constexpr (CG == 2) umma_commit_pair(drain);
+        else umma_commit(drain);
         volatile int no_abort = 0;
         mbar_wait(drain, 0, &no_abort, nullptr);
       }
@@ -457,7 +583,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       const TcProblem &p = g.prob[c.pi];
       if (!mbar_wait(&tfull[acc], acc_phase, abort, g.errword)) break;
       tc_fence_after();
-      const int gm = c.mt * BM + row;
+      const int mrow0 = c.mt * (BM * CG) + int(rank) * BM;  // this CTA's first accumulator row
+      const int gm = mrow0 + row;
       const bool row_ok = gm < p.M;
       const float alpha = p.alpha, beta = p.beta, diag = p.diag;
       if (p.coalesced == 1 || p.coalesced == 3) {
@@ -466,7 +593,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
         // rows x 128 contiguous bytes (mode 1), or, for rows that are not
         // 16-byte aligned (mode 3), one row x 128 bytes in 4-byte words
         unsigned char *ew = epi + quarter * (32 * S::EPI_ROW);
-        const int m_base = c.mt * BM + quarter * 32;
+        const int m_base = mrow0 + quarter * 32;
         bf16 *obase = p.outD + int64_t(c.b) * p.od_b;
         const int sub = lane & 7, rsub = lane >> 3;
         for (int cc = 0; cc < BN / 64; ++cc) {
@@ -552,7 +679,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
         // plain fp32 output: each 32-column chunk (128 B per row) goes row-wise
         // into this warp's staging rows, then out four rows x 128 B at a time
         unsigned char *ew = epi + quarter * (32 * S::EPI_ROW);
-        const int m_base = c.mt * BM + quarter * 32;
+        const int m_base = mrow0 + quarter * 32;
         float *obase = p.outF + int64_t(c.b) * p.of_b;
         const int sub = lane & 7, rsub = lane >> 3;
         unsigned char *myrow = ew + lane * S::EPI_ROW;
@@ -672,7 +799,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {  // the accumulator is released on the CTA that issues the MMAs
+        if constexpr (CG == 2) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[acc]), 0));
+        else mbar_arrive(&tempty[acc]);
+      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -681,10 +811,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
   }
 
   tc_fence_before();
-  __syncthreads();
+  // a pair frees its TMEM together, after every MMA of the pair has completed
+  // and both CTAs' epilogues have read their accumulators
+  if constexpr (CG == 2) cluster_sync_all();
+  else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, S::TMEM_COLS);
+    if constexpr (CG == 2) tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
+    else tmem_dealloc(tmem_base, S::TMEM_COLS);
   }
 }
 
@@ -738,13 +872,24 @@ bool make_map(CUtensorMap *map, const void *base, int64_t inner, int64_t outer, 
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// CTA pairs: POET_GEMM_PAIRS=0 turns them off (the single-CTA engine serves
+// every shape), =2 uses them for every streaming launch with problems at least
+// 256 rows tall (tests cover the pair engine at small sizes this way).
+const int g_pairs_mode = [] {
+  const char *e = std::getenv("POET_GEMM_PAIRS");
+  if (e && e[0] == '0') return 0;
+  if (e && e[0] == '2') return 2;
+  return 1;
+}();
+
 // Operand majors and tile width of a supported problem.
 struct TcPlan {
   bool A_MN, B_MN;
   int BN;
   bool bstat;  // B-stationary (whole B of a batch resident; contiguous tiles per CTA)
+  int cg = 1;  // CTAs per MMA: 2 = CTA pairs on 256 x 256 tiles
   bool operator==(const TcPlan &o) const {
-    return A_MN == o.A_MN && B_MN == o.B_MN && BN == o.BN && bstat == o.bstat;
+    return A_MN == o.A_MN && B_MN == o.B_MN && BN == o.BN && bstat == o.bstat && cg == o.cg;
   }
 };
 TcPlan plan_of(const Gemm &g) {
@@ -762,7 +907,7 @@ TcPlan plan_of(const Gemm &g) {
 // Fill one problem of a group (tiles use split-K only for atomic outputs).
 bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, CUtensorMap *ma, CUtensorMap *mb) {
   p->M = g.M; p->N = g.N; p->K = g.K; p->batch = g.batch;
-  p->num_m = (g.M + BM - 1) / BM;
+  p->num_m = (g.M + BM * t.cg - 1) / (BM * t.cg);
   p->num_n = (g.N + t.BN - 1) / t.BN;
   p->nk = (g.K + BK - 1) / BK;
   int splits = g.atomic ? (split_want < p->nk ? split_want : p->nk) : 1;
@@ -774,6 +919,9 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   p->outF = g.outF; p->of_m = g.of_m; p->of_b = g.of_b;
   p->outD = static_cast<bf16 *>(g.outD); p->od_m = g.od_m; p->od_b = g.od_b;
   p->atomic = g.atomic ? 1 : 0;
+  // consecutive tiles (one wave of persistent CTAs) share the slabs of the
+  // larger operand, which is then read from HBM about once
+  p->m_fast = g.N > g.M ? 1 : 0;
   // staged epilogue for a single plain output (1: bf16, 16-byte aligned rows;
   // 3: bf16, any rows; 2: fp32, 16-byte aligned rows); the per-row path
   // handles addends, pairs of outputs and split-K reductions
@@ -787,17 +935,18 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   if (!t.A_MN) ok = make_map(ma, g.A, g.K, g.M, g.batch, g.a_m, g.a_b, 64, BM);
   else ok = make_map(ma, g.A, g.M, g.K, g.batch, g.a_k, g.a_b, 64, 64);
   if (ok) {
-    if (!t.B_MN) ok = make_map(mb, g.B, g.K, g.N, g.batch, g.b_n, g.b_b, 64, t.BN);
+    if (!t.B_MN) ok = make_map(mb, g.B, g.K, g.N, g.batch, g.b_n, g.b_b, 64, t.BN / t.cg);
     else ok = make_map(mb, g.B, g.N, g.K, g.batch, g.b_k, g.b_b, 64, 64);
   }
   return ok;
 }
 
-template <bool A_MN, bool B_MN, int BN, int MAXP, bool BSTAT = false>
+template <bool A_MN, bool B_MN, int BN, int MAXP, bool BSTAT = false, int CG = 1>
 poet_status launch(const TcGroup<MAXP> &grp, cudaStream_t st) {
-  using S = Smem<BN, BSTAT>;
-  auto kern = gemm_tc_kernel<A_MN, B_MN, BN, MAXP, BSTAT>;
+  using S = Smem<BN, BSTAT, CG>;
+  auto kern = gemm_tc_kernel<A_MN, B_MN, BN, MAXP, BSTAT, CG>;
   static bool configured[64] = {};
+  static int max_pairs[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
@@ -805,8 +954,34 @@ poet_status launch(const TcGroup<MAXP> &grp, cudaStream_t st) {
     configured[dev] = true;
   }
   const int64_t tiles = grp.tile_start[grp.count];
-  const int64_t grid = tiles < num_sms() ? tiles : num_sms();
-  kern<<<int(grid), NTHREADS, S::BYTES, st>>>(grp);
+  if constexpr (CG == 1) {
+    const int64_t grid = tiles < num_sms() ? tiles : num_sms();
+    kern<<<int(grid), NTHREADS, S::BYTES, st>>>(grp);
+  } else {
+    // persistent CTA pairs: one cluster of two CTAs per pair of SMs, as many
+    // as can be resident at once
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = S::BYTES;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (dev < 64 && max_pairs[dev] == 0) {
+      cfg.gridDim = dim3(2 * (num_sms() / 2));
+      int n = 0;
+      POET_CUDA_TRY(cudaOccupancyMaxActiveClusters(&n, kern, &cfg));
+      max_pairs[dev] = n > 0 ? n : num_sms() / 2;
+    }
+    const int64_t cap = dev < 64 ? max_pairs[dev] : num_sms() / 2;
+    const int64_t pairs = tiles < cap ? tiles : cap;
+    cfg.gridDim = dim3(unsigned(2 * pairs));
+    POET_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, grp));
+  }
   count_launch();
   return launch_status("gemm_tc");
 }
@@ -816,7 +991,7 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
   static thread_local TcGroup<MAXP> grp;  // large: keep it off the stack
   int64_t base_tiles = 0;
   for (int i = 0; i < n; ++i) {
-    const int64_t mt = (gs[i].M + BM - 1) / BM, nt = (gs[i].N + t.BN - 1) / t.BN;
+    const int64_t mt = (gs[i].M + BM * t.cg - 1) / (BM * t.cg), nt = (gs[i].N + t.BN - 1) / t.BN;
     base_tiles += mt * nt * gs[i].batch;
   }
   // Split K (atomic outputs only) into s parts, s chosen so that the tiles
@@ -826,7 +1001,7 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
   bool any_atomic = false;
   for (int i = 0; i < n; ++i) any_atomic |= gs[i].atomic;
   if (any_atomic && base_tiles > 0) {
-    const int64_t sms = num_sms();
+    const int64_t sms = num_sms() / t.cg;  // concurrent tile workers: CTAs or CTA pairs
     double best = 0.0;
     for (int sp = 1; sp <= 16; ++sp) {
       const int64_t tiles = base_tiles * sp;
@@ -859,6 +1034,12 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
     if (!t.A_MN && t.B_MN) return launch<false, true, 128, MAXP>(grp, st);
     if (t.A_MN && !t.B_MN) return launch<true, false, 128, MAXP>(grp, st);
     return launch<true, true, 128, MAXP>(grp, st);
+  }
+  if (t.cg == 2) {
+    if (!t.A_MN && !t.B_MN) return launch<false, false, 256, MAXP, false, 2>(grp, st);
+    if (!t.A_MN && t.B_MN) return launch<false, true, 256, MAXP, false, 2>(grp, st);
+    if (t.A_MN && !t.B_MN) return launch<true, false, 256, MAXP, false, 2>(grp, st);
+    return launch<true, true, 256, MAXP, false, 2>(grp, st);
   }
   if (!t.A_MN && !t.B_MN) return launch<false, false, 256, MAXP>(grp, st);
   if (!t.A_MN && t.B_MN) return launch<false, true, 256, MAXP>(grp, st);
@@ -896,8 +1077,22 @@ TcPlan narrowed(TcPlan t, int64_t tiles, bool any_atomic) {
   return t;
 }
 
+// Large streaming launches run on CTA pairs (256 x 256 tiles, each CTA loading
+// half of B): every problem at least 512 rows tall and enough pair tiles for
+// every pair of SMs.
+TcPlan paired(TcPlan t, const Gemm *gs, int n) {
+  if (t.BN != 256 || t.bstat || g_pairs_mode == 0) return t;
+  int64_t pair_tiles = 0;
+  for (int i = 0; i < n; ++i) {
+    if (gs[i].M < (g_pairs_mode == 2 ? 256 : 512)) return t;
+    pair_tiles += int64_t((gs[i].M + 2 * BM - 1) / (2 * BM)) * ((gs[i].N + 255) / 256) * gs[i].batch;
+  }
+  if (g_pairs_mode == 2 || pair_tiles >= num_sms() / 2) t.cg = 2;
+  return t;
+}
+
 poet_status gemm_tc(const Gemm &g, cudaStream_t st) {
-  return run_group<1>(&g, 1, narrowed(plan_of(g), wide_tiles(g), g.atomic), st);
+  return run_group<1>(&g, 1, paired(narrowed(plan_of(g), wide_tiles(g), g.atomic), &g, 1), st);
 }
 
 // Runs many independent problems: tensor-core problems that share operand
@@ -929,7 +1124,7 @@ poet_status gemm_tc_many(const Gemm *gs, int count, cudaStream_t st) {
         tiles += wide_tiles(v[i + j]);
         any_atomic |= v[i + j].atomic;
       }
-      const TcPlan t = narrowed(plans[b], tiles, any_atomic);
+      const TcPlan t = paired(narrowed(plans[b], tiles, any_atomic), v.data() + i, n);
       if (n == 1) POET_TRY(run_group<1>(v.data() + i, 1, t, st));
       else POET_TRY(run_group<kGroupMax>(v.data() + i, n, t, st));
     }
