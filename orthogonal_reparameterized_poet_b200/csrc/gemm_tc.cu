@@ -307,10 +307,11 @@ struct Smem {
   static constexpr int STAGE_BYTES = BSTAT ? A_BYTES : A_BYTES + B_BYTES;
   static constexpr int STAGES = BSTAT ? 4 : (CG == 2 ? 6 : (BN == 256 ? 4 : 6));
   static constexpr int BRES_BYTES = BSTAT ? KB_MAX * B_BYTES : 0;  // resident B
-  // epilogue staging: per epilogue warp 32 rows x 128 B (one 64-column bf16
-  // chunk), rows padded to 144 B so row-wise writes and line-wise reads both
-  // take the minimum number of shared-memory wavefronts
-  static constexpr int EPI_ROW = 144;
+  // epilogue staging: per epilogue warp 32 rows of one 64-column bf16 chunk
+  // (plus up to 16 elements of shift and carry for rows that are not 16-byte
+  // aligned), rows 176 B apart (11 16-byte units) so row-wise writes and
+  // line-wise reads both take the minimum number of shared-memory wavefronts
+  static constexpr int EPI_ROW = 176;
   static constexpr int EPI_BYTES = 4 * 32 * EPI_ROW;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr size_t BYTES =
@@ -590,12 +591,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       if (p.coalesced == 1 || p.coalesced == 3) {
         // plain bf16 output: each 64-column chunk goes row-wise into this warp's
         // staging rows, then out with every store instruction covering four
-        // rows x 128 contiguous bytes (mode 1), or, for rows that are not
-        // 16-byte aligned (mode 3), one row x 128 bytes in 4-byte words
+        // rows x 128 contiguous bytes.
+        // Mode 3 (rows not 16-byte aligned): a row's chunk is staged shifted by
+        // the row's misalignment q (elements mod 8 of the tile's first column),
+        // so that the 16-byte units of the output row are 16-byte units of the
+        // staging row; the last q columns of a chunk carry over to the front of
+        // the next one.  Units then go out exactly as in mode 1, and only the
+        // first 8 - q and last q columns of a tile row (16-byte units shared
+        // with the neighbouring tiles) are written as single elements.
         unsigned char *ew = epi + quarter * (32 * S::EPI_ROW);
         const int m_base = mrow0 + quarter * 32;
         bf16 *obase = p.outD + int64_t(c.b) * p.od_b;
         const int sub = lane & 7, rsub = lane >> 3;
+        const int nt0 = c.nt * BN;
+        const bool mis_rows = p.coalesced == 3;
+        const bool my_row_ok = m_base + lane < p.M;
+        uint16_t *myout = reinterpret_cast<uint16_t *>(obase + int64_t(m_base + lane) * p.od_m + nt0);
+        const int qrow = mis_rows ? int((reinterpret_cast<uintptr_t>(myout) >> 1) & 7) : 0;
         for (int cc = 0; cc < BN / 64; ++cc) {
           uint32_t r0[32], r1[32];
           __syncwarp();
@@ -603,9 +615,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
           tmem_ld32(taddr, r0);
           tmem_ld32(taddr + 32, r1);
           tmem_ld_wait();
-          const int gn0 = c.nt * BN + cc * 64;
+          const int gn0 = nt0 + cc * 64;
           if (gn0 >= p.N) continue;  // the same for the whole warp
           unsigned char *myrow = ew + lane * S::EPI_ROW;
+          uint16_t *row16 = reinterpret_cast<uint16_t *>(myrow);
+          if (mis_rows && cc > 0) *reinterpret_cast<uint4 *>(myrow + 16) = *reinterpret_cast<const uint4 *>(myrow + 144);
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const uint32_t *src = q < 4 ? r0 + 8 * q : r1 + 8 * (q - 4);
@@ -618,41 +632,48 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
             pk.y = *reinterpret_cast<uint32_t *>(&h1);
             pk.z = *reinterpret_cast<uint32_t *>(&h2);
             pk.w = *reinterpret_cast<uint32_t *>(&h3);
-            *reinterpret_cast<uint4 *>(myrow + q * 16) = pk;
+            if (!mis_rows) {
+              *reinterpret_cast<uint4 *>(myrow + q * 16) = pk;
+            } else {  // elements 8 + qrow + 8q ... (2-byte aligned)
+              uint16_t *d = row16 + 8 + qrow + 8 * q;
+              d[0] = uint16_t(pk.x); d[1] = uint16_t(pk.x >> 16);
+              d[2] = uint16_t(pk.y); d[3] = uint16_t(pk.y >> 16);
+              d[4] = uint16_t(pk.z); d[5] = uint16_t(pk.z >> 16);
+              d[6] = uint16_t(pk.w); d[7] = uint16_t(pk.w >> 16);
+            }
+          }
+          if (mis_rows && cc == 0 && qrow > 0 && my_row_ok) {
+            // head: columns [0, 8 - q) end the 16-byte unit the previous tile begins
+            for (int e = 0; e < 8 - qrow; ++e)
+              if (nt0 + e < p.N) myout[e] = row16[8 + qrow + e];
           }
           __syncwarp();
-          if (p.coalesced == 3) {
-            // one row per store instruction: lane l writes the 4-byte word
-            // holding elements e0 = 2l - mis and e0 + 1 (mis = 1 when the row
-            // segment starts 2 bytes past a 4-byte boundary; element 63 then
-            // goes separately).  Eight rows are read from shared memory before
-            // their stores are issued.
-            const int nv = min(64, p.N - gn0);
-            uint16_t *orow0 = reinterpret_cast<uint16_t *>(obase + int64_t(m_base) * p.od_m + gn0);
-            for (int r0 = 0; r0 < 32 && m_base + r0 < p.M; r0 += 8) {
-              uint32_t val[8];
-              uint16_t last[8];
-              int mis[8];
+          if (mis_rows) {
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const uint16_t *srow = reinterpret_cast<const uint16_t *>(ew + (r0 + j) * S::EPI_ROW);
-                mis[j] = int((reinterpret_cast<uintptr_t>(orow0 + int64_t(r0 + j) * p.od_m) >> 1) & 1);
-                const int e0 = 2 * lane - mis[j];  // >= -1; e0 + 1 <= 63
-                val[j] = uint32_t(srow[e0 < 0 ? 0 : e0]) | (uint32_t(srow[e0 + 1]) << 16);
-                last[j] = srow[63];
+            for (int it = 0; it < 8; ++it) {
+              const int rr = it * 4 + rsub;
+              const int gm = m_base + rr;
+              if (gm >= p.M) continue;
+              uint16_t *orow = reinterpret_cast<uint16_t *>(obase + int64_t(gm) * p.od_m + nt0);
+              const int qr = int((reinterpret_cast<uintptr_t>(orow) >> 1) & 7);
+              if (cc == 0 && qr > 0 && sub == 0) continue;  // the head, written above
+              const int col = cc * 64 - qr + 8 * sub;        // tile column of this 16-byte unit
+              if (nt0 + col >= p.N) continue;
+              const uint4 v = *reinterpret_cast<const uint4 *>(ew + rr * S::EPI_ROW + 16 + sub * 16);
+              if (nt0 + col + 8 <= p.N) {
+                *reinterpret_cast<uint4 *>(orow + col) = v;
+              } else {
+                const uint16_t *pv = reinterpret_cast<const uint16_t *>(&v);
+                for (int e = 0; e < 8; ++e)
+                  if (nt0 + col + e < p.N) orow[col + e] = pv[e];
               }
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                if (m_base + r0 + j >= p.M) break;  // the same for the whole warp
-                uint16_t *o = orow0 + int64_t(r0 + j) * p.od_m;
-                const int e0 = 2 * lane - mis[j];
-                if (e0 >= 0 && e0 + 1 < nv) {
-                  *reinterpret_cast<uint32_t *>(o + e0) = val[j];
-                } else {
-                  if (e0 >= 0 && e0 < nv) o[e0] = uint16_t(val[j]);
-                  if (e0 + 1 < nv) o[e0 + 1] = uint16_t(val[j] >> 16);
-                }
-                if (mis[j] && lane == 0 && 63 < nv) o[63] = last[j];
+            }
+            // tail after the tile's last chunk: its last q columns (staged at 72..)
+            const bool last_chunk = cc == BN / 64 - 1 || gn0 + 64 >= p.N;
+            if (last_chunk && qrow > 0 && my_row_ok) {
+              for (int e = 0; e < qrow; ++e) {
+                const int col = cc * 64 + 64 - qrow + e;
+                if (nt0 + col < p.N) myout[col] = row16[72 + e];
               }
             }
             continue;

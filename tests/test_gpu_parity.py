@@ -183,6 +183,10 @@ GEMM_CASES = [
     (I.BF16, 64, 40, 8, 1, "k", "k", 1.0, 0.0),
     (I.BF16, 2048, 1536, 2048, 1, "k", "k", 1.0, 0.0),
     (I.BF16, 2048, 1536, 2048, 1, "k", "n", 1.0, 0.0),
+    # output rows that are not 16-byte aligned (odd N = row stride), several N tiles
+    (I.BF16, 520, 777, 96, 1, "k", "k", 1.0, 0.0),
+    (I.BF16, 136, 515, 64, 2, "m", "k", -1.0, 0.0),
+    (I.BF16, 1100, 5461, 128, 1, "k", "k", 1.0, 0.0),
 ]
 
 
