@@ -62,6 +62,8 @@ def parse_args():
     ap.add_argument("--no-merge", action="store_true")
     ap.add_argument("--plan", choices=sorted(PLANS), default="auto",
                     help="where the primitives act: auto (cost model), token (activations) or weight (W0)")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eager launches instead of replaying each variant's step as a CUDA graph")
     ap.add_argument("--no-token-plan", action="store_true",
                     help="skip the second timed pass that runs every layer on the token plan")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (small profiling cases)")
@@ -390,7 +392,48 @@ def run_poet(args):
             elapsed, per_variant_ms = mx[0], mx[1:]
         return elapsed, per_variant_ms, trace, traces, launches, clk
 
-    elapsed, per_variant_ms, trace, traces, launches, clk = timed(args.steps, ClockSampler(smi_index))
+    # The kernel trace (per-kind times for the roofline) comes from eager steps.
+    # The headline time replays each variant's step captured as one CUDA graph
+    # (one process per GPU; every buffer is resident, so a step launches the
+    # same kernels on the same pointers every time).  Under data parallelism the
+    # step holds an NCCL all-reduce and stays eager.
+    use_graph = not args.no_graph and world == 1
+    e_elapsed, e_per_variant_ms, trace, traces, launches, e_clk = timed(args.steps, None if use_graph else
+                                                                        ClockSampler(smi_index))
+    graphs = None
+    if use_graph:
+        graphs = []
+        cap = torch.cuda.Stream()
+        for v in variants:
+            cap.wait_stream(torch.cuda.current_stream())
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph, stream=cap):
+                v.step(world)
+            torch.cuda.current_stream().wait_stream(cap)
+            graphs.append(gph)
+        for gph in graphs:  # warm replays
+            gph.replay()
+        torch.cuda.synchronize()
+        poet.poet_sync_status()
+        clocks = ClockSampler(smi_index)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in variants]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        clocks.start()
+        t0.record(stream)
+        for i, gph in enumerate(graphs):
+            ev[i][0].record(stream)
+            for _ in range(args.steps):
+                gph.replay()
+            ev[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        clk = clocks.stop()
+        poet.poet_sync_status()
+        elapsed = t0.elapsed_time(t1)
+        per_variant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(len(variants))]
+    else:
+        elapsed, per_variant_ms, clk = e_elapsed, e_per_variant_ms, e_clk
     plans_run = [v.plan_names() for v in variants]
 
     tokens_per_step = sum(v.T for v in variants) * world
@@ -495,6 +538,8 @@ def run_poet(args):
                      for i, v in enumerate(variants)},
         "value_merge_amortized": (round(tokens_per_step / ((ms_per_step + sum(merge.values()) / 400.0) / 1e3), 1)
                                   if merge else None),
+        "timing": {"mode": "cuda_graph" if use_graph else "eager",
+                   "eager_ms_per_step": round(e_elapsed / args.steps, 3)},
         "roofline": roof, "kernels": kernels, "gpu_launches": int(launches), "clocks": clk,
         "e2e": e2e, "cpu_baseline": cpu, "token_plan": token,
     }

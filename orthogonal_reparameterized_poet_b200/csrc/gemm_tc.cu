@@ -311,7 +311,7 @@ struct Smem {
   // (plus up to 16 elements of shift and carry for rows that are not 16-byte
   // aligned), rows 176 B apart (11 16-byte units) so row-wise writes and
   // line-wise reads both take the minimum number of shared-memory wavefronts
-  static constexpr int EPI_ROW = 176;
+  static constexpr int EPI_ROW = BSTAT ? 144 : 176;  // B-stationary launches have aligned rows only
   static constexpr int EPI_BYTES = 4 * 32 * EPI_ROW;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr size_t BYTES =
@@ -604,7 +604,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
         bf16 *obase = p.outD + int64_t(c.b) * p.od_b;
         const int sub = lane & 7, rsub = lane >> 3;
         const int nt0 = c.nt * BN;
-        const bool mis_rows = p.coalesced == 3;
+        const bool mis_rows = !BSTAT && p.coalesced == 3;  // B-stationary launches never get mode 3
         const bool my_row_ok = m_base + lane < p.M;
         uint16_t *myout = reinterpret_cast<uint16_t *>(obase + int64_t(m_base + lane) * p.od_m + nt0);
         const int qrow = mis_rows ? int((reinterpret_cast<uintptr_t>(myout) >> 1) & 7) : 0;
@@ -948,8 +948,10 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   // handles addends, pairs of outputs and split-K reductions
   p->coalesced = 0;
   const bool plain = !g.add && !g.atomic && g.diag == 0.f;
-  if (plain && g.outD && !g.outF)
+  if (plain && g.outD && !g.outF) {
     p->coalesced = aligned16(g.outD) && g.od_m % 8 == 0 && (g.batch == 1 || g.od_b % 8 == 0) ? 1 : 3;
+    if (t.bstat && p->coalesced == 3) p->coalesced = 0;  // the B-stationary kernels stage aligned rows only
+  }
   if (plain && g.outF && !g.outD && aligned16(g.outF) && g.of_m % 4 == 0 && (g.batch == 1 || g.of_b % 4 == 0))
     p->coalesced = 2;
   bool ok;
