@@ -56,7 +56,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["poet", "reference"], default="poet")
     ap.add_argument("--workload", choices=sorted(WORKLOAD_SETS), default="llama1.3b")
-    ap.add_argument("--e2e-steps", type=int, default=1)
+    ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-merge", action="store_true")
@@ -549,44 +549,112 @@ def run_poet(args):
 
 
 def run_e2e(args, variants, world):
-    """Same step through the public API with host buffers: every step copies the
-    step's inputs from pinned host memory and reads the results back."""
+    """The same steps through the public API with host buffers.  Every step
+    copies its inputs (x and dy of every linear shape) from pinned host memory
+    and reads its results (all dtheta, and y and dx of the first layer) back
+    into pinned host memory.  The copies run on a second stream, double
+    buffered: step i+1's inputs go up while step i computes, and step i's
+    results come down (from a device-side snapshot) while step i+1 computes.
+    The timed region spans the first upload to the last download."""
     import torch
 
     stream = torch.cuda.current_stream()
-    host_in, host_out = [], []
+    copy = torch.cuda.Stream()
+    # device inputs: set 0 = the tensors the variants hold, set 1 = copies (one per distinct tensor)
+    uniq = {}
     for v in variants:
         for d in (v.x, v.dy):
-            for key, t in d.items():
-                host_in.append((t, t.cpu().pin_memory()))
-        host_out.append((v.dtheta, torch.empty(v.dtheta.shape, dtype=v.dtheta.dtype, pin_memory=True)))
-        last_m = v.layers[0][2]
-        last_n = v.layers[0][3]
-        host_out.append((v.y[last_m], torch.empty(v.y[last_m].shape, dtype=v.y[last_m].dtype, pin_memory=True)))
-        host_out.append((v.dx[last_n], torch.empty(v.dx[last_n].shape, dtype=v.dx[last_n].dtype, pin_memory=True)))
-    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
-    d2h = sum(h.numel() * h.element_size() for _, h in host_out)
+            for t in d.values():
+                uniq[id(t)] = t
+    sets = [{k: t for k, t in uniq.items()}, {k: torch.empty_like(t) for k, t in uniq.items()}]
+    host_in = {k: t.cpu().pin_memory() for k, t in uniq.items()}
+    base = [({n: t for n, t in v.x.items()}, {m: t for m, t in v.dy.items()}) for v in variants]
 
-    def step():
-        for dev, host in host_in:
-            dev.copy_(host, non_blocking=True)
-        for v in variants:
-            v.step(world)
-        for dev, host in host_out:
-            host.copy_(dev, non_blocking=True)
+    def use_set(sidx):
+        for v, (bx, bdy) in zip(variants, base):
+            v.x = {n: sets[sidx][id(t)] for n, t in bx.items()}
+            v.dy = {m: sets[sidx][id(t)] for m, t in bdy.items()}
 
-    step()
+    # results: per variant dtheta, y and dx of the first layer; a device snapshot and a host copy per set
+    outs = []
+    for v in variants:
+        last_m, last_n = v.layers[0][2], v.layers[0][3]
+        outs += [v.dtheta, v.y[last_m], v.dx[last_n]]
+    snap = [[torch.empty_like(t) for t in outs] for _ in range(2)]
+    host_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs] for _ in range(2)]
+    h2d = sum(h.numel() * h.element_size() for h in host_in.values())
+    d2h = sum(h.numel() * h.element_size() for h in host_out[0])
+
+    use_graph = not args.no_graph and world == 1
+    graphs = None
+    if use_graph:  # one graph per variant and input set (the sets differ in pointers)
+        graphs = []
+        for sidx in range(2):
+            use_set(sidx)
+            row = []
+            for v in variants:
+                copy.wait_stream(stream)
+                gph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gph, stream=copy):
+                    v.step(world)
+                stream.wait_stream(copy)
+                row.append(gph)
+            graphs.append(row)
+        torch.cuda.synchronize()
+
+    ev_in = [torch.cuda.Event() for _ in range(2)]       # set s uploaded
+    ev_used = [torch.cuda.Event() for _ in range(2)]     # compute on set s finished
+    ev_snap = [torch.cuda.Event() for _ in range(2)]     # snapshot s written
+    ev_down = [torch.cuda.Event() for _ in range(2)]     # snapshot s downloaded
+
+    def upload(sidx, after_use):
+        with torch.cuda.stream(copy):
+            if after_use:
+                copy.wait_event(ev_used[sidx])
+            for k, h in host_in.items():
+                sets[sidx][k].copy_(h, non_blocking=True)
+            ev_in[sidx].record(copy)
+
+    def run(steps):
+        upload(0, False)
+        for i in range(steps):
+            sidx = i % 2
+            if i + 1 < steps:
+                upload(1 - sidx, i >= 1)
+            stream.wait_event(ev_in[sidx])
+            use_set(sidx)
+            if graphs is not None:
+                for gph in graphs[sidx]:
+                    gph.replay()
+            else:
+                for v in variants:
+                    v.step(world)
+            ev_used[sidx].record(stream)
+            if i >= 2:
+                stream.wait_event(ev_down[sidx])
+            for src, dst in zip(outs, snap[sidx]):
+                dst.copy_(src, non_blocking=True)
+            ev_snap[sidx].record(stream)
+            with torch.cuda.stream(copy):
+                copy.wait_event(ev_snap[sidx])
+                for src, dst in zip(snap[sidx], host_out[sidx]):
+                    dst.copy_(src, non_blocking=True)
+                ev_down[sidx].record(copy)
+        stream.wait_stream(copy)
+
+    run(2)  # warm
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(args.e2e_steps):
-        step()
+    run(args.e2e_steps)
     b.record(stream)
     b.synchronize()
+    use_set(0)
     ms = a.elapsed_time(b) / args.e2e_steps
     tokens = sum(v.T for v in variants) * world
     return {"value": round(tokens / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 3),
-            "steps": args.e2e_steps, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+            "steps": args.e2e_steps, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "copies": "second stream, double-buffered", "mode": "cuda_graph" if use_graph else "eager"}
 
 
 # ---------------------------------------------------------------------------- CPU oracle
