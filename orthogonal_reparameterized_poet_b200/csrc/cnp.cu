@@ -111,14 +111,6 @@ Gemm prim_gemm(const SideGeom &g, int dtype, const void *X, const void *Y, bool 
 
 }  // namespace
 
-poet_status f32_to_bf16(const float *in, void *out, int64_t n, cudaStream_t st) {
-  if (n <= 0) return POET_OK;
-  TraceScope ts("convert", 0.0, double(n) * 6.0, st);
-  f32_to_bf16_kernel<<<grid_for(n, 256), 256, 0, st>>>(in, static_cast<bf16 *>(out), n);
-  count_launch();
-  return launch_status("f32 to bf16");
-}
-
 poet_status pad_blocks(const float *G, const SideGeom &g, float *out, cudaStream_t st) {
   const int64_t n = g.all_elems();
   pad_blocks_kernel<<<grid_for(n, 256), 256, 0, st>>>(G, g.nprim, g.size, g.ld, out);

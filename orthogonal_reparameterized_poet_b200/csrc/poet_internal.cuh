@@ -141,9 +141,6 @@ poet_status copy_rows(int dtype, const void *src, int64_t ld_src, int64_t rows, 
 poet_status frame_f32_to_bf16(const float *D, int64_t ldD, const int32_t *rowmap, int64_t rows, int d,
                               const int32_t *perm, void *out, int64_t ld_out, cudaStream_t st);
 
-// out[e] = bf16(in[e]) for e < n.
-poet_status f32_to_bf16(const float *in, void *out, int64_t n, cudaStream_t st);
-
 // dst[dstrow(r)][perm[i]] = (i < split ? src1[r][i] : src2[r][i]); dstrow(r) = rowmap ? rowmap[r] : r.
 poet_status scatter_cols(int dtype, const void *src1, int64_t ld1, const void *src2, int64_t ld2,
                          int split, int64_t rows, int d, const int32_t *perm,
