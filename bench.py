@@ -43,7 +43,7 @@ PLAN_NAMES = {1: "token", 2: "weight"}
 
 # DRAM traffic / algorithmic bytes of one launch, from an ncu capture, with the
 # kernel revision (as named in poet_version()) the counters were taken on.
-NCU_TRAFFIC_RATIO = {"w0_fwd": (0.933, "gemm_tc r8"), "w0_bwd": (0.962, "gemm_tc r8"), "w_grad": (1.717, "gemm_tc r8")}
+NCU_TRAFFIC_RATIO = {"w0_fwd": (0.932, "gemm_tc r9"), "w0_bwd": (0.964, "gemm_tc r9"), "w_grad": (1.713, "gemm_tc r9")}
 NCU_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of every launch of one LLaMA-1.3B layer "
                       "(profiles/launches_llama1.3b_1layer.md), as a ratio to the algorithmic bytes of the "
                       "same launches, scaled to this run's launches")

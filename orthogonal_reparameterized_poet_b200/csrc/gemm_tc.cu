@@ -729,7 +729,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
             const float4 f = *reinterpret_cast<const float4 *>(ew + rr * S::EPI_ROW + sub * 16);
             if (gm < p.M && gn < p.N) {
               float *o = obase + int64_t(gm) * p.of_m + gn;
-              if (gn + 4 <= p.N) {
+              if (p.atomic) {  // split-K: float reductions at L2, four rows x 128 B per instruction
+                if (gn + 4 <= p.N) {
+                  red_add_v4(o, f.x, f.y, f.z, f.w);
+                } else {
+                  atomicAdd(o, f.x);  // gn < N
+                  if (gn + 1 < p.N) atomicAdd(o + 1, f.y);
+                  if (gn + 2 < p.N) atomicAdd(o + 2, f.z);
+                }
+              } else if (gn + 4 <= p.N) {
                 *reinterpret_cast<float4 *>(o) = f;
               } else {
                 o[0] = f.x;  // gn < N
@@ -944,15 +952,17 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   // larger operand, which is then read from HBM about once
   p->m_fast = g.N > g.M ? 1 : 0;
   // staged epilogue for a single plain output (1: bf16, 16-byte aligned rows;
-  // 3: bf16, any rows; 2: fp32, 16-byte aligned rows); the per-row path
-  // handles addends, pairs of outputs and split-K reductions
+  // 3: bf16, any rows; 2: fp32, 16-byte aligned rows, stored or reduced); the
+  // per-row path handles addends, pairs of outputs and unaligned fp32 rows
   p->coalesced = 0;
   const bool plain = !g.add && !g.atomic && g.diag == 0.f;
   if (plain && g.outD && !g.outF) {
     p->coalesced = aligned16(g.outD) && g.od_m % 8 == 0 && (g.batch == 1 || g.od_b % 8 == 0) ? 1 : 3;
     if (t.bstat && p->coalesced == 3) p->coalesced = 0;  // the B-stationary kernels stage aligned rows only
   }
-  if (plain && g.outF && !g.outD && aligned16(g.outF) && g.of_m % 4 == 0 && (g.batch == 1 || g.of_b % 4 == 0))
+  // fp32: plain stores or split-K reductions
+  if (!g.add && g.diag == 0.f && g.outF && !g.outD && aligned16(g.outF) && g.of_m % 4 == 0 &&
+      (g.batch == 1 || g.of_b % 4 == 0))
     p->coalesced = 2;
   bool ok;
   if (!t.A_MN) ok = make_map(ma, g.A, g.K, g.M, g.batch, g.a_m, g.a_b, 64, BM);
