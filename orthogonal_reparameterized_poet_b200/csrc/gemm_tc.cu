@@ -13,11 +13,21 @@
 //   warp 1     TMEM allocator + MMA issuer (one elected lane):
 //              tcgen05.mma.cta_group::1.kind::f16, M=128, N=BN, K=16
 //   warps 2-5  epilogue: tcgen05.ld 32x32b rows out of TMEM, alpha/addend/
-//              diagonal, bf16 and/or fp32 stores, or fp32 atomics (split-K)
+//              diagonal, bf16 and/or fp32 stores, or fp32 reductions (split-K);
+//              single plain outputs are staged through shared memory so that
+//              every store instruction covers four rows x 128 bytes
 // The accumulator is double-buffered in TMEM (2 x BN columns), so the
-// epilogue of one tile overlaps the MMAs of the next.  Every mbarrier wait is
-// bounded: after a time limit the CTA records ERR_TIMEOUT in the device status
-// word, stops, drains what it issued (bounded too), frees TMEM and returns.
+// epilogue of one tile overlaps the MMAs of the next.
+//
+// CTA pairs (CG = 2, large streaming launches): two CTAs of a cluster run
+// tcgen05.mma.cta_group::2 on 256 x 256 tiles.  Each loads its 128 rows of A
+// and half of B; rank 0 issues the MMAs; stage and accumulator barriers are
+// shared through multicast commits and remote arrivals; TMEM is allocated and
+// freed by both CTAs together.
+//
+// Every mbarrier wait is bounded: after a time limit the CTA records
+// ERR_TIMEOUT in the device status word, stops, drains what it issued (bounded
+// too), frees TMEM and returns.
 #include <cudaTypedefs.h>
 
 #include <cstdlib>
