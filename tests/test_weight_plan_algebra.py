@@ -1,0 +1,79 @@
+"""The weight plan's reassociation, restated on the CPU in float64 and checked
+against the oracle's dense forward and backward (no GPU).
+
+The weight plan applies the primitives to W0 instead of the activations:
+    H = R^ W0f,  F = W0f P^,  E_f = H P^  (frame, R^ / P^ = block-diagonal sides),
+    E = E_f taken back to natural order,  y = x E^T,  dx = dy E,
+    D = dy^T x,  D_f = D in the frame,
+    G_R[j] = D_f[rows j] F[rows j]^T,  G_P[j] = H[:, cols j]^T D_f[:, cols j].
+These are exact identities of y = R W0 P x; this test pins them independently
+of the CUDA path (the GPU tests then check the kernels against the oracle)."""
+import numpy as np
+import pytest
+
+from oracle import poet_oracle as O
+
+BS, FS = 0, 1
+
+CASES = [
+    # m, n, modeR, bR, modeP, bP, k, T
+    (300, 200, BS, 64, BS, 64, 2, 37),      # leftover identity indices on both sides
+    (301, 199, FS, 0, FS, 0, 3, 29),        # fully stochastic, odd sizes
+    (96, 160, FS, 0, BS, 16, 1, 21),        # mixed modes
+    (40, 24, BS, 64, BS, 64, 2, 9),         # b > d: no primitives
+    (64, 48, BS, 16, BS, 16, 0, 13),        # k = 0
+]
+
+
+def frame_side(d, blocks, mode, b):
+    """The side in its own frame: blockdiag(blocks, I), primitives on consecutive index ranges."""
+    nprim, size = O.side_shape(d, mode, b)
+    M = np.eye(d)
+    for j in range(nprim):
+        M[j * size:(j + 1) * size, j * size:(j + 1) * size] = blocks[j]
+    return M
+
+
+@pytest.mark.parametrize("m,n,modeR,bR,modeP,bP,k,T", CASES)
+def test_weight_plan_matches_dense_chain_rule(m, n, modeR, bR, modeP, bP, k, T):
+    rng = np.random.default_rng(m * 1000 + n)
+    W0 = rng.standard_normal((m, n))
+    X = rng.standard_normal((T, n))
+    dY = rng.standard_normal((T, m))
+    permR = O.draw_perm(5, m + n, 0, 0, m)
+    permP = O.draw_perm(5, m + n, 1, 0, n)
+    nR, sR = O.side_shape(m, modeR, bR)
+    nP, sP = O.side_shape(n, modeP, bP)
+    thR = 0.05 * rng.standard_normal(nR * O.n_skew(sR))
+    thP = 0.05 * rng.standard_normal(nP * O.n_skew(sP))
+    Rb = O.cayley_neumann(thR, nR, sR, k)
+    Pb = O.cayley_neumann(thP, nP, sP, k)
+
+    # oracle: dense matrices, per-token chain rule
+    R = O.dense_side(permR, Rb, modeR, bR)
+    P = O.dense_side(permP, Pb, modeP, bP)
+    Y_ref = O.forward(W0, R, P, X)
+    dX_ref, GR_ref, GP_ref = O.backward(W0, R, P, X, dY, permR, modeR, bR, permP, modeP, bP)
+
+    # weight plan, in the frame
+    W0f = W0[np.ix_(permR, permP)]
+    Rh, Ph = frame_side(m, Rb, modeR, bR), frame_side(n, Pb, modeP, bP)
+    H, F = Rh @ W0f, W0f @ Ph
+    E_f = H @ Ph
+    E = np.empty_like(W0)
+    E[np.ix_(permR, permP)] = E_f
+    Y = X @ E.T
+    dX = dY @ E
+    D_f = (dY.T @ X)[np.ix_(permR, permP)]
+    GR = np.stack([D_f[j * sR:(j + 1) * sR] @ F[j * sR:(j + 1) * sR].T for j in range(nR)]) if nR else np.zeros((0, sR, sR))
+    GP = np.stack([H[:, j * sP:(j + 1) * sP].T @ D_f[:, j * sP:(j + 1) * sP] for j in range(nP)]) if nP else np.zeros((0, sP, sP))
+
+    def close(a, b):
+        return np.linalg.norm(a - b) <= 1e-12 * max(1.0, np.linalg.norm(b))
+
+    assert close(Y, Y_ref)
+    assert close(dX, dX_ref)
+    assert GR.shape == GR_ref.shape and close(GR, GR_ref)
+    assert GP.shape == GP_ref.shape and close(GP, GP_ref)
+    # E is the dense R W0 P: the merge of the same step
+    assert close(E, O.merge(W0, R, P))
