@@ -38,6 +38,11 @@ Conventions (readings):
   * Cayley-Neumann of order k: R_blk = (I + Q) (I + Q + Q^2 + ... + Q^k), the
     Cayley map (I+Q)(I-Q)^-1 with the inverse replaced by its truncated series.
 
+The optimizer step on theta (``adamw_step``) is adjacent to the path: the
+pages name no optimizer, so it is the textbook AdamW update (decoupled weight
+decay, bias-corrected moments; Loshchilov & Hutter, "Decoupled Weight Decay
+Regularization") -- a reading.  Its pins are that update's own closed forms.
+
 Parity pins: every function here is checked in tests/test_oracle_pins.py
 against closed forms, exact identities, brute force or values printed on the
 pages.  ``draw_perm``'s generator is pinned to the published SplitMix64 test
@@ -328,3 +333,22 @@ def layer_step(W0, thetaR, thetaP, permR, permP, modeR, bR, modeP, bP, k, X, dY)
         "dthetaP": theta_grad(G_P, thetaP, sP, k),
         "W0_merged": merge(W0, R, P),
     }
+
+
+# --------------------------------------------------------------------------
+# adjacent: the optimizer step on the packed parameters (a reading)
+# --------------------------------------------------------------------------
+
+def adamw_step(theta, grad, m, v, lr, beta1, beta2, eps, weight_decay, step):
+    """One AdamW step, elementwise on the packed skew parameters: the first and
+    second moment estimates are updated, bias-corrected by 1 - beta**step, and
+    theta moves by lr * (m_hat / (sqrt(v_hat) + eps) + weight_decay * theta)
+    (decay decoupled from the gradient).  Returns (theta, m, v) after the step."""
+    theta = np.asarray(theta, dtype=np.float64)
+    grad = np.asarray(grad, dtype=np.float64)
+    m_new = beta1 * np.asarray(m, dtype=np.float64) + (1.0 - beta1) * grad
+    v_new = beta2 * np.asarray(v, dtype=np.float64) + (1.0 - beta2) * grad * grad
+    m_hat = m_new / (1.0 - beta1 ** step)
+    v_hat = v_new / (1.0 - beta2 ** step)
+    theta_new = theta - lr * (m_hat / (np.sqrt(v_hat) + eps) + weight_decay * theta)
+    return theta_new, m_new, v_new

@@ -330,6 +330,33 @@ def check_draw_perm(O):
     return bool(ok)
 
 
+# ---------------------------------------------------------------- optimizer step (adjacent)
+
+def check_adamw_closed_forms(O):
+    """Textbook AdamW properties that fix every term of the update."""
+    rng = np.random.default_rng(3)
+    theta = rng.standard_normal(64)
+    g = rng.standard_normal(64)
+    z = np.zeros(64)
+    lr, b1, b2, eps = 1e-3, 0.9, 0.999, 1e-8
+    # first step from zero moments: m_hat = g, v_hat = g^2, so the move is lr * g / (|g| + eps)
+    th1, m1, v1 = O.adamw_step(theta, g, z, z, lr, b1, b2, eps, 0.0, 1)
+    ok = np.allclose(th1, theta - lr * g / (np.abs(g) + eps), rtol=1e-14, atol=0)
+    ok &= np.allclose(m1, (1 - b1) * g, rtol=1e-15, atol=0) and np.allclose(v1, (1 - b2) * g * g, rtol=1e-15, atol=0)
+    # a constant gradient keeps the bias-corrected moments at g and g^2: the same move every step
+    th, m, v = theta, z, z
+    for step in range(1, 6):
+        th, m, v = O.adamw_step(th, g, m, v, lr, b1, b2, eps, 0.0, step)
+    ok &= np.allclose(th, theta - 5 * lr * g / (np.abs(g) + eps), rtol=1e-12, atol=1e-15)
+    # decoupled decay: with no gradient and zero moments only the decay moves theta
+    th2, m2, v2 = O.adamw_step(theta, z, z, z, lr, b1, b2, eps, 0.1, 1)
+    ok &= np.allclose(th2, theta * (1 - lr * 0.1), rtol=1e-15, atol=0) and not m2.any() and not v2.any()
+    # moments decay geometrically with no gradient
+    _, m3, v3 = O.adamw_step(theta, z, np.ones(64), 4 * np.ones(64), lr, b1, b2, eps, 0.0, 1000)
+    ok &= np.allclose(m3, b1) and np.allclose(v3, 4 * b2)
+    return bool(ok)
+
+
 # ---------------------------------------------------------------- bookkeeping
 
 def check_param_counts(O):
@@ -349,5 +376,5 @@ ALL_CHECKS = [
     check_dense_side_golden, check_dense_side_vs_loops, check_apply_side_rows, check_side_shapes,
     check_no_primitive_side,
     check_spectrum_preservation, check_merge_invariance, check_backward_finite_differences,
-    check_splitmix_golden, check_draw_perm, check_param_counts,
+    check_splitmix_golden, check_draw_perm, check_param_counts, check_adamw_closed_forms,
 ]

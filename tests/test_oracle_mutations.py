@@ -172,6 +172,27 @@ def _trainable_with_diag(dim_out, dim_in, mode, b):
     return total
 
 
+def _adamw_no_bias_correction(theta, grad, m, v, lr, beta1, beta2, eps, weight_decay, step):
+    m_new = beta1 * m + (1.0 - beta1) * grad
+    v_new = beta2 * v + (1.0 - beta2) * grad * grad
+    return theta - lr * (m_new / (np.sqrt(v_new) + eps) + weight_decay * theta), m_new, v_new
+
+
+def _adamw_coupled_decay(theta, grad, m, v, lr, beta1, beta2, eps, weight_decay, step):
+    grad = grad + weight_decay * theta  # L2 penalty folded into the gradient (Adam, not AdamW)
+    m_new = beta1 * m + (1.0 - beta1) * grad
+    v_new = beta2 * v + (1.0 - beta2) * grad * grad
+    m_hat, v_hat = m_new / (1.0 - beta1 ** step), v_new / (1.0 - beta2 ** step)
+    return theta - lr * m_hat / (np.sqrt(v_hat) + eps), m_new, v_new
+
+
+def _adamw_no_sqrt(theta, grad, m, v, lr, beta1, beta2, eps, weight_decay, step):
+    m_new = beta1 * m + (1.0 - beta1) * grad
+    v_new = beta2 * v + (1.0 - beta2) * grad * grad
+    m_hat, v_hat = m_new / (1.0 - beta1 ** step), v_new / (1.0 - beta2 ** step)
+    return theta - lr * (m_hat / (v_hat + eps) + weight_decay * theta), m_new, v_new
+
+
 MUTANTS = {
     "unpack transposed sign": dict(unpack_skew=_unpack_transposed),
     "unpack column-major": dict(unpack_skew=_unpack_colmajor),
@@ -191,6 +212,9 @@ MUTANTS = {
     "splitmix wrong final shift": dict(splitmix64=_splitmix_wrong_const),
     "perm sorted descending": dict(draw_perm=_draw_perm_descending),
     "trainable count includes diagonal": dict(trainable_params=_trainable_with_diag),
+    "adamw without bias correction": dict(adamw_step=_adamw_no_bias_correction),
+    "adamw with the decay in the gradient": dict(adamw_step=_adamw_coupled_decay),
+    "adamw without the square root": dict(adamw_step=_adamw_no_sqrt),
 }
 
 
