@@ -280,6 +280,23 @@ POET_API poet_status poet_resample(poet_layer *L, poet_stream stream);
 POET_API poet_status poet_draw_perm(uint64_t seed, int32_t layer_id, int32_t side, int32_t epoch,
                            int32_t dim, int32_t *perm, poet_stream stream);
 
+/* ---------------------------------------------------------------- optimizer step (adjacent) */
+
+/* One AdamW step on n packed parameters in place: the pages name no
+ * optimizer for the primitives' parameters, so this is the textbook update
+ * (Loshchilov & Hutter, "Decoupled Weight Decay Regularization"):
+ *   m <- beta1 m + (1 - beta1) g,   v <- beta2 v + (1 - beta2) g^2,
+ *   theta <- theta - lr * ( (m / (1 - beta1^step)) / (sqrt(v / (1 - beta2^step)) + eps)
+ *                           + weight_decay * theta ).
+ * theta, m, v: device float[n], updated; grad: device float[n] (e.g. the
+ * dtheta of poet_backward).  step >= 1 counts the updates so far including
+ * this one.  After poet_merge resets theta, the caller resets m, v and step.
+ * Host validation: n >= 0; pointers non-NULL and 4-byte aligned when n > 0;
+ * 0 <= beta1, beta2 < 1; eps > 0; lr, weight_decay >= 0 and finite. */
+POET_API poet_status poet_adamw_step(float *theta, const float *grad, float *m, float *v, int64_t n,
+                                     float lr, float beta1, float beta2, float eps, float weight_decay,
+                                     int32_t step, poet_stream stream);
+
 /* ---------------------------------------------------------------- utilities */
 
 /* Batched dense product on the library's GEMM engine, exported so that the

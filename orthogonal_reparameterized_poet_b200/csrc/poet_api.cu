@@ -19,6 +19,7 @@
 //             G_R[j] = D_f[rows j] F[rows j]^T,  G_P[j] = H[:, cols j]^T D_f[:, cols j]
 // (G_R = sum_t dyf_t vf_t^T with vf_t = F xf_t, and G_P = sum_t duf_t xf_t^T with
 // duf_t = H^T dyf_t, so both plans give the same gradients.)
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -874,6 +875,22 @@ poet_status poet_gemm(int32_t dtype, int32_t M, int32_t N, int32_t K, int32_t ba
   if (beta != 0.f) { p.add = C; p.add_dtype = dtype; p.add_m = ldc; p.add_b = sCb; p.beta = beta; }
   p.outD = C; p.od_m = ldc; p.od_b = sCb;
   return gemm_run(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+poet_status poet_adamw_step(float *theta, const float *grad, float *m, float *v, int64_t n, float lr, float beta1,
+                            float beta2, float eps, float weight_decay, int32_t step, poet_stream stream) {
+  clear_error();
+  POET_REQUIRE(n >= 0, "poet_adamw_step: n=%lld < 0", (long long)n);
+  POET_REQUIRE(step >= 1, "poet_adamw_step: step=%d < 1", step);
+  POET_REQUIRE(std::isfinite(lr) && lr >= 0.f && std::isfinite(weight_decay) && weight_decay >= 0.f,
+               "poet_adamw_step: lr and weight_decay must be finite and >= 0");
+  POET_REQUIRE(beta1 >= 0.f && beta1 < 1.f && beta2 >= 0.f && beta2 < 1.f, "poet_adamw_step: betas outside [0, 1)");
+  POET_REQUIRE(std::isfinite(eps) && eps > 0.f, "poet_adamw_step: eps must be > 0");
+  if (n == 0) return POET_OK;
+  auto ok = [](const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 3) == 0; };
+  POET_REQUIRE(ok(theta) && ok(grad) && ok(m) && ok(v), "poet_adamw_step: NULL or misaligned buffer");
+  return adamw_step(theta, grad, m, v, n, lr, beta1, beta2, eps, weight_decay, step,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 poet_status poet_selftest_bounded_wait(uint32_t timeout_us, poet_stream stream) {

@@ -163,6 +163,12 @@ size_t cnp_many_scratch_bytes(const SideGeom &g, int dtype);
 // out = G (dense [nprim][size][size]) re-laid as [nprim][ld][ld] with zero padding
 poet_status pad_blocks(const float *G, const SideGeom &g, float *out, cudaStream_t st);
 
+// ------------------------------------------------------------------ optimizer step
+
+// One AdamW step on n float parameters in place (see poet_adamw_step).
+poet_status adamw_step(float *theta, const float *grad, float *m, float *v, int64_t n, float lr, float beta1,
+                       float beta2, float eps, float weight_decay, int32_t step, cudaStream_t st);
+
 // ------------------------------------------------------------------ permutations
 
 poet_status draw_perm_dev(uint64_t seed, int32_t layer_id, int32_t side, int32_t epoch,

@@ -86,6 +86,9 @@ _SIGS = {
     "poet_cayley_neumann_grad_noalloc": (ctypes.c_int, [ctypes.POINTER(poet_side), ctypes.c_int32, ctypes.c_void_p,
                                                         ctypes.c_void_p, ctypes.c_void_p]),
     "poet_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_void_p]),
+    "poet_adamw_step": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_int64, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                       ctypes.c_float, ctypes.c_float, ctypes.c_int32, ctypes.c_void_p]),
     "poet_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "poet_launch_count": (ctypes.c_int64, []),
     "poet_trace_enable": (ctypes.c_int, [ctypes.c_int32]),
@@ -219,6 +222,16 @@ def poet_gemm_engine(dtype: int) -> int:
 
 def poet_selftest_bounded_wait(timeout_us: int, stream=None):
     _check(lib().poet_selftest_bounded_wait(timeout_us, _stream(stream)))
+
+
+def poet_adamw_step(theta, grad, m, v, lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=1,
+                    stream=None):
+    """One AdamW step on float tensors of equal length, in place on theta, m and v."""
+    n = theta.numel()
+    if not (grad.numel() == m.numel() == v.numel() == n):
+        raise ValueError("theta, grad, m and v must have the same length")
+    _check(lib().poet_adamw_step(_ptr(theta), _ptr(grad), _ptr(m), _ptr(v), n, lr, beta1, beta2, eps,
+                                 weight_decay, step, _stream(stream)))
 
 
 def poet_sync_status(stream=None):

@@ -127,3 +127,19 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(poet, "_LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError, match="not built"):
         poet.lib()
+
+
+def test_adamw_step_validation():
+    lib = poet.lib()
+    st = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(1 << 20)
+    call = lambda ptrs, n, lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, wd=0.0, step=1: lib.poet_adamw_step(
+        *ptrs, n, lr, b1, b2, eps, wd, step, st)
+    assert call((None, None, None, None), 0) == poet.OK            # nothing to do
+    assert call((None, None, None, None), 16) == poet.EINVAL       # NULL buffers
+    assert call((ctypes.c_void_p((1 << 20) + 2), fake, fake, fake), 16) == poet.EINVAL  # misaligned
+    assert call((fake,) * 4, 16, b1=1.0) == poet.EINVAL
+    assert call((fake,) * 4, 16, eps=0.0) == poet.EINVAL
+    assert call((fake,) * 4, 16, lr=-1.0) == poet.EINVAL
+    assert call((fake,) * 4, 16, step=0) == poet.EINVAL
+    assert call((fake,) * 4, -1) == poet.EINVAL

@@ -288,3 +288,35 @@ def test_many_sides_match_single_calls_and_oracle(cuda, which, plan):
         assert rel_fro(dP.cpu().numpy(), ref["dthetaP"]) <= tol
         assert rel_fro(dR.cpu().numpy(), dR1.cpu().numpy()) <= MANY_VS_SINGLE[which]
         assert rel_fro(dP.cpu().numpy(), dP1.cpu().numpy()) <= MANY_VS_SINGLE[which]
+
+
+# ------------------------------------------------------------------ optimizer step (adjacent)
+
+@pytest.mark.parametrize("n,offset", [(1, 0), (13, 0), (4099, 1), (1000003, 0), (1000003, 3)])
+def test_adamw_step_matches_oracle(cuda, n, offset):
+    """Three AdamW steps on the device against the float64 oracle; offset > 0
+    makes the buffers only 4-byte aligned (the scalar kernel)."""
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    rng = np.random.default_rng(n + offset)
+    theta0 = (0.02 * rng.standard_normal(n)).astype(np.float32)
+    grads = [rng.standard_normal(n).astype(np.float32) for _ in range(3)]
+    # the ABI takes float32 hyperparameters: the oracle gets the same rounded values
+    lr, b1, b2, eps, wd = (float(np.float32(h)) for h in (1e-3, 0.9, 0.999, 1e-8, 0.01))
+
+    def dev(a):
+        buf = cuda.zeros(n + offset, dtype=cuda.float32, device="cuda")
+        buf[offset:] = cuda.from_numpy(a).cuda()
+        return buf, buf[offset:]
+
+    (_, th), (_, m), (_, v) = dev(theta0), dev(np.zeros(n, np.float32)), dev(np.zeros(n, np.float32))
+    ref = (theta0.astype(np.float64), np.zeros(n), np.zeros(n))
+    for step, g in enumerate(grads, start=1):
+        _, gd = dev(g)
+        poet.poet_adamw_step(th, gd, m, v, lr, b1, b2, eps, wd, step)
+        # the oracle takes the same float32 inputs (theta and moments as the device holds them)
+        ref = O.adamw_step(ref[0], g.astype(np.float64), ref[1], ref[2], lr, b1, b2, eps, wd, step)
+    poet.poet_sync_status()
+    assert rel_fro(th.cpu().numpy(), ref[0]) <= 1e-6
+    assert rel_fro(m.cpu().numpy(), ref[1]) <= 1e-6
+    assert rel_fro(v.cpu().numpy(), ref[2]) <= 1e-6
