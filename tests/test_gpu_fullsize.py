@@ -1,5 +1,5 @@
-"""Parity at the benchmark's full size: LLaMA-1.3B shapes, 32768 tokens, layer
-0 of both variants (fully stochastic and block-stochastic b=256), built from
+"""Parity at the benchmark's full size: LLaMA-1.3B shapes, 32768 tokens, the
+first (and, for one shape, the last) layer of both variants (fully stochastic and block-stochastic b=256), built from
 the same seeded inputs and run through the same grouped calls bench.py times
 (poet_cayley_neumann_many, poet_forward, poet_backward_blocks,
 poet_cayley_neumann_grad_many, then poet_merge).
@@ -37,18 +37,20 @@ def cuda():
     return torch
 
 
-CASES = [("llama1.3b_fs", 4), ("llama1.3b_fs", 6), ("llama1.3b_bs256", 4), ("llama1.3b_bs256", 6)]
+# (variant, linear, layer): square (q), wide (gate) and tall (down) shapes; the first and last layer
+CASES = [("llama1.3b_fs", 0, 0), ("llama1.3b_fs", 4, 0), ("llama1.3b_fs", 6, 0), ("llama1.3b_fs", 4, 23),
+         ("llama1.3b_bs256", 0, 0), ("llama1.3b_bs256", 4, 0), ("llama1.3b_bs256", 6, 0)]
 # auto: the plan bench.py runs at this size (the weight plan); token: the other one
 PLANS = {"auto": 0, "token": 1}
 
 
 @pytest.mark.parametrize("plan", list(PLANS))
-@pytest.mark.parametrize("name,linear", CASES)
-def test_fullsize_sampled_parity(cuda, name, linear, plan):
+@pytest.mark.parametrize("name,linear,layer", CASES)
+def test_fullsize_sampled_parity(cuda, name, linear, layer, plan):
     from orthogonal_reparameterized_poet_b200 import poet
 
     wl = I.WORKLOADS[name]
-    layer, T, k, dt = 0, wl.tokens, wl.k, wl.dtype
+    T, k, dt = wl.tokens, wl.k, wl.dtype
     m, n = wl.linear_shapes()[linear]
     layer_id = layer * len(wl.linear_shapes()) + linear
     nR, sR = O.side_shape(m, wl.mode, wl.b)
