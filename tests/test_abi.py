@@ -143,3 +143,23 @@ def test_adamw_step_validation():
     assert call((fake,) * 4, 16, lr=-1.0) == poet.EINVAL
     assert call((fake,) * 4, 16, step=0) == poet.EINVAL
     assert call((fake,) * 4, -1) == poet.EINVAL
+
+
+@pytest.mark.parametrize("m,n,mode,b,dtype", [(512, 512, poet.FS, 0, poet.BF16), (1376, 512, poet.FS, 0, poet.BF16),
+                                              (2736, 1024, poet.BS, 256, poet.BF16), (5461, 2048, poet.BS, 256, poet.BF16),
+                                              (6912, 2560, poet.FS, 0, poet.BF16), (256, 256, poet.BS, 32, poet.F32)])
+def test_auto_plan_switches_once(m, n, mode, b, dtype):
+    """The cost model's choice is monotone in the token count: the token plan up
+    to some T, the weight plan beyond it (never back)."""
+    L = _layer(m, n, mode, b, 4, dtype)
+    plans = [poet.poet_plan_for(L, T) for T in [0, 1, 16, 64, 256, 1024, 2048, 4096, 8192, 16384, 32768, 1 << 20]]
+    assert set(plans) <= {poet.PLAN_TOKEN, poet.PLAN_WEIGHT}
+    first_weight = plans.index(poet.PLAN_WEIGHT) if poet.PLAN_WEIGHT in plans else len(plans)
+    assert all(p == poet.PLAN_TOKEN for p in plans[:first_weight])
+    assert all(p == poet.PLAN_WEIGHT for p in plans[first_weight:])
+    # the workspace and saved sizes follow the plan the layer runs
+    for T in (64, 32768):
+        L.plan = poet.poet_plan_for(L, T)
+        fixed = (poet.poet_saved_bytes(L, T), poet.poet_workspace_bytes(L, T))
+        L.plan = poet.PLAN_AUTO
+        assert (poet.poet_saved_bytes(L, T), poet.poet_workspace_bytes(L, T)) == fixed
