@@ -60,6 +60,7 @@ extern "C" {
 
 poet_status poet_cayley_neumann_grad_noalloc(const poet_side *side, int32_t dtype, const float *G, float *dtheta,
                                              poet_stream stream) {
+  CallRange nvtx_range("poet_cayley_neumann_grad_noalloc");
   clear_error();
   SideGeom g;
   POET_REQUIRE(side_geom(side, &g), "poet_cayley_neumann_grad_noalloc: malformed side");

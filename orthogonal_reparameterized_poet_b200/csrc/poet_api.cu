@@ -400,6 +400,7 @@ size_t poet_side_workspace_bytes(const poet_side *side, int32_t dtype) {
 }
 
 poet_status poet_cayley_neumann(const poet_side *side, int32_t dtype, void *ws, size_t ws_bytes, poet_stream stream) {
+  CallRange nvtx_range("poet_cayley_neumann");
   (void)ws; (void)ws_bytes;
   clear_error();
   SideGeom g;
@@ -413,6 +414,7 @@ poet_status poet_cayley_neumann(const poet_side *side, int32_t dtype, void *ws, 
 
 poet_status poet_cayley_neumann_grad(const poet_side *side, int32_t dtype, const float *G, float *dtheta, void *ws,
                                      size_t ws_bytes, poet_stream stream) {
+  CallRange nvtx_range("poet_cayley_neumann_grad");
   clear_error();
   SideGeom g;
   POET_REQUIRE(side_geom(side, &g), "poet_cayley_neumann_grad: malformed side");
@@ -563,6 +565,7 @@ static poet_status backward_weight(const poet_layer *L, const LayerGeom &lg, cha
 
 poet_status poet_forward(const poet_layer *L, const void *x, int64_t T, void *y, void *saved, void *ws,
                          size_t ws_bytes, poet_stream stream) {
+  CallRange nvtx_range("poet_forward");
   clear_error();
   LayerGeom lg;
   POET_TRY(check_layer(L, &lg, true));
@@ -675,6 +678,7 @@ static poet_status backward_core(const poet_layer *L, const LayerGeom &lg, int p
 
 poet_status poet_backward(const poet_layer *L, const void *x, const void *saved, const void *dy, int64_t T,
                           void *dx, float *dtheta_R, float *dtheta_P, void *ws, size_t ws_bytes, poet_stream stream) {
+  CallRange nvtx_range("poet_backward");
   clear_error();
   LayerGeom lg;
   POET_TRY(check_layer(L, &lg, true));
@@ -702,6 +706,7 @@ poet_status poet_backward(const poet_layer *L, const void *x, const void *saved,
 
 poet_status poet_backward_blocks(const poet_layer *L, const void *x, const void *saved, const void *dy, int64_t T,
                                  void *dx, float *G_R, float *G_P, void *ws, size_t ws_bytes, poet_stream stream) {
+  CallRange nvtx_range("poet_backward_blocks");
   clear_error();
   LayerGeom lg;
   POET_TRY(check_layer(L, &lg, true));
@@ -727,6 +732,7 @@ size_t poet_block_grad_bytes(const poet_side *side) {
 }
 
 poet_status poet_cayley_neumann_many(const poet_side *sides, int32_t count, int32_t dtype, poet_stream stream) {
+  CallRange nvtx_range("poet_cayley_neumann_many");
   clear_error();
   POET_REQUIRE(count >= 0 && (count == 0 || sides), "poet_cayley_neumann_many: bad side list");
   POET_REQUIRE(dtype == POET_F32 || dtype == POET_BF16, "poet_cayley_neumann_many: bad dtype %d", dtype);
@@ -754,6 +760,7 @@ size_t poet_cayley_neumann_grad_many_workspace_bytes(const poet_side *sides, int
 poet_status poet_cayley_neumann_grad_many(const poet_side *sides, const float *const *G, float *const *dtheta,
                                           int32_t count, int32_t dtype, void *ws, size_t ws_bytes,
                                           poet_stream stream) {
+  CallRange nvtx_range("poet_cayley_neumann_grad_many");
   clear_error();
   POET_REQUIRE(count >= 0 && (count == 0 || (sides && G && dtheta)), "poet_cayley_neumann_grad_many: bad lists");
   POET_REQUIRE(dtype == POET_F32 || dtype == POET_BF16, "poet_cayley_neumann_grad_many: bad dtype %d", dtype);
@@ -778,6 +785,7 @@ poet_status poet_cayley_neumann_grad_many(const poet_side *sides, const float *c
 }
 
 poet_status poet_prepare(poet_layer *L, poet_stream stream) {
+  CallRange nvtx_range("poet_prepare");
   clear_error();
   LayerGeom lg;
   POET_TRY(check_layer(L, &lg, false));
@@ -790,6 +798,7 @@ poet_status poet_prepare(poet_layer *L, poet_stream stream) {
 }
 
 poet_status poet_resample(poet_layer *L, poet_stream stream) {
+  CallRange nvtx_range("poet_resample");
   clear_error();
   POET_REQUIRE(L != nullptr, "poet_resample: layer is NULL");
   POET_REQUIRE(L->epoch >= 0 && L->epoch < 0x7FFFFFFF, "poet_resample: epoch %d cannot advance", L->epoch);
@@ -801,11 +810,13 @@ poet_status poet_resample(poet_layer *L, poet_stream stream) {
 
 poet_status poet_draw_perm(uint64_t seed, int32_t layer_id, int32_t side, int32_t epoch, int32_t dim, int32_t *perm,
                            poet_stream stream) {
+  CallRange nvtx_range("poet_draw_perm");
   clear_error();
   return draw_perm_dev(seed, layer_id, side, epoch, dim, perm, reinterpret_cast<cudaStream_t>(stream));
 }
 
 poet_status poet_merge(poet_layer *L, void *ws, size_t ws_bytes, poet_stream stream) {
+  CallRange nvtx_range("poet_merge");
   clear_error();
   LayerGeom lg;
   POET_TRY(check_layer(L, &lg, true));
@@ -862,6 +873,7 @@ poet_status poet_merge(poet_layer *L, void *ws, size_t ws_bytes, poet_stream str
 poet_status poet_gemm(int32_t dtype, int32_t M, int32_t N, int32_t K, int32_t batch, const void *A, int64_t sAm,
                       int64_t sAk, int64_t sAb, const void *B, int64_t sBn, int64_t sBk, int64_t sBb, void *C,
                       int64_t ldc, int64_t sCb, float alpha, float beta, poet_stream stream) {
+  CallRange nvtx_range("poet_gemm");
   clear_error();
   POET_REQUIRE(dtype == POET_F32 || dtype == POET_BF16, "poet_gemm: bad dtype %d", dtype);
   POET_REQUIRE(M >= 0 && N >= 0 && K >= 0 && batch >= 0, "poet_gemm: negative size");
@@ -879,6 +891,7 @@ poet_status poet_gemm(int32_t dtype, int32_t M, int32_t N, int32_t K, int32_t ba
 
 poet_status poet_adamw_step(float *theta, const float *grad, float *m, float *v, int64_t n, float lr, float beta1,
                             float beta2, float eps, float weight_decay, int32_t step, poet_stream stream) {
+  CallRange nvtx_range("poet_adamw_step");
   clear_error();
   POET_REQUIRE(n >= 0, "poet_adamw_step: n=%lld < 0", (long long)n);
   POET_REQUIRE(step >= 1, "poet_adamw_step: step=%d < 1", step);

@@ -64,6 +64,16 @@ struct TraceScope {
   cudaStream_t st = nullptr;
 };
 
+// An NVTX range around one ABI call on the calling thread (the kernels it
+// launches carry the call's name in a profiler's NVTX filters; TraceScope adds
+// a nested range per kernel kind).  No-ops unless a profiler is attached.
+struct CallRange {
+  explicit CallRange(const char *name);
+  ~CallRange();
+  CallRange(const CallRange &) = delete;
+  CallRange &operator=(const CallRange &) = delete;
+};
+
 // ------------------------------------------------------------------ geometry
 
 inline size_t esize(int dtype) { return dtype == POET_BF16 ? 2 : 4; }

@@ -6,6 +6,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "poet_internal.cuh"
 
 namespace poet {
@@ -40,7 +42,11 @@ cudaEvent_t take_event() {
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 bool trace_on() { return g_trace.load(std::memory_order_relaxed); }
 
+CallRange::CallRange(const char *name) { nvtxRangePushA(name); }
+CallRange::~CallRange() { nvtxRangePop(); }
+
 TraceScope::TraceScope(const char *kind, double flop, double bytes, cudaStream_t s) : st(s) {
+  nvtxRangePushA(kind);
   if (!trace_on()) return;
   std::lock_guard<std::mutex> lock(g_mu);
   Rec r{kind, flop, bytes, take_event(), take_event()};
@@ -51,9 +57,11 @@ TraceScope::TraceScope(const char *kind, double flop, double bytes, cudaStream_t
 }
 
 TraceScope::~TraceScope() {
-  if (slot < 0) return;
-  std::lock_guard<std::mutex> lock(g_mu);
-  cudaEventRecord(g_recs[slot].e1, st);
+  if (slot >= 0) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    cudaEventRecord(g_recs[slot].e1, st);
+  }
+  nvtxRangePop();
 }
 
 }  // namespace poet
