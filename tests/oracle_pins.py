@@ -330,6 +330,15 @@ def check_draw_perm(O):
     return bool(ok)
 
 
+def check_perm_stream_seed_golden(O):
+    """The mixing of (seed, layer, side, epoch) into the key stream's seed, on
+    tuples whose SplitMix64 inputs are published test-vector points (the
+    expected values were derived by hand, tests/golden/perm_stream_seed.json)."""
+    g = load_golden("perm_stream_seed.json")
+    return all(O.perm_stream_seed(int(c["seed"]), c["layer_id"], c["side"], c["epoch"]) == int(c["h"])
+               for c in g["cases"])
+
+
 # ---------------------------------------------------------------- optimizer step (adjacent)
 
 def check_adamw_closed_forms(O):
@@ -376,5 +385,5 @@ ALL_CHECKS = [
     check_dense_side_golden, check_dense_side_vs_loops, check_apply_side_rows, check_side_shapes,
     check_no_primitive_side,
     check_spectrum_preservation, check_merge_invariance, check_backward_finite_differences,
-    check_splitmix_golden, check_draw_perm, check_param_counts, check_adamw_closed_forms,
+    check_splitmix_golden, check_perm_stream_seed_golden, check_draw_perm, check_param_counts, check_adamw_closed_forms,
 ]

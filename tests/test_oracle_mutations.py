@@ -164,6 +164,24 @@ def _draw_perm_descending(seed, layer_id, side, epoch, dim):
     return np.asarray(sorted(range(dim), key=lambda i: (-keys[i], i)), dtype=np.int32)
 
 
+_M64 = (1 << 64) - 1
+
+
+def _stream_seed_side_epoch_swapped(seed, layer_id, side, epoch):
+    inner = splitmix64((((layer_id & 0xFFFFFFFF) << 32) ^ ((side & 1) << 1) ^ (epoch & 0x7FFFFFFF)) & _M64)  # noqa: F821
+    return splitmix64((seed ^ inner) & _M64)  # noqa: F821
+
+
+def _stream_seed_no_inner_step(seed, layer_id, side, epoch):
+    inner = (((layer_id & 0xFFFFFFFF) << 32) ^ ((epoch & 0x7FFFFFFF) << 1) ^ (side & 1)) & _M64
+    return splitmix64((seed ^ inner) & _M64)  # noqa: F821
+
+
+def _stream_seed_layer_unshifted(seed, layer_id, side, epoch):
+    inner = splitmix64(((layer_id & 0xFFFFFFFF) ^ ((epoch & 0x7FFFFFFF) << 1) ^ (side & 1)) & _M64)  # noqa: F821
+    return splitmix64((seed ^ inner) & _M64)  # noqa: F821
+
+
 def _trainable_with_diag(dim_out, dim_in, mode, b):
     total = 0
     for d in (dim_out, dim_in):
@@ -211,6 +229,9 @@ MUTANTS = {
     "merge wrong operand order": dict(merge=_merge_wrong_order),
     "splitmix wrong final shift": dict(splitmix64=_splitmix_wrong_const),
     "perm sorted descending": dict(draw_perm=_draw_perm_descending),
+    "stream seed with side and epoch terms swapped": dict(perm_stream_seed=_stream_seed_side_epoch_swapped),
+    "stream seed without the inner SplitMix64 step": dict(perm_stream_seed=_stream_seed_no_inner_step),
+    "stream seed with the layer not shifted": dict(perm_stream_seed=_stream_seed_layer_unshifted),
     "trainable count includes diagonal": dict(trainable_params=_trainable_with_diag),
     "adamw without bias correction": dict(adamw_step=_adamw_no_bias_correction),
     "adamw with the decay in the gradient": dict(adamw_step=_adamw_coupled_decay),
