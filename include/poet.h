@@ -27,9 +27,13 @@
  *  - Status: arguments are validated on the host before anything is
  *    launched; a bad argument returns POET_EINVAL and launches nothing.  A
  *    failed CUDA launch returns POET_ECUDA.  Device-side errors (a bounded
- *    wait that ran out) are recorded in a device status word that
- *    poet_sync_status() reads.  poet_last_error() describes the last failure
- *    of the calling thread.
+ *    wait that ran out, a perm entry out of range) are recorded in a device
+ *    status word that poet_sync_status() reads; kernels never dereference an
+ *    index they found out of range.  poet_last_error() describes the last
+ *    failure of the calling thread.
+ *  - The library caches per-device addresses of its own device variables
+ *    (the status word, the allocation-free entry point's scratch).  Do not
+ *    use it across a cudaDeviceReset of a device it has run on.
  *
  * One side (R: dim = m, P: dim = n) -- readings of [P1] Key results
  * ("POET-FS (b=1/2)", "POET-BS (b=256)"); the pages fix no layout:
@@ -89,7 +93,9 @@ typedef enum {
   POET_EINVAL = 1,     /* bad argument; nothing was launched */
   POET_ECUDA = 2,      /* a CUDA call or launch failed */
   POET_ETIMEOUT = 3,   /* a device-side bounded wait ran out (see poet_sync_status) */
-  POET_ENOMEM_WS = 4   /* the workspace passed is smaller than required */
+  POET_ENOMEM_WS = 4,  /* the workspace passed is smaller than required */
+  POET_EBOUNDS = 5     /* a kernel met an index out of range in a caller-written perm
+                          (outside [0, dim)) and skipped it (see poet_sync_status) */
 } poet_status;
 
 typedef enum { POET_F32 = 0, POET_BF16 = 1 } poet_dtype;
@@ -349,7 +355,9 @@ POET_API poet_status poet_selftest_bounded_wait(uint32_t timeout_us, poet_stream
 
 /* Synchronize the stream, then read and clear the device status word.
  * Returns POET_ETIMEOUT if a kernel gave up a bounded wait since the last
- * call, POET_ECUDA on a CUDA error, POET_OK otherwise. */
+ * call, else POET_EBOUNDS if a kernel skipped an index out of range (a
+ * permutation entry outside [0, dim); the results of that call are not
+ * meaningful), POET_ECUDA on a CUDA error, POET_OK otherwise. */
 POET_API poet_status poet_sync_status(poet_stream stream);
 
 /* Text of the last failure on the calling thread ("" if none). */

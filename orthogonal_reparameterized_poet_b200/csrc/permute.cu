@@ -9,6 +9,11 @@
 // One kernel serves both directions as a row gather out[r][j] = in[r][map[j]]:
 //   gather  (natural -> frame): map = perm
 //   scatter (frame -> natural): map = perm^-1, built in shared memory
+// Indices come from the caller (perm, row maps): an entry out of range is
+// never dereferenced.  A perm entry outside [0, d) leaves its map slot at 0 (a
+// valid column), a row-map entry outside [0, rows) skips that output row, and
+// either sets ERR_BOUNDS in the device status word (poet_sync_status reports
+// POET_EBOUNDS).
 // Each CTA keeps map (uint16) in shared memory and streams its rows through a
 // ring of NB row slots filled by cp.async 16-byte copies, prefetching NB-1
 // rows ahead, so the loads, the shared-memory gather and the 16-byte global
@@ -39,6 +44,7 @@ struct PermArgs {
   const int32_t *dst_rowmap;          // destination row of output row r (nullptr: r)
   int slot;                           // slot stride (elements, multiple of 16 bytes)
   int map_len;                        // map entries allocated (>= round_up(d, 8) + 8)
+  unsigned *errword;                  // ERR_BOUNDS is OR-ed in for an index out of range
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
@@ -155,13 +161,24 @@ __global__ void __launch_bounds__(NT) permute_rows_kernel(const PermArgs<T> a) {
   const int nthr = blockDim.x, warps = nthr / 32;
   for (int i = threadIdx.x; i < a.map_len; i += nthr) map[i] = 0;
   __syncthreads();
+  bool bad = false;
   if (!a.perm) {  // identity: a plain row copy (re-striding)
     for (int i = threadIdx.x; i < d; i += nthr) map[i] = uint16_t(i);
   } else if (a.inverse) {
-    for (int i = threadIdx.x; i < d; i += nthr) map[a.perm[i]] = uint16_t(i);
+    for (int i = threadIdx.x; i < d; i += nthr) {
+      const int p = a.perm[i];
+      if (unsigned(p) < unsigned(d)) map[p] = uint16_t(i);
+      else bad = true;
+    }
   } else {
-    for (int i = threadIdx.x; i < d; i += nthr) map[i] = uint16_t(a.perm[i]);
+    for (int i = threadIdx.x; i < d; i += nthr) {
+      const int p = a.perm[i];
+      const bool ok = unsigned(p) < unsigned(d);
+      map[i] = ok ? uint16_t(p) : uint16_t(0);
+      bad |= !ok;
+    }
   }
+  if (bad && a.errword) atomicOr(a.errword, ERR_BOUNDS);
   __syncthreads();  // the only block-wide barriers: map is complete
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -170,19 +187,26 @@ __global__ void __launch_bounds__(NT) permute_rows_kernel(const PermArgs<T> a) {
   const int64_t first = int64_t(blockIdx.x) * warps + warp, stride = int64_t(gridDim.x) * warps;
   const int64_t count = first < a.rows ? (a.rows - first + stride - 1) / stride : 0;
 
-  auto src1_row = [&](int64_t r) {
-    return a.src1 + (a.src_rowmap ? int64_t(a.src_rowmap[r]) : r) * a.ld1;
+  // source and destination row of output row r; -1 when a row map's entry is out of range
+  auto src_row = [&](int64_t r) -> int64_t {
+    if (!a.src_rowmap) return r;
+    const int64_t s = a.src_rowmap[r];
+    return s >= 0 && s < a.rows ? s : -1;
+  };
+  auto dst_row = [&](int64_t r) -> int64_t {
+    if (!a.dst_rowmap) return r;
+    const int64_t s = a.dst_rowmap[r];
+    return s >= 0 && s < a.rows ? s : -1;
   };
   auto issue = [&](int64_t k) {
     const int64_t r = first + k * stride;
+    const int64_t sr = src_row(r);
+    if (sr < 0 || dst_row(r) < 0) return;  // skipped row: nothing to load
     T *slot = ring + int64_t(k % NBW) * a.slot;
-    const T *r1 = src1_row(r);
+    const T *r1 = a.src1 + sr * a.ld1;
     const int off = misalign(r1);
     load_part(r1, 0, split, slot, off, lane);
-    if (split < d) {
-      const T *r2 = a.src2 + (a.src_rowmap ? int64_t(a.src_rowmap[r]) : r) * a.ld2;
-      load_part(r2, split, d, slot, off, lane);
-    }
+    if (split < d) load_part(a.src2 + sr * a.ld2, split, d, slot, off, lane);
   };
 
   if (count > 0) issue(0);
@@ -193,8 +217,14 @@ __global__ void __launch_bounds__(NT) permute_rows_kernel(const PermArgs<T> a) {
     cp_async_wait_one();  // this lane's copies of row k have landed
     __syncwarp();         // ... and every other lane's (scalar edges included)
     const int64_t r = first + k * stride;
-    const T *s = ring + int64_t(k % NBW) * a.slot + misalign(src1_row(r));
-    T *drow = a.dst1 + (a.dst_rowmap ? int64_t(a.dst_rowmap[r]) : r) * a.ldd1;
+    const int64_t sr = src_row(r), dr = dst_row(r);
+    if (sr < 0 || dr < 0) {  // a row map entry out of range: skip the row, report it
+      if (lane == 0 && a.errword) atomicOr(a.errword, ERR_BOUNDS);
+      __syncwarp();
+      continue;
+    }
+    const T *s = ring + int64_t(k % NBW) * a.slot + misalign(a.src1 + sr * a.ld1);
+    T *drow = a.dst1 + dr * a.ldd1;
     T *d2row = a.dst2 ? a.dst2 + r * a.ldd2 : nullptr;
     switch (misalign(drow)) {
       case 0: emit_row<T, 0>(a, map, s, drow, d2row, lane); break;
@@ -260,23 +290,37 @@ __global__ void __launch_bounds__(256) restride_kernel(const unsigned char *__re
 
 // out[a][c] = bf16(D[rowmap[a]][perm[c]]): a float matrix gathered into the
 // frame and rounded in one pass.  One block per output row at a time; the
-// source row is read through L1 (it is reused by the block's gathers).
+// source row is read through L1 (it is reused by the block's gathers).  An
+// index out of range (rowmap outside [0, rows), perm outside [0, d)) is not
+// read: its output is 0 and ERR_BOUNDS is set in the status word.
 __global__ void __launch_bounds__(256) frame_f32_to_bf16_kernel(const float *__restrict__ D, int64_t ldD,
                                                                 const int32_t *__restrict__ rowmap, int64_t rows,
                                                                 int d, const int32_t *__restrict__ perm,
-                                                                bf16 *__restrict__ out, int64_t ld_out) {
+                                                                bf16 *__restrict__ out, int64_t ld_out,
+                                                                unsigned *errword) {
+  bool bad = false;
   for (int64_t a = blockIdx.x; a < rows; a += gridDim.x) {
-    const float *src = D + int64_t(__ldg(rowmap + a)) * ldD;
+    const int64_t sr = __ldg(rowmap + a);
+    const bool row_ok = sr >= 0 && sr < rows;
+    bad |= !row_ok;
+    const float *src = D + (row_ok ? sr : 0) * ldD;
     bf16 *orow = out + a * ld_out;
     for (int c = 2 * threadIdx.x; c < d; c += 2 * blockDim.x) {
       if (c + 1 < d) {
         const int2 pc = *reinterpret_cast<const int2 *>(perm + c);
-        *reinterpret_cast<__nv_bfloat162 *>(orow + c) = __floats2bfloat162_rn(__ldg(src + pc.x), __ldg(src + pc.y));
+        const bool okx = row_ok && unsigned(pc.x) < unsigned(d), oky = row_ok && unsigned(pc.y) < unsigned(d);
+        bad |= !(okx && oky);
+        *reinterpret_cast<__nv_bfloat162 *>(orow + c) =
+            __floats2bfloat162_rn(okx ? __ldg(src + pc.x) : 0.f, oky ? __ldg(src + pc.y) : 0.f);
       } else {
-        orow[c] = __float2bfloat16_rn(__ldg(src + perm[c]));
+        const int pc = perm[c];
+        const bool ok = row_ok && unsigned(pc) < unsigned(d);
+        bad |= !ok;
+        orow[c] = __float2bfloat16_rn(ok ? __ldg(src + pc) : 0.f);
       }
     }
   }
+  if (bad && errword) atomicOr(errword, ERR_BOUNDS);
 }
 
 template <typename T>
@@ -304,6 +348,7 @@ poet_status launch_permute(PermArgs<T> a, cudaStream_t st, const char *kind) {
   const int64_t want = (a.rows + warps - 1) / warps;
   const int64_t cap = int64_t(num_sms()) * per_sm;
   const int grid = int(want < cap ? want : cap);
+  a.errword = device_errword();
   TraceScope ts(kind, 0.0, double(a.rows) * a.d * sizeof(T) * 2.0, st);
   permute_rows_kernel<T><<<grid, warps * 32, smem, st>>>(a);
   count_launch();
@@ -342,7 +387,8 @@ poet_status frame_f32_to_bf16(const float *D, int64_t ldD, const int32_t *rowmap
   TraceScope ts("frame", 0.0, double(rows) * d * 6.0, st);
   const int64_t cap = int64_t(num_sms()) * 8;
   const int grid = int(rows < cap ? rows : cap);
-  frame_f32_to_bf16_kernel<<<grid, 256, 0, st>>>(D, ldD, rowmap, rows, d, perm, static_cast<bf16 *>(out), ld_out);
+  frame_f32_to_bf16_kernel<<<grid, 256, 0, st>>>(D, ldD, rowmap, rows, d, perm, static_cast<bf16 *>(out), ld_out,
+                                                  device_errword());
   count_launch();
   return launch_status("frame");
 }

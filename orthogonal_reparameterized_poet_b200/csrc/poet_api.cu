@@ -924,8 +924,8 @@ poet_status poet_sync_status(poet_stream stream) {
     unsigned zero = 0;
     POET_CUDA_TRY(cudaMemcpy(ew, &zero, sizeof(zero), cudaMemcpyHostToDevice));
     set_error("device status word 0x%x (%s%s)", word, (word & ERR_TIMEOUT) ? "bounded wait ran out " : "",
-              (word & ERR_BOUNDS) ? "index out of bounds" : "");
-    return POET_ETIMEOUT;
+              (word & ERR_BOUNDS) ? "index out of range skipped" : "");
+    return (word & ERR_TIMEOUT) ? POET_ETIMEOUT : POET_EBOUNDS;
   }
   return POET_OK;
 }

@@ -15,7 +15,7 @@ import torch
 F32, BF16 = 0, 1
 BS, FS = 0, 1
 PLAN_AUTO, PLAN_TOKEN, PLAN_WEIGHT = 0, 1, 2
-OK, EINVAL, ECUDA, ETIMEOUT, ENOMEM_WS = 0, 1, 2, 3, 4
+OK, EINVAL, ECUDA, ETIMEOUT, ENOMEM_WS, EBOUNDS = 0, 1, 2, 3, 4, 5
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpoet.so")
 _lib = None

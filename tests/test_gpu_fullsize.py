@@ -1,20 +1,23 @@
-"""Parity at the benchmark's full size: LLaMA-1.3B shapes, 32768 tokens, the
-first (and, for one shape, the last) layer of both variants (fully stochastic and block-stochastic b=256), built from
-the same seeded inputs and run through the same grouped calls bench.py times
-(poet_cayley_neumann_many, poet_forward, poet_backward_blocks,
-poet_cayley_neumann_grad_many, then poet_merge).
+"""Parity at full size, on the LLaMA-350M (block-stochastic b=256, 16384
+tokens), LLaMA-1.3B (fully stochastic and block-stochastic b=256, 32768
+tokens) and LLaMA-3B (fully stochastic, 16384 tokens) layer sets: the square
+(q), wide (gate) and tall (down) shapes of the first, middle and last layer,
+built from the same seeded inputs bench.py draws and run through the same
+grouped calls it times (poet_cayley_neumann_many, poet_forward,
+poet_backward_blocks, poet_cayley_neumann_grad_many, then poet_merge).
 
-The oracle cannot afford the whole layer at this size, so it computes sampled
+The oracle cannot afford a whole layer at this size, so it computes sampled
 outputs one by one from their definitions:
   * y and dx on 16 sampled tokens (per-token products through the primitives);
-  * dtheta of sampled primitives, whose block gradient sums over all 32768
-    tokens (only the primitive's own columns of v = W0 P x or du = W0^T R^T dy
-    are formed);
+  * dtheta of sampled primitives, whose block gradient sums over every token
+    (only the primitive's own columns of v = W0 P x or du = W0^T R^T dy are
+    formed);
   * sampled rows of the merged W0;
   * every permutation, bit-exact.
-Fully stochastic sides of size 2730 are checked through y, dx and the merge
-(their dtheta costs minutes of float64 CPU time); their 1024-sized sides are
-checked directly."""
+Fully stochastic primitives larger than 1280 (2730 at LLaMA-1.3B, 3456 at
+LLaMA-3B) cost seconds of float64 CPU time each: their dtheta is compared in
+the cases marked full_dtheta and checked through y, dx and the merge in the
+others."""
 import numpy as np
 import pytest
 
@@ -37,18 +40,40 @@ def cuda():
     return torch
 
 
-# (variant, linear, layer): square (q), wide (gate) and tall (down) shapes; the first and last layer
-CASES = [("llama1.3b_fs", 0, 0), ("llama1.3b_fs", 4, 0), ("llama1.3b_fs", 6, 0), ("llama1.3b_fs", 4, 23),
-         ("llama1.3b_bs256", 0, 0), ("llama1.3b_bs256", 4, 0), ("llama1.3b_bs256", 6, 0)]
-# auto: the plan bench.py runs at this size (the weight plan); token: the other one
+# (variant, linear, layer, full_dtheta): q, gate and down of the first, middle and last layer
+CASES = [("llama1.3b_fs", 0, 0, False), ("llama1.3b_fs", 4, 0, True), ("llama1.3b_fs", 6, 0, False),
+         ("llama1.3b_fs", 4, 23, False),
+         ("llama1.3b_bs256", 0, 0, False), ("llama1.3b_bs256", 4, 0, False), ("llama1.3b_bs256", 6, 0, False),
+         ("llama350m_bs256", 0, 0, False), ("llama350m_bs256", 4, 0, False), ("llama350m_bs256", 6, 0, False),
+         ("llama350m_bs256", 0, 12, False), ("llama350m_bs256", 4, 12, False), ("llama350m_bs256", 6, 12, False),
+         ("llama350m_bs256", 0, 23, False), ("llama350m_bs256", 4, 23, False), ("llama350m_bs256", 6, 23, False),
+         ("llama3b_fs", 0, 0, False), ("llama3b_fs", 4, 0, True), ("llama3b_fs", 6, 0, True),
+         ("llama3b_fs", 0, 16, False), ("llama3b_fs", 4, 16, False), ("llama3b_fs", 6, 16, False),
+         ("llama3b_fs", 0, 31, False), ("llama3b_fs", 4, 31, False), ("llama3b_fs", 6, 31, False)]
+# auto: the plan bench.py runs at these sizes (the weight plan); token: the other one, on the first layer
 PLANS = {"auto": 0, "token": 1}
+PARAMS = [(c, p) for c in CASES for p in PLANS if p == "auto" or c[2] == 0]
+DTHETA_MAX_SIZE = 1280  # larger fully stochastic primitives: only where full_dtheta
 
 
-@pytest.mark.parametrize("plan", list(PLANS))
-@pytest.mark.parametrize("name,linear,layer", CASES)
-def test_fullsize_sampled_parity(cuda, name, linear, layer, plan):
+_ACT = {}
+
+
+def _activations(wl, d, grad):
+    """x or dy of width d exactly as bench.py draws them on rank 0 (shared by every layer of that width)."""
+    key = (wl.seed, d, wl.tokens, wl.dtype, grad)
+    if key not in _ACT:
+        if len(_ACT) >= 4:
+            _ACT.clear()
+        _ACT[key] = I.activations(wl.seed, d, wl.tokens, d, wl.dtype, grad=grad)
+    return _ACT[key]
+
+
+@pytest.mark.parametrize("case,plan", PARAMS, ids=[f"{c[0]}-{c[1]}-{c[2]}-{p}" for c, p in PARAMS])
+def test_fullsize_sampled_parity(cuda, case, plan):
     from orthogonal_reparameterized_poet_b200 import poet
 
+    name, linear, layer, full_dtheta = case
     wl = I.WORKLOADS[name]
     T, k, dt = wl.tokens, wl.k, wl.dtype
     m, n = wl.linear_shapes()[linear]
@@ -59,8 +84,8 @@ def test_fullsize_sampled_parity(cuda, name, linear, layer, plan):
     W0 = I.w0(wl.seed, layer, linear, m, n, dt)
     thR = I.theta(wl.seed, layer, linear, 0, nR * O.n_skew(sR), wl.sigma)
     thP = I.theta(wl.seed, layer, linear, 1, nP * O.n_skew(sP), wl.sigma)
-    X = I.activations(wl.seed, n, T, n, dt)
-    dY = I.activations(wl.seed, m, T, m, dt, grad=True)
+    X = _activations(wl, n, False)
+    dY = _activations(wl, m, True)
 
     # ---------------- CUDA path, bench launch configuration
     tdt = poet.torch_dtype(dt)
@@ -106,7 +131,7 @@ def test_fullsize_sampled_parity(cuda, name, linear, layer, plan):
     assert rel_fro(dx_s, dx_ref) <= tol
     # dtheta of sampled primitives (block gradient over all tokens)
     rng = np.random.default_rng(7)
-    if sP <= 1024:
+    if sP <= DTHETA_MAX_SIZE or full_dtheta:
         dV = O.apply_side_rows(dY, permR, RbT, wl.mode, wl.b)  # R^T dy for every token
         for j in sorted(rng.choice(nP, min(2, nP), replace=False)):
             J = permP[j * sP:(j + 1) * sP]
@@ -116,7 +141,7 @@ def test_fullsize_sampled_parity(cuda, name, linear, layer, plan):
             ref = O.theta_grad_block(G, thP[j * per:(j + 1) * per].astype(np.float64), sP, k)
             assert rel_fro(dthP[j * per:(j + 1) * per], ref) <= tol
         del dV
-    if sR <= 1024:
+    if sR <= DTHETA_MAX_SIZE or full_dtheta:
         U = O.apply_side_rows(X, permP, Pb, wl.mode, wl.b)         # P x for every token
         for j in sorted(rng.choice(nR, min(2, nR), replace=False)):
             Iset = permR[j * sR:(j + 1) * sR]

@@ -58,6 +58,8 @@ CNP_CASES = [
     (1024, I.BS, 256, 4, 0.02, I.BF16),
     (1376, I.FS, 0, 4, 0.02, I.BF16),
     (5461, I.FS, 0, 4, 0.02, I.BF16),
+    (2560, I.FS, 0, 4, 0.02, I.BF16),   # LLaMA-3B hidden side: one 1280 x 1280 primitive
+    (6912, I.FS, 0, 4, 0.02, I.BF16),   # LLaMA-3B FFN side: one 3456 x 3456 primitive
     (301, I.FS, 0, 2, 0.03, I.F32),
 ]
 
@@ -163,6 +165,55 @@ def test_zero_tokens(cuda, plan):
     poet.poet_sync_status()
     assert y.shape == (0, case.m) and dx.shape == (0, case.n)
     assert not dthR.any().item() and not dthP.any().item()
+
+
+@pytest.mark.parametrize("plan", list(PLANS))
+def test_resume_is_bit_exact(cuda, plan):
+    """Checkpoint and resume: a layer's state is W0, theta_R, theta_P and its
+    integers (seed, layer_id, epoch, modes, b, k, plan).  After a step, a
+    merge-then-reinitialize and a second parameter change, a new layer built
+    from that state reproduces the permutations, the frame copy of W0 and the
+    forward output bit for bit."""
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    case = Case(640, 512, I.BS, 128, I.FS, 0, 4, 200, I.BF16, 0.02, layer_id=31, epoch=3)
+    W0, thR, thP, x, dy = case.arrays()
+    tdt = poet.torch_dtype(case.dtype)
+    xt, dyt = cuda.from_numpy(x).to("cuda", tdt), cuda.from_numpy(dy).to("cuda", tdt)
+
+    def build(W0d, tR, tP, epoch):
+        L = poet.PoetLayer(W0d, tR, tP, mode=case.modeR, b=case.bR, modeP=case.modeP, bP=case.bP, k=case.k,
+                           seed=case.seed, layer_id=case.layer_id, epoch=epoch, plan=PLANS[plan])
+        L.prepare()
+        L.cayley_neumann()
+        return L
+
+    L1 = build(cuda.from_numpy(W0).to("cuda", tdt), cuda.from_numpy(thR).cuda(), cuda.from_numpy(thP).cuda(),
+               case.epoch)
+    _, saved = L1.forward(xt)
+    _, dR, dP = L1.backward(saved, dyt, x=xt)
+    L1.theta_R.sub_(0.5 * dR)
+    L1.theta_P.sub_(0.5 * dP)
+    L1.cayley_neumann()
+    L1.merge()
+    L1.resample()
+    L1.theta_R.copy_(cuda.from_numpy(I.theta(5, 0, 0, 0, L1.theta_R.numel(), 0.02)).cuda())
+    L1.cayley_neumann()
+    y1, _ = L1.forward(xt)
+    poet.poet_sync_status()
+    # the checkpoint: tensors and integers only
+    ck = (L1.W0.clone(), L1.theta_R.clone(), L1.theta_P.clone(), L1.epoch)
+    L2 = build(*ck)
+    y2, _ = L2.forward(xt)
+    poet.poet_sync_status()
+    assert L2.epoch == case.epoch + 1
+    assert cuda.equal(L2.perm_R, L1.perm_R) and cuda.equal(L2.perm_P, L1.perm_P)
+    es = 2 if case.dtype == I.BF16 else 4
+    ldn = (case.n + 63) // 64 * 64
+    f1 = L1.W0f[: case.m * ldn * es].view(cuda.uint8).reshape(case.m, ldn * es)[:, : case.n * es]
+    f2 = L2.W0f[: case.m * ldn * es].view(cuda.uint8).reshape(case.m, ldn * es)[:, : case.n * es]
+    assert cuda.equal(f1, f2)
+    assert cuda.equal(y1, y2)
 
 
 # ------------------------------------------------------------------ GEMM engine
