@@ -39,6 +39,11 @@ WORKLOAD_SETS = {
 }
 METRIC = "POET layer fwd+bwd tokens/s at LLaMA-1.3B shapes; % of TC/HBM roofline"
 PLANS = {"auto": 0, "token": 1, "weight": 2}
+
+
+def row_stride(d):
+    """Row stride of the bench's activations: the width rounded up to 8 elements (16-byte aligned bf16 rows)."""
+    return (d + 7) // 8 * 8
 PLAN_NAMES = {1: "token", 2: "weight"}
 
 # DRAM traffic / algorithmic bytes of one launch, from an ncu capture, with the
@@ -67,6 +72,12 @@ def parse_args():
     ap.add_argument("--no-token-plan", action="store_true",
                     help="skip the second timed pass that runs every layer on the token plan")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (small profiling cases)")
+    ap.add_argument("--tokens", type=int, default=0, help="override the token count (small profiling cases)")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip timing the other LLaMA layer sets after the headline")
+    ap.add_argument("--probe", default="",
+                    help="measure only this one of the other layer sets or small-block probes and print its line "
+                         "(profiling)")
     return ap.parse_args()
 
 
@@ -178,23 +189,28 @@ class Variant:
         for a, b in nth:
             self.dslices.append((self.dtheta[off:off + a], self.dtheta[off + a:off + a + b]))
             off += a + b
-        # per-shape activations (each rank draws its own tokens)
+        # per-shape activations (each rank draws its own tokens), in rows whose
+        # stride is the width rounded up to 8 elements (16-byte aligned rows)
         self.x, self.dy, self.y, self.dx = {}, {}, {}, {}
+
+        def rows(d):
+            return torch.zeros(self.T, row_stride(d), dtype=tdt, device=device)[:, :d]
+
         def act(d, grad):
             key = (wl.seed + 7919 * rank, d, self.T, wl.dtype, grad)
             if key not in act_cache:  # the variants of one model see the same tokens
-                act_cache[key] = torch.from_numpy(
-                    I.activations(wl.seed + 7919 * rank, d, self.T, d, wl.dtype, grad=grad)).to(device=device,
-                                                                                             dtype=tdt)
+                t = rows(d)
+                t.copy_(torch.from_numpy(I.activations(wl.seed + 7919 * rank, d, self.T, d, wl.dtype, grad=grad)))
+                act_cache[key] = t
             return act_cache[key]
 
         for (m, n) in set(shapes):
             if n not in self.x:
                 self.x[n] = act(n, False)
-                self.dx[n] = torch.empty(self.T, n, dtype=tdt, device=device)
+                self.dx[n] = rows(n)
             if m not in self.dy:
                 self.dy[m] = act(m, True)
-                self.y[m] = torch.empty(self.T, m, dtype=tdt, device=device)
+                self.y[m] = rows(m)
         # saved activations: one buffer per linear position, shared by the variants (they run one after the other)
         self.saved = []
         for i, (_, _, _, _, L) in enumerate(self.layers):
@@ -206,9 +222,21 @@ class Variant:
                 else:
                     saved_pool.append(buf)
             self.saved.append(saved_pool[i])
-        self.ws_need = max(max(L.workspace_bytes(self.T), L.workspace_bytes(0)) for (_, _, _, _, L) in self.layers)
+        self.per_call = len(shapes)  # the grouped calls take one block's linears at a time
+        self.ws_need = self._ws_need()
         self.ws = None
         self.input_bytes = sum(v.numel() * v.element_size() for v in list(self.x.values()) + list(self.dy.values()))
+
+    def _ws_need(self):
+        from orthogonal_reparameterized_poet_b200 import poet
+
+        pl = [L for (_, _, _, _, L) in self.layers]
+        need = max(L.workspace_bytes(0) for L in pl)  # merge
+        for c0 in range(0, len(pl), self.per_call):
+            chunk = self.layers[c0:c0 + self.per_call]
+            need = max(need, poet.many_workspace_bytes([c[4] for c in chunk], self.T,
+                                                       [self.dy[c[2]] for c in chunk]))
+        return need
 
     def use_plan(self, plan, saved_pool, device):
         """Run every layer on `plan` from now on; grow the shared saved buffers to fit."""
@@ -223,7 +251,7 @@ class Variant:
                 saved_pool[i] = None
                 saved_pool[i] = torch.empty(need, dtype=torch.uint8, device=device)
             self.saved[i] = saved_pool[i]
-        self.ws_need = max(max(L.workspace_bytes(self.T), L.workspace_bytes(0)) for (_, _, _, _, L) in self.layers)
+        self.ws_need = self._ws_need()
 
     def plan_names(self):
         return "+".join(sorted({PLAN_NAMES[L.plan_for(self.T)] for (_, _, _, _, L) in self.layers}))
@@ -254,12 +282,16 @@ class Variant:
 
         pl = [L for (_, _, _, _, L) in self.layers]
         poet.cayley_neumann_many(pl)  # a1 for every primitive of every layer
-        for i, (_, _, m, n, L) in enumerate(self.layers):
-            L.forward(self.x[n], y=self.y[m], saved=self.saved[i], ws=self.ws)
-        for i in reversed(range(len(self.layers))):
-            _, _, m, n, L = self.layers[i]
-            L.backward_blocks(self.saved[i], self.dy[m], self.G[i][0], self.G[i][1], dx=self.dx[n], ws=self.ws,
-                              x=self.x[n])
+        k = self.per_call
+        for c0 in range(0, len(pl), k):  # a2..a4, one block's linears per grouped call
+            ch = self.layers[c0:c0 + k]
+            poet.forward_many([c[4] for c in ch], [self.x[c[3]] for c in ch], [self.y[c[2]] for c in ch],
+                              self.saved[c0:c0 + k], self.ws)
+        for c0 in reversed(range(0, len(pl), k)):  # a5..a7, blocks in reverse order
+            ch = self.layers[c0:c0 + k]
+            poet.backward_blocks_many([c[4] for c in ch], [self.x[c[3]] for c in ch], self.saved[c0:c0 + k],
+                                      [self.dy[c[2]] for c in ch], [self.dx[c[3]] for c in ch],
+                                      self.G[c0:c0 + k], self.ws)
         for c0 in range(0, len(pl), self.chunk):  # a8 for every layer, in grouped launches
             poet.cayley_neumann_grad_many(pl[c0:c0 + self.chunk], self.G[c0:c0 + self.chunk],
                                           self.dslices[c0:c0 + self.chunk], self.gws)
@@ -267,6 +299,18 @@ class Variant:
             from orthogonal_reparameterized_poet_b200 import dp
 
             dp.allreduce_gradients_(self.dtheta)
+
+    def merge_flop(self):
+        """Algorithmic flops of one merge of every linear: the R blocks on W0's
+        rows and the P blocks on its columns, 2 (c_R n s_R + m c_P s_P)."""
+        from orthogonal_reparameterized_poet_b200 import poet
+
+        total = 0.0
+        for (_, _, m, n, L) in self.layers:
+            nR, sR = poet.side_geometry(m, self.wl.mode, self.wl.b)
+            nP, sP = poet.side_geometry(n, self.wl.mode, self.wl.b)
+            total += 2.0 * (nR * sR * n * sR + m * nP * sP * sP)
+        return total
 
     def merge_all(self):
         for (_, _, _, _, L) in self.layers:
@@ -294,6 +338,116 @@ def kernel_table(rows, steps):
     return out
 
 
+def roofline_of(rows, version):
+    """Roofline of the dominant kind of a trace: achieved = its algorithmic flops
+    (or bytes) over its CUDA-event time, against the measured sustained bf16
+    peak (or the copy bandwidth) that its flop/byte ratio selects."""
+    peaks = load_peaks()
+    if not rows:
+        return None
+    dominant = max(rows, key=lambda k: rows[k]["ms"])
+    r = rows[dominant]
+    intensity = r["flop"] / r["bytes"] if r["bytes"] else float("inf")
+    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    avg_ms = r["ms"] / r["launches"]
+    if intensity >= ridge:
+        achieved = r["flop"] / (r["ms"] / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_kind": "bf16 sustained, " + peaks["source"]}
+    else:
+        achieved = r["bytes"] / (r["ms"] / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "unit": "GB/s", "peak_kind": "copy, " + peaks["source"]}
+    traffic = None
+    ratio = NCU_TRAFFIC_RATIO.get(dominant)
+    if ratio and ratio[1] in version:  # counters taken on this kernel revision
+        traffic = round(ratio[0] * r["bytes"] / r["launches"])
+    roof.update({"kernel": dominant, "achieved": round(achieved, 1), "peak": peak,
+                 "frac": round(achieved / peak, 4), "traffic": traffic, "avg_launch_ms": round(avg_ms, 4),
+                 "launches": r["launches"], "algorithmic_per_launch": {
+                     "flop": r["flop"] / r["launches"], "bytes": r["bytes"] / r["launches"]},
+                 "traffic_source": NCU_TRAFFIC_SOURCE})
+    return roof
+
+
+# The other layer sets of the pages' LLaMA family, measured after the headline
+# in the same run (each built, timed and freed in turn).
+OTHER_WORKLOADS = ["single256_fp32_bs32", "llama60m_fs", "llama350m_bs256", "llama3b_fs"]
+
+
+# Small primitives (size 32) at a token count whose block passes exceed L2: the
+# small-block kernels against the copy bandwidth (token plan).
+SMALLB_PROBES = {"smallb_fp32_b32_T262144": ("single256_fp32_bs32", {"tokens": 262144}),
+                 "smallb_bf16_b32_T262144": ("single256_fp32_bs32", {"tokens": 262144, "dtype": 1, "k": 4,
+                                                                    "sigma": 0.02})}
+
+
+def measure_workload(name, args, device, rank, plan, overrides=None):
+    """tokens/s of one workload's step (CUDA-graph replay, inputs resident), its
+    per-kind trace and dominant-kernel roofline, and its merge time."""
+    import dataclasses
+
+    import torch
+
+    from orthogonal_reparameterized_poet_b200 import inputs as I
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    wl = I.WORKLOADS[name]
+    if overrides:
+        wl = dataclasses.replace(wl, **overrides)
+    v = Variant(wl, rank, device, {}, {}, [], plan)
+    v.ws = torch.empty(max(v.ws_need, 1), dtype=torch.uint8, device=device)
+    gws_need = v.alloc_grads(device, chunk=4 * len(wl.linear_shapes()))
+    v.gws = torch.empty(max(gws_need, 1), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 1)):
+        v.step()
+    poet.poet_sync_status()
+    poet.poet_trace_enable(True)
+    for _ in range(args.steps):
+        v.step()
+    trace = poet.poet_trace_read()
+    poet.poet_trace_enable(False)
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    gph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gph, stream=cap):
+        v.step()
+    stream.wait_stream(cap)
+    gph.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        gph.replay()
+    b.record(stream)
+    b.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    poet.poet_sync_status()
+    m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    m0.record(stream)
+    v.merge_all()
+    m1.record(stream)
+    m1.synchronize()
+    poet.poet_sync_status()
+    rows = {k: dict(r) for k, r in trace.items()}
+    roof = roofline_of(rows, poet.poet_version())
+    out = {"tok_s": round(v.T / (ms / 1e3), 1), "ms": round(ms, 3), "tokens": v.T, "layers": wl.layers,
+           "mode": "FS" if wl.mode == I.FS else f"BS{wl.b}", "dtype": "f32" if wl.dtype == I.F32 else "bf16",
+           "plan": v.plan_names(), "merge_ms": round(m0.elapsed_time(m1), 3),
+           "merge_tflops": round(v.merge_flop() / (m0.elapsed_time(m1) / 1e3) / 1e12, 1),
+           "kernel": roof["kernel"] if roof else None, "bound": roof["bound"] if roof else None,
+           "frac": roof["frac"] if roof else None,
+           "per_kind_ms": {k: round(r["ms"] / args.steps, 3) for k, r in
+                           sorted(rows.items(), key=lambda kv: -kv[1]["ms"])[:6]}}
+    if overrides:  # probes: every kind's bandwidth and fraction of its roofline
+        out["kinds"] = {k: [r["gbs"], r["frac"], r["bound"]] for k, r in kernel_table(rows, args.steps).items()}
+    del gph, v
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_poet(args):
     import torch
 
@@ -318,10 +472,10 @@ def run_poet(args):
     poet.lib()
 
     wls = [I.WORKLOADS[name] for name in WORKLOAD_SETS[args.workload]]
-    if args.layers:
+    if args.layers or args.tokens:
         import dataclasses
 
-        wls = [dataclasses.replace(w, layers=args.layers) for w in wls]
+        wls = [dataclasses.replace(w, layers=args.layers or w.layers, tokens=args.tokens or w.tokens) for w in wls]
     w0_cache, act_cache, saved_pool = {}, {}, []
     variants = [Variant(wl, rank, device, w0_cache, act_cache, saved_pool, PLANS[args.plan]) for wl in wls]
     del w0_cache
@@ -486,32 +640,8 @@ def run_poet(args):
             dist.destroy_process_group()
         return
 
-    peaks = load_peaks()
     rows = {k: dict(v) for k, v in trace.items()}
-    dominant = max(rows, key=lambda k: rows[k]["ms"]) if rows else None
-    roof = None
-    if dominant:
-        r = rows[dominant]
-        intensity = r["flop"] / r["bytes"] if r["bytes"] else float("inf")
-        ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-        avg_ms = r["ms"] / r["launches"]
-        if intensity >= ridge:
-            achieved = r["flop"] / (r["ms"] / 1e3) / 1e12
-            peak = peaks["bf16_tflops_sustained"]
-            roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_kind": "bf16 sustained, " + peaks["source"]}
-        else:
-            achieved = r["bytes"] / (r["ms"] / 1e3) / 1e9
-            peak = peaks["hbm_gbs"]
-            roof = {"bound": "hbm", "unit": "GB/s", "peak_kind": "copy, " + peaks["source"]}
-        traffic = None
-        ratio = NCU_TRAFFIC_RATIO.get(dominant)
-        if ratio and ratio[1] in poet.poet_version():  # counters taken on this kernel revision
-            traffic = round(ratio[0] * r["bytes"] / r["launches"])
-        roof.update({"kernel": dominant, "achieved": round(achieved, 1), "peak": peak,
-                     "frac": round(achieved / peak, 4), "traffic": traffic, "avg_launch_ms": round(avg_ms, 4),
-                     "launches": r["launches"], "algorithmic_per_launch": {
-                         "flop": r["flop"] / r["launches"], "bytes": r["bytes"] / r["launches"]},
-                     "traffic_source": NCU_TRAFFIC_SOURCE})
+    roof = roofline_of(rows, poet.poet_version())
     kernels = kernel_table(rows, args.steps)
 
     cpu = None
@@ -529,10 +659,14 @@ def run_poet(args):
                    "variants": [{"name": v.wl.name, "mode": "FS" if v.wl.mode == I.FS else "BS", "b": v.wl.b,
                                  "k": v.wl.k, "plan": plans_run[i]} for i, v in enumerate(variants)],
                    "plan_requested": args.plan,
-                   "parallelism": f"dp{world}", "l2": "inputs larger than L2 (no flush needed)"},
+                   "parallelism": f"dp{world}", "l2": "inputs larger than L2 (no flush needed)",
+                   "activation_rows": "row stride = width rounded up to 8 elements (16-byte aligned rows)",
+                   "linears_per_call": variants[0].per_call},
         "variants": {v.wl.name: {"ms_per_step": round(per_variant_ms[i] / args.steps, 3),
                                  "tokens_per_s": round(v.T * world / (per_variant_ms[i] / args.steps / 1e3), 1),
                                  "merge_ms": round(merge.get(v.wl.name, float("nan")), 3) if merge else None,
+                                 "merge_tflops": (round(v.merge_flop() / (merge[v.wl.name] / 1e3) / 1e12, 1)
+                                                  if merge else None),
                                  "kernels_ms_per_step": {k: round(r["ms"] / args.steps, 2) for k, r in
                                                          sorted(traces[i].items(), key=lambda kv: -kv[1]["ms"])}}
                      for i, v in enumerate(variants)},
@@ -543,6 +677,25 @@ def run_poet(args):
         "roofline": roof, "kernels": kernels, "gpu_launches": int(launches), "clocks": clk,
         "e2e": e2e, "cpu_baseline": cpu, "token_plan": token,
     }
+    out["roofline"]["per_kind_ms_frac"] = {k: [r["ms_per_step"], r["frac"], r["bound"]] for k, r in kernels.items()}
+    if not args.no_other_workloads and world == 1:
+        # the other layer sets, one at a time, after the headline's buffers are freed
+        del variants, ws, gws, saved_pool, act_cache, graphs, e2e, token
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        others = {}
+        for name in OTHER_WORKLOADS:
+            others[name] = measure_workload(name, args, device, rank, PLANS[args.plan])
+            if not args.no_cpu_baseline:
+                wl = I.WORKLOADS[name]
+                full = wl.tokens * wl.layers <= 4096  # the small sets: every token of the layer set
+                one = cpu_baseline([wl], budget_s=6.0, threads=1, full=full)
+                allc = cpu_baseline([wl], budget_s=6.0, full=full)
+                others[name].update({"cpu_1t_tok_s": one["value"], "cpu_all_tok_s": allc["value"],
+                                     "cpu_cores": allc["cores"], "cpu_full": full})
+        for name, (base, ov) in SMALLB_PROBES.items():
+            others[name] = measure_workload(base, args, device, rank, PLANS["token"], ov)
+        out["workloads"] = others
     print(json.dumps(out), flush=True)
     if dist is not None:
         dist.destroy_process_group()
@@ -560,14 +713,20 @@ def run_e2e(args, variants, world):
 
     stream = torch.cuda.current_stream()
     copy = torch.cuda.Stream()
-    # device inputs: set 0 = the tensors the variants hold, set 1 = copies (one per distinct tensor)
+    def whole_rows(t):
+        """The activation's padded rows (a dense view), so that copies of it are plain memory copies."""
+        return t.as_strided((t.shape[0], t.stride(0)), (t.stride(0), 1)) if t.dim() == 2 else t
+
+    # device inputs: set 0 = the tensors the variants hold, set 1 = copies (one per distinct tensor),
+    # each in the same padded row layout
     uniq = {}
     for v in variants:
         for d in (v.x, v.dy):
             for t in d.values():
                 uniq[id(t)] = t
-    sets = [{k: t for k, t in uniq.items()}, {k: torch.empty_like(t) for k, t in uniq.items()}]
-    host_in = {k: t.cpu().pin_memory() for k, t in uniq.items()}
+    second = {k: torch.empty_like(whole_rows(t))[:, : t.shape[1]] for k, t in uniq.items()}
+    sets = [{k: t for k, t in uniq.items()}, second]
+    host_in = {k: whole_rows(t).cpu().pin_memory() for k, t in uniq.items()}
     base = [({n: t for n, t in v.x.items()}, {m: t for m, t in v.dy.items()}) for v in variants]
 
     def use_set(sidx):
@@ -579,7 +738,7 @@ def run_e2e(args, variants, world):
     outs = []
     for v in variants:
         last_m, last_n = v.layers[0][2], v.layers[0][3]
-        outs += [v.dtheta, v.y[last_m], v.dx[last_n]]
+        outs += [v.dtheta, whole_rows(v.y[last_m]), whole_rows(v.dx[last_n])]
     snap = [[torch.empty_like(t) for t in outs] for _ in range(2)]
     host_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs] for _ in range(2)]
     h2d = sum(h.numel() * h.element_size() for h in host_in.values())
@@ -612,7 +771,7 @@ def run_e2e(args, variants, world):
             if after_use:
                 copy.wait_event(ev_used[sidx])
             for k, h in host_in.items():
-                sets[sidx][k].copy_(h, non_blocking=True)
+                whole_rows(sets[sidx][k]).copy_(h, non_blocking=True)
             ev_in[sidx].record(copy)
 
     def run(steps):
@@ -659,9 +818,20 @@ def run_e2e(args, variants, world):
 
 # ---------------------------------------------------------------------------- CPU oracle
 
-def cpu_baseline(wls, budget_s=25.0):
+def cpu_baseline(wls, budget_s=25.0, threads=None, full=False):
     """The float64 CPU oracle, as it stands, on a bounded sample of the same
-    workload, extrapolated to the full step in tokens/s."""
+    workload, extrapolated to the full step in tokens/s (full: every token of
+    one layer set).  threads: BLAS threads to allow (None: as configured)."""
+    import contextlib
+
+    from threadpoolctl import threadpool_info, threadpool_limits
+
+    ctx = threadpool_limits(limits=threads, user_api="blas") if threads else contextlib.nullcontext()
+    with ctx:
+        return _cpu_baseline(wls, budget_s, full)
+
+
+def _cpu_baseline(wls, budget_s, full):
     import numpy as np
     from threadpoolctl import threadpool_info
 
@@ -674,7 +844,7 @@ def cpu_baseline(wls, budget_s=25.0):
     t_start = time.perf_counter()
     for wl in wls:
         shapes = wl.linear_shapes()
-        Ts = 64
+        Ts = wl.tokens if full else 64
         # token-independent part: Cayley-Neumann forward + backward, once per distinct primitive size
         cnp_s = {}
         for (m, n) in set(shapes):
@@ -717,7 +887,8 @@ def cpu_baseline(wls, budget_s=25.0):
         total_s += per_layer * wl.layers
         total_tokens += wl.tokens
         sample_desc.append(f"{wl.name}: Cayley-Neumann fwd+bwd once per distinct primitive size "
-                           f"{sorted(cnp_s)}, dense fwd+bwd of {Ts} tokens once per distinct linear shape")
+                           f"{sorted(cnp_s)}, dense fwd+bwd of {Ts} tokens once per distinct linear shape"
+                           + ("" if Ts < wl.tokens else " (all tokens)"))
         if time.perf_counter() - t_start > budget_s:
             break
     wall = time.perf_counter() - t_start
@@ -754,8 +925,26 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_probe(args):
+    import torch
+
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    torch.cuda.set_device(0)
+    poet.lib()
+    if args.probe in SMALLB_PROBES:
+        base, ov = SMALLB_PROBES[args.probe]
+        res = measure_workload(base, args, torch.device("cuda", 0), 0, PLANS["token"], ov)
+    else:
+        res = measure_workload(args.probe, args, torch.device("cuda", 0), 0, PLANS[args.plan])
+    print(json.dumps({"probe": args.probe, **res}), flush=True)
+
+
 def main():
     args = parse_args()
+    if args.probe:
+        run_probe(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

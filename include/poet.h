@@ -244,6 +244,43 @@ POET_API poet_status poet_backward_blocks(const poet_layer *L, const void *x, co
                                           const void *dy, int64_t T, void *dx, float *G_R,
                                           float *G_P, void *ws, size_t ws_bytes, poet_stream stream);
 
+/* ---- many layers' forward and backward
+ *
+ * The forward and a5..a7 of count independent layers (for example every
+ * linear of a layer set whose inputs are all at hand, or q, k and v of one
+ * block, which share their input).  Same results as poet_forward and
+ * poet_backward_blocks on each layer (the per-primitive gradients, whose
+ * products are summed over split ranges, agree to rounding); the difference
+ * is the launches: under the weight plan the weight-sized products of every
+ * layer share grouped tensor-core launches, their permutations share one
+ * launch, and the T-sized GEMMs of all layers run as one grouped launch.
+ * Token-plan layers in the list run one after another.
+ *  - layers: count complete layers of one element type (state from
+ *    poet_cayley_neumann, W0f from poet_prepare / poet_resample / poet_merge),
+ *    each with its plan as poet_plan_for(&layers[i], T) says.
+ *  - x[i] (T x n_i), y[i] (T x m_i), dy[i] (T x m_i), dx[i] (T x n_i): device,
+ *    row-major with row strides ldx[i], ldy[i], lddy[i], lddx[i] elements
+ *    (>= the width; a NULL stride list means contiguous rows).  Rows whose
+ *    start is 16-byte aligned (stride x element size a multiple of 16, base
+ *    16-byte aligned) are read and written in place; other x and dy rows are
+ *    first copied into 16-byte aligned rows.
+ *  - saved[i]: device, poet_saved_bytes(&layers[i], T) bytes, 256-byte aligned.
+ *  - G_R[i], G_P[i]: device, poet_block_grad_bytes each, 16-byte aligned,
+ *    overwritten.
+ *  - ws: device, poet_many_workspace_bytes(layers, count, T, lddy) bytes,
+ *    256-byte aligned; one size serves both calls. */
+POET_API size_t poet_many_workspace_bytes(const poet_layer *layers, int32_t count, int64_t T, const int64_t *lddy);
+
+POET_API poet_status poet_forward_many(const poet_layer *layers, int32_t count, const void *const *x,
+                                       const int64_t *ldx, int64_t T, void *const *y, const int64_t *ldy,
+                                       void *const *saved, void *ws, size_t ws_bytes, poet_stream stream);
+
+POET_API poet_status poet_backward_blocks_many(const poet_layer *layers, int32_t count, const void *const *x,
+                                               const int64_t *ldx, const void *const *saved,
+                                               const void *const *dy, const int64_t *lddy, int64_t T,
+                                               void *const *dx, const int64_t *lddx, float *const *G_R,
+                                               float *const *G_P, void *ws, size_t ws_bytes, poet_stream stream);
+
 /* Workspace bytes of poet_cayley_neumann_grad_many for these sides. */
 POET_API size_t poet_cayley_neumann_grad_many_workspace_bytes(const poet_side *sides, int32_t count,
                                                               int32_t dtype);
@@ -302,6 +339,39 @@ POET_API poet_status poet_draw_perm(uint64_t seed, int32_t layer_id, int32_t sid
 POET_API poet_status poet_adamw_step(float *theta, const float *grad, float *m, float *v, int64_t n,
                                      float lr, float beta1, float beta2, float eps, float weight_decay,
                                      int32_t step, poet_stream stream);
+
+/* AdamW hyperparameters of one step (see poet_adamw_step). */
+typedef struct {
+  float lr, beta1, beta2, eps, weight_decay;
+  int32_t step;    /* >= 1: updates so far including this one */
+} poet_adamw_hparams;
+
+/* a8 for count sides, with the AdamW step of poet_adamw_step applied to each
+ * side's theta (in place, side->theta) in the same kernel that packs the
+ * gradient: per parameter the gradient is formed, the moments m[i], v[i]
+ * (device float, theta layout) are updated and theta moves, with no pass of
+ * the gradient through memory.  dtheta[i] may be NULL (not written) or a
+ * buffer that also receives the gradient.  Same gradient as
+ * poet_cayley_neumann_grad_many, same update as poet_adamw_step on it.
+ * Workspace as poet_cayley_neumann_grad_many.  For data-parallel training,
+ * where the gradient is summed over ranks before the update, use
+ * poet_cayley_neumann_grad_many, the all-reduce, then poet_adamw_step. */
+POET_API poet_status poet_cayley_neumann_grad_many_adamw(const poet_side *sides, const float *const *G,
+                                                         float *const *m, float *const *v,
+                                                         float *const *dtheta, int32_t count, int32_t dtype,
+                                                         const poet_adamw_hparams *h, void *ws, size_t ws_bytes,
+                                                         poet_stream stream);
+
+/* poet_merge, then the AdamW moments of both sides reset to zero (the
+ * parameters restart at theta = 0; the caller restarts its step count).
+ * m_R, v_R: device float[R's theta length]; m_P, v_P: the same for P (any of
+ * them may be NULL when that side has no parameters). */
+POET_API poet_status poet_merge_reset_moments(poet_layer *L, float *m_R, float *v_R, float *m_P, float *v_P,
+                                              void *ws, size_t ws_bytes, poet_stream stream);
+
+/* The workspace size query under the name of the pages' boundary sketch: the
+ * same value as poet_workspace_bytes. */
+POET_API size_t poet_workspace_size(const poet_layer *L, int64_t T);
 
 /* ---------------------------------------------------------------- utilities */
 

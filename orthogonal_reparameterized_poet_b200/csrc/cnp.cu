@@ -5,7 +5,19 @@
 // map (I+Q)(I-Q)^-1 of a skew-symmetric Q with the inverse replaced by its
 // Neumann series truncated after Q^k:  B = (I + Q)(I + Q + ... + Q^k).
 //
-// Forward, by Horner's rule on the series:
+// Order 4 (the order the pages' LLaMA runs use) is evaluated by powers of
+// S = Q^2, with T = S^2:
+//   B = Q C + D0,   C = 2I + 2S + T,   D0 = I + 2S + 2T
+// (3 GEMMs).  The state keeps Q, S, C, T and D0.  Its gradient, G = dL/dB:
+// theta enters Q antisymmetrically (Q[a,c] = theta = -Q[c,a]), so only the
+// antisymmetric part of dL/dQ reaches dtheta; S, T and C are symmetric, so
+// only the symmetric parts of dL/dS and dL/dT matter:
+//   QG = Q G,  GC = G C,  dT_s = sym(2G - QG),  W = dT_s S,
+//   dS_s = sym(2G - 2 QG) + W + W^T,  Y = dS_s Q,  D = G C - 2 Y,
+//   dtheta[a,c] = D[a,c] - D[c,a]                       (sym(X) = (X + X^T)/2)
+// (4 GEMMs, in three grouped launches).
+//
+// Every other order, by Horner's rule on the series:
 //   S_1 = I + Q,  S_{l+1} = I + Q S_l (l = 1..k-1),  B = (I + Q) S_k = S_1 S_k
 // (k GEMMs of size^3; k = 0 gives B = I + Q).  Q and S_1..S_k are kept in
 // the side state for the backward.
@@ -30,27 +42,8 @@ __device__ __forceinline__ int64_t packed_index(int a, int c, int size) {
 template <typename T> __device__ __forceinline__ T from_f(float v);
 template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
-
-// Q and S_1 = I + Q (or B = I + Q when k == 0) for every primitive; padding is zero.
-template <typename T>
-__global__ void unpack_kernel(const float *__restrict__ theta, int nprim, int size, int ld,
-                              T *__restrict__ Q, T *__restrict__ IplusQ) {
-  const int64_t blk = int64_t(ld) * ld;
-  const int64_t total = blk * nprim;
-  const int64_t per = int64_t(size) * (size - 1) / 2;
-  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
-    const int j = int(e / blk);
-    const int a = int((e % blk) / ld), c = int(e % ld);
-    float q = 0.f, eye = 0.f;
-    if (a < size && c < size) {
-      if (a < c) q = theta[j * per + packed_index(a, c, size)];
-      else if (a > c) q = -theta[j * per + packed_index(c, a, size)];
-      else eye = 1.f;
-    }
-    Q[e] = from_f<T>(q);
-    IplusQ[e] = from_f<T>(q + eye);
-  }
-}
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(bf16 v) { return __bfloat162float(v); }
 
 // dtheta[j][idx(a,c)] = D[a,c] - D[c,a] with D = dQ (+ A1 when given)
 __global__ void pack_grad_kernel(const float *__restrict__ dQ, const float *__restrict__ A1, int nprim, int size,
@@ -86,6 +79,13 @@ __global__ void f32_to_bf16_kernel(const float *__restrict__ in, bf16 *__restric
   for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x)
     out[e] = __float2bfloat16_rn(in[e]);
 }
+
+}  // namespace
+
+// Order 4 is evaluated by powers of S = Q^2 (see the top of this file).
+bool by_powers(const SideGeom &g) { return g.k == 4; }
+
+namespace {
 
 int grid_for(int64_t n, int threads) {
   int64_t g = (n + threads - 1) / threads;
@@ -126,40 +126,17 @@ size_t cnp_scratch_bytes(const SideGeom &g, int dtype) {
 }
 
 poet_status cnp_forward(const poet_side *side, const SideGeom &g, int dtype, cudaStream_t st) {
-  if (g.nprim == 0) return POET_OK;
-  const StateLayout L = state_layout(g, dtype);
-  char *base = static_cast<char *>(side->state);
-  void *R = base + L.R, *Q = base + L.Q;
-  const int64_t n = g.all_elems();
-  void *first = g.k == 0 ? R : static_cast<void *>(base + L.S1);
-  if (dtype == POET_BF16)
-    unpack_kernel<bf16><<<grid_for(n, 256), 256, 0, st>>>(side->theta, g.nprim, g.size, g.ld, static_cast<bf16 *>(Q),
-                                                          static_cast<bf16 *>(first));
-  else
-    unpack_kernel<float><<<grid_for(n, 256), 256, 0, st>>>(side->theta, g.nprim, g.size, g.ld, static_cast<float *>(Q),
-                                                           static_cast<float *>(first));
-  count_launch();
-  POET_TRY(launch_status("cnp unpack"));
-  for (int l = 1; l <= g.k; ++l) {
-    void *S = base + L.S1 + size_t(l - 1) * L.term;
-    Gemm p;
-    if (l < g.k) {                               // S_{l+1} = I + Q S_l
-      p = prim_gemm(g, dtype, Q, S, false, "cnp_fwd");
-      p.diag = 1.f;
-      p.outD = base + L.S1 + size_t(l) * L.term;
-    } else {                                     // B = (I + Q) S_k = S_1 S_k
-      p = prim_gemm(g, dtype, base + L.S1, S, false, "cnp_fwd");
-      p.outD = R;
-    }
-    p.od_m = g.ld; p.od_b = g.blk_elems();
-    POET_TRY(gemm_run(p, st));
-  }
-  return POET_OK;
+  return cnp_forward_many(side, &g, 1, dtype, st);  // one code path: a single side is a list of one
 }
 
 poet_status cnp_backward(const poet_side *side, const SideGeom &g, int dtype, const float *G, float *dtheta,
                          void *scratch, cudaStream_t st) {
   if (g.nprim == 0 || g.size < 2) return POET_OK;
+  if (by_powers(g)) {  // order 4: the grouped path on a list of one side (cnp_scratch_bytes >= its scratch)
+    void *sc = scratch;
+    float *dth = dtheta;
+    return cnp_backward_many(side, &g, 1, dtype, &G, &dth, &sc, st);
+  }
   const StateLayout L = state_layout(g, dtype);
   char *base = static_cast<char *>(side->state);
   const void *Q = base + L.Q;
@@ -228,8 +205,9 @@ poet_status cnp_backward(const poet_side *side, const SideGeom &g, int dtype, co
 // ---------------------------------------------------------------- many sides
 //
 // The element-wise steps of many sides (unpacking theta, rounding G to the
-// operand type, packing dQ into dtheta) run as one launch per step over a
-// table of up to kSidesMax sides; each block works inside one side.
+// operand type, the symmetric combinations of the order-4 gradient, packing
+// dQ into dtheta) run as one launch per step over a table of up to kSidesMax
+// sides; each block works inside one side.
 
 namespace {
 
@@ -240,12 +218,20 @@ struct SideTable {
   int count;
   int64_t block_start[kSidesMax + 1];
   const void *src[kSidesMax];
+  const void *src2[kSidesMax];
+  const void *src3[kSidesMax];
   void *dst[kSidesMax];
   void *dst2[kSidesMax];
+  void *dst3[kSidesMax];
   int nprim[kSidesMax], size[kSidesMax], ld[kSidesMax];
   int terms[kSidesMax];          // pack: partial products summed onto src
   int64_t stride[kSidesMax];     // pack: floats between partial products
+  float coef[kSidesMax];         // pack: weight of the partial products
+  float *theta[kSidesMax];       // pack with an optimizer step: parameters, first and second moments
+  float *m1[kSidesMax];
+  float *m2[kSidesMax];
 };
+static_assert(sizeof(SideTable) <= 32000, "side table exceeds the kernel parameter limit");
 
 __device__ __forceinline__ int side_of_block(const SideTable &t) {
   int lo = 0, hi = t.count - 1;
@@ -256,7 +242,9 @@ __device__ __forceinline__ int side_of_block(const SideTable &t) {
   return lo;
 }
 
-// unpack_kernel for many sides: src = theta, dst = Q, dst2 = S_1 (or B when k = 0)
+// src = theta, dst = Q, dst2 = S_1 = I + Q (or B = I + Q when k = 0; nullptr:
+// not written), dst3 = B whose padding (rows or columns >= size) is zeroed
+// (nullptr: none).  Padding of Q and S_1 is zero.
 template <typename T>
 __global__ void __launch_bounds__(256) unpack_many_kernel(const __grid_constant__ SideTable t) {
   const int i = side_of_block(t);
@@ -266,19 +254,49 @@ __global__ void __launch_bounds__(256) unpack_many_kernel(const __grid_constant_
   const float *theta = static_cast<const float *>(t.src[i]);
   T *Q = static_cast<T *>(t.dst[i]);
   T *IplusQ = static_cast<T *>(t.dst2[i]);
+  T *Bpad = static_cast<T *>(t.dst3[i]);
   const int64_t e0 = (int64_t(blockIdx.x) - t.block_start[i]) * (256 * kItems);
   const int64_t e1 = e0 + 256 * kItems < total ? e0 + 256 * kItems : total;
   for (int64_t e = e0 + threadIdx.x; e < e1; e += 256) {
     const int j = int(e / blk);
     const int a = int((e % blk) / ld), c = int(e % ld);
     float q = 0.f, eye = 0.f;
-    if (a < size && c < size) {
+    const bool inside = a < size && c < size;
+    if (inside) {
       if (a < c) q = theta[j * per + packed_index(a, c, size)];
       else if (a > c) q = -theta[j * per + packed_index(c, a, size)];
       else eye = 1.f;
     }
     Q[e] = from_f<T>(q);
-    IplusQ[e] = from_f<T>(q + eye);
+    if (IplusQ) IplusQ[e] = from_f<T>(q + eye);
+    if (Bpad && !inside) Bpad[e] = from_f<T>(0.f);
+  }
+}
+
+// Order 4: from S (src) and T = S^2 (src2), C = 2I + 2S + T (dst) and
+// D0 = I + 2S + 2T (dst2); padding zero.
+template <typename T>
+__global__ void __launch_bounds__(256) powers_combine_kernel(const __grid_constant__ SideTable t) {
+  const int i = side_of_block(t);
+  const int size = t.size[i], ld = t.ld[i];
+  const int64_t blk = int64_t(ld) * ld, total = blk * t.nprim[i];
+  const T *S = static_cast<const T *>(t.src[i]);
+  const T *Tp = static_cast<const T *>(t.src2[i]);
+  T *C = static_cast<T *>(t.dst[i]);
+  T *D0 = static_cast<T *>(t.dst2[i]);
+  const int64_t e0 = (int64_t(blockIdx.x) - t.block_start[i]) * (256 * kItems);
+  const int64_t e1 = e0 + 256 * kItems < total ? e0 + 256 * kItems : total;
+  for (int64_t e = e0 + threadIdx.x; e < e1; e += 256) {
+    const int a = int((e % blk) / ld), c = int(e % ld);
+    float cv = 0.f, dv = 0.f;
+    if (a < size && c < size) {
+      const float sv = to_f(S[e]), tv = to_f(Tp[e]);
+      const float eye = a == c ? 1.f : 0.f;
+      cv = 2.f * eye + 2.f * sv + tv;
+      dv = eye + 2.f * sv + 2.f * tv;
+    }
+    C[e] = from_f<T>(cv);
+    D0[e] = from_f<T>(dv);
   }
 }
 
@@ -293,50 +311,130 @@ __global__ void __launch_bounds__(256) round_many_kernel(const __grid_constant__
   for (int64_t e = e0 + threadIdx.x; e < e1; e += 256) out[e] = __float2bfloat16_rn(G[e]);
 }
 
-// dst = dtheta: dtheta[j][idx(a,c)] = D[a][c] - D[c][a] with D = src +
-// sum_{t < terms} dst2 + t * stride (all float [nprim][ld][ld]).  One block
-// per pair of 32 x 32 tiles (ta <= tc) of one primitive; both tiles are summed
-// row-contiguously into shared memory and the transposed read comes from there.
-__global__ void __launch_bounds__(256) pack_many_kernel(const __grid_constant__ SideTable t) {
-  __shared__ float t1[PACK_T][PACK_T + 1], t2[PACK_T][PACK_T + 1];
-  const int i = side_of_block(t);
-  const int size = t.size[i], ld = t.ld[i];
+// Tile pair (ta <= tc, 32 x 32 tiles) of primitive j handled by this block.
+struct TilePair {
+  int j, ta, tc;
+};
+__device__ __forceinline__ TilePair tile_pair(const SideTable &t, int i) {
+  const int size = t.size[i];
   const int tiles = (size + PACK_T - 1) / PACK_T;
   const int pairs = tiles * (tiles + 1) / 2;
   const int64_t local = int64_t(blockIdx.x) - t.block_start[i];
-  const int j = int(local / pairs);
+  TilePair p;
+  p.j = int(local / pairs);
   int ta = 0, rem = int(local % pairs);
   while (rem >= tiles - ta) { rem -= tiles - ta; ++ta; }
-  const int tc = ta + rem;
-  const int64_t off = int64_t(j) * ld * ld;
+  p.ta = ta;
+  p.tc = ta + rem;
+  return p;
+}
+
+// Order-4 gradient, symmetric combinations: dst = sum_q c_q (X_q + X_q^T)
+// over X_0 = src, X_1 = src2 and X_2 = src3 (float [nprim][ld][ld]; src3 may
+// be nullptr), in the operand type.  One block per pair of 32 x 32 tiles
+// (ta <= tc) of one primitive; both tiles of every input are read
+// row-contiguously into shared memory and both output tiles are written.
+template <typename T>
+__global__ void __launch_bounds__(256) sym_many_kernel(const __grid_constant__ SideTable t, float c0, float c1,
+                                                        float c2) {
+  __shared__ float u1[PACK_T][PACK_T + 1], u2[PACK_T][PACK_T + 1];
+  const int i = side_of_block(t);
+  const int size = t.size[i], ld = t.ld[i];
+  const TilePair tp = tile_pair(t, i);
+  const int64_t off = int64_t(tp.j) * ld * ld;
+  const float *X[3] = {static_cast<const float *>(t.src[i]), static_cast<const float *>(t.src2[i]),
+                       static_cast<const float *>(t.src3[i])};
+  const float cf[3] = {c0, c1, c2};
+  T *out = static_cast<T *>(t.dst[i]) + off;
+  const int x = threadIdx.x % PACK_T;
+  // u1[y][x] = sum c_q X_q[ta*32+y][tc*32+x],  u2[y][x] = sum c_q X_q[tc*32+y][ta*32+x]
+  for (int y = threadIdx.x / PACK_T; y < PACK_T; y += 256 / PACK_T) {
+    const int a1 = tp.ta * PACK_T + y, b1 = tp.tc * PACK_T + x;
+    const int a2 = tp.tc * PACK_T + y, b2 = tp.ta * PACK_T + x;
+    float v1 = 0.f, v2 = 0.f;
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      if (!X[q]) continue;
+      if (a1 < size && b1 < size) v1 += cf[q] * X[q][off + int64_t(a1) * ld + b1];
+      if (a2 < size && b2 < size) v2 += cf[q] * X[q][off + int64_t(a2) * ld + b2];
+    }
+    u1[y][x] = v1;
+    u2[y][x] = v2;
+  }
+  __syncthreads();
+  // out[ta*32+y][tc*32+x] = u1[y][x] + u2[x][y];  out[tc*32+y][ta*32+x] = u2[y][x] + u1[x][y]
+  for (int y = threadIdx.x / PACK_T; y < PACK_T; y += 256 / PACK_T) {
+    const int a1 = tp.ta * PACK_T + y, b1 = tp.tc * PACK_T + x;
+    const int a2 = tp.tc * PACK_T + y, b2 = tp.ta * PACK_T + x;
+    if (a1 < size && b1 < size) out[int64_t(a1) * ld + b1] = from_f<T>(u1[y][x] + u2[x][y]);
+    if (tp.ta != tp.tc && a2 < size && b2 < size) out[int64_t(a2) * ld + b2] = from_f<T>(u2[y][x] + u1[x][y]);
+  }
+}
+
+// dst = dtheta: dtheta[j][idx(a,c)] = D[a][c] - D[c][a] with D = src +
+// coef * sum_{q < terms} dst2 + q * stride (all float [nprim][ld][ld]).  One
+// block per pair of 32 x 32 tiles (ta <= tc) of one primitive; both tiles are
+// summed row-contiguously into shared memory and the transposed read comes
+// from there.  With ADAM, each parameter's gradient also drives its AdamW
+// step (theta, m1, m2 updated in place; dst may be nullptr).
+template <bool ADAM>
+__global__ void __launch_bounds__(256) pack_many_kernel(const __grid_constant__ SideTable t, const AdamW h) {
+  __shared__ float t1[PACK_T][PACK_T + 1], t2[PACK_T][PACK_T + 1];
+  const int i = side_of_block(t);
+  const int size = t.size[i], ld = t.ld[i];
+  const TilePair tp = tile_pair(t, i);
+  const int64_t off = int64_t(tp.j) * ld * ld;
   const float *dQ = static_cast<const float *>(t.src[i]) + off;
   const int terms = t.terms[i];
+  const float coef = t.coef[i];
   const float *P = terms ? static_cast<const float *>(t.dst2[i]) + off : nullptr;
   const int64_t stride = t.stride[i];
-  float *dtheta = static_cast<float *>(t.dst[i]) + int64_t(j) * (int64_t(size) * (size - 1) / 2);
+  float *dtheta = t.dst[i] ? static_cast<float *>(t.dst[i]) + int64_t(tp.j) * (int64_t(size) * (size - 1) / 2)
+                           : nullptr;
   const int x = threadIdx.x % PACK_T;
   for (int y = threadIdx.x / PACK_T; y < PACK_T; y += 256 / PACK_T) {
-    const int a1 = ta * PACK_T + y, c1 = tc * PACK_T + x;
-    const int a2 = tc * PACK_T + y, c2 = ta * PACK_T + x;
+    const int a1 = tp.ta * PACK_T + y, c1 = tp.tc * PACK_T + x;
+    const int a2 = tp.tc * PACK_T + y, c2 = tp.ta * PACK_T + x;
     float v1 = 0.f, v2 = 0.f;
     if (a1 < size && c1 < size) {
       const int64_t o = int64_t(a1) * ld + c1;
-      v1 = dQ[o];
-      for (int q = 0; q < terms; ++q) v1 += P[q * stride + o];
+      float acc = 0.f;
+      for (int q = 0; q < terms; ++q) acc += P[q * stride + o];
+      v1 = dQ[o] + coef * acc;
     }
     if (a2 < size && c2 < size) {
       const int64_t o = int64_t(a2) * ld + c2;
-      v2 = dQ[o];
-      for (int q = 0; q < terms; ++q) v2 += P[q * stride + o];
+      float acc = 0.f;
+      for (int q = 0; q < terms; ++q) acc += P[q * stride + o];
+      v2 = dQ[o] + coef * acc;
     }
     t1[y][x] = v1;
     t2[y][x] = v2;
   }
   __syncthreads();
+  const int64_t pbase = int64_t(tp.j) * (int64_t(size) * (size - 1) / 2);
   for (int y = threadIdx.x / PACK_T; y < PACK_T; y += 256 / PACK_T) {
-    const int a = ta * PACK_T + y, c = tc * PACK_T + x;
-    if (a < c && c < size) dtheta[packed_index(a, c, size)] = t1[y][x] - t2[x][y];
+    const int a = tp.ta * PACK_T + y, c = tp.tc * PACK_T + x;
+    if (a < c && c < size) {
+      const int64_t idx = packed_index(a, c, size);
+      const float g = t1[y][x] - t2[x][y];
+      if (!ADAM || t.dst[i]) dtheta[idx] = g;
+      if constexpr (ADAM) {
+        const int64_t e = pbase + idx;
+        float th = t.theta[i][e], mm = t.m1[i][e], vv = t.m2[i][e];
+        adamw_one(th, g, mm, vv, h);
+        t.theta[i][e] = th;
+        t.m1[i][e] = mm;
+        t.m2[i][e] = vv;
+      }
+    }
   }
+}
+
+int64_t elem_blocks(const SideGeom &g) { return (g.all_elems() + 256 * kItems - 1) / (256 * kItems); }
+int64_t pair_blocks(const SideGeom &g) {
+  const int64_t tiles = (g.size + PACK_T - 1) / PACK_T;
+  return int64_t(g.nprim) * tiles * (tiles + 1) / 2;
 }
 
 // Fill a table with the sides of idx[0..n) (blocks per side from `blocks`) and launch.
@@ -346,24 +444,46 @@ poet_status many_launch(const std::vector<int> &idx, Blocks blocks, SideTable &t
     const int n = int(idx.size() - c0 < size_t(kSidesMax) ? idx.size() - c0 : size_t(kSidesMax));
     t.count = n;
     t.block_start[0] = 0;
-    for (int q = 0; q < n; ++q) t.block_start[q + 1] = t.block_start[q] + blocks(idx[c0 + q], q);
+    for (int q = 0; q < n; ++q) {
+      t.src[q] = t.src2[q] = t.src3[q] = nullptr;
+      t.dst[q] = t.dst2[q] = t.dst3[q] = nullptr;
+      t.theta[q] = t.m1[q] = t.m2[q] = nullptr;
+      t.terms[q] = 0;
+      t.stride[q] = 0;
+      t.coef[q] = 1.f;
+      t.block_start[q + 1] = t.block_start[q] + blocks(idx[c0 + q], q);
+    }
     if (t.block_start[n] == 0) continue;
     POET_TRY(launch(t, int(c0), n));
   }
   return POET_OK;
 }
 
+// Byte offsets of the order-4 terms in a side state: S, C, T, D0 take the
+// slots of S_1..S_4.
+struct PowersLayout {
+  size_t S, C, T, D0;
+};
+PowersLayout powers_layout(const StateLayout &L) {
+  return {L.S1, L.S1 + L.term, L.S1 + 2 * L.term, L.S1 + 3 * L.term};
+}
+
 }  // namespace
 
 poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int count, int dtype, cudaStream_t st) {
-  std::vector<int> idx;
+  std::vector<int> idx, horner, pw;
   int kmax = 0;
   for (int i = 0; i < count; ++i) {
     if (geoms[i].nprim == 0) continue;
     idx.push_back(i);
-    if (geoms[i].k > kmax) kmax = geoms[i].k;
+    if (by_powers(geoms[i])) {
+      pw.push_back(i);
+    } else {
+      horner.push_back(i);
+      if (geoms[i].k > kmax) kmax = geoms[i].k;
+    }
   }
-  // theta -> Q and S_1 (or B when k = 0), every side in one launch
+  // theta -> Q, and S_1 (or B when k = 0) for Horner's rule; every side in one launch
   static thread_local SideTable t;
   POET_TRY(many_launch(idx, [&](int i, int q) {
     const SideGeom &g = geoms[i];
@@ -371,9 +491,10 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
     char *base = static_cast<char *>(sides[i].state);
     t.src[q] = sides[i].theta;
     t.dst[q] = base + L.Q;
-    t.dst2[q] = g.k == 0 ? base + L.R : base + L.S1;
+    t.dst2[q] = by_powers(g) ? nullptr : (g.k == 0 ? base + L.R : base + L.S1);
+    t.dst3[q] = g.k == 0 ? nullptr : base + L.R;
     t.nprim[q] = g.nprim; t.size[q] = g.size; t.ld[q] = g.ld;
-    return (g.all_elems() + 256 * kItems - 1) / (256 * kItems);
+    return elem_blocks(g);
   }, t, [&](const SideTable &tt, int, int) {
     const int blocks = int(tt.block_start[tt.count]);
     if (dtype == POET_BF16) unpack_many_kernel<bf16><<<blocks, 256, 0, st>>>(tt);
@@ -382,9 +503,10 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
     return launch_status("cnp unpack");
   }));
   std::vector<Gemm> gs;
+  // Horner's rule: one grouped launch per order
   for (int l = 1; l <= kmax; ++l) {
     gs.clear();
-    for (int i : idx) {
+    for (int i : horner) {
       const SideGeom &g = geoms[i];
       if (g.k < l) continue;
       const StateLayout L = state_layout(g, dtype);
@@ -404,46 +526,101 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
     }
     POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
   }
-  return POET_OK;
+  if (pw.empty()) return POET_OK;
+  // order 4 by powers: S = Q Q, T = S S, then C and D0, then B = Q C + D0
+  auto powers_step = [&](int step) {
+    gs.clear();
+    for (int i : pw) {
+      const SideGeom &g = geoms[i];
+      const StateLayout L = state_layout(g, dtype);
+      const PowersLayout W = powers_layout(L);
+      char *base = static_cast<char *>(sides[i].state);
+      Gemm p;
+      if (step == 0) {
+        p = prim_gemm(g, dtype, base + L.Q, base + L.Q, false, "cnp_fwd");
+        p.outD = base + W.S;
+      } else if (step == 1) {
+        p = prim_gemm(g, dtype, base + W.S, base + W.S, false, "cnp_fwd");
+        p.outD = base + W.T;
+      } else {
+        p = prim_gemm(g, dtype, base + L.Q, base + W.C, false, "cnp_fwd");
+        p.add = base + W.D0; p.add_dtype = dtype; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 1.f;
+        p.outD = base + L.R;
+      }
+      p.od_m = g.ld; p.od_b = g.blk_elems();
+      gs.push_back(p);
+    }
+    return gemm_run_many(gs.data(), int(gs.size()), st);
+  };
+  POET_TRY(powers_step(0));
+  POET_TRY(powers_step(1));
+  POET_TRY(many_launch(pw, [&](int i, int q) {
+    const SideGeom &g = geoms[i];
+    const PowersLayout W = powers_layout(state_layout(g, dtype));
+    char *base = static_cast<char *>(sides[i].state);
+    t.src[q] = base + W.S;
+    t.src2[q] = base + W.T;
+    t.dst[q] = base + W.C;
+    t.dst2[q] = base + W.D0;
+    t.nprim[q] = g.nprim; t.size[q] = g.size; t.ld[q] = g.ld;
+    return elem_blocks(g);
+  }, t, [&](const SideTable &tt, int, int) {
+    const int blocks = int(tt.block_start[tt.count]);
+    if (dtype == POET_BF16) powers_combine_kernel<bf16><<<blocks, 256, 0, st>>>(tt);
+    else powers_combine_kernel<float><<<blocks, 256, 0, st>>>(tt);
+    count_launch();
+    return launch_status("cnp combine");
+  }));
+  return powers_step(2);
 }
 
-// Many sides: the same gradient reorganised for grouped launches.  The chain
-// A_k = S_1^T G, A_l = -Q A_{l+1} takes one grouped launch per order (all
-// sides; S_1^T is read straight from the stored S_1 as a transposed operand).
-// One more launch forms every partial product P_k = G S_k^T,
-// P_l = A_{l+1} S_l^T (l < k) of every side, each into its own float buffer,
-// and one launch packs D - D^T into dtheta with D = A_1 + P_1 + ... + P_k.
+// Many sides: the same gradient reorganised for grouped launches.
+//  - Horner's rule: the chain A_k = S_1^T G, A_l = -Q A_{l+1} takes one grouped
+//    launch per order (all sides; S_1^T is read straight from the stored S_1
+//    as a transposed operand).  One more launch forms every partial product
+//    P_k = G S_k^T, P_l = A_{l+1} S_l^T (l < k) of every side, each into its
+//    own float buffer, and one launch packs D - D^T into dtheta with
+//    D = A_1 + P_1 + ... + P_k.
+//  - order 4 by powers: QG = Q G and GC = G C in one launch, dT_s, W = dT_s S,
+//    dS_s, Y = dS_s Q, then D = GC - 2 Y packed (see the top of this file).
 // Every product writes one plain output, which the tensor-core engine stores
 // through its staged epilogue.
 size_t cnp_many_scratch_bytes(const SideGeom &g, int dtype) {
   if (g.nprim == 0 || g.size < 2 || g.k == 0) return 0;
   const size_t f = align256(size_t(g.all_elems()) * 4);
   const size_t d = align256(size_t(g.all_elems()) * esize(dtype));
+  // order 4: G operand copy, QG then Y (f32), GC (f32), dT_s then dS_s (operand type), W (f32)
+  if (by_powers(g)) return 2 * d + 3 * f;
   // G operand copy, A_k..A_2 (dtype), A_1 (f32), P_1..P_k (f32)
   return d + size_t(g.k - 1) * d + f + size_t(g.k) * f;
 }
 
 poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int count, int dtype,
-                              const float *const *G, float *const *dtheta, void *const *scratch, cudaStream_t st) {
+                              const float *const *G, float *const *dtheta, void *const *scratch, cudaStream_t st,
+                              const AdamW *adam, float *const *m, float *const *v) {
   struct Work {
     const void *Q, *Gop;
     const char *S1;
     size_t term;
-    char *X;   // A_{l+1} for l = 1..k-1 at X + (l-1) * xb (dtype)
+    char *X;   // Horner: A_{l+1} for l = 1..k-1 at X + (l-1) * xb (dtype)
     size_t xb;
-    float *A1;  // A_1
-    float *P;   // P_l at P + (l-1) * pstride
+    float *A1;  // Horner: A_1
+    float *P;   // Horner: P_l at P + (l-1) * pstride
     int64_t pstride;
+    // order 4 by powers
+    const void *S, *C;
+    float *QGY, *GC, *W;
+    void *dT;
   };
   std::vector<Work> w(count);
-  std::vector<int> chain, all;  // sides with k >= 1; every side with parameters
+  std::vector<int> chain, all, pw, rounded;  // Horner sides with k >= 1; every side; order-4 sides; G to round
   int kmax = 0;
   for (int i = 0; i < count; ++i) {
     const SideGeom &g = geoms[i];
     if (g.nprim == 0 || g.size < 2) continue;
     all.push_back(i);
     if (g.k == 0) continue;  // B = I + Q: dQ = G
-    chain.push_back(i);
+    rounded.push_back(i);
     const StateLayout L = state_layout(g, dtype);
     const char *base = static_cast<const char *>(sides[i].state);
     const size_t db = align256(size_t(g.all_elems()) * esize(dtype));
@@ -451,9 +628,21 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
     char *s = static_cast<char *>(scratch[i]);
     Work &x = w[i];
     x.Q = base + L.Q;
+    x.Gop = dtype == POET_BF16 ? static_cast<const void *>(s) : static_cast<const void *>(G[i]);
+    if (by_powers(g)) {
+      pw.push_back(i);
+      const PowersLayout P = powers_layout(L);
+      x.S = base + P.S;
+      x.C = base + P.C;
+      x.QGY = reinterpret_cast<float *>(s + db);
+      x.GC = reinterpret_cast<float *>(s + db + fb);
+      x.dT = s + db + 2 * fb;
+      x.W = reinterpret_cast<float *>(s + 2 * db + 2 * fb);
+      continue;
+    }
+    chain.push_back(i);
     x.S1 = base + L.S1;
     x.term = L.term;
-    x.Gop = dtype == POET_BF16 ? static_cast<const void *>(s) : static_cast<const void *>(G[i]);
     x.X = s + db;
     x.xb = db;
     x.A1 = reinterpret_cast<float *>(s + size_t(g.k) * db);
@@ -463,23 +652,73 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
   }
   static thread_local SideTable t;
   if (dtype == POET_BF16) {  // G rounded to the operand type, every side in one launch
-    POET_TRY(many_launch(chain, [&](int i, int q) {
+    POET_TRY(many_launch(rounded, [&](int i, int q) {
       const SideGeom &g = geoms[i];
       t.src[q] = G[i];
       t.dst[q] = const_cast<void *>(w[i].Gop);
       t.nprim[q] = g.nprim; t.size[q] = g.size; t.ld[q] = g.ld;
-      return (g.all_elems() + 256 * kItems - 1) / (256 * kItems);
+      return elem_blocks(g);
     }, t, [&](const SideTable &tt, int, int) {
       round_many_kernel<<<int(tt.block_start[tt.count]), 256, 0, st>>>(tt);
       count_launch();
       return launch_status("cnp G to bf16");
     }));
   }
+  std::vector<Gemm> gs;
+  auto fout = [](Gemm &p, const SideGeom &g, float *o) { p.outF = o; p.of_m = g.ld; p.of_b = g.blk_elems(); };
+  // ---- order 4 by powers
+  if (!pw.empty()) {
+    gs.clear();
+    for (int i : pw) {  // QG = Q G, GC = G C
+      const SideGeom &g = geoms[i];
+      Gemm a = prim_gemm(g, dtype, w[i].Q, w[i].Gop, false, "cnp_bwd");
+      fout(a, g, w[i].QGY);
+      gs.push_back(a);
+      Gemm b = prim_gemm(g, dtype, w[i].Gop, w[i].C, false, "cnp_bwd");
+      fout(b, g, w[i].GC);
+      gs.push_back(b);
+    }
+    POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
+    auto sym = [&](bool second) {  // dT_s = sym(2G - QG), then dS_s = sym(2G - 2 QG) + W + W^T
+      return many_launch(pw, [&](int i, int q) {
+        const SideGeom &g = geoms[i];
+        t.src[q] = G[i];
+        t.src2[q] = w[i].QGY;
+        t.src3[q] = second ? w[i].W : nullptr;
+        t.dst[q] = w[i].dT;
+        t.nprim[q] = g.nprim; t.size[q] = g.size; t.ld[q] = g.ld;
+        return pair_blocks(g);
+      }, t, [&](const SideTable &tt, int, int) {
+        const int blocks = int(tt.block_start[tt.count]);
+        const float c1 = second ? -1.f : -0.5f, c2 = second ? 1.f : 0.f;
+        if (dtype == POET_BF16) sym_many_kernel<bf16><<<blocks, 256, 0, st>>>(tt, 1.f, c1, c2);
+        else sym_many_kernel<float><<<blocks, 256, 0, st>>>(tt, 1.f, c1, c2);
+        count_launch();
+        return launch_status("cnp symmetric part");
+      });
+    };
+    POET_TRY(sym(false));
+    gs.clear();
+    for (int i : pw) {  // W = dT_s S
+      Gemm a = prim_gemm(geoms[i], dtype, w[i].dT, w[i].S, false, "cnp_bwd");
+      fout(a, geoms[i], w[i].W);
+      gs.push_back(a);
+    }
+    POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
+    POET_TRY(sym(true));
+    gs.clear();
+    for (int i : pw) {  // Y = dS_s Q (over QG, which is no longer needed)
+      Gemm a = prim_gemm(geoms[i], dtype, w[i].dT, w[i].Q, false, "cnp_bwd");
+      fout(a, geoms[i], w[i].QGY);
+      gs.push_back(a);
+    }
+    POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
+  }
+  // ---- Horner's rule
   // X_l, the left factor of P_l: G for l = k, else A_{l+1}
   auto Xop = [&](int i, int l) -> const void * {
     return l == geoms[i].k ? w[i].Gop : static_cast<const void *>(w[i].X + size_t(l - 1) * w[i].xb);
   };
-  std::vector<Gemm> gs;
   // the chain, one order per launch (sides with a smaller k finish early)
   for (int step = 0; step < kmax; ++step) {
     gs.clear();
@@ -497,11 +736,11 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
         a.alpha = -1.f;
       }
       if (l == 1) {
-        a.outF = x.A1; a.of_m = g.ld; a.of_b = g.blk_elems();
+        fout(a, g, x.A1);
       } else if (dtype == POET_BF16) {
         a.outD = x.X + size_t(l - 2) * x.xb; a.od_m = g.ld; a.od_b = g.blk_elems();
       } else {
-        a.outF = reinterpret_cast<float *>(x.X + size_t(l - 2) * x.xb); a.of_m = g.ld; a.of_b = g.blk_elems();
+        fout(a, g, reinterpret_cast<float *>(x.X + size_t(l - 2) * x.xb));
       }
       gs.push_back(a);
     }
@@ -513,24 +752,40 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
     const SideGeom &g = geoms[i];
     for (int l = g.k; l >= 1; --l) {
       Gemm p = prim_gemm(g, dtype, Xop(i, l), w[i].S1 + size_t(l - 1) * w[i].term, true, "cnp_bwd");
-      p.outF = w[i].P + (l - 1) * w[i].pstride; p.of_m = g.ld; p.of_b = g.blk_elems();
+      fout(p, g, w[i].P + (l - 1) * w[i].pstride);
       gs.push_back(p);
     }
   }
   POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
-  // dtheta = D - D^T with D = A_1 + sum P_l (k = 0: D = G), every side in one launch
+  // dtheta = D - D^T, every side in one launch:  k = 0: D = G;  Horner: D = A_1 + sum P_l;
+  // order 4: D = GC - 2 Y
   return many_launch(all, [&](int i, int q) {
     const SideGeom &g = geoms[i];
-    t.src[q] = g.k == 0 ? static_cast<const void *>(G[i]) : static_cast<const void *>(w[i].A1);
-    t.dst2[q] = g.k == 0 ? nullptr : static_cast<void *>(w[i].P);
-    t.terms[q] = g.k;
-    t.stride[q] = g.k == 0 ? 0 : w[i].pstride;
-    t.dst[q] = dtheta[i];
+    if (g.k == 0) {
+      t.src[q] = G[i];
+    } else if (by_powers(g)) {
+      t.src[q] = w[i].GC;
+      t.dst2[q] = w[i].QGY;
+      t.terms[q] = 1;
+      t.coef[q] = -2.f;
+    } else {
+      t.src[q] = w[i].A1;
+      t.dst2[q] = w[i].P;
+      t.terms[q] = g.k;
+      t.stride[q] = w[i].pstride;
+    }
+    t.dst[q] = dtheta ? dtheta[i] : nullptr;
+    if (adam) {
+      t.theta[q] = sides[i].theta;
+      t.m1[q] = m[i];
+      t.m2[q] = v[i];
+    }
     t.nprim[q] = g.nprim; t.size[q] = g.size; t.ld[q] = g.ld;
-    const int64_t tiles = (g.size + PACK_T - 1) / PACK_T;
-    return int64_t(g.nprim) * tiles * (tiles + 1) / 2;
+    return pair_blocks(g);
   }, t, [&](const SideTable &tt, int, int) {
-    pack_many_kernel<<<int(tt.block_start[tt.count]), 256, 0, st>>>(tt);
+    const int blocks = int(tt.block_start[tt.count]);
+    if (adam) pack_many_kernel<true><<<blocks, 256, 0, st>>>(tt, *adam);
+    else pack_many_kernel<false><<<blocks, 256, 0, st>>>(tt, AdamW{});
     count_launch();
     return launch_status("cnp pack");
   });

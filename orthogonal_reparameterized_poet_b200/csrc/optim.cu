@@ -14,19 +14,6 @@
 namespace poet {
 namespace {
 
-struct AdamW {
-  float lr, beta1, beta2, eps, wd;
-  float bc1, bc2;  // 1 - beta^step
-};
-
-__device__ __forceinline__ void adamw_one(float &theta, float g, float &m, float &v, const AdamW &h) {
-  m = h.beta1 * m + (1.f - h.beta1) * g;
-  v = h.beta2 * v + (1.f - h.beta2) * g * g;
-  const float m_hat = m / h.bc1;
-  const float v_hat = v / h.bc2;
-  theta = theta - h.lr * (m_hat / (sqrtf(v_hat) + h.eps) + h.wd * theta);
-}
-
 __global__ void adamw_vec4_kernel(float4 *__restrict__ theta, const float4 *__restrict__ grad, float4 *__restrict__ m,
                                   float4 *__restrict__ v, int64_t n4, const AdamW h) {
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n4; i += int64_t(gridDim.x) * blockDim.x) {
@@ -50,13 +37,18 @@ __global__ void adamw_kernel(float *__restrict__ theta, const float *__restrict_
 
 }  // namespace
 
-poet_status adamw_step(float *theta, const float *grad, float *m, float *v, int64_t n, float lr, float beta1,
-                       float beta2, float eps, float weight_decay, int32_t step, cudaStream_t st) {
-  if (n == 0) return POET_OK;
+AdamW adamw_of(float lr, float beta1, float beta2, float eps, float weight_decay, int32_t step) {
   AdamW h;
   h.lr = lr; h.beta1 = beta1; h.beta2 = beta2; h.eps = eps; h.wd = weight_decay;
   h.bc1 = float(1.0 - std::pow(double(beta1), double(step)));
   h.bc2 = float(1.0 - std::pow(double(beta2), double(step)));
+  return h;
+}
+
+poet_status adamw_step(float *theta, const float *grad, float *m, float *v, int64_t n, float lr, float beta1,
+                       float beta2, float eps, float weight_decay, int32_t step, cudaStream_t st) {
+  if (n == 0) return POET_OK;
+  const AdamW h = adamw_of(lr, beta1, beta2, eps, weight_decay, step);
   const bool vec = ((reinterpret_cast<uintptr_t>(theta) | reinterpret_cast<uintptr_t>(grad) |
                      reinterpret_cast<uintptr_t>(m) | reinterpret_cast<uintptr_t>(v)) & 15) == 0;
   const int threads = 256;

@@ -22,6 +22,7 @@
 // length) use 16-byte copies for the aligned body and scalar copies for the
 // edges; shared and global addresses stay congruent modulo 16.
 #include <type_traits>
+#include <vector>
 
 #include "poet_internal.cuh"
 
@@ -42,8 +43,7 @@ struct PermArgs {
   T *dst1; int64_t ldd1;              // output rows
   T *dst2; int64_t ldd2; int dsplit;  // columns >= dsplit also go here (nullptr: none)
   const int32_t *dst_rowmap;          // destination row of output row r (nullptr: r)
-  int slot;                           // slot stride (elements, multiple of 16 bytes)
-  int map_len;                        // map entries allocated (>= round_up(d, 8) + 8)
+  int64_t map_rows;                   // row-map entries must lie in [0, map_rows) (0: rows)
   unsigned *errword;                  // ERR_BOUNDS is OR-ed in for an index out of range
 };
 
@@ -152,93 +152,118 @@ __device__ __forceinline__ void emit_row(const PermArgs<T> &a, const uint16_t *m
   }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(NT) permute_rows_kernel(const PermArgs<T> a) {
+// Up to MAXP independent row permutations in one launch.  Problem p owns the
+// global rows [row_start[p], row_start[p+1]); CTA c works through the
+// contiguous global rows [total*c/G, total*(c+1)/G), one segment per problem
+// it touches, and rebuilds its shared-memory map at the start of each segment.
+template <typename T, int MAXP>
+struct PermGroup {
+  PermArgs<T> prob[MAXP];
+  int64_t row_start[MAXP + 1];
+  int count;
+  int slot;     // ring slot stride (elements, multiple of 16 bytes), for the widest problem
+  int map_len;  // map entries allocated (>= round_up(max d, 8) + 8)
+};
+
+template <typename T, int MAXP>
+__global__ void __launch_bounds__(NT) permute_rows_kernel(const __grid_constant__ PermGroup<T, MAXP> g) {
   constexpr int VEC = 16 / sizeof(T);
   extern __shared__ __align__(16) unsigned char smem_raw[];
   uint16_t *map = reinterpret_cast<uint16_t *>(smem_raw);
-  const int d = a.d;
   const int nthr = blockDim.x, warps = nthr / 32;
-  for (int i = threadIdx.x; i < a.map_len; i += nthr) map[i] = 0;
-  __syncthreads();
-  bool bad = false;
-  if (!a.perm) {  // identity: a plain row copy (re-striding)
-    for (int i = threadIdx.x; i < d; i += nthr) map[i] = uint16_t(i);
-  } else if (a.inverse) {
-    for (int i = threadIdx.x; i < d; i += nthr) {
-      const int p = a.perm[i];
-      if (unsigned(p) < unsigned(d)) map[p] = uint16_t(i);
-      else bad = true;
-    }
-  } else {
-    for (int i = threadIdx.x; i < d; i += nthr) {
-      const int p = a.perm[i];
-      const bool ok = unsigned(p) < unsigned(d);
-      map[i] = ok ? uint16_t(p) : uint16_t(0);
-      bad |= !ok;
-    }
-  }
-  if (bad && a.errword) atomicOr(a.errword, ERR_BOUNDS);
-  __syncthreads();  // the only block-wide barriers: map is complete
-
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  T *ring = reinterpret_cast<T *>(smem_raw + size_t(a.map_len) * 2) + int64_t(warp) * NBW * a.slot;
-  const int split = a.split < d ? a.split : d;
-  const int64_t first = int64_t(blockIdx.x) * warps + warp, stride = int64_t(gridDim.x) * warps;
-  const int64_t count = first < a.rows ? (a.rows - first + stride - 1) / stride : 0;
+  T *ring = reinterpret_cast<T *>(smem_raw + size_t(g.map_len) * 2) + int64_t(warp) * NBW * g.slot;
+  const int64_t total = g.row_start[g.count];
+  const int64_t r0 = total * blockIdx.x / gridDim.x, r1 = total * (blockIdx.x + 1) / gridDim.x;
+  int p = 0;
+  for (int64_t seg = r0; seg < r1;) {
+    while (g.row_start[p + 1] <= seg) ++p;
+    const PermArgs<T> &a = g.prob[p];
+    const int64_t seg_end = r1 < g.row_start[p + 1] ? r1 : g.row_start[p + 1];
+    const int64_t lo = seg - g.row_start[p], hi = seg_end - g.row_start[p];  // rows [lo, hi) of problem p
+    seg = seg_end;
+    const int d = a.d;
+    __syncthreads();  // the previous segment's readers of map are done
+    for (int i = threadIdx.x; i < g.map_len; i += nthr) map[i] = 0;
+    __syncthreads();
+    bool bad = false;
+    if (!a.perm) {  // identity: a plain row copy
+      for (int i = threadIdx.x; i < d; i += nthr) map[i] = uint16_t(i);
+    } else if (a.inverse) {
+      for (int i = threadIdx.x; i < d; i += nthr) {
+        const int pi = a.perm[i];
+        if (unsigned(pi) < unsigned(d)) map[pi] = uint16_t(i);
+        else bad = true;
+      }
+    } else {
+      for (int i = threadIdx.x; i < d; i += nthr) {
+        const int pi = a.perm[i];
+        const bool ok = unsigned(pi) < unsigned(d);
+        map[i] = ok ? uint16_t(pi) : uint16_t(0);
+        bad |= !ok;
+      }
+    }
+    if (bad && a.errword) atomicOr(a.errword, ERR_BOUNDS);
+    __syncthreads();  // map is complete
 
-  // source and destination row of output row r; -1 when a row map's entry is out of range
-  auto src_row = [&](int64_t r) -> int64_t {
-    if (!a.src_rowmap) return r;
-    const int64_t s = a.src_rowmap[r];
-    return s >= 0 && s < a.rows ? s : -1;
-  };
-  auto dst_row = [&](int64_t r) -> int64_t {
-    if (!a.dst_rowmap) return r;
-    const int64_t s = a.dst_rowmap[r];
-    return s >= 0 && s < a.rows ? s : -1;
-  };
-  auto issue = [&](int64_t k) {
-    const int64_t r = first + k * stride;
-    const int64_t sr = src_row(r);
-    if (sr < 0 || dst_row(r) < 0) return;  // skipped row: nothing to load
-    T *slot = ring + int64_t(k % NBW) * a.slot;
-    const T *r1 = a.src1 + sr * a.ld1;
-    const int off = misalign(r1);
-    load_part(r1, 0, split, slot, off, lane);
-    if (split < d) load_part(a.src2 + sr * a.ld2, split, d, slot, off, lane);
-  };
+    const int split = a.split < d ? a.split : d;
+    const int64_t first = lo + warp, stride = warps;
+    const int64_t count = first < hi ? (hi - first + stride - 1) / stride : 0;
 
-  if (count > 0) issue(0);
-  cp_async_commit();
-  for (int64_t k = 0; k < count; ++k) {
-    if (k + 1 < count) issue(k + 1);
+    // source and destination row of output row r; -1 when a row map's entry is out of range
+    const int64_t map_rows = a.map_rows > 0 ? a.map_rows : a.rows;
+    auto src_row = [&](int64_t r) -> int64_t {
+      if (!a.src_rowmap) return r;
+      const int64_t s = a.src_rowmap[r];
+      return s >= 0 && s < map_rows ? s : -1;
+    };
+    auto dst_row = [&](int64_t r) -> int64_t {
+      if (!a.dst_rowmap) return r;
+      const int64_t s = a.dst_rowmap[r];
+      return s >= 0 && s < map_rows ? s : -1;
+    };
+    auto issue = [&](int64_t k) {
+      const int64_t r = first + k * stride;
+      const int64_t sr = src_row(r);
+      if (sr < 0 || dst_row(r) < 0) return;  // skipped row: nothing to load
+      T *slot = ring + int64_t(k % NBW) * g.slot;
+      const T *row1 = a.src1 + sr * a.ld1;
+      const int off = misalign(row1);
+      load_part(row1, 0, split, slot, off, lane);
+      if (split < d) load_part(a.src2 + sr * a.ld2, split, d, slot, off, lane);
+    };
+
+    if (count > 0) issue(0);
     cp_async_commit();
-    cp_async_wait_one();  // this lane's copies of row k have landed
-    __syncwarp();         // ... and every other lane's (scalar edges included)
-    const int64_t r = first + k * stride;
-    const int64_t sr = src_row(r), dr = dst_row(r);
-    if (sr < 0 || dr < 0) {  // a row map entry out of range: skip the row, report it
-      if (lane == 0 && a.errword) atomicOr(a.errword, ERR_BOUNDS);
-      __syncwarp();
-      continue;
+    for (int64_t k = 0; k < count; ++k) {
+      if (k + 1 < count) issue(k + 1);
+      cp_async_commit();
+      cp_async_wait_one();  // this lane's copies of row k have landed
+      __syncwarp();         // ... and every other lane's (scalar edges included)
+      const int64_t r = first + k * stride;
+      const int64_t sr = src_row(r), dr = dst_row(r);
+      if (sr < 0 || dr < 0) {  // a row map entry out of range: skip the row, report it
+        if (lane == 0 && a.errword) atomicOr(a.errword, ERR_BOUNDS);
+        __syncwarp();
+        continue;
+      }
+      const T *sl = ring + int64_t(k % NBW) * g.slot + misalign(a.src1 + sr * a.ld1);
+      T *drow = a.dst1 + dr * a.ldd1;
+      T *d2row = a.dst2 ? a.dst2 + r * a.ldd2 : nullptr;
+      switch (misalign(drow)) {
+        case 0: emit_row<T, 0>(a, map, sl, drow, d2row, lane); break;
+        case 1: emit_row<T, 1>(a, map, sl, drow, d2row, lane); break;
+        case 2: emit_row<T, 2>(a, map, sl, drow, d2row, lane); break;
+        case 3: emit_row<T, 3>(a, map, sl, drow, d2row, lane); break;
+        case 4: if constexpr (VEC == 8) emit_row<T, 4>(a, map, sl, drow, d2row, lane); break;
+        case 5: if constexpr (VEC == 8) emit_row<T, 5>(a, map, sl, drow, d2row, lane); break;
+        case 6: if constexpr (VEC == 8) emit_row<T, 6>(a, map, sl, drow, d2row, lane); break;
+        default: if constexpr (VEC == 8) emit_row<T, 7>(a, map, sl, drow, d2row, lane); break;
+      }
+      __syncwarp();  // slot k % NBW may be refilled by the next iteration's prefetch
     }
-    const T *s = ring + int64_t(k % NBW) * a.slot + misalign(a.src1 + sr * a.ld1);
-    T *drow = a.dst1 + dr * a.ldd1;
-    T *d2row = a.dst2 ? a.dst2 + r * a.ldd2 : nullptr;
-    switch (misalign(drow)) {
-      case 0: emit_row<T, 0>(a, map, s, drow, d2row, lane); break;
-      case 1: emit_row<T, 1>(a, map, s, drow, d2row, lane); break;
-      case 2: emit_row<T, 2>(a, map, s, drow, d2row, lane); break;
-      case 3: emit_row<T, 3>(a, map, s, drow, d2row, lane); break;
-      case 4: if constexpr (VEC == 8) emit_row<T, 4>(a, map, s, drow, d2row, lane); break;
-      case 5: if constexpr (VEC == 8) emit_row<T, 5>(a, map, s, drow, d2row, lane); break;
-      case 6: if constexpr (VEC == 8) emit_row<T, 6>(a, map, s, drow, d2row, lane); break;
-      default: if constexpr (VEC == 8) emit_row<T, 7>(a, map, s, drow, d2row, lane); break;
-    }
-    __syncwarp();  // slot k % NBW may be refilled by the next iteration's prefetch
+    cp_async_wait_all();
   }
-  cp_async_wait_all();
 }
 
 // Plain row copy to 16-byte aligned destination rows (re-striding rows whose
@@ -289,22 +314,42 @@ __global__ void __launch_bounds__(256) restride_kernel(const unsigned char *__re
 }
 
 // out[a][c] = bf16(D[rowmap[a]][perm[c]]): a float matrix gathered into the
-// frame and rounded in one pass.  One block per output row at a time; the
-// source row is read through L1 (it is reused by the block's gathers).  An
-// index out of range (rowmap outside [0, rows), perm outside [0, d)) is not
-// read: its output is 0 and ERR_BOUNDS is set in the status word.
-__global__ void __launch_bounds__(256) frame_f32_to_bf16_kernel(const float *__restrict__ D, int64_t ldD,
-                                                                const int32_t *__restrict__ rowmap, int64_t rows,
-                                                                int d, const int32_t *__restrict__ perm,
-                                                                bf16 *__restrict__ out, int64_t ld_out,
-                                                                unsigned *errword) {
+// frame and rounded in one pass, for up to kFrameMax matrices per launch
+// (matrix p owns the global rows [row_start[p], row_start[p+1])).  One block
+// per output row at a time; the source row is read through L1 (it is reused
+// by the block's gathers).  An index out of range (rowmap outside [0, rows),
+// perm outside [0, d)) is not read: its output is 0 and ERR_BOUNDS is set in
+// the status word.
+constexpr int kFrameMax = 64;
+struct FrameGroup {
+  const float *D[kFrameMax];
+  int64_t ldD[kFrameMax];
+  const int32_t *rowmap[kFrameMax];
+  const int32_t *perm[kFrameMax];
+  bf16 *out[kFrameMax];
+  int64_t ld_out[kFrameMax];
+  int64_t rows[kFrameMax];
+  int d[kFrameMax];
+  int64_t row_start[kFrameMax + 1];
+  int count;
+  unsigned *errword;
+};
+static_assert(sizeof(FrameGroup) <= 32000, "frame table exceeds the kernel parameter limit");
+
+__global__ void __launch_bounds__(256) frame_f32_to_bf16_kernel(const __grid_constant__ FrameGroup g) {
   bool bad = false;
-  for (int64_t a = blockIdx.x; a < rows; a += gridDim.x) {
-    const int64_t sr = __ldg(rowmap + a);
+  const int64_t total = g.row_start[g.count];
+  int p = 0;
+  for (int64_t gr = blockIdx.x; gr < total; gr += gridDim.x) {
+    while (g.row_start[p + 1] <= gr) ++p;  // rows are visited in increasing order
+    const int64_t a = gr - g.row_start[p], rows = g.rows[p];
+    const int d = g.d[p];
+    const int32_t *perm = g.perm[p];
+    const int64_t sr = __ldg(g.rowmap[p] + a);
     const bool row_ok = sr >= 0 && sr < rows;
     bad |= !row_ok;
-    const float *src = D + (row_ok ? sr : 0) * ldD;
-    bf16 *orow = out + a * ld_out;
+    const float *src = g.D[p] + (row_ok ? sr : 0) * g.ldD[p];
+    bf16 *orow = g.out[p] + a * g.ld_out[p];
     for (int c = 2 * threadIdx.x; c < d; c += 2 * blockDim.x) {
       if (c + 1 < d) {
         const int2 pc = *reinterpret_cast<const int2 *>(perm + c);
@@ -320,39 +365,101 @@ __global__ void __launch_bounds__(256) frame_f32_to_bf16_kernel(const float *__r
       }
     }
   }
-  if (bad && errword) atomicOr(errword, ERR_BOUNDS);
+  if (bad && g.errword) atomicOr(g.errword, ERR_BOUNDS);
 }
 
-template <typename T>
-poet_status launch_permute(PermArgs<T> a, cudaStream_t st, const char *kind) {
-  if (a.rows <= 0 || a.d <= 0) return POET_OK;
-  POET_REQUIRE(a.d <= 65535, "permute: dimension %d too large", a.d);
+// dst[p][0 .. n[p]) = 0 for up to kFrameMax float buffers (16-byte vectors
+// where a buffer is 16-byte aligned).
+struct ZeroGroup {
+  float *dst[kFrameMax];
+  int64_t n[kFrameMax];
+  int count;
+};
+__global__ void __launch_bounds__(256) zero_many_kernel(const __grid_constant__ ZeroGroup g) {
+  for (int p = 0; p < g.count; ++p) {
+    float *d = g.dst[p];
+    const int64_t n = g.n[p];
+    const int64_t tid = blockIdx.x * int64_t(blockDim.x) + threadIdx.x, nth = int64_t(gridDim.x) * blockDim.x;
+    if ((reinterpret_cast<uintptr_t>(d) & 15) == 0) {
+      const int64_t n4 = n / 4;
+      for (int64_t i = tid; i < n4; i += nth) reinterpret_cast<float4 *>(d)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int64_t i = n4 * 4 + tid; i < n; i += nth) d[i] = 0.f;
+    } else {
+      for (int64_t i = tid; i < n; i += nth) d[i] = 0.f;
+    }
+  }
+}
+
+// Launches the problems of one table: the ring slot fits the widest row, as
+// many warps as shared memory allows (at most MAX_WARPS), and a grid of the
+// CTAs that can be resident at once (fewer for little work).
+template <typename T, int MAXP>
+poet_status launch_permute_group(PermGroup<T, MAXP> &grp, cudaStream_t st, const char *kind) {
   constexpr int VEC = 16 / sizeof(T);
-  a.slot = int(round_up(a.d + VEC, VEC));
-  a.map_len = int(round_up(a.d, 8) + 8);
-  const size_t budget = 220 * 1024, per_warp = size_t(NBW) * a.slot * sizeof(T);
-  int warps = int((budget - size_t(a.map_len) * 2) / per_warp);
+  int dmax = 0;
+  double bytes = 0.0;
+  grp.row_start[0] = 0;
+  for (int i = 0; i < grp.count; ++i) {
+    const PermArgs<T> &a = grp.prob[i];
+    POET_REQUIRE(a.d >= 1 && a.d <= 65535, "permute: dimension %d outside [1, 65535]", a.d);
+    if (a.d > dmax) dmax = a.d;
+    grp.row_start[i + 1] = grp.row_start[i] + (a.rows > 0 ? a.rows : 0);
+    bytes += double(a.rows) * a.d * sizeof(T) * 2.0;
+  }
+  const int64_t total = grp.row_start[grp.count];
+  if (total <= 0) return POET_OK;
+  grp.slot = int(round_up(dmax + VEC, VEC));
+  grp.map_len = int(round_up(dmax, 8) + 8);
+  const size_t budget = 220 * 1024, per_warp = size_t(NBW) * grp.slot * sizeof(T);
+  int warps = int((budget - size_t(grp.map_len) * 2) / per_warp);
   if (warps > MAX_WARPS) warps = MAX_WARPS;
-  POET_REQUIRE(warps >= 1, "permute: rows of %d elements do not fit in shared memory", a.d);
-  const size_t smem = size_t(a.map_len) * 2 + size_t(warps) * per_warp;
+  POET_REQUIRE(warps >= 1, "permute: rows of %d elements do not fit in shared memory", dmax);
+  const size_t smem = size_t(grp.map_len) * 2 + size_t(warps) * per_warp;
+  auto kern = permute_rows_kernel<T, MAXP>;
   static int configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && configured[dev] < int(smem)) {
-    POET_CUDA_TRY(cudaFuncSetAttribute(permute_rows_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+    POET_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
     configured[dev] = int(smem);
   }
   int per_sm = 0;
-  POET_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_rows_kernel<T>, warps * 32, smem));
+  POET_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, warps * 32, smem));
   if (per_sm < 1) per_sm = 1;
-  const int64_t want = (a.rows + warps - 1) / warps;
+  const int64_t want = (total + warps - 1) / warps;
   const int64_t cap = int64_t(num_sms()) * per_sm;
   const int grid = int(want < cap ? want : cap);
-  a.errword = device_errword();
-  TraceScope ts(kind, 0.0, double(a.rows) * a.d * sizeof(T) * 2.0, st);
-  permute_rows_kernel<T><<<grid, warps * 32, smem, st>>>(a);
+  unsigned *ew = device_errword();
+  for (int i = 0; i < grp.count; ++i) grp.prob[i].errword = ew;
+  TraceScope ts(kind, 0.0, bytes, st);
+  kern<<<grid, warps * 32, smem, st>>>(grp);
   count_launch();
   return launch_status(kind);
+}
+
+template <typename T>
+poet_status launch_permute(const PermArgs<T> &a, cudaStream_t st, const char *kind) {
+  if (a.rows <= 0 || a.d <= 0) return POET_OK;
+  PermGroup<T, 1> grp;
+  grp.prob[0] = a;
+  grp.count = 1;
+  return launch_permute_group(grp, st, kind);
+}
+
+constexpr int kPermMax = 64;
+static_assert(sizeof(PermGroup<float, kPermMax>) <= 32000, "permute table exceeds the kernel parameter limit");
+
+template <typename T>
+poet_status launch_permute_many(const std::vector<PermArgs<T>> &v, cudaStream_t st, const char *kind) {
+  static thread_local PermGroup<T, kPermMax> grp;  // large: keep it off the stack
+  for (size_t i0 = 0; i0 < v.size(); i0 += kPermMax) {
+    grp.count = 0;
+    for (size_t i = i0; i < v.size() && i < i0 + kPermMax; ++i)
+      if (v[i].rows > 0 && v[i].d > 0) grp.prob[grp.count++] = v[i];
+    if (grp.count == 0) continue;
+    POET_TRY(launch_permute_group(grp, st, kind));
+  }
+  return POET_OK;
 }
 
 }  // namespace
@@ -378,19 +485,85 @@ poet_status gather_cols(int dtype, const void *src, int64_t ld_src, const int32_
   return dtype == POET_BF16 ? fill(static_cast<bf16 *>(nullptr)) : fill(static_cast<float *>(nullptr));
 }
 
+poet_status frame_many(const std::vector<FrameItem> &v, cudaStream_t st) {
+  static thread_local FrameGroup grp;
+  for (size_t i0 = 0; i0 < v.size(); i0 += kFrameMax) {
+    grp.count = 0;
+    grp.row_start[0] = 0;
+    double bytes = 0.0;
+    for (size_t i = i0; i < v.size() && i < i0 + kFrameMax; ++i) {
+      const FrameItem &f = v[i];
+      if (f.rows <= 0 || f.d <= 0) continue;
+      POET_REQUIRE((reinterpret_cast<uintptr_t>(f.out) & 3) == 0 && f.ld_out % 2 == 0 &&
+                       (reinterpret_cast<uintptr_t>(f.perm) & 7) == 0,
+                   "frame: output rows must be 4-byte aligned and perm 8-byte aligned");
+      const int q = grp.count++;
+      grp.D[q] = f.D; grp.ldD[q] = f.ldD; grp.rowmap[q] = f.rowmap; grp.perm[q] = f.perm;
+      grp.out[q] = static_cast<bf16 *>(f.out); grp.ld_out[q] = f.ld_out; grp.rows[q] = f.rows; grp.d[q] = f.d;
+      grp.row_start[q + 1] = grp.row_start[q] + f.rows;
+      bytes += double(f.rows) * f.d * 6.0;
+    }
+    if (grp.count == 0) continue;
+    grp.errword = device_errword();
+    const int64_t total = grp.row_start[grp.count];
+    const int64_t cap = int64_t(num_sms()) * 8;
+    const int grid = int(total < cap ? total : cap);
+    TraceScope ts("frame", 0.0, bytes, st);
+    frame_f32_to_bf16_kernel<<<grid, 256, 0, st>>>(grp);
+    count_launch();
+    POET_TRY(launch_status("frame"));
+  }
+  return POET_OK;
+}
+
 poet_status frame_f32_to_bf16(const float *D, int64_t ldD, const int32_t *rowmap, int64_t rows, int d,
                               const int32_t *perm, void *out, int64_t ld_out, cudaStream_t st) {
-  POET_REQUIRE((reinterpret_cast<uintptr_t>(out) & 3) == 0 && ld_out % 2 == 0 &&
-                   (reinterpret_cast<uintptr_t>(perm) & 7) == 0,
-               "frame: output rows must be 4-byte aligned and perm 8-byte aligned");
-  if (rows <= 0 || d <= 0) return POET_OK;
-  TraceScope ts("frame", 0.0, double(rows) * d * 6.0, st);
-  const int64_t cap = int64_t(num_sms()) * 8;
-  const int grid = int(rows < cap ? rows : cap);
-  frame_f32_to_bf16_kernel<<<grid, 256, 0, st>>>(D, ldD, rowmap, rows, d, perm, static_cast<bf16 *>(out), ld_out,
-                                                  device_errword());
-  count_launch();
-  return launch_status("frame");
+  return frame_many({FrameItem{D, ldD, rowmap, rows, d, perm, out, ld_out}}, st);
+}
+
+poet_status zero_many(const std::vector<std::pair<float *, int64_t>> &v, cudaStream_t st) {
+  static thread_local ZeroGroup grp;
+  for (size_t i0 = 0; i0 < v.size(); i0 += kFrameMax) {
+    grp.count = 0;
+    int64_t most = 0;
+    for (size_t i = i0; i < v.size() && i < i0 + kFrameMax; ++i) {
+      if (!v[i].first || v[i].second <= 0) continue;
+      grp.dst[grp.count] = v[i].first;
+      grp.n[grp.count++] = v[i].second;
+      if (v[i].second > most) most = v[i].second;
+    }
+    if (grp.count == 0) continue;
+    const int64_t want = (most / 4 + 255) / 256, cap = int64_t(num_sms()) * 4;
+    const int grid = int(want < 1 ? 1 : (want < cap ? want : cap));
+    zero_many_kernel<<<grid, 256, 0, st>>>(grp);
+    count_launch();
+    POET_TRY(launch_status("zero"));
+  }
+  return POET_OK;
+}
+
+poet_status permute_many(int dtype, const std::vector<RowPermute> &v, cudaStream_t st, const char *kind) {
+  auto run = [&](auto *tag) {
+    using T = std::remove_pointer_t<decltype(tag)>;
+    std::vector<PermArgs<T>> args;
+    args.reserve(v.size());
+    for (const RowPermute &r : v) {
+      PermArgs<T> a{};
+      a.src1 = static_cast<const T *>(r.src1); a.ld1 = r.ld1;
+      a.src2 = static_cast<const T *>(r.src2 ? r.src2 : r.src1); a.ld2 = r.src2 ? r.ld2 : r.ld1;
+      a.split = r.src2 ? r.split : r.d;
+      a.src_rowmap = r.src_rowmap;
+      a.rows = r.rows; a.d = r.d;
+      a.perm = r.perm; a.inverse = r.inverse;
+      a.dst1 = static_cast<T *>(r.dst); a.ldd1 = r.ldd;
+      a.dst2 = nullptr; a.ldd2 = 0; a.dsplit = r.d;
+      a.dst_rowmap = r.dst_rowmap;
+      a.map_rows = r.map_rows;
+      args.push_back(a);
+    }
+    return launch_permute_many<T>(args, st, kind);
+  };
+  return dtype == POET_BF16 ? run(static_cast<bf16 *>(nullptr)) : run(static_cast<float *>(nullptr));
 }
 
 poet_status copy_rows(int dtype, const void *src, int64_t ld_src, int64_t rows, int d, void *dst, int64_t ld_dst,

@@ -236,6 +236,7 @@ size_t side_ws_bytes(const SideGeom &g, int dtype) {
 Gemm blockdiag(const SideGeom &g, int dtype, int64_t T, const void *X, int64_t ldx, const void *Blk, bool trans,
                void *C, int64_t ldc) {
   Gemm p;
+  p.small = SMALL_RIGHT;
   p.tag = trans ? "blk_bwd" : "blk_fwd";
   p.M = int(T); p.N = g.size; p.K = g.size; p.batch = g.nprim;
   p.dtype = dtype;
@@ -251,6 +252,7 @@ Gemm blockdiag(const SideGeom &g, int dtype, int64_t T, const void *X, int64_t l
 //   Gout[j][a][c] += sum_t D[t][j*s + a] * V[t][j*s + c]
 Gemm blockgrad(const SideGeom &g, int dtype, int64_t T, const void *D, const void *V, int64_t ld, float *Gout) {
   Gemm p;
+  p.small = SMALL_GRAD;
   p.tag = "blk_grad";
   p.M = g.size; p.N = g.size; p.K = int(T); p.batch = g.nprim;
   p.dtype = dtype;
@@ -271,6 +273,7 @@ Gemm left_blocks(const poet_layer *L, const LayerGeom &lg, const void *src, void
   const SideGeom &g = lg.R;
   const int64_t ldw = lg.ldn;
   Gemm p;
+  p.small = SMALL_LEFT;
   p.tag = tag;
   p.M = g.size; p.N = int(lg.n); p.K = g.size; p.batch = g.nprim; p.dtype = lg.dtype;
   p.A = state_R(&L->R, g, lg.dtype); p.a_m = g.ld; p.a_k = 1; p.a_b = g.blk_elems();
@@ -294,6 +297,7 @@ Gemm right_blocks(const poet_layer *L, const LayerGeom &lg, const void *src, voi
   const SideGeom &g = lg.P;
   const int64_t ldw = lg.ldn;
   Gemm p;
+  p.small = SMALL_RIGHT;
   p.tag = tag;
   p.M = int(lg.m); p.N = g.size; p.K = g.size; p.batch = g.nprim; p.dtype = lg.dtype;
   p.A = src; p.a_m = ldw; p.a_k = 1; p.a_b = g.size;
@@ -314,6 +318,9 @@ poet_status right_tail(const LayerGeom &lg, const void *src, void *out, cudaStre
 
 poet_status gemm_run(const Gemm &g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.batch <= 0) return POET_OK;
+  bool done = false;
+  POET_TRY(smallb_dispatch(g, st, &done));
+  if (done) return POET_OK;
   const double mnb = double(g.M) * g.N * g.batch;
   const double bytes = double(esize(g.dtype)) * (double(g.M) + g.N) * g.K * g.batch +
                        mnb * ((g.outF ? 4.0 : 0.0) + (g.outD ? double(esize(g.dtype)) : 0.0) +
@@ -325,6 +332,15 @@ poet_status gemm_run(const Gemm &g, cudaStream_t st) {
 
 poet_status gemm_run_many(const Gemm *gs, int count, cudaStream_t st) {
   if (count <= 0) return POET_OK;
+  std::vector<Gemm> rest;  // what the small-block kernels do not take
+  for (int i = 0; i < count; ++i) {
+    bool done = false;
+    if (gs[i].M > 0 && gs[i].N > 0 && gs[i].batch > 0) POET_TRY(smallb_dispatch(gs[i], st, &done));
+    if (!done) rest.push_back(gs[i]);
+  }
+  if (rest.empty()) return POET_OK;
+  gs = rest.data();
+  count = int(rest.size());
   double flop = 0.0, bytes = 0.0;
   for (int i = 0; i < count; ++i) {
     const Gemm &g = gs[i];
@@ -349,7 +365,7 @@ extern "C" {
 const char *poet_last_error(void) { return g_last_error; }
 
 // The kernel revisions name the code that profiles/ counters were taken on.
-const char *poet_version(void) { return "libpoet 0.3 (sm_100a; gemm_tc r9; permute r3; restride r1; cnp r2)"; }
+const char *poet_version(void) { return "libpoet 0.4 (sm_100a; gemm_tc r9; permute r4; restride r1; cnp r3; smallb r1)"; }
 
 size_t poet_side_state_bytes(const poet_side *side, int32_t dtype) {
   SideGeom g;
@@ -434,166 +450,290 @@ poet_status poet_cayley_neumann_grad(const poet_side *side, int32_t dtype, const
 }
 
 // ------------------------------------------------------------------ weight plan
+//
+// Every weight-plan call works on a list of layers, so that the weight-sized
+// products of many layers share grouped tensor-core launches and their
+// permutations share one launch; the single-layer entry points pass a list of
+// one.  With c_R = R.covered and c_P = P.covered (frame indices acted on):
+//   H = R W0f on the rows [0, c_R)            (the other rows of H are W0f's)
+//   F = W0f P on the columns [0, c_P)         (the other columns are W0f's)
+//   E_f = H P on the rows [0, c_R) and columns [0, c_P)
+// and E = E_f unframed, reading E_f / H on the rows [0, c_R) and F / W0f on
+// the others, each split at the column c_P.  The backward's per-primitive
+// products split their K range the same way, so the leftover rows and
+// columns are read from W0f in place.  Only when c_P is not a 16-byte
+// column offset (a TMA operand must start on one) are F's leftover columns
+// copied from W0f.
 
-// E_f = R W0f P in the frame (H = R W0f and F = W0f P kept for the backward),
-// then E = E_f in natural order.  Weight-sized work only.
-static poet_status weight_factors(const poet_layer *L, const LayerGeom &lg, char *sv, const WeightSaved &ly, void *Ef,
-                                  cudaStream_t st) {
-  const int dt = lg.dtype;
-  const void *W0f = L->W0f;
-  const void *Hs = W0f, *Es = W0f;
-  if (lg.R.nprim > 0) {
-    POET_TRY(gemm_run(left_blocks(L, lg, W0f, sv + ly.H, "w_prep"), st));
-    POET_TRY(left_tail(lg, W0f, sv + ly.H, st));
-    Hs = sv + ly.H;
-    Es = Hs;
-  }
-  if (lg.P.nprim > 0) {
-    Gemm two[2] = {right_blocks(L, lg, W0f, sv + ly.F, "w_prep"), right_blocks(L, lg, Hs, Ef, "w_prep")};
-    POET_TRY(gemm_run_many(two, 2, st));
-    POET_TRY(right_tail(lg, W0f, sv + ly.F, st));
-    POET_TRY(right_tail(lg, Hs, Ef, st));
-    Es = Ef;
-  }
-  // E[R.perm[i]][P.perm[j]] = E_f[i][j]
-  return scatter_cols(dt, Es, lg.ldn, Es, lg.ldn, int(lg.n), lg.m, int(lg.n), L->P.perm, sv + ly.E, lg.ldn,
-                      L->R.perm, st, "unframe");
+namespace {
+
+struct WFwd {          // one layer of a grouped weight-plan forward
+  const poet_layer *L;
+  LayerGeom lg;
+  const void *x; int64_t ldx;
+  void *y; int64_t ldy;
+  char *sv;            // saved buffer (weight_saved layout)
+  void *Ef;            // m x ldn scratch in the storage type (E_f)
+};
+
+struct WBwd {          // one layer of a grouped weight-plan backward
+  const poet_layer *L;
+  LayerGeom lg;
+  const void *x; int64_t ldx;
+  const char *sv;
+  const void *dy; int64_t lddy;
+  void *dx; int64_t lddx;
+  float *GR, *GP;      // per-primitive gradients (overwritten)
+  void *act1;          // T x ldm scratch for a re-strided dy (used when dy's rows are not 16-byte aligned)
+  float *D;            // m x ldn float scratch
+  void *Df;            // m x ldn scratch in the storage type (D framed)
+};
+
+// c_P is a column offset a TMA operand can start at
+bool col_split_ok(const LayerGeom &lg) { return (int64_t(lg.P.covered) * int64_t(esize(lg.dtype))) % 16 == 0; }
+bool f_tail_copied(const LayerGeom &lg) {
+  return lg.P.nprim > 0 && lg.P.covered < lg.n && !col_split_ok(lg);
 }
 
-static poet_status forward_weight(const poet_layer *L, const LayerGeom &lg, const void *x, int64_t T, void *y,
-                                  void *saved, char *wb, const WsLayout &w, cudaStream_t st) {
-  const int dt = lg.dtype;
-  char *sv = static_cast<char *>(saved);
-  const WeightSaved ly = weight_saved(lg, T);
-  POET_TRY(weight_factors(L, lg, sv, ly, wb + w.Z, st));
-  // x as a GEMM operand needs 16-byte aligned rows
-  const void *xa = x;
-  int64_t ldx = lg.n;
-  if (!rows16(x, lg.n, dt)) {
-    POET_TRY(copy_rows(dt, x, lg.n, T, int(lg.n), sv + ly.xp, lg.ldn, st));
-    xa = sv + ly.xp;
-    ldx = lg.ldn;
-  }
-  Gemm p;  // y = x E^T
-  p.tag = "w0_fwd";
-  p.M = int(T); p.N = int(lg.m); p.K = int(lg.n); p.dtype = dt;
-  p.A = xa; p.a_m = ldx; p.a_k = 1;
-  p.B = sv + ly.E; p.b_n = lg.ldn; p.b_k = 1;
-  p.outD = y; p.od_m = lg.m;
-  return gemm_run(p, st);
+const char *at(const void *base, int64_t elems, int dtype) {
+  return static_cast<const char *>(base) + elems * int64_t(esize(dtype));
 }
 
-static poet_status backward_weight(const poet_layer *L, const LayerGeom &lg, char *wb, const WsLayout &w,
-                                   const void *x, const void *saved, const void *dy, int64_t T, void *dx, float *GR,
-                                   float *GP, cudaStream_t st) {
-  const int dt = lg.dtype;
-  const SideGeom &gR = lg.R, &gP = lg.P;
-  const char *sv = static_cast<const char *>(saved);
-  const WeightSaved ly = weight_saved(lg, T);
-  const void *xa = x;
-  int64_t ldx = lg.n;
-  if (!rows16(x, lg.n, dt)) { xa = sv + ly.xp; ldx = lg.ldn; }  // the forward's re-strided copy
-  const void *dya = dy;
-  int64_t ldy = lg.m;
-  if (!rows16(dy, lg.m, dt)) {
-    POET_TRY(copy_rows(dt, dy, lg.m, T, int(lg.m), wb + w.act1, lg.ldm, st));
-    dya = wb + w.act1;
-    ldy = lg.ldm;
+poet_status forward_weight_many(std::vector<WFwd> &v, int64_t T, cudaStream_t st) {
+  std::vector<Gemm> gs;
+  std::vector<RowPermute> perms;
+  if (v.empty()) return POET_OK;
+  const int dt = v[0].lg.dtype;
+  // H = R W0f (rows < c_R) and F = W0f P (columns < c_P), every layer in one grouped launch
+  for (WFwd &f : v) {
+    const WeightSaved ly = weight_saved(f.lg, T);
+    if (f.lg.R.nprim > 0) gs.push_back(left_blocks(f.L, f.lg, f.L->W0f, f.sv + ly.H, "w_prep"));
+    if (f.lg.P.nprim > 0) gs.push_back(right_blocks(f.L, f.lg, f.L->W0f, f.sv + ly.F, "w_prep"));
   }
-  {  // dx = dy E
+  POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
+  // F's leftover columns, where the backward cannot read them from W0f in place
+  for (WFwd &f : v) {
+    if (!f_tail_copied(f.lg)) continue;
+    const WeightSaved ly = weight_saved(f.lg, T);
+    RowPermute r;
+    r.src1 = at(f.L->W0f, f.lg.P.covered, dt); r.ld1 = f.lg.ldn;
+    r.rows = f.lg.m; r.d = int(f.lg.n - f.lg.P.covered);
+    r.dst = const_cast<char *>(at(f.sv + ly.F, f.lg.P.covered, dt)); r.ldd = f.lg.ldn;
+    perms.push_back(r);
+  }
+  POET_TRY(permute_many(dt, perms, st, "copy"));
+  // E_f = H P on the rows < c_R
+  gs.clear();
+  for (WFwd &f : v) {
+    if (f.lg.R.nprim == 0 || f.lg.P.nprim == 0) continue;
+    const WeightSaved ly = weight_saved(f.lg, T);
+    Gemm p = right_blocks(f.L, f.lg, f.sv + ly.H, f.Ef, "w_prep");
+    p.M = f.lg.R.covered;
+    gs.push_back(p);
+  }
+  POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
+  // E[R.perm[i]][P.perm[j]] = E_f[i][j], every layer in one launch
+  perms.clear();
+  for (WFwd &f : v) {
+    const LayerGeom &lg = f.lg;
+    const WeightSaved ly = weight_saved(lg, T);
+    const int64_t cR = lg.R.covered, cP = lg.P.covered;
+    const char *W0f = static_cast<const char *>(f.L->W0f);
+    RowPermute r;
+    r.ld1 = r.ld2 = lg.ldn;
+    r.d = int(lg.n);
+    r.perm = f.L->P.perm; r.inverse = 1;
+    r.dst = f.sv + ly.E; r.ldd = lg.ldn;
+    r.map_rows = lg.m;
+    if (cR > 0) {  // rows acted on by R: E_f (columns < c_P) and H
+      RowPermute a = r;
+      a.src1 = cP > 0 ? static_cast<const void *>(f.Ef) : f.sv + ly.H;
+      a.src2 = cP > 0 && cP < lg.n ? f.sv + ly.H : nullptr;
+      a.split = int(cP);
+      a.rows = cR;
+      a.dst_rowmap = f.L->R.perm;
+      perms.push_back(a);
+    }
+    if (cR < lg.m) {  // the other rows: F (columns < c_P) and W0f
+      RowPermute b = r;
+      b.src1 = at(cP > 0 ? static_cast<const void *>(f.sv + ly.F) : W0f, cR * lg.ldn, dt);
+      b.src2 = cP > 0 && cP < lg.n ? at(W0f, cR * lg.ldn, dt) : nullptr;
+      b.split = int(cP);
+      b.rows = lg.m - cR;
+      b.dst_rowmap = f.L->R.perm + cR;
+      perms.push_back(b);
+    }
+  }
+  POET_TRY(permute_many(dt, perms, st, "unframe"));
+  // y = x E^T, every layer in one grouped launch (x re-strided first where its rows are not 16-byte aligned)
+  gs.clear();
+  for (WFwd &f : v) {
+    const LayerGeom &lg = f.lg;
+    const WeightSaved ly = weight_saved(lg, T);
+    const void *xa = f.x;
+    int64_t ldx = f.ldx;
+    if (!rows16(f.x, f.ldx, dt)) {
+      POET_TRY(copy_rows(dt, f.x, f.ldx, T, int(lg.n), f.sv + ly.xp, lg.ldn, st));
+      xa = f.sv + ly.xp;
+      ldx = lg.ldn;
+    }
+    Gemm p;
+    p.tag = "w0_fwd";
+    p.M = int(T); p.N = int(lg.m); p.K = int(lg.n); p.dtype = dt;
+    p.A = xa; p.a_m = ldx; p.a_k = 1;
+    p.B = f.sv + ly.E; p.b_n = lg.ldn; p.b_k = 1;
+    p.outD = f.y; p.od_m = f.ldy;
+    gs.push_back(p);
+  }
+  return gemm_run_many(gs.data(), int(gs.size()), st);
+}
+
+poet_status backward_weight_many(std::vector<WBwd> &v, int64_t T, cudaStream_t st) {
+  if (v.empty()) return POET_OK;
+  const int dt = v[0].lg.dtype;
+  std::vector<Gemm> gs;
+  std::vector<const void *> xa(v.size()), dya(v.size());
+  std::vector<int64_t> ldxa(v.size()), ldya(v.size());
+  // dx = dy E, every layer in one grouped launch
+  for (size_t i = 0; i < v.size(); ++i) {
+    WBwd &b = v[i];
+    const LayerGeom &lg = b.lg;
+    const WeightSaved ly = weight_saved(lg, T);
+    xa[i] = b.x; ldxa[i] = b.ldx;
+    if (!rows16(b.x, b.ldx, dt)) { xa[i] = b.sv + ly.xp; ldxa[i] = lg.ldn; }  // the forward's re-strided copy
+    dya[i] = b.dy; ldya[i] = b.lddy;
+    if (!rows16(b.dy, b.lddy, dt)) {
+      POET_TRY(copy_rows(dt, b.dy, b.lddy, T, int(lg.m), b.act1, lg.ldm, st));
+      dya[i] = b.act1; ldya[i] = lg.ldm;
+    }
     Gemm p;
     p.tag = "w0_bwd";
     p.M = int(T); p.N = int(lg.n); p.K = int(lg.m); p.dtype = dt;
-    p.A = dya; p.a_m = ldy; p.a_k = 1;
-    p.B = sv + ly.E; p.b_n = 1; p.b_k = lg.ldn;
-    p.outD = dx; p.od_m = lg.n;
-    POET_TRY(gemm_run(p, st));
+    p.A = dya[i]; p.a_m = ldya[i]; p.a_k = 1;
+    p.B = b.sv + ly.E; p.b_n = 1; p.b_k = lg.ldn;
+    p.outD = b.dx; p.od_m = b.lddx;
+    gs.push_back(p);
   }
-  if (gR.nprim == 0 && gP.nprim == 0) return POET_OK;
-  // D = dy^T x (natural order, float, split over tokens)
-  float *D = reinterpret_cast<float *>(wb + w.D);
-  float *D2 = reinterpret_cast<float *>(wb + w.D2);
-  const size_t wsz = size_t(lg.m) * lg.ldn;
-  POET_CUDA_TRY(cudaMemsetAsync(D, 0, wsz * 4, st));
-  {
+  POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
+  // D = dy^T x (natural order, float, split over tokens) for the layers with primitives
+  std::vector<std::pair<float *, int64_t>> zero;
+  gs.clear();
+  for (size_t i = 0; i < v.size(); ++i) {
+    WBwd &b = v[i];
+    const LayerGeom &lg = b.lg;
+    if (lg.R.nprim == 0 && lg.P.nprim == 0) continue;
+    zero.emplace_back(b.D, lg.m * lg.ldn);
     Gemm p;
     p.tag = "w_grad";
     p.M = int(lg.m); p.N = int(lg.n); p.K = int(T); p.dtype = dt;
-    p.A = dya; p.a_m = 1; p.a_k = ldy;
-    p.B = xa; p.b_n = 1; p.b_k = ldx;
-    p.outF = D; p.of_m = lg.ldn;
+    p.A = dya[i]; p.a_m = 1; p.a_k = ldya[i];
+    p.B = xa[i]; p.b_n = 1; p.b_k = ldxa[i];
+    p.outF = b.D; p.of_m = lg.ldn;
     p.atomic = true;
-    POET_TRY(gemm_run(p, st));
+    gs.push_back(p);
   }
-  // D_f[i][j] = D[R.perm[i]][P.perm[j]], in the element type of the GEMMs
-  const void *Df;
+  if (gs.empty()) return POET_OK;
+  POET_TRY(zero_many(zero, st));
+  POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
+  // D_f[i][j] = D[R.perm[i]][P.perm[j]] in the storage type, every layer in one launch
   if (dt == POET_BF16) {
-    POET_TRY(frame_f32_to_bf16(D, lg.ldn, L->R.perm, lg.m, int(lg.n), L->P.perm, wb + w.Z, lg.ldn, st));
-    Df = wb + w.Z;
+    std::vector<FrameItem> fr;
+    for (WBwd &b : v) {
+      if (b.lg.R.nprim == 0 && b.lg.P.nprim == 0) continue;
+      fr.push_back(FrameItem{b.D, b.lg.ldn, b.L->R.perm, b.lg.m, int(b.lg.n), b.L->P.perm, b.Df, b.lg.ldn});
+    }
+    POET_TRY(frame_many(fr, st));
   } else {
-    POET_TRY(gather_cols(POET_F32, D, lg.ldn, L->R.perm, lg.m, int(lg.n), L->P.perm, D2, lg.ldn, nullptr, 0,
-                         int(lg.n), st, "frame"));
-    Df = D2;
+    std::vector<RowPermute> fr;
+    for (WBwd &b : v) {
+      if (b.lg.R.nprim == 0 && b.lg.P.nprim == 0) continue;
+      RowPermute r;
+      r.src1 = b.D; r.ld1 = b.lg.ldn;
+      r.src_rowmap = b.L->R.perm;
+      r.rows = b.lg.m; r.d = int(b.lg.n);
+      r.perm = b.L->P.perm;
+      r.dst = b.Df; r.ldd = b.lg.ldn;
+      fr.push_back(r);
+    }
+    POET_TRY(permute_many(POET_F32, fr, st, "frame"));
   }
-  const void *Fs = gP.nprim > 0 ? static_cast<const void *>(sv + ly.F) : L->W0f;
-  const void *Hs = gR.nprim > 0 ? static_cast<const void *>(sv + ly.H) : L->W0f;
-  // the per-primitive products are small (K = n or m): split over K, summed in place
-  Gemm g2[2];
-  int ng = 0;
-  if (gR.nprim > 0) POET_CUDA_TRY(cudaMemsetAsync(GR, 0, size_t(gR.all_elems()) * 4, st));
-  if (gP.nprim > 0) POET_CUDA_TRY(cudaMemsetAsync(GP, 0, size_t(gP.all_elems()) * 4, st));
-  if (gR.nprim > 0) {  // G_R[j] = D_f[rows j] F[rows j]^T
-    Gemm &p = g2[ng++];
-    p.tag = "blk_grad";
-    p.M = gR.size; p.N = gR.size; p.K = int(lg.n); p.batch = gR.nprim; p.dtype = dt;
-    p.A = Df; p.a_m = lg.ldn; p.a_k = 1; p.a_b = int64_t(gR.size) * lg.ldn;
-    p.B = Fs; p.b_n = lg.ldn; p.b_k = 1; p.b_b = int64_t(gR.size) * lg.ldn;
-    p.outF = GR; p.of_m = gR.ld; p.of_b = gR.blk_elems();
-    p.atomic = true;
+  // G_R[j] = D_f[rows j] F[rows j]^T,  G_P[j] = H[:, cols j]^T D_f[:, cols j]
+  // (small products: split over K and summed in place; leftover ranges of K read from W0f)
+  zero.clear();
+  gs.clear();
+  for (WBwd &b : v) {
+    const LayerGeom &lg = b.lg;
+    const SideGeom &gR = lg.R, &gP = lg.P;
+    const WeightSaved ly = weight_saved(lg, T);
+    const char *W0f = static_cast<const char *>(b.L->W0f);
+    const int64_t cR = gR.covered, cP = gP.covered;
+    if (gR.nprim > 0) {
+      zero.emplace_back(b.GR, gR.all_elems());
+      Gemm p;
+      p.tag = "blk_grad";
+      p.M = gR.size; p.N = gR.size; p.batch = gR.nprim; p.dtype = dt;
+      p.a_m = lg.ldn; p.a_k = 1; p.a_b = int64_t(gR.size) * lg.ldn;
+      p.b_n = lg.ldn; p.b_k = 1; p.b_b = int64_t(gR.size) * lg.ldn;
+      p.outF = b.GR; p.of_m = gR.ld; p.of_b = gR.blk_elems();
+      p.atomic = true;
+      if (gP.nprim > 0 && cP < lg.n && col_split_ok(lg)) {
+        Gemm q = p;  // K in [0, c_P): F
+        q.K = int(cP); q.A = b.Df; q.B = b.sv + ly.F;
+        gs.push_back(q);
+        q.K = int(lg.n - cP); q.A = at(b.Df, cP, dt); q.B = at(W0f, cP, dt);  // K in [c_P, n): W0f
+        gs.push_back(q);
+      } else {
+        p.K = int(lg.n); p.A = b.Df;
+        p.B = gP.nprim > 0 ? static_cast<const void *>(b.sv + ly.F) : W0f;  // F with its leftover columns, or W0f
+        gs.push_back(p);
+      }
+    }
+    if (gP.nprim > 0) {
+      zero.emplace_back(b.GP, gP.all_elems());
+      Gemm p;
+      p.small = SMALL_GRAD;  // G_P[j] = sum over rows of H[:, cols j] x D_f[:, cols j]
+      p.tag = "blk_grad";
+      p.M = gP.size; p.N = gP.size; p.batch = gP.nprim; p.dtype = dt;
+      p.a_m = 1; p.a_k = lg.ldn; p.a_b = gP.size;
+      p.b_n = 1; p.b_k = lg.ldn; p.b_b = gP.size;
+      p.outF = b.GP; p.of_m = gP.ld; p.of_b = gP.blk_elems();
+      p.atomic = true;
+      if (gR.nprim > 0) {
+        Gemm q = p;  // K in [0, c_R): H
+        q.K = int(cR); q.A = b.sv + ly.H; q.B = b.Df;
+        gs.push_back(q);
+        if (cR < lg.m) {  // K in [c_R, m): W0f
+          q.K = int(lg.m - cR); q.A = at(W0f, cR * lg.ldn, dt); q.B = at(b.Df, cR * lg.ldn, dt);
+          gs.push_back(q);
+        }
+      } else {
+        p.K = int(lg.m); p.A = W0f; p.B = b.Df;
+        gs.push_back(p);
+      }
+    }
   }
-  if (gP.nprim > 0) {  // G_P[j] = H[:, cols j]^T D_f[:, cols j]
-    Gemm &p = g2[ng++];
-    p.tag = "blk_grad";
-    p.M = gP.size; p.N = gP.size; p.K = int(lg.m); p.batch = gP.nprim; p.dtype = dt;
-    p.A = Hs; p.a_m = 1; p.a_k = lg.ldn; p.a_b = gP.size;
-    p.B = Df; p.b_n = 1; p.b_k = lg.ldn; p.b_b = gP.size;
-    p.outF = GP; p.of_m = gP.ld; p.of_b = gP.blk_elems();
-    p.atomic = true;
-  }
-  return gemm_run_many(g2, ng, st);
+  POET_TRY(zero_many(zero, st));
+  return gemm_run_many(gs.data(), int(gs.size()), st);
 }
 
-poet_status poet_forward(const poet_layer *L, const void *x, int64_t T, void *y, void *saved, void *ws,
-                         size_t ws_bytes, poet_stream stream) {
-  CallRange nvtx_range("poet_forward");
-  clear_error();
-  LayerGeom lg;
-  POET_TRY(check_layer(L, &lg, true));
-  POET_REQUIRE(T >= 0 && T <= (int64_t(1) << 31) - 1, "poet_forward: T=%lld out of range", (long long)T);
-  if (T == 0) return POET_OK;
-  POET_REQUIRE(x && y && aligned_elem(x, lg.dtype) && aligned_elem(y, lg.dtype), "poet_forward: x/y NULL or misaligned");
-  POET_REQUIRE(saved && aligned256(saved), "poet_forward: saved NULL or not 256-byte aligned");
-  const int plan = resolve_plan(lg, T);
-  const WsLayout w = ws_layout(lg, T, plan);
-  if (!ws || ws_bytes < w.bytes || !aligned256(ws)) {
-    set_error("poet_forward: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, w.bytes);
-    return POET_ENOMEM_WS;
-  }
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (plan == POET_PLAN_WEIGHT) return forward_weight(L, lg, x, T, y, saved, static_cast<char *>(ws), w, st);
+}  // namespace
+
+// Token plan forward (the primitives act on the activations); x and y rows
+// ldx and ldy elements apart.
+static poet_status forward_token(const poet_layer *L, const LayerGeom &lg, const void *x, int64_t ldx, int64_t T,
+                                 void *y, int64_t ldy, void *saved, char *wb, const WsLayout &w, cudaStream_t st) {
   const int dt = lg.dtype;
   const size_t es = esize(dt);
   char *sv = static_cast<char *>(saved);
   void *xf = sv;
   void *vf = sv + align256(size_t(T) * lg.ldn * es);
-  char *wb = static_cast<char *>(ws);
   void *uf = wb + w.act1;
   void *yf = wb + w.act2;
   const SideGeom &gR = lg.R, &gP = lg.P;
 
   // a2: gather x into the P frame; the identity tail goes straight to uf
   const bool tailP = gP.nprim > 0 && gP.covered < lg.n;
-  POET_TRY(gather_cols(dt, x, lg.n, nullptr, T, int(lg.n), L->P.perm, xf, lg.ldn, tailP ? uf : nullptr, lg.ldn,
+  POET_TRY(gather_cols(dt, x, ldx, nullptr, T, int(lg.n), L->P.perm, xf, lg.ldn, tailP ? uf : nullptr, lg.ldn,
                        gP.covered, st));
   const void *u = xf;
   if (gP.nprim > 0) {
@@ -616,7 +756,78 @@ poet_status poet_forward(const poet_layer *L, const void *x, int64_t T, void *y,
     POET_TRY(gemm_run(blockdiag(gR, dt, T, vf, lg.ldm, state_R(&L->R, gR, dt), false, yf, lg.ldm), st));
     ysrc = yf;
   }
-  return scatter_cols(dt, ysrc, lg.ldm, vf, lg.ldm, gR.covered, T, int(lg.m), L->R.perm, y, lg.m, nullptr, st);
+  return scatter_cols(dt, ysrc, lg.ldm, vf, lg.ldm, gR.covered, T, int(lg.m), L->R.perm, y, ldy, nullptr, st);
+}
+
+
+poet_status poet_forward(const poet_layer *L, const void *x, int64_t T, void *y, void *saved, void *ws,
+                         size_t ws_bytes, poet_stream stream) {
+  CallRange nvtx_range("poet_forward");
+  clear_error();
+  LayerGeom lg;
+  POET_TRY(check_layer(L, &lg, true));
+  POET_REQUIRE(T >= 0 && T <= (int64_t(1) << 31) - 1, "poet_forward: T=%lld out of range", (long long)T);
+  if (T == 0) return POET_OK;
+  POET_REQUIRE(x && y && aligned_elem(x, lg.dtype) && aligned_elem(y, lg.dtype), "poet_forward: x/y NULL or misaligned");
+  POET_REQUIRE(saved && aligned256(saved), "poet_forward: saved NULL or not 256-byte aligned");
+  const int plan = resolve_plan(lg, T);
+  const WsLayout w = ws_layout(lg, T, plan);
+  if (!ws || ws_bytes < w.bytes || !aligned256(ws)) {
+    set_error("poet_forward: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, w.bytes);
+    return POET_ENOMEM_WS;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (plan == POET_PLAN_WEIGHT) {
+    std::vector<WFwd> one{WFwd{L, lg, x, lg.n, y, lg.m, static_cast<char *>(saved), static_cast<char *>(ws) + w.Z}};
+    return forward_weight_many(one, T, st);
+  }
+  return forward_token(L, lg, x, lg.n, T, y, lg.m, saved, static_cast<char *>(ws), w, st);
+}
+
+// Token plan backward a5..a7 (dx and the per-primitive gradients); dy and dx
+// rows lddy and lddx elements apart.
+static poet_status backward_token(const poet_layer *L, const LayerGeom &lg, char *wb, const WsLayout &w,
+                                  const void *saved, const void *dy, int64_t lddy, int64_t T, void *dx, int64_t lddx,
+                                  float *GR, float *GP, cudaStream_t st) {
+  const int dt = lg.dtype;
+  const size_t es = esize(dt);
+  const SideGeom &gR = lg.R, &gP = lg.P;
+  const char *sv = static_cast<const char *>(saved);
+  const void *xf = sv;
+  const void *vf = sv + align256(size_t(T) * lg.ldn * es);
+  void *dyf = wb + w.act1, *dvf = wb + w.act2, *duf = wb + w.act3, *dxf = wb + w.act1;
+
+  // a5: gather dy into the R frame (tail straight to dvf), dv = R^T dy, G_R
+  const bool tailR = gR.nprim > 0 && gR.covered < lg.m;
+  POET_TRY(gather_cols(dt, dy, lddy, nullptr, T, int(lg.m), L->R.perm, dyf, lg.ldm, tailR ? dvf : nullptr, lg.ldm,
+                       gR.covered, st));
+  const void *dv = dyf;
+  if (gR.nprim > 0) {
+    POET_TRY(gemm_run(blockdiag(gR, dt, T, dyf, lg.ldm, state_R(&L->R, gR, dt), true, dvf, lg.ldm), st));
+    dv = dvf;
+    POET_CUDA_TRY(cudaMemsetAsync(GR, 0, size_t(gR.all_elems()) * 4, st));
+    POET_TRY(gemm_run(blockgrad(gR, dt, T, dyf, vf, lg.ldm, GR), st));
+  }
+  // a6: du = dv W0f
+  {
+    Gemm p;
+    p.tag = "w0_bwd";
+    p.M = int(T); p.N = int(lg.n); p.K = int(lg.m); p.dtype = dt;
+    p.A = dv; p.a_m = lg.ldm; p.a_k = 1;
+    p.B = L->W0f; p.b_n = 1; p.b_k = lg.ldn;
+    p.outD = duf; p.od_m = lg.ldn;
+    POET_TRY(gemm_run(p, st));
+  }
+  // a7: G_P, dx = P^T du, scatter (tail straight from du)
+  const void *dxsrc = duf;
+  if (gP.nprim > 0) {
+    POET_CUDA_TRY(cudaMemsetAsync(GP, 0, size_t(gP.all_elems()) * 4, st));
+    POET_TRY(gemm_run(blockgrad(gP, dt, T, duf, xf, lg.ldn, GP), st));
+    POET_TRY(gemm_run(blockdiag(gP, dt, T, duf, lg.ldn, state_R(&L->P, gP, dt), true, dxf, lg.ldn), st));
+    dxsrc = dxf;
+  }
+  POET_TRY(scatter_cols(dt, dxsrc, lg.ldn, duf, lg.ldn, gP.covered, T, int(lg.n), L->P.perm, dx, lddx, nullptr, st));
+  return POET_OK;
 }
 
 static poet_status backward_core(const poet_layer *L, const LayerGeom &lg, int plan, char *wb, const WsLayout &w,
@@ -629,46 +840,15 @@ static poet_status backward_core(const poet_layer *L, const LayerGeom &lg, int p
     POET_REQUIRE(dy && dx && aligned_elem(dy, dt) && aligned_elem(dx, dt), "backward: dy/dx NULL or misaligned");
     POET_REQUIRE(x && aligned_elem(x, dt), "backward: x NULL or misaligned (the weight plan reads x)");
     POET_REQUIRE(saved && aligned256(saved), "backward: saved NULL or not 256-byte aligned");
-    return backward_weight(L, lg, wb, w, x, saved, dy, T, dx, GR, GP, st);
+    std::vector<WBwd> one{WBwd{L, lg, x, lg.n, static_cast<const char *>(saved), dy, lg.m, dx, lg.n, GR, GP,
+                               wb + w.act1, reinterpret_cast<float *>(wb + w.D),
+                               lg.dtype == POET_BF16 ? static_cast<void *>(wb + w.Z) : static_cast<void *>(wb + w.D2)}};
+    return backward_weight_many(one, T, st);
   }
   if (T > 0) {
     POET_REQUIRE(dy && dx && aligned_elem(dy, dt) && aligned_elem(dx, dt), "backward: dy/dx NULL or misaligned");
     POET_REQUIRE(saved && aligned256(saved), "backward: saved NULL or not 256-byte aligned");
-    const char *sv = static_cast<const char *>(saved);
-    const void *xf = sv;
-    const void *vf = sv + align256(size_t(T) * lg.ldn * es);
-    void *dyf = wb + w.act1, *dvf = wb + w.act2, *duf = wb + w.act3, *dxf = wb + w.act1;
-
-    // a5: gather dy into the R frame (tail straight to dvf), dv = R^T dy, G_R
-    const bool tailR = gR.nprim > 0 && gR.covered < lg.m;
-    POET_TRY(gather_cols(dt, dy, lg.m, nullptr, T, int(lg.m), L->R.perm, dyf, lg.ldm, tailR ? dvf : nullptr, lg.ldm,
-                         gR.covered, st));
-    const void *dv = dyf;
-    if (gR.nprim > 0) {
-      POET_TRY(gemm_run(blockdiag(gR, dt, T, dyf, lg.ldm, state_R(&L->R, gR, dt), true, dvf, lg.ldm), st));
-      dv = dvf;
-      POET_CUDA_TRY(cudaMemsetAsync(GR, 0, size_t(gR.all_elems()) * 4, st));
-      POET_TRY(gemm_run(blockgrad(gR, dt, T, dyf, vf, lg.ldm, GR), st));
-    }
-    // a6: du = dv W0f
-    {
-      Gemm p;
-      p.tag = "w0_bwd";
-      p.M = int(T); p.N = int(lg.n); p.K = int(lg.m); p.dtype = dt;
-      p.A = dv; p.a_m = lg.ldm; p.a_k = 1;
-      p.B = L->W0f; p.b_n = 1; p.b_k = lg.ldn;
-      p.outD = duf; p.od_m = lg.ldn;
-      POET_TRY(gemm_run(p, st));
-    }
-    // a7: G_P, dx = P^T du, scatter (tail straight from du)
-    const void *dxsrc = duf;
-    if (gP.nprim > 0) {
-      POET_CUDA_TRY(cudaMemsetAsync(GP, 0, size_t(gP.all_elems()) * 4, st));
-      POET_TRY(gemm_run(blockgrad(gP, dt, T, duf, xf, lg.ldn, GP), st));
-      POET_TRY(gemm_run(blockdiag(gP, dt, T, duf, lg.ldn, state_R(&L->P, gP, dt), true, dxf, lg.ldn), st));
-      dxsrc = dxf;
-    }
-    POET_TRY(scatter_cols(dt, dxsrc, lg.ldn, duf, lg.ldn, gP.covered, T, int(lg.n), L->P.perm, dx, lg.n, nullptr, st));
+    POET_TRY(backward_token(L, lg, wb, w, saved, dy, lg.m, T, dx, lg.n, GR, GP, st));
   } else {
     if (gR.nprim > 0) POET_CUDA_TRY(cudaMemsetAsync(GR, 0, size_t(gR.all_elems()) * 4, st));
     if (gP.nprim > 0) POET_CUDA_TRY(cudaMemsetAsync(GP, 0, size_t(gP.all_elems()) * 4, st));
@@ -725,10 +905,189 @@ poet_status poet_backward_blocks(const poet_layer *L, const void *x, const void 
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
+// Workspace of the grouped calls.  Token-plan layers run one after another,
+// each with its single-layer workspace at offset 0; every weight-plan layer
+// has a region of its own after that: D (float m x ldn), D_f (m x ldn in the
+// storage type; the forward keeps E_f there) and, when dy's rows are not
+// 16-byte aligned, a re-strided copy of dy (T x ldm).
+struct ManyLayout {
+  std::vector<int> plan;
+  std::vector<size_t> region;   // weight-plan layers: offset of the layer's region
+  std::vector<char> dy_copy;    // weight-plan layers: the region holds a re-strided dy
+  size_t D_bytes(const LayerGeom &lg) const { return align256(size_t(lg.m) * lg.ldn * 4); }
+  size_t Df_bytes(const LayerGeom &lg) const { return align256(size_t(lg.m) * lg.ldn * esize(lg.dtype)); }
+  size_t bytes = 0;
+};
+
+static ManyLayout many_layout(const std::vector<LayerGeom> &geoms, int64_t T, const int64_t *lddy) {
+  ManyLayout M;
+  const size_t n = geoms.size();
+  M.plan.resize(n);
+  M.region.assign(n, 0);
+  M.dy_copy.assign(n, 0);
+  size_t token = 0;
+  for (size_t i = 0; i < n; ++i) {
+    M.plan[i] = resolve_plan(geoms[i], T);
+    if (M.plan[i] == POET_PLAN_TOKEN) {
+      const size_t b = ws_layout(geoms[i], T, POET_PLAN_TOKEN).bytes;
+      if (b > token) token = b;
+    }
+  }
+  size_t off = align256(token);
+  for (size_t i = 0; i < n; ++i) {
+    if (M.plan[i] != POET_PLAN_WEIGHT) continue;
+    const LayerGeom &lg = geoms[i];
+    const int64_t ld = lddy ? lddy[i] : lg.m;
+    M.region[i] = off;
+    off += M.D_bytes(lg) + M.Df_bytes(lg);
+    if ((ld * int64_t(esize(lg.dtype))) % 16 != 0) {
+      M.dy_copy[i] = 1;
+      off += align256(size_t(T) * lg.ldm * esize(lg.dtype));
+    }
+  }
+  M.bytes = off;
+  return M;
+}
+
+// Validation shared by the grouped calls: every layer complete and of one
+// element type, T in range, row strides at least the rows' widths.
+static poet_status check_many(const char *fn, const poet_layer *layers, int32_t count, int64_t T,
+                              std::vector<LayerGeom> *geoms) {
+  POET_REQUIRE(count >= 0 && (count == 0 || layers), "%s: bad layer list", fn);
+  POET_REQUIRE(T >= 0 && T <= (int64_t(1) << 31) - 1, "%s: T=%lld out of range", fn, (long long)T);
+  geoms->resize(count);
+  for (int i = 0; i < count; ++i) {
+    poet_status st = check_layer(&layers[i], &(*geoms)[i], true);
+    if (st != POET_OK) return st;
+    POET_REQUIRE(layers[i].dtype == layers[0].dtype, "%s: layer %d has another element type than layer 0", fn, i);
+  }
+  return POET_OK;
+}
+
+static poet_status check_rows(const char *fn, const char *what, int i, const void *p, int64_t ld, int64_t width,
+                              int dtype) {
+  POET_REQUIRE(p && aligned_elem(p, dtype), "%s: %s[%d] NULL or misaligned", fn, what, i);
+  POET_REQUIRE(ld >= width, "%s: row stride of %s[%d] (%lld) below its width %lld", fn, what, i, (long long)ld,
+               (long long)width);
+  return POET_OK;
+}
+
 size_t poet_block_grad_bytes(const poet_side *side) {
   SideGeom g;
   if (!side_geom(side, &g)) return 0;
   return size_t(g.all_elems()) * 4;
+}
+
+size_t poet_many_workspace_bytes(const poet_layer *layers, int32_t count, int64_t T, const int64_t *lddy) {
+  if (count < 0 || (count > 0 && !layers) || T < 0) return 0;
+  std::vector<LayerGeom> geoms(count);
+  for (int i = 0; i < count; ++i)
+    if (!shape_geom(&layers[i], &geoms[i])) return 0;
+  return many_layout(geoms, T, lddy).bytes;
+}
+
+poet_status poet_forward_many(const poet_layer *layers, int32_t count, const void *const *x, const int64_t *ldx,
+                              int64_t T, void *const *y, const int64_t *ldy, void *const *saved, void *ws,
+                              size_t ws_bytes, poet_stream stream) {
+  CallRange nvtx_range("poet_forward_many");
+  clear_error();
+  std::vector<LayerGeom> geoms;
+  POET_TRY(check_many("poet_forward_many", layers, count, T, &geoms));
+  if (count == 0 || T == 0) return POET_OK;
+  POET_REQUIRE(x && y && saved, "poet_forward_many: x, y and saved lists must not be NULL");
+  for (int i = 0; i < count; ++i) {
+    const LayerGeom &lg = geoms[i];
+    POET_TRY(check_rows("poet_forward_many", "x", i, x[i], ldx ? ldx[i] : lg.n, lg.n, lg.dtype));
+    POET_TRY(check_rows("poet_forward_many", "y", i, y[i], ldy ? ldy[i] : lg.m, lg.m, lg.dtype));
+    POET_REQUIRE(saved[i] && aligned256(saved[i]), "poet_forward_many: saved[%d] NULL or not 256-byte aligned", i);
+  }
+  const ManyLayout M = many_layout(geoms, T, nullptr);
+  if (!ws || ws_bytes < M.bytes || !aligned256(ws)) {
+    set_error("poet_forward_many: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, M.bytes);
+    return POET_ENOMEM_WS;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char *wb = static_cast<char *>(ws);
+  std::vector<WFwd> wl;
+  for (int i = 0; i < count; ++i) {
+    if (M.plan[i] != POET_PLAN_WEIGHT) continue;
+    const LayerGeom &lg = geoms[i];
+    wl.push_back(WFwd{&layers[i], lg, x[i], ldx ? ldx[i] : lg.n, y[i], ldy ? ldy[i] : lg.m,
+                      static_cast<char *>(saved[i]), wb + M.region[i] + M.D_bytes(lg)});
+  }
+  POET_TRY(forward_weight_many(wl, T, st));
+  for (int i = 0; i < count; ++i) {  // token-plan layers, one after another
+    if (M.plan[i] != POET_PLAN_TOKEN) continue;
+    const LayerGeom &lg = geoms[i];
+    POET_TRY(forward_token(&layers[i], lg, x[i], ldx ? ldx[i] : lg.n, T, y[i], ldy ? ldy[i] : lg.m, saved[i], wb,
+                           ws_layout(lg, T, POET_PLAN_TOKEN), st));
+  }
+  return POET_OK;
+}
+
+poet_status poet_backward_blocks_many(const poet_layer *layers, int32_t count, const void *const *x,
+                                      const int64_t *ldx, const void *const *saved, const void *const *dy,
+                                      const int64_t *lddy, int64_t T, void *const *dx, const int64_t *lddx,
+                                      float *const *G_R, float *const *G_P, void *ws, size_t ws_bytes,
+                                      poet_stream stream) {
+  CallRange nvtx_range("poet_backward_blocks_many");
+  clear_error();
+  std::vector<LayerGeom> geoms;
+  POET_TRY(check_many("poet_backward_blocks_many", layers, count, T, &geoms));
+  if (count == 0) return POET_OK;
+  POET_REQUIRE(G_R && G_P, "poet_backward_blocks_many: G_R and G_P lists must not be NULL");
+  for (int i = 0; i < count; ++i) {
+    POET_REQUIRE(geoms[i].R.nprim == 0 || (G_R[i] && (reinterpret_cast<uintptr_t>(G_R[i]) & 15) == 0),
+                 "poet_backward_blocks_many: G_R[%d] NULL or not 16-byte aligned", i);
+    POET_REQUIRE(geoms[i].P.nprim == 0 || (G_P[i] && (reinterpret_cast<uintptr_t>(G_P[i]) & 15) == 0),
+                 "poet_backward_blocks_many: G_P[%d] NULL or not 16-byte aligned", i);
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {  // no tokens: every per-primitive gradient is zero
+    std::vector<std::pair<float *, int64_t>> zero;
+    for (int i = 0; i < count; ++i) {
+      if (geoms[i].R.nprim > 0) zero.emplace_back(G_R[i], geoms[i].R.all_elems());
+      if (geoms[i].P.nprim > 0) zero.emplace_back(G_P[i], geoms[i].P.all_elems());
+    }
+    return zero_many(zero, st);
+  }
+  POET_REQUIRE(x && saved && dy && dx, "poet_backward_blocks_many: x, saved, dy and dx lists must not be NULL");
+  const ManyLayout M = many_layout(geoms, T, lddy);
+  for (int i = 0; i < count; ++i) {
+    const LayerGeom &lg = geoms[i];
+    const int64_t ld_dy = lddy ? lddy[i] : lg.m;
+    POET_TRY(check_rows("poet_backward_blocks_many", "dy", i, dy[i], ld_dy, lg.m, lg.dtype));
+    POET_TRY(check_rows("poet_backward_blocks_many", "dx", i, dx[i], lddx ? lddx[i] : lg.n, lg.n, lg.dtype));
+    POET_REQUIRE(saved[i] && aligned256(saved[i]), "poet_backward_blocks_many: saved[%d] NULL or not 256-byte aligned",
+                 i);
+    if (M.plan[i] == POET_PLAN_WEIGHT) {
+      POET_TRY(check_rows("poet_backward_blocks_many", "x", i, x[i], ldx ? ldx[i] : lg.n, lg.n, lg.dtype));
+      POET_REQUIRE(M.dy_copy[i] || rows16(dy[i], ld_dy, lg.dtype),
+                   "poet_backward_blocks_many: dy[%d] must start on a 16-byte boundary (its row stride is)", i);
+    }
+  }
+  if (!ws || ws_bytes < M.bytes || !aligned256(ws)) {
+    set_error("poet_backward_blocks_many: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, M.bytes);
+    return POET_ENOMEM_WS;
+  }
+  char *wb = static_cast<char *>(ws);
+  std::vector<WBwd> wl;
+  for (int i = 0; i < count; ++i) {
+    if (M.plan[i] != POET_PLAN_WEIGHT) continue;
+    const LayerGeom &lg = geoms[i];
+    char *r = wb + M.region[i];
+    wl.push_back(WBwd{&layers[i], lg, x[i], ldx ? ldx[i] : lg.n, static_cast<const char *>(saved[i]), dy[i],
+                      lddy ? lddy[i] : lg.m, dx[i], lddx ? lddx[i] : lg.n, G_R[i], G_P[i],
+                      r + M.D_bytes(lg) + M.Df_bytes(lg), reinterpret_cast<float *>(r), r + M.D_bytes(lg)});
+  }
+  POET_TRY(backward_weight_many(wl, T, st));
+  for (int i = 0; i < count; ++i) {  // token-plan layers, one after another
+    if (M.plan[i] != POET_PLAN_TOKEN) continue;
+    const LayerGeom &lg = geoms[i];
+    POET_TRY(backward_token(&layers[i], lg, wb, ws_layout(lg, T, POET_PLAN_TOKEN), saved[i], dy[i],
+                            lddy ? lddy[i] : lg.m, T, dx[i], lddx ? lddx[i] : lg.n, G_R[i], G_P[i], st));
+  }
+  return POET_OK;
 }
 
 poet_status poet_cayley_neumann_many(const poet_side *sides, int32_t count, int32_t dtype, poet_stream stream) {
@@ -757,31 +1116,68 @@ size_t poet_cayley_neumann_grad_many_workspace_bytes(const poet_side *sides, int
   return total;
 }
 
+static poet_status grad_many_impl(const char *fn, const poet_side *sides, const float *const *G,
+                                  float *const *dtheta, int32_t count, int32_t dtype, void *ws, size_t ws_bytes,
+                                  cudaStream_t st, const AdamW *adam, float *const *m, float *const *v) {
+  POET_REQUIRE(count >= 0 && (count == 0 || (sides && G && (dtheta || adam))), "%s: bad lists", fn);
+  POET_REQUIRE(!adam || count == 0 || (m && v), "%s: moment lists must not be NULL", fn);
+  POET_REQUIRE(dtype == POET_F32 || dtype == POET_BF16, "%s: bad dtype %d", fn, dtype);
+  std::vector<SideGeom> geoms(count);
+  std::vector<void *> scratch(count, nullptr);
+  size_t off = 0;
+  auto ok4 = [](const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 3) == 0; };
+  for (int i = 0; i < count; ++i) {
+    POET_REQUIRE(side_geom(&sides[i], &geoms[i]), "%s: side %d malformed", fn, i);
+    if (geoms[i].nprim == 0 || geoms[i].size < 2) continue;
+    POET_REQUIRE(sides[i].state && aligned256(sides[i].state) && G[i] && (reinterpret_cast<uintptr_t>(G[i]) & 15) == 0,
+                 "%s: side %d state/G NULL or misaligned", fn, i);
+    if (adam) {
+      POET_REQUIRE(ok4(sides[i].theta) && ok4(m[i]) && ok4(v[i]) && (!dtheta || !dtheta[i] || ok4(dtheta[i])),
+                   "%s: side %d theta/m/v NULL or misaligned", fn, i);
+    } else {
+      POET_REQUIRE(dtheta[i] != nullptr, "%s: side %d dtheta is NULL", fn, i);
+    }
+    scratch[i] = static_cast<char *>(ws) + off;
+    off += align256(cnp_many_scratch_bytes(geoms[i], dtype));
+  }
+  if (off > 0 && (!ws || ws_bytes < off || !aligned256(ws))) {
+    set_error("%s: workspace %zu bytes, need %zu (256-byte aligned)", fn, ws_bytes, off);
+    return POET_ENOMEM_WS;
+  }
+  return cnp_backward_many(sides, geoms.data(), count, dtype, G, dtheta, scratch.data(), st, adam, m, v);
+}
+
 poet_status poet_cayley_neumann_grad_many(const poet_side *sides, const float *const *G, float *const *dtheta,
                                           int32_t count, int32_t dtype, void *ws, size_t ws_bytes,
                                           poet_stream stream) {
   CallRange nvtx_range("poet_cayley_neumann_grad_many");
   clear_error();
-  POET_REQUIRE(count >= 0 && (count == 0 || (sides && G && dtheta)), "poet_cayley_neumann_grad_many: bad lists");
-  POET_REQUIRE(dtype == POET_F32 || dtype == POET_BF16, "poet_cayley_neumann_grad_many: bad dtype %d", dtype);
-  std::vector<SideGeom> geoms(count);
-  std::vector<void *> scratch(count, nullptr);
-  size_t off = 0;
-  for (int i = 0; i < count; ++i) {
-    POET_REQUIRE(side_geom(&sides[i], &geoms[i]), "poet_cayley_neumann_grad_many: side %d malformed", i);
-    if (geoms[i].nprim == 0 || geoms[i].size < 2) continue;
-    POET_REQUIRE(sides[i].state && aligned256(sides[i].state) && G[i] && dtheta[i] &&
-                     (reinterpret_cast<uintptr_t>(G[i]) & 15) == 0,
-                 "poet_cayley_neumann_grad_many: side %d state/G/dtheta NULL or misaligned", i);
-    scratch[i] = static_cast<char *>(ws) + off;
-    off += align256(cnp_many_scratch_bytes(geoms[i], dtype));
-  }
-  if (off > 0 && (!ws || ws_bytes < off || !aligned256(ws))) {
-    set_error("poet_cayley_neumann_grad_many: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, off);
-    return POET_ENOMEM_WS;
-  }
-  return cnp_backward_many(sides, geoms.data(), count, dtype, G, dtheta, scratch.data(),
-                           reinterpret_cast<cudaStream_t>(stream));
+  return grad_many_impl("poet_cayley_neumann_grad_many", sides, G, dtheta, count, dtype, ws, ws_bytes,
+                        reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr);
+}
+
+static poet_status check_adamw(const char *fn, float lr, float beta1, float beta2, float eps, float weight_decay,
+                               int32_t step) {
+  POET_REQUIRE(step >= 1, "%s: step=%d < 1", fn, step);
+  POET_REQUIRE(std::isfinite(lr) && lr >= 0.f && std::isfinite(weight_decay) && weight_decay >= 0.f,
+               "%s: lr and weight_decay must be finite and >= 0", fn);
+  POET_REQUIRE(beta1 >= 0.f && beta1 < 1.f && beta2 >= 0.f && beta2 < 1.f, "%s: betas outside [0, 1)", fn);
+  POET_REQUIRE(std::isfinite(eps) && eps > 0.f, "%s: eps must be > 0", fn);
+  return POET_OK;
+}
+
+poet_status poet_cayley_neumann_grad_many_adamw(const poet_side *sides, const float *const *G, float *const *m,
+                                                float *const *v, float *const *dtheta, int32_t count,
+                                                int32_t dtype, const poet_adamw_hparams *h, void *ws,
+                                                size_t ws_bytes, poet_stream stream) {
+  CallRange nvtx_range("poet_cayley_neumann_grad_many_adamw");
+  clear_error();
+  const char *fn = "poet_cayley_neumann_grad_many_adamw";
+  POET_REQUIRE(h != nullptr, "%s: hyperparameters are NULL", fn);
+  POET_TRY(check_adamw(fn, h->lr, h->beta1, h->beta2, h->eps, h->weight_decay, h->step));
+  const AdamW a = adamw_of(h->lr, h->beta1, h->beta2, h->eps, h->weight_decay, h->step);
+  return grad_many_impl(fn, sides, G, dtheta, count, dtype, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
+                        &a, m, v);
 }
 
 poet_status poet_prepare(poet_layer *L, poet_stream stream) {
@@ -870,6 +1266,25 @@ poet_status poet_merge(poet_layer *L, void *ws, size_t ws_bytes, poet_stream str
   return POET_OK;
 }
 
+poet_status poet_merge_reset_moments(poet_layer *L, float *m_R, float *v_R, float *m_P, float *v_P, void *ws,
+                                     size_t ws_bytes, poet_stream stream) {
+  CallRange nvtx_range("poet_merge_reset_moments");
+  clear_error();
+  LayerGeom lg;
+  POET_TRY(check_layer(L, &lg, true));
+  const int64_t nR = int64_t(lg.R.nprim) * lg.R.packed_per(), nP = int64_t(lg.P.nprim) * lg.P.packed_per();
+  auto ok4 = [](const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 3) == 0; };
+  POET_REQUIRE(nR == 0 || (ok4(m_R) && ok4(v_R)), "poet_merge_reset_moments: R moments NULL or misaligned");
+  POET_REQUIRE(nP == 0 || (ok4(m_P) && ok4(v_P)), "poet_merge_reset_moments: P moments NULL or misaligned");
+  POET_TRY(poet_merge(L, ws, ws_bytes, stream));
+  std::vector<std::pair<float *, int64_t>> zero;
+  if (nR > 0) { zero.emplace_back(m_R, nR); zero.emplace_back(v_R, nR); }
+  if (nP > 0) { zero.emplace_back(m_P, nP); zero.emplace_back(v_P, nP); }
+  return zero_many(zero, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t poet_workspace_size(const poet_layer *L, int64_t T) { return poet_workspace_bytes(L, T); }
+
 poet_status poet_gemm(int32_t dtype, int32_t M, int32_t N, int32_t K, int32_t batch, const void *A, int64_t sAm,
                       int64_t sAk, int64_t sAb, const void *B, int64_t sBn, int64_t sBk, int64_t sBb, void *C,
                       int64_t ldc, int64_t sCb, float alpha, float beta, poet_stream stream) {
@@ -894,11 +1309,7 @@ poet_status poet_adamw_step(float *theta, const float *grad, float *m, float *v,
   CallRange nvtx_range("poet_adamw_step");
   clear_error();
   POET_REQUIRE(n >= 0, "poet_adamw_step: n=%lld < 0", (long long)n);
-  POET_REQUIRE(step >= 1, "poet_adamw_step: step=%d < 1", step);
-  POET_REQUIRE(std::isfinite(lr) && lr >= 0.f && std::isfinite(weight_decay) && weight_decay >= 0.f,
-               "poet_adamw_step: lr and weight_decay must be finite and >= 0");
-  POET_REQUIRE(beta1 >= 0.f && beta1 < 1.f && beta2 >= 0.f && beta2 < 1.f, "poet_adamw_step: betas outside [0, 1)");
-  POET_REQUIRE(std::isfinite(eps) && eps > 0.f, "poet_adamw_step: eps must be > 0");
+  POET_TRY(check_adamw("poet_adamw_step", lr, beta1, beta2, eps, weight_decay, step));
   if (n == 0) return POET_OK;
   auto ok = [](const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 3) == 0; };
   POET_REQUIRE(ok(theta) && ok(grad) && ok(m) && ok(v), "poet_adamw_step: NULL or misaligned buffer");

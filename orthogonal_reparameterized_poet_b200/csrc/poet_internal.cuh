@@ -6,6 +6,9 @@
 #include <stdint.h>
 #include <stddef.h>
 
+#include <utility>
+#include <vector>
+
 #include "poet.h"
 
 namespace poet {
@@ -119,7 +122,14 @@ struct Gemm {
   void *outD = nullptr; int64_t od_m = 0, od_b = 0;
   bool atomic = false;
   const char *tag = "gemm";                   // kind for tracing
+  // A block-diagonal product of one side's primitives, which primitives of
+  // size <= 32 run on the small-block kernels instead:
+  //   SMALL_RIGHT: out[r][j*s + a] = sum_c A[r][j*s + c] B_j(a, c)  (M = rows, N = K = s)
+  //   SMALL_LEFT:  out[j*s + a][k] = sum_c A_j[a][c] B[j*s + c][k]  (M = K = s, N = columns)
+  //   SMALL_GRAD:  outF_j[a][c] += sum_r A[r][j*s + a] B[r][j*s + c] (M = N = s, K = rows)
+  int small = 0;
 };
+enum { SMALL_RIGHT = 1, SMALL_LEFT = 2, SMALL_GRAD = 3 };
 
 poet_status gemm_run(const Gemm &g, cudaStream_t st);       // picks the engine
 poet_status gemm_simt(const Gemm &g, cudaStream_t st);      // CUDA-core FMA engine
@@ -132,6 +142,19 @@ poet_status gemm_run_many(const Gemm *gs, int count, cudaStream_t st);
 // One CTA whose bounded wait on a barrier nothing arrives on runs out (tests failure detection).
 poet_status selftest_bounded_wait(uint32_t timeout_us, cudaStream_t st);
 bool gemm_tc_enabled();
+
+// Small-block kernels (primitive size <= 32, CUDA cores; see smallb.cu).
+bool smallb_supported(int size);
+poet_status smallb_right(int dtype, const void *X, int64_t ldx, int64_t rows, const void *M, int64_t ldm,
+                         int64_t bstride, int nprim, int s, bool trans, void *out, int64_t ldo, cudaStream_t st,
+                         const char *kind);
+poet_status smallb_left(int dtype, const void *X, int64_t ldx, int64_t cols, const void *M, int64_t ldm,
+                        int64_t bstride, int nprim, int s, bool trans, void *out, int64_t ldo, cudaStream_t st,
+                        const char *kind);
+poet_status smallb_grad(int dtype, const void *D, const void *V, int64_t ld, int64_t rows, int nprim, int s, float *G,
+                        int64_t ldg, int64_t gstride, cudaStream_t st);
+// Runs g on the small-block kernels if it is a marked block product they serve (*done = true).
+poet_status smallb_dispatch(const Gemm &g, cudaStream_t st, bool *done);
 
 // ------------------------------------------------------------------ data movement
 
@@ -157,6 +180,59 @@ poet_status scatter_cols(int dtype, const void *src1, int64_t ld1, const void *s
                          void *dst, int64_t ld_dst, const int32_t *rowmap, cudaStream_t st,
                          const char *kind = "scatter");
 
+// Many row permutations in one launch (weight-sized matrices of several
+// layers).  Output row r of item i: dst[dstrow(r)][j] = src(r)[map[j]] for
+// j < d, where src(r) = row srcrow(r) of src1 for columns < split and of src2
+// for columns >= split (src2 = nullptr: src1 only), map = perm (inverse = 0),
+// perm^-1 (inverse = 1) or the identity (perm = nullptr), and srcrow/dstrow
+// are the row maps (nullptr: r) whose entries must lie in [0, map_rows)
+// (map_rows = 0: [0, rows)).  Rows may start at any element boundary.
+struct RowPermute {
+  const void *src1 = nullptr; int64_t ld1 = 0;
+  const void *src2 = nullptr; int64_t ld2 = 0; int split = 0;
+  const int32_t *src_rowmap = nullptr;
+  int64_t rows = 0; int d = 0;
+  const int32_t *perm = nullptr; int inverse = 0;
+  void *dst = nullptr; int64_t ldd = 0;
+  const int32_t *dst_rowmap = nullptr;
+  int64_t map_rows = 0;
+};
+poet_status permute_many(int dtype, const std::vector<RowPermute> &v, cudaStream_t st, const char *kind);
+
+// out[a][c] = bf16(D[rowmap[a]][perm[c]]) for several matrices in one launch.
+struct FrameItem {
+  const float *D; int64_t ldD;
+  const int32_t *rowmap; int64_t rows; int d;
+  const int32_t *perm;
+  void *out; int64_t ld_out;
+};
+poet_status frame_many(const std::vector<FrameItem> &v, cudaStream_t st);
+
+// Zero several float buffers in one launch.
+poet_status zero_many(const std::vector<std::pair<float *, int64_t>> &v, cudaStream_t st);
+
+// ------------------------------------------------------------------ optimizer step
+
+// AdamW hyperparameters of one step with the bias corrections 1 - beta^step.
+struct AdamW {
+  float lr, beta1, beta2, eps, wd;
+  float bc1, bc2;
+};
+AdamW adamw_of(float lr, float beta1, float beta2, float eps, float weight_decay, int32_t step);
+
+// One parameter's AdamW update (decoupled weight decay, bias-corrected moments).
+__device__ __forceinline__ void adamw_one(float &theta, float g, float &m, float &v, const AdamW &h) {
+  m = h.beta1 * m + (1.f - h.beta1) * g;
+  v = h.beta2 * v + (1.f - h.beta2) * g * g;
+  const float m_hat = m / h.bc1;
+  const float v_hat = v / h.bc2;
+  theta = theta - h.lr * (m_hat / (sqrtf(v_hat) + h.eps) + h.wd * theta);
+}
+
+// One AdamW step on n float parameters in place (see poet_adamw_step).
+poet_status adamw_step(float *theta, const float *grad, float *m, float *v, int64_t n, float lr, float beta1,
+                       float beta2, float eps, float weight_decay, int32_t step, cudaStream_t st);
+
 // ------------------------------------------------------------------ Cayley-Neumann
 
 poet_status cnp_forward(const poet_side *side, const SideGeom &g, int dtype, cudaStream_t st);
@@ -167,17 +243,14 @@ size_t cnp_scratch_bytes(const SideGeom &g, int dtype);
 // The same for many sides at once; their GEMM steps share grouped launches.
 // G[i]: float [nprim][ld][ld]; scratch[i]: cnp_many_scratch_bytes(geoms[i], dtype) bytes each.
 poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int count, int dtype, cudaStream_t st);
+// With adam != nullptr the packing also applies that AdamW step to each side's
+// theta with moments m[i], v[i] (dtheta[i] may then be nullptr).
 poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int count, int dtype,
-                              const float *const *G, float *const *dtheta, void *const *scratch, cudaStream_t st);
+                              const float *const *G, float *const *dtheta, void *const *scratch, cudaStream_t st,
+                              const AdamW *adam = nullptr, float *const *m = nullptr, float *const *v = nullptr);
 size_t cnp_many_scratch_bytes(const SideGeom &g, int dtype);
 // out = G (dense [nprim][size][size]) re-laid as [nprim][ld][ld] with zero padding
 poet_status pad_blocks(const float *G, const SideGeom &g, float *out, cudaStream_t st);
-
-// ------------------------------------------------------------------ optimizer step
-
-// One AdamW step on n float parameters in place (see poet_adamw_step).
-poet_status adamw_step(float *theta, const float *grad, float *m, float *v, int64_t n, float lr, float beta1,
-                       float beta2, float eps, float weight_decay, int32_t step, cudaStream_t st);
 
 // ------------------------------------------------------------------ permutations
 

@@ -39,6 +39,11 @@ class poet_layer(ctypes.Structure):
                 ("R", poet_side), ("P", poet_side)]
 
 
+class poet_adamw_hparams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
+                ("weight_decay", ctypes.c_float), ("step", ctypes.c_int32)]
+
+
 class poet_trace_row(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_char * 32), ("launches", ctypes.c_int64), ("ms", ctypes.c_double),
                 ("flop", ctypes.c_double), ("bytes", ctypes.c_double)]
@@ -78,6 +83,16 @@ _SIGS = {
     "poet_backward_blocks": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "poet_many_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_layer), ctypes.c_int32, ctypes.c_int64,
+                                                     ctypes.c_void_p]),
+    "poet_forward_many": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "poet_backward_blocks_many": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_int32, ctypes.c_void_p,
+                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                                 ctypes.c_void_p]),
     "poet_cayley_neumann_grad_many_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_side), ctypes.c_int32,
                                                                         ctypes.c_int32]),
     "poet_cayley_neumann_grad_many": (ctypes.c_int, [ctypes.POINTER(poet_side), ctypes.POINTER(ctypes.c_void_p),
@@ -85,6 +100,14 @@ _SIGS = {
                                                      ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "poet_cayley_neumann_grad_noalloc": (ctypes.c_int, [ctypes.POINTER(poet_side), ctypes.c_int32, ctypes.c_void_p,
                                                         ctypes.c_void_p, ctypes.c_void_p]),
+    "poet_cayley_neumann_grad_many_adamw": (ctypes.c_int, [ctypes.POINTER(poet_side), ctypes.c_void_p, ctypes.c_void_p,
+                                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                                           ctypes.c_int32, ctypes.POINTER(poet_adamw_hparams),
+                                                           ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "poet_merge_reset_moments": (ctypes.c_int, [ctypes.POINTER(poet_layer), ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                                ctypes.c_void_p]),
+    "poet_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(poet_layer), ctypes.c_int64]),
     "poet_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_void_p]),
     "poet_adamw_step": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_int64, ctypes.c_float, ctypes.c_float, ctypes.c_float,
@@ -438,3 +461,84 @@ def cayley_neumann_grad_many(layers, G, dtheta, ws, stream=None):
     sides = [s for L in layers for s in (L.struct.R, L.struct.P)]
     poet_cayley_neumann_grad_many(sides, [t for pair in G for t in pair], [t for pair in dtheta for t in pair],
                                   layers[0].dtype, ws, stream)
+
+
+# ------------------------------------------------------------------ many layers' forward and backward
+
+def _layer_array(structs):
+    arr = (poet_layer * max(len(structs), 1))()
+    for i, L in enumerate(structs):
+        arr[i] = L
+    return arr
+
+
+def _ptrs(ts):
+    return (ctypes.c_void_p * max(len(ts), 1))(*[None if t is None else t.data_ptr() for t in ts])
+
+
+def _rows(ts):
+    """Row strides (elements) of 2-D tensors whose rows are contiguous."""
+    for t in ts:
+        if t is not None and t.dim() == 2 and t.shape[1] > 1 and t.stride(1) != 1:
+            raise ValueError("activation rows must be contiguous (stride(1) == 1)")
+    return (ctypes.c_int64 * max(len(ts), 1))(*[0 if t is None else (t.stride(0) if t.dim() == 2 else 0)
+                                                for t in ts])
+
+
+def poet_many_workspace_bytes(structs, T: int, lddy=None) -> int:
+    lds = None if lddy is None else (ctypes.c_int64 * max(len(lddy), 1))(*lddy)
+    return lib().poet_many_workspace_bytes(_layer_array(structs), len(structs), T, lds)
+
+
+def poet_forward_many(structs, x, T: int, y, saved, ws, stream=None):
+    """x, y: lists of 2-D device tensors (rows contiguous; any row stride >= the width)."""
+    _check(lib().poet_forward_many(_layer_array(structs), len(structs), _ptrs(x), _rows(x), T, _ptrs(y), _rows(y),
+                                   _ptrs(saved), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def poet_backward_blocks_many(structs, x, saved, dy, T: int, dx, G_R, G_P, ws, stream=None):
+    _check(lib().poet_backward_blocks_many(_layer_array(structs), len(structs), _ptrs(x), _rows(x), _ptrs(saved),
+                                           _ptrs(dy), _rows(dy), T, _ptrs(dx), _rows(dx), _ptrs(G_R), _ptrs(G_P),
+                                           _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def many_workspace_bytes(layers, T: int, dy=None) -> int:
+    """Workspace of forward_many / backward_blocks_many over these PoetLayers (dy: the upstream
+    gradient tensors, whose row strides decide whether a re-strided copy is needed)."""
+    lddy = None if dy is None else [t.stride(0) for t in dy]
+    return poet_many_workspace_bytes([L.struct for L in layers], T, lddy)
+
+
+def forward_many(layers, x, y, saved, ws, stream=None):
+    """Forward of independent PoetLayers in grouped launches: y[i] = layer_i(x[i])."""
+    if layers:
+        poet_forward_many([L.struct for L in layers], x, x[0].shape[0], y, saved, ws, stream)
+
+
+def backward_blocks_many(layers, x, saved, dy, dx, G, ws, stream=None):
+    """a5..a7 of independent PoetLayers in grouped launches; G = [(G_R, G_P), ...]."""
+    if layers:
+        poet_backward_blocks_many([L.struct for L in layers], x, saved, dy, dy[0].shape[0], dx,
+                                  [g[0] for g in G], [g[1] for g in G], ws, stream)
+
+
+# ------------------------------------------------------------------ a8 with the optimizer step fused
+
+def poet_cayley_neumann_grad_many_adamw(sides, G, m, v, dtype: int, ws, lr, beta1=0.9, beta2=0.999, eps=1e-8,
+                                        weight_decay=0.0, step=1, dtheta=None, stream=None):
+    """a8 for every side with the AdamW step applied to each side's theta in the packing kernel."""
+    h = poet_adamw_hparams(lr, beta1, beta2, eps, weight_decay, step)
+    n = len(sides)
+    dp = None if dtheta is None else _ptrs(dtheta)
+    _check(lib().poet_cayley_neumann_grad_many_adamw(_side_array(sides), _ptrs(G), _ptrs(m), _ptrs(v), dp, n, dtype,
+                                                     ctypes.byref(h), _ptr(ws), 0 if ws is None else ws.numel(),
+                                                     _stream(stream)))
+
+
+def poet_merge_reset_moments(layer: poet_layer, m_R, v_R, m_P, v_P, ws, stream=None):
+    _check(lib().poet_merge_reset_moments(ctypes.byref(layer), _ptr(m_R), _ptr(v_R), _ptr(m_P), _ptr(v_P), _ptr(ws),
+                                          ws.numel(), _stream(stream)))
+
+
+def poet_workspace_size(layer: poet_layer, T: int) -> int:
+    return lib().poet_workspace_size(ctypes.byref(layer), T)

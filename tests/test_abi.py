@@ -163,3 +163,42 @@ def test_auto_plan_switches_once(m, n, mode, b, dtype):
         fixed = (poet.poet_saved_bytes(L, T), poet.poet_workspace_bytes(L, T))
         L.plan = poet.PLAN_AUTO
         assert (poet.poet_saved_bytes(L, T), poet.poet_workspace_bytes(L, T)) == fixed
+
+
+def test_many_layer_calls_validate_and_size():
+    """The grouped calls: sizes grow with the list, a re-strided dy costs
+    workspace, and bad lists are rejected before anything is launched."""
+    lib = poet.lib()
+
+    def layer(m, n, dtype=poet.BF16, plan=poet.PLAN_WEIGHT, fake=1 << 20):
+        L = poet.poet_layer()
+        L.m, L.n, L.dtype, L.plan = m, n, dtype, plan
+        for sd, d in ((L.R, m), (L.P, n)):
+            sd.dim, sd.mode, sd.b, sd.k = d, poet.BS, 256, 4
+            sd.perm, sd.theta, sd.state = fake, fake, fake
+        L.W0, L.W0f = fake, fake
+        return L
+
+    one = poet.poet_many_workspace_bytes([layer(2048, 2048)], 4096)
+    two = poet.poet_many_workspace_bytes([layer(2048, 2048), layer(5461, 2048)], 4096)
+    assert 0 < one < two
+    # dy rows of 5461 bf16 elements are not 16-byte aligned: room for a re-strided copy
+    plain = poet.poet_many_workspace_bytes([layer(5461, 2048)], 4096, [5464])
+    odd = poet.poet_many_workspace_bytes([layer(5461, 2048)], 4096, [5461])
+    assert odd - plain >= 4096 * 5504 * 2
+    st = ctypes.c_void_p(0)
+    arr = (poet.poet_layer * 2)(layer(256, 256), layer(256, 256, dtype=poet.F32))
+    fake = (ctypes.c_void_p * 2)(1 << 20, 1 << 20)
+    # mixed element types
+    assert lib.poet_forward_many(arr, 2, fake, None, 16, fake, None, fake, ctypes.c_void_p(1 << 20), 1 << 30,
+                                 st) == poet.EINVAL
+    # a row stride below the width
+    arr1 = (poet.poet_layer * 1)(layer(256, 256))
+    ld = (ctypes.c_int64 * 1)(255)
+    assert lib.poet_forward_many(arr1, 1, fake, ld, 16, fake, None, fake, ctypes.c_void_p(1 << 20), 1 << 30,
+                                 st) == poet.EINVAL
+    # workspace too small
+    assert lib.poet_forward_many(arr1, 1, fake, None, 16, fake, None, fake, ctypes.c_void_p(1 << 20), 256,
+                                 st) == poet.ENOMEM_WS
+    assert lib.poet_backward_blocks_many(arr1, 1, fake, None, fake, fake, None, 16, fake, None, None, None,
+                                         ctypes.c_void_p(1 << 20), 1 << 30, st) == poet.EINVAL

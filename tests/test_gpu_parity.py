@@ -111,6 +111,9 @@ LAYER_CASES = {
     "b1_no_params": Case(40, 24, I.BS, 1, I.BS, 1, 2, 9, I.F32, 0.05),
     "b_gt_dim": Case(40, 24, I.BS, 64, I.BS, 64, 2, 9, I.F32, 0.05),
     "single_token": Case(128, 64, I.BS, 32, I.FS, 0, 2, 1, I.F32, 0.05),
+    # primitives of size <= 32 (the small-block kernels): bf16 b = 32 / 16, and fully stochastic sides of 30 / 25
+    "smallb_bs32_bf16": Case(512, 384, I.BS, 32, I.BS, 16, 4, 300, I.BF16, 0.02, layer_id=15),
+    "smallb_fs_fp32": Case(60, 50, I.FS, 0, I.FS, 0, 3, 70, I.F32, 0.05, layer_id=16),
 }
 
 
@@ -371,3 +374,187 @@ def test_adamw_step_matches_oracle(cuda, n, offset):
     assert rel_fro(th.cpu().numpy(), ref[0]) <= 1e-6
     assert rel_fro(m.cpu().numpy(), ref[1]) <= 1e-6
     assert rel_fro(v.cpu().numpy(), ref[2]) <= 1e-6
+
+
+# ------------------------------------------------------------------ grouped forward / backward of many layers
+
+GROUPED_SETS = {
+    "bf16": [  # (case, plan): FS and BS, leftover indices, an FS side whose covered width is not a 16-byte
+               # column offset (199 -> 99), sides without primitives, and token- and weight-plan layers in one list
+        (Case(512, 512, I.FS, 0, I.FS, 0, 4, 300, I.BF16, 0.02, layer_id=41), 2),
+        (Case(1376, 512, I.FS, 0, I.FS, 0, 4, 300, I.BF16, 0.02, layer_id=42), 2),
+        (Case(1024, 768, I.BS, 256, I.BS, 256, 4, 300, I.BF16, 0.02, layer_id=43), 2),
+        (Case(300, 200, I.BS, 64, I.BS, 64, 2, 300, I.BF16, 0.05, layer_id=44), 2),
+        (Case(301, 199, I.FS, 0, I.FS, 0, 3, 300, I.BF16, 0.03, layer_id=45), 2),
+        (Case(200, 341, I.BS, 64, I.FS, 0, 4, 300, I.BF16, 0.03, layer_id=46), 2),
+        (Case(40, 24, I.BS, 64, I.BS, 64, 2, 300, I.BF16, 0.05, layer_id=47), 2),
+        (Case(640, 512, I.BS, 128, I.FS, 0, 2, 300, I.BF16, 0.03, layer_id=48), 1),
+        (Case(512, 384, I.FS, 0, I.BS, 128, 4, 300, I.BF16, 0.02, layer_id=49), 0),
+        (Case(256, 200, I.BS, 32, I.BS, 16, 3, 300, I.BF16, 0.03, layer_id=50), 2),
+    ],
+    "f32": [
+        (Case(301, 200, I.FS, 0, I.BS, 48, 3, 130, I.F32, 0.03, layer_id=51), 2),
+        (Case(200, 301, I.BS, 64, I.FS, 0, 1, 130, I.F32, 0.03, layer_id=52), 2),
+        (Case(96, 130, I.FS, 0, I.FS, 0, 0, 130, I.F32, 0.03, layer_id=53), 1),
+    ],
+}
+
+
+@pytest.mark.parametrize("strided", [False, True])
+@pytest.mark.parametrize("which", sorted(GROUPED_SETS))
+def test_grouped_forward_backward_match_single_calls_and_oracle(cuda, which, strided):
+    """poet_forward_many / poet_backward_blocks_many against the single-layer
+    calls and the oracle.  strided: every activation lives in a wider row
+    (x: odd stride, so it is re-strided; y and dx: odd strides, written by the
+    unaligned epilogue; dy: a 16-byte aligned stride, read in place)."""
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    sets = GROUPED_SETS[which]
+    T = sets[0][0].T
+    built = [_make_layer(cuda, c, plan) for c, plan in sets]
+    layers = [b[0] for b in built]
+    poet.cayley_neumann_many(layers)
+    tdt = poet.torch_dtype(sets[0][0].dtype)
+
+    def strided_copy(t, extra):
+        if not strided:
+            return t.clone()
+        buf = cuda.zeros(t.shape[0], t.shape[1] + extra, dtype=t.dtype, device="cuda")
+        buf[:, : t.shape[1]] = t
+        return buf[:, : t.shape[1]]
+
+    xs = [strided_copy(b[1], 5) for b in built]
+    dys = [strided_copy(b[2], 8) for b in built]
+    ys = [strided_copy(cuda.zeros(T, c.m, dtype=tdt, device="cuda"), 3) for c, _ in sets]
+    dxs = [strided_copy(cuda.zeros(T, c.n, dtype=tdt, device="cuda"), 1) for c, _ in sets]
+    saved = [L.saved_buffer(T) for L in layers]
+    Gs = [L.block_grad_buffers() for L in layers]
+    ws = cuda.empty(max(poet.many_workspace_bytes(layers, T, dys), 1), dtype=cuda.uint8, device="cuda")
+    poet.forward_many(layers, xs, ys, saved, ws)
+    poet.backward_blocks_many(layers, xs, saved, dys, dxs, Gs, ws)
+    poet.poet_sync_status()
+    tol = TOL[sets[0][0].dtype]
+    for (L, xt, dyt, arrs), (case, plan), y, dx, (gR, gP) in zip(built, sets, ys, dxs, Gs):
+        y1, sv1 = L.forward(xt)
+        g1R, g1P = L.block_grad_buffers()
+        dx1 = L.backward_blocks(sv1, dyt, g1R, g1P, x=xt)
+        poet.poet_sync_status()
+        assert rel_fro(y.float().cpu().numpy(), y1.float().cpu().numpy()) <= 1e-5
+        assert rel_fro(dx.float().cpu().numpy(), dx1.float().cpu().numpy()) <= 1e-5
+        ref = run_oracle(case, *arrs)
+        assert rel_fro(y.float().cpu().numpy(), ref["Y"]) <= tol
+        assert rel_fro(dx.float().cpu().numpy(), ref["dX"]) <= tol
+        for g, g1, (nprim, size), key in ((gR, g1R, L.geom_R, "G_R"), (gP, g1P, L.geom_P, "G_P")):
+            if nprim == 0:
+                continue
+            ld = (size + 7) // 8 * 8
+            got = g[: nprim * ld * ld].reshape(nprim, ld, ld)[:, :size, :size].cpu().numpy()
+            one = g1[: nprim * ld * ld].reshape(nprim, ld, ld)[:, :size, :size].cpu().numpy()
+            assert rel_fro(got, one) <= MANY_VS_SINGLE[which]
+            assert rel_fro(got, ref[key]) <= tol, (case, key)
+
+
+def test_grouped_backward_with_no_tokens_zeroes_the_gradients(cuda):
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    sets = GROUPED_SETS["bf16"][:3]
+    layers = [_make_layer(cuda, c, plan)[0] for c, plan in sets]
+    poet.cayley_neumann_many(layers)
+    Gs = [L.block_grad_buffers() for L in layers]
+    for gR, gP in Gs:
+        gR.fill_(1.0)
+        gP.fill_(1.0)
+    ws = cuda.empty(max(poet.many_workspace_bytes(layers, 0), 1), dtype=cuda.uint8, device="cuda")
+    e = [cuda.empty(0, L.m, dtype=cuda.bfloat16, device="cuda") for L in layers]
+    f = [cuda.empty(0, L.n, dtype=cuda.bfloat16, device="cuda") for L in layers]
+    poet.backward_blocks_many(layers, f, [L.saved_buffer(0) for L in layers], e, f, Gs, ws)
+    poet.poet_sync_status()
+    for (gR, gP), L in zip(Gs, layers):
+        nR, sR = L.geom_R
+        nP, sP = L.geom_P
+        assert not gR[: nR * ((sR + 7) // 8 * 8) ** 2].any().item()
+        assert not gP[: nP * ((sP + 7) // 8 * 8) ** 2].any().item()
+
+
+# ------------------------------------------------------------------ a8 with the AdamW step fused
+
+@pytest.mark.parametrize("which", sorted(MANY_SETS))
+def test_fused_adamw_matches_separate_step_and_oracle(cuda, which):
+    """poet_cayley_neumann_grad_many_adamw against poet_cayley_neumann_grad_many
+    followed by poet_adamw_step (bitwise: the same gradient and the same update
+    arithmetic), and the update against the oracle's AdamW step on the
+    oracle's gradient.  Moments start nonzero and step = 3, so that every term
+    of the update matters."""
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    cases = MANY_SETS[which]
+    built = [_make_layer(cuda, c) for c in cases]
+    layers = [b[0] for b in built]
+    poet.cayley_neumann_many(layers)
+    G = []
+    for L, xt, dyt, _ in built:
+        _, saved = L.forward(xt)
+        gR, gP = L.block_grad_buffers()
+        L.backward_blocks(saved, dyt, gR, gP, x=xt)
+        G.append((gR, gP))
+    sides = [s for L in layers for s in (L.struct.R, L.struct.P)]
+    Gl = [g for pair in G for g in pair]
+    rng = np.random.default_rng(3)
+    hp = dict(lr=float(np.float32(1e-3)), beta1=float(np.float32(0.9)), beta2=float(np.float32(0.999)),
+              eps=float(np.float32(1e-8)), weight_decay=float(np.float32(0.01)), step=3)
+    th0 = [t.clone() for L in layers for t in (L.theta_R, L.theta_P)]
+    m0 = [cuda.from_numpy((0.01 * rng.standard_normal(t.numel())).astype(np.float32)).cuda() for t in th0]
+    v0 = [cuda.from_numpy((1e-4 * rng.random(t.numel())).astype(np.float32)).cuda() for t in th0]
+    ws = cuda.empty(max(poet.cayley_neumann_grad_many_workspace_bytes(layers), 1), dtype=cuda.uint8, device="cuda")
+    # separate: gradient, then the optimizer kernel
+    dth = [cuda.empty_like(t) for t in th0]
+    poet.poet_cayley_neumann_grad_many(sides, Gl, dth, layers[0].dtype, ws)
+    th_a, m_a, v_a = [t.clone() for t in th0], [t.clone() for t in m0], [t.clone() for t in v0]
+    for t, g, m, v in zip(th_a, dth, m_a, v_a):
+        if t.numel():
+            poet.poet_adamw_step(t, g, m, v, **hp)
+    # fused: the sides' own theta is updated in place
+    m_b, v_b = [t.clone() for t in m0], [t.clone() for t in v0]
+    dth_b = [cuda.full_like(t, float("nan")) for t in th0]
+    poet.poet_cayley_neumann_grad_many_adamw(sides, Gl, m_b, v_b, layers[0].dtype, ws, dtheta=dth_b, **hp)
+    poet.poet_sync_status()
+    th_b = [t for L in layers for t in (L.theta_R, L.theta_P)]
+    for a, b in zip(dth, dth_b):
+        assert cuda.equal(a, b)
+    for a, b in zip(th_a, th_b):
+        assert cuda.equal(a, b)
+    for a, b in zip(m_a + v_a, m_b + v_b):
+        assert cuda.equal(a, b)
+    # the update against the oracle's AdamW step on the oracle's gradient
+    for (L, xt, dyt, arrs), case, i in zip(built, cases, range(len(cases))):
+        ref = run_oracle(case, *arrs)
+        for s, key in ((0, "dthetaR"), (1, "dthetaP")):
+            k = 2 * i + s
+            if not th0[k].numel():
+                continue
+            t_ref, m_ref, _ = O.adamw_step(th0[k].double().cpu().numpy(), ref[key], m0[k].double().cpu().numpy(),
+                                           v0[k].double().cpu().numpy(), **hp)
+            d_got = (th_b[k].double() - th0[k].double()).cpu().numpy()
+            assert rel_fro(d_got, t_ref - th0[k].double().cpu().numpy()) <= TOL[case.dtype]
+            assert rel_fro(m_b[k].cpu().numpy(), m_ref) <= TOL[case.dtype]
+
+
+def test_merge_reset_moments(cuda):
+    """poet_merge_reset_moments: the merge of poet_merge (bitwise, on an
+    identical layer), theta reset, and the moments of both sides zero."""
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    case = MANY_SETS["bf16"][2]
+    L1, _, _, _ = _make_layer(cuda, case)
+    L2, _, _, _ = _make_layer(cuda, case)
+    for L in (L1, L2):
+        L.cayley_neumann()
+    mR, vR = cuda.ones_like(L1.theta_R), cuda.ones_like(L1.theta_R)
+    mP, vP = cuda.ones_like(L1.theta_P), cuda.ones_like(L1.theta_P)
+    L1.merge()
+    poet.poet_merge_reset_moments(L2.struct, mR, vR, mP, vP, L2.workspace(0))
+    poet.poet_sync_status()
+    assert cuda.equal(L1.W0, L2.W0)
+    assert not L2.theta_R.any().item() and not L2.theta_P.any().item()
+    for t in (mR, vR, mP, vP):
+        assert not t.any().item()

@@ -77,3 +77,80 @@ def test_weight_plan_matches_dense_chain_rule(m, n, modeR, bR, modeP, bP, k, T):
     assert GP.shape == GP_ref.shape and close(GP, GP_ref)
     # E is the dense R W0 P: the merge of the same step
     assert close(E, O.merge(W0, R, P))
+
+
+@pytest.mark.parametrize("m,n,modeR,bR,modeP,bP,k,T", CASES + [(200, 341, BS, 64, FS, 0, 4, 11),
+                                                               (512, 384, FS, 0, BS, 128, 2, 7)])
+@pytest.mark.parametrize("f_tail", [False, True])
+def test_weight_plan_partial_buffers(m, n, modeR, bR, modeP, bP, k, T, f_tail):
+    """The weight plan as the grouped kernels evaluate it: H only on the rows
+    the R primitives cover (c_R), F and E_f only on the columns the P
+    primitives cover (c_P); E is unframed from E_f / H on rows < c_R and from
+    F / W0f on the others, split at column c_P; the per-primitive gradients
+    split their K range at c_P (G_R) and c_R (G_P), reading the leftover
+    range from W0f.  f_tail: F's leftover columns copied from W0f instead of
+    the K split (the kernels do this when c_P is not a 16-byte column
+    offset).  Regions no kernel writes hold NaN, so a read of one shows."""
+    rng = np.random.default_rng(m * 7 + n)
+    W0 = rng.standard_normal((m, n))
+    X = rng.standard_normal((T, n))
+    dY = rng.standard_normal((T, m))
+    permR = O.draw_perm(3, m + n, 0, 1, m)
+    permP = O.draw_perm(3, m + n, 1, 1, n)
+    nR, sR = O.side_shape(m, modeR, bR)
+    nP, sP = O.side_shape(n, modeP, bP)
+    Rb = O.cayley_neumann(0.05 * rng.standard_normal(nR * O.n_skew(sR)), nR, sR, k)
+    Pb = O.cayley_neumann(0.05 * rng.standard_normal(nP * O.n_skew(sP)), nP, sP, k)
+    R = O.dense_side(permR, Rb, modeR, bR)
+    P = O.dense_side(permP, Pb, modeP, bP)
+    Y_ref = O.forward(W0, R, P, X)
+    dX_ref, GR_ref, GP_ref = O.backward(W0, R, P, X, dY, permR, modeR, bR, permP, modeP, bP)
+
+    cR, cP = nR * sR, nP * sP
+    W0f = W0[np.ix_(permR, permP)]
+    nan = np.full((m, n), np.nan)
+    H, F, Ef = nan.copy(), nan.copy(), nan.copy()
+    for j in range(nR):  # H = R^ W0f on the covered rows
+        H[j * sR:(j + 1) * sR] = Rb[j] @ W0f[j * sR:(j + 1) * sR]
+    for j in range(nP):  # F = W0f P^ on the covered columns
+        F[:, j * sP:(j + 1) * sP] = W0f[:, j * sP:(j + 1) * sP] @ Pb[j]
+    if f_tail and nP:
+        F[:, cP:] = W0f[:, cP:]
+    if nR and nP:  # E_f = H P^ on the covered rows and columns
+        for j in range(nP):
+            Ef[:cR, j * sP:(j + 1) * sP] = H[:cR, j * sP:(j + 1) * sP] @ Pb[j]
+    # unframe: rows < c_R from E_f (columns < c_P) and H; the others from F (columns < c_P) and W0f
+    Efull = np.empty((m, n))
+    top = Ef if nP else H
+    Efull[:cR, :cP] = top[:cR, :cP]
+    Efull[:cR, cP:] = H[:cR, cP:]
+    bot = F if nP else W0f
+    Efull[cR:, :cP] = bot[cR:, :cP]
+    Efull[cR:, cP:] = W0f[cR:, cP:]
+    E = np.empty((m, n))
+    E[np.ix_(permR, permP)] = Efull
+    Y = X @ E.T
+    dX = dY @ E
+    D_f = (dY.T @ X)[np.ix_(permR, permP)]
+    GR = np.zeros((nR, sR, sR))
+    for j in range(nR):
+        rows = slice(j * sR, (j + 1) * sR)
+        if nP and cP < n and not f_tail:  # K split at c_P: F, then W0f
+            GR[j] = D_f[rows, :cP] @ F[rows, :cP].T + D_f[rows, cP:] @ W0f[rows, cP:].T
+        else:
+            GR[j] = D_f[rows] @ (F if nP else W0f)[rows].T
+    GP = np.zeros((nP, sP, sP))
+    for j in range(nP):
+        cols = slice(j * sP, (j + 1) * sP)
+        if nR:  # K split at c_R: H, then W0f
+            GP[j] = H[:cR, cols].T @ D_f[:cR, cols] + W0f[cR:, cols].T @ D_f[cR:, cols]
+        else:
+            GP[j] = W0f[:, cols].T @ D_f[:, cols]
+
+    def close(a, b):
+        return np.isfinite(a).all() and np.linalg.norm(a - b) <= 1e-12 * max(1.0, np.linalg.norm(b))
+
+    assert close(Y, Y_ref)
+    assert close(dX, dX_ref)
+    assert GR.shape == GR_ref.shape and close(GR, GR_ref)
+    assert GP.shape == GP_ref.shape and close(GP, GP_ref)
