@@ -689,10 +689,16 @@ def run_poet(args):
             if not args.no_cpu_baseline:
                 wl = I.WORKLOADS[name]
                 full = wl.tokens * wl.layers <= 4096  # the small sets: every token of the layer set
-                one = cpu_baseline([wl], budget_s=6.0, threads=1, full=full)
+                widest = max(max(m, n) for m, n in wl.linear_shapes())
+                # one thread only where the widest primitive is <= 1024 (a 3456-wide Cayley-Neumann
+                # gradient alone takes about a minute on one core)
+                one_ok = wl.mode == I.BS or widest // 2 <= 1024
+                one = cpu_baseline([wl], budget_s=6.0, threads=1, full=full) if one_ok else None
                 allc = cpu_baseline([wl], budget_s=6.0, full=full)
-                others[name].update({"cpu_1t_tok_s": one["value"], "cpu_all_tok_s": allc["value"],
-                                     "cpu_cores": allc["cores"], "cpu_full": full})
+                others[name].update({"cpu_1t_tok_s": one["value"] if one else None,
+                                     "cpu_all_tok_s": allc["value"], "cpu_cores": allc["cores"], "cpu_full": full})
+                if not one:
+                    others[name]["cpu_1t_note"] = "not timed: primitives wider than 1024 (minutes on one core)"
         for name, (base, ov) in SMALLB_PROBES.items():
             others[name] = measure_workload(base, args, device, rank, PLANS["token"], ov)
         out["workloads"] = others

@@ -919,7 +919,9 @@ struct ManyLayout {
   size_t bytes = 0;
 };
 
-static ManyLayout many_layout(const std::vector<LayerGeom> &geoms, int64_t T, const int64_t *lddy) {
+// dy_copies: reserve re-strided dy copies (the backward); the forward never reads dy.
+static ManyLayout many_layout(const std::vector<LayerGeom> &geoms, int64_t T, const int64_t *lddy,
+                              bool dy_copies = true) {
   ManyLayout M;
   const size_t n = geoms.size();
   M.plan.resize(n);
@@ -940,7 +942,7 @@ static ManyLayout many_layout(const std::vector<LayerGeom> &geoms, int64_t T, co
     const int64_t ld = lddy ? lddy[i] : lg.m;
     M.region[i] = off;
     off += M.D_bytes(lg) + M.Df_bytes(lg);
-    if ((ld * int64_t(esize(lg.dtype))) % 16 != 0) {
+    if (dy_copies && (ld * int64_t(esize(lg.dtype))) % 16 != 0) {
       M.dy_copy[i] = 1;
       off += align256(size_t(T) * lg.ldm * esize(lg.dtype));
     }
@@ -1001,7 +1003,7 @@ poet_status poet_forward_many(const poet_layer *layers, int32_t count, const voi
     POET_TRY(check_rows("poet_forward_many", "y", i, y[i], ldy ? ldy[i] : lg.m, lg.m, lg.dtype));
     POET_REQUIRE(saved[i] && aligned256(saved[i]), "poet_forward_many: saved[%d] NULL or not 256-byte aligned", i);
   }
-  const ManyLayout M = many_layout(geoms, T, nullptr);
+  const ManyLayout M = many_layout(geoms, T, nullptr, false);
   if (!ws || ws_bytes < M.bytes || !aligned256(ws)) {
     set_error("poet_forward_many: workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, M.bytes);
     return POET_ENOMEM_WS;

@@ -35,14 +35,18 @@ template <typename T> __device__ __forceinline__ void stf(T *p, float v);
 template <> __device__ __forceinline__ void stf<float>(float *p, float v) { *p = v; }
 template <> __device__ __forceinline__ void stf<bf16>(bf16 *p, float v) { *p = __float2bfloat16_rn(v); }
 
-// Stage block j as float in shared memory, Ms[a][c] = M_j(a, c) (row stride SB).
+// Stage block j as float in shared memory, Ms[a][c] = M_j(a, c) (row stride SB);
+// every entry outside the s x s block is zero, since the products read whole
+// rows of SB entries (0 * an unset entry could be NaN).
 template <typename T>
 __device__ __forceinline__ void stage_block(const T *M, int64_t ldm, int64_t bstride, int j, int s, bool trans,
                                             float *Ms) {
   const T *Mj = M + int64_t(j) * bstride;
-  for (int e = threadIdx.x; e < s * s; e += blockDim.x) {
-    const int a = e / s, c = e % s;
-    Ms[a * SB + c] = trans ? ldf(Mj + int64_t(c) * ldm + a) : ldf(Mj + int64_t(a) * ldm + c);
+  for (int e = threadIdx.x; e < SB * SB; e += blockDim.x) {
+    const int a = e / SB, c = e % SB;
+    float v = 0.f;
+    if (a < s && c < s) v = trans ? ldf(Mj + int64_t(c) * ldm + a) : ldf(Mj + int64_t(a) * ldm + c);
+    Ms[e] = v;
   }
 }
 
