@@ -448,6 +448,88 @@ def measure_workload(name, args, device, rank, plan, overrides=None):
     return out
 
 
+# One LLaMA block around seven POET linears (forward, backward and the grouped
+# a8 of its fourteen sides) at LLaMA-1.3B shapes: hidden 2048, FFN 5461, 32
+# heads of 64, 16 sequences of 2048 tokens.
+BLOCK_WORKLOADS = {"llama1.3b_block_fs": ("llama1.3b_fs", 32, 64, 2048),
+                   "llama1.3b_block_bs256": ("llama1.3b_bs256", 32, 64, 2048)}
+
+
+def measure_block(name, args, device):
+    import torch
+
+    from orthogonal_reparameterized_poet_b200 import inputs as I
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    base, heads, head_dim, seq = BLOCK_WORKLOADS[name]
+    wl = I.WORKLOADS[base]
+    T = wl.tokens
+    layers = []
+    for t, (m, n) in enumerate(wl.linear_shapes()):
+        nR, sR = poet.side_geometry(m, wl.mode, wl.b)
+        nP, sP = poet.side_geometry(n, wl.mode, wl.b)
+        W0 = torch.from_numpy(I.w0(wl.seed, 0, t, m, n, wl.dtype)).to(device=device, dtype=torch.bfloat16)
+        thR = torch.from_numpy(I.theta(wl.seed, 0, t, 0, nR * sR * (sR - 1) // 2, wl.sigma)).to(device)
+        thP = torch.from_numpy(I.theta(wl.seed, 0, t, 1, nP * sP * (sP - 1) // 2, wl.sigma)).to(device)
+        L = poet.PoetLayer(W0, thR, thP, mode=wl.mode, b=wl.b, k=wl.k, seed=wl.seed, layer_id=t)
+        L.prepare()
+        layers.append(L)
+    blk = poet.PoetBlock(layers, seq, heads, head_dim)
+    h = torch.from_numpy(I.activations(wl.seed, wl.hidden, T, wl.hidden, wl.dtype)).to(device, torch.bfloat16)
+    dout = torch.from_numpy(I.activations(wl.seed, wl.hidden, T, wl.hidden, wl.dtype, grad=True)).to(device,
+                                                                                                     torch.bfloat16)
+    out = torch.empty_like(h)
+    dh = torch.empty_like(h)
+    saved = torch.empty(blk.saved_bytes(T), dtype=torch.uint8, device=device)
+    G = [L.block_grad_buffers() for L in layers]
+    dth = [(torch.empty_like(L.theta_R), torch.empty_like(L.theta_P)) for L in layers]
+    gws = torch.empty(max(poet.cayley_neumann_grad_many_workspace_bytes(layers), 1), dtype=torch.uint8,
+                      device=device)
+    blk.workspace(T)
+
+    def step():
+        poet.cayley_neumann_many(layers)
+        blk.forward(h, out=out, saved=saved)
+        blk.backward(saved, dout, dh=dh, G=G)
+        poet.cayley_neumann_grad_many(layers, G, dth, gws)
+
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 1)):
+        step()
+    poet.poet_sync_status()
+    poet.poet_trace_enable(True)
+    for _ in range(args.steps):
+        step()
+    rows = poet.poet_trace_read()
+    poet.poet_trace_enable(False)
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    gph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gph, stream=cap):
+        step()
+    stream.wait_stream(cap)
+    gph.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        gph.replay()
+    b.record(stream)
+    b.synchronize()
+    poet.poet_sync_status()
+    ms = a.elapsed_time(b) / args.steps
+    roof = roofline_of({k: dict(r) for k, r in rows.items()}, poet.poet_version())
+    res = {"tok_s": round(T / (ms / 1e3), 1), "ms": round(ms, 3), "tokens": T, "seq_len": seq, "heads": heads,
+           "head_dim": head_dim, "mode": "FS" if wl.mode == I.FS else f"BS{wl.b}", "plan": "auto",
+           "kernel": roof["kernel"] if roof else None, "frac": roof["frac"] if roof else None,
+           "per_kind_ms": {k: round(r["ms"] / args.steps, 3) for k, r in
+                           sorted(rows.items(), key=lambda kv: -kv[1]["ms"])[:8]}}
+    del gph, blk, layers, saved, G, dth, gws
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_poet(args):
     import torch
 
@@ -701,6 +783,8 @@ def run_poet(args):
                     others[name]["cpu_1t_note"] = "not timed: primitives wider than 1024 (minutes on one core)"
         for name, (base, ov) in SMALLB_PROBES.items():
             others[name] = measure_workload(base, args, device, rank, PLANS["token"], ov)
+        for name in BLOCK_WORKLOADS:
+            others[name] = measure_block(name, args, device)
         out["workloads"] = others
     print(json.dumps(out), flush=True)
     if dist is not None:
@@ -941,6 +1025,8 @@ def run_probe(args):
     if args.probe in SMALLB_PROBES:
         base, ov = SMALLB_PROBES[args.probe]
         res = measure_workload(base, args, torch.device("cuda", 0), 0, PLANS["token"], ov)
+    elif args.probe in BLOCK_WORKLOADS:
+        res = measure_block(args.probe, args, torch.device("cuda", 0))
     else:
         res = measure_workload(args.probe, args, torch.device("cuda", 0), 0, PLANS[args.plan])
     print(json.dumps({"probe": args.probe, **res}), flush=True)

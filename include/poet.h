@@ -373,6 +373,51 @@ POET_API poet_status poet_merge_reset_moments(poet_layer *L, float *m_R, float *
  * same value as poet_workspace_bytes. */
 POET_API size_t poet_workspace_size(const poet_layer *L, int64_t T);
 
+/* ---------------------------------------------------------------- one LLaMA block (adjacent)
+ *
+ * The pages train LLaMA models whose linears are POET layers ([P1]
+ * Experimental setup); these calls run one such block on synthetic tokens,
+ * forward and backward, with the published LLaMA design around the seven
+ * linears: pre-normalization by RMSNorm (gains 1, not trained; eps inside the
+ * square root), rotary position embedding on interleaved pairs (2i, 2i+1) of
+ * each head (angle pos * rope_base^(-2i/head_dim), positions counted within
+ * each sequence of seq_len tokens), causal multi-head attention with scores
+ * scaled by 1/sqrt(head_dim), SwiGLU (down(silu(gate(x)) * up(x))) and
+ * residual connections.  The readings are the library's; the pages restate
+ * none of the block.  Attention materializes the scores (float) and the
+ * probabilities (bf16, kept for the backward) of every head: T/seq_len x heads
+ * x seq_len^2 each.  bf16 only. */
+typedef struct {
+  int32_t seq_len;    /* tokens per sequence (a multiple of 8); T must be a multiple of it */
+  int32_t heads;      /* attention heads */
+  int32_t head_dim;   /* width of one head (a multiple of 8); heads * head_dim = hidden */
+  float rope_base;    /* rotary base (LLaMA: 10000) */
+  float norm_eps;     /* RMSNorm epsilon (LLaMA: 1e-6) */
+  poet_layer lin[7];  /* q, k, v, o (hidden x hidden), gate, up (ffn x hidden), down (hidden x ffn),
+                         each prepared (poet_prepare) with its sides materialized */
+} poet_llama_block;
+
+/* Bytes of the buffer the block's forward saves for its backward at T tokens (0 if invalid). */
+POET_API size_t poet_llama_block_saved_bytes(const poet_llama_block *blk, int64_t T);
+
+/* Bytes of workspace the block's forward and backward need at T tokens (0 if invalid). */
+POET_API size_t poet_llama_block_workspace_bytes(const poet_llama_block *blk, int64_t T);
+
+/* out = the block applied to h (device T x hidden bf16, contiguous rows, 16-byte
+ * aligned); saved: device, poet_llama_block_saved_bytes, 256-byte aligned;
+ * ws: device, poet_llama_block_workspace_bytes, 256-byte aligned. */
+POET_API poet_status poet_llama_block_forward(const poet_llama_block *blk, const void *h, int64_t T, void *out,
+                                              void *saved, void *ws, size_t ws_bytes, poet_stream stream);
+
+/* For upstream gradient dout (device T x hidden bf16): dh (device T x hidden
+ * bf16) and every linear's per-primitive gradients G[2i] = G_R, G[2i+1] = G_P
+ * of lin[i] (device, poet_block_grad_bytes each, 16-byte aligned, overwritten);
+ * the skew-parameter gradients follow with poet_cayley_neumann_grad_many on
+ * the fourteen sides.  saved: the buffer the forward filled for the same h. */
+POET_API poet_status poet_llama_block_backward(const poet_llama_block *blk, const void *saved, const void *dout,
+                                               int64_t T, void *dh, float *const *G, void *ws, size_t ws_bytes,
+                                               poet_stream stream);
+
 /* ---------------------------------------------------------------- utilities */
 
 /* Batched dense product on the library's GEMM engine, exported so that the

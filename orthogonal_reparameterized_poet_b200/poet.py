@@ -39,6 +39,11 @@ class poet_layer(ctypes.Structure):
                 ("R", poet_side), ("P", poet_side)]
 
 
+class poet_llama_block(ctypes.Structure):
+    _fields_ = [("seq_len", ctypes.c_int32), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float), ("lin", poet_layer * 7)]
+
+
 class poet_adamw_hparams(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
                 ("weight_decay", ctypes.c_float), ("step", ctypes.c_int32)]
@@ -108,6 +113,14 @@ _SIGS = {
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                                 ctypes.c_void_p]),
     "poet_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(poet_layer), ctypes.c_int64]),
+    "poet_llama_block_saved_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_llama_block), ctypes.c_int64]),
+    "poet_llama_block_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(poet_llama_block), ctypes.c_int64]),
+    "poet_llama_block_forward": (ctypes.c_int, [ctypes.POINTER(poet_llama_block), ctypes.c_void_p, ctypes.c_int64,
+                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                                ctypes.c_void_p]),
+    "poet_llama_block_backward": (ctypes.c_int, [ctypes.POINTER(poet_llama_block), ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_size_t, ctypes.c_void_p]),
     "poet_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_void_p]),
     "poet_adamw_step": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_int64, ctypes.c_float, ctypes.c_float, ctypes.c_float,
@@ -542,3 +555,75 @@ def poet_merge_reset_moments(layer: poet_layer, m_R, v_R, m_P, v_P, ws, stream=N
 
 def poet_workspace_size(layer: poet_layer, T: int) -> int:
     return lib().poet_workspace_size(ctypes.byref(layer), T)
+
+
+# ------------------------------------------------------------------ one LLaMA block around seven POET linears
+
+class PoetBlock:
+    """One LLaMA block whose linears q, k, v, o, gate, up, down are PoetLayers
+    (bf16).  forward() saves what backward() needs; backward() returns dh and
+    the packed-skew gradients of the fourteen sides (a8 grouped)."""
+
+    NAMES = ("q", "k", "v", "o", "gate", "up", "down")
+
+    def __init__(self, layers, seq_len, heads, head_dim, rope_base=10000.0, norm_eps=1e-6):
+        if len(layers) != 7:
+            raise ValueError("a block takes seven PoetLayers: q, k, v, o, gate, up, down")
+        self.layers = list(layers)
+        self.hidden = layers[0].m
+        b = poet_llama_block()
+        b.seq_len, b.heads, b.head_dim, b.rope_base, b.norm_eps = seq_len, heads, head_dim, rope_base, norm_eps
+        self._b = b
+        self._sync()
+        self._ws = {}
+
+    def _sync(self):
+        for i, L in enumerate(self.layers):
+            self._b.lin[i] = L.struct
+
+    @property
+    def struct(self):
+        self._sync()
+        return self._b
+
+    def saved_bytes(self, T):
+        return lib().poet_llama_block_saved_bytes(ctypes.byref(self.struct), T)
+
+    def workspace(self, T):
+        if T not in self._ws:
+            n = lib().poet_llama_block_workspace_bytes(ctypes.byref(self.struct), T)
+            self._ws[T] = torch.empty(max(n, 1), dtype=torch.uint8, device=self.layers[0].W0.device)
+        return self._ws[T]
+
+    def forward(self, h, out=None, saved=None, stream=None):
+        T = h.shape[0]
+        if out is None:
+            out = torch.empty_like(h)
+        if saved is None:
+            saved = torch.empty(max(self.saved_bytes(T), 1), dtype=torch.uint8, device=h.device)
+        ws = self.workspace(T)
+        _check(lib().poet_llama_block_forward(ctypes.byref(self.struct), _ptr(h), T, _ptr(out), _ptr(saved), _ptr(ws),
+                                              ws.numel(), _stream(stream)))
+        return out, saved
+
+    def backward(self, saved, dout, dh=None, G=None, stream=None):
+        """dh and G = [(G_R, G_P), ...] per linear (per-primitive gradients)."""
+        T = dout.shape[0]
+        if dh is None:
+            dh = torch.empty_like(dout)
+        if G is None:
+            G = [L.block_grad_buffers() for L in self.layers]
+        ws = self.workspace(T)
+        gp = _ptrs([g for pair in G for g in pair])
+        _check(lib().poet_llama_block_backward(ctypes.byref(self.struct), _ptr(saved), _ptr(dout), T, _ptr(dh), gp,
+                                               _ptr(ws), ws.numel(), _stream(stream)))
+        return dh, G
+
+    def theta_grads(self, G, ws=None, stream=None):
+        """a8 of the fourteen sides: [(dtheta_R, dtheta_P), ...]."""
+        dth = [(torch.empty_like(L.theta_R), torch.empty_like(L.theta_P)) for L in self.layers]
+        if ws is None:
+            n = cayley_neumann_grad_many_workspace_bytes(self.layers)
+            ws = torch.empty(max(n, 1), dtype=torch.uint8, device=self.layers[0].W0.device)
+        cayley_neumann_grad_many(self.layers, G, dth, ws, stream)
+        return dth
