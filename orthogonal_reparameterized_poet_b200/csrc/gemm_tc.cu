@@ -55,6 +55,7 @@ struct TcProblem {
   int atomic;
   int coalesced;  // plain bf16 output, 16-byte aligned rows: stores staged through shared memory
   int m_fast;     // tile order: M tiles fastest (N > M: CTAs of a wave share B slabs)
+  int group_m;    // split-K: M tiles per group (a group runs all its splits before the next group)
 };
 
 // A launch: up to MAXP independent problems sharing operand majors and tile
@@ -289,6 +290,29 @@ __device__ __forceinline__ TileCoord decode(int64_t tile, const TcGroup<MAXP> &g
   c.pi = lo;
   const TcProblem &p = g.prob[lo];
   int64_t t = tile - g.tile_start[lo];
+  if (p.splits > 1) {
+    // split-K: groups of group_m M tiles; a group's tiles run split by split,
+    // so its part of the float output is reduced into while it is in L2
+    const int64_t per_b = int64_t(p.num_m) * p.num_n * p.splits;
+    c.b = int(t / per_b);
+    t %= per_b;
+    const int64_t full = int64_t(p.group_m) * p.num_n * p.splits;
+    const int grp = int(t / full);
+    t %= full;
+    const int m0 = grp * p.group_m;
+    const int gm = p.num_m - m0 < p.group_m ? p.num_m - m0 : p.group_m;  // the last group may be smaller
+    const int64_t per_split = int64_t(gm) * p.num_n;
+    c.s = int(t / per_split);
+    t %= per_split;
+    if (p.m_fast) {
+      c.mt = m0 + int(t % gm);
+      c.nt = int(t / gm);
+    } else {
+      c.nt = int(t % p.num_n);
+      c.mt = m0 + int(t / p.num_n);
+    }
+    return c;
+  }
   if (p.m_fast) {
     c.mt = int(t % p.num_m);
     t /= p.num_m;
@@ -961,6 +985,14 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   // consecutive tiles (one wave of persistent CTAs) share the slabs of the
   // larger operand, which is then read from HBM about once
   p->m_fast = g.N > g.M ? 1 : 0;
+  // split-K groups: about one wave of tile workers (CTAs or CTA pairs) per group
+  {
+    const int workers = num_sms() / t.cg;
+    int gm = workers / (p->num_n > 0 ? p->num_n : 1);
+    if (gm < 1) gm = 1;
+    if (gm > p->num_m) gm = p->num_m;
+    p->group_m = gm;
+  }
   // staged epilogue for a single plain output (1: bf16, 16-byte aligned rows;
   // 3: bf16, any rows; 2: fp32, 16-byte aligned rows, stored or reduced); the
   // per-row path handles addends, pairs of outputs and unaligned fp32 rows
