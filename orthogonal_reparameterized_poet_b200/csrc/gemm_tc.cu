@@ -808,17 +808,39 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(r[j]);
         if (p.add) {
+          // the addend's 32 values of this row: 16-byte vector loads when the chunk is whole and aligned
           const int64_t off = int64_t(c.b) * p.add_b + int64_t(gm) * p.add_m + gn0;
           if (p.add_f32) {
             const float *a = static_cast<const float *>(p.add) + off;
+            if (nvalid == 32 && (reinterpret_cast<uintptr_t>(a) & 15) == 0) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nvalid) v[j] += beta * a[j];
+              for (int j = 0; j < 32; j += 4) {
+                const float4 q = *reinterpret_cast<const float4 *>(a + j);
+                v[j] += beta * q.x; v[j + 1] += beta * q.y; v[j + 2] += beta * q.z; v[j + 3] += beta * q.w;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nvalid) v[j] += beta * a[j];
+            }
           } else {
             const uint16_t *a = static_cast<const uint16_t *>(p.add) + off;
+            if (nvalid == 32 && (reinterpret_cast<uintptr_t>(a) & 15) == 0) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nvalid) v[j] += beta * bf16_bits_to_float(a[j]);
+              for (int j = 0; j < 32; j += 8) {
+                const uint4 q = *reinterpret_cast<const uint4 *>(a + j);
+                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  v[j + 2 * e] += beta * bf16_bits_to_float(uint16_t(w[e] & 0xFFFFu));
+                  v[j + 2 * e + 1] += beta * bf16_bits_to_float(uint16_t(w[e] >> 16));
+                }
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nvalid) v[j] += beta * bf16_bits_to_float(a[j]);
+            }
           }
         }
         if (diag != 0.f && gm >= gn0 && gm < gn0 + 32) {

@@ -21,6 +21,7 @@
 // flight.  Rows whose start is not 16-byte aligned (natural rows of odd
 // length) use 16-byte copies for the aligned body and scalar copies for the
 // edges; shared and global addresses stay congruent modulo 16.
+#include <algorithm>
 #include <type_traits>
 #include <vector>
 
@@ -337,6 +338,10 @@ struct FrameGroup {
 static_assert(sizeof(FrameGroup) <= 32000, "frame table exceeds the kernel parameter limit");
 
 __global__ void __launch_bounds__(256) frame_f32_to_bf16_kernel(const __grid_constant__ FrameGroup g) {
+  // a row of D is staged in shared memory with 16-byte copies (coalesced), then
+  // gathered from there; rows whose start is not 16-byte aligned are gathered
+  // from global memory directly
+  extern __shared__ __align__(16) float srow[];
   bool bad = false;
   const int64_t total = g.row_start[g.count];
   int p = 0;
@@ -349,19 +354,29 @@ __global__ void __launch_bounds__(256) frame_f32_to_bf16_kernel(const __grid_con
     const bool row_ok = sr >= 0 && sr < rows;
     bad |= !row_ok;
     const float *src = g.D[p] + (row_ok ? sr : 0) * g.ldD[p];
+    const bool staged = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+    if (staged) {
+      __syncthreads();  // the previous row's readers of srow are done
+      const int units = d / 4;
+      for (int u = threadIdx.x; u < units; u += blockDim.x) cp_async16(srow + 4 * u, src + 4 * u);
+      for (int c = 4 * units + threadIdx.x; c < d; c += blockDim.x) srow[c] = src[c];
+      cp_async_wait_all();
+      __syncthreads();
+    }
     bf16 *orow = g.out[p] + a * g.ld_out[p];
     for (int c = 2 * threadIdx.x; c < d; c += 2 * blockDim.x) {
       if (c + 1 < d) {
         const int2 pc = *reinterpret_cast<const int2 *>(perm + c);
         const bool okx = row_ok && unsigned(pc.x) < unsigned(d), oky = row_ok && unsigned(pc.y) < unsigned(d);
         bad |= !(okx && oky);
-        *reinterpret_cast<__nv_bfloat162 *>(orow + c) =
-            __floats2bfloat162_rn(okx ? __ldg(src + pc.x) : 0.f, oky ? __ldg(src + pc.y) : 0.f);
+        const float vx = okx ? (staged ? srow[pc.x] : __ldg(src + pc.x)) : 0.f;
+        const float vy = oky ? (staged ? srow[pc.y] : __ldg(src + pc.y)) : 0.f;
+        *reinterpret_cast<__nv_bfloat162 *>(orow + c) = __floats2bfloat162_rn(vx, vy);
       } else {
         const int pc = perm[c];
         const bool ok = row_ok && unsigned(pc) < unsigned(d);
         bad |= !ok;
-        orow[c] = __float2bfloat16_rn(ok ? __ldg(src + pc) : 0.f);
+        orow[c] = __float2bfloat16_rn(ok ? (staged ? srow[pc] : __ldg(src + pc)) : 0.f);
       }
     }
   }
@@ -449,15 +464,33 @@ poet_status launch_permute(const PermArgs<T> &a, cudaStream_t st, const char *ki
 constexpr int kPermMax = 64;
 static_assert(sizeof(PermGroup<float, kPermMax>) <= 32000, "permute table exceeds the kernel parameter limit");
 
+// Problems are launched in buckets of similar row width (the ring slot of a
+// launch fits its widest row, so a narrow row sharing a launch with a wide one
+// would get fewer CTAs per SM than on its own), up to kPermMax per launch.
 template <typename T>
 poet_status launch_permute_many(const std::vector<PermArgs<T>> &v, cudaStream_t st, const char *kind) {
   static thread_local PermGroup<T, kPermMax> grp;  // large: keep it off the stack
-  for (size_t i0 = 0; i0 < v.size(); i0 += kPermMax) {
+  auto width_class = [](int d) {  // row bytes rounded up to a power of two
+    int c = 0;
+    while ((int64_t(1) << c) < int64_t(d) * int64_t(sizeof(T))) ++c;
+    return c;
+  };
+  std::vector<int> classes;
+  for (const PermArgs<T> &a : v)
+    if (a.rows > 0 && a.d > 0) classes.push_back(width_class(a.d));
+  std::sort(classes.begin(), classes.end());
+  classes.erase(std::unique(classes.begin(), classes.end()), classes.end());
+  for (int cls : classes) {
     grp.count = 0;
-    for (size_t i = i0; i < v.size() && i < i0 + kPermMax; ++i)
-      if (v[i].rows > 0 && v[i].d > 0) grp.prob[grp.count++] = v[i];
-    if (grp.count == 0) continue;
-    POET_TRY(launch_permute_group(grp, st, kind));
+    for (const PermArgs<T> &a : v) {
+      if (a.rows <= 0 || a.d <= 0 || width_class(a.d) != cls) continue;
+      grp.prob[grp.count++] = a;
+      if (grp.count == kPermMax) {
+        POET_TRY(launch_permute_group(grp, st, kind));
+        grp.count = 0;
+      }
+    }
+    if (grp.count > 0) POET_TRY(launch_permute_group(grp, st, kind));
   }
   return POET_OK;
 }
@@ -505,11 +538,26 @@ poet_status frame_many(const std::vector<FrameItem> &v, cudaStream_t st) {
     }
     if (grp.count == 0) continue;
     grp.errword = device_errword();
+    int dmax = 0;
+    for (int q = 0; q < grp.count; ++q) dmax = grp.d[q] > dmax ? grp.d[q] : dmax;
+    const size_t smem = size_t(dmax) * 4;  // one staged row of the widest matrix
+    POET_REQUIRE(smem <= 200 * 1024, "frame: rows of %d floats do not fit in shared memory", dmax);
+    static int configured[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (smem > 48 * 1024 && dev < 64 && configured[dev] < int(smem)) {
+      POET_CUDA_TRY(cudaFuncSetAttribute(frame_f32_to_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(smem)));
+      configured[dev] = int(smem);
+    }
+    int per_sm = 0;
+    POET_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, frame_f32_to_bf16_kernel, 256, smem));
+    if (per_sm < 1) per_sm = 1;
     const int64_t total = grp.row_start[grp.count];
-    const int64_t cap = int64_t(num_sms()) * 8;
+    const int64_t cap = int64_t(num_sms()) * per_sm;
     const int grid = int(total < cap ? total : cap);
     TraceScope ts("frame", 0.0, bytes, st);
-    frame_f32_to_bf16_kernel<<<grid, 256, 0, st>>>(grp);
+    frame_f32_to_bf16_kernel<<<grid, 256, smem, st>>>(grp);
     count_launch();
     POET_TRY(launch_status("frame"));
   }

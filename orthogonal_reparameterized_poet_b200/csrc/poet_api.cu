@@ -365,7 +365,7 @@ extern "C" {
 const char *poet_last_error(void) { return g_last_error; }
 
 // The kernel revisions name the code that profiles/ counters were taken on.
-const char *poet_version(void) { return "libpoet 0.4 (sm_100a; gemm_tc r10; permute r4; restride r1; cnp r3; smallb r1; block r1)"; }
+const char *poet_version(void) { return "libpoet 0.4 (sm_100a; gemm_tc r11; permute r5; restride r1; cnp r3; smallb r1; block r1)"; }
 
 size_t poet_side_state_bytes(const poet_side *side, int32_t dtype) {
   SideGeom g;
@@ -460,10 +460,10 @@ poet_status poet_cayley_neumann_grad(const poet_side *side, int32_t dtype, const
 //   E_f = H P on the rows [0, c_R) and columns [0, c_P)
 // and E = E_f unframed, reading E_f / H on the rows [0, c_R) and F / W0f on
 // the others, each split at the column c_P.  The backward's per-primitive
-// products split their K range the same way, so the leftover rows and
-// columns are read from W0f in place.  Only when c_P is not a 16-byte
-// column offset (a TMA operand must start on one) are F's leftover columns
-// copied from W0f.
+// products read whole rows of F and whole columns of H, so H's leftover rows
+// and F's leftover columns are copied from W0f once (one grouped launch):
+// reading them from W0f in place would split each product's K range into two
+// problems, doubling its split-K float reductions, which costs more.
 
 namespace {
 
@@ -489,12 +489,6 @@ struct WBwd {          // one layer of a grouped weight-plan backward
   void *Df;            // m x ldn scratch in the storage type (D framed)
 };
 
-// c_P is a column offset a TMA operand can start at
-bool col_split_ok(const LayerGeom &lg) { return (int64_t(lg.P.covered) * int64_t(esize(lg.dtype))) % 16 == 0; }
-bool f_tail_copied(const LayerGeom &lg) {
-  return lg.P.nprim > 0 && lg.P.covered < lg.n && !col_split_ok(lg);
-}
-
 const char *at(const void *base, int64_t elems, int dtype) {
   return static_cast<const char *>(base) + elems * int64_t(esize(dtype));
 }
@@ -511,15 +505,24 @@ poet_status forward_weight_many(std::vector<WFwd> &v, int64_t T, cudaStream_t st
     if (f.lg.P.nprim > 0) gs.push_back(right_blocks(f.L, f.lg, f.L->W0f, f.sv + ly.F, "w_prep"));
   }
   POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
-  // F's leftover columns, where the backward cannot read them from W0f in place
+  // H's leftover rows and F's leftover columns (the identity part of each side), for the backward
   for (WFwd &f : v) {
-    if (!f_tail_copied(f.lg)) continue;
     const WeightSaved ly = weight_saved(f.lg, T);
-    RowPermute r;
-    r.src1 = at(f.L->W0f, f.lg.P.covered, dt); r.ld1 = f.lg.ldn;
-    r.rows = f.lg.m; r.d = int(f.lg.n - f.lg.P.covered);
-    r.dst = const_cast<char *>(at(f.sv + ly.F, f.lg.P.covered, dt)); r.ldd = f.lg.ldn;
-    perms.push_back(r);
+    const int64_t cR = f.lg.R.covered, cP = f.lg.P.covered;
+    if (f.lg.R.nprim > 0 && f.lg.P.nprim > 0 && cR < f.lg.m) {
+      RowPermute r;
+      r.src1 = at(f.L->W0f, cR * f.lg.ldn, dt); r.ld1 = f.lg.ldn;
+      r.rows = f.lg.m - cR; r.d = int(f.lg.n);
+      r.dst = const_cast<char *>(at(f.sv + ly.H, cR * f.lg.ldn, dt)); r.ldd = f.lg.ldn;
+      perms.push_back(r);
+    }
+    if (f.lg.P.nprim > 0 && f.lg.R.nprim > 0 && cP < f.lg.n) {
+      RowPermute r;
+      r.src1 = at(f.L->W0f, cP, dt); r.ld1 = f.lg.ldn;
+      r.rows = f.lg.m; r.d = int(f.lg.n - cP);
+      r.dst = const_cast<char *>(at(f.sv + ly.F, cP, dt)); r.ldd = f.lg.ldn;
+      perms.push_back(r);
+    }
   }
   POET_TRY(permute_many(dt, perms, st, "copy"));
   // E_f = H P on the rows < c_R
@@ -658,7 +661,7 @@ poet_status backward_weight_many(std::vector<WBwd> &v, int64_t T, cudaStream_t s
     POET_TRY(permute_many(POET_F32, fr, st, "frame"));
   }
   // G_R[j] = D_f[rows j] F[rows j]^T,  G_P[j] = H[:, cols j]^T D_f[:, cols j]
-  // (small products: split over K and summed in place; leftover ranges of K read from W0f)
+  // (small products: split over K and summed in place)
   zero.clear();
   gs.clear();
   for (WBwd &b : v) {
@@ -666,50 +669,30 @@ poet_status backward_weight_many(std::vector<WBwd> &v, int64_t T, cudaStream_t s
     const SideGeom &gR = lg.R, &gP = lg.P;
     const WeightSaved ly = weight_saved(lg, T);
     const char *W0f = static_cast<const char *>(b.L->W0f);
-    const int64_t cR = gR.covered, cP = gP.covered;
-    if (gR.nprim > 0) {
+    if (gR.nprim > 0) {  // G_R[j] = D_f[rows j] F[rows j]^T  (F = W0f when P has no primitives)
       zero.emplace_back(b.GR, gR.all_elems());
       Gemm p;
       p.tag = "blk_grad";
-      p.M = gR.size; p.N = gR.size; p.batch = gR.nprim; p.dtype = dt;
-      p.a_m = lg.ldn; p.a_k = 1; p.a_b = int64_t(gR.size) * lg.ldn;
+      p.M = gR.size; p.N = gR.size; p.K = int(lg.n); p.batch = gR.nprim; p.dtype = dt;
+      p.A = b.Df; p.a_m = lg.ldn; p.a_k = 1; p.a_b = int64_t(gR.size) * lg.ldn;
+      p.B = gP.nprim > 0 ? static_cast<const void *>(b.sv + ly.F) : W0f;
       p.b_n = lg.ldn; p.b_k = 1; p.b_b = int64_t(gR.size) * lg.ldn;
       p.outF = b.GR; p.of_m = gR.ld; p.of_b = gR.blk_elems();
       p.atomic = true;
-      if (gP.nprim > 0 && cP < lg.n && col_split_ok(lg)) {
-        Gemm q = p;  // K in [0, c_P): F
-        q.K = int(cP); q.A = b.Df; q.B = b.sv + ly.F;
-        gs.push_back(q);
-        q.K = int(lg.n - cP); q.A = at(b.Df, cP, dt); q.B = at(W0f, cP, dt);  // K in [c_P, n): W0f
-        gs.push_back(q);
-      } else {
-        p.K = int(lg.n); p.A = b.Df;
-        p.B = gP.nprim > 0 ? static_cast<const void *>(b.sv + ly.F) : W0f;  // F with its leftover columns, or W0f
-        gs.push_back(p);
-      }
+      gs.push_back(p);
     }
-    if (gP.nprim > 0) {
+    if (gP.nprim > 0) {  // G_P[j] = H[:, cols j]^T D_f[:, cols j]  (H = W0f when R has no primitives)
       zero.emplace_back(b.GP, gP.all_elems());
       Gemm p;
-      p.small = SMALL_GRAD;  // G_P[j] = sum over rows of H[:, cols j] x D_f[:, cols j]
+      p.small = SMALL_GRAD;  // the sum runs over the rows
       p.tag = "blk_grad";
-      p.M = gP.size; p.N = gP.size; p.batch = gP.nprim; p.dtype = dt;
+      p.M = gP.size; p.N = gP.size; p.K = int(lg.m); p.batch = gP.nprim; p.dtype = dt;
+      p.A = gR.nprim > 0 ? static_cast<const void *>(b.sv + ly.H) : W0f;
       p.a_m = 1; p.a_k = lg.ldn; p.a_b = gP.size;
-      p.b_n = 1; p.b_k = lg.ldn; p.b_b = gP.size;
+      p.B = b.Df; p.b_n = 1; p.b_k = lg.ldn; p.b_b = gP.size;
       p.outF = b.GP; p.of_m = gP.ld; p.of_b = gP.blk_elems();
       p.atomic = true;
-      if (gR.nprim > 0) {
-        Gemm q = p;  // K in [0, c_R): H
-        q.K = int(cR); q.A = b.sv + ly.H; q.B = b.Df;
-        gs.push_back(q);
-        if (cR < lg.m) {  // K in [c_R, m): W0f
-          q.K = int(lg.m - cR); q.A = at(W0f, cR * lg.ldn, dt); q.B = at(b.Df, cR * lg.ldn, dt);
-          gs.push_back(q);
-        }
-      } else {
-        p.K = int(lg.m); p.A = W0f; p.B = b.Df;
-        gs.push_back(p);
-      }
+      gs.push_back(p);
     }
   }
   POET_TRY(zero_many(zero, st));

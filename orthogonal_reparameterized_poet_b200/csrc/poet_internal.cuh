@@ -221,12 +221,16 @@ struct AdamW {
 AdamW adamw_of(float lr, float beta1, float beta2, float eps, float weight_decay, int32_t step);
 
 // One parameter's AdamW update (decoupled weight decay, bias-corrected moments).
+// Every operation is an explicitly rounded single-precision intrinsic, so the
+// compiler contracts none of them into fused multiply-adds and every kernel
+// that calls this function performs exactly the same arithmetic.
 __device__ __forceinline__ void adamw_one(float &theta, float g, float &m, float &v, const AdamW &h) {
-  m = h.beta1 * m + (1.f - h.beta1) * g;
-  v = h.beta2 * v + (1.f - h.beta2) * g * g;
-  const float m_hat = m / h.bc1;
-  const float v_hat = v / h.bc2;
-  theta = theta - h.lr * (m_hat / (sqrtf(v_hat) + h.eps) + h.wd * theta);
+  m = __fadd_rn(__fmul_rn(h.beta1, m), __fmul_rn(__fsub_rn(1.f, h.beta1), g));
+  v = __fadd_rn(__fmul_rn(h.beta2, v), __fmul_rn(__fmul_rn(__fsub_rn(1.f, h.beta2), g), g));
+  const float m_hat = __fdiv_rn(m, h.bc1);
+  const float v_hat = __fdiv_rn(v, h.bc2);
+  const float step = __fadd_rn(__fdiv_rn(m_hat, __fadd_rn(__fsqrt_rn(v_hat), h.eps)), __fmul_rn(h.wd, theta));
+  theta = __fsub_rn(theta, __fmul_rn(h.lr, step));
 }
 
 // One AdamW step on n float parameters in place (see poet_adamw_step).

@@ -81,16 +81,15 @@ def test_weight_plan_matches_dense_chain_rule(m, n, modeR, bR, modeP, bP, k, T):
 
 @pytest.mark.parametrize("m,n,modeR,bR,modeP,bP,k,T", CASES + [(200, 341, BS, 64, FS, 0, 4, 11),
                                                                (512, 384, FS, 0, BS, 128, 2, 7)])
-@pytest.mark.parametrize("f_tail", [False, True])
-def test_weight_plan_partial_buffers(m, n, modeR, bR, modeP, bP, k, T, f_tail):
-    """The weight plan as the grouped kernels evaluate it: H only on the rows
-    the R primitives cover (c_R), F and E_f only on the columns the P
-    primitives cover (c_P); E is unframed from E_f / H on rows < c_R and from
-    F / W0f on the others, split at column c_P; the per-primitive gradients
-    split their K range at c_P (G_R) and c_R (G_P), reading the leftover
-    range from W0f.  f_tail: F's leftover columns copied from W0f instead of
-    the K split (the kernels do this when c_P is not a 16-byte column
-    offset).  Regions no kernel writes hold NaN, so a read of one shows."""
+def test_weight_plan_partial_buffers(m, n, modeR, bR, modeP, bP, k, T):
+    """The weight plan as the grouped kernels evaluate it: H computed on the
+    rows the R primitives cover (c_R), F on the columns the P primitives cover
+    (c_P), E_f = H P on both; when both sides have primitives, H's other rows
+    and F's other columns are copied from W0f; E is unframed from E_f / H on
+    rows < c_R and from F / W0f on the others, split at column c_P; G_R reads
+    whole rows of F (W0f without P primitives), G_P whole columns of H (W0f
+    without R primitives).  Regions no kernel writes hold NaN, so a read of
+    one shows."""
     rng = np.random.default_rng(m * 7 + n)
     W0 = rng.standard_normal((m, n))
     X = rng.standard_normal((T, n))
@@ -114,10 +113,10 @@ def test_weight_plan_partial_buffers(m, n, modeR, bR, modeP, bP, k, T, f_tail):
         H[j * sR:(j + 1) * sR] = Rb[j] @ W0f[j * sR:(j + 1) * sR]
     for j in range(nP):  # F = W0f P^ on the covered columns
         F[:, j * sP:(j + 1) * sP] = W0f[:, j * sP:(j + 1) * sP] @ Pb[j]
-    if f_tail and nP:
+    if nR and nP:  # the leftover rows of H and columns of F, copied from W0f
+        H[cR:] = W0f[cR:]
         F[:, cP:] = W0f[:, cP:]
-    if nR and nP:  # E_f = H P^ on the covered rows and columns
-        for j in range(nP):
+        for j in range(nP):  # E_f = H P^ on the covered rows and columns
             Ef[:cR, j * sP:(j + 1) * sP] = H[:cR, j * sP:(j + 1) * sP] @ Pb[j]
     # unframe: rows < c_R from E_f (columns < c_P) and H; the others from F (columns < c_P) and W0f
     Efull = np.empty((m, n))
@@ -132,20 +131,12 @@ def test_weight_plan_partial_buffers(m, n, modeR, bR, modeP, bP, k, T, f_tail):
     Y = X @ E.T
     dX = dY @ E
     D_f = (dY.T @ X)[np.ix_(permR, permP)]
-    GR = np.zeros((nR, sR, sR))
-    for j in range(nR):
-        rows = slice(j * sR, (j + 1) * sR)
-        if nP and cP < n and not f_tail:  # K split at c_P: F, then W0f
-            GR[j] = D_f[rows, :cP] @ F[rows, :cP].T + D_f[rows, cP:] @ W0f[rows, cP:].T
-        else:
-            GR[j] = D_f[rows] @ (F if nP else W0f)[rows].T
-    GP = np.zeros((nP, sP, sP))
-    for j in range(nP):
-        cols = slice(j * sP, (j + 1) * sP)
-        if nR:  # K split at c_R: H, then W0f
-            GP[j] = H[:cR, cols].T @ D_f[:cR, cols] + W0f[cR:, cols].T @ D_f[cR:, cols]
-        else:
-            GP[j] = W0f[:, cols].T @ D_f[:, cols]
+    Fg = F if nP else W0f
+    Hg = H if nR else W0f
+    GR = np.stack([D_f[j * sR:(j + 1) * sR] @ Fg[j * sR:(j + 1) * sR].T for j in range(nR)]) if nR else \
+        np.zeros((0, sR, sR))
+    GP = np.stack([Hg[:, j * sP:(j + 1) * sP].T @ D_f[:, j * sP:(j + 1) * sP] for j in range(nP)]) if nP else \
+        np.zeros((0, sP, sP))
 
     def close(a, b):
         return np.isfinite(a).all() and np.linalg.norm(a - b) <= 1e-12 * max(1.0, np.linalg.norm(b))
