@@ -431,6 +431,13 @@ __global__ void __launch_bounds__(256) pack_many_kernel(const __grid_constant__ 
   }
 }
 
+// Logical elements (nprim * size^2) of the sides in a table, for the trace's bytes.
+double table_elems(const SideTable &t) {
+  double e = 0.0;
+  for (int q = 0; q < t.count; ++q) e += double(t.nprim[q]) * t.size[q] * t.size[q];
+  return e;
+}
+
 int64_t elem_blocks(const SideGeom &g) { return (g.all_elems() + 256 * kItems - 1) / (256 * kItems); }
 int64_t pair_blocks(const SideGeom &g) {
   const int64_t tiles = (g.size + PACK_T - 1) / PACK_T;
@@ -497,6 +504,7 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
     return elem_blocks(g);
   }, t, [&](const SideTable &tt, int, int) {
     const int blocks = int(tt.block_start[tt.count]);
+    TraceScope ts("cnp_elem", 0.0, table_elems(tt) * (2.0 * esize(dtype) + 2.0), st);
     if (dtype == POET_BF16) unpack_many_kernel<bf16><<<blocks, 256, 0, st>>>(tt);
     else unpack_many_kernel<float><<<blocks, 256, 0, st>>>(tt);
     count_launch();
@@ -566,6 +574,7 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
     return elem_blocks(g);
   }, t, [&](const SideTable &tt, int, int) {
     const int blocks = int(tt.block_start[tt.count]);
+    TraceScope ts("cnp_elem", 0.0, table_elems(tt) * 4.0 * esize(dtype), st);
     if (dtype == POET_BF16) powers_combine_kernel<bf16><<<blocks, 256, 0, st>>>(tt);
     else powers_combine_kernel<float><<<blocks, 256, 0, st>>>(tt);
     count_launch();
@@ -659,6 +668,7 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
       t.nprim[q] = g.nprim; t.size[q] = g.size; t.ld[q] = g.ld;
       return elem_blocks(g);
     }, t, [&](const SideTable &tt, int, int) {
+      TraceScope ts("cnp_elem", 0.0, table_elems(tt) * 6.0, st);
       round_many_kernel<<<int(tt.block_start[tt.count]), 256, 0, st>>>(tt);
       count_launch();
       return launch_status("cnp G to bf16");
@@ -691,6 +701,7 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
       }, t, [&](const SideTable &tt, int, int) {
         const int blocks = int(tt.block_start[tt.count]);
         const float c1 = second ? -1.f : -0.5f, c2 = second ? 1.f : 0.f;
+        TraceScope ts("cnp_elem", 0.0, table_elems(tt) * ((second ? 12.0 : 8.0) + esize(dtype)), st);
         if (dtype == POET_BF16) sym_many_kernel<bf16><<<blocks, 256, 0, st>>>(tt, 1.f, c1, c2);
         else sym_many_kernel<float><<<blocks, 256, 0, st>>>(tt, 1.f, c1, c2);
         count_launch();
@@ -784,6 +795,9 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
     return pair_blocks(g);
   }, t, [&](const SideTable &tt, int, int) {
     const int blocks = int(tt.block_start[tt.count]);
+    double terms = 0.0;
+    for (int q = 0; q < tt.count; ++q) terms += double(tt.nprim[q]) * tt.size[q] * tt.size[q] * (1 + tt.terms[q]);
+    TraceScope ts("cnp_elem", 0.0, terms * 4.0 + table_elems(tt) * (adam ? 14.0 : 2.0), st);
     if (adam) pack_many_kernel<true><<<blocks, 256, 0, st>>>(tt, *adam);
     else pack_many_kernel<false><<<blocks, 256, 0, st>>>(tt, AdamW{});
     count_launch();

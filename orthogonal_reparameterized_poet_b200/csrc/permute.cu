@@ -583,6 +583,9 @@ poet_status zero_many(const std::vector<std::pair<float *, int64_t>> &v, cudaStr
     if (grp.count == 0) continue;
     const int64_t want = (most / 4 + 255) / 256, cap = int64_t(num_sms()) * 4;
     const int grid = int(want < 1 ? 1 : (want < cap ? want : cap));
+    double bytes = 0.0;
+    for (int q = 0; q < grp.count; ++q) bytes += double(grp.n[q]) * 4.0;
+    TraceScope ts("zero", 0.0, bytes, st);
     zero_many_kernel<<<grid, 256, 0, st>>>(grp);
     count_launch();
     POET_TRY(launch_status("zero"));
