@@ -6,16 +6,19 @@
 // Neumann series truncated after Q^k:  B = (I + Q)(I + Q + ... + Q^k).
 //
 // Order 4 (the order the pages' LLaMA runs use) is evaluated by powers of
-// S = Q^2, with T = S^2:
-//   B = Q C + D0,   C = 2I + 2S + T,   D0 = I + 2S + 2T
-// (3 GEMMs).  The state keeps Q, S, C, T and D0.  Its gradient, G = dL/dB:
-// theta enters Q antisymmetrically (Q[a,c] = theta = -Q[c,a]), so only the
-// antisymmetric part of dL/dQ reaches dtheta; S, T and C are symmetric, so
-// only the symmetric parts of dL/dS and dL/dT matter:
-//   QG = Q G,  GC = G C,  dT_s = sym(2G - QG),  W = dT_s S,
-//   dS_s = sym(2G - 2 QG) + W + W^T,  Y = dS_s Q,  D = G C - 2 Y,
-//   dtheta[a,c] = D[a,c] - D[c,a]                       (sym(X) = (X + X^T)/2)
-// (4 GEMMs, in three grouped launches).
+// S = Q^2, with T = S^2:  B = Q C + D0,  C = 2I + 2S + T,  D0 = I + 2S + 2T,
+// as three GEMMs whose epilogues add the rest:
+//   S = Q Q,   C = S S + 2S + 2I,   B = (Q + 2I) C - 2S - 3I
+// (the last equals Q C + D0).  The state keeps Q, Q + 2I, S and C.  Its
+// gradient, G = dL/dB: theta enters Q antisymmetrically (Q[a,c] = theta =
+// -Q[c,a]), so only the antisymmetric part of dL/dQ reaches dtheta; S, T and C
+// are symmetric, so only the symmetric parts of dL/dS and dL/dT matter:
+//   dT_s = sym(2G - QG),  W = dT_s S,  dS_s = sym(2G - 2QG) + W + W^T,
+//   D = G C - 2 dS_s Q,  dtheta[a,c] = D[a,c] - D[c,a]   (sym(X) = (X + X^T)/2)
+// evaluated as four GEMMs (three grouped launches) with the sums in their
+// epilogues:  U = G - Q G and G C;  V = dT_s S + U with dT_s = sym(G + U);
+// D = G C - 2 (V + V^T) Q;  so the element-wise passes between them read one
+// or two matrices each.
 //
 // Every other order, by Horner's rule on the series:
 //   S_1 = I + Q,  S_{l+1} = I + Q S_l (l = 1..k-1),  B = (I + Q) S_k = S_1 S_k
@@ -219,7 +222,6 @@ struct SideTable {
   int64_t block_start[kSidesMax + 1];
   const void *src[kSidesMax];
   const void *src2[kSidesMax];
-  const void *src3[kSidesMax];
   void *dst[kSidesMax];
   void *dst2[kSidesMax];
   void *dst3[kSidesMax];
@@ -242,9 +244,10 @@ __device__ __forceinline__ int side_of_block(const SideTable &t) {
   return lo;
 }
 
-// src = theta, dst = Q, dst2 = S_1 = I + Q (or B = I + Q when k = 0; nullptr:
-// not written), dst3 = B whose padding (rows or columns >= size) is zeroed
-// (nullptr: none).  Padding of Q and S_1 is zero.
+// src = theta, dst = Q, dst2 = Q + coef I (Horner's S_1 = I + Q, or B = I + Q
+// when k = 0, with coef 1; Q + 2I for order 4; nullptr: not written), dst3 = B
+// whose padding (rows or columns >= size) is zeroed (nullptr: none).  Padding
+// of Q and dst2 is zero.
 template <typename T>
 __global__ void __launch_bounds__(256) unpack_many_kernel(const __grid_constant__ SideTable t) {
   const int i = side_of_block(t);
@@ -268,35 +271,8 @@ __global__ void __launch_bounds__(256) unpack_many_kernel(const __grid_constant_
       else eye = 1.f;
     }
     Q[e] = from_f<T>(q);
-    if (IplusQ) IplusQ[e] = from_f<T>(q + eye);
+    if (IplusQ) IplusQ[e] = from_f<T>(q + t.coef[i] * eye);
     if (Bpad && !inside) Bpad[e] = from_f<T>(0.f);
-  }
-}
-
-// Order 4: from S (src) and T = S^2 (src2), C = 2I + 2S + T (dst) and
-// D0 = I + 2S + 2T (dst2); padding zero.
-template <typename T>
-__global__ void __launch_bounds__(256) powers_combine_kernel(const __grid_constant__ SideTable t) {
-  const int i = side_of_block(t);
-  const int size = t.size[i], ld = t.ld[i];
-  const int64_t blk = int64_t(ld) * ld, total = blk * t.nprim[i];
-  const T *S = static_cast<const T *>(t.src[i]);
-  const T *Tp = static_cast<const T *>(t.src2[i]);
-  T *C = static_cast<T *>(t.dst[i]);
-  T *D0 = static_cast<T *>(t.dst2[i]);
-  const int64_t e0 = (int64_t(blockIdx.x) - t.block_start[i]) * (256 * kItems);
-  const int64_t e1 = e0 + 256 * kItems < total ? e0 + 256 * kItems : total;
-  for (int64_t e = e0 + threadIdx.x; e < e1; e += 256) {
-    const int a = int((e % blk) / ld), c = int(e % ld);
-    float cv = 0.f, dv = 0.f;
-    if (a < size && c < size) {
-      const float sv = to_f(S[e]), tv = to_f(Tp[e]);
-      const float eye = a == c ? 1.f : 0.f;
-      cv = 2.f * eye + 2.f * sv + tv;
-      dv = eye + 2.f * sv + 2.f * tv;
-    }
-    C[e] = from_f<T>(cv);
-    D0[e] = from_f<T>(dv);
   }
 }
 
@@ -329,22 +305,20 @@ __device__ __forceinline__ TilePair tile_pair(const SideTable &t, int i) {
   return p;
 }
 
-// Order-4 gradient, symmetric combinations: dst = sum_q c_q (X_q + X_q^T)
-// over X_0 = src, X_1 = src2 and X_2 = src3 (float [nprim][ld][ld]; src3 may
-// be nullptr), in the operand type.  One block per pair of 32 x 32 tiles
+// Order-4 gradient, symmetric combinations: dst = c0 (X_0 + X_0^T) + c1 (X_1 +
+// X_1^T) over X_0 = src and X_1 = src2 (float [nprim][ld][ld]; src2 may be
+// nullptr), in the operand type.  One block per pair of 32 x 32 tiles
 // (ta <= tc) of one primitive; both tiles of every input are read
 // row-contiguously into shared memory and both output tiles are written.
 template <typename T>
-__global__ void __launch_bounds__(256) sym_many_kernel(const __grid_constant__ SideTable t, float c0, float c1,
-                                                        float c2) {
+__global__ void __launch_bounds__(256) sym_many_kernel(const __grid_constant__ SideTable t, float c0, float c1) {
   __shared__ float u1[PACK_T][PACK_T + 1], u2[PACK_T][PACK_T + 1];
   const int i = side_of_block(t);
   const int size = t.size[i], ld = t.ld[i];
   const TilePair tp = tile_pair(t, i);
   const int64_t off = int64_t(tp.j) * ld * ld;
-  const float *X[3] = {static_cast<const float *>(t.src[i]), static_cast<const float *>(t.src2[i]),
-                       static_cast<const float *>(t.src3[i])};
-  const float cf[3] = {c0, c1, c2};
+  const float *X[2] = {static_cast<const float *>(t.src[i]), static_cast<const float *>(t.src2[i])};
+  const float cf[2] = {c0, c1};
   T *out = static_cast<T *>(t.dst[i]) + off;
   const int x = threadIdx.x % PACK_T;
   // u1[y][x] = sum c_q X_q[ta*32+y][tc*32+x],  u2[y][x] = sum c_q X_q[tc*32+y][ta*32+x]
@@ -353,7 +327,7 @@ __global__ void __launch_bounds__(256) sym_many_kernel(const __grid_constant__ S
     const int a2 = tp.tc * PACK_T + y, b2 = tp.ta * PACK_T + x;
     float v1 = 0.f, v2 = 0.f;
 #pragma unroll
-    for (int q = 0; q < 3; ++q) {
+    for (int q = 0; q < 2; ++q) {
       if (!X[q]) continue;
       if (a1 < size && b1 < size) v1 += cf[q] * X[q][off + int64_t(a1) * ld + b1];
       if (a2 < size && b2 < size) v2 += cf[q] * X[q][off + int64_t(a2) * ld + b2];
@@ -452,7 +426,7 @@ poet_status many_launch(const std::vector<int> &idx, Blocks blocks, SideTable &t
     t.count = n;
     t.block_start[0] = 0;
     for (int q = 0; q < n; ++q) {
-      t.src[q] = t.src2[q] = t.src3[q] = nullptr;
+      t.src[q] = t.src2[q] = nullptr;
       t.dst[q] = t.dst2[q] = t.dst3[q] = nullptr;
       t.theta[q] = t.m1[q] = t.m2[q] = nullptr;
       t.terms[q] = 0;
@@ -466,14 +440,12 @@ poet_status many_launch(const std::vector<int> &idx, Blocks blocks, SideTable &t
   return POET_OK;
 }
 
-// Byte offsets of the order-4 terms in a side state: S, C, T, D0 take the
-// slots of S_1..S_4.
+// Byte offsets of the order-4 terms in a side state: Q + 2I, S and C take the
+// slots of S_1..S_3.
 struct PowersLayout {
-  size_t S, C, T, D0;
+  size_t Q2, S, C;
 };
-PowersLayout powers_layout(const StateLayout &L) {
-  return {L.S1, L.S1 + L.term, L.S1 + 2 * L.term, L.S1 + 3 * L.term};
-}
+PowersLayout powers_layout(const StateLayout &L) { return {L.S1, L.S1 + L.term, L.S1 + 2 * L.term}; }
 
 }  // namespace
 
@@ -498,7 +470,8 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
     char *base = static_cast<char *>(sides[i].state);
     t.src[q] = sides[i].theta;
     t.dst[q] = base + L.Q;
-    t.dst2[q] = by_powers(g) ? nullptr : (g.k == 0 ? base + L.R : base + L.S1);
+    t.dst2[q] = g.k == 0 ? base + L.R : base + L.S1;  // B = I + Q, S_1 = I + Q, or Q + 2I (order 4)
+    t.coef[q] = by_powers(g) ? 2.f : 1.f;
     t.dst3[q] = g.k == 0 ? nullptr : base + L.R;
     t.nprim[q] = g.nprim; t.size[q] = g.size; t.ld[q] = g.ld;
     return elem_blocks(g);
@@ -535,8 +508,8 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
     POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
   }
   if (pw.empty()) return POET_OK;
-  // order 4 by powers: S = Q Q, T = S S, then C and D0, then B = Q C + D0
-  auto powers_step = [&](int step) {
+  // order 4 by powers: S = Q Q, C = S S + 2S + 2I, B = (Q + 2I) C - 2S - 3I
+  for (int step = 0; step < 3; ++step) {
     gs.clear();
     for (int i : pw) {
       const SideGeom &g = geoms[i];
@@ -549,38 +522,21 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
         p.outD = base + W.S;
       } else if (step == 1) {
         p = prim_gemm(g, dtype, base + W.S, base + W.S, false, "cnp_fwd");
-        p.outD = base + W.T;
+        p.add = base + W.S; p.add_dtype = dtype; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 2.f;
+        p.diag = 2.f;
+        p.outD = base + W.C;
       } else {
-        p = prim_gemm(g, dtype, base + L.Q, base + W.C, false, "cnp_fwd");
-        p.add = base + W.D0; p.add_dtype = dtype; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 1.f;
+        p = prim_gemm(g, dtype, base + W.Q2, base + W.C, false, "cnp_fwd");
+        p.add = base + W.S; p.add_dtype = dtype; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = -2.f;
+        p.diag = -3.f;
         p.outD = base + L.R;
       }
       p.od_m = g.ld; p.od_b = g.blk_elems();
       gs.push_back(p);
     }
-    return gemm_run_many(gs.data(), int(gs.size()), st);
-  };
-  POET_TRY(powers_step(0));
-  POET_TRY(powers_step(1));
-  POET_TRY(many_launch(pw, [&](int i, int q) {
-    const SideGeom &g = geoms[i];
-    const PowersLayout W = powers_layout(state_layout(g, dtype));
-    char *base = static_cast<char *>(sides[i].state);
-    t.src[q] = base + W.S;
-    t.src2[q] = base + W.T;
-    t.dst[q] = base + W.C;
-    t.dst2[q] = base + W.D0;
-    t.nprim[q] = g.nprim; t.size[q] = g.size; t.ld[q] = g.ld;
-    return elem_blocks(g);
-  }, t, [&](const SideTable &tt, int, int) {
-    const int blocks = int(tt.block_start[tt.count]);
-    TraceScope ts("cnp_elem", 0.0, table_elems(tt) * 4.0 * esize(dtype), st);
-    if (dtype == POET_BF16) powers_combine_kernel<bf16><<<blocks, 256, 0, st>>>(tt);
-    else powers_combine_kernel<float><<<blocks, 256, 0, st>>>(tt);
-    count_launch();
-    return launch_status("cnp combine");
-  }));
-  return powers_step(2);
+    POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
+  }
+  return POET_OK;
 }
 
 // Many sides: the same gradient reorganised for grouped launches.
@@ -590,15 +546,15 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
 //    P_k = G S_k^T, P_l = A_{l+1} S_l^T (l < k) of every side, each into its
 //    own float buffer, and one launch packs D - D^T into dtheta with
 //    D = A_1 + P_1 + ... + P_k.
-//  - order 4 by powers: QG = Q G and GC = G C in one launch, dT_s, W = dT_s S,
-//    dS_s, Y = dS_s Q, then D = GC - 2 Y packed (see the top of this file).
+//  - order 4 by powers: U = G - Q G and G C in one launch, dT_s, V = dT_s S + U,
+//    dS_s, D = G C - 2 dS_s Q, then D packed (see the top of this file).
 // Every product writes one plain output, which the tensor-core engine stores
 // through its staged epilogue.
 size_t cnp_many_scratch_bytes(const SideGeom &g, int dtype) {
   if (g.nprim == 0 || g.size < 2 || g.k == 0) return 0;
   const size_t f = align256(size_t(g.all_elems()) * 4);
   const size_t d = align256(size_t(g.all_elems()) * esize(dtype));
-  // order 4: G operand copy, QG then Y (f32), GC (f32), dT_s then dS_s (operand type), W (f32)
+  // order 4: G operand copy, U then D (f32), G C (f32), dT_s then dS_s (operand type), V (f32)
   if (by_powers(g)) return 2 * d + 3 * f;
   // G operand copy, A_k..A_2 (dtype), A_1 (f32), P_1..P_k (f32)
   return d + size_t(g.k - 1) * d + f + size_t(g.k) * f;
@@ -618,8 +574,8 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
     int64_t pstride;
     // order 4 by powers
     const void *S, *C;
-    float *QGY, *GC, *W;
-    void *dT;
+    float *UD, *GC, *V;  // U, then D; G C; V
+    void *dT;            // dT_s, then dS_s (operand type)
   };
   std::vector<Work> w(count);
   std::vector<int> chain, all, pw, rounded;  // Horner sides with k >= 1; every side; order-4 sides; G to round
@@ -643,10 +599,10 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
       const PowersLayout P = powers_layout(L);
       x.S = base + P.S;
       x.C = base + P.C;
-      x.QGY = reinterpret_cast<float *>(s + db);
+      x.UD = reinterpret_cast<float *>(s + db);
       x.GC = reinterpret_cast<float *>(s + db + fb);
       x.dT = s + db + 2 * fb;
-      x.W = reinterpret_cast<float *>(s + 2 * db + 2 * fb);
+      x.V = reinterpret_cast<float *>(s + 2 * db + 2 * fb);
       continue;
     }
     chain.push_back(i);
@@ -679,48 +635,55 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
   // ---- order 4 by powers
   if (!pw.empty()) {
     gs.clear();
-    for (int i : pw) {  // QG = Q G, GC = G C
+    for (int i : pw) {  // U = G - Q G, GC = G C
       const SideGeom &g = geoms[i];
       Gemm a = prim_gemm(g, dtype, w[i].Q, w[i].Gop, false, "cnp_bwd");
-      fout(a, g, w[i].QGY);
+      a.alpha = -1.f;
+      a.add = G[i]; a.add_dtype = POET_F32; a.add_m = g.ld; a.add_b = g.blk_elems(); a.beta = 1.f;
+      fout(a, g, w[i].UD);
       gs.push_back(a);
       Gemm b = prim_gemm(g, dtype, w[i].Gop, w[i].C, false, "cnp_bwd");
       fout(b, g, w[i].GC);
       gs.push_back(b);
     }
     POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
-    auto sym = [&](bool second) {  // dT_s = sym(2G - QG), then dS_s = sym(2G - 2 QG) + W + W^T
+    // dT_s = sym(G + U) = (G + G^T + U + U^T) / 2, then dS_s = V + V^T
+    auto sym = [&](bool second) {
       return many_launch(pw, [&](int i, int q) {
         const SideGeom &g = geoms[i];
-        t.src[q] = G[i];
-        t.src2[q] = w[i].QGY;
-        t.src3[q] = second ? w[i].W : nullptr;
+        t.src[q] = second ? static_cast<const void *>(w[i].V) : static_cast<const void *>(G[i]);
+        t.src2[q] = second ? nullptr : w[i].UD;
         t.dst[q] = w[i].dT;
         t.nprim[q] = g.nprim; t.size[q] = g.size; t.ld[q] = g.ld;
         return pair_blocks(g);
       }, t, [&](const SideTable &tt, int, int) {
         const int blocks = int(tt.block_start[tt.count]);
-        const float c1 = second ? -1.f : -0.5f, c2 = second ? 1.f : 0.f;
-        TraceScope ts("cnp_elem", 0.0, table_elems(tt) * ((second ? 12.0 : 8.0) + esize(dtype)), st);
-        if (dtype == POET_BF16) sym_many_kernel<bf16><<<blocks, 256, 0, st>>>(tt, 1.f, c1, c2);
-        else sym_many_kernel<float><<<blocks, 256, 0, st>>>(tt, 1.f, c1, c2);
+        const float c0 = second ? 1.f : 0.5f, c1 = second ? 0.f : 0.5f;
+        TraceScope ts("cnp_elem", 0.0, table_elems(tt) * ((second ? 4.0 : 8.0) + esize(dtype)), st);
+        if (dtype == POET_BF16) sym_many_kernel<bf16><<<blocks, 256, 0, st>>>(tt, c0, c1);
+        else sym_many_kernel<float><<<blocks, 256, 0, st>>>(tt, c0, c1);
         count_launch();
         return launch_status("cnp symmetric part");
       });
     };
     POET_TRY(sym(false));
     gs.clear();
-    for (int i : pw) {  // W = dT_s S
-      Gemm a = prim_gemm(geoms[i], dtype, w[i].dT, w[i].S, false, "cnp_bwd");
-      fout(a, geoms[i], w[i].W);
+    for (int i : pw) {  // V = dT_s S + U
+      const SideGeom &g = geoms[i];
+      Gemm a = prim_gemm(g, dtype, w[i].dT, w[i].S, false, "cnp_bwd");
+      a.add = w[i].UD; a.add_dtype = POET_F32; a.add_m = g.ld; a.add_b = g.blk_elems(); a.beta = 1.f;
+      fout(a, g, w[i].V);
       gs.push_back(a);
     }
     POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
     POET_TRY(sym(true));
     gs.clear();
-    for (int i : pw) {  // Y = dS_s Q (over QG, which is no longer needed)
-      Gemm a = prim_gemm(geoms[i], dtype, w[i].dT, w[i].Q, false, "cnp_bwd");
-      fout(a, geoms[i], w[i].QGY);
+    for (int i : pw) {  // D = GC - 2 dS_s Q (over U, which is no longer needed)
+      const SideGeom &g = geoms[i];
+      Gemm a = prim_gemm(g, dtype, w[i].dT, w[i].Q, false, "cnp_bwd");
+      a.alpha = -2.f;
+      a.add = w[i].GC; a.add_dtype = POET_F32; a.add_m = g.ld; a.add_b = g.blk_elems(); a.beta = 1.f;
+      fout(a, g, w[i].UD);
       gs.push_back(a);
     }
     POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
@@ -769,16 +732,13 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
   }
   POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
   // dtheta = D - D^T, every side in one launch:  k = 0: D = G;  Horner: D = A_1 + sum P_l;
-  // order 4: D = GC - 2 Y
+  // order 4: D as formed above
   return many_launch(all, [&](int i, int q) {
     const SideGeom &g = geoms[i];
     if (g.k == 0) {
       t.src[q] = G[i];
     } else if (by_powers(g)) {
-      t.src[q] = w[i].GC;
-      t.dst2[q] = w[i].QGY;
-      t.terms[q] = 1;
-      t.coef[q] = -2.f;
+      t.src[q] = w[i].UD;
     } else {
       t.src[q] = w[i].A1;
       t.dst2[q] = w[i].P;
