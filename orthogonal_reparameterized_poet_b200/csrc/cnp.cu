@@ -8,17 +8,21 @@
 // Order 4 (the order the pages' LLaMA runs use) is evaluated by powers of
 // S = Q^2, with T = S^2:  B = Q C + D0,  C = 2I + 2S + T,  D0 = I + 2S + 2T,
 // as three GEMMs whose epilogues add the rest:
-//   S = Q Q,   C = S S + 2S + 2I,   B = (Q + 2I) C - 2S - 3I
-// (the last equals Q C + D0).  The state keeps Q, Q + 2I, S and C.  Its
+//   S = Q Q,   C' = S S + 2S,   B = (Q + 2I) C' + 2Q - 2S + I
+// with C' = C - 2I (the last equals Q C + D0).  No stored matrix carries a
+// multiple of I (Q + 2I differs from Q only on its zero diagonal, where 2 is
+// exact), so bf16 storage rounds the small parts only: a stored C, whose
+// diagonal is near 2, would put its rounding, doubled, on B's diagonal.  The
+// state keeps Q, Q + 2I, S and C'.  Its
 // gradient, G = dL/dB: theta enters Q antisymmetrically (Q[a,c] = theta =
 // -Q[c,a]), so only the antisymmetric part of dL/dQ reaches dtheta; S, T and C
 // are symmetric, so only the symmetric parts of dL/dS and dL/dT matter:
 //   dT_s = sym(2G - QG),  W = dT_s S,  dS_s = sym(2G - 2QG) + W + W^T,
 //   D = G C - 2 dS_s Q,  dtheta[a,c] = D[a,c] - D[c,a]   (sym(X) = (X + X^T)/2)
 // evaluated as four GEMMs (three grouped launches) with the sums in their
-// epilogues:  U = G - Q G and G C;  V = dT_s S + U with dT_s = sym(G + U);
-// D = G C - 2 (V + V^T) Q;  so the element-wise passes between them read one
-// or two matrices each.
+// epilogues:  U = G - Q G and G C = G C' + 2G;  V = dT_s S + U with
+// dT_s = sym(G + U);  D = G C - 2 (V + V^T) Q;  so the element-wise passes
+// between them read one or two matrices each.
 //
 // Every other order, by Horner's rule on the series:
 //   S_1 = I + Q,  S_{l+1} = I + Q S_l (l = 1..k-1),  B = (I + Q) S_k = S_1 S_k
@@ -440,8 +444,8 @@ poet_status many_launch(const std::vector<int> &idx, Blocks blocks, SideTable &t
   return POET_OK;
 }
 
-// Byte offsets of the order-4 terms in a side state: Q + 2I, S and C take the
-// slots of S_1..S_3.
+// Byte offsets of the order-4 terms in a side state: Q + 2I, S and C' = C - 2I
+// take the slots of S_1..S_3.
 struct PowersLayout {
   size_t Q2, S, C;
 };
@@ -508,7 +512,7 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
     POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
   }
   if (pw.empty()) return POET_OK;
-  // order 4 by powers: S = Q Q, C = S S + 2S + 2I, B = (Q + 2I) C - 2S - 3I
+  // order 4 by powers: S = Q Q, C' = S S + 2S, B = (Q + 2I) C' + 2Q - 2S + I
   for (int step = 0; step < 3; ++step) {
     gs.clear();
     for (int i : pw) {
@@ -523,12 +527,12 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
       } else if (step == 1) {
         p = prim_gemm(g, dtype, base + W.S, base + W.S, false, "cnp_fwd");
         p.add = base + W.S; p.add_dtype = dtype; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 2.f;
-        p.diag = 2.f;
         p.outD = base + W.C;
       } else {
         p = prim_gemm(g, dtype, base + W.Q2, base + W.C, false, "cnp_fwd");
-        p.add = base + W.S; p.add_dtype = dtype; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = -2.f;
-        p.diag = -3.f;
+        p.add = base + L.Q; p.add_dtype = dtype; p.add_m = g.ld; p.add_b = g.blk_elems(); p.beta = 2.f;
+        p.add2 = base + W.S; p.add2_dtype = dtype; p.add2_m = g.ld; p.add2_b = g.blk_elems(); p.beta2 = -2.f;
+        p.diag = 1.f;
         p.outD = base + L.R;
       }
       p.od_m = g.ld; p.od_b = g.blk_elems();
@@ -546,7 +550,7 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
 //    P_k = G S_k^T, P_l = A_{l+1} S_l^T (l < k) of every side, each into its
 //    own float buffer, and one launch packs D - D^T into dtheta with
 //    D = A_1 + P_1 + ... + P_k.
-//  - order 4 by powers: U = G - Q G and G C in one launch, dT_s, V = dT_s S + U,
+//  - order 4 by powers: U = G - Q G and G C = G C' + 2G in one launch, dT_s, V = dT_s S + U,
 //    dS_s, D = G C - 2 dS_s Q, then D packed (see the top of this file).
 // Every product writes one plain output, which the tensor-core engine stores
 // through its staged epilogue.
@@ -573,7 +577,7 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
     float *P;   // Horner: P_l at P + (l-1) * pstride
     int64_t pstride;
     // order 4 by powers
-    const void *S, *C;
+    const void *S, *C;   // S and C' = C - 2I
     float *UD, *GC, *V;  // U, then D; G C; V
     void *dT;            // dT_s, then dS_s (operand type)
   };
@@ -635,7 +639,7 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
   // ---- order 4 by powers
   if (!pw.empty()) {
     gs.clear();
-    for (int i : pw) {  // U = G - Q G, GC = G C
+    for (int i : pw) {  // U = G - Q G, GC = G C' + 2G
       const SideGeom &g = geoms[i];
       Gemm a = prim_gemm(g, dtype, w[i].Q, w[i].Gop, false, "cnp_bwd");
       a.alpha = -1.f;
@@ -643,6 +647,7 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
       fout(a, g, w[i].UD);
       gs.push_back(a);
       Gemm b = prim_gemm(g, dtype, w[i].Gop, w[i].C, false, "cnp_bwd");
+      b.add = G[i]; b.add_dtype = POET_F32; b.add_m = g.ld; b.add_b = g.blk_elems(); b.beta = 2.f;
       fout(b, g, w[i].GC);
       gs.push_back(b);
     }

@@ -87,6 +87,7 @@ __global__ void __launch_bounds__(NT) gemm_simt_kernel(Gemm g, int splitk, int k
         continue;
       }
       if (g.add) v += g.beta * ld_any(g.add, g.add_dtype, int64_t(b) * g.add_b + int64_t(gm) * g.add_m + gn);
+      if (g.add2) v += g.beta2 * ld_any(g.add2, g.add2_dtype, int64_t(b) * g.add2_b + int64_t(gm) * g.add2_m + gn);
       if (gm == gn) v += g.diag;
       if (g.outF) g.outF[int64_t(b) * g.of_b + int64_t(gm) * g.of_m + gn] = v;
       if (g.outD) st_from_float<T>(static_cast<T *>(g.outD) + int64_t(b) * g.od_b + int64_t(gm) * g.od_m + gn, v);

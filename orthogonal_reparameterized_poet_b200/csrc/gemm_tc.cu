@@ -12,7 +12,7 @@
 //   warp 0     TMA producer (one elected lane) filling a STAGES-deep ring
 //   warp 1     TMEM allocator + MMA issuer (one elected lane):
 //              tcgen05.mma.cta_group::1.kind::f16, M=128, N=BN, K=16
-//   warps 2-5  epilogue: tcgen05.ld 32x32b rows out of TMEM, alpha/addend/
+//   warps 2-5  epilogue: tcgen05.ld 32x32b rows out of TMEM, alpha/addends/
 //              diagonal, bf16 and/or fp32 stores, or fp32 reductions (split-K);
 //              single plain outputs are staged through shared memory so that
 //              every store instruction covers four rows x 128 bytes
@@ -50,6 +50,7 @@ struct TcProblem {
   int num_m, num_n, nk, kchunk, splits;
   float alpha, beta, diag;
   const void *add; int add_f32; int64_t add_m, add_b;
+  const void *add2; int add2_f32; int64_t add2_m, add2_b; float beta2;  // a second addend
   float *outF; int64_t of_m, of_b;
   bf16 *outD; int64_t od_m, od_b;
   int atomic;
@@ -353,6 +354,43 @@ struct Smem {
 };
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
+
+// v[j] += beta * Add[off + j] for the j < nvalid values of one row chunk (Add
+// float or bf16): 16-byte vector loads when the chunk is whole and aligned.
+__device__ __forceinline__ void add_row(const void *add, int f32, int64_t off, float beta, int nvalid, float (&v)[32]) {
+  if (f32) {
+    const float *a = static_cast<const float *>(add) + off;
+    if (nvalid == 32 && (reinterpret_cast<uintptr_t>(a) & 15) == 0) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const float4 q = *reinterpret_cast<const float4 *>(a + j);
+        v[j] += beta * q.x; v[j + 1] += beta * q.y; v[j + 2] += beta * q.z; v[j + 3] += beta * q.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < nvalid) v[j] += beta * a[j];
+    }
+  } else {
+    const uint16_t *a = static_cast<const uint16_t *>(add) + off;
+    if (nvalid == 32 && (reinterpret_cast<uintptr_t>(a) & 15) == 0) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) {
+        const uint4 q = *reinterpret_cast<const uint4 *>(a + j);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[j + 2 * e] += beta * bf16_bits_to_float(uint16_t(w[e] & 0xFFFFu));
+          v[j + 2 * e + 1] += beta * bf16_bits_to_float(uint16_t(w[e] >> 16));
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < nvalid) v[j] += beta * bf16_bits_to_float(a[j]);
+    }
+  }
+}
 
 // out[0..3] += (a, b, c, d) as one 16-byte reduction at L2
 __device__ __forceinline__ void red_add_v4(float *out, float a, float b, float c, float d) {
@@ -807,42 +845,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(r[j]);
-        if (p.add) {
-          // the addend's 32 values of this row: 16-byte vector loads when the chunk is whole and aligned
-          const int64_t off = int64_t(c.b) * p.add_b + int64_t(gm) * p.add_m + gn0;
-          if (p.add_f32) {
-            const float *a = static_cast<const float *>(p.add) + off;
-            if (nvalid == 32 && (reinterpret_cast<uintptr_t>(a) & 15) == 0) {
-#pragma unroll
-              for (int j = 0; j < 32; j += 4) {
-                const float4 q = *reinterpret_cast<const float4 *>(a + j);
-                v[j] += beta * q.x; v[j + 1] += beta * q.y; v[j + 2] += beta * q.z; v[j + 3] += beta * q.w;
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (j < nvalid) v[j] += beta * a[j];
-            }
-          } else {
-            const uint16_t *a = static_cast<const uint16_t *>(p.add) + off;
-            if (nvalid == 32 && (reinterpret_cast<uintptr_t>(a) & 15) == 0) {
-#pragma unroll
-              for (int j = 0; j < 32; j += 8) {
-                const uint4 q = *reinterpret_cast<const uint4 *>(a + j);
-                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  v[j + 2 * e] += beta * bf16_bits_to_float(uint16_t(w[e] & 0xFFFFu));
-                  v[j + 2 * e + 1] += beta * bf16_bits_to_float(uint16_t(w[e] >> 16));
-                }
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (j < nvalid) v[j] += beta * bf16_bits_to_float(a[j]);
-            }
-          }
-        }
+        if (p.add) add_row(p.add, p.add_f32, int64_t(c.b) * p.add_b + int64_t(gm) * p.add_m + gn0, beta, nvalid, v);
+        if (p.add2) add_row(p.add2, p.add2_f32, int64_t(c.b) * p.add2_b + int64_t(gm) * p.add2_m + gn0, p.beta2, nvalid, v);
         if (diag != 0.f && gm >= gn0 && gm < gn0 + 32) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -1001,6 +1005,8 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   p->splits = (p->nk + p->kchunk - 1) / p->kchunk;
   p->alpha = g.alpha; p->beta = g.beta; p->diag = g.diag;
   p->add = g.add; p->add_f32 = g.add_dtype == POET_F32; p->add_m = g.add_m; p->add_b = g.add_b;
+  p->add2 = g.add2; p->add2_f32 = g.add2_dtype == POET_F32; p->add2_m = g.add2_m; p->add2_b = g.add2_b;
+  p->beta2 = g.beta2;
   p->outF = g.outF; p->of_m = g.of_m; p->of_b = g.of_b;
   p->outD = static_cast<bf16 *>(g.outD); p->od_m = g.od_m; p->od_b = g.od_b;
   p->atomic = g.atomic ? 1 : 0;
@@ -1019,13 +1025,13 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   // 3: bf16, any rows; 2: fp32, 16-byte aligned rows, stored or reduced); the
   // per-row path handles addends, pairs of outputs and unaligned fp32 rows
   p->coalesced = 0;
-  const bool plain = !g.add && !g.atomic && g.diag == 0.f;
+  const bool plain = !g.add && !g.add2 && !g.atomic && g.diag == 0.f;
   if (plain && g.outD && !g.outF) {
     p->coalesced = aligned16(g.outD) && g.od_m % 8 == 0 && (g.batch == 1 || g.od_b % 8 == 0) ? 1 : 3;
     if (t.bstat && p->coalesced == 3) p->coalesced = 0;  // the B-stationary kernels stage aligned rows only
   }
   // fp32: plain stores or split-K reductions
-  if (!g.add && g.diag == 0.f && g.outF && !g.outD && aligned16(g.outF) && g.of_m % 4 == 0 &&
+  if (!g.add && !g.add2 && g.diag == 0.f && g.outF && !g.outD && aligned16(g.outF) && g.of_m % 4 == 0 &&
       (g.batch == 1 || g.of_b % 4 == 0))
     p->coalesced = 2;
   bool ok;
@@ -1160,7 +1166,8 @@ bool gemm_tc_supported(const Gemm &g) {
   const bool b_mn = g.b_n == 1 && g.b_k % 8 == 0 && g.b_k >= 1;
   if (!(a_k || a_mn) || !(b_k || b_mn)) return false;
   if (g.batch > 1 && (g.a_b % 8 != 0 || g.b_b % 8 != 0 || g.a_b <= 0 || g.b_b <= 0)) return false;
-  if (g.atomic && (g.add || g.outD || !g.outF)) return false;
+  if (g.atomic && (g.add || g.add2 || g.outD || !g.outF)) return false;
+  if (g.add2 && !g.add) return false;
   return true;
 }
 

@@ -324,7 +324,8 @@ poet_status gemm_run(const Gemm &g, cudaStream_t st) {
   const double mnb = double(g.M) * g.N * g.batch;
   const double bytes = double(esize(g.dtype)) * (double(g.M) + g.N) * g.K * g.batch +
                        mnb * ((g.outF ? 4.0 : 0.0) + (g.outD ? double(esize(g.dtype)) : 0.0) +
-                              (g.add ? double(esize(g.add_dtype)) : 0.0));
+                              (g.add ? double(esize(g.add_dtype)) : 0.0) +
+                              (g.add2 ? double(esize(g.add2_dtype)) : 0.0));
   TraceScope ts(g.tag, 2.0 * mnb * g.K, bytes, st);
   if (gemm_tc_enabled() && gemm_tc_supported(g)) return gemm_tc(g, st);
   return gemm_simt(g, st);
@@ -348,7 +349,7 @@ poet_status gemm_run_many(const Gemm *gs, int count, cudaStream_t st) {
     flop += 2.0 * mnb * g.K;
     bytes += double(esize(g.dtype)) * (double(g.M) + g.N) * g.K * g.batch +
              mnb * ((g.outF ? 4.0 : 0.0) + (g.outD ? double(esize(g.dtype)) : 0.0) +
-                    (g.add ? double(esize(g.add_dtype)) : 0.0));
+                    (g.add ? double(esize(g.add_dtype)) : 0.0) + (g.add2 ? double(esize(g.add2_dtype)) : 0.0));
   }
   TraceScope ts(gs[0].tag, flop, bytes, st);
   return gemm_tc_many(gs, count, st);

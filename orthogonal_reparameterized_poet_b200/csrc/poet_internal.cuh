@@ -106,7 +106,8 @@ StateLayout state_layout(const SideGeom &g, int dtype);
 
 // ------------------------------------------------------------------ GEMM engine
 //
-//   v(b,i,j) = alpha * sum_l A(b,i,l) * B(b,j,l)  (+ beta * Add(b,i,j)) (+ diag if i == j)
+//   v(b,i,j) = alpha * sum_l A(b,i,l) * B(b,j,l)  (+ beta * Add(b,i,j)) (+ beta2 * Add2(b,i,j))
+//              (+ diag if i == j)
 //   A(b,i,l) = A[b*a_b + i*a_m + l*a_k], B(b,j,l) = B[b*b_b + j*b_n + l*b_k]
 // then v is stored to outF (float) and/or outD (element type `dtype`), or
 // added atomically into outF (split-K allowed).
@@ -117,6 +118,7 @@ struct Gemm {
   const void *B = nullptr; int64_t b_n = 0, b_k = 0, b_b = 0;
   float alpha = 1.f;
   const void *add = nullptr; int add_dtype = POET_F32; int64_t add_m = 0, add_b = 0; float beta = 0.f;
+  const void *add2 = nullptr; int add2_dtype = POET_F32; int64_t add2_m = 0, add2_b = 0; float beta2 = 0.f;
   float diag = 0.f;
   float *outF = nullptr; int64_t of_m = 0, of_b = 0;
   void *outD = nullptr; int64_t od_m = 0, od_b = 0;

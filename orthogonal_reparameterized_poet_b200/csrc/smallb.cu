@@ -255,7 +255,7 @@ poet_status smallb_grad(int dtype, const void *D, const void *V, int64_t ld, int
 
 poet_status smallb_dispatch(const Gemm &g, cudaStream_t st, bool *done) {
   *done = false;
-  if (!g.small || g.alpha != 1.f || g.add || g.diag != 0.f) return POET_OK;
+  if (!g.small || g.alpha != 1.f || g.add || g.add2 || g.diag != 0.f) return POET_OK;
   if (g.small == SMALL_RIGHT) {
     // A = X (K contiguous, blocks s apart), B_j(a, c) = B[a][c] (b_n = ld) or B[c][a] (b_n = 1)
     if (!smallb_supported(g.K) || g.N != g.K || g.a_k != 1 || g.a_b != g.K || !g.outD || g.outF || g.od_b != g.K)
