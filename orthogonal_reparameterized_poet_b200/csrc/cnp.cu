@@ -219,7 +219,6 @@ poet_status cnp_backward(const poet_side *side, const SideGeom &g, int dtype, co
 namespace {
 
 constexpr int kSidesMax = 64;
-constexpr int kItems = 4;  // elements per thread in the element-wise many-side kernels
 
 struct SideTable {
   int count;
@@ -248,65 +247,105 @@ __device__ __forceinline__ int side_of_block(const SideTable &t) {
   return lo;
 }
 
+// Tile pair (ta <= tc, 32 x 32 tiles over [0, span)) of primitive j handled by
+// this block: the pairs of a primitive are numbered row by row (ta, then tc),
+// and the row of a number comes from the quadratic formula, then is corrected
+// by one step where float rounding put it off.
+struct TilePair {
+  int j, ta, tc;
+};
+__device__ __forceinline__ TilePair tile_pair(const SideTable &t, int i, int span) {
+  const int tiles = (span + PACK_T - 1) / PACK_T;
+  const int pairs = tiles * (tiles + 1) / 2;
+  const int64_t local = int64_t(blockIdx.x) - t.block_start[i];
+  TilePair p;
+  p.j = int(local / pairs);
+  const int r = int(local % pairs);
+  // row ta starts at start(ta) = ta * tiles - ta (ta - 1) / 2
+  const float b = 2.f * float(tiles) + 1.f;
+  int ta = int(0.5f * (b - sqrtf(fmaxf(b * b - 8.f * float(r), 0.f))));
+  ta = ta < 0 ? 0 : (ta > tiles - 1 ? tiles - 1 : ta);
+  while (ta + 1 < tiles && (ta + 1) * tiles - (ta + 1) * ta / 2 <= r) ++ta;
+  while (ta > 0 && ta * tiles - ta * (ta - 1) / 2 > r) --ta;
+  p.ta = ta;
+  p.tc = ta + (r - (ta * tiles - ta * (ta - 1) / 2));
+  return p;
+}
+
 // src = theta, dst = Q, dst2 = Q + coef I (Horner's S_1 = I + Q, or B = I + Q
 // when k = 0, with coef 1; Q + 2I for order 4; nullptr: not written), dst3 = B
 // whose padding (rows or columns >= size) is zeroed (nullptr: none).  Padding
-// of Q and dst2 is zero.
+// of Q and dst2 is zero.  One block per pair of 32 x 32 tiles (ta <= tc) over
+// [0, ld): theta of the upper tile is read row-contiguously into shared
+// memory, and the tile and its mirror (negated, transposed) are written.
 template <typename T>
 __global__ void __launch_bounds__(256) unpack_many_kernel(const __grid_constant__ SideTable t) {
+  __shared__ float u[PACK_T][PACK_T + 1];
   const int i = side_of_block(t);
   const int size = t.size[i], ld = t.ld[i];
-  const int64_t blk = int64_t(ld) * ld, total = blk * t.nprim[i];
+  const TilePair tp = tile_pair(t, i, ld);
   const int64_t per = int64_t(size) * (size - 1) / 2;
-  const float *theta = static_cast<const float *>(t.src[i]);
-  T *Q = static_cast<T *>(t.dst[i]);
-  T *IplusQ = static_cast<T *>(t.dst2[i]);
-  T *Bpad = static_cast<T *>(t.dst3[i]);
-  const int64_t e0 = (int64_t(blockIdx.x) - t.block_start[i]) * (256 * kItems);
-  const int64_t e1 = e0 + 256 * kItems < total ? e0 + 256 * kItems : total;
-  for (int64_t e = e0 + threadIdx.x; e < e1; e += 256) {
-    const int j = int(e / blk);
-    const int a = int((e % blk) / ld), c = int(e % ld);
-    float q = 0.f, eye = 0.f;
-    const bool inside = a < size && c < size;
-    if (inside) {
-      if (a < c) q = theta[j * per + packed_index(a, c, size)];
-      else if (a > c) q = -theta[j * per + packed_index(c, a, size)];
-      else eye = 1.f;
+  const float *theta = static_cast<const float *>(t.src[i]) + int64_t(tp.j) * per;
+  const int64_t off = int64_t(tp.j) * ld * ld;
+  T *Q = static_cast<T *>(t.dst[i]) + off;
+  T *Q2 = t.dst2[i] ? static_cast<T *>(t.dst2[i]) + off : nullptr;
+  T *Bpad = t.dst3[i] ? static_cast<T *>(t.dst3[i]) + off : nullptr;
+  const float coef = t.coef[i];
+  const int x = threadIdx.x % PACK_T;
+  // u[y][x] = Q[ta*32+y][tc*32+x] where a < c < size, else 0
+  for (int y = threadIdx.x / PACK_T; y < PACK_T; y += 256 / PACK_T) {
+    const int a = tp.ta * PACK_T + y, c = tp.tc * PACK_T + x;
+    u[y][x] = (a < c && c < size) ? theta[packed_index(a, c, size)] : 0.f;
+  }
+  __syncthreads();
+  for (int y = threadIdx.x / PACK_T; y < PACK_T; y += 256 / PACK_T) {
+    {  // tile (ta, tc); on the diagonal tile the lower part is the mirror
+      const int a = tp.ta * PACK_T + y, c = tp.tc * PACK_T + x;
+      if (a < ld && c < ld) {
+        const float q = (tp.ta == tp.tc && a > c) ? -u[x][y] : u[y][x];
+        const float eye = (a == c && a < size) ? 1.f : 0.f;
+        const int64_t e = int64_t(a) * ld + c;
+        Q[e] = from_f<T>(q);
+        if (Q2) Q2[e] = from_f<T>(q + coef * eye);
+        if (Bpad && (a >= size || c >= size)) Bpad[e] = from_f<T>(0.f);
+      }
     }
-    Q[e] = from_f<T>(q);
-    if (IplusQ) IplusQ[e] = from_f<T>(q + t.coef[i] * eye);
-    if (Bpad && !inside) Bpad[e] = from_f<T>(0.f);
+    if (tp.ta != tp.tc) {  // tile (tc, ta): Q[a][c] = -Q[c][a]
+      const int a = tp.tc * PACK_T + y, c = tp.ta * PACK_T + x;
+      if (a < ld && c < ld) {
+        const float q = -u[x][y];
+        const int64_t e = int64_t(a) * ld + c;
+        Q[e] = from_f<T>(q);
+        if (Q2) Q2[e] = from_f<T>(q);
+        if (Bpad && (a >= size || c >= size)) Bpad[e] = from_f<T>(0.f);
+      }
+    }
   }
 }
 
-// src = G (float), dst = its bf16 copy, nprim * ld * ld elements
+// src = G (float), dst = its bf16 copy, nprim * ld * ld elements; eight per
+// thread, as two 16-byte loads and one 16-byte store where both are aligned
+constexpr int kRoundItems = 8;
 __global__ void __launch_bounds__(256) round_many_kernel(const __grid_constant__ SideTable t) {
   const int i = side_of_block(t);
   const int64_t total = int64_t(t.ld[i]) * t.ld[i] * t.nprim[i];
   const float *G = static_cast<const float *>(t.src[i]);
   bf16 *out = static_cast<bf16 *>(t.dst[i]);
-  const int64_t e0 = (int64_t(blockIdx.x) - t.block_start[i]) * (256 * kItems);
-  const int64_t e1 = e0 + 256 * kItems < total ? e0 + 256 * kItems : total;
-  for (int64_t e = e0 + threadIdx.x; e < e1; e += 256) out[e] = __float2bfloat16_rn(G[e]);
-}
-
-// Tile pair (ta <= tc, 32 x 32 tiles) of primitive j handled by this block.
-struct TilePair {
-  int j, ta, tc;
-};
-__device__ __forceinline__ TilePair tile_pair(const SideTable &t, int i) {
-  const int size = t.size[i];
-  const int tiles = (size + PACK_T - 1) / PACK_T;
-  const int pairs = tiles * (tiles + 1) / 2;
-  const int64_t local = int64_t(blockIdx.x) - t.block_start[i];
-  TilePair p;
-  p.j = int(local / pairs);
-  int ta = 0, rem = int(local % pairs);
-  while (rem >= tiles - ta) { rem -= tiles - ta; ++ta; }
-  p.ta = ta;
-  p.tc = ta + rem;
-  return p;
+  const bool vec = ((reinterpret_cast<uintptr_t>(G) | reinterpret_cast<uintptr_t>(out)) & 15) == 0;
+  const int64_t e = (int64_t(blockIdx.x) - t.block_start[i]) * (256 * kRoundItems) + int64_t(threadIdx.x) * kRoundItems;
+  if (vec && e + kRoundItems <= total) {
+    const float4 lo = *reinterpret_cast<const float4 *>(G + e), hi = *reinterpret_cast<const float4 *>(G + e + 4);
+    const __nv_bfloat162 h0 = __floats2bfloat162_rn(lo.x, lo.y), h1 = __floats2bfloat162_rn(lo.z, lo.w);
+    const __nv_bfloat162 h2 = __floats2bfloat162_rn(hi.x, hi.y), h3 = __floats2bfloat162_rn(hi.z, hi.w);
+    uint4 pk;
+    pk.x = *reinterpret_cast<const uint32_t *>(&h0);
+    pk.y = *reinterpret_cast<const uint32_t *>(&h1);
+    pk.z = *reinterpret_cast<const uint32_t *>(&h2);
+    pk.w = *reinterpret_cast<const uint32_t *>(&h3);
+    *reinterpret_cast<uint4 *>(out + e) = pk;
+  } else {
+    for (int64_t q = e; q < e + kRoundItems && q < total; ++q) out[q] = __float2bfloat16_rn(G[q]);
+  }
 }
 
 // Order-4 gradient, symmetric combinations: dst = c0 (X_0 + X_0^T) + c1 (X_1 +
@@ -319,7 +358,7 @@ __global__ void __launch_bounds__(256) sym_many_kernel(const __grid_constant__ S
   __shared__ float u1[PACK_T][PACK_T + 1], u2[PACK_T][PACK_T + 1];
   const int i = side_of_block(t);
   const int size = t.size[i], ld = t.ld[i];
-  const TilePair tp = tile_pair(t, i);
+  const TilePair tp = tile_pair(t, i, size);
   const int64_t off = int64_t(tp.j) * ld * ld;
   const float *X[2] = {static_cast<const float *>(t.src[i]), static_cast<const float *>(t.src2[i])};
   const float cf[2] = {c0, c1};
@@ -360,7 +399,7 @@ __global__ void __launch_bounds__(256) pack_many_kernel(const __grid_constant__ 
   __shared__ float t1[PACK_T][PACK_T + 1], t2[PACK_T][PACK_T + 1];
   const int i = side_of_block(t);
   const int size = t.size[i], ld = t.ld[i];
-  const TilePair tp = tile_pair(t, i);
+  const TilePair tp = tile_pair(t, i, size);
   const int64_t off = int64_t(tp.j) * ld * ld;
   const float *dQ = static_cast<const float *>(t.src[i]) + off;
   const int terms = t.terms[i];
@@ -416,11 +455,13 @@ double table_elems(const SideTable &t) {
   return e;
 }
 
-int64_t elem_blocks(const SideGeom &g) { return (g.all_elems() + 256 * kItems - 1) / (256 * kItems); }
-int64_t pair_blocks(const SideGeom &g) {
-  const int64_t tiles = (g.size + PACK_T - 1) / PACK_T;
+int64_t round_blocks(const SideGeom &g) { return (g.all_elems() + 256 * kRoundItems - 1) / (256 * kRoundItems); }
+// tile pairs (ta <= tc) over [0, span) of every primitive
+int64_t pairs_over(const SideGeom &g, int span) {
+  const int64_t tiles = (span + PACK_T - 1) / PACK_T;
   return int64_t(g.nprim) * tiles * (tiles + 1) / 2;
 }
+int64_t pair_blocks(const SideGeom &g) { return pairs_over(g, g.size); }
 
 // Fill a table with the sides of idx[0..n) (blocks per side from `blocks`) and launch.
 template <typename Launch, typename Blocks>
@@ -478,7 +519,7 @@ poet_status cnp_forward_many(const poet_side *sides, const SideGeom *geoms, int 
     t.coef[q] = by_powers(g) ? 2.f : 1.f;
     t.dst3[q] = g.k == 0 ? nullptr : base + L.R;
     t.nprim[q] = g.nprim; t.size[q] = g.size; t.ld[q] = g.ld;
-    return elem_blocks(g);
+    return pairs_over(g, g.ld);
   }, t, [&](const SideTable &tt, int, int) {
     const int blocks = int(tt.block_start[tt.count]);
     TraceScope ts("cnp_elem", 0.0, table_elems(tt) * (2.0 * esize(dtype) + 2.0), st);
@@ -626,7 +667,7 @@ poet_status cnp_backward_many(const poet_side *sides, const SideGeom *geoms, int
       t.src[q] = G[i];
       t.dst[q] = const_cast<void *>(w[i].Gop);
       t.nprim[q] = g.nprim; t.size[q] = g.size; t.ld[q] = g.ld;
-      return elem_blocks(g);
+      return round_blocks(g);
     }, t, [&](const SideTable &tt, int, int) {
       TraceScope ts("cnp_elem", 0.0, table_elems(tt) * 6.0, st);
       round_many_kernel<<<int(tt.block_start[tt.count]), 256, 0, st>>>(tt);

@@ -1093,27 +1093,36 @@ template <int MAXP>
 poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
   static thread_local TcGroup<MAXP> grp;  // large: keep it off the stack
   int64_t base_tiles = 0;
+  double kb_sum = 0.0;  // k-blocks summed over the base tiles
   for (int i = 0; i < n; ++i) {
     const int64_t mt = (gs[i].M + BM * t.cg - 1) / (BM * t.cg), nt = (gs[i].N + t.BN - 1) / t.BN;
     base_tiles += mt * nt * gs[i].batch;
+    kb_sum += double(mt * nt * gs[i].batch) * double((gs[i].K + BK - 1) / BK);
   }
-  // Split K (atomic outputs only) into s parts, s chosen so that the tiles
-  // fill whole waves of persistent CTAs: take the smallest s within 2% of the
-  // best wave efficiency tiles / (ceil(tiles / SMs) * SMs), s <= 16.
+  // Split K (atomic outputs only) into s parts.  A tile of k k-blocks takes
+  // about max(k, kEpiKb) + 1 k-block times (its float reduction takes about
+  // kEpiKb, overlapped with the next tile's products), and the tiles run in
+  // ceil(tiles / workers) waves; s minimizes waves(s) * (max(kavg / s,
+  // kEpiKb) + 1), the smallest s within 1% of the best, s <= 16.  (Filling
+  // waves alone picked up to 15 splits of 2048-deep products whose every
+  // 3-k-block tile then waited on a whole tile's reduction.)
   int split_want = 1;
   bool any_atomic = false;
   for (int i = 0; i < n; ++i) any_atomic |= gs[i].atomic;
   if (any_atomic && base_tiles > 0) {
-    const int64_t sms = num_sms() / t.cg;  // concurrent tile workers: CTAs or CTA pairs
+    constexpr double kEpiKb = 6.0;
+    const int64_t workers = num_sms() / t.cg;  // concurrent tile workers: CTAs or CTA pairs
+    const double kavg = kb_sum / double(base_tiles);
+    double cost[17] = {};
     double best = 0.0;
     for (int sp = 1; sp <= 16; ++sp) {
-      const int64_t tiles = base_tiles * sp;
-      const double eff = double(tiles) / double(((tiles + sms - 1) / sms) * sms);
-      if (eff > best + 0.02) {
-        best = eff;
-        split_want = sp;
-      }
+      const int64_t waves = (base_tiles * sp + workers - 1) / workers;
+      const double per = kavg / sp;
+      cost[sp] = double(waves) * ((per > kEpiKb ? per : kEpiKb) + 1.0);
+      if (sp == 1 || cost[sp] < best) best = cost[sp];
     }
+    for (int sp = 1; sp <= 16; ++sp)
+      if (cost[sp] <= 1.01 * best) { split_want = sp; break; }
   }
   grp.count = n;
   grp.errword = device_errword();
