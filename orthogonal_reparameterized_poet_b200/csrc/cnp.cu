@@ -348,6 +348,49 @@ __global__ void __launch_bounds__(256) round_many_kernel(const __grid_constant__
   }
 }
 
+// The tile-pair kernels below give each thread four consecutive columns of
+// one row of a 32 x 32 tile: threadIdx.x / 8 is the row, (threadIdx.x % 8) * 4
+// the first column, so that a warp reads four rows x 128 contiguous bytes.
+
+// v[e] = sum_q cf_q X_q[row][col + e] for e < 4 (0 outside [0, size)^2); one
+// 16-byte load per matrix when the four columns are inside and aligned.
+__device__ __forceinline__ void load_quad(const float *const *X, const float *cf, int nx, int row, int col, int size,
+                                          int ld, bool vec, float (&v)[4]) {
+  v[0] = v[1] = v[2] = v[3] = 0.f;
+  if (row >= size || col >= size) return;
+  const int64_t o = int64_t(row) * ld + col;
+  for (int q = 0; q < nx; ++q) {
+    if (!X[q]) continue;
+    if (vec && col + 4 <= size) {
+      const float4 f = *reinterpret_cast<const float4 *>(X[q] + o);
+      v[0] += cf[q] * f.x; v[1] += cf[q] * f.y; v[2] += cf[q] * f.z; v[3] += cf[q] * f.w;
+    } else {
+      for (int e = 0; e < 4 && col + e < size; ++e) v[e] += cf[q] * X[q][o + e];
+    }
+  }
+}
+
+// out[row][col + e] = v[e] for the columns inside [0, size): one 8-byte
+// (bf16) or 16-byte (float) store when all four are inside and aligned.
+template <typename T>
+__device__ __forceinline__ void store_quad(T *out, int row, int col, int size, int ld, bool vec, const float (&v)[4]) {
+  if (row >= size || col >= size) return;
+  T *o = out + int64_t(row) * ld + col;
+  if (vec && col + 4 <= size) {
+    if constexpr (sizeof(T) == 2) {
+      const __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t *>(&h0);
+      pk.y = *reinterpret_cast<const uint32_t *>(&h1);
+      *reinterpret_cast<uint2 *>(o) = pk;
+    } else {
+      *reinterpret_cast<float4 *>(o) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+  } else {
+    for (int e = 0; e < 4 && col + e < size; ++e) o[e] = from_f<T>(v[e]);
+  }
+}
+
 // Order-4 gradient, symmetric combinations: dst = c0 (X_0 + X_0^T) + c1 (X_1 +
 // X_1^T) over X_0 = src and X_1 = src2 (float [nprim][ld][ld]; src2 may be
 // nullptr), in the operand type.  One block per pair of 32 x 32 tiles
@@ -360,32 +403,32 @@ __global__ void __launch_bounds__(256) sym_many_kernel(const __grid_constant__ S
   const int size = t.size[i], ld = t.ld[i];
   const TilePair tp = tile_pair(t, i, size);
   const int64_t off = int64_t(tp.j) * ld * ld;
-  const float *X[2] = {static_cast<const float *>(t.src[i]), static_cast<const float *>(t.src2[i])};
+  const float *X[2] = {static_cast<const float *>(t.src[i]) + off,
+                       t.src2[i] ? static_cast<const float *>(t.src2[i]) + off : nullptr};
   const float cf[2] = {c0, c1};
   T *out = static_cast<T *>(t.dst[i]) + off;
-  const int x = threadIdx.x % PACK_T;
+  const bool vec = ((reinterpret_cast<uintptr_t>(X[0]) | reinterpret_cast<uintptr_t>(X[1]) |
+                     reinterpret_cast<uintptr_t>(out)) & 15) == 0;
+  const int y = threadIdx.x / 8, x = (threadIdx.x % 8) * 4;
   // u1[y][x] = sum c_q X_q[ta*32+y][tc*32+x],  u2[y][x] = sum c_q X_q[tc*32+y][ta*32+x]
-  for (int y = threadIdx.x / PACK_T; y < PACK_T; y += 256 / PACK_T) {
-    const int a1 = tp.ta * PACK_T + y, b1 = tp.tc * PACK_T + x;
-    const int a2 = tp.tc * PACK_T + y, b2 = tp.ta * PACK_T + x;
-    float v1 = 0.f, v2 = 0.f;
+  float v1[4], v2[4];
+  load_quad(X, cf, 2, tp.ta * PACK_T + y, tp.tc * PACK_T + x, size, ld, vec, v1);
+  load_quad(X, cf, 2, tp.tc * PACK_T + y, tp.ta * PACK_T + x, size, ld, vec, v2);
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      if (!X[q]) continue;
-      if (a1 < size && b1 < size) v1 += cf[q] * X[q][off + int64_t(a1) * ld + b1];
-      if (a2 < size && b2 < size) v2 += cf[q] * X[q][off + int64_t(a2) * ld + b2];
-    }
-    u1[y][x] = v1;
-    u2[y][x] = v2;
+  for (int e = 0; e < 4; ++e) {
+    u1[y][x + e] = v1[e];
+    u2[y][x + e] = v2[e];
   }
   __syncthreads();
   // out[ta*32+y][tc*32+x] = u1[y][x] + u2[x][y];  out[tc*32+y][ta*32+x] = u2[y][x] + u1[x][y]
-  for (int y = threadIdx.x / PACK_T; y < PACK_T; y += 256 / PACK_T) {
-    const int a1 = tp.ta * PACK_T + y, b1 = tp.tc * PACK_T + x;
-    const int a2 = tp.tc * PACK_T + y, b2 = tp.ta * PACK_T + x;
-    if (a1 < size && b1 < size) out[int64_t(a1) * ld + b1] = from_f<T>(u1[y][x] + u2[x][y]);
-    if (tp.ta != tp.tc && a2 < size && b2 < size) out[int64_t(a2) * ld + b2] = from_f<T>(u2[y][x] + u1[x][y]);
+  float w1[4], w2[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    w1[e] = u1[y][x + e] + u2[x + e][y];
+    w2[e] = u2[y][x + e] + u1[x + e][y];
   }
+  store_quad(out, tp.ta * PACK_T + y, tp.tc * PACK_T + x, size, ld, vec, w1);
+  if (tp.ta != tp.tc) store_quad(out, tp.tc * PACK_T + y, tp.ta * PACK_T + x, size, ld, vec, w2);
 }
 
 // dst = dtheta: dtheta[j][idx(a,c)] = D[a][c] - D[c][a] with D = src +
@@ -408,41 +451,50 @@ __global__ void __launch_bounds__(256) pack_many_kernel(const __grid_constant__ 
   const int64_t stride = t.stride[i];
   float *dtheta = t.dst[i] ? static_cast<float *>(t.dst[i]) + int64_t(tp.j) * (int64_t(size) * (size - 1) / 2)
                            : nullptr;
-  const int x = threadIdx.x % PACK_T;
-  for (int y = threadIdx.x / PACK_T; y < PACK_T; y += 256 / PACK_T) {
-    const int a1 = tp.ta * PACK_T + y, c1 = tp.tc * PACK_T + x;
-    const int a2 = tp.tc * PACK_T + y, c2 = tp.ta * PACK_T + x;
-    float v1 = 0.f, v2 = 0.f;
-    if (a1 < size && c1 < size) {
-      const int64_t o = int64_t(a1) * ld + c1;
-      float acc = 0.f;
-      for (int q = 0; q < terms; ++q) acc += P[q * stride + o];
-      v1 = dQ[o] + coef * acc;
+  const bool vec = ((reinterpret_cast<uintptr_t>(dQ) | reinterpret_cast<uintptr_t>(P)) & 15) == 0 && stride % 4 == 0;
+  const int y = threadIdx.x / 8, x = (threadIdx.x % 8) * 4;
+  // t1[y][x] = D[ta*32+y][tc*32+x],  t2[y][x] = D[tc*32+y][ta*32+x]
+  auto load_d = [&](int row, int col, float (&v)[4]) {
+    const float *one[1] = {dQ};
+    const float cf1[1] = {1.f};
+    load_quad(one, cf1, 1, row, col, size, ld, vec, v);
+    if (terms == 0) return;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int q = 0; q < terms; ++q) {
+      const float *pq[1] = {P + q * stride};
+      float w[4];
+      load_quad(pq, cf1, 1, row, col, size, ld, vec, w);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] += w[e];
     }
-    if (a2 < size && c2 < size) {
-      const int64_t o = int64_t(a2) * ld + c2;
-      float acc = 0.f;
-      for (int q = 0; q < terms; ++q) acc += P[q * stride + o];
-      v2 = dQ[o] + coef * acc;
-    }
-    t1[y][x] = v1;
-    t2[y][x] = v2;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] += coef * acc[e];
+  };
+  float v1[4], v2[4];
+  load_d(tp.ta * PACK_T + y, tp.tc * PACK_T + x, v1);
+  load_d(tp.tc * PACK_T + y, tp.ta * PACK_T + x, v2);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    t1[y][x + e] = v1[e];
+    t2[y][x + e] = v2[e];
   }
   __syncthreads();
   const int64_t pbase = int64_t(tp.j) * (int64_t(size) * (size - 1) / 2);
-  for (int y = threadIdx.x / PACK_T; y < PACK_T; y += 256 / PACK_T) {
-    const int a = tp.ta * PACK_T + y, c = tp.tc * PACK_T + x;
+  const int a = tp.ta * PACK_T + y;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int c = tp.tc * PACK_T + x + e;
     if (a < c && c < size) {
       const int64_t idx = packed_index(a, c, size);
-      const float g = t1[y][x] - t2[x][y];
+      const float g = t1[y][x + e] - t2[x + e][y];
       if (!ADAM || t.dst[i]) dtheta[idx] = g;
       if constexpr (ADAM) {
-        const int64_t e = pbase + idx;
-        float th = t.theta[i][e], mm = t.m1[i][e], vv = t.m2[i][e];
+        const int64_t q = pbase + idx;
+        float th = t.theta[i][q], mm = t.m1[i][q], vv = t.m2[i][q];
         adamw_one(th, g, mm, vv, h);
-        t.theta[i][e] = th;
-        t.m1[i][e] = mm;
-        t.m2[i][e] = vv;
+        t.theta[i][q] = th;
+        t.m1[i][q] = mm;
+        t.m2[i][q] = vv;
       }
     }
   }

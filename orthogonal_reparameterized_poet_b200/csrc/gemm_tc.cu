@@ -54,7 +54,7 @@ struct TcProblem {
   float *outF; int64_t of_m, of_b;
   bf16 *outD; int64_t od_m, od_b;
   int atomic;
-  int coalesced;  // plain bf16 output, 16-byte aligned rows: stores staged through shared memory
+  int coalesced;  // staged epilogue mode (0: per row; 1, 3: bf16; 2: fp32; 4: addends, diagonal, pairs)
   int m_fast;     // tile order: M tiles fastest (N > M: CTAs of a wave share B slabs)
   int group_m;    // split-K: M tiles per group (a group runs all its splits before the next group)
 };
@@ -388,6 +388,31 @@ __device__ __forceinline__ void add_row(const void *add, int f32, int64_t off, f
 #pragma unroll
       for (int j = 0; j < 32; ++j)
         if (j < nvalid) v[j] += beta * bf16_bits_to_float(a[j]);
+    }
+  }
+}
+
+// v[0..nv) += beta * Add[off ..): one 16-byte (float) or 8-byte (bf16) load
+// when all four values are wanted (the staged epilogue's addends are aligned).
+__device__ __forceinline__ void add_quad(const void *add, int f32, int64_t off, float beta, int nv, float (&v)[4]) {
+  if (f32) {
+    const float *a = static_cast<const float *>(add) + off;
+    if (nv == 4) {
+      const float4 q = *reinterpret_cast<const float4 *>(a);
+      v[0] += beta * q.x; v[1] += beta * q.y; v[2] += beta * q.z; v[3] += beta * q.w;
+    } else {
+      for (int e = 0; e < nv; ++e) v[e] += beta * a[e];
+    }
+  } else {
+    const uint16_t *a = static_cast<const uint16_t *>(add) + off;
+    if (nv == 4) {
+      const uint2 q = *reinterpret_cast<const uint2 *>(a);
+      v[0] += beta * bf16_bits_to_float(uint16_t(q.x & 0xFFFFu));
+      v[1] += beta * bf16_bits_to_float(uint16_t(q.x >> 16));
+      v[2] += beta * bf16_bits_to_float(uint16_t(q.y & 0xFFFFu));
+      v[3] += beta * bf16_bits_to_float(uint16_t(q.y >> 16));
+    } else {
+      for (int e = 0; e < nv; ++e) v[e] += beta * bf16_bits_to_float(a[e]);
     }
   }
 }
@@ -819,6 +844,71 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
             }
           }
         }
+      } else if (p.coalesced == 4) {
+        // addends and/or a diagonal, fp32 and/or bf16 outputs (aligned rows):
+        // staged as in mode 2, then each thread finishes four columns of a
+        // row, so that a warp's addend loads and stores cover four rows x 32
+        // contiguous columns
+        unsigned char *ew = epi + quarter * (32 * S::EPI_ROW);
+        const int m_base = mrow0 + quarter * 32;
+        const int sub = lane & 7, rsub = lane >> 3;
+        unsigned char *myrow = ew + lane * S::EPI_ROW;
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          uint32_t r[32];
+          __syncwarp();
+          tmem_ld32(tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN + cc * 32), r);
+          tmem_ld_wait();
+          const int gn0 = c.nt * BN + cc * 32;
+          if (gn0 >= p.N) continue;  // the same for the whole warp
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float4 f;
+            f.x = alpha * __uint_as_float(r[4 * q]);
+            f.y = alpha * __uint_as_float(r[4 * q + 1]);
+            f.z = alpha * __uint_as_float(r[4 * q + 2]);
+            f.w = alpha * __uint_as_float(r[4 * q + 3]);
+            *reinterpret_cast<float4 *>(myrow + q * 16) = f;
+          }
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + rsub;
+            const int gm = m_base + rr;
+            const int gn = gn0 + sub * 4;
+            if (gm >= p.M || gn >= p.N) continue;
+            const float4 f = *reinterpret_cast<const float4 *>(ew + rr * S::EPI_ROW + sub * 16);
+            float v[4] = {f.x, f.y, f.z, f.w};
+            const int nv = min(4, p.N - gn);
+            if (p.add) add_quad(p.add, p.add_f32, int64_t(c.b) * p.add_b + int64_t(gm) * p.add_m + gn, beta, nv, v);
+            if (p.add2)
+              add_quad(p.add2, p.add2_f32, int64_t(c.b) * p.add2_b + int64_t(gm) * p.add2_m + gn, p.beta2, nv, v);
+            if (diag != 0.f) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (gn + e == gm) v[e] += diag;
+            }
+            if (p.outF) {
+              float *o = p.outF + int64_t(c.b) * p.of_b + int64_t(gm) * p.of_m + gn;
+              if (nv == 4) {
+                *reinterpret_cast<float4 *>(o) = make_float4(v[0], v[1], v[2], v[3]);
+              } else {
+                for (int e = 0; e < nv; ++e) o[e] = v[e];
+              }
+            }
+            if (p.outD) {
+              bf16 *o = p.outD + int64_t(c.b) * p.od_b + int64_t(gm) * p.od_m + gn;
+              if (nv == 4) {
+                const __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
+                uint2 pk;
+                pk.x = *reinterpret_cast<const uint32_t *>(&h0);
+                pk.y = *reinterpret_cast<const uint32_t *>(&h1);
+                *reinterpret_cast<uint2 *>(o) = pk;
+              } else {
+                for (int e = 0; e < nv; ++e) o[e] = __float2bfloat16_rn(v[e]);
+              }
+            }
+          }
+        }
       } else
       for (int cc = 0; cc < BN / 32; ++cc) {
         uint32_t r[32];
@@ -1034,6 +1124,20 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   if (!g.add && !g.add2 && g.diag == 0.f && g.outF && !g.outD && aligned16(g.outF) && g.of_m % 4 == 0 &&
       (g.batch == 1 || g.of_b % 4 == 0))
     p->coalesced = 2;
+  // 4: addends, a diagonal or a pair of outputs, every row 16-byte (fp32) or
+  // 8-byte (bf16) aligned
+  if (p->coalesced == 0 && !g.atomic && (g.add || g.diag != 0.f || (g.outF && g.outD))) {
+    auto rows_ok = [&](const void *ptr, bool f32, int64_t ld, int64_t bs) {
+      const uintptr_t a = reinterpret_cast<uintptr_t>(ptr);
+      return (a & (f32 ? 15 : 7)) == 0 && ld % 4 == 0 && (g.batch == 1 || bs % 4 == 0);
+    };
+    bool ok4 = g.outF || g.outD;
+    if (g.outF) ok4 = ok4 && rows_ok(g.outF, true, g.of_m, g.of_b);
+    if (g.outD) ok4 = ok4 && rows_ok(g.outD, false, g.od_m, g.od_b);
+    if (g.add) ok4 = ok4 && rows_ok(g.add, g.add_dtype == POET_F32, g.add_m, g.add_b);
+    if (g.add2) ok4 = ok4 && rows_ok(g.add2, g.add2_dtype == POET_F32, g.add2_m, g.add2_b);
+    if (ok4) p->coalesced = 4;
+  }
   bool ok;
   if (!t.A_MN) ok = make_map(ma, g.A, g.K, g.M, g.batch, g.a_m, g.a_b, 64, BM);
   else ok = make_map(ma, g.A, g.M, g.K, g.batch, g.a_k, g.a_b, 64, 64);
