@@ -30,6 +30,7 @@
 // too), frees TMEM and returns.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdlib>
 #include <mutex>
 #include <vector>
@@ -392,27 +393,29 @@ __device__ __forceinline__ void add_row(const void *add, int f32, int64_t off, f
   }
 }
 
-// v[0..nv) += beta * Add[off ..): one 16-byte (float) or 8-byte (bf16) load
-// when all four values are wanted (the staged epilogue's addends are aligned).
-__device__ __forceinline__ void add_quad(const void *add, int f32, int64_t off, float beta, int nv, float (&v)[4]) {
+// q[0..nv) = Add[off ..) as float (0 past nv): one 16-byte (float) or
+// 8-byte (bf16) load when all four values are wanted (the staged epilogue's
+// addends are aligned).
+__device__ __forceinline__ void load_quad(const void *add, int f32, int64_t off, int nv, float (&q)[4]) {
+  q[0] = q[1] = q[2] = q[3] = 0.f;
   if (f32) {
     const float *a = static_cast<const float *>(add) + off;
     if (nv == 4) {
-      const float4 q = *reinterpret_cast<const float4 *>(a);
-      v[0] += beta * q.x; v[1] += beta * q.y; v[2] += beta * q.z; v[3] += beta * q.w;
+      const float4 v = *reinterpret_cast<const float4 *>(a);
+      q[0] = v.x; q[1] = v.y; q[2] = v.z; q[3] = v.w;
     } else {
-      for (int e = 0; e < nv; ++e) v[e] += beta * a[e];
+      for (int e = 0; e < nv; ++e) q[e] = a[e];
     }
   } else {
     const uint16_t *a = static_cast<const uint16_t *>(add) + off;
     if (nv == 4) {
-      const uint2 q = *reinterpret_cast<const uint2 *>(a);
-      v[0] += beta * bf16_bits_to_float(uint16_t(q.x & 0xFFFFu));
-      v[1] += beta * bf16_bits_to_float(uint16_t(q.x >> 16));
-      v[2] += beta * bf16_bits_to_float(uint16_t(q.y & 0xFFFFu));
-      v[3] += beta * bf16_bits_to_float(uint16_t(q.y >> 16));
+      const uint2 v = *reinterpret_cast<const uint2 *>(a);
+      q[0] = bf16_bits_to_float(uint16_t(v.x & 0xFFFFu));
+      q[1] = bf16_bits_to_float(uint16_t(v.x >> 16));
+      q[2] = bf16_bits_to_float(uint16_t(v.y & 0xFFFFu));
+      q[3] = bf16_bits_to_float(uint16_t(v.y >> 16));
     } else {
-      for (int e = 0; e < nv; ++e) v[e] += beta * bf16_bits_to_float(a[e]);
+      for (int e = 0; e < nv; ++e) q[e] = bf16_bits_to_float(a[e]);
     }
   }
 }
@@ -450,12 +453,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
   const bool leader = rank == 0;
   const int64_t units = CG == 2 ? int64_t(cluster_count()) : int64_t(gridDim.x);
   const int64_t unit = CG == 2 ? int64_t(cluster_id()) : int64_t(blockIdx.x);
-  // Tiles of this CTA (pair): strided over the grid (streaming), or one
-  // contiguous range (B-stationary, so that consecutive tiles share their B operand).
+  // Tiles of this CTA (pair): one contiguous range (B-stationary, so that
+  // consecutive tiles share their B operand), or one tile of each wave of
+  // `units` consecutive tiles (streaming), the waves taken in alternating
+  // directions.  The host orders a launch's problems by decreasing K, so the
+  // long tiles come first and the short ones of the later waves even out
+  // what the long ones left; within a wave the tiles stay consecutive, which
+  // keeps their shared operand slabs together in L2.
   const int64_t per_cta = (tiles + units - 1) / units;
   const int64_t t_first = BSTAT ? unit * per_cta : unit;
-  const int64_t t_step = BSTAT ? 1 : units;
   const int64_t t_end = BSTAT ? (t_first + per_cta < tiles ? t_first + per_cta : tiles) : tiles;
+  auto tile_of = [&](int64_t k) -> int64_t {
+    if (BSTAT) return t_first + k;
+    return k * units + ((k & 1) ? units - 1 - unit : unit);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -499,7 +510,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       uint32_t bfree_phase = 0;
       uint32_t bloads = 0;
       const uint32_t full0 = CG == 2 ? mapa_shared(smem_u32(full), 0) : 0;  // rank 0's full[0]
-      for (int64_t tile = t_first; tile < t_end && !*abort; tile += t_step) {
+      for (int64_t k = 0;; ++k) {
+        const int64_t tile = tile_of(k);
+        if (tile >= t_end || *abort) break;
         const TileCoord c = decode(tile, g);
         const TcProblem &p = g.prob[c.pi];
         const CUtensorMap *ma = &g.ma[c.pi];
@@ -608,7 +621,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       bool issued = false;
       int res_pi = -1, res_b = -1;  // B-stationary: operand currently resident
       uint32_t bfull_phase = 0;
-      for (int64_t tile = t_first; tile < t_end && !*abort; tile += t_step) {
+      for (int64_t k = 0;; ++k) {
+        const int64_t tile = tile_of(k);
+        if (tile >= t_end || *abort) break;
         const TileCoord c = decode(tile, g);
         const TcProblem &p = g.prob[c.pi];
         const int kb0 = c.s * p.kchunk;
@@ -650,9 +665,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
         else umma_commit(&tfull[acc]);
         if constexpr (BSTAT) {
           // the resident B is released after the last tile that reads it
-          bool last_use = tile + t_step >= t_end;
+          bool last_use = tile_of(k + 1) >= t_end;
           if (!last_use) {
-            const TileCoord nc = decode(tile + t_step, g);
+            const TileCoord nc = decode(tile_of(k + 1), g);
             last_use = nc.pi != c.pi || nc.b != c.b;
           }
           if (last_use) umma_commit(bfree);
@@ -676,7 +691,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int64_t tile = t_first; tile < t_end && !*abort; tile += t_step) {
+    for (int64_t k = 0;; ++k) {
+      const int64_t tile = tile_of(k);
+      if (tile >= t_end || *abort) break;
       const TileCoord c = decode(tile, g);
       const TcProblem &p = g.prob[c.pi];
       if (!mbar_wait(&tfull[acc], acc_phase, abort, g.errword)) break;
@@ -870,6 +887,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
             *reinterpret_cast<float4 *>(myrow + q * 16) = f;
           }
           __syncwarp();
+          // every addend value of this thread's eight quads is loaded before
+          // any store (one load latency per chunk, not one per quad: the
+          // stores could alias the addends for all the compiler knows)
+          float qa[8][4], qb[8][4];
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int gm = m_base + it * 4 + rsub;
+            const int gn = gn0 + sub * 4;
+            const bool in = gm < p.M && gn < p.N;
+            const int nv = in ? min(4, p.N - gn) : 0;
+            if (p.add) load_quad(p.add, p.add_f32, int64_t(c.b) * p.add_b + int64_t(gm) * p.add_m + gn, nv, qa[it]);
+            if (p.add2)
+              load_quad(p.add2, p.add2_f32, int64_t(c.b) * p.add2_b + int64_t(gm) * p.add2_m + gn, nv, qb[it]);
+          }
 #pragma unroll
           for (int it = 0; it < 8; ++it) {
             const int rr = it * 4 + rsub;
@@ -879,9 +910,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
             const float4 f = *reinterpret_cast<const float4 *>(ew + rr * S::EPI_ROW + sub * 16);
             float v[4] = {f.x, f.y, f.z, f.w};
             const int nv = min(4, p.N - gn);
-            if (p.add) add_quad(p.add, p.add_f32, int64_t(c.b) * p.add_b + int64_t(gm) * p.add_m + gn, beta, nv, v);
-            if (p.add2)
-              add_quad(p.add2, p.add2_f32, int64_t(c.b) * p.add2_b + int64_t(gm) * p.add2_m + gn, p.beta2, nv, v);
+            if (p.add) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) v[e] += beta * qa[it][e];
+            }
+            if (p.add2) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) v[e] += p.beta2 * qb[it][e];
+            }
             if (diag != 0.f) {
 #pragma unroll
               for (int e = 0; e < 4; ++e)
@@ -1061,6 +1097,14 @@ const int g_pairs_mode = [] {
   return 1;
 }();
 
+// Split-K: POET_GEMM_SPLITK_MAX=n caps the number of K splits of a launch with
+// float-reduced outputs (default 16; 1 turns split-K off).
+const int g_splitk_max = [] {
+  const char *e = std::getenv("POET_GEMM_SPLITK_MAX");
+  const int v = e ? std::atoi(e) : 16;
+  return v < 1 ? 1 : (v > 16 ? 16 : v);
+}();
+
 // Operand majors and tile width of a supported problem.
 struct TcPlan {
   bool A_MN, B_MN;
@@ -1099,7 +1143,7 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   p->beta2 = g.beta2;
   p->outF = g.outF; p->of_m = g.of_m; p->of_b = g.of_b;
   p->outD = static_cast<bf16 *>(g.outD); p->od_m = g.od_m; p->od_b = g.od_b;
-  p->atomic = g.atomic ? 1 : 0;
+  p->atomic = g.atomic && p->splits > 1 ? 1 : 0;  // one split: the zeroed output is simply stored
   // consecutive tiles (one wave of persistent CTAs) share the slabs of the
   // larger operand, which is then read from HBM about once
   p->m_fast = g.N > g.M ? 1 : 0;
@@ -1219,22 +1263,27 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
     const double kavg = kb_sum / double(base_tiles);
     double cost[17] = {};
     double best = 0.0;
-    for (int sp = 1; sp <= 16; ++sp) {
+    for (int sp = 1; sp <= g_splitk_max; ++sp) {
       const int64_t waves = (base_tiles * sp + workers - 1) / workers;
       const double per = kavg / sp;
       cost[sp] = double(waves) * ((per > kEpiKb ? per : kEpiKb) + 1.0);
       if (sp == 1 || cost[sp] < best) best = cost[sp];
     }
-    for (int sp = 1; sp <= 16; ++sp)
+    for (int sp = 1; sp <= g_splitk_max; ++sp)
       if (cost[sp] <= 1.01 * best) { split_want = sp; break; }
   }
+  // problems in decreasing K order (their tiles' length; ties keep the list order)
+  int order[MAXP];
+  for (int i = 0; i < n; ++i) order[i] = i;
+  std::stable_sort(order, order + n, [&](int a, int b) { return gs[a].K > gs[b].K; });
   grp.count = n;
   grp.errword = device_errword();
   grp.tile_start[0] = 0;
   for (int i = 0; i < n; ++i) {
     TcProblem &p = grp.prob[i];
-    if (!fill_problem(gs[i], t, split_want, &p, &grp.ma[i], &grp.mb[i])) {
-      set_error("gemm_tc: tensor map encoding failed (M=%d N=%d K=%d)", gs[i].M, gs[i].N, gs[i].K);
+    const Gemm &gi = gs[order[i]];
+    if (!fill_problem(gi, t, split_want, &p, &grp.ma[i], &grp.mb[i])) {
+      set_error("gemm_tc: tensor map encoding failed (M=%d N=%d K=%d)", gi.M, gi.N, gi.K);
       return POET_ECUDA;
     }
     grp.tile_start[i + 1] = grp.tile_start[i] + int64_t(p.num_m) * p.num_n * p.splits * p.batch;

@@ -109,8 +109,9 @@ StateLayout state_layout(const SideGeom &g, int dtype);
 //   v(b,i,j) = alpha * sum_l A(b,i,l) * B(b,j,l)  (+ beta * Add(b,i,j)) (+ beta2 * Add2(b,i,j))
 //              (+ diag if i == j)
 //   A(b,i,l) = A[b*a_b + i*a_m + l*a_k], B(b,j,l) = B[b*b_b + j*b_n + l*b_k]
-// then v is stored to outF (float) and/or outD (element type `dtype`), or
-// added atomically into outF (split-K allowed).
+// then v is stored to outF (float) and/or outD (element type `dtype`).  With
+// `atomic`, outF holds zeros on entry and the engine may split K, adding the
+// partial sums into it (or store v when it does not split).
 struct Gemm {
   int M = 0, N = 0, K = 0, batch = 1;
   int dtype = POET_F32;                       // type of A, B, outD
