@@ -1105,6 +1105,13 @@ const int g_splitk_max = [] {
   return v < 1 ? 1 : (v > 16 ? 16 : v);
 }();
 
+// Staged epilogue for addends, diagonals and paired outputs (mode 4):
+// POET_GEMM_EPI4=1 turns it on; by default such products take the per-row path.
+const bool g_epi4 = [] {
+  const char *e = std::getenv("POET_GEMM_EPI4");
+  return e && e[0] == '1';
+}();
+
 // Operand majors and tile width of a supported problem.
 struct TcPlan {
   bool A_MN, B_MN;
@@ -1170,7 +1177,7 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
     p->coalesced = 2;
   // 4: addends, a diagonal or a pair of outputs, every row 16-byte (fp32) or
   // 8-byte (bf16) aligned
-  if (p->coalesced == 0 && !g.atomic && (g.add || g.diag != 0.f || (g.outF && g.outD))) {
+  if (g_epi4 && p->coalesced == 0 && !g.atomic && (g.add || g.diag != 0.f || (g.outF && g.outD))) {
     auto rows_ok = [&](const void *ptr, bool f32, int64_t ld, int64_t bs) {
       const uintptr_t a = reinterpret_cast<uintptr_t>(ptr);
       return (a & (f32 ? 15 : 7)) == 0 && ld % 4 == 0 && (g.batch == 1 || bs % 4 == 0);

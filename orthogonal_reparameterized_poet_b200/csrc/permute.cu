@@ -323,14 +323,11 @@ __global__ void __launch_bounds__(256) restride_kernel(const unsigned char *__re
 
 // out[a][c] = bf16(D[rowmap[a]][perm[c]]): a float matrix gathered into the
 // frame and rounded in one pass, for up to kFrameMax matrices per launch
-// (matrix p owns the global rows [row_start[p], row_start[p+1])).  CTA c
-// works through the contiguous global rows [total*c/G, total*(c+1)/G), one
-// segment per matrix it touches: it keeps that matrix's column map (uint16)
-// in shared memory and streams the source rows through two row slots, the
-// next row's 16-byte cp.async copies in flight while the current row is
-// gathered.  An index out of range (rowmap outside [0, rows), perm outside
-// [0, d)) is not read: its output is 0 and ERR_BOUNDS is set in the status
-// word.
+// (matrix p owns the global rows [row_start[p], row_start[p+1])).  One block
+// per output row at a time; the source row is read through L1 (it is reused
+// by the block's gathers).  An index out of range (rowmap outside [0, rows),
+// perm outside [0, d)) is not read: its output is 0 and ERR_BOUNDS is set in
+// the status word.
 constexpr int kFrameMax = 64;
 struct FrameGroup {
   const float *D[kFrameMax];
@@ -343,76 +340,53 @@ struct FrameGroup {
   int d[kFrameMax];
   int64_t row_start[kFrameMax + 1];
   int count;
-  int map_len;  // map entries (a multiple of 8 >= the widest d)
-  int slot;     // floats per row slot (a multiple of 4 >= the widest d)
   unsigned *errword;
 };
 static_assert(sizeof(FrameGroup) <= 32000, "frame table exceeds the kernel parameter limit");
 
 __global__ void __launch_bounds__(256) frame_f32_to_bf16_kernel(const __grid_constant__ FrameGroup g) {
-  extern __shared__ __align__(16) unsigned char fsm[];
-  uint16_t *map = reinterpret_cast<uint16_t *>(fsm);
-  float *slots = reinterpret_cast<float *>(fsm + size_t(g.map_len) * 2);
+  // a row of D is staged in shared memory with 16-byte copies (coalesced), then
+  // gathered from there; rows whose start is not 16-byte aligned are gathered
+  // from global memory directly
+  extern __shared__ __align__(16) float srow[];
   bool bad = false;
   const int64_t total = g.row_start[g.count];
-  const int64_t r0 = total * blockIdx.x / gridDim.x, r1 = total * (blockIdx.x + 1) / gridDim.x;
   int p = 0;
-  for (int64_t seg = r0; seg < r1;) {
-    while (g.row_start[p + 1] <= seg) ++p;
-    const int64_t seg_end = r1 < g.row_start[p + 1] ? r1 : g.row_start[p + 1];
-    const int64_t lo = seg - g.row_start[p], hi = seg_end - g.row_start[p];  // rows [lo, hi) of matrix p
-    seg = seg_end;
+  for (int64_t gr = blockIdx.x; gr < total; gr += gridDim.x) {
+    while (g.row_start[p + 1] <= gr) ++p;  // rows are visited in increasing order
+    const int64_t a = gr - g.row_start[p], rows = g.rows[p];
     const int d = g.d[p];
-    const int64_t rows = g.rows[p];
-    const float *D = g.D[p];
-    __syncthreads();  // the previous segment's readers of map and slots are done
-    for (int c = threadIdx.x; c < d; c += blockDim.x) {
-      const int pc = g.perm[p][c];
-      const bool ok = unsigned(pc) < unsigned(d);
-      map[c] = ok ? uint16_t(pc) : uint16_t(0);
-      bad |= !ok;
+    const int32_t *perm = g.perm[p];
+    const int64_t sr = __ldg(g.rowmap[p] + a);
+    const bool row_ok = sr >= 0 && sr < rows;
+    bad |= !row_ok;
+    const float *src = g.D[p] + (row_ok ? sr : 0) * g.ldD[p];
+    const bool staged = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+    if (staged) {
+      __syncthreads();  // the previous row's readers of srow are done
+      const int units = d / 4;
+      for (int u = threadIdx.x; u < units; u += blockDim.x) cp_async16(srow + 4 * u, src + 4 * u);
+      for (int c = 4 * units + threadIdx.x; c < d; c += blockDim.x) srow[c] = src[c];
+      cp_async_wait_all();
+      __syncthreads();
     }
-    // source row of output row a, or nullptr (its row-map entry is out of range)
-    auto src_of = [&](int64_t a) -> const float * {
-      const int64_t sr = __ldg(g.rowmap[p] + a);
-      return sr >= 0 && sr < rows ? D + sr * g.ldD[p] : nullptr;
-    };
-    auto issue = [&](int64_t a, float *slot) {
-      const float *src = src_of(a);
-      if (src) {
-        if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
-          const int units = d / 4;
-          for (int u = threadIdx.x; u < units; u += blockDim.x) cp_async16(slot + 4 * u, src + 4 * u);
-          for (int c = 4 * units + threadIdx.x; c < d; c += blockDim.x) slot[c] = src[c];
-        } else {
-          for (int c = threadIdx.x; c < d; c += blockDim.x) slot[c] = src[c];
-        }
+    bf16 *orow = g.out[p] + a * g.ld_out[p];
+    for (int c = 2 * threadIdx.x; c < d; c += 2 * blockDim.x) {
+      if (c + 1 < d) {
+        const int2 pc = *reinterpret_cast<const int2 *>(perm + c);
+        const bool okx = row_ok && unsigned(pc.x) < unsigned(d), oky = row_ok && unsigned(pc.y) < unsigned(d);
+        bad |= !(okx && oky);
+        const float vx = okx ? (staged ? srow[pc.x] : __ldg(src + pc.x)) : 0.f;
+        const float vy = oky ? (staged ? srow[pc.y] : __ldg(src + pc.y)) : 0.f;
+        *reinterpret_cast<__nv_bfloat162 *>(orow + c) = __floats2bfloat162_rn(vx, vy);
+      } else {
+        const int pc = perm[c];
+        const bool ok = row_ok && unsigned(pc) < unsigned(d);
+        bad |= !ok;
+        orow[c] = __float2bfloat16_rn(ok ? (staged ? srow[pc] : __ldg(src + pc)) : 0.f);
       }
-      cp_async_commit();
-    };
-    if (lo < hi) issue(lo, slots);
-    for (int64_t a = lo; a < hi; ++a) {
-      float *cur = slots + int64_t((a - lo) & 1) * g.slot;
-      float *nxt = slots + int64_t(((a - lo) & 1) ^ 1) * g.slot;
-      if (a + 1 < hi) issue(a + 1, nxt);
-      else cp_async_commit();
-      cp_async_wait_one();  // this thread's copies of row a have landed
-      __syncthreads();      // everyone's (and the map)
-      const bool row_ok = src_of(a) != nullptr;
-      bad |= !row_ok;
-      bf16 *orow = g.out[p] + a * g.ld_out[p];
-      for (int c = 2 * threadIdx.x; c < d; c += 2 * blockDim.x) {
-        if (c + 1 < d) {
-          const float vx = row_ok ? cur[map[c]] : 0.f, vy = row_ok ? cur[map[c + 1]] : 0.f;
-          *reinterpret_cast<__nv_bfloat162 *>(orow + c) = __floats2bfloat162_rn(vx, vy);
-        } else {
-          orow[c] = __float2bfloat16_rn(row_ok ? cur[map[c]] : 0.f);
-        }
-      }
-      __syncthreads();  // row a's readers are done before its slot is refilled
     }
   }
-  cp_async_wait_all();
   if (bad && g.errword) atomicOr(g.errword, ERR_BOUNDS);
 }
 
@@ -573,9 +547,7 @@ poet_status frame_many(const std::vector<FrameItem> &v, cudaStream_t st) {
     grp.errword = device_errword();
     int dmax = 0;
     for (int q = 0; q < grp.count; ++q) dmax = grp.d[q] > dmax ? grp.d[q] : dmax;
-    grp.map_len = int(round_up(dmax, 8));
-    grp.slot = int(round_up(dmax, 4));
-    const size_t smem = size_t(grp.map_len) * 2 + 2 * size_t(grp.slot) * 4;  // map and two row slots
+    const size_t smem = size_t(dmax) * 4;  // one staged row of the widest matrix
     POET_REQUIRE(smem <= 200 * 1024, "frame: rows of %d floats do not fit in shared memory", dmax);
     static int configured[64] = {};
     int dev = 0;
