@@ -55,7 +55,7 @@ struct TcProblem {
   float *outF; int64_t of_m, of_b;
   bf16 *outD; int64_t od_m, od_b;
   int atomic;
-  int coalesced;  // staged epilogue mode (0: per row; 1, 3: bf16; 2: fp32; 4: addends, diagonal, pairs)
+  int coalesced;  // staged epilogue mode (0: per row; 1, 3: bf16; 2: fp32)
   int m_fast;     // tile order: M tiles fastest (N > M: CTAs of a wave share B slabs)
   int group_m;    // split-K: M tiles per group (a group runs all its splits before the next group)
 };
@@ -389,33 +389,6 @@ __device__ __forceinline__ void add_row(const void *add, int f32, int64_t off, f
 #pragma unroll
       for (int j = 0; j < 32; ++j)
         if (j < nvalid) v[j] += beta * bf16_bits_to_float(a[j]);
-    }
-  }
-}
-
-// q[0..nv) = Add[off ..) as float (0 past nv): one 16-byte (float) or
-// 8-byte (bf16) load when all four values are wanted (the staged epilogue's
-// addends are aligned).
-__device__ __forceinline__ void load_quad(const void *add, int f32, int64_t off, int nv, float (&q)[4]) {
-  q[0] = q[1] = q[2] = q[3] = 0.f;
-  if (f32) {
-    const float *a = static_cast<const float *>(add) + off;
-    if (nv == 4) {
-      const float4 v = *reinterpret_cast<const float4 *>(a);
-      q[0] = v.x; q[1] = v.y; q[2] = v.z; q[3] = v.w;
-    } else {
-      for (int e = 0; e < nv; ++e) q[e] = a[e];
-    }
-  } else {
-    const uint16_t *a = static_cast<const uint16_t *>(add) + off;
-    if (nv == 4) {
-      const uint2 v = *reinterpret_cast<const uint2 *>(a);
-      q[0] = bf16_bits_to_float(uint16_t(v.x & 0xFFFFu));
-      q[1] = bf16_bits_to_float(uint16_t(v.x >> 16));
-      q[2] = bf16_bits_to_float(uint16_t(v.y & 0xFFFFu));
-      q[3] = bf16_bits_to_float(uint16_t(v.y >> 16));
-    } else {
-      for (int e = 0; e < nv; ++e) q[e] = bf16_bits_to_float(a[e]);
     }
   }
 }
@@ -861,90 +834,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
             }
           }
         }
-      } else if (p.coalesced == 4) {
-        // addends and/or a diagonal, fp32 and/or bf16 outputs (aligned rows):
-        // staged as in mode 2, then each thread finishes four columns of a
-        // row, so that a warp's addend loads and stores cover four rows x 32
-        // contiguous columns
-        unsigned char *ew = epi + quarter * (32 * S::EPI_ROW);
-        const int m_base = mrow0 + quarter * 32;
-        const int sub = lane & 7, rsub = lane >> 3;
-        unsigned char *myrow = ew + lane * S::EPI_ROW;
-        for (int cc = 0; cc < BN / 32; ++cc) {
-          uint32_t r[32];
-          __syncwarp();
-          tmem_ld32(tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN + cc * 32), r);
-          tmem_ld_wait();
-          const int gn0 = c.nt * BN + cc * 32;
-          if (gn0 >= p.N) continue;  // the same for the whole warp
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float4 f;
-            f.x = alpha * __uint_as_float(r[4 * q]);
-            f.y = alpha * __uint_as_float(r[4 * q + 1]);
-            f.z = alpha * __uint_as_float(r[4 * q + 2]);
-            f.w = alpha * __uint_as_float(r[4 * q + 3]);
-            *reinterpret_cast<float4 *>(myrow + q * 16) = f;
-          }
-          __syncwarp();
-          // every addend value of this thread's eight quads is loaded before
-          // any store (one load latency per chunk, not one per quad: the
-          // stores could alias the addends for all the compiler knows)
-          float qa[8][4], qb[8][4];
-#pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int gm = m_base + it * 4 + rsub;
-            const int gn = gn0 + sub * 4;
-            const bool in = gm < p.M && gn < p.N;
-            const int nv = in ? min(4, p.N - gn) : 0;
-            if (p.add) load_quad(p.add, p.add_f32, int64_t(c.b) * p.add_b + int64_t(gm) * p.add_m + gn, nv, qa[it]);
-            if (p.add2)
-              load_quad(p.add2, p.add2_f32, int64_t(c.b) * p.add2_b + int64_t(gm) * p.add2_m + gn, nv, qb[it]);
-          }
-#pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int rr = it * 4 + rsub;
-            const int gm = m_base + rr;
-            const int gn = gn0 + sub * 4;
-            if (gm >= p.M || gn >= p.N) continue;
-            const float4 f = *reinterpret_cast<const float4 *>(ew + rr * S::EPI_ROW + sub * 16);
-            float v[4] = {f.x, f.y, f.z, f.w};
-            const int nv = min(4, p.N - gn);
-            if (p.add) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) v[e] += beta * qa[it][e];
-            }
-            if (p.add2) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) v[e] += p.beta2 * qb[it][e];
-            }
-            if (diag != 0.f) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (gn + e == gm) v[e] += diag;
-            }
-            if (p.outF) {
-              float *o = p.outF + int64_t(c.b) * p.of_b + int64_t(gm) * p.of_m + gn;
-              if (nv == 4) {
-                *reinterpret_cast<float4 *>(o) = make_float4(v[0], v[1], v[2], v[3]);
-              } else {
-                for (int e = 0; e < nv; ++e) o[e] = v[e];
-              }
-            }
-            if (p.outD) {
-              bf16 *o = p.outD + int64_t(c.b) * p.od_b + int64_t(gm) * p.od_m + gn;
-              if (nv == 4) {
-                const __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
-                uint2 pk;
-                pk.x = *reinterpret_cast<const uint32_t *>(&h0);
-                pk.y = *reinterpret_cast<const uint32_t *>(&h1);
-                *reinterpret_cast<uint2 *>(o) = pk;
-              } else {
-                for (int e = 0; e < nv; ++e) o[e] = __float2bfloat16_rn(v[e]);
-              }
-            }
-          }
-        }
       } else
       for (int cc = 0; cc < BN / 32; ++cc) {
         uint32_t r[32];
@@ -1105,13 +994,6 @@ const int g_splitk_max = [] {
   return v < 1 ? 1 : (v > 16 ? 16 : v);
 }();
 
-// Staged epilogue for addends, diagonals and paired outputs (mode 4):
-// POET_GEMM_EPI4=1 turns it on; by default such products take the per-row path.
-const bool g_epi4 = [] {
-  const char *e = std::getenv("POET_GEMM_EPI4");
-  return e && e[0] == '1';
-}();
-
 // Operand majors and tile width of a supported problem.
 struct TcPlan {
   bool A_MN, B_MN;
@@ -1175,20 +1057,6 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
   if (!g.add && !g.add2 && g.diag == 0.f && g.outF && !g.outD && aligned16(g.outF) && g.of_m % 4 == 0 &&
       (g.batch == 1 || g.of_b % 4 == 0))
     p->coalesced = 2;
-  // 4: addends, a diagonal or a pair of outputs, every row 16-byte (fp32) or
-  // 8-byte (bf16) aligned
-  if (g_epi4 && p->coalesced == 0 && !g.atomic && (g.add || g.diag != 0.f || (g.outF && g.outD))) {
-    auto rows_ok = [&](const void *ptr, bool f32, int64_t ld, int64_t bs) {
-      const uintptr_t a = reinterpret_cast<uintptr_t>(ptr);
-      return (a & (f32 ? 15 : 7)) == 0 && ld % 4 == 0 && (g.batch == 1 || bs % 4 == 0);
-    };
-    bool ok4 = g.outF || g.outD;
-    if (g.outF) ok4 = ok4 && rows_ok(g.outF, true, g.of_m, g.of_b);
-    if (g.outD) ok4 = ok4 && rows_ok(g.outD, false, g.od_m, g.od_b);
-    if (g.add) ok4 = ok4 && rows_ok(g.add, g.add_dtype == POET_F32, g.add_m, g.add_b);
-    if (g.add2) ok4 = ok4 && rows_ok(g.add2, g.add2_dtype == POET_F32, g.add2_m, g.add2_b);
-    if (ok4) p->coalesced = 4;
-  }
   bool ok;
   if (!t.A_MN) ok = make_map(ma, g.A, g.K, g.M, g.batch, g.a_m, g.a_b, 64, BM);
   else ok = make_map(ma, g.A, g.M, g.K, g.batch, g.a_k, g.a_b, 64, 64);
