@@ -109,6 +109,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity.  Returns false (after
 // recording ERR_TIMEOUT and raising the CTA's abort flag) if it runs out, or
 // if another role of the CTA has already aborted.
@@ -613,9 +626,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
         bool ok = true;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort, g.errword)) { ok = false; break; }
-          tc_fence_after();
+        // The k-blocks go two at a time: both stages' barriers are tested back
+        // to back, so that the two tests' round trips overlap.  A barrier test
+        // sits on this thread's path between k-blocks, and one per k-block
+        // left the tensor pipe idle about a third of the time.
+        auto issue_kb = [&](int kb) {
           const uint32_t sa = smem_u32(stage_base + size_t(stage) * S::STAGE_BYTES);
           const uint32_t sb = BSTAT ? smem_u32(bres + size_t(kb) * S::B_BYTES) : sa + S::A_BYTES;
 #pragma unroll
@@ -632,6 +647,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
             stage = 0;
             phase ^= 1;
           }
+        };
+        for (int kb = kb0; kb < kb1; kb += 2) {
+          const bool two = kb + 1 < kb1;
+          const int s1 = stage + 1 == STAGES ? 0 : stage + 1;
+          const uint32_t ph1 = stage + 1 == STAGES ? phase ^ 1 : phase;
+          const bool r0 = mbar_test(&full[stage], phase);
+          const bool r1 = !two || mbar_test(&full[s1], ph1);
+          if (!r0 && !mbar_wait(&full[stage], phase, abort, g.errword)) { ok = false; break; }
+          tc_fence_after();
+          issue_kb(kb);
+          if (!two) break;
+          if (!r1 && !mbar_wait(&full[stage], phase, abort, g.errword)) { ok = false; break; }
+          tc_fence_after();
+          issue_kb(kb + 1);
         }
         if (!ok) break;
         if constexpr (CG == 2) umma_commit_pair_both(&tfull[acc]);
