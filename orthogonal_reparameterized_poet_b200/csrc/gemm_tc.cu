@@ -626,10 +626,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
         bool ok = true;
-        // The k-blocks go two at a time: both stages' barriers are tested back
-        // to back, so that the two tests' round trips overlap.  A barrier test
-        // sits on this thread's path between k-blocks, and one per k-block
-        // left the tensor pipe idle about a third of the time.
+        // The barrier of the next k-block's stage is tested before this
+        // k-block's MMAs are issued, so that the test's round trip overlaps
+        // the issue.  A test on the path between k-blocks left the tensor pipe
+        // idle about a third of the time.
         auto issue_kb = [&](int kb) {
           const uint32_t sa = smem_u32(stage_base + size_t(stage) * S::STAGE_BYTES);
           const uint32_t sb = BSTAT ? smem_u32(bres + size_t(kb) * S::B_BYTES) : sa + S::A_BYTES;
@@ -648,19 +648,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
             phase ^= 1;
           }
         };
-        for (int kb = kb0; kb < kb1; kb += 2) {
-          const bool two = kb + 1 < kb1;
+        bool ready = kb0 < kb1 && mbar_test(&full[stage], phase);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!ready && !mbar_wait(&full[stage], phase, abort, g.errword)) { ok = false; break; }
+          tc_fence_after();
           const int s1 = stage + 1 == STAGES ? 0 : stage + 1;
           const uint32_t ph1 = stage + 1 == STAGES ? phase ^ 1 : phase;
-          const bool r0 = mbar_test(&full[stage], phase);
-          const bool r1 = !two || mbar_test(&full[s1], ph1);
-          if (!r0 && !mbar_wait(&full[stage], phase, abort, g.errword)) { ok = false; break; }
-          tc_fence_after();
+          ready = kb + 1 < kb1 && mbar_test(&full[s1], ph1);
           issue_kb(kb);
-          if (!two) break;
-          if (!r1 && !mbar_wait(&full[stage], phase, abort, g.errword)) { ok = false; break; }
-          tc_fence_after();
-          issue_kb(kb + 1);
         }
         if (!ok) break;
         if constexpr (CG == 2) umma_commit_pair_both(&tfull[acc]);
