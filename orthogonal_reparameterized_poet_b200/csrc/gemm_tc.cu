@@ -607,6 +607,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       bool issued = false;
       int res_pi = -1, res_b = -1;  // B-stationary: operand currently resident
       uint32_t bfull_phase = 0;
+      bool ready = false;  // the next k-block's stage has been seen full
       for (int64_t k = 0;; ++k) {
         const int64_t tile = tile_of(k);
         if (tile >= t_end || *abort) break;
@@ -648,13 +649,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
             phase ^= 1;
           }
         };
-        bool ready = kb0 < kb1 && mbar_test(&full[stage], phase);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!ready && !mbar_wait(&full[stage], phase, abort, g.errword)) { ok = false; break; }
           tc_fence_after();
           const int s1 = stage + 1 == STAGES ? 0 : stage + 1;
           const uint32_t ph1 = stage + 1 == STAGES ? phase ^ 1 : phase;
-          ready = kb + 1 < kb1 && mbar_test(&full[s1], ph1);
+          ready = mbar_test(&full[s1], ph1);  // the ring runs on across tiles
           issue_kb(kb);
         }
         if (!ok) break;
