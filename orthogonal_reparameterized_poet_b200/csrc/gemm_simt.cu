@@ -25,6 +25,7 @@ __device__ __forceinline__ float ld_any(const void *p, int dtype, int64_t i) {
 
 template <typename T>
 __global__ void __launch_bounds__(NT) gemm_simt_kernel(Gemm g, int splitk, int kchunk) {
+  const bool reduce = g.atomic && splitk > 1;  // partial sums added into the zeroed output
   __shared__ float As[TK][TM + 1];
   __shared__ float Bs[TK][TN + 1];
   const int tid = threadIdx.x;
@@ -82,7 +83,7 @@ __global__ void __launch_bounds__(NT) gemm_simt_kernel(Gemm g, int splitk, int k
       const int gn = n0 + tx + 16 * j;
       if (gn >= g.N) continue;
       float v = g.alpha * acc[i][j];
-      if (g.atomic) {
+      if (reduce) {
         atomicAdd(g.outF + int64_t(b) * g.of_b + int64_t(gm) * g.of_m + gn, v);
         continue;
       }
@@ -115,6 +116,7 @@ poet_status gemm_simt(const Gemm &g, cudaStream_t st) {
   if (g.K == 0) kchunk = 0;
   POET_REQUIRE(int64_t(g.batch) * splitk <= 65535 && mt <= 65535, "gemm grid too large (M=%d batch=%d)", g.M, g.batch);
   dim3 grid(nt, mt, g.batch * splitk);
+  if (g.atomic && splitk > 1) POET_TRY(zero_output(g.outF, g.M, g.N, g.of_m, g.batch, g.of_b, st));
   if (g.dtype == POET_BF16)
     gemm_simt_kernel<bf16><<<grid, NT, 0, st>>>(g, splitk, kchunk);
   else

@@ -1148,16 +1148,20 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
   }
   // Split K (atomic outputs only) into s parts.  A tile of k k-blocks takes
   // about max(k, kEpiKb) + 1 k-block times (its float reduction takes about
-  // kEpiKb, overlapped with the next tile's products), and the tiles run in
-  // ceil(tiles / workers) waves; s minimizes waves(s) * (max(kavg / s,
-  // kEpiKb) + 1), the smallest s within 1% of the best, s <= 16.  (Filling
-  // waves alone picked up to 15 splits of 2048-deep products whose every
-  // 3-k-block tile then waited on a whole tile's reduction.)
+  // kEpiKb, overlapped with the next tile's products), the tiles run in
+  // ceil(tiles / workers) waves, and each further split costs about 3.5% more
+  // (the output is zeroed and reduced into through L2: measured on the
+  // weight plan's 32768-token products, three splits ran 4% slower than one);
+  // s minimizes waves(s) * (max(kavg / s, kEpiKb) + 1) * (1 + 0.035 (s - 1)),
+  // the smallest s within 1% of the best, s <= 16.  (Filling waves alone
+  // picked up to 15 splits of 2048-deep products whose every 3-k-block tile
+  // then waited on a whole tile's reduction.)
   int split_want = 1;
   bool any_atomic = false;
   for (int i = 0; i < n; ++i) any_atomic |= gs[i].atomic;
   if (any_atomic && base_tiles > 0) {
     constexpr double kEpiKb = 6.0;
+    constexpr double kSplitCost = 0.035;  // each further split: zeroing and reducing the whole output
     const int64_t workers = num_sms() / t.cg;  // concurrent tile workers: CTAs or CTA pairs
     const double kavg = kb_sum / double(base_tiles);
     double cost[17] = {};
@@ -1165,7 +1169,7 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
     for (int sp = 1; sp <= g_splitk_max; ++sp) {
       const int64_t waves = (base_tiles * sp + workers - 1) / workers;
       const double per = kavg / sp;
-      cost[sp] = double(waves) * ((per > kEpiKb ? per : kEpiKb) + 1.0);
+      cost[sp] = double(waves) * ((per > kEpiKb ? per : kEpiKb) + 1.0) * (1.0 + kSplitCost * (sp - 1));
       if (sp == 1 || cost[sp] < best) best = cost[sp];
     }
     for (int sp = 1; sp <= g_splitk_max; ++sp)
@@ -1186,6 +1190,7 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
       return POET_ECUDA;
     }
     grp.tile_start[i + 1] = grp.tile_start[i] + int64_t(p.num_m) * p.num_n * p.splits * p.batch;
+    if (p.atomic) POET_TRY(zero_output(gi.outF, gi.M, gi.N, gi.of_m, gi.batch, gi.of_b, st));  // split: reduced into
   }
   if constexpr (MAXP == 1) {
     if (t.bstat && !t.A_MN) {

@@ -412,6 +412,23 @@ __global__ void __launch_bounds__(256) zero_many_kernel(const __grid_constant__ 
   }
 }
 
+// out[b*ldb + r*ldm + c] = 0 for b < batch, r < M, c < N; 16-byte stores where
+// rows allow.
+__global__ void __launch_bounds__(256) zero_output_kernel(float *out, int M, int N, int64_t ldm, int batch,
+                                                          int64_t ldb) {
+  const bool vec = (reinterpret_cast<uintptr_t>(out) & 15) == 0 && ldm % 4 == 0 && (batch == 1 || ldb % 4 == 0);
+  const int units = vec ? (N + 3) / 4 : N;  // 16-byte units (the last may be partial) or single columns
+  const int64_t rows = int64_t(batch) * M;
+  for (int64_t row = blockIdx.y * int64_t(blockDim.y) + threadIdx.y; row < rows; row += int64_t(gridDim.y) * blockDim.y) {
+    float *o = out + (row / M) * ldb + (row % M) * ldm;
+    for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < units; u += gridDim.x * blockDim.x) {
+      if (vec && 4 * u + 4 <= N) *reinterpret_cast<float4 *>(o + 4 * u) = make_float4(0.f, 0.f, 0.f, 0.f);
+      else if (vec) { for (int c = 4 * u; c < N; ++c) o[c] = 0.f; }
+      else o[u] = 0.f;
+    }
+  }
+}
+
 // Launches the problems of one table: the ring slot fits the widest row, as
 // many warps as shared memory allows (at most MAX_WARPS), and a grid of the
 // CTAs that can be resident at once (fewer for little work).
@@ -574,6 +591,19 @@ poet_status frame_many(const std::vector<FrameItem> &v, cudaStream_t st) {
 poet_status frame_f32_to_bf16(const float *D, int64_t ldD, const int32_t *rowmap, int64_t rows, int d,
                               const int32_t *perm, void *out, int64_t ld_out, cudaStream_t st) {
   return frame_many({FrameItem{D, ldD, rowmap, rows, d, perm, out, ld_out}}, st);
+}
+
+poet_status zero_output(float *out, int M, int N, int64_t ldm, int batch, int64_t ldb, cudaStream_t st) {
+  if (M <= 0 || N <= 0 || batch <= 0) return POET_OK;
+  const int64_t rows = int64_t(batch) * M;
+  const dim3 block(32, 8);
+  const int gx = int(((N + 3) / 4 + 31) / 32);
+  const int64_t gy_want = (rows + 7) / 8, gy_cap = int64_t(num_sms()) * 8;
+  const dim3 grid(unsigned(gx > 0 ? gx : 1), unsigned(gy_want < gy_cap ? gy_want : gy_cap));
+  TraceScope ts("zero", 0.0, double(rows) * N * 4.0, st);
+  zero_output_kernel<<<grid, block, 0, st>>>(out, M, N, ldm, batch, ldb);
+  count_launch();
+  return launch_status("zero");
 }
 
 poet_status zero_many(const std::vector<std::pair<float *, int64_t>> &v, cudaStream_t st) {

@@ -366,7 +366,7 @@ extern "C" {
 const char *poet_last_error(void) { return g_last_error; }
 
 // The kernel revisions name the code that profiles/ counters were taken on.
-const char *poet_version(void) { return "libpoet 0.4 (sm_100a; gemm_tc r19; permute r7; restride r1; cnp r6; smallb r1; block r1)"; }
+const char *poet_version(void) { return "libpoet 0.4 (sm_100a; gemm_tc r20; permute r8; restride r1; cnp r6; smallb r2; block r1)"; }
 
 size_t poet_side_state_bytes(const poet_side *side, int32_t dtype) {
   SideGeom g;
@@ -619,14 +619,12 @@ poet_status backward_weight_many(std::vector<WBwd> &v, int64_t T, cudaStream_t s
     gs.push_back(p);
   }
   POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
-  // D = dy^T x (natural order, float, split over tokens) for the layers with primitives
-  std::vector<std::pair<float *, int64_t>> zero;
+  // D = dy^T x (natural order, float, possibly split over tokens) for the layers with primitives
   gs.clear();
   for (size_t i = 0; i < v.size(); ++i) {
     WBwd &b = v[i];
     const LayerGeom &lg = b.lg;
     if (lg.R.nprim == 0 && lg.P.nprim == 0) continue;
-    zero.emplace_back(b.D, lg.m * lg.ldn);
     Gemm p;
     p.tag = "w_grad";
     p.M = int(lg.m); p.N = int(lg.n); p.K = int(T); p.dtype = dt;
@@ -637,7 +635,6 @@ poet_status backward_weight_many(std::vector<WBwd> &v, int64_t T, cudaStream_t s
     gs.push_back(p);
   }
   if (gs.empty()) return POET_OK;
-  POET_TRY(zero_many(zero, st));
   POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
   // D_f[i][j] = D[R.perm[i]][P.perm[j]] in the storage type, every layer in one launch
   if (dt == POET_BF16) {
@@ -662,8 +659,7 @@ poet_status backward_weight_many(std::vector<WBwd> &v, int64_t T, cudaStream_t s
     POET_TRY(permute_many(POET_F32, fr, st, "frame"));
   }
   // G_R[j] = D_f[rows j] F[rows j]^T,  G_P[j] = H[:, cols j]^T D_f[:, cols j]
-  // (small products: split over K and summed in place)
-  zero.clear();
+  // (small products: possibly split over K and summed in place)
   gs.clear();
   for (WBwd &b : v) {
     const LayerGeom &lg = b.lg;
@@ -671,7 +667,6 @@ poet_status backward_weight_many(std::vector<WBwd> &v, int64_t T, cudaStream_t s
     const WeightSaved ly = weight_saved(lg, T);
     const char *W0f = static_cast<const char *>(b.L->W0f);
     if (gR.nprim > 0) {  // G_R[j] = D_f[rows j] F[rows j]^T  (F = W0f when P has no primitives)
-      zero.emplace_back(b.GR, gR.all_elems());
       Gemm p;
       p.tag = "blk_grad";
       p.M = gR.size; p.N = gR.size; p.K = int(lg.n); p.batch = gR.nprim; p.dtype = dt;
@@ -683,7 +678,6 @@ poet_status backward_weight_many(std::vector<WBwd> &v, int64_t T, cudaStream_t s
       gs.push_back(p);
     }
     if (gP.nprim > 0) {  // G_P[j] = H[:, cols j]^T D_f[:, cols j]  (H = W0f when R has no primitives)
-      zero.emplace_back(b.GP, gP.all_elems());
       Gemm p;
       p.small = SMALL_GRAD;  // the sum runs over the rows
       p.tag = "blk_grad";
@@ -696,7 +690,6 @@ poet_status backward_weight_many(std::vector<WBwd> &v, int64_t T, cudaStream_t s
       gs.push_back(p);
     }
   }
-  POET_TRY(zero_many(zero, st));
   return gemm_run_many(gs.data(), int(gs.size()), st);
 }
 
@@ -789,7 +782,6 @@ static poet_status backward_token(const poet_layer *L, const LayerGeom &lg, char
   if (gR.nprim > 0) {
     POET_TRY(gemm_run(blockdiag(gR, dt, T, dyf, lg.ldm, state_R(&L->R, gR, dt), true, dvf, lg.ldm), st));
     dv = dvf;
-    POET_CUDA_TRY(cudaMemsetAsync(GR, 0, size_t(gR.all_elems()) * 4, st));
     POET_TRY(gemm_run(blockgrad(gR, dt, T, dyf, vf, lg.ldm, GR), st));
   }
   // a6: du = dv W0f
@@ -805,7 +797,6 @@ static poet_status backward_token(const poet_layer *L, const LayerGeom &lg, char
   // a7: G_P, dx = P^T du, scatter (tail straight from du)
   const void *dxsrc = duf;
   if (gP.nprim > 0) {
-    POET_CUDA_TRY(cudaMemsetAsync(GP, 0, size_t(gP.all_elems()) * 4, st));
     POET_TRY(gemm_run(blockgrad(gP, dt, T, duf, xf, lg.ldn, GP), st));
     POET_TRY(gemm_run(blockdiag(gP, dt, T, duf, lg.ldn, state_R(&L->P, gP, dt), true, dxf, lg.ldn), st));
     dxsrc = dxf;

@@ -110,8 +110,9 @@ StateLayout state_layout(const SideGeom &g, int dtype);
 //              (+ diag if i == j)
 //   A(b,i,l) = A[b*a_b + i*a_m + l*a_k], B(b,j,l) = B[b*b_b + j*b_n + l*b_k]
 // then v is stored to outF (float) and/or outD (element type `dtype`).  With
-// `atomic`, outF holds zeros on entry and the engine may split K, adding the
-// partial sums into it (or store v when it does not split).
+// `atomic` (outF only, no addend or diagonal) the engine may split K: it then
+// zeroes outF and adds the partial sums into it; outF's prior content is never
+// used.
 struct Gemm {
   int M = 0, N = 0, K = 0, batch = 1;
   int dtype = POET_F32;                       // type of A, B, outD
@@ -135,6 +136,9 @@ struct Gemm {
 enum { SMALL_RIGHT = 1, SMALL_LEFT = 2, SMALL_GRAD = 3 };
 
 poet_status gemm_run(const Gemm &g, cudaStream_t st);       // picks the engine
+// out[b*ldb + r*ldm + c] = 0 for b < batch, r < M, c < N (an output about to
+// receive reductions).
+poet_status zero_output(float *out, int M, int N, int64_t ldm, int batch, int64_t ldb, cudaStream_t st);
 poet_status gemm_simt(const Gemm &g, cudaStream_t st);      // CUDA-core FMA engine
 bool gemm_tc_supported(const Gemm &g);                      // tcgen05 engine can take g
 poet_status gemm_tc(const Gemm &g, cudaStream_t st);        // tcgen05 engine

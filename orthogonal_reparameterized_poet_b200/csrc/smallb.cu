@@ -241,6 +241,7 @@ poet_status smallb_grad(int dtype, const void *D, const void *V, int64_t ld, int
   POET_REQUIRE(smallb_supported(s) && nprim <= 65535, "smallb: primitive size %d or count %d out of range", s, nprim);
   const int64_t per = rows_per_cta(rows, nprim);
   const dim3 grid(unsigned((rows + per - 1) / per), unsigned(nprim));
+  POET_TRY(zero_output(G, s, s, ldg, nprim, gstride, st));  // the CTAs' sums are added into it
   const double elems = double(rows) * nprim * s;
   TraceScope ts("blk_grad", 2.0 * elems * s, elems * esize(dtype) * 2.0, st);
   if (dtype == POET_BF16)
