@@ -1146,23 +1146,24 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
     base_tiles += mt * nt * gs[i].batch;
     kb_sum += double(mt * nt * gs[i].batch) * double((gs[i].K + BK - 1) / BK);
   }
-  // Split K (atomic outputs only) into s parts.  A tile of k k-blocks takes
+  // Split K (atomic outputs only) into s parts, for launches of less than two
+  // full waves only: on the weight plan's launches of 4-11 waves (tiles of
+  // 16-512 k-blocks) one split beat every other.  A tile of k k-blocks takes
   // about max(k, kEpiKb) + 1 k-block times (its float reduction takes about
   // kEpiKb, overlapped with the next tile's products), the tiles run in
   // ceil(tiles / workers) waves, and each further split costs about 3.5% more
-  // (the output is zeroed and reduced into through L2: measured on the
-  // weight plan's 32768-token products, three splits ran 4% slower than one);
-  // s minimizes waves(s) * (max(kavg / s, kEpiKb) + 1) * (1 + 0.035 (s - 1)),
-  // the smallest s within 1% of the best, s <= 16.  (Filling waves alone
-  // picked up to 15 splits of 2048-deep products whose every 3-k-block tile
-  // then waited on a whole tile's reduction.)
+  // (the output is zeroed and reduced into through L2); s minimizes
+  // waves(s) * (max(kavg / s, kEpiKb) + 1) * (1 + 0.035 (s - 1)), the smallest
+  // s within 1% of the best.  (Filling waves alone picked up to 15 splits of
+  // 2048-deep products whose every 3-k-block tile then waited on a whole
+  // tile's reduction.)
   int split_want = 1;
   bool any_atomic = false;
   for (int i = 0; i < n; ++i) any_atomic |= gs[i].atomic;
-  if (any_atomic && base_tiles > 0) {
+  const int64_t workers = num_sms() / t.cg;  // concurrent tile workers: CTAs or CTA pairs
+  if (any_atomic && base_tiles > 0 && base_tiles < 2 * workers) {
     constexpr double kEpiKb = 6.0;
     constexpr double kSplitCost = 0.035;  // each further split: zeroing and reducing the whole output
-    const int64_t workers = num_sms() / t.cg;  // concurrent tile workers: CTAs or CTA pairs
     const double kavg = kb_sum / double(base_tiles);
     double cost[17] = {};
     double best = 0.0;
