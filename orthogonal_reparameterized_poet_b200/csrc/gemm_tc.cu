@@ -1176,6 +1176,7 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
     for (int sp = 1; sp <= g_splitk_max; ++sp)
       if (cost[sp] <= 1.01 * best) { split_want = sp; break; }
   }
+  std::vector<ZeroRegion> zero;  // outputs of split problems, zeroed in one launch before the products
   // problems in decreasing K order (their tiles' length; ties keep the list order)
   int order[MAXP];
   for (int i = 0; i < n; ++i) order[i] = i;
@@ -1191,8 +1192,9 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
       return POET_ECUDA;
     }
     grp.tile_start[i + 1] = grp.tile_start[i] + int64_t(p.num_m) * p.num_n * p.splits * p.batch;
-    if (p.atomic) POET_TRY(zero_output(gi.outF, gi.M, gi.N, gi.of_m, gi.batch, gi.of_b, st));  // split: reduced into
+    if (p.atomic) zero.push_back(ZeroRegion{gi.outF, gi.M, gi.N, gi.of_m, gi.batch, gi.of_b});  // split: reduced into
   }
+  if (!zero.empty()) POET_TRY(zero_outputs(zero, st));
   if constexpr (MAXP == 1) {
     if (t.bstat && !t.A_MN) {
       if (!t.B_MN) return launch<false, false, 256, MAXP, true>(grp, st);

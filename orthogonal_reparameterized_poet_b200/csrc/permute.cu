@@ -412,18 +412,23 @@ __global__ void __launch_bounds__(256) zero_many_kernel(const __grid_constant__ 
   }
 }
 
-// out[b*ldb + r*ldm + c] = 0 for b < batch, r < M, c < N; 16-byte stores where
-// rows allow.
-__global__ void __launch_bounds__(256) zero_output_kernel(float *out, int M, int N, int64_t ldm, int batch,
-                                                          int64_t ldb) {
-  const bool vec = (reinterpret_cast<uintptr_t>(out) & 15) == 0 && ldm % 4 == 0 && (batch == 1 || ldb % 4 == 0);
-  const int units = vec ? (N + 3) / 4 : N;  // 16-byte units (the last may be partial) or single columns
-  const int64_t rows = int64_t(batch) * M;
+// out_p[b*ldb + r*ldm + c] = 0 for b < batch, r < M, c < N of up to kZeroMax
+// regions p (blockIdx.z); 16-byte stores where rows allow.
+constexpr int kZeroMax = 64;
+struct ZeroTable {
+  ZeroRegion reg[kZeroMax];
+  int count;
+};
+__global__ void __launch_bounds__(256) zero_output_kernel(const __grid_constant__ ZeroTable t) {
+  const ZeroRegion &r = t.reg[blockIdx.z];
+  const bool vec = (reinterpret_cast<uintptr_t>(r.out) & 15) == 0 && r.ldm % 4 == 0 && (r.batch == 1 || r.ldb % 4 == 0);
+  const int units = vec ? (r.N + 3) / 4 : r.N;  // 16-byte units (the last may be partial) or single columns
+  const int64_t rows = int64_t(r.batch) * r.M;
   for (int64_t row = blockIdx.y * int64_t(blockDim.y) + threadIdx.y; row < rows; row += int64_t(gridDim.y) * blockDim.y) {
-    float *o = out + (row / M) * ldb + (row % M) * ldm;
+    float *o = r.out + (row / r.M) * r.ldb + (row % r.M) * r.ldm;
     for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < units; u += gridDim.x * blockDim.x) {
-      if (vec && 4 * u + 4 <= N) *reinterpret_cast<float4 *>(o + 4 * u) = make_float4(0.f, 0.f, 0.f, 0.f);
-      else if (vec) { for (int c = 4 * u; c < N; ++c) o[c] = 0.f; }
+      if (vec && 4 * u + 4 <= r.N) *reinterpret_cast<float4 *>(o + 4 * u) = make_float4(0.f, 0.f, 0.f, 0.f);
+      else if (vec) { for (int c = 4 * u; c < r.N; ++c) o[c] = 0.f; }
       else o[u] = 0.f;
     }
   }
@@ -593,17 +598,37 @@ poet_status frame_f32_to_bf16(const float *D, int64_t ldD, const int32_t *rowmap
   return frame_many({FrameItem{D, ldD, rowmap, rows, d, perm, out, ld_out}}, st);
 }
 
+poet_status zero_outputs(const std::vector<ZeroRegion> &v, cudaStream_t st) {
+  static thread_local ZeroTable t;
+  for (size_t i0 = 0; i0 < v.size(); i0 += kZeroMax) {
+    t.count = 0;
+    int nmax = 1;
+    int64_t rmax = 1;
+    double bytes = 0.0;
+    for (size_t i = i0; i < v.size() && i < i0 + kZeroMax; ++i) {
+      const ZeroRegion &r = v[i];
+      if (r.M <= 0 || r.N <= 0 || r.batch <= 0) continue;
+      t.reg[t.count++] = r;
+      nmax = r.N > nmax ? r.N : nmax;
+      const int64_t rows = int64_t(r.batch) * r.M;
+      rmax = rows > rmax ? rows : rmax;
+      bytes += double(rows) * r.N * 4.0;
+    }
+    if (t.count == 0) continue;
+    const dim3 block(32, 8);
+    const int64_t gy_want = (rmax + 7) / 8, gy_cap = int64_t(num_sms()) * 8 / t.count + 1;
+    const dim3 grid(unsigned(((nmax + 3) / 4 + 31) / 32), unsigned(gy_want < gy_cap ? gy_want : gy_cap),
+                    unsigned(t.count));
+    TraceScope ts("zero", 0.0, bytes, st);
+    zero_output_kernel<<<grid, block, 0, st>>>(t);
+    count_launch();
+    POET_TRY(launch_status("zero"));
+  }
+  return POET_OK;
+}
+
 poet_status zero_output(float *out, int M, int N, int64_t ldm, int batch, int64_t ldb, cudaStream_t st) {
-  if (M <= 0 || N <= 0 || batch <= 0) return POET_OK;
-  const int64_t rows = int64_t(batch) * M;
-  const dim3 block(32, 8);
-  const int gx = int(((N + 3) / 4 + 31) / 32);
-  const int64_t gy_want = (rows + 7) / 8, gy_cap = int64_t(num_sms()) * 8;
-  const dim3 grid(unsigned(gx > 0 ? gx : 1), unsigned(gy_want < gy_cap ? gy_want : gy_cap));
-  TraceScope ts("zero", 0.0, double(rows) * N * 4.0, st);
-  zero_output_kernel<<<grid, block, 0, st>>>(out, M, N, ldm, batch, ldb);
-  count_launch();
-  return launch_status("zero");
+  return zero_outputs({ZeroRegion{out, M, N, ldm, batch, ldb}}, st);
 }
 
 poet_status zero_many(const std::vector<std::pair<float *, int64_t>> &v, cudaStream_t st) {

@@ -139,6 +139,10 @@ poet_status gemm_run(const Gemm &g, cudaStream_t st);       // picks the engine
 // out[b*ldb + r*ldm + c] = 0 for b < batch, r < M, c < N (an output about to
 // receive reductions).
 poet_status zero_output(float *out, int M, int N, int64_t ldm, int batch, int64_t ldb, cudaStream_t st);
+struct ZeroRegion {
+  float *out; int M, N; int64_t ldm; int batch; int64_t ldb;
+};
+poet_status zero_outputs(const std::vector<ZeroRegion> &v, cudaStream_t st);  // many regions, one launch
 poet_status gemm_simt(const Gemm &g, cudaStream_t st);      // CUDA-core FMA engine
 bool gemm_tc_supported(const Gemm &g);                      // tcgen05 engine can take g
 poet_status gemm_tc(const Gemm &g, cudaStream_t st);        // tcgen05 engine
