@@ -48,8 +48,8 @@ PLAN_NAMES = {1: "token", 2: "weight"}
 
 # DRAM traffic / algorithmic bytes of one launch, from an ncu capture, with the
 # kernel revision (as named in poet_version()) the counters were taken on.
-NCU_TRAFFIC_RATIO = {"w0_fwd": (1.018, "gemm_tc r16;"), "w0_bwd": (1.034, "gemm_tc r16;"),
-                     "w_grad": (2.808, "gemm_tc r16;")}
+NCU_TRAFFIC_RATIO = {"w0_fwd": (0.999, "gemm_tc r22;"), "w0_bwd": (1.025, "gemm_tc r22;"),
+                     "w_grad": (1.273, "gemm_tc r22;")}
 NCU_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the grouped launch of one LLaMA-1.3B "
                       "layer at 16384 tokens (profiles/w0_gemm_llama1.3b_layer_T16384.md), as a ratio to the "
                       "algorithmic bytes of that launch, scaled to this run's launches")
