@@ -808,18 +808,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
           }
         }
       } else if (p.coalesced == 2) {
-        // fp32 output: each 32-column chunk (128 B per row) goes row-wise into
-        // this warp's staging rows, then out four rows x 128 B at a time; a
-        // float addend (aligned rows) is read four rows x 128 B at a time too,
-        // all eight of a thread's quads before any store
+        // plain fp32 output: each 32-column chunk (128 B per row) goes row-wise
+        // into this warp's staging rows, then out four rows x 128 B at a time
         unsigned char *ew = epi + quarter * (32 * S::EPI_ROW);
         const int m_base = mrow0 + quarter * 32;
         float *obase = p.outF + int64_t(c.b) * p.of_b;
         const int sub = lane & 7, rsub = lane >> 3;
         unsigned char *myrow = ew + lane * S::EPI_ROW;
-        const float *abase = p.add ? static_cast<const float *>(p.add) + int64_t(c.b) * p.add_b +
-                                         int64_t(m_base + rsub) * p.add_m + sub * 4
-                                   : nullptr;
         for (int cc = 0; cc < BN / 32; ++cc) {
           uint32_t r[32];
           __syncwarp();
@@ -837,35 +832,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
             *reinterpret_cast<float4 *>(myrow + q * 16) = f;
           }
           __syncwarp();
-          float4 qa[8];
-          if (abase) {
-#pragma unroll
-            for (int it = 0; it < 8; ++it) {
-              const int gm = m_base + it * 4 + rsub, gn = gn0 + sub * 4;
-              qa[it] = make_float4(0.f, 0.f, 0.f, 0.f);
-              if (gm < p.M && gn + 4 <= p.N) {
-                qa[it] = *reinterpret_cast<const float4 *>(abase + int64_t(it * 4) * p.add_m + gn0);
-              } else if (gm < p.M && gn < p.N) {
-                const float *a = abase + int64_t(it * 4) * p.add_m + gn0;
-                qa[it].x = a[0];
-                if (gn + 1 < p.N) qa[it].y = a[1];
-                if (gn + 2 < p.N) qa[it].z = a[2];
-              }
-            }
-          }
 #pragma unroll
           for (int it = 0; it < 8; ++it) {
             const int rr = it * 4 + rsub;
             const int gm = m_base + rr;
             const int gn = gn0 + sub * 4;
-            float4 f = *reinterpret_cast<const float4 *>(ew + rr * S::EPI_ROW + sub * 16);
-            if (abase) {
-              f.x += beta * qa[it].x; f.y += beta * qa[it].y; f.z += beta * qa[it].z; f.w += beta * qa[it].w;
-            }
-            if (diag != 0.f && gm >= gn && gm < gn + 4) {
-              const int e = gm - gn;
-              if (e == 0) f.x += diag; else if (e == 1) f.y += diag; else if (e == 2) f.z += diag; else f.w += diag;
-            }
+            const float4 f = *reinterpret_cast<const float4 *>(ew + rr * S::EPI_ROW + sub * 16);
             if (gm < p.M && gn < p.N) {
               float *o = obase + int64_t(gm) * p.of_m + gn;
               if (p.atomic) {  // split-K: float reductions at L2, four rows x 128 B per instruction
@@ -1046,13 +1018,6 @@ const int g_splitk_max = [] {
   return v < 1 ? 1 : (v > 16 ? 16 : v);
 }();
 
-// POET_GEMM_STAGED_ADD=1: products with a float addend and float output take
-// the staged fp32 epilogue instead of the per-row path.
-const bool g_staged_add = [] {
-  const char *e = std::getenv("POET_GEMM_STAGED_ADD");
-  return e && e[0] == '1';
-}();
-
 // Operand majors and tile width of a supported problem.
 struct TcPlan {
   bool A_MN, B_MN;
@@ -1112,12 +1077,9 @@ bool fill_problem(const Gemm &g, const TcPlan &t, int split_want, TcProblem *p, 
     p->coalesced = aligned16(g.outD) && g.od_m % 8 == 0 && (g.batch == 1 || g.od_b % 8 == 0) ? 1 : 3;
     if (t.bstat && p->coalesced == 3) p->coalesced = 0;  // the B-stationary kernels stage aligned rows only
   }
-  // fp32: plain stores or split-K reductions, or (POET_GEMM_STAGED_ADD=1) a
-  // float addend and a diagonal with aligned rows
-  const bool f32_out = g.outF && !g.outD && aligned16(g.outF) && g.of_m % 4 == 0 && (g.batch == 1 || g.of_b % 4 == 0);
-  if (f32_out && !g.add && !g.add2 && g.diag == 0.f) p->coalesced = 2;
-  if (g_staged_add && f32_out && !g.atomic && !g.add2 && g.add && g.add_dtype == POET_F32 && aligned16(g.add) &&
-      g.add_m % 4 == 0 && (g.batch == 1 || g.add_b % 4 == 0))
+  // fp32: plain stores or split-K reductions
+  if (!g.add && !g.add2 && g.diag == 0.f && g.outF && !g.outD && aligned16(g.outF) && g.of_m % 4 == 0 &&
+      (g.batch == 1 || g.of_b % 4 == 0))
     p->coalesced = 2;
   bool ok;
   if (!t.A_MN) ok = make_map(ma, g.A, g.K, g.M, g.batch, g.a_m, g.a_b, 64, BM);
