@@ -257,10 +257,10 @@ struct TilePair {
 __device__ __forceinline__ TilePair tile_pair(const SideTable &t, int i, int span) {
   const int tiles = (span + PACK_T - 1) / PACK_T;
   const int pairs = tiles * (tiles + 1) / 2;
-  const int64_t local = int64_t(blockIdx.x) - t.block_start[i];
+  const int local = int(int64_t(blockIdx.x) - t.block_start[i]);  // 32-bit division below
   TilePair p;
-  p.j = int(local / pairs);
-  const int r = int(local % pairs);
+  p.j = local / pairs;
+  const int r = local - p.j * pairs;
   // row ta starts at start(ta) = ta * tiles - ta (ta - 1) / 2
   const float b = 2.f * float(tiles) + 1.f;
   int ta = int(0.5f * (b - sqrtf(fmaxf(b * b - 8.f * float(r), 0.f))));
