@@ -70,7 +70,6 @@ struct TcGroup {
   TcProblem prob[MAXP];
   int64_t tile_start[MAXP + 1];
   int count;
-  int prefetch_add;  // per-row epilogue: prefetch the next chunk's addends into L1
   unsigned *errword;
 };
 
@@ -405,10 +404,6 @@ __device__ __forceinline__ void add_row(const void *add, int f32, int64_t off, f
         if (j < nvalid) v[j] += beta * bf16_bits_to_float(a[j]);
     }
   }
-}
-
-__device__ __forceinline__ void prefetch_l1(const void *p) {
-  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
 
 // out[0..3] += (a, b, c, d) as one 16-byte reduction at L2
@@ -868,13 +863,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
         uint32_t r[32];
         __syncwarp();
         tmem_ld32(tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN + cc * 32), r);
-        const int gn0 = c.nt * BN + cc * 32;
-        if (g.prefetch_add && row_ok && gn0 + 32 < p.N && cc + 1 < BN / 32) {
-          // the next chunk's addend bytes of this row, on their way to L1 while this chunk is finished
-          if (p.add) prefetch_l1(static_cast<const char *>(p.add) + (int64_t(c.b) * p.add_b + int64_t(gm) * p.add_m + gn0 + 32) * (p.add_f32 ? 4 : 2));
-          if (p.add2) prefetch_l1(static_cast<const char *>(p.add2) + (int64_t(c.b) * p.add2_b + int64_t(gm) * p.add2_m + gn0 + 32) * (p.add2_f32 ? 4 : 2));
-        }
         tmem_ld_wait();
+        const int gn0 = c.nt * BN + cc * 32;
         if (!row_ok || gn0 >= p.N) continue;
         const int nvalid = min(32, p.N - gn0);
         if (p.atomic) {
@@ -1026,13 +1016,6 @@ const int g_splitk_max = [] {
   const char *e = std::getenv("POET_GEMM_SPLITK_MAX");
   const int v = e ? std::atoi(e) : 16;
   return v < 1 ? 1 : (v > 16 ? 16 : v);
-}();
-
-// POET_GEMM_PREFETCH_ADD=1: the per-row epilogue prefetches the next chunk's
-// addend bytes into L1.
-const int g_prefetch_add = [] {
-  const char *e = std::getenv("POET_GEMM_PREFETCH_ADD");
-  return e && e[0] == '1' ? 1 : 0;
 }();
 
 // Operand majors and tile width of a supported problem.
@@ -1199,7 +1182,6 @@ poet_status run_group(const Gemm *gs, int n, const TcPlan &t, cudaStream_t st) {
   for (int i = 0; i < n; ++i) order[i] = i;
   std::stable_sort(order, order + n, [&](int a, int b) { return gs[a].K > gs[b].K; });
   grp.count = n;
-  grp.prefetch_add = g_prefetch_add;
   grp.errword = device_errword();
   grp.tile_start[0] = 0;
   for (int i = 0; i < n; ++i) {
