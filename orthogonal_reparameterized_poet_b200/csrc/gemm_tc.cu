@@ -1018,6 +1018,13 @@ const int g_splitk_max = [] {
   return v < 1 ? 1 : (v > 16 ? 16 : v);
 }();
 
+// POET_GEMM_BSTAT=0 turns the B-stationary kernels off (such problems stream
+// both operands).
+const bool g_bstat = [] {
+  const char *e = std::getenv("POET_GEMM_BSTAT");
+  return !(e && e[0] == '0');
+}();
+
 // Operand majors and tile width of a supported problem.
 struct TcPlan {
   bool A_MN, B_MN;
@@ -1036,7 +1043,7 @@ TcPlan plan_of(const Gemm &g) {
   // token-streaming products against a small operand (block-diagonal passes
   // with 256-wide blocks): keep B resident when it fits and many M tiles
   // share it
-  t.bstat = t.BN == 256 && g.N <= 256 && g.K <= KB_MAX * BK && g.M >= 8 * BM && !g.atomic;
+  t.bstat = g_bstat && t.BN == 256 && g.N <= 256 && g.K <= KB_MAX * BK && g.M >= 8 * BM && !g.atomic;
   return t;
 }
 
