@@ -464,7 +464,8 @@ poet_status poet_cayley_neumann_grad(const poet_side *side, int32_t dtype, const
 // products read whole rows of F and whole columns of H, so H's leftover rows
 // and F's leftover columns are copied from W0f once (one grouped launch):
 // reading them from W0f in place would split each product's K range into two
-// problems, doubling its split-K float reductions, which costs more.
+// problems summed into one output, i.e. float reductions where one plain store
+// suffices.
 
 namespace {
 
@@ -619,7 +620,7 @@ poet_status backward_weight_many(std::vector<WBwd> &v, int64_t T, cudaStream_t s
     gs.push_back(p);
   }
   POET_TRY(gemm_run_many(gs.data(), int(gs.size()), st));
-  // D = dy^T x (natural order, float, possibly split over tokens) for the layers with primitives
+  // D = dy^T x (natural order, float) for the layers with primitives
   gs.clear();
   for (size_t i = 0; i < v.size(); ++i) {
     WBwd &b = v[i];
@@ -659,7 +660,7 @@ poet_status backward_weight_many(std::vector<WBwd> &v, int64_t T, cudaStream_t s
     POET_TRY(permute_many(POET_F32, fr, st, "frame"));
   }
   // G_R[j] = D_f[rows j] F[rows j]^T,  G_P[j] = H[:, cols j]^T D_f[:, cols j]
-  // (small products: possibly split over K and summed in place)
+  // (the engine splits K only for launches of less than two waves)
   gs.clear();
   for (WBwd &b : v) {
     const LayerGeom &lg = b.lg;
