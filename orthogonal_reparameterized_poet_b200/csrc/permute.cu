@@ -323,12 +323,11 @@ __global__ void __launch_bounds__(256) restride_kernel(const unsigned char *__re
 
 // out[a][c] = bf16(D[rowmap[a]][perm[c]]): a float matrix gathered into the
 // frame and rounded in one pass, for up to kFrameMax matrices per launch
-// (matrix p owns the global rows [row_start[p], row_start[p+1])).  CTA c
-// works through the contiguous global rows [total*c/G, total*(c+1)/G) with two
-// row slots in shared memory: the next row's 16-byte cp.async copies are in
-// flight while the current row is gathered (perm read through L1) and stored.
-// An index out of range (rowmap outside [0, rows), perm outside [0, d)) is not
-// read: its output is 0 and ERR_BOUNDS is set in the status word.
+// (matrix p owns the global rows [row_start[p], row_start[p+1])).  One block
+// per output row at a time; the source row is read through L1 (it is reused
+// by the block's gathers).  An index out of range (rowmap outside [0, rows),
+// perm outside [0, d)) is not read: its output is 0 and ERR_BOUNDS is set in
+// the status word.
 constexpr int kFrameMax = 64;
 struct FrameGroup {
   const float *D[kFrameMax];
@@ -341,83 +340,53 @@ struct FrameGroup {
   int d[kFrameMax];
   int64_t row_start[kFrameMax + 1];
   int count;
-  int slot;  // floats per row slot (a multiple of 4 >= the widest d)
   unsigned *errword;
 };
 static_assert(sizeof(FrameGroup) <= 32000, "frame table exceeds the kernel parameter limit");
 
 __global__ void __launch_bounds__(256) frame_f32_to_bf16_kernel(const __grid_constant__ FrameGroup g) {
-  extern __shared__ __align__(16) float slots[];
+  // a row of D is staged in shared memory with 16-byte copies (coalesced), then
+  // gathered from there; rows whose start is not 16-byte aligned are gathered
+  // from global memory directly
+  extern __shared__ __align__(16) float srow[];
   bool bad = false;
   const int64_t total = g.row_start[g.count];
-  const int64_t r0 = total * blockIdx.x / gridDim.x, r1 = total * (blockIdx.x + 1) / gridDim.x;
-  // matrix, row and source of global row gr (rows are visited in increasing order)
-  struct Row {
-    int p;
-    int64_t a;
-    const float *src;  // nullptr: the row-map entry is out of range
-  };
-  int pscan = 0;
-  auto locate = [&](int64_t gr) {
-    while (g.row_start[pscan + 1] <= gr) ++pscan;
-    Row r;
-    r.p = pscan;
-    r.a = gr - g.row_start[pscan];
-    const int64_t sr = __ldg(g.rowmap[pscan] + r.a);
-    r.src = sr >= 0 && sr < g.rows[pscan] ? g.D[pscan] + sr * g.ldD[pscan] : nullptr;
-    return r;
-  };
-  auto issue = [&](const Row &r, float *slot) {
-    const int d = g.d[r.p];
-    if (r.src) {
-      if ((reinterpret_cast<uintptr_t>(r.src) & 15) == 0) {
-        const int units = d / 4;
-        for (int u = threadIdx.x; u < units; u += blockDim.x) cp_async16(slot + 4 * u, r.src + 4 * u);
-        for (int c = 4 * units + threadIdx.x; c < d; c += blockDim.x) slot[c] = r.src[c];
-      } else {
-        for (int c = threadIdx.x; c < d; c += blockDim.x) slot[c] = r.src[c];
-      }
-    }
-    cp_async_commit();
-  };
-  Row cur{}, nxt{};
-  if (r0 < r1) {
-    cur = locate(r0);
-    issue(cur, slots);
-  }
-  for (int64_t gr = r0; gr < r1; ++gr) {
-    float *cs = slots + int64_t((gr - r0) & 1) * g.slot;
-    if (gr + 1 < r1) {
-      nxt = locate(gr + 1);
-      issue(nxt, slots + int64_t(((gr - r0) & 1) ^ 1) * g.slot);
-    } else {
-      cp_async_commit();
-    }
-    cp_async_wait_one();  // this thread's copies of row gr have landed
-    __syncthreads();      // everyone's
-    const int d = g.d[cur.p];
-    const int32_t *perm = g.perm[cur.p];
-    const bool row_ok = cur.src != nullptr;
+  int p = 0;
+  for (int64_t gr = blockIdx.x; gr < total; gr += gridDim.x) {
+    while (g.row_start[p + 1] <= gr) ++p;  // rows are visited in increasing order
+    const int64_t a = gr - g.row_start[p], rows = g.rows[p];
+    const int d = g.d[p];
+    const int32_t *perm = g.perm[p];
+    const int64_t sr = __ldg(g.rowmap[p] + a);
+    const bool row_ok = sr >= 0 && sr < rows;
     bad |= !row_ok;
-    bf16 *orow = g.out[cur.p] + cur.a * g.ld_out[cur.p];
+    const float *src = g.D[p] + (row_ok ? sr : 0) * g.ldD[p];
+    const bool staged = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+    if (staged) {
+      __syncthreads();  // the previous row's readers of srow are done
+      const int units = d / 4;
+      for (int u = threadIdx.x; u < units; u += blockDim.x) cp_async16(srow + 4 * u, src + 4 * u);
+      for (int c = 4 * units + threadIdx.x; c < d; c += blockDim.x) srow[c] = src[c];
+      cp_async_wait_all();
+      __syncthreads();
+    }
+    bf16 *orow = g.out[p] + a * g.ld_out[p];
     for (int c = 2 * threadIdx.x; c < d; c += 2 * blockDim.x) {
       if (c + 1 < d) {
         const int2 pc = *reinterpret_cast<const int2 *>(perm + c);
         const bool okx = row_ok && unsigned(pc.x) < unsigned(d), oky = row_ok && unsigned(pc.y) < unsigned(d);
         bad |= !(okx && oky);
-        *reinterpret_cast<__nv_bfloat162 *>(orow + c) =
-            __floats2bfloat162_rn(okx ? cs[pc.x] : 0.f, oky ? cs[pc.y] : 0.f);
+        const float vx = okx ? (staged ? srow[pc.x] : __ldg(src + pc.x)) : 0.f;
+        const float vy = oky ? (staged ? srow[pc.y] : __ldg(src + pc.y)) : 0.f;
+        *reinterpret_cast<__nv_bfloat162 *>(orow + c) = __floats2bfloat162_rn(vx, vy);
       } else {
         const int pc = perm[c];
         const bool ok = row_ok && unsigned(pc) < unsigned(d);
         bad |= !ok;
-        orow[c] = __float2bfloat16_rn(ok ? cs[pc] : 0.f);
+        orow[c] = __float2bfloat16_rn(ok ? (staged ? srow[pc] : __ldg(src + pc)) : 0.f);
       }
     }
-    __syncthreads();  // row gr's readers are done before its slot is refilled
-    cur = nxt;
   }
-  cp_async_wait_all();
   if (bad && g.errword) atomicOr(g.errword, ERR_BOUNDS);
 }
 
@@ -600,8 +569,7 @@ poet_status frame_many(const std::vector<FrameItem> &v, cudaStream_t st) {
     grp.errword = device_errword();
     int dmax = 0;
     for (int q = 0; q < grp.count; ++q) dmax = grp.d[q] > dmax ? grp.d[q] : dmax;
-    grp.slot = int(round_up(dmax, 4));
-    const size_t smem = 2 * size_t(grp.slot) * 4;  // two row slots of the widest matrix
+    const size_t smem = size_t(dmax) * 4;  // one staged row of the widest matrix
     POET_REQUIRE(smem <= 200 * 1024, "frame: rows of %d floats do not fit in shared memory", dmax);
     static int configured[64] = {};
     int dev = 0;
