@@ -319,23 +319,35 @@ class Variant:
             L.resample()
 
 
-def kernel_table(rows, steps):
-    """Per trace kind: launches, ms per step, share, and the fraction of the
-    roofline that bounds it (tensor when its flop/byte is above the ridge of
-    the measured peaks, HBM otherwise)."""
+def trace_on(poet):
+    """Start the library's per-kind event trace, with the ridge of the measured
+    peaks splitting launches into tensor- and HBM-bound ones."""
     peaks = load_peaks()
-    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    poet.poet_trace_set_ridge(peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9))
+    poet.poet_trace_enable(True)
+
+
+def kernel_table(rows, steps):
+    """Per trace kind: launches, ms per step, share, achieved TFLOP/s and GB/s,
+    and the fraction of its roofline.  Every launch is held to its own bound:
+    the library sums the flops of the launches whose flop/byte is at or above
+    the ridge of the measured peaks (flop_tc) and the bytes of the others
+    (bytes_hbm), so the roofline time is flop_tc / tensor peak + bytes_hbm /
+    copy peak and frac = that time over the measured one.  `bound` names the
+    larger of the two terms."""
+    peaks = load_peaks()
+    pt, ph = peaks["bf16_tflops_sustained"] * 1e12, peaks["hbm_gbs"] * 1e9
     total = sum(x["ms"] for x in rows.values()) or 1.0
     out = {}
     for k, r in sorted(rows.items(), key=lambda kv: -kv[1]["ms"]):
         sec = r["ms"] / 1e3
         tf = r["flop"] / sec / 1e12 if sec and r["flop"] else None
         gb = r["bytes"] / sec / 1e9 if sec else None
-        tensor = r["flop"] and r["bytes"] and r["flop"] / r["bytes"] >= ridge
-        frac = (tf / peaks["bf16_tflops_sustained"]) if tensor else (gb / peaks["hbm_gbs"] if gb else None)
+        t_tc, t_hbm = r.get("flop_tc", 0.0) / pt, r.get("bytes_hbm", 0.0) / ph
+        frac = (t_tc + t_hbm) / sec if sec and (t_tc or t_hbm) else None
         out[k] = {"launches": r["launches"], "ms_per_step": round(r["ms"] / steps, 3), "share": round(r["ms"] / total, 4),
                   "tflops": round(tf, 1) if tf else None, "gbs": round(gb, 1) if gb else None,
-                  "bound": "tensor" if tensor else "hbm", "frac": round(frac, 4) if frac is not None else None}
+                  "bound": "tensor" if t_tc >= t_hbm else "hbm", "frac": round(frac, 4) if frac is not None else None}
     return out
 
 
@@ -404,7 +416,7 @@ def measure_workload(name, args, device, rank, plan, overrides=None):
     for _ in range(max(args.warmup, 1)):
         v.step()
     poet.poet_sync_status()
-    poet.poet_trace_enable(True)
+    trace_on(poet)
     for _ in range(args.steps):
         v.step()
     trace = poet.poet_trace_read()
@@ -498,7 +510,7 @@ def measure_block(name, args, device):
     for _ in range(max(args.warmup, 1)):
         step()
     poet.poet_sync_status()
-    poet.poet_trace_enable(True)
+    trace_on(poet)
     for _ in range(args.steps):
         step()
     rows = poet.poet_trace_read()
@@ -595,7 +607,7 @@ def run_poet(args):
         torch.cuda.synchronize()
         if clocks:
             clocks.start()
-        poet.poet_trace_enable(True)
+        trace_on(poet)
         launches0 = poet.poet_launch_count()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
@@ -618,7 +630,8 @@ def run_poet(args):
         trace = {}
         for tr in traces:
             for k, r in tr.items():
-                a = trace.setdefault(k, {"launches": 0, "ms": 0.0, "flop": 0.0, "bytes": 0.0})
+                a = trace.setdefault(k, {"launches": 0, "ms": 0.0, "flop": 0.0, "bytes": 0.0, "flop_tc": 0.0,
+                                         "bytes_hbm": 0.0})
                 for f in a:
                     a[f] += r[f]
         poet.poet_sync_status()

@@ -440,13 +440,19 @@ POET_API int32_t poet_gemm_engine(int32_t dtype);
 /* ---------------------------------------------------------------- accounting */
 
 /* One kind of work with its recorded launches, CUDA-event time and
- * algorithmic flops / bytes (the operation's own operand sizes, not counters). */
+ * algorithmic flops / bytes (the operation's own operand sizes, not counters).
+ * flop_tc sums the flops of the launches whose flop / byte ratio is at or
+ * above the ridge set by poet_trace_set_ridge, bytes_hbm the bytes of the
+ * others, so that flop_tc / (tensor peak) + bytes_hbm / (copy peak) is the
+ * kind's roofline time with every launch held to its own bound. */
 typedef struct {
   char kind[32];
   int64_t launches;
   double ms;
   double flop;
   double bytes;
+  double flop_tc;
+  double bytes_hbm;
 } poet_trace_row;
 
 /* Kernels this library has launched since it was loaded (all devices). */
@@ -456,6 +462,10 @@ POET_API int64_t poet_launch_count(void);
  * around each unit of work, tagged by kind.  Recording adds host calls
  * between launches but no device work. */
 POET_API poet_status poet_trace_enable(int32_t on);
+
+/* The flop / byte ratio that splits launches into flop_tc and bytes_hbm
+ * (the tensor peak over the copy peak; 216 until set).  EINVAL unless > 0. */
+POET_API poet_status poet_trace_set_ridge(double flop_per_byte);
 
 /* Wait for the recorded events, aggregate them by kind into rows (at most
  * max_rows, sorted by kind), forget them, and return the rows written. */

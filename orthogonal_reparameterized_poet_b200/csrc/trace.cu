@@ -15,6 +15,7 @@ namespace {
 
 std::atomic<long long> g_launches{0};
 std::atomic<bool> g_trace{false};
+std::atomic<double> g_ridge{216.0};  // flop per byte: measured bf16 peak over copy peak
 
 struct Rec {
   std::string kind;
@@ -77,9 +78,16 @@ poet_status poet_trace_enable(int32_t on) {
   return POET_OK;
 }
 
+poet_status poet_trace_set_ridge(double flop_per_byte) {
+  POET_REQUIRE(flop_per_byte > 0.0, "poet_trace_set_ridge: ridge %g must be positive", flop_per_byte);
+  g_ridge.store(flop_per_byte);
+  return POET_OK;
+}
+
 int32_t poet_trace_read(poet_trace_row *rows, int32_t max_rows) {
   std::lock_guard<std::mutex> lock(g_mu);
   std::map<std::string, poet_trace_row> agg;
+  const double ridge = g_ridge.load();
   for (auto &r : g_recs) {
     float ms = 0.f;
     if (cudaEventSynchronize(r.e1) == cudaSuccess) cudaEventElapsedTime(&ms, r.e0, r.e1);
@@ -88,6 +96,10 @@ int32_t poet_trace_read(poet_trace_row *rows, int32_t max_rows) {
     a.ms += ms;
     a.flop += r.flop;
     a.bytes += r.bytes;
+    if (r.flop > 0.0 && r.flop >= ridge * r.bytes)
+      a.flop_tc += r.flop;
+    else
+      a.bytes_hbm += r.bytes;
     g_pool.push_back(r.e0);
     g_pool.push_back(r.e1);
   }

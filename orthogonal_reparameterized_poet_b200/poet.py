@@ -51,7 +51,8 @@ class poet_adamw_hparams(ctypes.Structure):
 
 class poet_trace_row(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_char * 32), ("launches", ctypes.c_int64), ("ms", ctypes.c_double),
-                ("flop", ctypes.c_double), ("bytes", ctypes.c_double)]
+                ("flop", ctypes.c_double), ("bytes", ctypes.c_double), ("flop_tc", ctypes.c_double),
+                ("bytes_hbm", ctypes.c_double)]
 
 
 _SIGS = {
@@ -129,6 +130,7 @@ _SIGS = {
     "poet_launch_count": (ctypes.c_int64, []),
     "poet_trace_enable": (ctypes.c_int, [ctypes.c_int32]),
     "poet_trace_read": (ctypes.c_int32, [ctypes.POINTER(poet_trace_row), ctypes.c_int32]),
+    "poet_trace_set_ridge": (ctypes.c_int, [ctypes.c_double]),
     "poet_last_error": (ctypes.c_char_p, []),
     "poet_version": (ctypes.c_char_p, []),
 }
@@ -314,12 +316,19 @@ def poet_trace_enable(on: bool):
     _check(lib().poet_trace_enable(1 if on else 0))
 
 
+def poet_trace_set_ridge(flop_per_byte: float):
+    _check(lib().poet_trace_set_ridge(float(flop_per_byte)))
+
+
 def poet_trace_read() -> dict:
-    """{kind: {"launches", "ms", "flop", "bytes"}} of the work recorded since tracing was enabled."""
+    """{kind: {"launches", "ms", "flop", "bytes", "flop_tc", "bytes_hbm"}} of the work recorded since
+    tracing was enabled (flop_tc / bytes_hbm: the flops of the launches at or above the ridge, the
+    bytes of the others)."""
     rows = (poet_trace_row * 64)()
     n = lib().poet_trace_read(rows, 64)
     return {rows[i].kind.decode(): {"launches": rows[i].launches, "ms": rows[i].ms, "flop": rows[i].flop,
-                                    "bytes": rows[i].bytes} for i in range(n)}
+                                    "bytes": rows[i].bytes, "flop_tc": rows[i].flop_tc,
+                                    "bytes_hbm": rows[i].bytes_hbm} for i in range(n)}
 
 
 def poet_version() -> str:

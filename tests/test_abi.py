@@ -120,6 +120,9 @@ def test_host_validation_rejects_bad_arguments():
     bad.P.dim = 256
     assert lib.poet_merge(ctypes.byref(bad), None, 0, st) == poet.EINVAL
     assert lib.poet_gemm(7, 1, 1, 1, 1, None, 0, 0, 0, None, 0, 0, 0, None, 1, 0, 1.0, 0.0, st) == poet.EINVAL
+    assert lib.poet_trace_set_ridge(0.0) == poet.EINVAL
+    assert lib.poet_trace_set_ridge(-5.0) == poet.EINVAL
+    assert lib.poet_trace_set_ridge(216.0) == poet.OK
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

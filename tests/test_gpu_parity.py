@@ -251,6 +251,39 @@ def test_tensor_core_engine_is_live(cuda):
     assert poet.poet_gemm_engine(I.F32) == 0
 
 
+def test_trace_splits_launches_at_the_ridge(cuda):
+    """The per-kind trace holds each launch to its own bound: a K = 4096 bf16
+    product (about 1000 flop per byte) lands in flop_tc, the AdamW pass (no
+    flops) in bytes_hbm, and a ridge above every launch moves the product's
+    bytes to bytes_hbm."""
+    from orthogonal_reparameterized_poet_b200 import poet
+
+    M = N = 512
+    K = 4096
+    A = cuda.randn(M, K, device="cuda").to(cuda.bfloat16)
+    B = cuda.randn(N, K, device="cuda").to(cuda.bfloat16)
+    C = cuda.empty(M, N, device="cuda", dtype=cuda.bfloat16)
+    theta, grad, m, v = (cuda.zeros(4096, device="cuda") for _ in range(4))
+    try:
+        poet.poet_trace_set_ridge(216.0)
+        poet.poet_trace_enable(True)
+        poet.poet_gemm(I.BF16, M, N, K, 1, A, (K, 1, M * K), B, (K, 1, N * K), C, N, M * N)
+        poet.poet_adamw_step(theta, grad, m, v, 1e-3)
+        rows = poet.poet_trace_read()
+        poet.poet_trace_set_ridge(1e9)
+        poet.poet_gemm(I.BF16, M, N, K, 1, A, (K, 1, M * K), B, (K, 1, N * K), C, N, M * N)
+        high = poet.poet_trace_read()
+    finally:
+        poet.poet_trace_enable(False)
+        poet.poet_trace_set_ridge(216.0)
+    poet.poet_sync_status()
+    g, a, h = rows["gemm"], rows["adamw"], high["gemm"]
+    assert g["launches"] == 1 and g["flop"] == 2.0 * M * N * K and g["flop_tc"] == g["flop"] and g["bytes_hbm"] == 0
+    assert a["flop"] == 0 and a["flop_tc"] == 0 and a["bytes_hbm"] == a["bytes"] > 0
+    assert h["flop_tc"] == 0 and h["bytes_hbm"] == h["bytes"] == g["bytes"] > 0
+    assert g["ms"] > 0 and a["ms"] > 0
+
+
 @pytest.mark.parametrize("dtype,M,N,K,batch,amaj,bmaj,alpha,beta", GEMM_CASES)
 def test_gemm_engine(cuda, dtype, M, N, K, batch, amaj, bmaj, alpha, beta):
     from orthogonal_reparameterized_poet_b200 import poet
