@@ -184,7 +184,6 @@ __global__ void __launch_bounds__(SB_WARPS * 32) smallb_grad_kernel(const T *__r
   }
 }
 
-// Row ranges per block for about four CTAs per SM over all blocks (at least 64 rows each).
 // right for bf16 blocks of 16 or 32 on the tensor cores: mma.sync
 // m16n8k16 (bf16 in, float accumulate), which takes the s multiply-adds per
 // output off the CUDA cores (the CUDA-core kernel above is bound by them and
@@ -264,6 +263,109 @@ __global__ void __launch_bounds__(SB_WARPS * 32) smallb_right_mma_kernel(const b
   }
 }
 
+// grad for bf16 blocks of 16 or 32 on the tensor cores: G_j = D_j^T V_j is a
+// product over the rows, and both operands hold the rows as their strided
+// dimension, so each warp stages 32 rows of D_j and V_j in its own shared
+// memory (rows padded to S + 8 elements: eight 16-byte row segments of an
+// ldmatrix then fall on distinct banks) and takes the fragments with
+// ldmatrix.trans, which hands every lane two consecutive rows of one column.
+// A(a, r) = D[r][j*S + a], B(r, c) = V[r][j*S + c]; the accumulators of the
+// S x S block stay in registers over the CTA's rows, then the warps are summed
+// with shared atomics and added to G with one float atomic per element.
+__device__ __forceinline__ void ldsm_x4_trans(const void *p, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+  const uint32_t a = uint32_t(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(a));
+}
+
+template <int S>
+__global__ void __launch_bounds__(SB_WARPS * 32) smallb_grad_mma_kernel(const bf16 *__restrict__ D,
+                                                                        const bf16 *__restrict__ V, int64_t ld,
+                                                                        int64_t rows, int64_t rows_per_cta,
+                                                                        float *__restrict__ G, int64_t ldg,
+                                                                        int64_t gstride) {
+  constexpr int MT = S / 16, NT = S / 8, RW = 32, LDS = S + 8, CH = S / 8;  // CH: 16-byte chunks per row
+  __shared__ __align__(16) bf16 sd[SB_WARPS][RW][LDS];
+  __shared__ __align__(16) bf16 sv[SB_WARPS][RW][LDS];
+  __shared__ float red[S][S + 1];
+  const int j = blockIdx.y;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int g = lane >> 2, q = lane & 3;
+  for (int e = threadIdx.x; e < S * (S + 1); e += blockDim.x) (&red[0][0])[e] = 0.f;
+  const int64_t r_begin = int64_t(blockIdx.x) * rows_per_cta;
+  const int64_t r_end = r_begin + rows_per_cta < rows ? r_begin + rows_per_cta : rows;
+  const bf16 *Dj = D + int64_t(j) * S;
+  const bf16 *Vj = V + int64_t(j) * S;
+  float acc[MT][NT][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+  // ldmatrix addresses: lane i of matrix (lane / 8) gives row (lane % 8) of that 8 x 8 matrix
+  const int mi = lane >> 3, mr = lane & 7;
+  for (int64_t r0 = r_begin + warp * RW; r0 < r_end; r0 += SB_WARPS * RW) {
+    uint4 dbuf[RW * CH / 32], vbuf[RW * CH / 32];
+#pragma unroll
+    for (int i = 0; i < RW * CH / 32; ++i) {
+      const int idx = lane + 32 * i, r = idx / CH, ch = idx % CH;
+      const bool ok = r0 + r < r_end;
+      dbuf[i] = ok ? *reinterpret_cast<const uint4 *>(Dj + (r0 + r) * ld + ch * 8) : make_uint4(0, 0, 0, 0);
+      vbuf[i] = ok ? *reinterpret_cast<const uint4 *>(Vj + (r0 + r) * ld + ch * 8) : make_uint4(0, 0, 0, 0);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < RW * CH / 32; ++i) {
+      const int idx = lane + 32 * i, r = idx / CH, ch = idx % CH;
+      *reinterpret_cast<uint4 *>(&sd[warp][r][ch * 8]) = dbuf[i];
+      *reinterpret_cast<uint4 *>(&sv[warp][r][ch * 8]) = vbuf[i];
+    }
+    __syncwarp();
+#pragma unroll
+    for (int k0 = 0; k0 < RW; k0 += 16) {
+      uint32_t af[MT][4], bfr[NT][2];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)  // matrix i: rows k0 + 8 (i & 2 ? 1 : 0), columns 16 mt + 8 (i & 1)
+        ldsm_x4_trans(&sd[warp][k0 + ((mi & 2) ? 8 : 0) + mr][mt * 16 + ((mi & 1) ? 8 : 0)], af[mt][0], af[mt][1],
+                      af[mt][2], af[mt][3]);
+#pragma unroll
+      for (int np = 0; np < NT / 2; ++np)  // matrix i: rows k0 + 8 (i & 1), columns 16 np + 8 (i & 2 ? 1 : 0)
+        ldsm_x4_trans(&sv[warp][k0 + ((mi & 1) ? 8 : 0) + mr][np * 16 + ((mi & 2) ? 8 : 0)], bfr[2 * np][0],
+                      bfr[2 * np][1], bfr[2 * np + 1][0], bfr[2 * np + 1][1]);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          asm volatile(
+              "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+              "{%0, %1, %2, %3};"
+              : "+f"(acc[mt][nt][0]), "+f"(acc[mt][nt][1]), "+f"(acc[mt][nt][2]), "+f"(acc[mt][nt][3])
+              : "r"(af[mt][0]), "r"(af[mt][1]), "r"(af[mt][2]), "r"(af[mt][3]), "r"(bfr[nt][0]), "r"(bfr[nt][1]));
+    }
+    __syncwarp();
+  }
+  __syncthreads();  // red zeroed
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int a = mt * 16 + g, c = nt * 8 + 2 * q;
+      atomicAdd(&red[a][c], acc[mt][nt][0]);
+      atomicAdd(&red[a][c + 1], acc[mt][nt][1]);
+      atomicAdd(&red[a + 8][c], acc[mt][nt][2]);
+      atomicAdd(&red[a + 8][c + 1], acc[mt][nt][3]);
+    }
+  __syncthreads();
+  float *Gj = G + int64_t(j) * gstride;
+  for (int e = threadIdx.x; e < S * S; e += blockDim.x) {
+    const int a = e / S, c = e % S;
+    atomicAdd(Gj + int64_t(a) * ldg + c, red[a][c]);
+  }
+}
+
+// Row ranges per block for about four CTAs per SM over all blocks (at least 64 rows each).
 int64_t rows_per_cta(int64_t rows, int nprim) {
   int64_t ranges = (int64_t(num_sms()) * 4 + nprim - 1) / nprim;
   int64_t per = (rows + ranges - 1) / ranges;
@@ -335,7 +437,17 @@ poet_status smallb_grad(int dtype, const void *D, const void *V, int64_t ld, int
   POET_TRY(zero_output(G, s, s, ldg, nprim, gstride, st));  // the CTAs' sums are added into it
   const double elems = double(rows) * nprim * s;
   TraceScope ts("blk_grad", 2.0 * elems * s, elems * esize(dtype) * 2.0, st);
-  if (dtype == POET_BF16)
+  const bool chunks_ok = ((reinterpret_cast<uintptr_t>(D) | reinterpret_cast<uintptr_t>(V)) & 15) == 0 && ld % 8 == 0;
+  if (dtype == POET_BF16 && (s == 16 || s == 32) && chunks_ok) {
+    if (s == 32)
+      smallb_grad_mma_kernel<32><<<grid, SB_WARPS * 32, 0, st>>>(static_cast<const bf16 *>(D),
+                                                                 static_cast<const bf16 *>(V), ld, rows, per, G, ldg,
+                                                                 gstride);
+    else
+      smallb_grad_mma_kernel<16><<<grid, SB_WARPS * 32, 0, st>>>(static_cast<const bf16 *>(D),
+                                                                 static_cast<const bf16 *>(V), ld, rows, per, G, ldg,
+                                                                 gstride);
+  } else if (dtype == POET_BF16)
     smallb_grad_kernel<bf16><<<grid, SB_WARPS * 32, 0, st>>>(
         static_cast<const bf16 *>(D), static_cast<const bf16 *>(V), ld, rows, per, s, G, ldg, gstride);
   else
