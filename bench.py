@@ -47,9 +47,11 @@ def row_stride(d):
 PLAN_NAMES = {1: "token", 2: "weight"}
 
 # DRAM traffic / algorithmic bytes of one launch, from an ncu capture, with the
-# kernel revision (as named in poet_version()) the counters were taken on.
-NCU_TRAFFIC_RATIO = {"w0_fwd": (0.999, "gemm_tc r22;"), "w0_bwd": (1.025, "gemm_tc r22;"),
-                     "w_grad": (1.273, "gemm_tc r22;")}
+# engine revisions (as named in poet_version()) that run that launch unchanged:
+# the counters were taken on r22; r25 changes only the plan of grouped launches
+# whose problems are at most 256 columns wide, which these launches are not.
+_T_SIZED = ("gemm_tc r22;", "gemm_tc r25;")
+NCU_TRAFFIC_RATIO = {"w0_fwd": (0.999, _T_SIZED), "w0_bwd": (1.025, _T_SIZED), "w_grad": (1.273, _T_SIZED)}
 NCU_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the grouped launch of one LLaMA-1.3B "
                       "layer at 16384 tokens (profiles/w0_gemm_llama1.3b_layer_T16384.md), as a ratio to the "
                       "algorithmic bytes of that launch, scaled to this run's launches")
@@ -373,7 +375,7 @@ def roofline_of(rows, version):
         roof = {"bound": "hbm", "unit": "GB/s", "peak_kind": "copy, " + peaks["source"]}
     traffic = None
     ratio = NCU_TRAFFIC_RATIO.get(dominant)
-    if ratio and ratio[1] in version:  # counters taken on this kernel revision
+    if ratio and any(r in version for r in ratio[1]):  # counters valid for this kernel revision
         traffic = round(ratio[0] * r["bytes"] / r["launches"])
     roof.update({"kernel": dominant, "achieved": round(achieved, 1), "peak": peak,
                  "frac": round(achieved / peak, 4), "traffic": traffic, "avg_launch_ms": round(avg_ms, 4),

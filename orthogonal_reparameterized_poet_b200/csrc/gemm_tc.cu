@@ -1304,7 +1304,11 @@ poet_status gemm_tc_many(const Gemm *gs, int count, cudaStream_t st) {
         tiles += wide_tiles(v[i + j]);
         any_atomic |= v[i + j].atomic;
       }
-      const TcPlan t = paired(narrowed(plans[b], tiles, any_atomic), v.data() + i, n);
+      // only single-problem launches have a B-stationary kernel: a grouped
+      // launch of such problems streams, and then on CTA pairs where they qualify
+      TcPlan base = plans[b];
+      if (n > 1) base.bstat = false;
+      const TcPlan t = paired(narrowed(base, tiles, any_atomic), v.data() + i, n);
       if (n == 1) POET_TRY(run_group<1>(v.data() + i, 1, t, st));
       else POET_TRY(run_group<kGroupMax>(v.data() + i, n, t, st));
     }
