@@ -692,7 +692,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_tc_kernel(const __grid_const
       const int64_t tile = tile_of(k);
       if (tile >= t_end || *abort) break;
       const TileCoord c = decode(tile, g);
-      const TcProblem &p = g.prob[c.pi];
+      // A copy, not a reference: the problem's fields then live in registers.
+      // Read in place, every use went back to the kernel's parameter space
+      // (each asm with a memory clobber forces a reload), which cost about a
+      // quarter of a tile's epilogue.
+      const TcProblem p = g.prob[c.pi];
       if (!mbar_wait(&tfull[acc], acc_phase, abort, g.errword)) break;
       tc_fence_after();
       const int mrow0 = c.mt * (BM * CG) + int(rank) * BM;  // this CTA's first accumulator row
