@@ -197,6 +197,103 @@ __device__ __forceinline__ uint32_t bf16_pair(bf16 lo, bf16 hi) {
   return uint32_t(__bfloat16_as_ushort(lo)) | (uint32_t(__bfloat16_as_ushort(hi)) << 16);
 }
 
+__device__ __forceinline__ void ldsm_x4(const void *p, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+  const uint32_t a = uint32_t(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x4_trans(const void *p, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+  const uint32_t a = uint32_t(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(a));
+}
+
+// The same product for 16-byte aligned rows, with every global access a
+// 16-byte unit: each warp stages 32 rows of X_j in its own shared memory
+// (rows padded to S + 8 elements, so that the eight row segments of an
+// ldmatrix fall on distinct banks), takes the A fragments with ldmatrix,
+// writes the outputs back over the same rows and stores them as 16-byte
+// units.  (The 4-byte fragment loads and stores of the kernel below keep
+// L1/TEX busy well before HBM.)
+template <int S>
+__global__ void __launch_bounds__(SB_WARPS * 32) smallb_right_mma_staged_kernel(
+    const bf16 *__restrict__ X, int64_t ldx, int64_t rows, int64_t rows_per_cta, const bf16 *__restrict__ M,
+    int64_t ldm, int64_t bstride, int trans, bf16 *__restrict__ out, int64_t ldo) {
+  constexpr int KS = S / 16, NT = S / 8, RW = 32, LDS = S + 8, CH = S / 8, PER = RW * CH / 32;
+  __shared__ __align__(16) bf16 sx[SB_WARPS][RW][LDS];
+  const int j = blockIdx.y;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int g = lane >> 2, q = lane & 3, mi = lane >> 3, mr = lane & 7;
+  const bf16 *Mj = M + int64_t(j) * bstride;
+  auto m_at = [&](int a, int c) { return trans ? Mj[int64_t(c) * ldm + a] : Mj[int64_t(a) * ldm + c]; };
+  uint32_t bfr[KS][NT][2];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int a = nt * 8 + g, c = ks * 16 + 2 * q;
+      bfr[ks][nt][0] = bf16_pair(m_at(a, c), m_at(a, c + 1));
+      bfr[ks][nt][1] = bf16_pair(m_at(a, c + 8), m_at(a, c + 9));
+    }
+  const int64_t r_begin = int64_t(blockIdx.x) * rows_per_cta;
+  const int64_t r_end = r_begin + rows_per_cta < rows ? r_begin + rows_per_cta : rows;
+  const bf16 *Xj = X + int64_t(j) * S;
+  bf16 *Oj = out + int64_t(j) * S;
+  bf16(*tile)[LDS] = sx[warp];
+  for (int64_t r0 = r_begin + warp * RW; r0 < r_end; r0 += SB_WARPS * RW) {
+    uint4 buf[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int idx = lane + 32 * i, r = idx / CH, ch = idx % CH;
+      buf[i] = r0 + r < r_end ? *reinterpret_cast<const uint4 *>(Xj + (r0 + r) * ldx + ch * 8) : make_uint4(0, 0, 0, 0);
+    }
+    __syncwarp();  // the previous rows' outputs have left the tile
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int idx = lane + 32 * i, r = idx / CH, ch = idx % CH;
+      *reinterpret_cast<uint4 *>(&tile[r][ch * 8]) = buf[i];
+    }
+    __syncwarp();
+#pragma unroll
+    for (int mt = 0; mt < RW / 16; ++mt) {
+      uint32_t af[KS][4];
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks)  // matrix i: rows 16 mt + 8 (i & 1), columns 16 ks + 8 (i >> 1)
+        ldsm_x4(&tile[mt * 16 + (mi & 1) * 8 + mr][ks * 16 + (mi >> 1) * 8], af[ks][0], af[ks][1], af[ks][2],
+                af[ks][3]);
+      float acc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks)
+          asm volatile(
+              "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+              "{%0, %1, %2, %3};"
+              : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
+              : "r"(af[ks][0]), "r"(af[ks][1]), "r"(af[ks][2]), "r"(af[ks][3]), "r"(bfr[ks][nt][0]),
+                "r"(bfr[ks][nt][1]));
+      }
+      __syncwarp();  // every lane's fragments of these 16 rows are in registers
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int c = nt * 8 + 2 * q;
+        *reinterpret_cast<__nv_bfloat162 *>(&tile[mt * 16 + g][c]) = __floats2bfloat162_rn(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<__nv_bfloat162 *>(&tile[mt * 16 + g + 8][c]) = __floats2bfloat162_rn(acc[nt][2], acc[nt][3]);
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int idx = lane + 32 * i, r = idx / CH, ch = idx % CH;
+      if (r0 + r < r_end)
+        *reinterpret_cast<uint4 *>(Oj + (r0 + r) * ldo + ch * 8) = *reinterpret_cast<const uint4 *>(&tile[r][ch * 8]);
+    }
+  }
+}
+
 template <int S>
 __global__ void __launch_bounds__(SB_WARPS * 32) smallb_right_mma_kernel(const bf16 *__restrict__ X, int64_t ldx,
                                                                          int64_t rows, int64_t rows_per_cta,
@@ -272,12 +369,6 @@ __global__ void __launch_bounds__(SB_WARPS * 32) smallb_right_mma_kernel(const b
 // A(a, r) = D[r][j*S + a], B(r, c) = V[r][j*S + c]; the accumulators of the
 // S x S block stay in registers over the CTA's rows, then the warps are summed
 // with shared atomics and added to G with one float atomic per element.
-__device__ __forceinline__ void ldsm_x4_trans(const void *p, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
-  const uint32_t a = uint32_t(__cvta_generic_to_shared(p));
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(a));
-}
 
 template <int S>
 __global__ void __launch_bounds__(SB_WARPS * 32) smallb_grad_mma_kernel(const bf16 *__restrict__ D,
@@ -387,7 +478,18 @@ poet_status smallb_right(int dtype, const void *X, int64_t ldx, int64_t rows, co
   TraceScope ts(kind, 2.0 * elems * s, elems * esize(dtype) * 2.0, st);
   const bool pairs_ok = ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(out)) & 3) == 0 &&
                         ldx % 2 == 0 && ldo % 2 == 0;
-  if (dtype == POET_BF16 && (s == 16 || s == 32) && pairs_ok) {
+  const bool units_ok = ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(out)) & 15) == 0 &&
+                        ldx % 8 == 0 && ldo % 8 == 0;
+  if (dtype == POET_BF16 && (s == 16 || s == 32) && units_ok) {
+    if (s == 32)
+      smallb_right_mma_staged_kernel<32><<<grid, SB_WARPS * 32, 0, st>>>(
+          static_cast<const bf16 *>(X), ldx, rows, per, static_cast<const bf16 *>(M), ldm, bstride, trans ? 1 : 0,
+          static_cast<bf16 *>(out), ldo);
+    else
+      smallb_right_mma_staged_kernel<16><<<grid, SB_WARPS * 32, 0, st>>>(
+          static_cast<const bf16 *>(X), ldx, rows, per, static_cast<const bf16 *>(M), ldm, bstride, trans ? 1 : 0,
+          static_cast<bf16 *>(out), ldo);
+  } else if (dtype == POET_BF16 && (s == 16 || s == 32) && pairs_ok) {
     if (s == 32)
       smallb_right_mma_kernel<32><<<grid, SB_WARPS * 32, 0, st>>>(static_cast<const bf16 *>(X), ldx, rows, per,
                                                                   static_cast<const bf16 *>(M), ldm, bstride,
