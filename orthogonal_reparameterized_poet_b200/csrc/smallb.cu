@@ -184,15 +184,6 @@ __global__ void __launch_bounds__(SB_WARPS * 32) smallb_grad_kernel(const T *__r
   }
 }
 
-// right for bf16 blocks of 16 or 32 on the tensor cores: mma.sync
-// m16n8k16 (bf16 in, float accumulate), which takes the s multiply-adds per
-// output off the CUDA cores (the CUDA-core kernel above is bound by them and
-// by its broadcast reads).  blockIdx.y = block j; each warp holds M_j's
-// fragments in registers and takes 16 rows at a time.  Fragment layouts of
-// m16n8k16 (g = lane / 4, q = lane % 4): A regs = X[g][2q..], X[g+8][2q..],
-// X[g][2q+8..], X[g+8][2q+8..]; B regs = M(n=g, k=2q..), M(g, 2q+8..);
-// C = out[g][2q..], out[g+8][2q..]; every register holds two consecutive
-// bf16 (the lower column in the low half).
 __device__ __forceinline__ uint32_t bf16_pair(bf16 lo, bf16 hi) {
   return uint32_t(__bfloat16_as_ushort(lo)) | (uint32_t(__bfloat16_as_ushort(hi)) << 16);
 }
@@ -210,13 +201,20 @@ __device__ __forceinline__ void ldsm_x4_trans(const void *p, uint32_t &r0, uint3
                : "r"(a));
 }
 
-// The same product for 16-byte aligned rows, with every global access a
-// 16-byte unit: each warp stages 32 rows of X_j in its own shared memory
-// (rows padded to S + 8 elements, so that the eight row segments of an
-// ldmatrix fall on distinct banks), takes the A fragments with ldmatrix,
-// writes the outputs back over the same rows and stores them as 16-byte
-// units.  (The 4-byte fragment loads and stores of the kernel below keep
-// L1/TEX busy well before HBM.)
+// right for bf16 blocks of 16 or 32 with 16-byte aligned rows, on the tensor
+// cores: mma.sync m16n8k16 (bf16 in, float accumulate) takes the s
+// multiply-adds per output off the CUDA cores (the CUDA-core kernel above is
+// bound by them and by its broadcast reads).  blockIdx.y = block j.  Each
+// warp holds M_j's B fragments in registers, stages 32 rows of X_j in its own
+// shared memory with 16-byte loads (rows padded to S + 8 elements, so that
+// the eight row segments of an ldmatrix fall on distinct banks), takes the A
+// fragments with ldmatrix, writes the outputs back over the same rows and
+// stores them as 16-byte units.  Fragment layouts of m16n8k16 (g = lane / 4,
+// q = lane % 4): A regs = X[g][2q..], X[g+8][2q..], X[g][2q+8..],
+// X[g+8][2q+8..]; B regs = M(n=g, k=2q..), M(g, 2q+8..); C = out[g][2q..],
+// out[g+8][2q..]; every register holds two consecutive bf16 (the lower
+// column in the low half).  Fragments built from 4-byte global loads and
+// stores instead kept L1/TEX at 87 % at half the copy peak.
 template <int S>
 __global__ void __launch_bounds__(SB_WARPS * 32) smallb_right_mma_staged_kernel(
     const bf16 *__restrict__ X, int64_t ldx, int64_t rows, int64_t rows_per_cta, const bf16 *__restrict__ M,
@@ -290,72 +288,6 @@ __global__ void __launch_bounds__(SB_WARPS * 32) smallb_right_mma_staged_kernel(
       const int idx = lane + 32 * i, r = idx / CH, ch = idx % CH;
       if (r0 + r < r_end)
         *reinterpret_cast<uint4 *>(Oj + (r0 + r) * ldo + ch * 8) = *reinterpret_cast<const uint4 *>(&tile[r][ch * 8]);
-    }
-  }
-}
-
-template <int S>
-__global__ void __launch_bounds__(SB_WARPS * 32) smallb_right_mma_kernel(const bf16 *__restrict__ X, int64_t ldx,
-                                                                         int64_t rows, int64_t rows_per_cta,
-                                                                         const bf16 *__restrict__ M, int64_t ldm,
-                                                                         int64_t bstride, int trans,
-                                                                         bf16 *__restrict__ out, int64_t ldo) {
-  constexpr int KS = S / 16, NT = S / 8;
-  const int j = blockIdx.y;
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int g = lane >> 2, q = lane & 3;
-  const bf16 *Mj = M + int64_t(j) * bstride;
-  auto m_at = [&](int a, int c) { return trans ? Mj[int64_t(c) * ldm + a] : Mj[int64_t(a) * ldm + c]; };
-  uint32_t bfr[KS][NT][2];
-#pragma unroll
-  for (int ks = 0; ks < KS; ++ks)
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int a = nt * 8 + g, c = ks * 16 + 2 * q;
-      bfr[ks][nt][0] = bf16_pair(m_at(a, c), m_at(a, c + 1));
-      bfr[ks][nt][1] = bf16_pair(m_at(a, c + 8), m_at(a, c + 9));
-    }
-  const int64_t r_begin = int64_t(blockIdx.x) * rows_per_cta;
-  const int64_t r_end = r_begin + rows_per_cta < rows ? r_begin + rows_per_cta : rows;
-  const bf16 *Xj = X + int64_t(j) * S;
-  bf16 *Oj = out + int64_t(j) * S;
-  // U tiles of 16 rows per warp iteration, all loads issued before the MMAs
-  // (about 2 KB of each warp's reads in flight)
-  constexpr int U = 64 / S;
-  for (int64_t r0 = r_begin + warp * 16 * U; r0 < r_end; r0 += SB_WARPS * 16 * U) {
-    uint32_t afr[U][KS][4];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t ra = r0 + u * 16 + g, rb = ra + 8;
-      const bool oka = ra < r_end, okb = rb < r_end;
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        const int c = ks * 16 + 2 * q;
-        afr[u][ks][0] = oka ? *reinterpret_cast<const uint32_t *>(Xj + ra * ldx + c) : 0u;
-        afr[u][ks][1] = okb ? *reinterpret_cast<const uint32_t *>(Xj + rb * ldx + c) : 0u;
-        afr[u][ks][2] = oka ? *reinterpret_cast<const uint32_t *>(Xj + ra * ldx + c + 8) : 0u;
-        afr[u][ks][3] = okb ? *reinterpret_cast<const uint32_t *>(Xj + rb * ldx + c + 8) : 0u;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t ra = r0 + u * 16 + g, rb = ra + 8;
-      const bool oka = ra < r_end, okb = rb < r_end;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks)
-          asm volatile(
-              "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-              "{%0, %1, %2, %3};"
-              : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
-              : "r"(afr[u][ks][0]), "r"(afr[u][ks][1]), "r"(afr[u][ks][2]), "r"(afr[u][ks][3]),
-                "r"(bfr[ks][nt][0]), "r"(bfr[ks][nt][1]));
-        const int c = nt * 8 + 2 * q;
-        if (oka) *reinterpret_cast<__nv_bfloat162 *>(Oj + ra * ldo + c) = __floats2bfloat162_rn(acc[0], acc[1]);
-        if (okb) *reinterpret_cast<__nv_bfloat162 *>(Oj + rb * ldo + c) = __floats2bfloat162_rn(acc[2], acc[3]);
-      }
     }
   }
 }
@@ -476,8 +408,6 @@ poet_status smallb_right(int dtype, const void *X, int64_t ldx, int64_t rows, co
   const dim3 grid(unsigned((rows + per - 1) / per), unsigned(nprim));
   const double elems = double(rows) * nprim * s;
   TraceScope ts(kind, 2.0 * elems * s, elems * esize(dtype) * 2.0, st);
-  const bool pairs_ok = ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(out)) & 3) == 0 &&
-                        ldx % 2 == 0 && ldo % 2 == 0;
   const bool units_ok = ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(out)) & 15) == 0 &&
                         ldx % 8 == 0 && ldo % 8 == 0;
   if (dtype == POET_BF16 && (s == 16 || s == 32) && units_ok) {
@@ -489,15 +419,6 @@ poet_status smallb_right(int dtype, const void *X, int64_t ldx, int64_t rows, co
       smallb_right_mma_staged_kernel<16><<<grid, SB_WARPS * 32, 0, st>>>(
           static_cast<const bf16 *>(X), ldx, rows, per, static_cast<const bf16 *>(M), ldm, bstride, trans ? 1 : 0,
           static_cast<bf16 *>(out), ldo);
-  } else if (dtype == POET_BF16 && (s == 16 || s == 32) && pairs_ok) {
-    if (s == 32)
-      smallb_right_mma_kernel<32><<<grid, SB_WARPS * 32, 0, st>>>(static_cast<const bf16 *>(X), ldx, rows, per,
-                                                                  static_cast<const bf16 *>(M), ldm, bstride,
-                                                                  trans ? 1 : 0, static_cast<bf16 *>(out), ldo);
-    else
-      smallb_right_mma_kernel<16><<<grid, SB_WARPS * 32, 0, st>>>(static_cast<const bf16 *>(X), ldx, rows, per,
-                                                                  static_cast<const bf16 *>(M), ldm, bstride,
-                                                                  trans ? 1 : 0, static_cast<bf16 *>(out), ldo);
   } else if (dtype == POET_BF16)
     smallb_right_kernel<bf16><<<grid, SB_WARPS * 32, 0, st>>>(static_cast<const bf16 *>(X), ldx, rows, per,
                                                               static_cast<const bf16 *>(M), ldm, bstride, s,
