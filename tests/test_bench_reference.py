@@ -35,3 +35,26 @@ def test_reference_arm_prints_one_contract_line():
 
 def test_reference_arm_other_ranks_do_no_work():
     assert _run({"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_kernel_table_holds_each_launch_to_its_own_bound():
+    """The per-kind roofline fraction: the roofline time of the tensor-bound
+    launches' flops at the tensor peak plus the HBM-bound launches' bytes at
+    the copy peak, over the measured time.  A kind with one launch of each
+    kind gets the sum of both terms; `bound` names the larger."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    peaks = bench.load_peaks()
+    pt, ph = peaks["bf16_tflops_sustained"] * 1e12, peaks["hbm_gbs"] * 1e9
+    t_tc, t_hbm = 1e-3, 3e-3  # seconds of roofline time in each term
+    rows = {"mixed": {"launches": 2, "ms": 8.0, "flop": t_tc * pt + 1e9, "bytes": 5e9 + t_hbm * ph,
+                      "flop_tc": t_tc * pt, "bytes_hbm": t_hbm * ph},
+            "copy": {"launches": 1, "ms": 1.0, "flop": 0.0, "bytes": 0.5 * 1e-3 * ph, "flop_tc": 0.0,
+                     "bytes_hbm": 0.5 * 1e-3 * ph}}
+    tab = bench.kernel_table(rows, steps=1)
+    assert abs(tab["mixed"]["frac"] - 0.5) < 1e-4 and tab["mixed"]["bound"] == "hbm"
+    assert abs(tab["copy"]["frac"] - 0.5) < 1e-4 and tab["copy"]["bound"] == "hbm" and tab["copy"]["tflops"] is None
+    rows["mixed"]["bytes_hbm"] = 0.0
+    tab = bench.kernel_table(rows, steps=1)
+    assert abs(tab["mixed"]["frac"] - 0.125) < 1e-4 and tab["mixed"]["bound"] == "tensor"
