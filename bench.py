@@ -50,8 +50,9 @@ PLAN_NAMES = {1: "token", 2: "weight"}
 # engine revisions (as named in poet_version()) that run that launch unchanged:
 # the counters were taken on r22; r25 changes only the plan of grouped launches
 # whose problems are at most 256 columns wide, which these launches are not;
-# r26 keeps the epilogue's problem fields in registers (instructions, not bytes).
-_T_SIZED = ("gemm_tc r22;", "gemm_tc r25;", "gemm_tc r26;")
+# r26 keeps the epilogue's problem fields in registers (instructions, not bytes);
+# r27 returns the grouped launches of r25 to single CTAs.
+_T_SIZED = ("gemm_tc r22;", "gemm_tc r25;", "gemm_tc r26;", "gemm_tc r27;")
 NCU_TRAFFIC_RATIO = {"w0_fwd": (0.999, _T_SIZED), "w0_bwd": (1.025, _T_SIZED), "w_grad": (1.273, _T_SIZED)}
 NCU_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the grouped launch of one LLaMA-1.3B "
                       "layer at 16384 tokens (profiles/w0_gemm_llama1.3b_layer_T16384.md), as a ratio to the "

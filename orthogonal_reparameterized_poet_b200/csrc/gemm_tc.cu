@@ -1308,11 +1308,14 @@ poet_status gemm_tc_many(const Gemm *gs, int count, cudaStream_t st) {
         tiles += wide_tiles(v[i + j]);
         any_atomic |= v[i + j].atomic;
       }
-      // only single-problem launches have a B-stationary kernel: a grouped
-      // launch of such problems streams, and then on CTA pairs where they qualify
-      TcPlan base = plans[b];
-      if (n > 1) base.bstat = false;
-      const TcPlan t = paired(narrowed(base, tiles, any_atomic), v.data() + i, n);
+      // Only single-problem launches have a B-stationary kernel.  A grouped
+      // launch of such problems (at most 256 columns, K <= 256) streams on
+      // single CTAs with 256-wide tiles: their time goes to the epilogue (four
+      // k-blocks of MMA per tile), which CTA pairs do not shorten, and pairs
+      // measured 5-8 % slower on them.
+      TcPlan t = plans[b];
+      if (!(t.bstat && n > 1)) t = paired(narrowed(t, tiles, any_atomic), v.data() + i, n);
+      else t.bstat = false;
       if (n == 1) POET_TRY(run_group<1>(v.data() + i, 1, t, st));
       else POET_TRY(run_group<kGroupMax>(v.data() + i, n, t, st));
     }

@@ -366,7 +366,7 @@ extern "C" {
 const char *poet_last_error(void) { return g_last_error; }
 
 // The kernel revisions name the code that profiles/ counters were taken on.
-const char *poet_version(void) { return "libpoet 0.4 (sm_100a; gemm_tc r26; permute r9; restride r1; cnp r7; smallb r6; block r1)"; }
+const char *poet_version(void) { return "libpoet 0.4 (sm_100a; gemm_tc r27; permute r9; restride r1; cnp r7; smallb r6; block r1)"; }
 
 size_t poet_side_state_bytes(const poet_side *side, int32_t dtype) {
   SideGeom g;
